@@ -1,0 +1,116 @@
+"""LiteAttention skip update over a denoising chain, fp64 (oracle only).
+
+Follows the LiteAttention write-up (arXiv 2511.11062):
+* section 5: a block whose local maximum lies far below the accumulated
+  (running) maximum contributes an exponentially suppressed amount, the test
+  is local to each block;
+* sections 2, 3 and 6: the decision is recorded in a persistent tile-level
+  skip mask that later denoising steps reuse; a skipped tile is not loaded,
+  multiplied or exponentiated at all.
+
+Readings (stated because the page gives prose only):
+* k-blocks of q-block i are visited in ascending j among those with
+  mask[i, j] != 0 and skip_in[i, j] == 0;
+* m_r is the running maximum of the logits of row r over the blocks visited
+  before j; l_r(j) is the maximum of row r over block j's valid columns;
+* block j (not the first visited) gets a new skip bit iff l_r(j) < m_r - eps
+  for every valid row r of the q-block; eps is in natural-log logit units;
+* the output of the detecting step still includes block j; the bit takes
+  effect from the next step: skip_out = skip_in | new_bits.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+from .attention import _f64, _nblocks, _mask4
+
+
+def lite_qblock(qh, kh, vh, block, keep_row, i, eps, scale):
+    """(O rows, LSE rows, new-bit row, margin row) for one q-block.
+
+    margin[j] = max_r (l_r(j) - m_r + eps) for tested blocks (NaN elsewhere);
+    the new bit is set iff margin[j] < 0.
+    """
+    N = qh.shape[0]
+    d = vh.shape[1]
+    nkb = keep_row.shape[0]
+    r0, r1 = i * block, min(N, (i + 1) * block)
+    visited = np.nonzero(keep_row)[0]
+    new = np.zeros(nkb, dtype=np.uint8)
+    margin = np.full(nkb, np.nan)
+    if visited.size == 0:
+        return np.zeros((r1 - r0, d)), np.full(r1 - r0, -np.inf), new, margin
+    cols = [np.arange(j * block, min(N, (j + 1) * block)) for j in visited]
+    c = np.concatenate(cols)
+    s = (qh[r0:r1] @ kh[c].T) * scale
+    running = np.full(r1 - r0, -np.inf)
+    off = 0
+    for n_vis, j in enumerate(visited):
+        w = cols[n_vis].shape[0]
+        local = s[:, off:off + w].max(axis=1)
+        if n_vis > 0:
+            mg = np.max(local - running + eps)
+            margin[j] = mg
+            if mg < 0:
+                new[j] = 1
+        running = np.maximum(running, local)
+        off += w
+    m = s.max(axis=1, keepdims=True)
+    e = np.exp(s - m)
+    z = e.sum(axis=1, keepdims=True)
+    return (e / z) @ vh[c], (m + np.log(z))[:, 0], new, margin
+
+
+def lite_step(q, k, v, block, mask=None, skip_in=None, eps=10.0, scale=None, qblocks=None):
+    """One denoising step of block attention with the LiteAttention skip update.
+
+    Effective keep = mask & ~skip_in.  Returns (O, LSE, skip_out, margin) with
+    skip_out = skip_in | new bits, or a dict {(b,h,i): (O, LSE, skip_out_row,
+    margin_row)} when ``qblocks`` is given.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, N, d = q.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    nqb = nkb = _nblocks(N, block)
+    m4 = _mask4(mask, B, H, nqb, nkb)
+    if skip_in is None:
+        s4 = np.zeros((B, H, nqb, nkb), dtype=np.uint8)
+    else:
+        s4 = np.asarray(skip_in.detach().cpu().numpy() if hasattr(skip_in, "detach") else skip_in)
+        s4 = np.broadcast_to(s4, (B, H, nqb, nkb))
+
+    def one(b, h, i):
+        keep = (m4[b, h, i] != 0) & (s4[b, h, i] == 0)
+        o, lse, new, mg = lite_qblock(q[b, h], k[b, h], v[b, h], block, keep, i, eps, scale)
+        return o, lse, (s4[b, h, i] | new).astype(np.uint8), mg
+
+    if qblocks is not None:
+        return {key: one(*key) for key in qblocks}
+    O = np.zeros((B, H, N, d))
+    L = np.zeros((B, H, N))
+    S = np.zeros((B, H, nqb, nkb), dtype=np.uint8)
+    M = np.full((B, H, nqb, nkb), np.nan)
+    for b in range(B):
+        for h in range(H):
+            for i in range(nqb):
+                r0, r1 = i * block, min(N, (i + 1) * block)
+                O[b, h, r0:r1], L[b, h, r0:r1], S[b, h, i], M[b, h, i] = one(b, h, i)
+    return O, L, S, M
+
+
+def lite_chain(steps_inputs, block, eps, mask=None, skip0=None, feed=None):
+    """Run lite_step over a sequence of (q, k, v) denoising inputs.
+
+    ``feed(s, skip_out)`` may replace the skip mask handed to step s+1 (used
+    for teacher forcing against another implementation).  Returns a list of
+    per-step (O, LSE, skip_out, margin).
+    """
+    out = []
+    skip = skip0
+    for s, (q, k, v) in enumerate(steps_inputs):
+        O, L, S, M = lite_step(q, k, v, block, mask, skip, eps)
+        out.append((O, L, S, M))
+        skip = S if feed is None else feed(s, S)
+    return out
