@@ -1,0 +1,364 @@
+"""Benchmark: block-sparse attention with the LiteAttention skip chain on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--no-e2e] [--no-cpu-baseline]
+
+Default workload: the Wan2.1-14B-like 720p LiteAttention step (B=1, H=40,
+d=128, 21 x 45 x 80 grid = 75,600 tokens, block 128, eps = 10): each bench
+step is one denoising step's attention call, sa_sparse_attn_fwd with an
+all-kept mask, skip_in = the previous step's skip_out, and a fresh skip_out
+(the whole hot path of this workload; the skip test is fused in the kernel).
+Each step's Q/K/V are that denoising step's drifted inputs (x <- 0.98 x +
+0.2 xi), drawn on the device before the timed region; 3 x 774 MB per step is
+far larger than L2, so no flush is needed between steps.
+
+Printed metric: executed TFLOP/s of the attention forward (4 * d * sum over
+visited (q-block, k-block) pairs of valid rows x valid columns), with ms per
+call, density and the dense-equivalent rate alongside.  With N > 1 GPUs each
+rank runs its own copy of the workload (heads are independent; weak scaling,
+no collective on the data path) and the value is total FLOPs / max-over-ranks
+time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sparse attn ms/call, executed TFLOP/s & % B200 BF16 tensor peak at 75.6K tok"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"sa_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", str(self.dev)], stdout=self.out,
+                                         stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.close()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = max(mx, float(parts[2]))
+                except ValueError:
+                    continue
+                for nm, val in zip(names, parts[5:9]):
+                    if val.lower() == "active":
+                        reasons.add(nm)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def executed_flops(skip_in, N, block, d, mask=None):
+    """4 * d * sum over visited (i, j) of valid rows_i * valid cols_j."""
+    nb = -(-N // block)
+    rows = torch.full((nb,), float(block), device=skip_in.device, dtype=torch.float64)
+    rows[-1] = N - (nb - 1) * block
+    vis = (1 - skip_in.to(torch.float64))
+    if mask is not None:
+        vis = vis * (mask != 0).to(torch.float64)
+    per_bh = torch.einsum("i,bhij,j->bh", rows, vis, rows)
+    return float(4.0 * d * per_bh.sum().item())
+
+
+# ----------------------------------------------------------------- our arm ---
+
+def run_ours(args, rank, world, local):
+    from block_sparse_attention_flash_b200 import inputs, ops, build
+
+    wl = inputs.WORKLOADS[args.workload]
+    if wl.kind != "lite":
+        raise SystemExit("bench.py times the LiteAttention chain workload")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    build.build()
+    ops.lib()
+    B, H, N, d, block, eps = wl.B, wl.H, wl.N, wl.d, wl.block, wl.eps
+    nb = wl.nblocks
+    nsteps = args.warmup + args.steps
+
+    # Per-step inputs, drawn on the device before timing (the chain's drift).
+    q0, k0, v0 = inputs.rff_qkv(wl, device=dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(wl.seed + 1 + 1000 * rank)
+    qkv = [(q0, k0, v0)]
+    for s in range(1, nsteps):
+        q, k, v = qkv[-1]
+        qkv.append((inputs.drift(q, g), inputs.drift(k, g), inputs.drift(v, g)))
+    skips = [torch.zeros(B, H, nb, nb, dtype=torch.uint8, device=dev) for _ in range(nsteps + 1)]
+    out = torch.empty_like(q0)
+    stream = torch.cuda.current_stream(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nsteps)]
+
+    def step(s):
+        q, k, v = qkv[s]
+        ev[s][0].record(stream)
+        ops.sa_sparse_attn_fwd(q, k, v, block, mask=None, skip_in=skips[s], skip_out=skips[s + 1], eps=eps,
+                               out=out, stream=stream)
+        ev[s][1].record(stream)
+
+    for s in range(args.warmup):
+        step(s)
+    ops.sa_get_device_status(stream)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(local)
+    clocks.start()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for s in range(args.warmup, nsteps):
+        step(s)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    if world > 1:
+        torch.distributed.barrier()
+    ops.sa_get_device_status(stream)
+    total_ms = t0.elapsed_time(t1)
+    kern_ms = [ev[s][0].elapsed_time(ev[s][1]) for s in range(args.warmup, nsteps)]
+    flops = [executed_flops(skips[s], N, block, d) for s in range(args.warmup, nsteps)]
+    dense = 4.0 * d * N * N * B * H
+    my = torch.tensor([total_ms, sum(flops)], dtype=torch.float64, device=dev)
+    if world > 1:
+        t = my[:1].clone()
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        f = my[1:].clone()
+        torch.distributed.all_reduce(f, op=torch.distributed.ReduceOp.SUM)
+        total_ms_max, flops_all = float(t.item()), float(f.item())
+    else:
+        total_ms_max, flops_all = total_ms, sum(flops)
+
+    # end-to-end through the public API with host buffers (rank-local)
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(ops, qkv[0], block, eps, nb, dev, stream, args.e2e_steps, world)
+
+    del qkv
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        q, k, v = (t[:, :1].cpu() for t in (q0, k0, v0))
+        cpu = cpu_sample(q, k, v, block, eps, args.cpu_seconds)
+
+    if rank != 0:
+        return None
+    peaks, src = load_peaks()
+    achieved = sum(flops) / (sum(kern_ms) * 1e-3) / 1e12
+    peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+    skip_rate = 1.0 - sum(flops) / (dense * len(flops))
+    line = {
+        "metric": METRIC,
+        "value": round(flops_all / (total_ms_max * 1e-3) / 1e12, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(total_ms_max / args.steps, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded random-Fourier-feature locality generator + denoising drift, drawn on device)",
+        "config": {"workload": wl.name, "B": B, "H": H, "N": N, "grid": [wl.T, wl.Hh, wl.Ww], "d": d,
+                   "block": block, "eps": eps, "mask": "all kept + LiteAttention skip chain",
+                   "l2": "inputs larger than L2 (3 x 774 MB per step)", "parallelism": f"replicas x{world}"},
+        "ms_per_call": round(statistics.median(kern_ms), 3),
+        "density": round(1.0 - skip_rate, 6),
+        "executed_tflops": round(achieved, 2),
+        "dense_equiv_tflops": round(dense / (statistics.median(kern_ms) * 1e-3) / 1e12, 2),
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "peak_source": f"{src} bf16_tflops_sustained",
+                     "frac_of_burst": round(achieved / float(peaks["bf16_tflops"]), 4), "traffic": None},
+        "gpu_launches": args.steps,
+        "clocks": clk,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+    }
+    return line
+
+
+def run_e2e(ops, qkv0, block, eps, nb, dev, stream, steps, world):
+    """Same metric through the public API with pinned host buffers: H2D of Q/K/V,
+    the attention call, D2H of O, every step inside the timed region."""
+    q0, k0, v0 = qkv0
+    B, H, N, d = q0.shape
+    hq, hk, hv = (t.cpu().pin_memory() for t in (q0, k0, v0))
+    ho = torch.empty_like(hq).pin_memory()
+    dq, dk, dv = (torch.empty_like(q0) for _ in range(3))
+    do = torch.empty_like(q0)
+    skips = [torch.zeros(B, H, nb, nb, dtype=torch.uint8, device=dev) for _ in range(steps + 2)]
+
+    def one(s):
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        ops.sa_sparse_attn_fwd(dq, dk, dv, block, skip_in=skips[s], skip_out=skips[s + 1], eps=eps, out=do,
+                               stream=stream)
+        ho.copy_(do, non_blocking=True)
+
+    one(0)
+    torch.cuda.synchronize(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for s in range(1, steps + 1):
+        one(s)
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = a.elapsed_time(b)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    flops = sum(executed_flops(skips[s], N, block, d) for s in range(1, steps + 1)) * world
+    return {"value": round(flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+            "h2d_bytes_per_step": 3 * q0.numel() * 2, "d2h_bytes_per_step": q0.numel() * 2,
+            "ms_per_step": round(ms / steps, 3), "steps": steps}
+
+
+# ------------------------------------------------------------ oracle timing ---
+
+def cpu_sample(q, k, v, block, eps, seconds):
+    """Time the fp64 oracle's lite_step on q-blocks of head 0, step 0, for about
+    `seconds` of host time; report its executed TFLOP/s."""
+    import numpy as np
+    from threadpoolctl import threadpool_info
+    import oracle
+
+    N, d = q.shape[2], q.shape[3]
+    nb = -(-N // block)
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    order = list(range(0, nb, max(1, nb // 64)))
+    done, flops = 0, 0.0
+    t0 = time.perf_counter()
+    for i in order:
+        oracle.lite_step(q, k, v, block, None, None, eps, qblocks=[(0, 0, i)])
+        rows = min(block, N - i * block)
+        flops += 4.0 * d * rows * N
+        done += 1
+        if time.perf_counter() - t0 > seconds:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"{done} q-blocks of head 0 at denoising step 0 (all {N} keys each), {dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    """The oracle as the reference arm: each step a bounded sample of the workload."""
+    from block_sparse_attention_flash_b200 import inputs
+
+    if rank != 0:
+        return None
+    wl = inputs.WORKLOADS[args.workload]
+    q, k, v = inputs.rff_qkv(wl, H=1)
+    per_step = max(1.0, args.ref_seconds / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        cpu_sample(q, k, v, wl.block, wl.eps, per_step)
+    vals = []
+    t0 = time.perf_counter()
+    last = None
+    for _ in range(args.steps):
+        last = cpu_sample(q, k, v, wl.block, wl.eps, per_step)
+        vals.append(last["value"])
+    dt = time.perf_counter() - t0
+    value = statistics.mean(vals)
+    return {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(dt * 1e3 / max(1, args.steps), 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded random-Fourier-feature locality generator)", "impl": "reference",
+            "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "N": wl.N, "d": wl.d, "block": wl.block,
+                       "eps": wl.eps},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": last["cores"], "kind": "oracle",
+                             "sample": last["sample"]},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="wan14b_720p_lite")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-seconds", type=float, default=60.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+    else:
+        if world > 1:
+            import datetime
+            torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                                 device_id=torch.device("cuda", local))
+        line = run_ours(args, rank, world, local)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,287 @@
+// sa_lib.cu — host side of the C ABI declared in include/sparse_attn.h.
+//
+// One translation unit holds every kernel (included below) so that the
+// per-device error word is a single __device__ variable.  Host code only
+// validates arguments, encodes TMA tensor maps, picks the kernel instance and
+// launches it on the caller's stream; all arithmetic runs on the GPU.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "sa_attn_fwd.cuh"
+#include "sa_common.cuh"
+#include "sa_masks.cuh"
+#include "sparse_attn.h"
+
+namespace {
+
+using sa::AttnParams;
+
+constexpr int kMaxDevices = 64;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+int ceil_div(long long a, long long b) { return static_cast<int>((a + b - 1) / b); }
+cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+sa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SA_OK : SA_ERR_CUDA; }
+
+// ---------------------------------------------------------- tensor maps ---
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// [B*H, rows, D] bf16 viewed as a 3D tensor (D innermost), 64 x 128 x 1 boxes,
+// 128-byte swizzle, zero fill outside the tensor.
+bool encode_rows_map(CUtensorMap* map, const void* base, int BH, int rows, int D, int box_rows) {
+  auto fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(rows) * D * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ----------------------------------------------- per-device kernel set-up ---
+struct DeviceInit {
+  std::once_flag flag;
+  cudaError_t err = cudaSuccess;
+};
+DeviceInit g_dev_init[kMaxDevices];
+
+cudaError_t init_device_kernels() {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  DeviceInit& di = g_dev_init[dev];
+  std::call_once(di.flag, [&di] {
+    cudaError_t r = cudaSuccess;
+    auto set = [&r](const void* fn, int bytes) {
+      if (r == cudaSuccess) r = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    };
+    set(reinterpret_cast<const void*>(&sa::attn_fwd_kernel<128, 128>), sa::AttnSmem<128>::kAlloc);
+    set(reinterpret_cast<const void*>(&sa::attn_fwd_kernel<128, 64>), sa::AttnSmem<128>::kAlloc);
+    set(reinterpret_cast<const void*>(&sa::attn_fwd_kernel<64, 128>), sa::AttnSmem<64>::kAlloc);
+    set(reinterpret_cast<const void*>(&sa::attn_fwd_kernel<64, 64>), sa::AttnSmem<64>::kAlloc);
+    set(reinterpret_cast<const void*>(&sa::block_select_kernel),
+        static_cast<int>(sa::select_smem_bytes(sa::kMaxSelect)));
+    di.err = r;
+  });
+  return di.err;
+}
+
+bool valid_dim(int d) { return d == 64 || d == 128; }
+bool valid_block(int b) { return b == 64 || b == 128; }
+
+}  // namespace
+
+extern "C" {
+
+const char* sa_status_string(sa_status s) {
+  switch (s) {
+    case SA_OK: return "SA_OK";
+    case SA_ERR_INVALID_ARG: return "SA_ERR_INVALID_ARG";
+    case SA_ERR_UNSUPPORTED: return "SA_ERR_UNSUPPORTED";
+    case SA_ERR_CUDA: return "SA_ERR_CUDA";
+    case SA_ERR_TIMEOUT: return "SA_ERR_TIMEOUT";
+  }
+  return "SA_ERR_UNKNOWN";
+}
+
+int sa_version(void) { return 100; }
+
+sa_status sa_get_device_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(as_stream(stream));
+  if (e != cudaSuccess) return SA_ERR_CUDA;
+  int word = 0;
+  e = cudaMemcpyFromSymbol(&word, sa::g_error_word, sizeof(int));
+  if (e != cudaSuccess) return SA_ERR_CUDA;
+  if (word != 0) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(sa::g_error_word, &zero, sizeof(int));
+    if (e != cudaSuccess) return SA_ERR_CUDA;
+  }
+  if (word & (1 << SA_ERR_TIMEOUT)) return SA_ERR_TIMEOUT;
+  return word ? SA_ERR_CUDA : SA_OK;
+}
+
+size_t sa_build_mask_workspace(int B, int H, int N, int d, int block) {
+  if (B <= 0 || H <= 0 || N <= 0 || d <= 0 || block <= 0) return 0;
+  const size_t nb = static_cast<size_t>(ceil_div(N, block));
+  const size_t bh = static_cast<size_t>(B) * H;
+  return (2 * bh * nb * d + bh * nb * nb) * sizeof(float);
+}
+
+sa_status sa_build_mask(const void* q, const void* k, int B, int H, int N, int d, int block, int mode, float tau,
+                        const float* level_frac, uint8_t* mask_out, float* scores_out, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  if (B < 0 || H < 0 || N < 0) return SA_ERR_INVALID_ARG;
+  if (mode != SA_MASK_TAU && mode != SA_MASK_LEVELS) return SA_ERR_INVALID_ARG;
+  if (mode == SA_MASK_TAU && !(tau > 0.f && tau <= 1.f)) return SA_ERR_INVALID_ARG;
+  int c0 = 0, c1 = 0, c2 = 0;
+  if (B == 0 || H == 0 || N == 0) return SA_OK;
+  if (!valid_dim(d) || !valid_block(block)) return SA_ERR_UNSUPPORTED;
+  if (!q || !k || !mask_out || !workspace) return SA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return SA_ERR_INVALID_ARG;
+  const int nb = ceil_div(N, block);
+  if (nb > sa::kMaxSelect) return SA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * H > 65535) return SA_ERR_UNSUPPORTED;
+  if (workspace_bytes < sa_build_mask_workspace(B, H, N, d, block)) return SA_ERR_INVALID_ARG;
+  if (mode == SA_MASK_LEVELS) {
+    if (!level_frac) return SA_ERR_INVALID_ARG;
+    float prev = 0.f;
+    for (int i = 0; i < 3; ++i) {
+      const float f = level_frac[i];
+      if (!(f >= prev && f <= 1.f)) return SA_ERR_INVALID_ARG;
+      prev = f;
+    }
+    c0 = static_cast<int>(std::ceil(static_cast<double>(level_frac[0]) * nb - 1e-9));
+    c1 = static_cast<int>(std::ceil(static_cast<double>(level_frac[1]) * nb - 1e-9));
+    c2 = static_cast<int>(std::ceil(static_cast<double>(level_frac[2]) * nb - 1e-9));
+  }
+  cudaError_t e = init_device_kernels();
+  if (e != cudaSuccess) return SA_ERR_CUDA;
+  const int BH = B * H;
+  float* qmean = static_cast<float*>(workspace);
+  float* kmean = qmean + static_cast<size_t>(BH) * nb * d;
+  float* scores = scores_out ? scores_out : kmean + static_cast<size_t>(BH) * nb * d;
+  cudaStream_t s = as_stream(stream);
+  const float scale = 1.0f / std::sqrt(static_cast<float>(d));
+  const auto* qb = static_cast<const __nv_bfloat16*>(q);
+  const auto* kb = static_cast<const __nv_bfloat16*>(k);
+  dim3 g1(nb, BH, 2), g2(ceil_div(nb, 32), ceil_div(nb, 32), BH);
+  if (d == 128) {
+    sa::block_means_kernel<128><<<g1, 128, 0, s>>>(qb, kb, N, block, nb, qmean, kmean);
+    sa::block_scores_kernel<128><<<g2, 256, 0, s>>>(qmean, kmean, nb, scale, scores);
+  } else {
+    sa::block_means_kernel<64><<<g1, 128, 0, s>>>(qb, kb, N, block, nb, qmean, kmean);
+    sa::block_scores_kernel<64><<<g2, 256, 0, s>>>(qmean, kmean, nb, scale, scores);
+  }
+  sa::block_select_kernel<<<static_cast<unsigned>(BH) * nb, sa::kSelectThreads, sa::select_smem_bytes(nb), s>>>(
+      scores, nb, mode, tau, c0, c1, c2, mask_out);
+  return cuda_status(cudaGetLastError());
+}
+
+sa_status sa_radial_mask(int T, int Hh, int Ww, int block, uint8_t* mask_out, void* stream) {
+  if (T < 0 || Hh < 0 || Ww < 0 || block <= 0) return SA_ERR_INVALID_ARG;
+  const long long N = static_cast<long long>(T) * Hh * Ww;
+  if (N == 0) return SA_OK;
+  if (!mask_out) return SA_ERR_INVALID_ARG;
+  if (N > (1ll << 30)) return SA_ERR_UNSUPPORTED;
+  const int nb = ceil_div(N, block);
+  const int F = Hh * Ww;
+  const int S = ceil_div(F, block);
+  sa::radial_mask_kernel<<<nb, 256, 0, as_stream(stream)>>>(nb, F, block, S, mask_out);
+  return cuda_status(cudaGetLastError());
+}
+
+sa_status sa_pyramid_pool(const void* k, const void* v, int B, int H, int N, int d, int block, void* const* k_pool,
+                          void* const* v_pool, void* stream) {
+  if (B < 0 || H < 0 || N < 0) return SA_ERR_INVALID_ARG;
+  if (B == 0 || H == 0 || N == 0) return SA_OK;
+  if (!valid_dim(d) || !valid_block(block)) return SA_ERR_UNSUPPORTED;
+  if (!k || !v || !k_pool || !v_pool) return SA_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v)) return SA_ERR_INVALID_ARG;
+  for (int i = 0; i < 3; ++i)
+    if (!k_pool[i] || !v_pool[i] || !aligned16(k_pool[i]) || !aligned16(v_pool[i])) return SA_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * H > 65535) return SA_ERR_UNSUPPORTED;
+  const int BH = B * H;
+  auto kp = [&](int i) { return static_cast<__nv_bfloat16*>(k_pool[i]); };
+  auto vp = [&](int i) { return static_cast<__nv_bfloat16*>(v_pool[i]); };
+  const auto* kb = static_cast<const __nv_bfloat16*>(k);
+  const auto* vb = static_cast<const __nv_bfloat16*>(v);
+  cudaStream_t s = as_stream(stream);
+  if (d == 128) {
+    dim3 g(ceil_div(N, 8 * 8), BH, 2);
+    sa::pyramid_pool_kernel<128><<<g, 128, 0, s>>>(kb, vb, N, kp(0), kp(1), kp(2), vp(0), vp(1), vp(2));
+  } else {
+    dim3 g(ceil_div(N, 8 * 16), BH, 2);
+    sa::pyramid_pool_kernel<64><<<g, 128, 0, s>>>(kb, vb, N, kp(0), kp(1), kp(2), vp(0), vp(1), vp(2));
+  }
+  return cuda_status(cudaGetLastError());
+}
+
+sa_status sa_sparse_attn_fwd(const void* q, const void* k, const void* v, int B, int H, int N, int d, int block,
+                             const uint8_t* mask, int64_t mask_sb, int64_t mask_sh, int64_t mask_si,
+                             const uint8_t* skip_in, uint8_t* skip_out, float eps, float scale, void* o,
+                             float* lse, void* stream) {
+  if (B < 0 || H < 0 || N < 0) return SA_ERR_INVALID_ARG;
+  if (std::isnan(eps) || eps < 0.f) return SA_ERR_INVALID_ARG;
+  if (std::isnan(scale) || scale < 0.f || std::isinf(scale)) return SA_ERR_INVALID_ARG;
+  if (B == 0 || H == 0 || N == 0) return SA_OK;
+  if (!valid_dim(d) || !valid_block(block)) return SA_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !o) return SA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return SA_ERR_INVALID_ARG;
+  if (mask && (mask_sb < 0 || mask_sh < 0 || mask_si < 0)) return SA_ERR_INVALID_ARG;
+  const int n_kv_tiles = ceil_div(N, sa::kTileN);
+  if (n_kv_tiles > sa::kMaxKvTiles) return SA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * H > 65535) return SA_ERR_UNSUPPORTED;
+  cudaError_t e = init_device_kernels();
+  if (e != cudaSuccess) return SA_ERR_CUDA;
+
+  const int BH = B * H;
+  CUtensorMap tq, tk, tv;
+  if (!encode_rows_map(&tq, q, BH, N, d, sa::kTileM) || !encode_rows_map(&tk, k, BH, N, d, sa::kTileN) ||
+      !encode_rows_map(&tv, v, BH, N, d, sa::kTileN))
+    return SA_ERR_CUDA;
+
+  if (scale == 0.f) scale = 1.0f / std::sqrt(static_cast<float>(d));
+  AttnParams p;
+  p.B = B;
+  p.H = H;
+  p.N = N;
+  p.nb = ceil_div(N, block);
+  p.n_kv_tiles = n_kv_tiles;
+  p.mask = mask;
+  p.msb = mask_sb;
+  p.msh = mask_sh;
+  p.msi = mask_si;
+  p.skip_in = skip_in;
+  p.skip_out = skip_out;
+  p.write_skip = skip_out != nullptr;
+  p.carry_skip = skip_out != nullptr && skip_out != skip_in;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.eps_raw = std::isinf(eps) ? INFINITY : eps / scale;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+
+  const int n_pairs = ceil_div(ceil_div(N, sa::kTileM), 2);
+  dim3 grid(n_pairs, BH);
+  cudaStream_t s = as_stream(stream);
+  if (d == 128 && block == 128)
+    sa::attn_fwd_kernel<128, 128><<<grid, sa::kAttnThreads, sa::AttnSmem<128>::kAlloc, s>>>(tq, tk, tv, p);
+  else if (d == 128 && block == 64)
+    sa::attn_fwd_kernel<128, 64><<<grid, sa::kAttnThreads, sa::AttnSmem<128>::kAlloc, s>>>(tq, tk, tv, p);
+  else if (d == 64 && block == 128)
+    sa::attn_fwd_kernel<64, 128><<<grid, sa::kAttnThreads, sa::AttnSmem<64>::kAlloc, s>>>(tq, tk, tv, p);
+  else
+    sa::attn_fwd_kernel<64, 64><<<grid, sa::kAttnThreads, sa::AttnSmem<64>::kAlloc, s>>>(tq, tk, tv, p);
+  return cuda_status(cudaGetLastError());
+}
+
+sa_status sa_pyramid_attn_fwd(const void* q, const void* k, const void* v, int B, int H, int N, int d, int block,
+                              const uint8_t* levels, int64_t lv_sb, int64_t lv_sh, int64_t lv_si,
+                              const void* const* k_pool, const void* const* v_pool, float scale, void* o, float* lse,
+                              void* stream) {
+  (void)q; (void)k; (void)v; (void)B; (void)H; (void)N; (void)d; (void)block; (void)levels;
+  (void)lv_sb; (void)lv_sh; (void)lv_si; (void)k_pool; (void)v_pool; (void)scale; (void)o; (void)lse; (void)stream;
+  return SA_ERR_UNSUPPORTED;
+}
+
+}  // extern "C"

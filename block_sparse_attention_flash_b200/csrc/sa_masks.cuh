@@ -1,0 +1,365 @@
+// sa_masks.cuh — block-mask construction and pyramid pooling kernels.
+//
+//   radial_mask_kernel     static radial mask (Radial Attention page, static
+//                          exponential-decay mask paragraphs)
+//   block_means_kernel     mean of each token block of Q and K (VMoBA write-up,
+//                          block scoring with pooled queries/keys)
+//   block_scores_kernel    S_ij = scale * qbar_i . kbar_j (one small fp32 GEMM
+//                          per head)
+//   block_select_kernel    per q-block row: tau-mass selection (VMoBA write-up,
+//                          threshold dynamic selection) or PSA level quotas
+//                          (PSA page, multi-level mask generator)
+//   pyramid_pool_kernel    mean of 2, 4, 8 consecutive tokens (PSA page,
+//                          pyramid KV by progressive average pooling)
+//
+// The readers are HBM-bound; loads are 16-byte vectors, consecutive threads
+// read consecutive 16-byte chunks of a row, and each thread keeps several rows
+// in flight before it reduces.
+#pragma once
+
+#include "sa_common.cuh"
+
+namespace sa {
+
+// ------------------------------------------------------------ radial mask ---
+__global__ void radial_mask_kernel(int nb, int F, int block, int S, uint8_t* __restrict__ out) {
+  const int i = blockIdx.x;
+  const long long fi_tok = static_cast<long long>(i) * block;
+  const int fi = static_cast<int>(fi_tok / F);
+  const int pi = static_cast<int>((fi_tok % F) / block);
+  for (int j = threadIdx.x; j < nb; j += blockDim.x) {
+    const long long fj_tok = static_cast<long long>(j) * block;
+    const int fj = static_cast<int>(fj_tok / F);
+    const int pj = static_cast<int>((fj_tok % F) / block);
+    const int dt = abs(fi - fj);
+    uint8_t keep;
+    if (dt <= 1) {
+      keep = 1;
+    } else {
+      const int k = 31 - __clz(dt);  // floor(log2 dt)
+      keep = (static_cast<long long>(abs(pi - pj)) << k) < static_cast<long long>(S) ? 1 : 0;
+    }
+    out[static_cast<size_t>(i) * nb + j] = keep;
+  }
+}
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float* f) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 v = __bfloat1622float2(h[i]);
+    f[2 * i] = v.x;
+    f[2 * i + 1] = v.y;
+  }
+}
+
+// ------------------------------------------------------------ block means ---
+// grid (nb, B*H, 2): z = 0 averages Q, z = 1 averages K.  128 threads: thread
+// (rg, ch) sums 16-byte chunk ch of rows rg, rg + RG, ...; smem reduces over rg.
+template <int D>
+__global__ void __launch_bounds__(128) block_means_kernel(const __nv_bfloat16* __restrict__ q,
+                                                          const __nv_bfloat16* __restrict__ k, int N, int block,
+                                                          int nb, float* __restrict__ qmean,
+                                                          float* __restrict__ kmean) {
+  constexpr int CH = D / 8;      // 16-byte chunks per row
+  constexpr int RG = 128 / CH;   // row groups
+  __shared__ float red[RG][D];
+  const int i = blockIdx.x, bh = blockIdx.y, z = blockIdx.z;
+  const __nv_bfloat16* x = (z == 0 ? q : k) + (static_cast<size_t>(bh) * N + static_cast<size_t>(i) * block) * D;
+  const int rows = min(block, N - i * block);
+  const int ch = threadIdx.x % CH, rg = threadIdx.x / CH;
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+  int r = rg;
+  for (; r + 3 * RG < rows; r += 4 * RG) {
+    uint4 u[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) u[j] = __ldg(reinterpret_cast<const uint4*>(x + static_cast<size_t>(r + j * RG) * D) + ch);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float f[8];
+      bf16x8_to_f32(u[j], f);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] += f[e];
+    }
+  }
+  for (; r < rows; r += RG) {
+    float f[8];
+    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(x + static_cast<size_t>(r) * D) + ch), f);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] += f[e];
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) red[rg][ch * 8 + e] = acc[e];
+  __syncthreads();
+  for (int c = threadIdx.x; c < D; c += 128) {
+    float s = 0.f;
+#pragma unroll
+    for (int g = 0; g < RG; ++g) s += red[g][c];
+    float* out = (z == 0 ? qmean : kmean) + (static_cast<size_t>(bh) * nb + i) * D;
+    out[c] = s / static_cast<float>(rows);
+  }
+}
+
+// ----------------------------------------------------------- block scores ---
+// grid (ceil(nb/32), ceil(nb/32), B*H), 256 threads; each thread 4 outputs of
+// a 32 x 32 tile of S = scale * Qbar Kbar^T, fp32 throughout.
+template <int D>
+__global__ void __launch_bounds__(256) block_scores_kernel(const float* __restrict__ qmean,
+                                                           const float* __restrict__ kmean, int nb, float scale,
+                                                           float* __restrict__ scores) {
+  __shared__ float sq[32][D + 1];
+  __shared__ float sk[32][D + 1];
+  const int bh = blockIdx.z;
+  const int i0 = blockIdx.y * 32, j0 = blockIdx.x * 32;
+  const float* qm = qmean + static_cast<size_t>(bh) * nb * D;
+  const float* km = kmean + static_cast<size_t>(bh) * nb * D;
+  for (int idx = threadIdx.x; idx < 32 * D; idx += 256) {
+    const int rr = idx / D, c = idx % D;
+    sq[rr][c] = (i0 + rr < nb) ? qm[static_cast<size_t>(i0 + rr) * D + c] : 0.f;
+    sk[rr][c] = (j0 + rr < nb) ? km[static_cast<size_t>(j0 + rr) * D + c] : 0.f;
+  }
+  __syncthreads();
+  const int jj = threadIdx.x & 31;
+  const int ib = (threadIdx.x >> 5) * 4;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+  for (int c = 0; c < D; ++c) {
+    const float kv = sk[jj][c];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) acc[u] = fmaf(sq[ib + u][c], kv, acc[u]);
+  }
+  const int j = j0 + jj;
+  if (j < nb) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + ib + u;
+      if (i < nb) scores[(static_cast<size_t>(bh) * nb + i) * nb + j] = acc[u] * scale;
+    }
+  }
+}
+
+// ---------------------------------------------------------- block select ---
+constexpr int kSelectThreads = 256;
+constexpr int kMaxSelect = 4096;
+
+// Order-preserving map of a float to an unsigned key (larger float -> larger key).
+__device__ __forceinline__ uint32_t float_order_key(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float block_reduce_max(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  __syncthreads();
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  v = (l < kSelectThreads / 32) ? red[l] : -__int_as_float(0x7f800000);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ float block_reduce_sum(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  __syncthreads();
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  v = (l < kSelectThreads / 32) ? red[l] : 0.f;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__host__ __device__ inline int select_pow2(int nb) {
+  int P = 32;
+  while (P < nb) P <<= 1;
+  return P;
+}
+__host__ __device__ inline size_t select_smem_bytes(int nb) {
+  return static_cast<size_t>(select_pow2(nb)) * 13;
+}
+
+// One CTA per (b, h, i).  Keys (descending score, then ascending j) are
+// bitonic-sorted in shared memory; TAU mode takes an exclusive prefix sum of
+// the probabilities in that order, LEVELS mode uses the rank directly.
+__global__ void __launch_bounds__(kSelectThreads) block_select_kernel(const float* __restrict__ scores, int nb,
+                                                                      int mode, float tau, int c0, int c1, int c2,
+                                                                      uint8_t* __restrict__ mask_out) {
+  // dynamic shared memory: keys[P] (8 B), prob[P] (4 B), out_row[P] (1 B)
+  extern __shared__ unsigned long long select_smem[];
+  __shared__ float red[32];
+  __shared__ float part[kSelectThreads];
+  int P = 32;
+  while (P < nb) P <<= 1;
+  unsigned long long* keys = select_smem;
+  float* prob = reinterpret_cast<float*>(keys + P);
+  uint8_t* out_row = reinterpret_cast<uint8_t*>(prob + P);
+  const size_t row = blockIdx.x;
+  const float* srow = scores + row * nb;
+
+  float mx = -__int_as_float(0x7f800000);
+  for (int j = threadIdx.x; j < P; j += kSelectThreads) {
+    if (j < nb) {
+      const float sc = srow[j];
+      prob[j] = sc;
+      mx = fmaxf(mx, sc);
+      keys[j] = (static_cast<unsigned long long>(~float_order_key(sc)) << 32) | static_cast<unsigned>(j);
+    } else {
+      keys[j] = ~0ull;
+    }
+  }
+  if (mode == SA_MASK_TAU) {
+    mx = block_reduce_max(mx, red);
+    float sum = 0.f;
+    for (int j = threadIdx.x; j < nb; j += kSelectThreads) {
+      const float e = expf(prob[j] - mx);
+      prob[j] = e;
+      sum += e;
+    }
+    sum = block_reduce_sum(sum, red);
+    const float inv = 1.f / sum;
+    for (int j = threadIdx.x; j < nb; j += kSelectThreads) prob[j] *= inv;
+  }
+  __syncthreads();
+
+  // bitonic sort, ascending keys
+  for (int k = 2; k <= P; k <<= 1) {
+    for (int jj = k >> 1; jj > 0; jj >>= 1) {
+      for (int i = threadIdx.x; i < P; i += kSelectThreads) {
+        const int ixj = i ^ jj;
+        if (ixj > i) {
+          const unsigned long long a = keys[i], b = keys[ixj];
+          const bool up = (i & k) == 0;
+          if ((a > b) == up) {
+            keys[i] = b;
+            keys[ixj] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+
+  if (mode == SA_MASK_TAU) {
+    // exclusive scan of prob in sorted order: each thread a contiguous run
+    const int per = (nb + kSelectThreads - 1) / kSelectThreads;
+    const int r0 = threadIdx.x * per, r1 = min(nb, r0 + per);
+    float s = 0.f;
+    for (int r = r0; r < r1; ++r) s += prob[static_cast<unsigned>(keys[r])];
+    part[threadIdx.x] = s;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      // scan of the 256 partial sums by one warp (8 per lane)
+      float v[8];
+      float tot = 0.f;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        v[u] = part[threadIdx.x * 8 + u];
+        tot += v[u];
+      }
+      float inc = tot;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, inc, o);
+        if (threadIdx.x >= o) inc += y;
+      }
+      float run = inc - tot;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float x = v[u];
+        part[threadIdx.x * 8 + u] = run;
+        run += x;
+      }
+    }
+    __syncthreads();
+    float before = part[threadIdx.x];
+    for (int r = r0; r < r1; ++r) {
+      const unsigned j = static_cast<unsigned>(keys[r]);
+      out_row[j] = before < tau ? 1 : 0;
+      before += prob[j];
+    }
+  } else {
+    for (int r = threadIdx.x; r < nb; r += kSelectThreads) {
+      const unsigned j = static_cast<unsigned>(keys[r]);
+      out_row[j] = r < c0 ? 1 : (r < c1 ? 2 : (r < c2 ? 3 : 4));
+    }
+  }
+  __syncthreads();
+  uint8_t* mrow = mask_out + row * nb;
+  for (int j = threadIdx.x; j < nb; j += kSelectThreads) mrow[j] = out_row[j];
+}
+
+// ----------------------------------------------------------- pyramid pool ---
+// grid (ceil(N / (8 * GPB)), B*H, 2); z = 0 pools K, z = 1 pools V.  Thread
+// (g, ch) owns the 8-token group g of the CTA and 16-byte chunk ch: it loads
+// the 8 rows once and writes the c = 2, 4 and 8 means of that chunk.
+template <int D>
+__global__ void __launch_bounds__(128) pyramid_pool_kernel(const __nv_bfloat16* __restrict__ k,
+                                                           const __nv_bfloat16* __restrict__ v, int N,
+                                                           __nv_bfloat16* __restrict__ k2,
+                                                           __nv_bfloat16* __restrict__ k4,
+                                                           __nv_bfloat16* __restrict__ k8,
+                                                           __nv_bfloat16* __restrict__ v2,
+                                                           __nv_bfloat16* __restrict__ v4,
+                                                           __nv_bfloat16* __restrict__ v8) {
+  constexpr int CH = D / 8;
+  constexpr int GPB = 128 / CH;  // 8-token groups per CTA
+  const int bh = blockIdx.y, z = blockIdx.z;
+  const int g = blockIdx.x * GPB + threadIdx.x / CH;
+  const int ch = threadIdx.x % CH;
+  const int r0 = g * 8;
+  if (r0 >= N) return;
+  const int rows = min(8, N - r0);
+  const __nv_bfloat16* x = (z == 0 ? k : v) + (static_cast<size_t>(bh) * N + r0) * D;
+  float f[8][8];
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    if (r < rows) {
+      bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(x + static_cast<size_t>(r) * D) + ch), f[r]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) f[r][e] = 0.f;
+    }
+  }
+  __nv_bfloat16* o2 = z == 0 ? k2 : v2;
+  __nv_bfloat16* o4 = z == 0 ? k4 : v4;
+  __nv_bfloat16* o8 = z == 0 ? k8 : v8;
+  const size_t n2 = (N + 1) / 2, n4 = (N + 3) / 4, n8 = (N + 7) / 8;
+  auto store = [&](__nv_bfloat16* base, size_t nrows, size_t prow, const float* s, float inv) {
+    if (prow >= nrows) return;
+    uint4 w;
+    w.x = pack_bf16x2(s[0] * inv, s[1] * inv);
+    w.y = pack_bf16x2(s[2] * inv, s[3] * inv);
+    w.z = pack_bf16x2(s[4] * inv, s[5] * inv);
+    w.w = pack_bf16x2(s[6] * inv, s[7] * inv);
+    reinterpret_cast<uint4*>(base + (static_cast<size_t>(bh) * nrows + prow) * D)[ch] = w;
+  };
+  float s2[4][8], s4[2][8], s8[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) s2[u][e] = f[2 * u][e] + f[2 * u + 1][e];
+    s4[0][e] = s2[0][e] + s2[1][e];
+    s4[1][e] = s2[2][e] + s2[3][e];
+    s8[e] = s4[0][e] + s4[1][e];
+  }
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int cnt = min(2, max(0, rows - 2 * u));
+    if (cnt > 0) store(o2, n2, static_cast<size_t>(r0 / 2 + u), s2[u], 1.f / cnt);
+  }
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int cnt = min(4, max(0, rows - 4 * u));
+    if (cnt > 0) store(o4, n4, static_cast<size_t>(r0 / 4 + u), s4[u], 1.f / cnt);
+  }
+  store(o8, n8, static_cast<size_t>(r0 / 8), s8, 1.f / rows);
+}
+
+}  // namespace sa

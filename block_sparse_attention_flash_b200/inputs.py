@@ -72,8 +72,8 @@ WORKLOADS = {
 }
 
 
-def _gen(seed: int) -> torch.Generator:
-    g = torch.Generator(device="cpu")
+def _gen(seed: int, device="cpu") -> torch.Generator:
+    g = torch.Generator(device=device)
     g.manual_seed(int(seed))
     return g
 
@@ -86,31 +86,34 @@ def grid_coords(T: int, Hh: int, Ww: int) -> torch.Tensor:
     return torch.stack([t, h, w], dim=-1).reshape(-1, 3)
 
 
-def rff_qkv(wl: Workload, B: Optional[int] = None, H: Optional[int] = None):
+def rff_qkv(wl: Workload, B: Optional[int] = None, H: Optional[int] = None, device="cpu"):
     """Q, K, V bf16 [B, H, N, d] from the locality generator of ``wl``.
 
     Heads are drawn in order from one generator, so a run with fewer heads
     (H smaller than wl.H) yields exactly the first H heads of the full draw.
+    ``device="cuda"`` draws the same recipe with torch's CUDA generator (fast,
+    used for full-size timing runs); its values differ from the CPU draw, and
+    any oracle check of such inputs copies them to the host first.
     """
     B = wl.B if B is None else B
     H = wl.H if H is None else H
     N, d, D = wl.N, wl.d, RFF_FEATURES
-    coords = grid_coords(wl.T, wl.Hh, wl.Ww)
-    g = _gen(wl.seed)
-    q = torch.empty(B, H, N, d, dtype=torch.bfloat16)
+    coords = grid_coords(wl.T, wl.Hh, wl.Ww).to(device)
+    g = _gen(wl.seed, device)
+    q = torch.empty(B, H, N, d, dtype=torch.bfloat16, device=device)
     k = torch.empty_like(q)
     v = torch.empty_like(q)
-    sig = torch.tensor([wl.sigma_t, wl.sigma_s, wl.sigma_s], dtype=torch.float32)
+    sig = torch.tensor([wl.sigma_t, wl.sigma_s, wl.sigma_s], dtype=torch.float32, device=device)
     for b in range(B):
         for h in range(H):
-            omega = torch.randn(3, D, generator=g) / sig.view(3, 1)
-            phase = torch.rand(D, generator=g) * (2.0 * math.pi)
-            W = torch.randn(D, d, generator=g)
+            omega = torch.randn(3, D, generator=g, device=device) / sig.view(3, 1)
+            phase = torch.rand(D, generator=g, device=device) * (2.0 * math.pi)
+            W = torch.randn(D, d, generator=g, device=device)
             phi = torch.cos(coords @ omega + phase) * math.sqrt(2.0 / D)
             L = phi @ W
-            q[b, h] = (0.7 * L + 0.3 * torch.randn(N, d, generator=g)).to(torch.bfloat16)
-            k[b, h] = (0.7 * L + 0.3 * torch.randn(N, d, generator=g)).to(torch.bfloat16)
-            v[b, h] = torch.randn(N, d, generator=g).to(torch.bfloat16)
+            q[b, h] = (0.7 * L + 0.3 * torch.randn(N, d, generator=g, device=device)).to(torch.bfloat16)
+            k[b, h] = (0.7 * L + 0.3 * torch.randn(N, d, generator=g, device=device)).to(torch.bfloat16)
+            v[b, h] = torch.randn(N, d, generator=g, device=device).to(torch.bfloat16)
     return q, k, v
 
 
@@ -138,7 +141,7 @@ def bernoulli_block_mask(B: int, H: int, nqb: int, nkb: int, p: float, seed: int
 
 def drift(x: torch.Tensor, g: torch.Generator) -> torch.Tensor:
     """One denoising-drift step x -> bf16(0.98 x + 0.2 xi), xi ~ N(0,1)."""
-    xi = torch.randn(x.shape, generator=g)
+    xi = torch.randn(x.shape, generator=g, device=x.device)
     return (0.98 * x.float() + 0.2 * xi).to(torch.bfloat16)
 
 

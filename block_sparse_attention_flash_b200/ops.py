@@ -1,0 +1,220 @@
+"""Thin ctypes binding over libsparse_attn.so (argument marshalling only).
+
+Every function here has the name of the C entry point it calls, takes torch
+CUDA tensors, checks dtype / device / contiguity, passes raw device pointers
+and the current CUDA stream, and raises ``SparseAttnError`` on a non-OK
+status.  There is no CPU path: if the library is missing, or a tensor is not
+on a CUDA device, the call fails loudly.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libsparse_attn.so")
+
+SA_OK, SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_CUDA, SA_ERR_TIMEOUT = range(5)
+SA_MASK_TAU, SA_MASK_LEVELS = 0, 1
+
+_vp, _i32, _i64, _f32, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+
+_SIGNATURES = {
+    "sa_status_string": (ctypes.c_char_p, [_i32]),
+    "sa_version": (_i32, []),
+    "sa_get_device_status": (_i32, [_vp]),
+    "sa_build_mask_workspace": (_sz, [_i32, _i32, _i32, _i32, _i32]),
+    "sa_build_mask": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "sa_radial_mask": (_i32, [_i32, _i32, _i32, _i32, _vp, _vp]),
+    "sa_pyramid_pool": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
+    "sa_sparse_attn_fwd": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _i64, _i64, _i64,
+                                  _vp, _vp, _f32, _f32, _vp, _vp, _vp]),
+    "sa_pyramid_attn_fwd": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _i64, _i64, _i64,
+                                   _vp, _vp, _f32, _vp, _vp, _vp]),
+}
+
+_lib = None
+
+
+class SparseAttnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}")
+
+
+def lib() -> ctypes.CDLL:
+    """Load libsparse_attn.so once (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m block_sparse_attention_flash_b200.build`")
+        l = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(l, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = l
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().sa_status_string(status).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != SA_OK:
+        raise SparseAttnError(status, where)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dev(t: torch.Tensor, name: str, dtype: torch.dtype) -> int:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _opt(t: Optional[torch.Tensor], name: str, dtype: torch.dtype) -> Optional[int]:
+    return None if t is None else _dev(t, name, dtype)
+
+
+def _mask_strides(m: torch.Tensor, B: int, H: int, nb: int):
+    """(sb, sh, si) element strides for a [Nb,Nb], [H,Nb,Nb] or [B,H,Nb,Nb] mask."""
+    if m.shape[-1] != nb or m.shape[-2] != nb or m.stride(-1) != 1:
+        raise ValueError(f"mask must end in [{nb}, {nb}] with unit stride, got {tuple(m.shape)}")
+    if m.dim() == 2:
+        return 0, 0, m.stride(0)
+    if m.dim() == 3:
+        if m.shape[0] != H:
+            raise ValueError("3D mask must be [H, Nb, Nb]")
+        return 0, m.stride(0), m.stride(1)
+    if m.dim() == 4 and m.shape[0] == B and m.shape[1] == H:
+        return m.stride(0), m.stride(1), m.stride(2)
+    raise ValueError(f"mask shape {tuple(m.shape)} does not broadcast to [{B}, {H}, {nb}, {nb}]")
+
+
+def nblocks(N: int, block: int) -> int:
+    return -(-N // block)
+
+
+def sa_get_device_status(stream=None) -> None:
+    """Synchronise the stream and raise if a kernel recorded a device-side error."""
+    _check(lib().sa_get_device_status(_stream(stream)), "sa_get_device_status")
+
+
+def sa_radial_mask(T: int, Hh: int, Ww: int, block: int, out: Optional[torch.Tensor] = None,
+                   device=None, stream=None) -> torch.Tensor:
+    nb = nblocks(T * Hh * Ww, block)
+    if out is None:
+        out = torch.empty(nb, nb, dtype=torch.uint8, device=device or "cuda")
+    ptr = _dev(out, "out", torch.uint8)
+    _check(lib().sa_radial_mask(T, Hh, Ww, block, ptr, _stream(stream)), "sa_radial_mask")
+    return out
+
+
+def sa_build_mask_workspace(B: int, H: int, N: int, d: int, block: int) -> int:
+    return int(lib().sa_build_mask_workspace(B, H, N, d, block))
+
+
+def sa_build_mask(q: torch.Tensor, k: torch.Tensor, block: int, mode: str = "tau", tau: float = 0.9,
+                  level_frac: Sequence[float] = (0.1, 0.3, 0.6), mask_out: Optional[torch.Tensor] = None,
+                  scores_out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                  stream=None) -> torch.Tensor:
+    B, H, N, d = q.shape
+    nb = nblocks(N, block)
+    if mask_out is None:
+        mask_out = torch.empty(B, H, nb, nb, dtype=torch.uint8, device=q.device)
+    ws_bytes = sa_build_mask_workspace(B, H, N, d, block)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+    fr = (ctypes.c_float * 3)(*[float(x) for x in level_frac])
+    m = SA_MASK_TAU if mode == "tau" else SA_MASK_LEVELS
+    st = lib().sa_build_mask(_dev(q, "q", torch.bfloat16), _dev(k, "k", torch.bfloat16), B, H, N, d, block, m,
+                             float(tau), ctypes.cast(fr, ctypes.c_void_p), _dev(mask_out, "mask_out", torch.uint8),
+                             _opt(scores_out, "scores_out", torch.float32), _dev(workspace, "workspace", torch.uint8),
+                             workspace.numel(), _stream(stream))
+    _check(st, "sa_build_mask")
+    return mask_out
+
+
+def pool_rows(N: int, c: int) -> int:
+    return -(-N // c)
+
+
+def sa_pyramid_pool(k: torch.Tensor, v: torch.Tensor, block: int, k_pool=None, v_pool=None, stream=None):
+    B, H, N, d = k.shape
+    if k_pool is None:
+        k_pool = [torch.empty(B, H, pool_rows(N, c), d, dtype=k.dtype, device=k.device) for c in (2, 4, 8)]
+    if v_pool is None:
+        v_pool = [torch.empty(B, H, pool_rows(N, c), d, dtype=v.dtype, device=v.device) for c in (2, 4, 8)]
+    kp = (ctypes.c_void_p * 3)(*[_dev(t, "k_pool", torch.bfloat16) for t in k_pool])
+    vp = (ctypes.c_void_p * 3)(*[_dev(t, "v_pool", torch.bfloat16) for t in v_pool])
+    st = lib().sa_pyramid_pool(_dev(k, "k", torch.bfloat16), _dev(v, "v", torch.bfloat16), B, H, N, d, block,
+                               ctypes.cast(kp, ctypes.c_void_p), ctypes.cast(vp, ctypes.c_void_p), _stream(stream))
+    _check(st, "sa_pyramid_pool")
+    return k_pool, v_pool
+
+
+def sa_sparse_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block: int,
+                       mask: Optional[torch.Tensor] = None, skip_in: Optional[torch.Tensor] = None,
+                       skip_out: Optional[torch.Tensor] = None, eps: float = math.inf, scale: float = 0.0,
+                       out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                       stream=None) -> torch.Tensor:
+    """Block-sparse attention forward; returns O (and fills lse / skip_out if given)."""
+    B, H, N, d = q.shape
+    nb = nblocks(N, block)
+    if out is None:
+        out = torch.empty_like(q)
+    sb = sh = si = 0
+    mptr = None
+    if mask is not None:
+        if mask.dtype != torch.uint8 or not mask.is_cuda:
+            raise ValueError("mask must be a CUDA uint8 tensor")
+        sb, sh, si = _mask_strides(mask, B, H, nb)
+        mptr = mask.data_ptr()
+    for name, t in (("skip_in", skip_in), ("skip_out", skip_out)):
+        if t is not None and tuple(t.shape) != (B, H, nb, nb):
+            raise ValueError(f"{name} must be [{B}, {H}, {nb}, {nb}]")
+    st = lib().sa_sparse_attn_fwd(
+        _dev(q, "q", torch.bfloat16), _dev(k, "k", torch.bfloat16), _dev(v, "v", torch.bfloat16),
+        B, H, N, d, block, mptr, sb, sh, si,
+        _opt(skip_in, "skip_in", torch.uint8), _opt(skip_out, "skip_out", torch.uint8),
+        float(eps), float(scale), _dev(out, "out", torch.bfloat16), _opt(lse, "lse", torch.float32),
+        _stream(stream))
+    _check(st, "sa_sparse_attn_fwd")
+    return out
+
+
+def sa_pyramid_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block: int, levels: torch.Tensor,
+                        k_pool, v_pool, scale: float = 0.0, out: Optional[torch.Tensor] = None,
+                        lse: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """PSA multi-level attention forward over a level-code map (0 drop, 1+l level l)."""
+    B, H, N, d = q.shape
+    nb = nblocks(N, block)
+    if out is None:
+        out = torch.empty_like(q)
+    if levels.dtype != torch.uint8 or not levels.is_cuda:
+        raise ValueError("levels must be a CUDA uint8 tensor")
+    sb, sh, si = _mask_strides(levels, B, H, nb)
+    kp = (ctypes.c_void_p * 3)(*[_dev(t, "k_pool", torch.bfloat16) for t in k_pool])
+    vp = (ctypes.c_void_p * 3)(*[_dev(t, "v_pool", torch.bfloat16) for t in v_pool])
+    st = lib().sa_pyramid_attn_fwd(
+        _dev(q, "q", torch.bfloat16), _dev(k, "k", torch.bfloat16), _dev(v, "v", torch.bfloat16),
+        B, H, N, d, block, levels.data_ptr(), sb, sh, si,
+        ctypes.cast(kp, ctypes.c_void_p), ctypes.cast(vp, ctypes.c_void_p), float(scale),
+        _dev(out, "out", torch.bfloat16), _opt(lse, "lse", torch.float32), _stream(stream))
+    _check(st, "sa_pyramid_attn_fwd")
+    return out

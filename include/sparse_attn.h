@@ -1,0 +1,210 @@
+/*
+ * sparse_attn.h — C ABI of the block-sparse video attention library
+ * (libsparse_attn.so, CUDA for sm_100a / B200).
+ *
+ * The library computes non-causal softmax attention over the 3D
+ * (frame x height x width) token grid of a video diffusion transformer, where
+ * only selected (q-block, k-block) tiles are executed.  It has four parts:
+ *   sa_build_mask      mean-pooled block scores -> tau-mass mask or PSA level map
+ *   sa_radial_mask     static radial mask (window halves as frame distance doubles)
+ *   sa_pyramid_pool    PSA pyramid: mean-pooled K/V at 2, 4 and 8 tokens per key
+ *   sa_sparse_attn_fwd FlashAttention-style forward over kept tiles, with the
+ *                      LiteAttention skip-mask update fused in
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are caller-owned DEVICE memory.  Q, K, V and O are bf16,
+ *     contiguous [B, H, N, d] (d fastest), tokens in raster (t, h, w) order:
+ *     n = (t*Hh + h)*Ww + w.  Base pointers must be 16-byte aligned.
+ *   - Blocks are runs of `block` consecutive tokens; Nb = ceil(N / block).
+ *     The last block may be partial; means, maxima and softmax use its valid
+ *     tokens only.
+ *   - Block masks are uint8 [B, H, Nb, Nb] (q-block i, k-block j; j fastest).
+ *   - Every call is asynchronous on `stream` (a cudaStream_t, NULL = legacy
+ *     default stream).  Arguments are validated on the host before any launch;
+ *     a rejected call launches nothing and returns SA_ERR_INVALID_ARG or
+ *     SA_ERR_UNSUPPORTED.  No call falls back to another implementation.
+ *   - Device-side waits are bounded.  A wait that runs out records
+ *     SA_ERR_TIMEOUT in a per-device error word that sa_get_device_status
+ *     reads; the kernel then returns without hanging the GPU.
+ *   - The library allocates no device memory.  Scratch memory is passed in
+ *     by the caller (sa_build_mask's workspace).
+ *
+ * Citations name the web page the operation comes from and its section.
+ */
+#ifndef SPARSE_ATTN_H
+#define SPARSE_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SA_API __attribute__((visibility("default")))
+#else
+#define SA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SA_OK = 0,
+  SA_ERR_INVALID_ARG = 1,   /* bad pointer, alignment, size or value        */
+  SA_ERR_UNSUPPORTED = 2,   /* valid but not built (e.g. d not in {64,128}) */
+  SA_ERR_CUDA = 3,          /* a CUDA runtime call failed                   */
+  SA_ERR_TIMEOUT = 4        /* a device-side bounded wait ran out           */
+} sa_status;
+
+enum { SA_MASK_TAU = 0, SA_MASK_LEVELS = 1 };
+
+/* Human-readable name of a status code (static string, never NULL). */
+SA_API const char* sa_status_string(sa_status s);
+
+/* Library version, major*10000 + minor*100 + patch. */
+SA_API int sa_version(void);
+
+/*
+ * sa_get_device_status — synchronise `stream`, then read and clear the
+ * current device's error word.  Returns SA_OK, SA_ERR_TIMEOUT (a kernel's
+ * bounded wait ran out; its outputs are undefined) or SA_ERR_CUDA (the
+ * synchronisation itself failed).
+ */
+SA_API sa_status sa_get_device_status(void* stream);
+
+/*
+ * sa_build_mask_workspace — bytes of device scratch sa_build_mask needs:
+ * the fp32 block means of Q and K (2 * B*H*Nb*d floats) plus the fp32 block
+ * scores (B*H*Nb*Nb floats).  The caller allocates it (any 256-byte aligned
+ * buffer of at least this size).
+ */
+SA_API size_t sa_build_mask_workspace(int B, int H, int N, int d, int block);
+
+/*
+ * sa_build_mask — dynamic block mask from mean-pooled block scores.
+ *   VMoBA write-up (arXiv 2506.23858), "threshold dynamic selection" and
+ *   "global block selection" paragraphs: block importance from pooled
+ *   query/key blocks scored with one matrix product, blocks kept until the
+ *   selected attention mass reaches a threshold; PSA page (arXiv 2512.04025),
+ *   multi-level mask generator paragraph, for SA_MASK_LEVELS.
+ *
+ * Computes q_i = mean of Q rows in block i, k_j likewise (fp32), the score
+ * S_ij = q_i . k_j / sqrt(d), then per row (b, h, i):
+ *   SA_MASK_TAU:    P_i = softmax_j(S_i); visit j by descending S (ties: lower
+ *                   j first); mask[j] = 1 iff the mass of the blocks visited
+ *                   before j is < tau (the block that crosses tau is kept).
+ *   SA_MASK_LEVELS: rank r_j of S_ij in the same order; with quotas
+ *                   c_l = ceil(level_frac[l] * Nb) (cumulative fractions,
+ *                   non-decreasing), code = 1 if r < c_0, 2 if r < c_1,
+ *                   3 if r < c_2, else 4 (code = pyramid level + 1).
+ * Arguments
+ *   q, k        bf16 [B,H,N,d] device, read only.
+ *   tau         (0, 1]; used for SA_MASK_TAU.
+ *   level_frac  HOST pointer to 3 floats in [0,1]; used for SA_MASK_LEVELS.
+ *   mask_out    uint8 [B,H,Nb,Nb] device, written in full.
+ *   scores_out  optional fp32 [B,H,Nb,Nb] device (NULL: kept in workspace).
+ *   workspace   device scratch of sa_build_mask_workspace() bytes.
+ * Limits: d in {64,128}, block in {64,128}, Nb <= 4096.
+ */
+SA_API sa_status sa_build_mask(const void* q, const void* k, int B, int H, int N, int d, int block,
+                        int mode, float tau, const float* level_frac,
+                        uint8_t* mask_out, float* scores_out,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * sa_radial_mask — static radial mask for a T x Hh x Ww grid.
+ *   "MIT实验室推出Radial Attention" (arXiv 2506.19852), spatio-temporal energy
+ *   decay and static-mask paragraphs: attention concentrates on nearby frames,
+ *   the spatial window shrinks exponentially with temporal distance, and the
+ *   mask is precomputed once (O(n log n) kept pairs).
+ *
+ * Block i's frame f_i and in-frame block position p_i are those of its first
+ * token (f = floor(i*block / F), p = floor((i*block mod F) / block),
+ * F = Hh*Ww), S = ceil(F / block).  mask[i][j] = 1 iff |f_i - f_j| <= 1 or
+ * |p_i - p_j| < S / 2^floor(log2 |f_i - f_j|).
+ *   mask_out  uint8 [Nb, Nb] device (broadcast over B and H by passing
+ *             batch/head strides of 0 to sa_sparse_attn_fwd).
+ */
+SA_API sa_status sa_radial_mask(int T, int Hh, int Ww, int block, uint8_t* mask_out, void* stream);
+
+/*
+ * sa_pyramid_pool — PSA pyramid KV construction.
+ *   PSA page ("浙江大学突破视频AI瓶颈:金字塔方法提升视频AI效率10倍",
+ *   arXiv 2512.04025), pyramid KV paragraph: the bottom level keeps the
+ *   original keys/values, each level up is an average pooling of the one below.
+ *
+ * For c in {2, 4, 8} (level 1, 2, 3): pooled[g] = mean of rows c*g ..
+ * min(N, c*g+c)-1 (fp32 sum of the bf16 inputs, rounded to bf16).  Groups
+ * never cross a block edge because block is a multiple of 8.
+ *   k, v            bf16 [B,H,N,d] device, read only.
+ *   k_pool, v_pool  HOST arrays of 3 device pointers, each bf16
+ *                   [B,H,ceil(N/c),d] for c = 2, 4, 8.
+ */
+SA_API sa_status sa_pyramid_pool(const void* k, const void* v, int B, int H, int N, int d, int block,
+                          void* const* k_pool, void* const* v_pool, void* stream);
+
+/*
+ * sa_sparse_attn_fwd — block-sparse attention forward with the LiteAttention
+ * skip update.
+ *   Block-sparse keep/drop attention: PSA page, block-sparse attention
+ *   paragraph.  Skip rule and persistent skip mask: LiteAttention write-up
+ *   (arXiv 2511.11062), sections 3 (full-iteration skips), 5 (skip condition)
+ *   and 6 (persistent tile-level skip mask; producer loads only non-skipped
+ *   tiles; per-warp recording with the cross-warp reduction at kernel end).
+ *
+ * For each row r of q-block i:  O_r = sum_c softmax(s_rc) v_c over the key
+ * columns c of every k-block j with mask[b,h,i,j] != 0 and skip_in[b,h,i,j]
+ * == 0, where s_rc = scale * q_r . k_c.  LSE_r = ln sum_c exp(s_rc).  A row
+ * with no visited block gets O = 0 and LSE = -inf.
+ * Skip update (only when skip_out != NULL): visited k-blocks are taken in
+ * ascending j; block j (not the first visited) gets skip_out = 1 iff
+ * max_c s_rc over block j < (running max of row r over the blocks visited
+ * before j) - eps for every valid row r of the q-block.  Block j still
+ * contributes to this call's O.  Every other byte of the row is written as
+ * skip_in's byte (0 when skip_in is NULL), so skip_out = skip_in | new bits;
+ * skip_out may alias skip_in.
+ * Arguments
+ *   q, k, v       bf16 [B,H,N,d] device.
+ *   mask          uint8 device, element (b,h,i,j) at b*mask_sb + h*mask_sh +
+ *                 i*mask_si + j; strides of 0 broadcast (e.g. a radial mask
+ *                 [Nb,Nb]: 0, 0, Nb).  NULL keeps every block.  Any nonzero
+ *                 byte keeps the block at full resolution.
+ *   skip_in       NULL or uint8 [B,H,Nb,Nb] device.
+ *   skip_out      NULL or uint8 [B,H,Nb,Nb] device (may equal skip_in).
+ *   eps           skip threshold in natural-log logit units (>= 0; +inf
+ *                 never skips).
+ *   scale         logit scale; 0 selects 1/sqrt(d).
+ *   o             bf16 [B,H,N,d] device, written for every valid row.
+ *   lse           NULL or fp32 [B,H,N] device.
+ * Limits: d in {64,128}, block in {64,128}, ceil(N/128) <= 4096, B*H <= 65535.
+ */
+SA_API sa_status sa_sparse_attn_fwd(const void* q, const void* k, const void* v,
+                             int B, int H, int N, int d, int block,
+                             const uint8_t* mask, int64_t mask_sb, int64_t mask_sh, int64_t mask_si,
+                             const uint8_t* skip_in, uint8_t* skip_out, float eps, float scale,
+                             void* o, float* lse, void* stream);
+
+/*
+ * sa_pyramid_attn_fwd — PSA multi-level attention forward.
+ *   PSA page, adaptive pyramid attention paragraph (pooled keys weighted so
+ *   that the probability distribution stays consistent) and decoupled
+ *   block-tile kernel paragraph (logical block size independent of the
+ *   hardware tile).
+ *
+ * levels is a uint8 [B,H,Nb,Nb] code map (strides as for `mask`): 0 drops
+ * k-block j, 1 attends to its original keys, 2/3/4 attend to its keys pooled
+ * by c = 2/4/8 (k_pool/v_pool from sa_pyramid_pool).  A pooled key of a group
+ * holding n tokens gets logit scale * q . k_pooled + ln(n).
+ *   k_pool, v_pool  HOST arrays of 3 device pointers (c = 2, 4, 8).
+ * Limits: as sa_sparse_attn_fwd, block == 64 or 128.
+ */
+SA_API sa_status sa_pyramid_attn_fwd(const void* q, const void* k, const void* v,
+                              int B, int H, int N, int d, int block,
+                              const uint8_t* levels, int64_t lv_sb, int64_t lv_sh, int64_t lv_si,
+                              const void* const* k_pool, const void* const* v_pool,
+                              float scale, void* o, float* lse, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPARSE_ATTN_H */

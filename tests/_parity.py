@@ -1,0 +1,64 @@
+"""Comparison helpers for GPU-vs-oracle parity tests.
+
+Tolerances (bf16 inputs and output, unit-variance data):
+  O    max-abs <= 2e-2 and mean-abs <= 2e-3 against the fp64 oracle;
+  LSE  abs <= 1e-3 (finite rows), identical -inf on rows with no visited block;
+  masks / skip bits: bit-exact except bits whose decision margin lies within
+  1e-3 of the cut (flagged by the oracle); flagged mismatches are counted and
+  returned, not failed.
+"""
+import numpy as np
+import torch
+
+O_MAX_ABS = 2e-2
+O_MEAN_ABS = 2e-3
+LSE_ABS = 1e-3
+
+
+def as_np(t):
+    if isinstance(t, torch.Tensor):
+        return t.detach().float().cpu().numpy() if t.is_floating_point() else t.detach().cpu().numpy()
+    return np.asarray(t)
+
+
+def check_o(o_gpu, o_ref, what=""):
+    g = as_np(o_gpu).astype(np.float64)
+    r = np.asarray(o_ref, dtype=np.float64)
+    assert g.shape == r.shape, (g.shape, r.shape)
+    assert np.all(np.isfinite(g)), f"{what}: non-finite output"
+    err = np.abs(g - r)
+    assert err.max() <= O_MAX_ABS, f"{what}: O max-abs {err.max():.3e}"
+    assert err.mean() <= O_MEAN_ABS, f"{what}: O mean-abs {err.mean():.3e}"
+    return float(err.max()), float(err.mean())
+
+
+def check_lse(l_gpu, l_ref, what=""):
+    g = as_np(l_gpu).astype(np.float64)
+    r = np.asarray(l_ref, dtype=np.float64)
+    fin = np.isfinite(r)
+    assert np.array_equal(np.isfinite(g), fin), f"{what}: -inf rows differ"
+    assert np.all(g[~fin] == -np.inf)
+    if fin.any():
+        err = np.abs(g[fin] - r[fin]).max()
+        assert err <= LSE_ABS, f"{what}: LSE abs {err:.3e}"
+
+
+def check_bits(b_gpu, b_ref, flags=None, what=""):
+    """Bit-exact compare; mismatches on flagged positions are tolerated and counted."""
+    g = as_np(b_gpu).astype(np.int64)
+    r = np.asarray(b_ref).astype(np.int64)
+    assert g.shape == r.shape, (g.shape, r.shape)
+    bad = g != r
+    if flags is not None:
+        f = np.asarray(flags, dtype=bool)
+        unflagged = bad & ~f
+        assert not unflagged.any(), f"{what}: {int(unflagged.sum())} unflagged mismatches"
+        return int((bad & f).sum())
+    assert not bad.any(), f"{what}: {int(bad.sum())} mismatches"
+    return 0
+
+
+def skip_flags(margin, eps_margin=1e-3):
+    """Flag skip decisions whose margin max_r(l_r - m_r + eps) is within 1e-3 of 0."""
+    m = np.asarray(margin)
+    return np.isfinite(m) & (np.abs(m) < eps_margin)

@@ -1,0 +1,111 @@
+"""Host-side checks of the C-ABI library (no GPU needed).
+
+The library must load, export every entry point the public header declares,
+and reject bad arguments on the host before touching the GPU.
+"""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+from block_sparse_attention_flash_b200 import build, ops
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return ops.lib()
+
+
+def _declared_symbols():
+    text = open(os.path.join(ROOT, "include", "sparse_attn.h")).read()
+    return sorted(set(re.findall(r"SA_API\s+[\w\s\*]*?\b(sa_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = _declared_symbols()
+    for n in ("sa_build_mask", "sa_radial_mask", "sa_pyramid_pool", "sa_sparse_attn_fwd",
+              "sa_pyramid_attn_fwd", "sa_get_device_status", "sa_build_mask_workspace"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared_symbols():
+        assert hasattr(lib, name), name
+        assert name in ops._SIGNATURES, name
+
+
+def test_status_strings_and_version(lib):
+    assert ops.status_string(0) == "SA_OK"
+    assert ops.status_string(4) == "SA_ERR_TIMEOUT"
+    assert lib.sa_version() >= 100
+
+
+def test_workspace_size(lib):
+    B, H, N, d, block = 1, 12, 32760, 128, 64
+    nb = -(-N // block)
+    assert ops.sa_build_mask_workspace(B, H, N, d, block) == 4 * (2 * B * H * nb * d + B * H * nb * nb)
+    assert ops.sa_build_mask_workspace(0, H, N, d, block) == 0
+
+
+def _attn(lib, **kw):
+    a = dict(q=16, k=16, v=16, B=1, H=1, N=256, d=128, block=128, mask=None, sb=0, sh=0, si=0,
+             skip_in=None, skip_out=None, eps=math.inf, scale=0.0, o=16, lse=None, stream=None)
+    a.update(kw)
+    return lib.sa_sparse_attn_fwd(a["q"], a["k"], a["v"], a["B"], a["H"], a["N"], a["d"], a["block"],
+                                  a["mask"], a["sb"], a["sh"], a["si"], a["skip_in"], a["skip_out"],
+                                  a["eps"], a["scale"], a["o"], a["lse"], a["stream"])
+
+
+def test_attention_argument_validation(lib):
+    assert _attn(lib, d=96) == ops.SA_ERR_UNSUPPORTED
+    assert _attn(lib, block=32) == ops.SA_ERR_UNSUPPORTED
+    assert _attn(lib, q=None) == ops.SA_ERR_INVALID_ARG
+    assert _attn(lib, k=24) == ops.SA_ERR_INVALID_ARG          # not 16-byte aligned
+    assert _attn(lib, eps=float("nan")) == ops.SA_ERR_INVALID_ARG
+    assert _attn(lib, eps=-1.0) == ops.SA_ERR_INVALID_ARG
+    assert _attn(lib, scale=-0.5) == ops.SA_ERR_INVALID_ARG
+    assert _attn(lib, N=128 * 4097) == ops.SA_ERR_UNSUPPORTED
+    assert _attn(lib, B=256, H=256) == ops.SA_ERR_UNSUPPORTED
+    assert _attn(lib, N=0) == ops.SA_OK                       # empty input: nothing to do
+    assert _attn(lib, B=0) == ops.SA_OK
+    assert _attn(lib, mask=16, sb=-1) == ops.SA_ERR_INVALID_ARG
+
+
+def test_mask_builder_argument_validation(lib):
+    fr = (ctypes.c_float * 3)(0.1, 0.3, 0.6)
+    bad = (ctypes.c_float * 3)(0.5, 0.3, 0.6)
+    f = lib.sa_build_mask
+    assert f(16, 16, 1, 1, 512, 64, 64, 0, 1.5, None, 16, None, 256, 1 << 20, None) == ops.SA_ERR_INVALID_ARG
+    assert f(16, 16, 1, 1, 512, 64, 64, 7, 0.9, None, 16, None, 256, 1 << 20, None) == ops.SA_ERR_INVALID_ARG
+    assert f(16, 16, 1, 1, 512, 64, 64, 1, 0.9, ctypes.cast(bad, ctypes.c_void_p), 16, None, 256, 1 << 20,
+             None) == ops.SA_ERR_INVALID_ARG
+    assert f(16, 16, 1, 1, 512, 64, 64, 1, 0.9, ctypes.cast(fr, ctypes.c_void_p), 16, None, 256, 16,
+             None) == ops.SA_ERR_INVALID_ARG                   # workspace too small
+    assert f(16, 16, 1, 1, 512, 64, 64, 0, 0.9, None, 16, None, 200, 1 << 20, None) == ops.SA_ERR_INVALID_ARG
+    assert f(16, 16, 1, 1, 512, 80, 64, 0, 0.9, None, 16, None, 256, 1 << 20, None) == ops.SA_ERR_UNSUPPORTED
+    assert f(16, 16, 1, 1, 0, 64, 64, 0, 0.9, None, 16, None, 256, 0, None) == ops.SA_OK
+
+
+def test_pool_and_radial_argument_validation(lib):
+    three = (ctypes.c_void_p * 3)(16, 32, 48)
+    holes = (ctypes.c_void_p * 3)(16, None, 48)
+    f = lib.sa_pyramid_pool
+    assert f(16, 16, 1, 1, 64, 128, 64, ctypes.cast(holes, ctypes.c_void_p), ctypes.cast(three, ctypes.c_void_p),
+             None) == ops.SA_ERR_INVALID_ARG
+    assert f(16, 16, 1, 1, 64, 100, 64, ctypes.cast(three, ctypes.c_void_p), ctypes.cast(three, ctypes.c_void_p),
+             None) == ops.SA_ERR_UNSUPPORTED
+    assert lib.sa_radial_mask(4, 8, 16, 0, 16, None) == ops.SA_ERR_INVALID_ARG
+    assert lib.sa_radial_mask(4, 8, 16, 64, None, None) == ops.SA_ERR_INVALID_ARG
+    assert lib.sa_radial_mask(0, 8, 16, 64, None, None) == ops.SA_OK
+
+
+def test_ops_refuse_cpu_tensors():
+    import torch
+    q = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16)
+    with pytest.raises((ValueError, RuntimeError)):
+        ops.sa_sparse_attn_fwd(q, q, q, 64, out=q.clone())

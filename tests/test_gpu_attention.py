@@ -1,0 +1,172 @@
+"""GPU parity: sa_sparse_attn_fwd (binary masks, LiteAttention skip update) vs the fp64 oracle."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_attention_flash_b200 import build, inputs, ops
+from oracle import masked_attention, lite_step, radial_mask
+from _parity import check_o, check_lse, check_bits, skip_flags
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    build.build()
+    ops.lib()
+    yield
+    ops.sa_get_device_status()
+
+
+def run_attn(q, k, v, block, mask=None, skip_in=None, skip_out=None, eps=math.inf, with_lse=True):
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    B, H, N, d = q.shape
+    # poison the output so unwritten rows show up
+    out = torch.full_like(qd, float("nan"))
+    lse = torch.full((B, H, N), float("nan"), device="cuda") if with_lse else None
+    ops.sa_sparse_attn_fwd(qd, kd, vd, block, mask=None if mask is None else mask.cuda(),
+                           skip_in=skip_in, skip_out=skip_out, eps=eps, out=out, lse=lse)
+    ops.sa_get_device_status()
+    return out.cpu(), (lse.cpu() if lse is not None else None)
+
+
+def test_tiny_all_ones_equals_dense():
+    wl = inputs.WORKLOADS["tiny"]
+    q, k, v = inputs.normal_qkv(wl.B, wl.H, wl.N, wl.d, wl.seed)
+    O, L = run_attn(q, k, v, wl.block)
+    Or, Lr = masked_attention(q, k, v, wl.block, None)
+    check_o(O, Or, "tiny dense")
+    check_lse(L, Lr, "tiny dense")
+
+
+def test_tiny_bernoulli_mask():
+    wl = inputs.WORKLOADS["tiny"]
+    q, k, v = inputs.normal_qkv(wl.B, wl.H, wl.N, wl.d, wl.seed)
+    m = inputs.bernoulli_block_mask(wl.B, wl.H, wl.nblocks, wl.nblocks, 0.5, wl.seed + 1)
+    O, L = run_attn(q, k, v, wl.block, m)
+    Or, Lr = masked_attention(q, k, v, wl.block, m)
+    check_o(O, Or, "tiny bernoulli")
+    check_lse(L, Lr, "tiny bernoulli")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("block", [64, 128])
+@pytest.mark.parametrize("N", [1, 77, 130, 1000, 2065])
+def test_ragged_random_masks(d, block, N):
+    B, H = 2, 2
+    q, k, v = inputs.normal_qkv(B, H, N, d, seed=N * 7 + d + block)
+    nb = -(-N // block)
+    m = inputs.bernoulli_block_mask(B, H, nb, nb, 0.45, seed=N + 3, force_diagonal=True)
+    if nb > 2:
+        m[0, 1, 1, :] = 0                      # a q-block with no kept block
+    O, L = run_attn(q, k, v, block, m)
+    Or, Lr = masked_attention(q, k, v, block, m)
+    check_o(O, Or, f"N={N} d={d} block={block}")
+    check_lse(L, Lr, f"N={N} d={d} block={block}")
+    if nb > 2:
+        rows = slice(block, min(N, 2 * block))
+        assert torch.all(O[0, 1, rows] == 0)
+        assert torch.all(L[0, 1, rows] == -math.inf)
+
+
+def test_unit_values_rows_sum_to_one():
+    B, H, N, d, block = 1, 3, 1500, 128, 128
+    q, k, _ = inputs.normal_qkv(B, H, N, d, seed=5)
+    v = torch.ones_like(q)
+    nb = -(-N // block)
+    m = inputs.bernoulli_block_mask(B, H, nb, nb, 0.3, seed=6)
+    O, _ = run_attn(q, k, v, block, m, with_lse=False)
+    assert torch.all((O.float() - 1.0).abs() <= 8e-3)
+
+
+def test_radial_mask_broadcast_over_heads():
+    T, Hh, Ww, block = 12, 8, 16, 128
+    wl = inputs.Workload("r", 1, 3, 128, T, Hh, Ww, block, "radial", seed=31)
+    q, k, v = inputs.rff_qkv(wl)
+    rm = torch.from_numpy(radial_mask(T, Hh, Ww, block))
+    O, L = run_attn(q, k, v, block, rm)             # [Nb, Nb] mask: strides (0, 0, Nb)
+    Or, Lr = masked_attention(q, k, v, block, rm.numpy())
+    check_o(O, Or, "radial broadcast")
+    check_lse(L, Lr, "radial broadcast")
+
+
+# ------------------------------------------------------------------ skip ---
+
+def _skip_run(q, k, v, block, mask, skip_in, eps, alias=False):
+    B, H, N, d = q.shape
+    nb = -(-N // block)
+    si = skip_in.cuda() if skip_in is not None else None
+    if alias:
+        so = si
+    else:
+        so = torch.full((B, H, nb, nb), 77, dtype=torch.uint8, device="cuda")
+    O, L = run_attn(q, k, v, block, mask, skip_in=si, skip_out=so, eps=eps)
+    return O, L, so.cpu()
+
+
+def _check_skip_step(q, k, v, block, mask, skip_in, eps, alias=False):
+    O, L, S = _skip_run(q, k, v, block, mask, skip_in, eps, alias)
+    Or, Lr, Sr, M = lite_step(q, k, v, block, None if mask is None else mask.numpy(),
+                              None if skip_in is None else skip_in.numpy(), eps)
+    check_o(O, Or, f"skip step eps={eps}")
+    check_lse(L, Lr, f"skip step eps={eps}")
+    nflag = check_bits(S, Sr, skip_flags(M), f"skip bits eps={eps}")
+    return S, Sr, nflag
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_hand_built_gap_of_twelve(d):
+    block, nb = 128, 5
+    N = block * nb
+    a = math.sqrt(6.0 * math.sqrt(d))
+    u = torch.zeros(d)
+    u[3] = 1.0
+    q = (a * u).repeat(N, 1).view(1, 1, N, d).to(torch.bfloat16)
+    k = (-a * u).repeat(N, 1)
+    k[:block] = a * u
+    k = k.view(1, 1, N, d).to(torch.bfloat16)
+    v = torch.randn(1, 1, N, d, generator=torch.Generator().manual_seed(0)).to(torch.bfloat16)
+    S, Sr, _ = _check_skip_step(q, k, v, block, None, None, eps=10.0)
+    assert S[0, 0, :, 1:].all() and not S[0, 0, :, 0].any()
+    S, _, _ = _check_skip_step(q, k, v, block, None, None, eps=1e6)
+    assert S.sum() == 0
+
+
+@pytest.mark.parametrize("block", [64, 128])
+def test_rff_skips_small_eps(block):
+    wl = inputs.Workload("s", 1, 3, 128, 8, 16, 24, block, "lite", seed=41, sigma_s=2.0, sigma_t=1.5)
+    q, k, v = inputs.rff_qkv(wl)
+    S, Sr, nflag = _check_skip_step(q, k, v, block, None, None, eps=1.0)
+    assert Sr.sum() > 0
+
+
+@pytest.mark.parametrize("block", [64, 128])
+def test_teacher_forced_chain_with_carry_and_alias(block):
+    wl = inputs.Workload("c", 1, 2, 128, 6, 16, 24, block, "lite", seed=43, sigma_s=2.0, sigma_t=1.5)
+    steps = list(inputs.lite_chain_inputs(wl, 4))
+    nb = wl.nblocks
+    mask = inputs.bernoulli_block_mask(1, wl.H, nb, nb, 0.8, seed=44)
+    skip = None
+    total = 0
+    for s, (q, k, v) in enumerate(steps):
+        S, Sr, _ = _check_skip_step(q, k, v, block, mask, skip, eps=1.2, alias=(s % 2 == 1 and skip is not None))
+        if skip is not None:
+            assert np.all(S.numpy() >= skip.numpy())      # monotone carry
+        skip = S                                           # teacher forcing: GPU bits feed both sides
+        total = int(S.sum())
+    assert total > 0
+
+
+def test_skip_in_blocks_are_not_visited():
+    B, H, N, d, block = 1, 2, 1024, 128, 128
+    q, k, v = inputs.normal_qkv(B, H, N, d, seed=9)
+    nb = N // block
+    skip_in = inputs.bernoulli_block_mask(B, H, nb, nb, 0.3, seed=10, force_diagonal=False)
+    skip_in[:, :, torch.arange(nb), torch.arange(nb)] = 0
+    O, L, S = _skip_run(q, k, v, block, None, skip_in, eps=math.inf)
+    Or, Lr = masked_attention(q, k, v, block, (1 - skip_in.numpy()))
+    check_o(O, Or, "skip_in honoured")
+    check_lse(L, Lr, "skip_in honoured")
+    assert torch.equal(S, skip_in)                     # eps = inf: carry only

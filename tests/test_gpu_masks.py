@@ -1,0 +1,101 @@
+"""GPU parity: radial mask, tau / level mask builder and pyramid pooling vs the oracle."""
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_attention_flash_b200 import build, inputs, ops
+from oracle import radial_mask, tau_mask, level_map, pyramid_pool
+from _parity import check_bits
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    build.build()
+    ops.lib()
+    yield
+    ops.sa_get_device_status()
+
+
+@pytest.mark.parametrize("T,Hh,Ww,block", [(4, 8, 16, 64), (21, 30, 52, 64), (33, 45, 80, 128),
+                                           (21, 45, 80, 128), (7, 5, 9, 64), (1, 1, 1, 128)])
+def test_radial_mask_bit_exact(T, Hh, Ww, block):
+    m = ops.sa_radial_mask(T, Hh, Ww, block)
+    ops.sa_get_device_status()
+    check_bits(m.cpu(), radial_mask(T, Hh, Ww, block), what=f"radial {T}x{Hh}x{Ww}/{block}")
+
+
+def _small_rff(block, d=128, H=3, seed=61):
+    wl = inputs.Workload("m", 1, H, d, 9, 20, 24, block, "tau", seed=seed)
+    return inputs.rff_qkv(wl)
+
+
+@pytest.mark.parametrize("block", [64, 128])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("tau", [0.5, 0.9])
+def test_tau_mask_small(block, d, tau):
+    q, k, _ = _small_rff(block, d)
+    m = ops.sa_build_mask(q.cuda(), k.cuda(), block, "tau", tau=tau)
+    ops.sa_get_device_status()
+    mr, flags, _ = tau_mask(q, k, block, tau, return_info=True)
+    check_bits(m.cpu(), mr, flags, f"tau block={block} d={d} tau={tau}")
+
+
+@pytest.mark.parametrize("block", [64, 128])
+def test_level_map_small(block):
+    q, k, _ = _small_rff(block)
+    m = ops.sa_build_mask(q.cuda(), k.cuda(), block, "levels", level_frac=(0.1, 0.3, 0.6))
+    ops.sa_get_device_status()
+    lr, flags, _ = level_map(q, k, block, (0.1, 0.3, 0.6), return_info=True)
+    check_bits(m.cpu(), lr, flags, f"levels block={block}")
+
+
+def test_scores_out_matches_oracle_scores():
+    q, k, _ = _small_rff(64)
+    nb = -(-q.shape[2] // 64)
+    sc = torch.empty(1, q.shape[1], nb, nb, device="cuda")
+    ops.sa_build_mask(q.cuda(), k.cuda(), 64, "tau", tau=0.9, scores_out=sc)
+    ops.sa_get_device_status()
+    _, _, S = tau_mask(q, k, 64, 0.9, return_info=True)
+    assert np.abs(sc.cpu().numpy() - S).max() < 1e-4
+
+
+def test_uniform_scores_keep_first_blocks():
+    """Q == 0 makes every score equal: the GPU must break ties by index."""
+    N, block = 64 * 42, 64            # tau * Nb = 31.5: no exact tie with the threshold
+    q = torch.zeros(1, 2, N, 128, dtype=torch.bfloat16)
+    k = torch.randn(1, 2, N, 128, generator=torch.Generator().manual_seed(3)).to(torch.bfloat16)
+    m = ops.sa_build_mask(q.cuda(), k.cuda(), block, "tau", tau=0.75).cpu()
+    nb = N // block
+    keep = int(np.ceil(0.75 * nb))
+    assert torch.all(m[..., :keep] == 1) and torch.all(m[..., keep:] == 0)
+    lv = ops.sa_build_mask(q.cuda(), k.cuda(), block, "levels", level_frac=(0.1, 0.3, 0.6)).cpu()
+    assert lv[0, 0, 0].tolist() == level_map(q[:, :1, :block * nb], k[:, :1], block)[0, 0, 0].tolist()
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("N", [64 * 5 + 24, 1000, 1003, 7])
+def test_pyramid_pool(d, N):
+    g = torch.Generator().manual_seed(N + d)
+    k = torch.randn(2, 2, N, d, generator=g).to(torch.bfloat16)
+    v = torch.randn(2, 2, N, d, generator=g).to(torch.bfloat16)
+    kp, vp = ops.sa_pyramid_pool(k.cuda(), v.cuda(), 64)
+    ops.sa_get_device_status()
+    for lvl, c in enumerate((2, 4, 8)):
+        for got, src in ((kp[lvl], k), (vp[lvl], v)):
+            ref = pyramid_pool(src, c)
+            err = np.abs(got.float().cpu().numpy() - ref)
+            # fp32 sum then one bf16 rounding: within half a bf16 ulp of the mean
+            assert np.all(err <= np.abs(ref) * 2.0 ** -8 + 1e-6), (c, float(err.max()))
+
+
+def test_tau_mask_wan13b_480p_full():
+    """Full-size tau mask of the 480p Wan2.1-1.3B-like workload (12 heads, 512 x 512 blocks)."""
+    wl = inputs.WORKLOADS["wan13b_480p_tau"]
+    q, k, _ = inputs.rff_qkv(wl)
+    m = ops.sa_build_mask(q.cuda(), k.cuda(), wl.block, "tau", tau=wl.tau)
+    ops.sa_get_device_status()
+    mr, flags, _ = tau_mask(q, k, wl.block, wl.tau, return_info=True)
+    nflag = check_bits(m.cpu(), mr, flags, "tau 480p full")
+    assert nflag <= 0.001 * mr.size
