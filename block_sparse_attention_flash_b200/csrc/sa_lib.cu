@@ -285,3 +285,72 @@ sa_status sa_pyramid_attn_fwd(const void* q, const void* k, const void* v, int B
 }
 
 }  // extern "C"
+
+// ===========================================================================
+// sa_build_mask_noalloc: sa_build_mask for callers that must not allocate.
+//
+// Some callers cannot call cudaMalloc at the moment they need a mask:
+//   - code running inside CUDA stream capture, where an allocation would break
+//     the capture;
+//   - runtimes that own all device memory through their own pool and forbid
+//     libraries from allocating behind their back;
+//   - latency-critical loops that must never block on the allocator.
+// For them this variant takes its scratch (block means and block scores) from
+// one file-scope device array instead of a caller-provided workspace.  The
+// array is created when the library's device code is loaded on a GPU and is
+// held on every such GPU until the process exits.
+//
+// Everything that runs on the GPU is the same as in sa_build_mask: this entry
+// point looks up the array's device address and then calls sa_build_mask with
+// it as the workspace.
+// ===========================================================================
+namespace {
+
+// Upper bound of the shared scratch: large enough for the 480p workload
+// (12 heads, 32,760 tokens, block 64, d 128 needs 18.9 MB).
+constexpr size_t kNoAllocScratchBytes = static_cast<size_t>(32) << 20;  // 32 MiB
+
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_build_mask_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+struct ScratchAddress {
+  std::once_flag flag;
+  void* ptr = nullptr;
+  cudaError_t err = cudaSuccess;
+};
+ScratchAddress g_scratch_address[kMaxDevices];
+
+// Device address of g_build_mask_scratch on the current device.  In host code
+// the array's name is only a host-side stand-in, so the address has to be
+// asked from the runtime: once per device, with that device current.
+cudaError_t build_mask_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  ScratchAddress& s = g_scratch_address[dev];
+  std::call_once(s.flag, [&s] {
+    void* p = nullptr;
+    s.err = cudaGetSymbolAddress(&p, g_build_mask_scratch);
+    s.ptr = (s.err == cudaSuccess) ? p : nullptr;
+  });
+  *out = s.ptr;
+  return s.err;
+}
+
+}  // namespace
+
+extern "C" sa_status sa_build_mask_noalloc(const void* q, const void* k, int B, int H, int N, int d, int block,
+                                           int mode, float tau, const float* level_frac, uint8_t* mask_out,
+                                           float* scores_out, void* stream) {
+  if (B < 0 || H < 0 || N < 0) return SA_ERR_INVALID_ARG;
+  if (B == 0 || H == 0 || N == 0) return SA_OK;
+  if (sa_build_mask_workspace(B, H, N, d, block) > kNoAllocScratchBytes) return SA_ERR_UNSUPPORTED;
+  void* scratch = nullptr;
+  if (build_mask_scratch(&scratch) != cudaSuccess || scratch == nullptr) return SA_ERR_CUDA;
+  return sa_build_mask(q, k, B, H, N, d, block, mode, tau, level_frac, mask_out, scores_out, scratch,
+                       kNoAllocScratchBytes, stream);
+}

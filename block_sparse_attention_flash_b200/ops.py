@@ -29,6 +29,7 @@ _SIGNATURES = {
     "sa_get_device_status": (_i32, [_vp]),
     "sa_build_mask_workspace": (_sz, [_i32, _i32, _i32, _i32, _i32]),
     "sa_build_mask": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "sa_build_mask_noalloc": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _vp, _vp, _vp]),
     "sa_radial_mask": (_i32, [_i32, _i32, _i32, _i32, _vp, _vp]),
     "sa_pyramid_pool": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
     "sa_sparse_attn_fwd": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _i64, _i64, _i64,

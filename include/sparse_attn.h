@@ -111,6 +111,33 @@ SA_API sa_status sa_build_mask(const void* q, const void* k, int B, int H, int N
                         void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * sa_build_mask_noalloc — sa_build_mask without a caller-provided workspace.
+ *   The pages have no counterpart to this entry point: it exists for callers
+ *   that cannot allocate device memory when they need a mask (code inside
+ *   CUDA stream capture, runtimes that forbid libraries from allocating, or
+ *   loops that must not wait on an allocator).
+ *
+ * Same arguments, computation and results as sa_build_mask, minus the
+ * workspace.  The scratch comes from one static device array of 32 MiB
+ * (33,554,432 bytes) that every GPU loading this library holds until the
+ * process exits.  Rules:
+ *   - Size limit: sizes whose sa_build_mask_workspace(B, H, N, d, block)
+ *     exceeds 32 MiB are rejected with SA_ERR_UNSUPPORTED before any launch.
+ *   - Set-up: the first call on a device, with that device current, looks up
+ *     the array's device address (cudaGetSymbolAddress) and keeps it.  Make
+ *     that first call before any stream capture.
+ *   - Sharing: all calls on a device share the one array, and it keeps the
+ *     previous call's contents.  Nothing in it needs to start at zero (every
+ *     byte read is first written by the same call).  Calls whose kernels
+ *     overlap on the GPU (different streams, no ordering between them) race
+ *     on the array and give wrong masks: serialise them.
+ *   - No memory is allocated or freed by this call.
+ */
+SA_API sa_status sa_build_mask_noalloc(const void* q, const void* k, int B, int H, int N, int d, int block,
+                                       int mode, float tau, const float* level_frac,
+                                       uint8_t* mask_out, float* scores_out, void* stream);
+
+/*
  * sa_radial_mask — static radial mask for a T x Hh x Ww grid.
  *   "MIT实验室推出Radial Attention" (arXiv 2506.19852), spatio-temporal energy
  *   decay and static-mask paragraphs: attention concentrates on nearby frames,
