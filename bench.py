@@ -273,6 +273,104 @@ def run_e2e(ops, qkv0, block, eps, nb, dev, stream, steps, world):
             "ms_per_step": round(ms / steps, 3), "steps": steps}
 
 
+# -------------------------------------------------------------- suite mode ---
+
+def _time(fn, reps, stream):
+    """Median ms of `fn` over `reps` launches (CUDA events on `stream`), after 3 warm-ups."""
+    for _ in range(3):
+        fn()
+    ts = []
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    return statistics.median(ts)
+
+
+def run_suite(args):
+    """Every workload's hot path on one GPU: one JSON line per workload."""
+    from block_sparse_attention_flash_b200 import inputs, ops, build
+
+    build.build()
+    ops.lib()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    peaks, src = load_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    tens = float(peaks["bf16_tflops"])
+    out = []
+
+    def attn_line(wl, name, ms, flops, extra):
+        dense = 4.0 * wl.d * wl.N * wl.N * wl.B * wl.H
+        d = {"workload": name, "N": wl.N, "H": wl.H, "d": wl.d, "block": wl.block, "ms_per_call": round(ms, 3),
+             "density": round(flops / dense, 5), "executed_tflops": round(flops / ms / 1e9, 1),
+             "dense_equiv_tflops": round(dense / ms / 1e9, 1),
+             "frac_of_bf16_burst": round(flops / ms / 1e9 / tens, 4), "peak_source": src}
+        d.update(extra)
+        return d
+
+    for name in ("wan13b_480p_tau", "hunyuan_720p_radial", "wan14b_720p_lite", "psa_480p_pyramid"):
+        wl = inputs.WORKLOADS[name]
+        q, k, v = inputs.rff_qkv(wl, device=dev)
+        nb = wl.nblocks
+        B, H, N, d = q.shape
+        o = torch.empty_like(q)
+        qk_bytes = 2 * B * H * N * d * 2
+        if wl.kind == "tau":
+            ws = torch.empty(ops.sa_build_mask_workspace(B, H, N, d, wl.block), dtype=torch.uint8, device=dev)
+            m = torch.empty(B, H, nb, nb, dtype=torch.uint8, device=dev)
+            ms_m = _time(lambda: ops.sa_build_mask(q, k, wl.block, "tau", tau=wl.tau, mask_out=m, workspace=ws),
+                         args.suite_reps, stream)
+            ms_a = _time(lambda: ops.sa_sparse_attn_fwd(q, k, v, wl.block, mask=m, out=o), args.suite_reps, stream)
+            flops = executed_flops(torch.zeros_like(m), N, wl.block, d, mask=m)
+            out.append(attn_line(wl, name, ms_a, flops, {
+                "mask_ms": round(ms_m, 4), "mask_gbs": round(qk_bytes / ms_m / 1e6, 1),
+                "mask_frac_of_hbm": round(qk_bytes / ms_m / 1e6 / hbm, 4)}))
+        elif wl.kind == "radial":
+            rm = ops.sa_radial_mask(wl.T, wl.Hh, wl.Ww, wl.block)
+            ms_r = _time(lambda: ops.sa_radial_mask(wl.T, wl.Hh, wl.Ww, wl.block, out=rm), args.suite_reps, stream)
+            ms_a = _time(lambda: ops.sa_sparse_attn_fwd(q, k, v, wl.block, mask=rm, out=o), args.suite_reps, stream)
+            m4 = rm.view(1, 1, nb, nb).expand(B, H, nb, nb)
+            flops = executed_flops(torch.zeros(B, H, nb, nb, dtype=torch.uint8, device=dev), N, wl.block, d,
+                                   mask=m4)
+            out.append(attn_line(wl, name, ms_a, flops, {"radial_mask_ms": round(ms_r, 4)}))
+        elif wl.kind == "lite":
+            skip_a = torch.zeros(B, H, nb, nb, dtype=torch.uint8, device=dev)
+            skip_b = torch.zeros_like(skip_a)
+            ms_a = _time(lambda: ops.sa_sparse_attn_fwd(q, k, v, wl.block, skip_in=skip_a, skip_out=skip_b,
+                                                        eps=wl.eps, out=o), args.suite_reps, stream)
+            flops = executed_flops(skip_a, N, wl.block, d)
+            out.append(attn_line(wl, name, ms_a, flops, {"eps": wl.eps, "skipped_next_step": int(skip_b.sum())}))
+        else:
+            kp, vp = ops.sa_pyramid_pool(k, v, wl.block)
+            ms_p = _time(lambda: ops.sa_pyramid_pool(k, v, wl.block, k_pool=kp, v_pool=vp), args.suite_reps, stream)
+            lv = ops.sa_build_mask(q, k, wl.block, "levels", level_frac=wl.level_frac)
+            ms_a = _time(lambda: ops.sa_pyramid_attn_fwd(q, k, v, wl.block, lv, kp, vp, out=o), args.suite_reps,
+                         stream)
+            # executed keys per (i, j): block >> level (valid rows x pooled cols)
+            rows = torch.full((nb,), float(wl.block), device=dev, dtype=torch.float64)
+            rows[-1] = N - (nb - 1) * wl.block
+            cols = torch.zeros(B, H, nb, nb, dtype=torch.float64, device=dev)
+            for lvl in range(4):
+                cnt = torch.full((nb,), float(wl.block >> lvl), device=dev, dtype=torch.float64)
+                cnt[-1] = -(-int(rows[-1].item()) // (1 << lvl))
+                cols += (lv == lvl + 1).to(torch.float64) * cnt.view(1, 1, 1, nb)
+            flops = float(4.0 * d * torch.einsum("i,bhij->", rows, cols).item())
+            pool_bytes = qk_bytes + qk_bytes * 7 // 8
+            out.append(attn_line(wl, name, ms_a, flops, {
+                "pool_ms": round(ms_p, 4), "pool_gbs": round(pool_bytes / ms_p / 1e6, 1),
+                "pool_frac_of_hbm": round(pool_bytes / ms_p / 1e6 / hbm, 4)}))
+        ops.sa_get_device_status()
+        del q, k, v, o
+        torch.cuda.empty_cache()
+    for line in out:
+        print(json.dumps(line), flush=True)
+
+
 # ------------------------------------------------------------ oracle timing ---
 
 def cpu_sample(q, k, v, block, eps, seconds):
@@ -342,7 +440,12 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-seconds", type=float, default=60.0)
+    ap.add_argument("--suite", action="store_true", help="time every workload's hot path (one line each)")
+    ap.add_argument("--suite-reps", type=int, default=10)
     args = ap.parse_args()
+    if args.suite:
+        run_suite(args)
+        return
     if args.warmup < 3:
         args.warmup = 3
     rank, world, local = dist_env()

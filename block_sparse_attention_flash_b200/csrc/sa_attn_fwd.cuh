@@ -5,24 +5,29 @@
 // of one (b, h) and walks the union of their kept 128-column kv tiles in
 // ascending order.  Each kv tile is loaded once by TMA and feeds both q-tiles.
 //
-// Roles (384 threads, one CTA per SM):
-//   warp 0      builds the kv-tile list from the mask / skip bytes, then one
-//               lane issues the TMA loads (Q once, K/V through a 2-stage ring;
-//               skipped tiles are never loaded: LiteAttention write-up,
-//               sections 3 and 6);
-//   warp 1      owns TMEM (512 columns) and one lane issues every tcgen05.mma:
-//               S_t = Q_t K^T (SS form) and O_t += P_t V (A operand P_t read
-//               from TMEM, where the softmax wrote it over S_t);
-//   warps 4-7   online softmax of q-tile 0 (one row per thread, TMEM lanes
-//               0-127), warps 8-11 the same for q-tile 1.  They evaluate the
-//               skip condition on the row maxima they compute anyway
-//               (LiteAttention write-up, section 5), record it per warp and
-//               reduce across warps only at the end (section 6).
+// Roles (640 threads = 20 warps, one CTA per SM; warps 2-3 only join the
+// final barrier, they keep the softmax warps aligned to TMEM lane quarters):
+//   warp 0       builds the kv-tile list from the mask / skip bytes, then one
+//                lane issues the TMA loads (Q once, K and V through 2-stage
+//                rings released separately; skipped tiles are never loaded:
+//                LiteAttention write-up, sections 3 and 6);
+//   warp 1       owns TMEM (512 columns) and one lane issues every
+//                tcgen05.mma: S_t = Q_t K^T (both operands from shared memory)
+//                and O_t += P_t V (A operand P_t read from TMEM, where the
+//                softmax wrote it over S_t);
+//   warps 4-11   online softmax of q-tile 0, warps 12-19 of q-tile 1.  Two
+//                threads per row: warps [4,8) take columns 0-63 of rows
+//                32*(warp%4) .. +31 (a warp may only touch its own TMEM lane
+//                quarter), warps [8,12) columns 64-127; the two halves swap
+//                their row maxima through shared memory once per kv tile.
+//                They evaluate the skip condition on the maxima they compute
+//                anyway (LiteAttention write-up, section 5), record it per
+//                warp and reduce across warps only at kernel end (section 6).
 //
 // TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [384,384+D).
 // Shared memory: Q0, Q1, K[2], V[2] tiles of 128 x D bf16 in the 128-byte
 // swizzled layout TMA writes (each 64-column half is a [128 x 128 B] slab),
-// the kv list, the per-warp skip votes and the mbarriers.
+// the kv list, the per-warp skip votes, the row-max exchange and mbarriers.
 //
 // Block size 64: a 128-row tile holds q-blocks 2i, 2i+1 and a 128-column kv
 // tile holds k-blocks 2j, 2j+1; the list keeps per-quadrant bits and the
@@ -37,7 +42,12 @@ constexpr int kTileM = 128;
 constexpr int kTileN = 128;
 constexpr int kStages = 2;
 constexpr int kMaxKvTiles = 4096;
-constexpr int kAttnThreads = 384;
+constexpr int kAttnWarps = 20;
+constexpr int kAttnThreads = kAttnWarps * 32;
+constexpr int kSoftmaxWarp0 = 4;
+// Within each 16-pair chunk of a row, pairs [kPolyPairFrom, 16) take 2^x from
+// the FMA-pipe polynomial instead of the MUFU unit (balances the two pipes).
+constexpr int kPolyPairFrom = 12;
 
 struct AttnParams {
   int B, H, N;
@@ -62,10 +72,12 @@ struct AttnSmem {
   static constexpr int kOffK = 2 * kTileBytes;
   static constexpr int kOffV = kOffK + kStages * kTileBytes;
   static constexpr int kOffList = kOffV + kStages * kTileBytes;
-  static constexpr int kVoteWords = kMaxKvTiles * 2 / 32;  // per (tile, warp)
+  static constexpr int kVoteWords = kMaxKvTiles / 32;      // per softmax warp
   static constexpr int kOffVotes = kOffList + kMaxKvTiles * 4;
-  static constexpr int kNumBars = 1 + 3 * kStages + 2 + 2 + 2 + 1;
-  static constexpr int kOffBar = kOffVotes + 2 * 4 * kVoteWords * 4;
+  static constexpr int kOffRed = kOffVotes + 16 * kVoteWords * 4;
+  static constexpr int kRedFloats = 2 * 2 * 2 * kTileM;    // [tile][parity][half][row]
+  static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2 + 2 + 1;
+  static constexpr int kOffBar = kOffRed + kRedFloats * 4;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffMisc + 64;
   static constexpr int kAlloc = kBytes + 1024;
@@ -73,6 +85,21 @@ struct AttnSmem {
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Named barrier over `nthreads` threads that also returns the AND of `v`
+// over all of them, so that every participant takes the same branch.
+__device__ __forceinline__ bool named_bar_and(int id, int nthreads, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %2, 0;\n\t"
+      "bar.red.and.pred po, %1, %3, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(r)
+      : "r"(id), "r"(static_cast<uint32_t>(v)), "r"(nthreads)
+      : "memory");
+  return r != 0;
 }
 
 template <int D, int BLK>
@@ -90,12 +117,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint32_t* list = reinterpret_cast<uint32_t*>(smem + L::kOffList);
   uint32_t* votes = reinterpret_cast<uint32_t*>(smem + L::kOffVotes);
+  float* red = reinterpret_cast<float*>(smem + L::kOffRed);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;
   uint64_t* v_full = bars + 1 + kStages;
-  uint64_t* kv_empty = bars + 1 + 2 * kStages;
-  uint64_t* s_ready = bars + 1 + 3 * kStages;
+  uint64_t* k_empty = bars + 1 + 2 * kStages;
+  uint64_t* v_empty = bars + 1 + 3 * kStages;
+  uint64_t* s_ready = bars + 1 + 4 * kStages;
   uint64_t* p_ready = s_ready + 2;
   uint64_t* o_final = p_ready + 2;
   uint64_t* mma_done = o_final + 2;
@@ -107,7 +136,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int b = bh / p.H, h = bh - (bh / p.H) * p.H;
   const int qtile0 = 2 * pair;
 
-  for (int i = threadIdx.x; i < 2 * 4 * L::kVoteWords; i += kAttnThreads) votes[i] = 0;
+  for (int i = threadIdx.x; i < 16 * L::kVoteWords; i += kAttnThreads) votes[i] = 0;
 
   if (warp == 0) {
     // ---- kv-tile list: union over the two q-tiles, per-quadrant keep bits ----
@@ -151,7 +180,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       misc[4] = 0;
       for (int i = 0; i < L::kNumBars; ++i) {
         const bool softmax_arrivals = (&bars[i] == &p_ready[0]) || (&bars[i] == &p_ready[1]);
-        mbar_init(&bars[i], softmax_arrivals ? 128u : 1u);
+        mbar_init(&bars[i], softmax_arrivals ? 256u : 1u);
       }
       fence_mbar_init();
       tma_prefetch_desc(&tmQ);
@@ -172,6 +201,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t sK = smem_addr(smem + L::kOffK);
   const uint32_t sV = smem_addr(smem + L::kOffV);
 
+  if (warp < kSoftmaxWarp0) {
+    // Register split: this warpgroup gives up registers the softmax rows use.
+    // Each role runs to its own final barrier so the two register budgets
+    // never meet in shared code.
+    setmaxnreg_dec<32>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer ---
     if (lane == 0 && n_list > 0) {
@@ -189,17 +223,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       int issued = 0;
       for (int e = 0; e < n_list; ++e) {
         const int s = e % kStages;
-        if (e >= kStages) {
-          if (misc[4] || !mbar_wait(&kv_empty[s], ((e / kStages) - 1) & 1)) {
-            misc[4] = 1;
-            break;
-          }
+        const uint32_t par = ((e / kStages) - 1) & 1;
+        if (e >= kStages && (misc[4] || !mbar_wait(&k_empty[s], par))) {
+          misc[4] = 1;
+          break;
         }
         const int row = static_cast<int>(list[e] & 0xFFFFu) * kTileN;
         mbar_arrive_expect_tx(&k_full[s], L::kTileBytes);
 #pragma unroll
         for (int hd = 0; hd < D / 64; ++hd)
           tma_load_3d(&tmK, &k_full[s], smem + L::kOffK + s * L::kTileBytes + hd * kHalfBytes, hd * 64, row, bh);
+        if (e >= kStages && !mbar_wait(&v_empty[s], par)) {
+          misc[4] = 1;
+          issued = e;
+          mbar_wait(&k_full[s], (e / kStages) & 1);
+          break;
+        }
         mbar_arrive_expect_tx(&v_full[s], L::kTileBytes);
 #pragma unroll
         for (int hd = 0; hd < D / 64; ++hd)
@@ -242,7 +281,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const uint64_t bdesc = smem_desc(vbase + kk * 16 * 128, kHalfBytes, 1024);
           mma_ts(d_tmem, a_tmem + kk * 8, bdesc, kIdescPV, (done_pv[t] == 0 && kk == 0) ? 0u : 1u);
         }
-        if (--users[s] == 0) mma_commit(&kv_empty[s]);
+        if (--users[s] == 0) mma_commit(&v_empty[s]);
         if (++done_pv[t] == cnt[t]) mma_commit(&o_final[t]);
         pend[t] = -1;
         return true;
@@ -251,6 +290,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       for (int e = 0; ok && e < n_list; ++e) {
         const int s = e % kStages;
         const uint32_t bits = list[e];
+        const int last_t = ((bits >> 20) & 0xFu) ? 1 : 0;
         bool k_waited = false;
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
@@ -279,6 +319,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                    kk > 0 ? 1u : 0u);
           }
           mma_commit(&s_ready[t]);
+          if (t == last_t) mma_commit(&k_empty[s]);
           pend[t] = e;
         }
         if (misc[4]) ok = false;
@@ -289,26 +330,43 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mma_commit(mma_done);
       mbar_wait(mma_done, 0);
     }
-  } else if (warp >= 4) {
+  }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+      tc_fence_after();
+      tmem_dealloc(tmem, 512);
+    }
+    return;
+  }
+
+  setmaxnreg_inc<112>();
+  {
     // ------------------------------------------------------------- softmax ---
-    const int t = (warp - 4) >> 2;
-    const int wq = warp & 3;
-    const int r = wq * 32 + lane;
+    const int sw = warp - kSoftmaxWarp0;       // 0..15
+    const int t = sw >> 3;                     // q-tile
+    const int hf = (sw >> 2) & 1;              // column half of the S tile
+    const int sub = warp & 3;                  // TMEM lane quarter = row group
+    const int r = sub * 32 + lane;
     const int row = (qtile0 + t) * kTileM + r;
     const bool row_valid = row < p.N;
     const int qh = (BLK == 64) ? (r >> 6) : 0;
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-    const uint32_t s_addr = lane_base + t * 128;
-    const uint32_t o_addr = lane_base + 256 + t * D;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(sub * 32) << 16);
+    const uint32_t s_addr = lane_base + t * 128 + hf * 64;     // this thread's 64 S columns
+    const uint32_t p_addr = lane_base + t * 128 + hf * 32;     // its 32 packed P columns
+    constexpr int kOCols = D / 2;                               // O columns this thread owns
+    const uint32_t o_addr = lane_base + 256 + t * D + hf * kOCols;
     const int cnt = misc[2 + t];
     const float sl2 = p.scale_log2;
     const float NEG_INF = -__int_as_float(0x7f800000);
+    const int bar_id = 1 + t;
+    float* red_t = red + t * (2 * 2 * kTileM);
 
-    float m_used = NEG_INF, m_true = NEG_INF, l_sum = 0.f;
+    float m_used = NEG_INF, m_true = NEG_INF, l_part = 0.f;
     uint32_t sphase = 0;
     int et = 0;
     bool ok = true;
-    uint32_t* my_votes = votes + (t * 4 + wq) * L::kVoteWords;
+    uint32_t* my_votes = votes + ((t * 4 + sub) * 2 + hf) * L::kVoteWords;
 
     if (cnt > 0) {
       for (int e = 0; e < n_list; ++e) {
@@ -316,56 +374,68 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const uint32_t bits = (ent >> (16 + 4 * t)) & 0xFu;
         if (!bits) continue;
         const int jt = static_cast<int>(ent & 0xFFFFu);
-        ok = mbar_wait(&s_ready[t], sphase);
-        ok = __all_sync(0xffffffffu, ok) && !misc[4];
+        // A bounded wait that runs out is only acted on at the barrier below,
+        // which every thread of the tile reaches, so no thread is left waiting.
+        const bool w_ok = __all_sync(0xffffffffu, mbar_wait(&s_ready[t], sphase));
+        sphase ^= 1u;
+        tc_fence_after();
+
+        float s[64];
+        if (w_ok) {
+          tmem_ld64(s_addr, s);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) s[c] = NEG_INF;
+        }
+
+        // mask columns past N and quadrants this row's q-block does not keep
+        const int valid_cols = min(64, p.N - jt * kTileN - hf * 64);
+        const bool keep_half = BLK == 128 ? true : ((bits >> (qh * 2 + hf)) & 1u);
+        if (valid_cols < 64 || !keep_half) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) s[c] = (keep_half && c < valid_cols) ? s[c] : NEG_INF;
+        }
+        float a0 = fmaxf(s[0], s[1]), a1 = fmaxf(s[2], s[3]);
+        float a2 = fmaxf(s[4], s[5]), a3 = fmaxf(s[6], s[7]);
+#pragma unroll
+        for (int c = 8; c < 64; c += 8) {
+          a0 = fmax3(a0, s[c + 0], s[c + 1]);
+          a1 = fmax3(a1, s[c + 2], s[c + 3]);
+          a2 = fmax3(a2, s[c + 4], s[c + 5]);
+          a3 = fmax3(a3, s[c + 6], s[c + 7]);
+        }
+        const float m_mine = fmax3(a0, a1, fmaxf(a2, a3));
+        // swap half maxima with the partner thread (same row, other half)
+        float* red_p = red_t + (et & 1) * (2 * kTileM);
+        red_p[hf * kTileM + r] = m_mine;
+        tc_fence_before();
+        ok = named_bar_and(bar_id, 256, w_ok && misc[4] == 0);
+        tc_fence_after();
         if (!ok) {
           misc[4] = 1;
           break;
         }
-        sphase ^= 1u;
-        tc_fence_after();
-
-        float s[kTileN];
-#pragma unroll
-        for (int c = 0; c < kTileN / 32; ++c) tmem_ld32(s_addr + c * 32, s + c * 32);
-
-        const int valid_cols = min(kTileN, p.N - jt * kTileN);
-        if (valid_cols < kTileN || (BLK == 64 && bits != 0xFu)) {
-          const bool k0 = BLK == 128 ? true : ((bits >> (qh * 2 + 0)) & 1u);
-          const bool k1 = BLK == 128 ? true : ((bits >> (qh * 2 + 1)) & 1u);
-#pragma unroll
-          for (int c = 0; c < kTileN; ++c) {
-            const bool keep = (c < valid_cols) && (c < 64 ? k0 : k1);
-            s[c] = keep ? s[c] : NEG_INF;
-          }
-        }
-        float mx0 = s[0], mx1 = s[64];
-#pragma unroll
-        for (int c = 1; c < 64; ++c) {
-          mx0 = fmaxf(mx0, s[c]);
-          mx1 = fmaxf(mx1, s[64 + c]);
-        }
+        const float m_other = red_p[(hf ^ 1) * kTileM + r];
+        const float mx0 = hf == 0 ? m_mine : m_other;
+        const float mx1 = hf == 0 ? m_other : m_mine;
         const float mx = fmaxf(mx0, mx1);
 
         if (p.write_skip) {
           if (BLK == 128) {
-            const bool pred = !row_valid || (mx < m_true - p.eps_raw);
+            if (hf == 0) {
+              const bool pred = !row_valid || (mx < m_true - p.eps_raw);
+              const bool all = __all_sync(0xffffffffu, pred);
+              if (lane == 0 && all) my_votes[e >> 5] |= 1u << (e & 31);
+            }
+          } else if ((bits >> (qh * 2 + hf)) & 1u) {
+            // k-block 2j is visited before 2j+1: half 1 tests against the
+            // running max including half 0 (-inf when half 0 is masked)
+            const float m_test = hf == 0 ? m_true : fmaxf(m_true, mx0);
+            const bool pred = !row_valid || (m_mine < m_test - p.eps_raw);
             const bool all = __all_sync(0xffffffffu, pred);
             if (lane == 0 && all) my_votes[e >> 5] |= 1u << (e & 31);
-            m_true = fmaxf(m_true, mx);
-          } else {
-#pragma unroll
-            for (int kh = 0; kh < 2; ++kh) {
-              if ((bits >> (qh * 2 + kh)) & 1u) {
-                const float mk = kh == 0 ? mx0 : mx1;
-                const bool pred = !row_valid || (mk < m_true - p.eps_raw);
-                const bool all = __all_sync(0xffffffffu, pred);
-                const int bi = e * 2 + kh;
-                if (lane == 0 && all) my_votes[bi >> 5] |= 1u << (bi & 31);
-                m_true = fmaxf(m_true, mk);
-              }
-            }
           }
+          m_true = fmaxf(m_true, mx);
         }
 
         // online softmax with a lazily updated reference maximum
@@ -373,11 +443,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (mx > m_used && (m_used == NEG_INF || (mx - m_used) * sl2 > 8.f)) {
           factor = (m_used == NEG_INF) ? 0.f : fast_exp2((m_used - mx) * sl2);
           m_used = mx;
-          l_sum *= factor;
+          l_part *= factor;
         }
         if (et > 0 && __any_sync(0xffffffffu, factor != 1.f)) {
 #pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
+          for (int c = 0; c < kOCols / 32; ++c) {
             float ov[32];
             tmem_ld32(o_addr + c * 32, ov);
 #pragma unroll
@@ -386,22 +456,33 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
           tmem_st_wait();
         }
+        // p = 2^(s*scale*log2e - m): pairs through packed fp32 ops; pairs
+        // kPolyPairFrom..15 of every 16 use the FMA-pipe polynomial.
         const float neg_m = (m_used == NEG_INF) ? 0.f : -m_used * sl2;
-        float acc0 = 0.f, acc1 = 0.f;
+        const float2 sl2v = make_float2(sl2, sl2), nmv = make_float2(neg_m, neg_m);
+        float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int c = 0; c < kTileN / 32; ++c) {
+        for (int ch = 0; ch < 2; ++ch) {
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float a = fast_exp2(fmaf(s[c * 32 + 2 * i], sl2, neg_m));
-            const float bb = fast_exp2(fmaf(s[c * 32 + 2 * i + 1], sl2, neg_m));
-            acc0 += a;
-            acc1 += bb;
-            pk[i] = pack_bf16x2(a, bb);
+            const int c = ch * 32 + 2 * i;
+            const float2 x = fma2(make_float2(s[c], s[c + 1]), sl2v, nmv);
+            float2 pe;
+            if (i >= kPolyPairFrom) {
+              pe = exp2_poly2(x);
+            } else {
+              pe.x = fast_exp2(x.x);
+              pe.y = fast_exp2(x.y);
+            }
+            if (i & 1) acc1 = add2(acc1, pe);
+            else acc0 = add2(acc0, pe);
+            pk[i] = pack_bf16x2(pe.x, pe.y);
           }
-          tmem_st16(s_addr + c * 16, pk);
+          tmem_st16(p_addr + ch * 16, pk);
         }
-        l_sum += acc0 + acc1;
+        const float2 at = add2(acc0, acc1);
+        l_part += at.x + at.y;
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&p_ready[t]);
@@ -416,10 +497,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (!ok) misc[4] = 1;
       tc_fence_after();
     }
+    // row sum = both halves' partial sums
+    float* red_l = red_t;
+    named_bar_sync(bar_id, 256);
+    red_l[hf * kTileM + r] = l_part;
+    named_bar_sync(bar_id, 256);
+    const float l_sum = l_part + red_l[(hf ^ 1) * kTileM + r];
     const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
-    __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * p.N + (row_valid ? row : 0)) * D;
+    __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * p.N + (row_valid ? row : 0)) * D + hf * kOCols;
 #pragma unroll 1
-    for (int c = 0; c < D / 32; ++c) {
+    for (int c = 0; c < kOCols / 32; ++c) {
       float ov[32];
       if (cnt > 0 && ok) {
         tmem_ld32(o_addr + c * 32, ov);
@@ -440,41 +527,39 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
       }
     }
-    if (p.lse && row_valid) {
+    if (p.lse && row_valid && hf == 0) {
       const float neg_m = (m_used == NEG_INF) ? 0.f : -m_used * sl2;
       p.lse[static_cast<size_t>(bh) * p.N + row] =
           l_sum > 0.f ? (log2f(l_sum) - neg_m) * 0.69314718055994531f : NEG_INF;
     }
 
     // ----------------------------------- skip bits: cross-warp AND at the end ---
-    if (p.write_skip && cnt > 0) {
-      named_bar_sync(1 + t, 128);
-      if (ok && !misc[4]) {
-        const int tid = wq * 32 + lane;
-        uint32_t* tv = votes + t * 4 * L::kVoteWords;
-        for (int e = tid; e < n_list; e += 128) {
-          const uint32_t ent = list[e];
-          const uint32_t bits = (ent >> (16 + 4 * t)) & 0xFu;
-          if (!bits) continue;
-          const int jt = static_cast<int>(ent & 0xFFFFu);
+    if (p.write_skip && cnt > 0 && ok && !misc[4]) {
+      const int tid = sw * 32 + lane - t * 256;   // 0..255 within the tile
+      // votes of the tile: [sub][half][words]
+      const uint32_t* tv = votes + t * 8 * L::kVoteWords;
+      for (int e = tid; e < n_list; e += 256) {
+        const uint32_t ent = list[e];
+        const uint32_t bits = (ent >> (16 + 4 * t)) & 0xFu;
+        if (!bits) continue;
+        const int jt = static_cast<int>(ent & 0xFFFFu);
+        const uint32_t word = e >> 5, bit = e & 31;
 #pragma unroll
-          for (int qq = 0; qq < QH; ++qq) {
+        for (int qq = 0; qq < QH; ++qq) {
 #pragma unroll
-            for (int kh = 0; kh < KH; ++kh) {
-              if (BLK == 64 && !((bits >> (qq * 2 + kh)) & 1u)) continue;
-              const int qb = (qtile0 + t) * QH + qq;
-              const int kb = jt * KH + kh;
-              const int bi = (BLK == 128) ? e : e * 2 + kh;
-              uint32_t all = 1u;
-              if (BLK == 128) {
+          for (int kh = 0; kh < KH; ++kh) {
+            if (BLK == 64 && !((bits >> (qq * 2 + kh)) & 1u)) continue;
+            const int qb = (qtile0 + t) * QH + qq;
+            const int kb = jt * KH + kh;
+            uint32_t all = 1u;
+            if (BLK == 128) {
 #pragma unroll
-                for (int w = 0; w < 4; ++w) all &= tv[w * L::kVoteWords + (bi >> 5)] >> (bi & 31);
-              } else {
+              for (int sb = 0; sb < 4; ++sb) all &= tv[(sb * 2 + 0) * L::kVoteWords + word] >> bit;
+            } else {
 #pragma unroll
-                for (int w = 2 * qq; w < 2 * qq + 2; ++w) all &= tv[w * L::kVoteWords + (bi >> 5)] >> (bi & 31);
-              }
-              p.skip_out[(static_cast<size_t>(bh) * p.nb + qb) * p.nb + kb] = static_cast<uint8_t>(all & 1u);
+              for (int sb = 2 * qq; sb < 2 * qq + 2; ++sb) all &= tv[(sb * 2 + kh) * L::kVoteWords + word] >> bit;
             }
+            p.skip_out[(static_cast<size_t>(bh) * p.nb + qb) * p.nb + kb] = static_cast<uint8_t>(all & 1u);
           }
         }
       }
@@ -483,10 +568,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, 512);
-  }
 }
 
 }  // namespace sa

@@ -14,6 +14,7 @@
 #include "sa_attn_fwd.cuh"
 #include "sa_common.cuh"
 #include "sa_masks.cuh"
+#include "sa_pyr_fwd.cuh"
 #include "sparse_attn.h"
 
 namespace {
@@ -79,6 +80,10 @@ cudaError_t init_device_kernels() {
     set(reinterpret_cast<const void*>(&sa::attn_fwd_kernel<128, 64>), sa::AttnSmem<128>::kAlloc);
     set(reinterpret_cast<const void*>(&sa::attn_fwd_kernel<64, 128>), sa::AttnSmem<64>::kAlloc);
     set(reinterpret_cast<const void*>(&sa::attn_fwd_kernel<64, 64>), sa::AttnSmem<64>::kAlloc);
+    set(reinterpret_cast<const void*>(&sa::pyr_fwd_kernel<128, 128>), sa::PyrSmem<128>::kAlloc);
+    set(reinterpret_cast<const void*>(&sa::pyr_fwd_kernel<128, 64>), sa::PyrSmem<128>::kAlloc);
+    set(reinterpret_cast<const void*>(&sa::pyr_fwd_kernel<64, 128>), sa::PyrSmem<64>::kAlloc);
+    set(reinterpret_cast<const void*>(&sa::pyr_fwd_kernel<64, 64>), sa::PyrSmem<64>::kAlloc);
     set(reinterpret_cast<const void*>(&sa::block_select_kernel),
         static_cast<int>(sa::select_smem_bytes(sa::kMaxSelect)));
     di.err = r;
@@ -165,7 +170,7 @@ sa_status sa_build_mask(const void* q, const void* k, int B, int H, int N, int d
   const float scale = 1.0f / std::sqrt(static_cast<float>(d));
   const auto* qb = static_cast<const __nv_bfloat16*>(q);
   const auto* kb = static_cast<const __nv_bfloat16*>(k);
-  dim3 g1(nb, BH, 2), g2(ceil_div(nb, 32), ceil_div(nb, 32), BH);
+  dim3 g1(nb, BH, 2), g2(ceil_div(nb, 64), ceil_div(nb, 64), BH);
   if (d == 128) {
     sa::block_means_kernel<128><<<g1, 128, 0, s>>>(qb, kb, N, block, nb, qmean, kmean);
     sa::block_scores_kernel<128><<<g2, 256, 0, s>>>(qmean, kmean, nb, scale, scores);
@@ -173,8 +178,23 @@ sa_status sa_build_mask(const void* q, const void* k, int B, int H, int N, int d
     sa::block_means_kernel<64><<<g1, 128, 0, s>>>(qb, kb, N, block, nb, qmean, kmean);
     sa::block_scores_kernel<64><<<g2, 256, 0, s>>>(qmean, kmean, nb, scale, scores);
   }
-  sa::block_select_kernel<<<static_cast<unsigned>(BH) * nb, sa::kSelectThreads, sa::select_smem_bytes(nb), s>>>(
-      scores, nb, mode, tau, c0, c1, c2, mask_out);
+  const long long nrows = static_cast<long long>(BH) * nb;
+  const unsigned warp_grid = static_cast<unsigned>((nrows + 3) / 4);
+  if (nb <= 32)
+    sa::block_select_warp_kernel<1><<<warp_grid, 128, 0, s>>>(scores, nb, nrows, mode, tau, c0, c1, c2, mask_out);
+  else if (nb <= 64)
+    sa::block_select_warp_kernel<2><<<warp_grid, 128, 0, s>>>(scores, nb, nrows, mode, tau, c0, c1, c2, mask_out);
+  else if (nb <= 128)
+    sa::block_select_warp_kernel<4><<<warp_grid, 128, 0, s>>>(scores, nb, nrows, mode, tau, c0, c1, c2, mask_out);
+  else if (nb <= 256)
+    sa::block_select_warp_kernel<8><<<warp_grid, 128, 0, s>>>(scores, nb, nrows, mode, tau, c0, c1, c2, mask_out);
+  else if (nb <= 512)
+    sa::block_select_warp_kernel<16><<<warp_grid, 128, 0, s>>>(scores, nb, nrows, mode, tau, c0, c1, c2, mask_out);
+  else if (nb <= 1024)
+    sa::block_select_warp_kernel<32><<<warp_grid, 128, 0, s>>>(scores, nb, nrows, mode, tau, c0, c1, c2, mask_out);
+  else
+    sa::block_select_kernel<<<static_cast<unsigned>(nrows), sa::kSelectThreads, sa::select_smem_bytes(nb), s>>>(
+        scores, nb, mode, tau, c0, c1, c2, mask_out);
   return cuda_status(cudaGetLastError());
 }
 
@@ -279,9 +299,59 @@ sa_status sa_pyramid_attn_fwd(const void* q, const void* k, const void* v, int B
                               const uint8_t* levels, int64_t lv_sb, int64_t lv_sh, int64_t lv_si,
                               const void* const* k_pool, const void* const* v_pool, float scale, void* o, float* lse,
                               void* stream) {
-  (void)q; (void)k; (void)v; (void)B; (void)H; (void)N; (void)d; (void)block; (void)levels;
-  (void)lv_sb; (void)lv_sh; (void)lv_si; (void)k_pool; (void)v_pool; (void)scale; (void)o; (void)lse; (void)stream;
-  return SA_ERR_UNSUPPORTED;
+  if (B < 0 || H < 0 || N < 0) return SA_ERR_INVALID_ARG;
+  if (std::isnan(scale) || scale < 0.f || std::isinf(scale)) return SA_ERR_INVALID_ARG;
+  if (B == 0 || H == 0 || N == 0) return SA_OK;
+  if (!valid_dim(d) || !valid_block(block)) return SA_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !o || !levels || !k_pool || !v_pool) return SA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return SA_ERR_INVALID_ARG;
+  if (lv_sb < 0 || lv_sh < 0 || lv_si < 0) return SA_ERR_INVALID_ARG;
+  for (int i = 0; i < 3; ++i)
+    if (!k_pool[i] || !v_pool[i] || !aligned16(k_pool[i]) || !aligned16(v_pool[i])) return SA_ERR_INVALID_ARG;
+  const int nb = ceil_div(N, block);
+  if (nb > sa::kPyrMaxBlocks) return SA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * H > 65535) return SA_ERR_UNSUPPORTED;
+  cudaError_t e = init_device_kernels();
+  if (e != cudaSuccess) return SA_ERR_CUDA;
+
+  const int BH = B * H;
+  CUtensorMap tq;
+  sa::PyrMaps maps;
+  if (!encode_rows_map(&tq, q, BH, N, d, sa::kTileM)) return SA_ERR_CUDA;
+  sa::PyrParams p;
+  for (int l = 0; l < 4; ++l) {
+    const int rows = ceil_div(N, 1 << l);
+    const void* kb = l == 0 ? k : k_pool[l - 1];
+    const void* vb = l == 0 ? v : v_pool[l - 1];
+    if (!encode_rows_map(&maps.k[l], kb, BH, rows, d, block >> l) ||
+        !encode_rows_map(&maps.v[l], vb, BH, rows, d, block >> l))
+      return SA_ERR_CUDA;
+    p.pool_rows[l] = rows;
+  }
+  if (scale == 0.f) scale = 1.0f / std::sqrt(static_cast<float>(d));
+  p.B = B;
+  p.H = H;
+  p.N = N;
+  p.nb = nb;
+  p.levels = levels;
+  p.lsb = lv_sb;
+  p.lsh = lv_sh;
+  p.lsi = lv_si;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  const int n_pairs = ceil_div(ceil_div(N, sa::kTileM), 2);
+  dim3 grid(n_pairs, BH);
+  cudaStream_t s = as_stream(stream);
+  if (d == 128 && block == 128)
+    sa::pyr_fwd_kernel<128, 128><<<grid, sa::kAttnThreads, sa::PyrSmem<128>::kAlloc, s>>>(tq, maps, p);
+  else if (d == 128 && block == 64)
+    sa::pyr_fwd_kernel<128, 64><<<grid, sa::kAttnThreads, sa::PyrSmem<128>::kAlloc, s>>>(tq, maps, p);
+  else if (d == 64 && block == 128)
+    sa::pyr_fwd_kernel<64, 128><<<grid, sa::kAttnThreads, sa::PyrSmem<64>::kAlloc, s>>>(tq, maps, p);
+  else
+    sa::pyr_fwd_kernel<64, 64><<<grid, sa::kAttnThreads, sa::PyrSmem<64>::kAlloc, s>>>(tq, maps, p);
+  return cuda_status(cudaGetLastError());
 }
 
 }  // extern "C"

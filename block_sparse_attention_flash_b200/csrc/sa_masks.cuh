@@ -103,39 +103,59 @@ __global__ void __launch_bounds__(128) block_means_kernel(const __nv_bfloat16* _
 }
 
 // ----------------------------------------------------------- block scores ---
-// grid (ceil(nb/32), ceil(nb/32), B*H), 256 threads; each thread 4 outputs of
-// a 32 x 32 tile of S = scale * Qbar Kbar^T, fp32 throughout.
+// grid (ceil(nb/64), ceil(nb/64), B*H), 256 threads; each thread owns a 4 x 4
+// patch of a 64 x 64 tile of S = scale * Qbar Kbar^T, fp32 throughout.  The
+// d dimension is walked in chunks of 32 staged (transposed) in shared memory.
 template <int D>
 __global__ void __launch_bounds__(256) block_scores_kernel(const float* __restrict__ qmean,
                                                            const float* __restrict__ kmean, int nb, float scale,
                                                            float* __restrict__ scores) {
-  __shared__ float sq[32][D + 1];
-  __shared__ float sk[32][D + 1];
+  __shared__ __align__(16) float sa[32][68];
+  __shared__ __align__(16) float sb[32][68];
   const int bh = blockIdx.z;
-  const int i0 = blockIdx.y * 32, j0 = blockIdx.x * 32;
+  const int i0 = blockIdx.y * 64, j0 = blockIdx.x * 64;
   const float* qm = qmean + static_cast<size_t>(bh) * nb * D;
   const float* km = kmean + static_cast<size_t>(bh) * nb * D;
-  for (int idx = threadIdx.x; idx < 32 * D; idx += 256) {
-    const int rr = idx / D, c = idx % D;
-    sq[rr][c] = (i0 + rr < nb) ? qm[static_cast<size_t>(i0 + rr) * D + c] : 0.f;
-    sk[rr][c] = (j0 + rr < nb) ? km[static_cast<size_t>(j0 + rr) * D + c] : 0.f;
-  }
-  __syncthreads();
-  const int jj = threadIdx.x & 31;
-  const int ib = (threadIdx.x >> 5) * 4;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  float acc[4][4];
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) acc[a][c] = 0.f;
+#pragma unroll 1
+  for (int kc = 0; kc < D; kc += 32) {
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int idx = threadIdx.x + u * 256;   // 512 float4 per operand chunk
+      const int rr = idx >> 3, c4 = (idx & 7) * 4;
+      const float4 av = (i0 + rr < nb) ? *reinterpret_cast<const float4*>(qm + static_cast<size_t>(i0 + rr) * D + kc + c4)
+                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4 bv = (j0 + rr < nb) ? *reinterpret_cast<const float4*>(km + static_cast<size_t>(j0 + rr) * D + kc + c4)
+                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+      sa[c4 + 0][rr] = av.x; sa[c4 + 1][rr] = av.y; sa[c4 + 2][rr] = av.z; sa[c4 + 3][rr] = av.w;
+      sb[c4 + 0][rr] = bv.x; sb[c4 + 1][rr] = bv.y; sb[c4 + 2][rr] = bv.z; sb[c4 + 3][rr] = bv.w;
+    }
+    __syncthreads();
 #pragma unroll 8
-  for (int c = 0; c < D; ++c) {
-    const float kv = sk[jj][c];
+    for (int k = 0; k < 32; ++k) {
+      const float4 a = *reinterpret_cast<const float4*>(&sa[k][ty * 4]);
+      const float4 bq = *reinterpret_cast<const float4*>(&sb[k][tx * 4]);
+      const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {bq.x, bq.y, bq.z, bq.w};
 #pragma unroll
-    for (int u = 0; u < 4; ++u) acc[u] = fmaf(sq[ib + u][c], kv, acc[u]);
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int w = 0; w < 4; ++w) acc[u][w] = fmaf(av[u], bv[w], acc[u][w]);
+    }
+    __syncthreads();
   }
-  const int j = j0 + jj;
-  if (j < nb) {
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int i = i0 + ib + u;
-      if (i < nb) scores[(static_cast<size_t>(bh) * nb + i) * nb + j] = acc[u] * scale;
+  for (int u = 0; u < 4; ++u) {
+    const int i = i0 + ty * 4 + u;
+    if (i >= nb) continue;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const int j = j0 + tx * 4 + w;
+      if (j < nb) scores[(static_cast<size_t>(bh) * nb + i) * nb + j] = acc[u][w] * scale;
     }
   }
 }
@@ -293,6 +313,112 @@ __global__ void __launch_bounds__(kSelectThreads) block_select_kernel(const floa
   __syncthreads();
   uint8_t* mrow = mask_out + row * nb;
   for (int j = threadIdx.x; j < nb; j += kSelectThreads) mrow[j] = out_row[j];
+}
+
+// Warp-per-row variant for rows of at most 32*E blocks (E <= 32): the keys
+// live in registers (E per lane, blocked: lane l holds ranks l*E .. l*E+E-1
+// after the sort) and the bitonic network uses in-register swaps for strides
+// below E and shuffles above.  Four rows per 128-thread CTA.
+template <int E>
+__global__ void __launch_bounds__(128) block_select_warp_kernel(const float* __restrict__ scores, int nb,
+                                                                long long nrows, int mode, float tau, int c0,
+                                                                int c1, int c2, uint8_t* __restrict__ mask_out) {
+  constexpr int P = 32 * E;
+  __shared__ uint8_t stage[4][P];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long row = static_cast<long long>(blockIdx.x) * 4 + warp;
+  if (row >= nrows) return;
+  const float* srow = scores + row * nb;
+  unsigned long long key[E];
+  float mx = -__int_as_float(0x7f800000);
+#pragma unroll
+  for (int k = 0; k < E; ++k) {
+    const int i = lane * E + k;
+    if (i < nb) {
+      const float sc = srow[i];
+      mx = fmaxf(mx, sc);
+      key[k] = (static_cast<unsigned long long>(~float_order_key(sc)) << 32) | static_cast<unsigned>(i);
+    } else {
+      key[k] = ~0ull;
+    }
+  }
+  float inv = 0.f;
+  if (mode == SA_MASK_TAU) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    float sum = 0.f;
+#pragma unroll
+    for (int k = 0; k < E; ++k) {
+      const int i = lane * E + k;
+      if (i < nb) sum += expf(srow[i] - mx);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    inv = 1.f / sum;
+  }
+  // bitonic sort, ascending keys (descending score, then ascending j)
+#pragma unroll
+  for (int size = 2; size <= P; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      if (stride >= E) {
+        const int lm = stride / E;
+        const bool lower = (lane & lm) == 0;
+#pragma unroll
+        for (int k = 0; k < E; ++k) {
+          const unsigned long long other = __shfl_xor_sync(0xffffffffu, key[k], lm);
+          const bool up = ((lane * E + k) & size) == 0;
+          const bool take_min = (up == lower);
+          key[k] = take_min ? (key[k] < other ? key[k] : other) : (key[k] > other ? key[k] : other);
+        }
+      } else {
+#pragma unroll
+        for (int k = 0; k < E; ++k) {
+          if ((k & stride) == 0) {
+            const int k2 = k | stride;
+            const bool up = ((lane * E + k) & size) == 0;
+            const unsigned long long a = key[k], b = key[k2];
+            if ((a > b) == up) {
+              key[k] = b;
+              key[k2] = a;
+            }
+          }
+        }
+      }
+    }
+  }
+  if (mode == SA_MASK_TAU) {
+    float pk[E];
+    float lsum = 0.f;
+#pragma unroll
+    for (int k = 0; k < E; ++k) {
+      const unsigned j = static_cast<unsigned>(key[k]);
+      pk[k] = key[k] != ~0ull ? expf(srow[j] - mx) * inv : 0.f;
+      lsum += pk[k];
+    }
+    float inc = lsum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
+    }
+    float before = inc - lsum;
+#pragma unroll
+    for (int k = 0; k < E; ++k) {
+      if (key[k] != ~0ull) stage[warp][static_cast<unsigned>(key[k])] = before < tau ? 1 : 0;
+      before += pk[k];
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < E; ++k) {
+      const int r = lane * E + k;
+      if (key[k] != ~0ull)
+        stage[warp][static_cast<unsigned>(key[k])] = r < c0 ? 1 : (r < c1 ? 2 : (r < c2 ? 3 : 4));
+    }
+  }
+  __syncwarp();
+  uint8_t* mrow = mask_out + row * nb;
+  for (int j = lane; j < nb; j += 32) mrow[j] = stage[warp][j];
 }
 
 // ----------------------------------------------------------- pyramid pool ---

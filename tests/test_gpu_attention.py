@@ -144,6 +144,9 @@ def test_rff_skips_small_eps(block):
 
 @pytest.mark.parametrize("block", [64, 128])
 def test_teacher_forced_chain_with_carry_and_alias(block):
+    """Four denoising steps.  Each step's skip_in is the oracle's skip_out of
+    the step before, handed to both sides, so a flagged bit cannot cascade and
+    no oracle input comes from the GPU."""
     wl = inputs.Workload("c", 1, 2, 128, 6, 16, 24, block, "lite", seed=43, sigma_s=2.0, sigma_t=1.5)
     steps = list(inputs.lite_chain_inputs(wl, 4))
     nb = wl.nblocks
@@ -154,8 +157,8 @@ def test_teacher_forced_chain_with_carry_and_alias(block):
         S, Sr, _ = _check_skip_step(q, k, v, block, mask, skip, eps=1.2, alias=(s % 2 == 1 and skip is not None))
         if skip is not None:
             assert np.all(S.numpy() >= skip.numpy())      # monotone carry
-        skip = S                                           # teacher forcing: GPU bits feed both sides
-        total = int(S.sum())
+        skip = torch.from_numpy(np.ascontiguousarray(Sr))
+        total = int(Sr.sum())
     assert total > 0
 
 

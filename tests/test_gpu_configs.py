@@ -1,0 +1,112 @@
+"""GPU parity at the workloads' full sizes, in the launch configuration the
+bench uses, on sampled outputs the oracle computes one q-block at a time.
+
+Inputs are drawn with the seeded generator on the device (the CPU draw of
+40 heads takes about a minute) and the heads the oracle needs are copied to
+the host.  Masks handed to the attention kernel come from the oracle, so no
+oracle input is ever produced by the CUDA library.
+"""
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_attention_flash_b200 import build, inputs, ops
+from oracle import masked_attention, lite_step, radial_mask, tau_mask
+from _parity import check_o, check_lse, check_bits, skip_flags
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    build.build()
+    ops.lib()
+    yield
+    ops.sa_get_device_status()
+
+
+def _sample_qblocks(nb, heads, per_head, seed):
+    g = np.random.default_rng(seed)
+    out = []
+    for h in heads:
+        rows = sorted(set([0, nb - 1] + list(g.choice(nb, size=per_head, replace=False))))
+        out += [(0, h, int(i)) for i in rows]
+    return out
+
+
+def _compare_rows(O, L, ref, block, N, what):
+    got_o, got_l, want_o, want_l = [], [], [], []
+    for (b, h, i), (o, l) in ref.items():
+        r0, r1 = i * block, min(N, (i + 1) * block)
+        got_o.append(O[b, h, r0:r1])
+        got_l.append(L[b, h, r0:r1])
+        want_o.append(o)
+        want_l.append(l)
+    check_o(torch.cat(got_o), np.concatenate(want_o), what)
+    check_lse(torch.cat(got_l), np.concatenate(want_l), what)
+
+
+def _head_slice(t, heads):
+    return t[:, heads].cpu()
+
+
+def test_hunyuan_720p_radial_full():
+    wl = inputs.WORKLOADS["hunyuan_720p_radial"]
+    q, k, v = inputs.rff_qkv(wl, device="cuda")
+    nb = wl.nblocks
+    rm = radial_mask(wl.T, wl.Hh, wl.Ww, wl.block)
+    lse = torch.empty(1, wl.H, wl.N, device="cuda")
+    O = ops.sa_sparse_attn_fwd(q, k, v, wl.block, mask=torch.from_numpy(rm).cuda(), lse=lse)
+    ops.sa_get_device_status()
+    heads = [0, 11, 23]
+    samples = _sample_qblocks(nb, range(len(heads)), 4, seed=1)
+    ref = masked_attention(_head_slice(q, heads), _head_slice(k, heads), _head_slice(v, heads), wl.block, rm,
+                           qblocks=samples)
+    _compare_rows(O[:, heads].cpu(), lse[:, heads].cpu(), ref, wl.block, wl.N, "radial 720p")
+
+
+def test_wan13b_480p_tau_full():
+    wl = inputs.WORKLOADS["wan13b_480p_tau"]
+    q, k, v = inputs.rff_qkv(wl, device="cuda")
+    nb = wl.nblocks
+    heads = [0, 5, 11]
+    qh, kh, vh = _head_slice(q, heads), _head_slice(k, heads), _head_slice(v, heads)
+    m_gpu = ops.sa_build_mask(q, k, wl.block, "tau", tau=wl.tau)
+    mr, flags, _ = tau_mask(qh, kh, wl.block, wl.tau, return_info=True)
+    check_bits(m_gpu[:, heads].cpu(), mr, flags, "tau mask 480p")
+    # attention on the oracle's mask for the sampled heads (all heads run)
+    m_all = m_gpu.clone()
+    m_all[:, heads] = torch.from_numpy(mr).cuda()
+    lse = torch.empty(1, wl.H, wl.N, device="cuda")
+    O = ops.sa_sparse_attn_fwd(q, k, v, wl.block, mask=m_all, lse=lse)
+    ops.sa_get_device_status()
+    samples = _sample_qblocks(nb, range(len(heads)), 4, seed=2)
+    ref = masked_attention(qh, kh, vh, wl.block, mr, qblocks=samples)
+    _compare_rows(O[:, heads].cpu(), lse[:, heads].cpu(), ref, wl.block, wl.N, "tau 480p attention")
+
+
+@pytest.mark.parametrize("eps", [10.0, 2.0])
+def test_wan14b_720p_lite_step_full(eps):
+    """One LiteAttention step at 75,600 tokens x 40 heads.  eps = 10 is the
+    workload's threshold (no block is skipped on this generator); eps = 2 makes
+    skips happen so that the bits are exercised at full size."""
+    wl = inputs.WORKLOADS["wan14b_720p_lite"]
+    q, k, v = inputs.rff_qkv(wl, device="cuda")
+    nb = wl.nblocks
+    skip_in = torch.zeros(1, wl.H, nb, nb, dtype=torch.uint8, device="cuda")
+    skip_out = torch.zeros_like(skip_in)
+    lse = torch.empty(1, wl.H, wl.N, device="cuda")
+    O = ops.sa_sparse_attn_fwd(q, k, v, wl.block, skip_in=skip_in, skip_out=skip_out, eps=eps, lse=lse)
+    ops.sa_get_device_status()
+    heads = [0, 13, 26, 39]
+    samples = _sample_qblocks(nb, range(len(heads)), 3, seed=3)
+    ref = lite_step(_head_slice(q, heads), _head_slice(k, heads), _head_slice(v, heads), wl.block, None, None,
+                    eps, qblocks=samples)
+    _compare_rows(O[:, heads].cpu(), lse[:, heads].cpu(), {key: val[:2] for key, val in ref.items()}, wl.block,
+                  wl.N, f"lite 720p eps={eps}")
+    S = skip_out[:, heads].cpu().numpy()
+    nflag_total = 0
+    for (b, hh, i), (_, _, srow, mrow) in ref.items():
+        nflag_total += check_bits(S[b, hh, i], srow, skip_flags(mrow), f"skip row {hh},{i}")
+    if eps == 2.0:
+        assert S.sum() > 0

@@ -99,3 +99,21 @@ def test_tau_mask_wan13b_480p_full():
     mr, flags, _ = tau_mask(q, k, wl.block, wl.tau, return_info=True)
     nflag = check_bits(m.cpu(), mr, flags, "tau 480p full")
     assert nflag <= 0.001 * mr.size
+
+
+@pytest.mark.parametrize("nb,mode", [(700, "tau"), (1000, "levels"), (1500, "tau"), (1500, "levels")])
+def test_select_paths_for_long_rows(nb, mode):
+    """Rows of 513-1024 blocks (widest register sort) and of more than 1024
+    blocks (shared-memory sort) against the oracle."""
+    block, d = 64, 64
+    N = block * nb - 17
+    g = torch.Generator().manual_seed(nb)
+    q = (torch.randn(1, 1, N, d, generator=g) * 0.5).to(torch.bfloat16)
+    k = (torch.randn(1, 1, N, d, generator=g) * 0.5).to(torch.bfloat16)
+    m = ops.sa_build_mask(q.cuda(), k.cuda(), block, mode, tau=0.6)
+    ops.sa_get_device_status()
+    if mode == "tau":
+        ref, flags, _ = tau_mask(q, k, block, 0.6, return_info=True)
+    else:
+        ref, flags, _ = level_map(q, k, block, (0.1, 0.3, 0.6), return_info=True)
+    check_bits(m.cpu(), ref, flags, f"{mode} nb={nb}")
