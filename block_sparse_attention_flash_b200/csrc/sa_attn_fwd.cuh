@@ -5,29 +5,34 @@
 // of one (b, h) and walks the union of their kept 128-column kv tiles in
 // ascending order.  Each kv tile is loaded once by TMA and feeds both q-tiles.
 //
-// Roles (640 threads = 20 warps, one CTA per SM; warps 2-3 only join the
-// final barrier, they keep the softmax warps aligned to TMEM lane quarters):
+// Roles (384 threads = 12 warps, one CTA per SM):
 //   warp 0       builds the kv-tile list from the mask / skip bytes, then one
 //                lane issues the TMA loads (Q once, K and V through 2-stage
 //                rings released separately; skipped tiles are never loaded:
 //                LiteAttention write-up, sections 3 and 6);
-//   warp 1       owns TMEM (512 columns) and one lane issues every
-//                tcgen05.mma: S_t = Q_t K^T (both operands from shared memory)
-//                and O_t += P_t V (A operand P_t read from TMEM, where the
-//                softmax wrote it over S_t);
-//   warps 4-11   online softmax of q-tile 0, warps 12-19 of q-tile 1.  Two
-//                threads per row: warps [4,8) take columns 0-63 of rows
-//                32*(warp%4) .. +31 (a warp may only touch its own TMEM lane
-//                quarter), warps [8,12) columns 64-127; the two halves swap
-//                their row maxima through shared memory once per kv tile.
-//                They evaluate the skip condition on the maxima they compute
-//                anyway (LiteAttention write-up, section 5), record it per
-//                warp and reduce across warps only at kernel end (section 6).
+//   warp 1       owns TMEM (512 columns); its lane 0 issues the tcgen05.mma of
+//                q-tile 0, warp 2's lane 0 those of q-tile 1, so that a tile's
+//                P -> PV hand-off never waits behind the other tile's issue:
+//                S_t = Q_t K^T (both operands in shared memory) and
+//                O_t += P_t V (A operand P_t in TMEM, written over S_t);
+//   warps 4-7    online softmax of q-tile 0, warps 8-11 of q-tile 1, one row
+//                per thread (a warp may only touch its own TMEM lane quarter).
+//                P goes back in two 64-column halves with one barrier each, so
+//                the first half of PV runs while the second half is computed.
+//                The two softmax warpgroups take turns (a token passed through
+//                the go barriers in list order), so that one tile's softmax
+//                runs while the tensor core works on the other tile instead of
+//                both competing for the same MUFU units.
+//                The skip condition is evaluated on the row maxima the softmax
+//                computes anyway (LiteAttention write-up, section 5), recorded
+//                per warp and reduced across warps at kernel end (section 6).
+// The producer/MMA warpgroup hands registers to the softmax warpgroups
+// (setmaxnreg); each role runs to its own final barrier.
 //
 // TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [384,384+D).
 // Shared memory: Q0, Q1, K[2], V[2] tiles of 128 x D bf16 in the 128-byte
 // swizzled layout TMA writes (each 64-column half is a [128 x 128 B] slab),
-// the kv list, the per-warp skip votes, the row-max exchange and mbarriers.
+// the kv list, the per-warp skip votes and the mbarriers.
 //
 // Block size 64: a 128-row tile holds q-blocks 2i, 2i+1 and a 128-column kv
 // tile holds k-blocks 2j, 2j+1; the list keeps per-quadrant bits and the
@@ -42,12 +47,15 @@ constexpr int kTileM = 128;
 constexpr int kTileN = 128;
 constexpr int kStages = 2;
 constexpr int kMaxKvTiles = 4096;
-constexpr int kAttnWarps = 20;
+constexpr int kAttnWarps = 12;
 constexpr int kAttnThreads = kAttnWarps * 32;
 constexpr int kSoftmaxWarp0 = 4;
 // Within each 16-pair chunk of a row, pairs [kPolyPairFrom, 16) take 2^x from
-// the FMA-pipe polynomial instead of the MUFU unit (balances the two pipes).
-constexpr int kPolyPairFrom = 12;
+// the FMA-pipe polynomial instead of the MUFU unit.  Measured on B200 with one
+// softmax warp per sub-partition, offloading 12-37 % of the pairs was slower
+// than none (the polynomial's issue cost exceeds the MUFU time it frees), so
+// the offload is off; the polynomial stays for the pyramid kernel's tuning.
+constexpr int kPolyPairFrom = 16;
 
 struct AttnParams {
   int B, H, N;
@@ -72,12 +80,12 @@ struct AttnSmem {
   static constexpr int kOffK = 2 * kTileBytes;
   static constexpr int kOffV = kOffK + kStages * kTileBytes;
   static constexpr int kOffList = kOffV + kStages * kTileBytes;
-  static constexpr int kVoteWords = kMaxKvTiles / 32;      // per softmax warp
+  static constexpr int kVoteWords = kMaxKvTiles * 2 / 32;  // per softmax warp
   static constexpr int kOffVotes = kOffList + kMaxKvTiles * 4;
-  static constexpr int kOffRed = kOffVotes + 16 * kVoteWords * 4;
-  static constexpr int kRedFloats = 2 * 2 * 2 * kTileM;    // [tile][parity][half][row]
-  static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2 + 2 + 1;
-  static constexpr int kOffBar = kOffRed + kRedFloats * 4;
+  // q_full, k_full[2], v_full[2], k_empty[2], v_empty[2], s_ready[2],
+  // pa[2], pb[2], o_final[2], mma_done[2], go[2]
+  static constexpr int kNumBars = 1 + 4 * kStages + 2 * 6;
+  static constexpr int kOffBar = kOffVotes + 8 * kVoteWords * 4;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffMisc + 64;
   static constexpr int kAlloc = kBytes + 1024;
@@ -102,6 +110,32 @@ __device__ __forceinline__ bool named_bar_and(int id, int nthreads, bool v) {
   return r != 0;
 }
 
+// p = 2^x for 64 logits s[c] (x = s * sl2 + neg_m), packed to 32 bf16 pairs;
+// returns the fp32 sum.  Pairs with (i & 15) >= kPolyPairFrom take 2^x from
+// the FMA-pipe polynomial, the rest from the MUFU ex2 (the MUFU unit is the
+// bottleneck of a softmax row; the polynomial fills issue slots it leaves).
+__device__ __forceinline__ float exp_pack_64(const float* s, float sl2, float neg_m, uint32_t* pk) {
+  float acc[8];
+#pragma unroll
+  for (int a = 0; a < 8; ++a) acc[a] = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const float x0 = fmaf(s[2 * i], sl2, neg_m), x1 = fmaf(s[2 * i + 1], sl2, neg_m);
+    float p0, p1;
+    if ((i & 15) >= kPolyPairFrom) {
+      p0 = exp2_poly(x0);
+      p1 = exp2_poly(x1);
+    } else {
+      p0 = fast_exp2(x0);
+      p1 = fast_exp2(x1);
+    }
+    acc[(2 * i) & 7] += p0;
+    acc[(2 * i + 1) & 7] += p1;
+    pk[i] = pack_bf16x2(p0, p1);
+  }
+  return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+}
+
 template <int D, int BLK>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -117,17 +151,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint32_t* list = reinterpret_cast<uint32_t*>(smem + L::kOffList);
   uint32_t* votes = reinterpret_cast<uint32_t*>(smem + L::kOffVotes);
-  float* red = reinterpret_cast<float*>(smem + L::kOffRed);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;
-  uint64_t* v_full = bars + 1 + kStages;
-  uint64_t* k_empty = bars + 1 + 2 * kStages;
-  uint64_t* v_empty = bars + 1 + 3 * kStages;
-  uint64_t* s_ready = bars + 1 + 4 * kStages;
-  uint64_t* p_ready = s_ready + 2;
-  uint64_t* o_final = p_ready + 2;
+  uint64_t* v_full = k_full + kStages;
+  uint64_t* k_empty = v_full + kStages;
+  uint64_t* v_empty = k_empty + kStages;
+  uint64_t* s_ready = v_empty + kStages;
+  uint64_t* pa = s_ready + 2;
+  uint64_t* pb = pa + 2;
+  uint64_t* o_final = pb + 2;
   uint64_t* mma_done = o_final + 2;
+  uint64_t* go = mma_done + 2;
   volatile int* misc = reinterpret_cast<volatile int*>(smem + L::kOffMisc);
   // misc[0] TMEM base, [1] list length, [2] / [3] kv tiles of q-tile 0 / 1, [4] abort flag
 
@@ -136,7 +171,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int b = bh / p.H, h = bh - (bh / p.H) * p.H;
   const int qtile0 = 2 * pair;
 
-  for (int i = threadIdx.x; i < 16 * L::kVoteWords; i += kAttnThreads) votes[i] = 0;
+  for (int i = threadIdx.x; i < 8 * L::kVoteWords; i += kAttnThreads) votes[i] = 0;
 
   if (warp == 0) {
     // ---- kv-tile list: union over the two q-tiles, per-quadrant keep bits ----
@@ -179,8 +214,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       misc[3] = c1;
       misc[4] = 0;
       for (int i = 0; i < L::kNumBars; ++i) {
-        const bool softmax_arrivals = (&bars[i] == &p_ready[0]) || (&bars[i] == &p_ready[1]);
-        mbar_init(&bars[i], softmax_arrivals ? 256u : 1u);
+        uint32_t count = 1;
+        if (&bars[i] == &k_empty[0] || &bars[i] == &k_empty[1] || &bars[i] == &v_empty[0] ||
+            &bars[i] == &v_empty[1])
+          count = 2;  // one arrival from each q-tile's MMA issuer
+        if (&bars[i] == &pa[0] || &bars[i] == &pa[1] || &bars[i] == &pb[0] || &bars[i] == &pb[1] ||
+            &bars[i] == &go[0] || &bars[i] == &go[1])
+          count = 128;  // every softmax thread of the tile
+        mbar_init(&bars[i], count);
       }
       fence_mbar_init();
       tma_prefetch_desc(&tmQ);
@@ -197,140 +238,130 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   const uint32_t tmem = static_cast<uint32_t>(misc[0]);
   const int n_list = misc[1];
-  const uint32_t sQ = smem_addr(smem + L::kOffQ);
-  const uint32_t sK = smem_addr(smem + L::kOffK);
-  const uint32_t sV = smem_addr(smem + L::kOffV);
 
   if (warp < kSoftmaxWarp0) {
-    // Register split: this warpgroup gives up registers the softmax rows use.
-    // Each role runs to its own final barrier so the two register budgets
-    // never meet in shared code.
-    setmaxnreg_dec<32>();
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer ---
-    if (lane == 0 && n_list > 0) {
-      const int cnt0 = misc[2], cnt1 = misc[3];
-      const uint32_t qbytes = static_cast<uint32_t>((cnt0 > 0) + (cnt1 > 0)) * L::kTileBytes;
-      mbar_arrive_expect_tx(q_full, qbytes);
-#pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        if ((t == 0 ? cnt0 : cnt1) == 0) continue;
-#pragma unroll
-        for (int hd = 0; hd < D / 64; ++hd)
-          tma_load_3d(&tmQ, q_full, smem + L::kOffQ + t * L::kTileBytes + hd * kHalfBytes, hd * 64,
-                      (qtile0 + t) * kTileM, bh);
-      }
-      int issued = 0;
-      for (int e = 0; e < n_list; ++e) {
-        const int s = e % kStages;
-        const uint32_t par = ((e / kStages) - 1) & 1;
-        if (e >= kStages && (misc[4] || !mbar_wait(&k_empty[s], par))) {
-          misc[4] = 1;
-          break;
-        }
-        const int row = static_cast<int>(list[e] & 0xFFFFu) * kTileN;
-        mbar_arrive_expect_tx(&k_full[s], L::kTileBytes);
-#pragma unroll
-        for (int hd = 0; hd < D / 64; ++hd)
-          tma_load_3d(&tmK, &k_full[s], smem + L::kOffK + s * L::kTileBytes + hd * kHalfBytes, hd * 64, row, bh);
-        if (e >= kStages && !mbar_wait(&v_empty[s], par)) {
-          misc[4] = 1;
-          issued = e;
-          mbar_wait(&k_full[s], (e / kStages) & 1);
-          break;
-        }
-        mbar_arrive_expect_tx(&v_full[s], L::kTileBytes);
-#pragma unroll
-        for (int hd = 0; hd < D / 64; ++hd)
-          tma_load_3d(&tmV, &v_full[s], smem + L::kOffV + s * L::kTileBytes + hd * kHalfBytes, hd * 64, row, bh);
-        issued = e + 1;
-      }
-      // Loads still in flight must land before the CTA can exit.
-      for (int e = (issued > kStages ? issued - kStages : 0); e < issued; ++e) {
-        const int s = e % kStages;
-        mbar_wait(&k_full[s], (e / kStages) & 1);
-        mbar_wait(&v_full[s], (e / kStages) & 1);
-      }
-      if ((cnt0 | cnt1) != 0) mbar_wait(q_full, 0);
-    }
-  } else if (warp == 1) {
-    // ----------------------------------------------------------- MMA issue ---
-    if (lane == 0 && n_list > 0) {
-      const int cnt[2] = {misc[2], misc[3]};
-      bool ok = mbar_wait(q_full, 0);
-      if (!ok) misc[4] = 1;
-      int pend[2] = {-1, -1};
-      int done_pv[2] = {0, 0};
-      uint32_t pphase[2] = {0u, 0u};
-      int users[kStages];
-#pragma unroll
-      for (int s = 0; s < kStages; ++s) users[s] = 0;
-
-      auto issue_pv = [&](int t) -> bool {
-        const int e = pend[t];
-        const int s = e % kStages;
-        if (!mbar_wait(&p_ready[t], pphase[t])) return false;
-        pphase[t] ^= 1u;
-        if (!mbar_wait(&v_full[s], (e / kStages) & 1)) return false;
-        tc_fence_after();
-        const uint32_t d_tmem = tmem + 256 + t * D;
-        const uint32_t a_tmem = tmem + t * 128;
-        const uint32_t vbase = sV + s * L::kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < kTileN / 16; ++kk) {
-          const uint64_t bdesc = smem_desc(vbase + kk * 16 * 128, kHalfBytes, 1024);
-          mma_ts(d_tmem, a_tmem + kk * 8, bdesc, kIdescPV, (done_pv[t] == 0 && kk == 0) ? 0u : 1u);
-        }
-        if (--users[s] == 0) mma_commit(&v_empty[s]);
-        if (++done_pv[t] == cnt[t]) mma_commit(&o_final[t]);
-        pend[t] = -1;
-        return true;
-      };
-
-      for (int e = 0; ok && e < n_list; ++e) {
-        const int s = e % kStages;
-        const uint32_t bits = list[e];
-        const int last_t = ((bits >> 20) & 0xFu) ? 1 : 0;
-        bool k_waited = false;
+    setmaxnreg_dec<56>();
+    if (warp == 0) {
+      // ---------------------------------------------------------- producer ---
+      if (lane == 0 && n_list > 0) {
+        const int cnt0 = misc[2], cnt1 = misc[3];
+        const uint32_t qbytes = static_cast<uint32_t>((cnt0 > 0) + (cnt1 > 0)) * L::kTileBytes;
+        mbar_arrive_expect_tx(q_full, qbytes);
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
-          if (pend[t] >= 0 && !issue_pv(t)) {
+          if ((t == 0 ? cnt0 : cnt1) == 0) continue;
+#pragma unroll
+          for (int hd = 0; hd < D / 64; ++hd)
+            tma_load_3d(&tmQ, q_full, smem + L::kOffQ + t * L::kTileBytes + hd * kHalfBytes, hd * 64,
+                        (qtile0 + t) * kTileM, bh);
+        }
+        int issued = 0;
+        for (int e = 0; e < n_list; ++e) {
+          const int s = e % kStages;
+          const uint32_t par = ((e / kStages) - 1) & 1;
+          if (e >= kStages && (misc[4] || !mbar_wait(&k_empty[s], par))) {
+            misc[4] = 1;
+            break;
+          }
+          const int row = static_cast<int>(list[e] & 0xFFFFu) * kTileN;
+          mbar_arrive_expect_tx(&k_full[s], L::kTileBytes);
+#pragma unroll
+          for (int hd = 0; hd < D / 64; ++hd)
+            tma_load_3d(&tmK, &k_full[s], smem + L::kOffK + s * L::kTileBytes + hd * kHalfBytes, hd * 64, row, bh);
+          if (e >= kStages && !mbar_wait(&v_empty[s], par)) {
+            misc[4] = 1;
+            issued = e;
+            mbar_wait(&k_full[s], (e / kStages) & 1);
+            break;
+          }
+          mbar_arrive_expect_tx(&v_full[s], L::kTileBytes);
+#pragma unroll
+          for (int hd = 0; hd < D / 64; ++hd)
+            tma_load_3d(&tmV, &v_full[s], smem + L::kOffV + s * L::kTileBytes + hd * kHalfBytes, hd * 64, row, bh);
+          issued = e + 1;
+        }
+        // Loads still in flight must land before the CTA can exit.
+        for (int e = (issued > kStages ? issued - kStages : 0); e < issued; ++e) {
+          const int s = e % kStages;
+          mbar_wait(&k_full[s], (e / kStages) & 1);
+          mbar_wait(&v_full[s], (e / kStages) & 1);
+        }
+        if ((cnt0 | cnt1) != 0) mbar_wait(q_full, 0);
+      }
+    } else if (warp <= 2) {
+      // ---------------------------------------------- MMA issue, q-tile t ---
+      const int t = warp - 1;
+      if (lane == 0 && n_list > 0) {
+        const int cnt = misc[2 + t];
+        bool ok = mbar_wait(q_full, 0);
+        const uint64_t dq = smem_desc(smem_addr(smem + L::kOffQ + t * L::kTileBytes), 16, 1024);
+        const uint64_t dk0 = smem_desc(smem_addr(smem + L::kOffK), 16, 1024);
+        const uint64_t dv0 = smem_desc(smem_addr(smem + L::kOffV), kHalfBytes, 1024);
+        constexpr uint64_t kStageStep = L::kTileBytes >> 4;   // descriptor units
+        const uint32_t s_tmem = tmem + t * 128;
+        const uint32_t o_tmem = tmem + 256 + t * D;
+        int pend = -1, done = 0;
+        uint32_t pph = 0;
+        // O_t += P_t V of entry `pend`: first half as soon as it is ready
+        auto issue_pv = [&]() -> bool {
+          const int ps = pend % kStages;
+          const uint64_t dv = dv0 + ps * kStageStep;
+          if (!mbar_wait(&pa[t], pph) || !mbar_wait(&v_full[ps], (pend / kStages) & 1)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ts(o_tmem, s_tmem + kk * 8, dv + ((kk * 16 * 128) >> 4), kIdescPV, (done == 0 && kk == 0) ? 0u : 1u);
+          if (!mbar_wait(&pb[t], pph)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 4; kk < 8; ++kk)
+            mma_ts(o_tmem, s_tmem + kk * 8, dv + ((kk * 16 * 128) >> 4), kIdescPV, 1u);
+          pph ^= 1u;
+          mma_commit(&v_empty[ps]);
+          if (++done == cnt) mma_commit(&o_final[t]);
+          pend = -1;
+          return true;
+        };
+        for (int e = 0; ok && e < n_list; ++e) {
+          const int s = e % kStages;
+          const uint32_t par = (e / kStages) & 1;
+          if (pend >= 0 && !issue_pv()) {
             ok = false;
             break;
           }
-          if (((bits >> (16 + 4 * t)) & 0xFu) == 0) continue;
-          if (!k_waited) {
-            if (!mbar_wait(&k_full[s], (e / kStages) & 1)) {
+          // every entry's K must have landed before this tile reports the slot
+          // free, so the two arrivals on k_empty / v_empty stay in one phase
+          if (!mbar_wait(&k_full[s], par)) {
+            ok = false;
+            break;
+          }
+          if ((list[e] >> (16 + 4 * t)) & 0xFu) {
+            tc_fence_after();
+            const uint64_t dk = dk0 + s * kStageStep;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint64_t off = static_cast<uint64_t>((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+              mma_ss(s_tmem, dq + off, dk + off, kIdescS, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(&s_ready[t]);
+            mma_commit(&k_empty[s]);
+            pend = e;
+          } else {
+            mma_commit(&k_empty[s]);
+            if (!mbar_wait(&v_full[s], par)) {
               ok = false;
               break;
             }
-            k_waited = true;
-            users[s] = 0;
+            mma_commit(&v_empty[s]);
           }
-          ++users[s];
-          tc_fence_after();
-          const uint32_t d_tmem = tmem + t * 128;
-          const uint32_t qbase = sQ + t * L::kTileBytes;
-          const uint32_t kbase = sK + s * L::kTileBytes;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-            mma_ss(d_tmem, smem_desc(qbase + off, 16, 1024), smem_desc(kbase + off, 16, 1024), kIdescS,
-                   kk > 0 ? 1u : 0u);
-          }
-          mma_commit(&s_ready[t]);
-          if (t == last_t) mma_commit(&k_empty[s]);
-          pend[t] = e;
+          if (misc[4]) ok = false;
         }
-        if (misc[4]) ok = false;
+        if (ok && pend >= 0 && !issue_pv()) ok = false;
+        if (!ok) misc[4] = 1;
+        mma_commit(&mma_done[t]);
+        mbar_wait(&mma_done[t], 0);
       }
-      for (int t = 0; ok && t < 2; ++t)
-        if (pend[t] >= 0 && !issue_pv(t)) ok = false;
-      if (!ok) misc[4] = 1;
-      mma_commit(mma_done);
-      mbar_wait(mma_done, 0);
     }
-  }
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -340,33 +371,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     return;
   }
 
-  setmaxnreg_inc<112>();
+  setmaxnreg_inc<224>();
   {
     // ------------------------------------------------------------- softmax ---
-    const int sw = warp - kSoftmaxWarp0;       // 0..15
-    const int t = sw >> 3;                     // q-tile
-    const int hf = (sw >> 2) & 1;              // column half of the S tile
-    const int sub = warp & 3;                  // TMEM lane quarter = row group
-    const int r = sub * 32 + lane;
+    const int t = (warp - kSoftmaxWarp0) >> 2;
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;
     const int row = (qtile0 + t) * kTileM + r;
     const bool row_valid = row < p.N;
     const int qh = (BLK == 64) ? (r >> 6) : 0;
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(sub * 32) << 16);
-    const uint32_t s_addr = lane_base + t * 128 + hf * 64;     // this thread's 64 S columns
-    const uint32_t p_addr = lane_base + t * 128 + hf * 32;     // its 32 packed P columns
-    constexpr int kOCols = D / 2;                               // O columns this thread owns
-    const uint32_t o_addr = lane_base + 256 + t * D + hf * kOCols;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    const uint32_t s_addr = lane_base + t * 128;
+    const uint32_t o_addr = lane_base + 256 + t * D;
     const int cnt = misc[2 + t];
     const float sl2 = p.scale_log2;
     const float NEG_INF = -__int_as_float(0x7f800000);
-    const int bar_id = 1 + t;
-    float* red_t = red + t * (2 * 2 * kTileM);
 
-    float m_used = NEG_INF, m_true = NEG_INF, l_part = 0.f;
-    uint32_t sphase = 0;
+    float m_used = NEG_INF, m_true = NEG_INF, l_sum = 0.f;
+    uint32_t sphase = 0, gphase = 0;
     int et = 0;
     bool ok = true;
-    uint32_t* my_votes = votes + ((t * 4 + sub) * 2 + hf) * L::kVoteWords;
+    uint32_t* my_votes = votes + (t * 4 + wq) * L::kVoteWords;
 
     if (cnt > 0) {
       for (int e = 0; e < n_list; ++e) {
@@ -374,68 +399,72 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const uint32_t bits = (ent >> (16 + 4 * t)) & 0xFu;
         if (!bits) continue;
         const int jt = static_cast<int>(ent & 0xFFFFu);
-        // A bounded wait that runs out is only acted on at the barrier below,
-        // which every thread of the tile reaches, so no thread is left waiting.
-        const bool w_ok = __all_sync(0xffffffffu, mbar_wait(&s_ready[t], sphase));
-        sphase ^= 1u;
-        tc_fence_after();
-
-        float s[64];
-        if (w_ok) {
-          tmem_ld64(s_addr, s);
-        } else {
-#pragma unroll
-          for (int c = 0; c < 64; ++c) s[c] = NEG_INF;
+        // wait for our turn unless this is the first (entry, tile) phase
+        const bool has_prior = e > 0 || (t == 1 && ((ent >> 16) & 0xFu) != 0);
+        bool w_ok = true;
+        if (has_prior) {
+          w_ok = mbar_wait(&go[t], gphase);
+          gphase ^= 1u;
         }
-
-        // mask columns past N and quadrants this row's q-block does not keep
-        const int valid_cols = min(64, p.N - jt * kTileN - hf * 64);
-        const bool keep_half = BLK == 128 ? true : ((bits >> (qh * 2 + hf)) & 1u);
-        if (valid_cols < 64 || !keep_half) {
-#pragma unroll
-          for (int c = 0; c < 64; ++c) s[c] = (keep_half && c < valid_cols) ? s[c] : NEG_INF;
-        }
-        float a0 = fmaxf(s[0], s[1]), a1 = fmaxf(s[2], s[3]);
-        float a2 = fmaxf(s[4], s[5]), a3 = fmaxf(s[6], s[7]);
-#pragma unroll
-        for (int c = 8; c < 64; c += 8) {
-          a0 = fmax3(a0, s[c + 0], s[c + 1]);
-          a1 = fmax3(a1, s[c + 2], s[c + 3]);
-          a2 = fmax3(a2, s[c + 4], s[c + 5]);
-          a3 = fmax3(a3, s[c + 6], s[c + 7]);
-        }
-        const float m_mine = fmax3(a0, a1, fmaxf(a2, a3));
-        // swap half maxima with the partner thread (same row, other half)
-        float* red_p = red_t + (et & 1) * (2 * kTileM);
-        red_p[hf * kTileM + r] = m_mine;
-        tc_fence_before();
-        ok = named_bar_and(bar_id, 256, w_ok && misc[4] == 0);
-        tc_fence_after();
+        ok = __all_sync(0xffffffffu, w_ok && mbar_wait(&s_ready[t], sphase)) && misc[4] == 0;
         if (!ok) {
           misc[4] = 1;
           break;
         }
-        const float m_other = red_p[(hf ^ 1) * kTileM + r];
-        const float mx0 = hf == 0 ? m_mine : m_other;
-        const float mx1 = hf == 0 ? m_other : m_mine;
+        sphase ^= 1u;
+        tc_fence_after();
+
+        float s[kTileN];
+        tmem_ld128(s_addr, s);
+
+        const int valid_cols = min(kTileN, p.N - jt * kTileN);
+        if (valid_cols < kTileN || (BLK == 64 && bits != 0xFu)) {
+          const bool k0 = BLK == 128 ? true : ((bits >> (qh * 2 + 0)) & 1u);
+          const bool k1 = BLK == 128 ? true : ((bits >> (qh * 2 + 1)) & 1u);
+#pragma unroll
+          for (int c = 0; c < kTileN; ++c) {
+            const bool keep = (c < valid_cols) && (c < 64 ? k0 : k1);
+            s[c] = keep ? s[c] : NEG_INF;
+          }
+        }
+        // row maxima of the two 64-column halves: four independent chains each
+        float mxh[2];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const float* sh = s + 64 * hh;
+          float a0 = fmaxf(sh[0], sh[1]), a1 = fmaxf(sh[2], sh[3]);
+          float a2 = fmaxf(sh[4], sh[5]), a3 = fmaxf(sh[6], sh[7]);
+#pragma unroll
+          for (int c = 8; c < 64; c += 8) {
+            a0 = fmax3(a0, sh[c + 0], sh[c + 1]);
+            a1 = fmax3(a1, sh[c + 2], sh[c + 3]);
+            a2 = fmax3(a2, sh[c + 4], sh[c + 5]);
+            a3 = fmax3(a3, sh[c + 6], sh[c + 7]);
+          }
+          mxh[hh] = fmax3(a0, a1, fmaxf(a2, a3));
+        }
+        const float mx0 = mxh[0], mx1 = mxh[1];
         const float mx = fmaxf(mx0, mx1);
 
         if (p.write_skip) {
           if (BLK == 128) {
-            if (hf == 0) {
-              const bool pred = !row_valid || (mx < m_true - p.eps_raw);
-              const bool all = __all_sync(0xffffffffu, pred);
-              if (lane == 0 && all) my_votes[e >> 5] |= 1u << (e & 31);
-            }
-          } else if ((bits >> (qh * 2 + hf)) & 1u) {
-            // k-block 2j is visited before 2j+1: half 1 tests against the
-            // running max including half 0 (-inf when half 0 is masked)
-            const float m_test = hf == 0 ? m_true : fmaxf(m_true, mx0);
-            const bool pred = !row_valid || (m_mine < m_test - p.eps_raw);
+            const bool pred = !row_valid || (mx < m_true - p.eps_raw);
             const bool all = __all_sync(0xffffffffu, pred);
             if (lane == 0 && all) my_votes[e >> 5] |= 1u << (e & 31);
+            m_true = fmaxf(m_true, mx);
+          } else {
+#pragma unroll
+            for (int kh = 0; kh < 2; ++kh) {
+              if ((bits >> (qh * 2 + kh)) & 1u) {
+                const float mk = kh == 0 ? mx0 : mx1;
+                const bool pred = !row_valid || (mk < m_true - p.eps_raw);
+                const bool all = __all_sync(0xffffffffu, pred);
+                const int bi = e * 2 + kh;
+                if (lane == 0 && all) my_votes[bi >> 5] |= 1u << (bi & 31);
+                m_true = fmaxf(m_true, mk);
+              }
+            }
           }
-          m_true = fmaxf(m_true, mx);
         }
 
         // online softmax with a lazily updated reference maximum
@@ -443,11 +472,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (mx > m_used && (m_used == NEG_INF || (mx - m_used) * sl2 > 8.f)) {
           factor = (m_used == NEG_INF) ? 0.f : fast_exp2((m_used - mx) * sl2);
           m_used = mx;
-          l_part *= factor;
+          l_sum *= factor;
         }
         if (et > 0 && __any_sync(0xffffffffu, factor != 1.f)) {
 #pragma unroll 1
-          for (int c = 0; c < kOCols / 32; ++c) {
+          for (int c = 0; c < D / 32; ++c) {
             float ov[32];
             tmem_ld32(o_addr + c * 32, ov);
 #pragma unroll
@@ -456,57 +485,47 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
           tmem_st_wait();
         }
-        // p = 2^(s*scale*log2e - m): pairs through packed fp32 ops; pairs
-        // kPolyPairFrom..15 of every 16 use the FMA-pipe polynomial.
         const float neg_m = (m_used == NEG_INF) ? 0.f : -m_used * sl2;
-        const float2 sl2v = make_float2(sl2, sl2), nmv = make_float2(neg_m, neg_m);
-        float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int ch = 0; ch < 2; ++ch) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int c = ch * 32 + 2 * i;
-            const float2 x = fma2(make_float2(s[c], s[c + 1]), sl2v, nmv);
-            float2 pe;
-            if (i >= kPolyPairFrom) {
-              pe = exp2_poly2(x);
-            } else {
-              pe.x = fast_exp2(x.x);
-              pe.y = fast_exp2(x.y);
-            }
-            if (i & 1) acc1 = add2(acc1, pe);
-            else acc0 = add2(acc0, pe);
-            pk[i] = pack_bf16x2(pe.x, pe.y);
-          }
-          tmem_st16(p_addr + ch * 16, pk);
+        // first 64 columns -> P[0, 32): the MMA warp starts PV on them at once
+        {
+          uint32_t pk[32];
+          l_sum += exp_pack_64(s, sl2, neg_m, pk);
+          tmem_st32(s_addr, reinterpret_cast<const float*>(pk));
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(&pa[t]);
         }
-        const float2 at = add2(acc0, acc1);
-        l_part += at.x + at.y;
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(&p_ready[t]);
+        {
+          uint32_t pk[32];
+          l_sum += exp_pack_64(s + 64, sl2, neg_m, pk);
+          tmem_st32(s_addr + 32, reinterpret_cast<const float*>(pk));
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(&pb[t]);
+        }
+        // pass the turn to the owner of the next (entry, tile) phase
+        if (t == 0 && ((ent >> 20) & 0xFu) != 0) {
+          mbar_arrive(&go[1]);
+        } else if (e + 1 < n_list) {
+          mbar_arrive(&go[((list[e + 1] >> 16) & 0xFu) != 0 ? 0 : 1]);
+        }
         ++et;
       }
     }
 
     // ------------------------------------------------------------ epilogue ---
     if (cnt > 0 && ok) {
-      ok = mbar_wait(&o_final[t], 0);
-      ok = __all_sync(0xffffffffu, ok);
+      ok = __all_sync(0xffffffffu, mbar_wait(&o_final[t], 0));
       if (!ok) misc[4] = 1;
       tc_fence_after();
     }
-    // row sum = both halves' partial sums
-    float* red_l = red_t;
-    named_bar_sync(bar_id, 256);
-    red_l[hf * kTileM + r] = l_part;
-    named_bar_sync(bar_id, 256);
-    const float l_sum = l_part + red_l[(hf ^ 1) * kTileM + r];
+    // A row that never saw a valid column keeps m_used = -inf: it is empty
+    // (O = 0, LSE = -inf) whatever the polynomial left in l_sum.
+    if (m_used == NEG_INF) l_sum = 0.f;
     const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
-    __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * p.N + (row_valid ? row : 0)) * D + hf * kOCols;
+    __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * p.N + (row_valid ? row : 0)) * D;
 #pragma unroll 1
-    for (int c = 0; c < kOCols / 32; ++c) {
+    for (int c = 0; c < D / 32; ++c) {
       float ov[32];
       if (cnt > 0 && ok) {
         tmem_ld32(o_addr + c * 32, ov);
@@ -527,45 +546,46 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
       }
     }
-    if (p.lse && row_valid && hf == 0) {
+    if (p.lse && row_valid) {
       const float neg_m = (m_used == NEG_INF) ? 0.f : -m_used * sl2;
       p.lse[static_cast<size_t>(bh) * p.N + row] =
           l_sum > 0.f ? (log2f(l_sum) - neg_m) * 0.69314718055994531f : NEG_INF;
     }
 
     // ----------------------------------- skip bits: cross-warp AND at the end ---
-    if (p.write_skip && cnt > 0 && ok && !misc[4]) {
-      const int tid = sw * 32 + lane - t * 256;   // 0..255 within the tile
-      // votes of the tile: [sub][half][words]
-      const uint32_t* tv = votes + t * 8 * L::kVoteWords;
-      for (int e = tid; e < n_list; e += 256) {
-        const uint32_t ent = list[e];
-        const uint32_t bits = (ent >> (16 + 4 * t)) & 0xFu;
-        if (!bits) continue;
-        const int jt = static_cast<int>(ent & 0xFFFFu);
-        const uint32_t word = e >> 5, bit = e & 31;
+    if (p.write_skip && cnt > 0) {
+      named_bar_sync(1 + t, 128);
+      if (ok && !misc[4]) {
+        const int tid = wq * 32 + lane;
+        uint32_t* tv = votes + t * 4 * L::kVoteWords;
+        for (int e = tid; e < n_list; e += 128) {
+          const uint32_t ent = list[e];
+          const uint32_t bits = (ent >> (16 + 4 * t)) & 0xFu;
+          if (!bits) continue;
+          const int jt = static_cast<int>(ent & 0xFFFFu);
 #pragma unroll
-        for (int qq = 0; qq < QH; ++qq) {
+          for (int qq = 0; qq < QH; ++qq) {
 #pragma unroll
-          for (int kh = 0; kh < KH; ++kh) {
-            if (BLK == 64 && !((bits >> (qq * 2 + kh)) & 1u)) continue;
-            const int qb = (qtile0 + t) * QH + qq;
-            const int kb = jt * KH + kh;
-            uint32_t all = 1u;
-            if (BLK == 128) {
+            for (int kh = 0; kh < KH; ++kh) {
+              if (BLK == 64 && !((bits >> (qq * 2 + kh)) & 1u)) continue;
+              const int qb = (qtile0 + t) * QH + qq;
+              const int kb = jt * KH + kh;
+              const int bi = (BLK == 128) ? e : e * 2 + kh;
+              uint32_t all = 1u;
+              if (BLK == 128) {
 #pragma unroll
-              for (int sb = 0; sb < 4; ++sb) all &= tv[(sb * 2 + 0) * L::kVoteWords + word] >> bit;
-            } else {
+                for (int w = 0; w < 4; ++w) all &= tv[w * L::kVoteWords + (bi >> 5)] >> (bi & 31);
+              } else {
 #pragma unroll
-              for (int sb = 2 * qq; sb < 2 * qq + 2; ++sb) all &= tv[(sb * 2 + kh) * L::kVoteWords + word] >> bit;
+                for (int w = 2 * qq; w < 2 * qq + 2; ++w) all &= tv[w * L::kVoteWords + (bi >> 5)] >> (bi & 31);
+              }
+              p.skip_out[(static_cast<size_t>(bh) * p.nb + qb) * p.nb + kb] = static_cast<uint8_t>(all & 1u);
             }
-            p.skip_out[(static_cast<size_t>(bh) * p.nb + qb) * p.nb + kb] = static_cast<uint8_t>(all & 1u);
           }
         }
       }
     }
   }
-
   tc_fence_before();
   __syncthreads();
 }

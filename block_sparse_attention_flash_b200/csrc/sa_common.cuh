@@ -52,14 +52,20 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
+// One potentially blocking test of the phase with the given parity.  The
+// suspend-time hint lets the waiting warp sleep (up to kSuspendHintNs) until
+// the phase completes instead of re-issuing, so waiting warps do not take
+// issue slots from the warps that share their SM sub-partition.
+constexpr uint32_t kSuspendHintNs = 100000;  // 100 us
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_addr(bar)), "r"(parity)
+      : "r"(smem_addr(bar)), "r"(parity), "r"(kSuspendHintNs)
       : "memory");
   return ok != 0;
 }
@@ -70,9 +76,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_timer_ns();
   while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 32; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait(bar, parity)) return true;
     if (global_timer_ns() - t0 > kWaitLimitNs) {
       record_error(SA_ERR_TIMEOUT);
       return false;
@@ -208,6 +212,29 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
 
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// 4 x (32 lanes x 32 columns) from TMEM into v[0..127], one wait for all four.
+__device__ __forceinline__ void tmem_ld128(uint32_t taddr, float* v) {
+  uint32_t* r = reinterpret_cast<uint32_t*>(v);
+#define SA_R8(b) "=r"(r[b]), "=r"(r[b + 1]), "=r"(r[b + 2]), "=r"(r[b + 3]), "=r"(r[b + 4]), "=r"(r[b + 5]), \
+                 "=r"(r[b + 6]), "=r"(r[b + 7])
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%128];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, "
+      "%45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%129];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%64, %65, %66, %67, %68, %69, %70, %71, %72, %73, %74, %75, %76, "
+      "%77, %78, %79, %80, %81, %82, %83, %84, %85, %86, %87, %88, %89, %90, %91, %92, %93, %94, %95}, [%130];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%96, %97, %98, %99, %100, %101, %102, %103, %104, %105, %106, "
+      "%107, %108, %109, %110, %111, %112, %113, %114, %115, %116, %117, %118, %119, %120, %121, %122, %123, %124, "
+      "%125, %126, %127}, [%131];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : SA_R8(0), SA_R8(8), SA_R8(16), SA_R8(24), SA_R8(32), SA_R8(40), SA_R8(48), SA_R8(56), SA_R8(64),
+        SA_R8(72), SA_R8(80), SA_R8(88), SA_R8(96), SA_R8(104), SA_R8(112), SA_R8(120)
+      : "r"(taddr), "r"(taddr + 32), "r"(taddr + 64), "r"(taddr + 96)
+      : "memory");
+#undef SA_R8
+}
+
 // 2 x (32 lanes x 32 columns) from TMEM into v[0..63], one wait for both.
 __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float* v) {
   uint32_t* r = reinterpret_cast<uint32_t*>(v);
@@ -271,6 +298,22 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   r.x = x.x <= -125.f ? 0.f : r.x;
   r.y = x.y <= -125.f ? 0.f : r.y;
   return r;
+}
+
+// Scalar 2^x on the FMA pipe, same split and polynomial as exp2_poly2 but
+// without the exact-zero guard: inputs at or below -125 (masked logits) give
+// a value below 2^-124 instead of 0.  Callers that can see a row made only of
+// masked logits must treat that row as empty themselves.
+__device__ __forceinline__ float exp2_poly(float x) {
+  constexpr float kRound = 12582912.0f;
+  x = fmaxf(x, -125.f);
+  const float j = x + kRound;
+  const float n = j - kRound;
+  const float f = x - n;
+  float q = fmaf(0.05517167f, f, 0.24261113f);
+  q = fmaf(q, f, 0.69326097f);
+  q = fmaf(q, f, 0.99992806f);
+  return __int_as_float(__float_as_int(q) + (__float_as_int(j) << 23));
 }
 
 // Per-warpgroup register budget changes (all four warps of a warpgroup

@@ -344,13 +344,13 @@ sa_status sa_pyramid_attn_fwd(const void* q, const void* k, const void* v, int B
   dim3 grid(n_pairs, BH);
   cudaStream_t s = as_stream(stream);
   if (d == 128 && block == 128)
-    sa::pyr_fwd_kernel<128, 128><<<grid, sa::kAttnThreads, sa::PyrSmem<128>::kAlloc, s>>>(tq, maps, p);
+    sa::pyr_fwd_kernel<128, 128><<<grid, sa::kPyrThreads, sa::PyrSmem<128>::kAlloc, s>>>(tq, maps, p);
   else if (d == 128 && block == 64)
-    sa::pyr_fwd_kernel<128, 64><<<grid, sa::kAttnThreads, sa::PyrSmem<128>::kAlloc, s>>>(tq, maps, p);
+    sa::pyr_fwd_kernel<128, 64><<<grid, sa::kPyrThreads, sa::PyrSmem<128>::kAlloc, s>>>(tq, maps, p);
   else if (d == 64 && block == 128)
-    sa::pyr_fwd_kernel<64, 128><<<grid, sa::kAttnThreads, sa::PyrSmem<64>::kAlloc, s>>>(tq, maps, p);
+    sa::pyr_fwd_kernel<64, 128><<<grid, sa::kPyrThreads, sa::PyrSmem<64>::kAlloc, s>>>(tq, maps, p);
   else
-    sa::pyr_fwd_kernel<64, 64><<<grid, sa::kAttnThreads, sa::PyrSmem<64>::kAlloc, s>>>(tq, maps, p);
+    sa::pyr_fwd_kernel<64, 64><<<grid, sa::kPyrThreads, sa::PyrSmem<64>::kAlloc, s>>>(tq, maps, p);
   return cuda_status(cudaGetLastError());
 }
 

@@ -15,7 +15,8 @@
 // the union of their (j, l) pairs; a segment carries a row mask (which of
 // the two q-blocks uses it) that becomes a -inf bias for the other rows.
 //
-// One CTA = two q-tiles (ping-pong as in sa_attn_fwd.cuh), but each q-tile has
+// One CTA = two q-tiles (ping-pong as in sa_attn_fwd.cuh), 16 softmax warps with
+// two threads per row (the halves swap row maxima once per key tile), but each q-tile has
 // its own packed key tiles; the entries of the two are interleaved.  K and V
 // segments arrive by TMA from one tensor map per pyramid level (level 0 is
 // the original K/V), into 2-stage rings released separately.  The producer
@@ -30,6 +31,9 @@
 namespace sa {
 
 constexpr int kPyrMaxBlocks = 1024;                 // k-blocks per sequence
+// 20 warps: producer, MMA, 2 idle, then 16 softmax warps (two threads per row)
+constexpr int kPyrWarps = 20;
+constexpr int kPyrThreads = kPyrWarps * 32;
 constexpr int kPyrMaxSegs = 2 * kPyrMaxBlocks;      // per q-tile (union of 2 q-blocks)
 
 struct PyrParams {
@@ -66,7 +70,7 @@ struct PyrMaps {
 };
 
 template <int D, int BLK>
-__global__ void __launch_bounds__(kAttnThreads, 1)
+__global__ void __launch_bounds__(kPyrThreads, 1)
     pyr_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ PyrMaps maps,
                    const PyrParams p) {
   using L = PyrSmem<D>;
