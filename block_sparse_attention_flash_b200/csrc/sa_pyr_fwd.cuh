@@ -15,9 +15,10 @@
 // the union of their (j, l) pairs; a segment carries a row mask (which of
 // the two q-blocks uses it) that becomes a -inf bias for the other rows.
 //
-// One CTA = two q-tiles (ping-pong as in sa_attn_fwd.cuh), 16 softmax warps with
-// two threads per row (the halves swap row maxima once per key tile), but each q-tile has
-// its own packed key tiles; the entries of the two are interleaved.  K and V
+// One CTA = two q-tiles with the same roles as sa_attn_fwd.cuh (one MMA issuer
+// per q-tile, one softmax thread per row, P handed over in two halves, the two
+// softmax warpgroups taking turns), but each q-tile has its own packed key
+// tiles; the entries of the two are interleaved.  K and V
 // segments arrive by TMA from one tensor map per pyramid level (level 0 is
 // the original K/V), into 2-stage rings released separately.  The producer
 // warp also writes, per stage, the per-column bias (log2 of the pooled token
@@ -31,8 +32,8 @@
 namespace sa {
 
 constexpr int kPyrMaxBlocks = 1024;                 // k-blocks per sequence
-// 20 warps: producer, MMA, 2 idle, then 16 softmax warps (two threads per row)
-constexpr int kPyrWarps = 20;
+// 12 warps: producer, two MMA issuers, one idle, two softmax warpgroups
+constexpr int kPyrWarps = 12;
 constexpr int kPyrThreads = kPyrWarps * 32;
 constexpr int kPyrMaxSegs = 2 * kPyrMaxBlocks;      // per q-tile (union of 2 q-blocks)
 
@@ -55,12 +56,12 @@ struct PyrSmem {
   static constexpr int kOffV = kOffK + kStages * kTileBytes;
   static constexpr int kOffSeg = kOffV + kStages * kTileBytes;         // [tile][kPyrMaxSegs] u32
   static constexpr int kOffBias = kOffSeg + 2 * kPyrMaxSegs * 4;       // [stage][half A/B][128] f32
-  static constexpr int kOffRed = kOffBias + kStages * 2 * kTileN * 4;
-  static constexpr int kRedFloats = 2 * 2 * 2 * kTileM;
-  static constexpr int kNumBars = 1 + 5 * kStages + 2 + 2 + 2 + 1;
-  static constexpr int kOffBar = kOffRed + kRedFloats * 4;
+  // q_full, k_full[2], v_full[2], k_empty[2], v_empty[2], b_full[2],
+  // s_ready[2], pa[2], pb[2], o_final[2], mma_done[2], go[2]
+  static constexpr int kNumBars = 1 + 5 * kStages + 2 * 6;
+  static constexpr int kOffBar = kOffBias + kStages * 2 * kTileN * 4;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr int kBytes = kOffMisc + 64;
+  static constexpr int kBytes = kOffMisc + 128;
   static constexpr int kAlloc = kBytes + 1024;
 };
 
@@ -83,7 +84,6 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint32_t* segs = reinterpret_cast<uint32_t*>(smem + L::kOffSeg);
   float* bias = reinterpret_cast<float*>(smem + L::kOffBias);
-  float* red = reinterpret_cast<float*>(smem + L::kOffRed);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;
@@ -92,11 +92,14 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
   uint64_t* v_empty = bars + 1 + 3 * kStages;
   uint64_t* b_full = bars + 1 + 4 * kStages;
   uint64_t* s_ready = bars + 1 + 5 * kStages;
-  uint64_t* p_ready = s_ready + 2;
-  uint64_t* o_final = p_ready + 2;
+  uint64_t* pa = s_ready + 2;
+  uint64_t* pb = pa + 2;
+  uint64_t* o_final = pb + 2;
   uint64_t* mma_done = o_final + 2;
+  uint64_t* go = mma_done + 2;
   volatile int* misc = reinterpret_cast<volatile int*>(smem + L::kOffMisc);
   // misc[0] TMEM base, [1]/[2] segments of q-tile 0/1, [3]/[4] key tiles of q-tile 0/1, [5] abort
+  volatile int* grp = misc + 8;   // producer scratch: owning lane of each 8-column group
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int pair = blockIdx.x, bh = blockIdx.y;
@@ -137,8 +140,14 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
     if (lane == 0) {
       misc[5] = 0;
       for (int i = 0; i < L::kNumBars; ++i) {
-        const bool softmax_arrivals = (&bars[i] == &p_ready[0]) || (&bars[i] == &p_ready[1]);
-        mbar_init(&bars[i], softmax_arrivals ? 256u : 1u);
+        uint32_t count = 1;
+        if (&bars[i] == &k_empty[0] || &bars[i] == &k_empty[1] || &bars[i] == &v_empty[0] ||
+            &bars[i] == &v_empty[1])
+          count = 2;  // one arrival from each q-tile's MMA issuer
+        if (&bars[i] == &pa[0] || &bars[i] == &pa[1] || &bars[i] == &pb[0] || &bars[i] == &pb[1] ||
+            &bars[i] == &go[0] || &bars[i] == &go[1])
+          count = 128;  // every softmax thread of the tile
+        mbar_init(&bars[i], count);
       }
       fence_mbar_init();
       tma_prefetch_desc(&tmQ);
@@ -165,12 +174,11 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
       k = m + (e - 2 * m);
     }
   };
-  const uint32_t sQ = smem_addr(smem + L::kOffQ);
   const uint32_t sK = smem_addr(smem + L::kOffK);
   const uint32_t sV = smem_addr(smem + L::kOffV);
 
   if (warp < kSoftmaxWarp0) {
-    setmaxnreg_dec<32>();
+    setmaxnreg_dec<56>();
   if (warp == 0) {
     // ------------------------------------------------------------ producer ---
     if (n_entries > 0) {
@@ -189,23 +197,34 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
       int cursor[2] = {0, 0};   // next segment of each q-tile
       int issued = 0;
       bool ok = true;
+      const float NEG_INF = -__int_as_float(0x7f800000);
       for (int e = 0; e < n_entries && ok; ++e) {
         int t, k;
         entry_of(e, t, k);
         const int s = e % kStages;
         const uint32_t par = ((e / kStages) - 1) & 1;
-        // segments of this key tile: [s0, s1)
+        // One lane per segment (a 128-key tile holds at most 128 / 8 = 16):
+        // a warp scan of the lengths gives each segment's column.
         const uint32_t* tseg = segs + t * kPyrMaxSegs;
         const int nseg = misc[1 + t];
-        const int s0 = cursor[t];
-        int s1 = s0, fill = 0;
-        while (s1 < nseg) {
-          const int len = BLK >> ((tseg[s1] >> 16) & 3u);
-          if (fill + len > kTileN) break;
-          fill += len;
-          ++s1;
+        const int gi = cursor[t] + lane;
+        const uint32_t sg = (lane < 16 && gi < nseg) ? tseg[gi] : 0u;
+        const int lvl = static_cast<int>((sg >> 16) & 3u);
+        const int len = (lane < 16 && gi < nseg) ? (BLK >> lvl) : 0;
+        int incl = len;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
         }
-        cursor[t] = s1;
+        const int col = incl - len;
+        const bool mine = len > 0 && incl <= kTileN;
+        const unsigned ball = __ballot_sync(0xffffffffu, mine);
+        const int nmine = __popc(ball);
+        const int fill = nmine > 0 ? __shfl_sync(0xffffffffu, incl, nmine - 1) : 0;
+        cursor[t] += nmine;
+        const int row = static_cast<int>(sg & 0xFFFFu) * len;
+
         if (e >= kStages) {
           bool w = lane == 0 ? (misc[5] == 0 && mbar_wait(&k_empty[s], par)) : true;
           if (!__shfl_sync(0xffffffffu, w, 0)) {
@@ -213,9 +232,9 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
             break;
           }
         }
-        // empty columns [fill, 128): zero K rows so masked products stay finite
         uint8_t* kst = smem + L::kOffK + s * L::kTileBytes;
         uint8_t* vst = smem + L::kOffV + s * L::kTileBytes;
+        // empty columns [fill, 128): zero K rows so masked products stay finite
         if (fill < kTileN) {
           for (int idx = lane; idx < (kTileN - fill) * 8 * (D / 64); idx += 32) {
             const int hd = idx / ((kTileN - fill) * 8);
@@ -223,21 +242,13 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
             reinterpret_cast<uint4*>(kst + hd * kHalfBytes + (fill + rem / 8) * 128)[rem % 8] = make_uint4(0, 0, 0, 0);
           }
           asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          __syncwarp();
         }
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&k_full[s], static_cast<uint32_t>(fill) * D * 2);
-          int col = 0;
-          for (int g = s0; g < s1; ++g) {
-            const uint32_t sg = tseg[g];
-            const int lvl = (sg >> 16) & 3u;
-            const int len = BLK >> lvl;
-            const int row = static_cast<int>(sg & 0xFFFFu) * len;
+        if (lane == 0) mbar_arrive_expect_tx(&k_full[s], static_cast<uint32_t>(fill) * D * 2);
+        __syncwarp();
+        if (mine) {
 #pragma unroll
-            for (int hd = 0; hd < D / 64; ++hd)
-              tma_load_3d(&maps.k[lvl], &k_full[s], kst + hd * kHalfBytes + col * 128, hd * 64, row, bh);
-            col += len;
-          }
+          for (int hd = 0; hd < D / 64; ++hd)
+            tma_load_3d(&maps.k[lvl], &k_full[s], kst + hd * kHalfBytes + col * 128, hd * 64, row, bh);
         }
         // V slot and the bias table of this stage are free once PV of entry e-2 is done
         if (e >= kStages) {
@@ -256,49 +267,46 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
           }
           asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         }
-        // per-column log2(count) bias for row halves A and B
+        // per-column log2(pooled token count) for row halves A and B: every
+        // lane takes columns lane, lane+32, ...; the owner of each 8-column
+        // group is looked up in grp[] and its fields fetched by shuffle
         float* bst = bias + s * 2 * kTileN;
-        {
-          const float NEG_INF = -__int_as_float(0x7f800000);
-          int col = 0;
-          for (int g = s0; g < s1; ++g) {
-            const uint32_t sg = tseg[g];
-            const int lvl = (sg >> 16) & 3u;
-            const int len = BLK >> lvl;
-            const uint32_t rm = (sg >> 18) & 3u;
-            const int g0 = static_cast<int>(sg & 0xFFFFu) * len;
-            for (int c = lane; c < len; c += 32) {
-              const int gr = g0 + c;
-              float bv = NEG_INF;
-              if (gr < p.pool_rows[lvl]) {
-                const int count = min(1 << lvl, p.N - (gr << lvl));
-                bv = log2f(static_cast<float>(count));
-              }
-              bst[col + c] = (rm & 1u) ? bv : NEG_INF;
-              bst[kTileN + col + c] = (QH == 1 ? (rm & 1u) : (rm & 2u)) ? bv : NEG_INF;
+        if (mine)
+          for (int g = col / 8; g < (col + len) / 8; ++g) grp[g] = lane;
+        __syncwarp();
+#pragma unroll
+        for (int cc = 0; cc < kTileN / 32; ++cc) {
+          const int c = cc * 32 + lane;
+          const int src = c < fill ? grp[c / 8] : 0;
+          const uint32_t sg_o = __shfl_sync(0xffffffffu, sg, src);
+          const int col_o = __shfl_sync(0xffffffffu, col, src);
+          const int row_o = __shfl_sync(0xffffffffu, row, src);
+          float bA = NEG_INF, bB = NEG_INF;
+          if (c < fill) {
+            const int lv = static_cast<int>((sg_o >> 16) & 3u);
+            const uint32_t rm = (sg_o >> 18) & 3u;
+            const int gr = row_o + (c - col_o);
+            float bv = NEG_INF;
+            if (gr < p.pool_rows[lv]) {
+              const int count = min(1 << lv, p.N - (gr << lv));
+              bv = count == (1 << lv) ? static_cast<float>(lv) : log2f(static_cast<float>(count));
             }
-            col += len;
+            bA = (rm & 1u) ? bv : NEG_INF;
+            bB = (QH == 1 ? (rm & 1u) : (rm & 2u)) ? bv : NEG_INF;
           }
-          for (int c = fill + lane; c < kTileN; c += 32) {
-            bst[c] = NEG_INF;
-            bst[kTileN + c] = NEG_INF;
-          }
+          bst[c] = bA;
+          bst[kTileN + c] = bB;
         }
         __syncwarp();
         if (lane == 0) {
           mbar_arrive(&b_full[s]);
           mbar_arrive_expect_tx(&v_full[s], static_cast<uint32_t>(fill) * D * 2);
-          int col = 0;
-          for (int g = s0; g < s1; ++g) {
-            const uint32_t sg = tseg[g];
-            const int lvl = (sg >> 16) & 3u;
-            const int len = BLK >> lvl;
-            const int row = static_cast<int>(sg & 0xFFFFu) * len;
+        }
+        __syncwarp();
+        if (mine) {
 #pragma unroll
-            for (int hd = 0; hd < D / 64; ++hd)
-              tma_load_3d(&maps.v[lvl], &v_full[s], vst + hd * kHalfBytes + col * 128, hd * 64, row, bh);
-            col += len;
-          }
+          for (int hd = 0; hd < D / 64; ++hd)
+            tma_load_3d(&maps.v[lvl], &v_full[s], vst + hd * kHalfBytes + col * 128, hd * 64, row, bh);
         }
         issued = e + 1;
       }
@@ -312,72 +320,78 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
         mbar_wait(q_full, 0);
       }
     }
-  } else if (warp == 1) {
-    // ----------------------------------------------------------- MMA issue ---
+  } else if (warp <= 2) {
+    // ---------------------------------------------- MMA issue, q-tile t ---
+    const int t = warp - 1;
     if (lane == 0 && n_entries > 0) {
+      const int cnt = ntile[t];
       bool ok = mbar_wait(q_full, 0);
-      int pend[2] = {-1, -1};
-      int done_pv[2] = {0, 0};
-      uint32_t pphase[2] = {0u, 0u};
-      auto issue_pv = [&](int t) -> bool {
-        const int e = pend[t];
-        const int s = e % kStages;
-        if (!mbar_wait(&p_ready[t], pphase[t])) return false;
-        pphase[t] ^= 1u;
-        if (!mbar_wait(&v_full[s], (e / kStages) & 1)) return false;
+      const uint64_t dq = smem_desc(smem_addr(smem + L::kOffQ + t * L::kTileBytes), 16, 1024);
+      const uint64_t dk0 = smem_desc(sK, 16, 1024);
+      const uint64_t dv0 = smem_desc(sV, kHalfBytes, 1024);
+      constexpr uint64_t kStageStep = L::kTileBytes >> 4;
+      const uint32_t s_tmem = tmem + t * 128;
+      const uint32_t o_tmem = tmem + 256 + t * D;
+      int pend = -1, done = 0;
+      uint32_t pph = 0;
+      auto issue_pv = [&]() -> bool {
+        const int ps = pend % kStages;
+        const uint64_t dv = dv0 + ps * kStageStep;
+        if (!mbar_wait(&pa[t], pph) || !mbar_wait(&v_full[ps], (pend / kStages) & 1)) return false;
         tc_fence_after();
-        const uint32_t d_tmem = tmem + 256 + t * D;
-        const uint32_t a_tmem = tmem + t * 128;
-        const uint32_t vbase = sV + s * L::kTileBytes;
 #pragma unroll
-        for (int kk = 0; kk < kTileN / 16; ++kk)
-          mma_ts(d_tmem, a_tmem + kk * 8, smem_desc(vbase + kk * 16 * 128, kHalfBytes, 1024), kIdescPV,
-                 (done_pv[t] == 0 && kk == 0) ? 0u : 1u);
-        mma_commit(&v_empty[s]);
-        if (++done_pv[t] == ntile[t]) mma_commit(&o_final[t]);
-        pend[t] = -1;
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ts(o_tmem, s_tmem + kk * 8, dv + ((kk * 16 * 128) >> 4), kIdescPV, (done == 0 && kk == 0) ? 0u : 1u);
+        if (!mbar_wait(&pb[t], pph)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 4; kk < 8; ++kk)
+          mma_ts(o_tmem, s_tmem + kk * 8, dv + ((kk * 16 * 128) >> 4), kIdescPV, 1u);
+        pph ^= 1u;
+        mma_commit(&v_empty[ps]);
+        if (++done == cnt) mma_commit(&o_final[t]);
+        pend = -1;
         return true;
       };
       for (int e = 0; ok && e < n_entries; ++e) {
-        int t, k;
-        entry_of(e, t, k);
+        int te, k;
+        entry_of(e, te, k);
         const int s = e % kStages;
-        // A PV two or more entries old holds the V slot (and bias table) of
-        // the stage the producer refills next: issue it now.  This matters
-        // once one q-tile has run out of key tiles and the other continues.
-        if (pend[t ^ 1] >= 0 && pend[t ^ 1] <= e - kStages && !issue_pv(t ^ 1)) {
+        const uint32_t par = (e / kStages) & 1;
+        if (pend >= 0 && !issue_pv()) {
           ok = false;
           break;
         }
-        // S_t(e) overwrites the TMEM columns P_t of the previous entry occupies
-        if (pend[t] >= 0 && !issue_pv(t)) {
+        // every entry's K must have landed before this tile reports the slot free
+        if (!mbar_wait(&k_full[s], par)) {
           ok = false;
           break;
         }
-        if (!mbar_wait(&k_full[s], (e / kStages) & 1)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t d_tmem = tmem + t * 128;
-        const uint32_t qbase = sQ + t * L::kTileBytes;
-        const uint32_t kbase = sK + s * L::kTileBytes;
+        if (te == t) {
+          tc_fence_after();
+          const uint64_t dk = dk0 + s * kStageStep;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-          mma_ss(d_tmem, smem_desc(qbase + off, 16, 1024), smem_desc(kbase + off, 16, 1024), kIdescS,
-                 kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t off = static_cast<uint64_t>((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+            mma_ss(s_tmem, dq + off, dk + off, kIdescS, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&s_ready[t]);
+          mma_commit(&k_empty[s]);
+          pend = e;
+        } else {
+          mma_commit(&k_empty[s]);
+          if (!mbar_wait(&v_full[s], par)) {
+            ok = false;
+            break;
+          }
+          mma_commit(&v_empty[s]);
         }
-        mma_commit(&s_ready[t]);
-        mma_commit(&k_empty[s]);
-        pend[t] = e;
         if (misc[5]) ok = false;
       }
-      for (int t = 0; ok && t < 2; ++t)
-        if (pend[t] >= 0 && !issue_pv(t)) ok = false;
+      if (ok && pend >= 0 && !issue_pv()) ok = false;
       if (!ok) misc[5] = 1;
-      mma_commit(mma_done);
-      mbar_wait(mma_done, 0);
+      mma_commit(&mma_done[t]);
+      mbar_wait(&mma_done[t], 0);
     }
   }
     tc_fence_before();
@@ -389,30 +403,24 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
     return;
   }
 
-  setmaxnreg_inc<112>();
+  setmaxnreg_inc<224>();
   {
     // ------------------------------------------------------------- softmax ---
-    const int sw = warp - kSoftmaxWarp0;
-    const int t = sw >> 3;
-    const int hf = (sw >> 2) & 1;
-    const int sub = warp & 3;
-    const int r = sub * 32 + lane;
+    const int t = (warp - kSoftmaxWarp0) >> 2;
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;
     const int row = (qtile0 + t) * kTileM + r;
     const bool row_valid = row < p.N;
     const int rh = (QH == 2) ? (r >> 6) : 0;   // which q-block of the tile (bias half)
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(sub * 32) << 16);
-    const uint32_t s_addr = lane_base + t * 128 + hf * 64;
-    const uint32_t p_addr = lane_base + t * 128 + hf * 32;
-    constexpr int kOCols = D / 2;
-    const uint32_t o_addr = lane_base + 256 + t * D + hf * kOCols;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    const uint32_t s_addr = lane_base + t * 128;
+    const uint32_t o_addr = lane_base + 256 + t * D;
     const int cnt = ntile[t];
     const float sl2 = p.scale_log2;
     const float NEG_INF = -__int_as_float(0x7f800000);
-    const int bar_id = 1 + t;
-    float* red_t = red + t * (2 * 2 * kTileM);
 
-    float m_used = NEG_INF, l_part = 0.f;
-    uint32_t sphase = 0;
+    float m_used = NEG_INF, l_sum = 0.f;
+    uint32_t sphase = 0, gphase = 0;
     int et = 0;
     bool ok = true;
     if (cnt > 0) {
@@ -421,57 +429,49 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
         entry_of(e, te, k);
         if (te != t) continue;
         const int st = e % kStages;
-        bool w_ok = mbar_wait(&s_ready[t], sphase);
-        w_ok = w_ok && mbar_wait(&b_full[st], (e / kStages) & 1);
-        w_ok = __all_sync(0xffffffffu, w_ok);
+        bool w_ok = true;
+        if (e > 0) {                       // wait for our turn
+          w_ok = mbar_wait(&go[t], gphase);
+          gphase ^= 1u;
+        }
+        w_ok = w_ok && mbar_wait(&s_ready[t], sphase) && mbar_wait(&b_full[st], (e / kStages) & 1);
+        ok = __all_sync(0xffffffffu, w_ok) && misc[5] == 0;
+        if (!ok) {
+          misc[5] = 1;
+          break;
+        }
         sphase ^= 1u;
         tc_fence_after();
-        float s[64];
-        if (w_ok) {
-          tmem_ld64(s_addr, s);
-        } else {
-#pragma unroll
-          for (int c = 0; c < 64; ++c) s[c] = 0.f;
-        }
+        float s[kTileN];
+        tmem_ld128(s_addr, s);
         // x = s * scale * log2e + log2(count), -inf on masked / empty columns
-        const float4* bsrc = reinterpret_cast<const float4*>(bias + st * 2 * kTileN + rh * kTileN + hf * 64);
+        const float4* bsrc = reinterpret_cast<const float4*>(bias + st * 2 * kTileN + rh * kTileN);
 #pragma unroll
-        for (int c4 = 0; c4 < 16; ++c4) {
+        for (int c4 = 0; c4 < 32; ++c4) {
           const float4 bv = bsrc[c4];
           s[4 * c4 + 0] = fmaf(s[4 * c4 + 0], sl2, bv.x);
           s[4 * c4 + 1] = fmaf(s[4 * c4 + 1], sl2, bv.y);
           s[4 * c4 + 2] = fmaf(s[4 * c4 + 2], sl2, bv.z);
           s[4 * c4 + 3] = fmaf(s[4 * c4 + 3], sl2, bv.w);
         }
-        float a0 = fmaxf(s[0], s[1]), a1 = fmaxf(s[2], s[3]);
-        float a2 = fmaxf(s[4], s[5]), a3 = fmaxf(s[6], s[7]);
+        float a[8];
 #pragma unroll
-        for (int c = 8; c < 64; c += 8) {
-          a0 = fmax3(a0, s[c + 0], s[c + 1]);
-          a1 = fmax3(a1, s[c + 2], s[c + 3]);
-          a2 = fmax3(a2, s[c + 4], s[c + 5]);
-          a3 = fmax3(a3, s[c + 6], s[c + 7]);
+        for (int u = 0; u < 8; ++u) a[u] = fmaxf(s[2 * u], s[2 * u + 1]);
+#pragma unroll
+        for (int c = 16; c < kTileN; c += 16) {
+#pragma unroll
+          for (int u = 0; u < 8; ++u) a[u] = fmax3(a[u], s[c + 2 * u], s[c + 2 * u + 1]);
         }
-        const float m_mine = fmax3(a0, a1, fmaxf(a2, a3));
-        float* red_p = red_t + (et & 1) * (2 * kTileM);
-        red_p[hf * kTileM + r] = m_mine;
-        tc_fence_before();
-        ok = named_bar_and(bar_id, 256, w_ok && misc[5] == 0);
-        tc_fence_after();
-        if (!ok) {
-          misc[5] = 1;
-          break;
-        }
-        const float mx = fmaxf(m_mine, red_p[(hf ^ 1) * kTileM + r]);
+        const float mx = fmaxf(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], fmax3(a[5], a[6], a[7])));
         float factor = 1.f;
         if (mx > m_used && (m_used == NEG_INF || mx - m_used > 8.f)) {
           factor = (m_used == NEG_INF) ? 0.f : fast_exp2(m_used - mx);
           m_used = mx;
-          l_part *= factor;
+          l_sum *= factor;
         }
         if (et > 0 && __any_sync(0xffffffffu, factor != 1.f)) {
 #pragma unroll 1
-          for (int c = 0; c < kOCols / 32; ++c) {
+          for (int c = 0; c < D / 32; ++c) {
             float ov[32];
             tmem_ld32(o_addr + c * 32, ov);
 #pragma unroll
@@ -481,50 +481,42 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
           tmem_st_wait();
         }
         const float neg_m = (m_used == NEG_INF) ? 0.f : -m_used;
-        const float2 nmv = make_float2(neg_m, neg_m);
-        float2 acc[4];
-#pragma unroll
-        for (int a = 0; a < 4; ++a) acc[a] = make_float2(0.f, 0.f);
-        uint32_t pk[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float2 x = add2(make_float2(s[2 * i], s[2 * i + 1]), nmv);
-          float2 pe;
-          if ((i & 15) >= kPolyPairFrom) {
-            pe = exp2_poly2(x);
-          } else {
-            pe.x = fast_exp2(x.x);
-            pe.y = fast_exp2(x.y);
-          }
-          acc[i & 3] = add2(acc[i & 3], pe);
-          pk[i] = pack_bf16x2(pe.x, pe.y);
+        {
+          uint32_t pk[32];
+          l_sum += exp_pack_64(s, 1.f, neg_m, pk);
+          tmem_st32(s_addr, reinterpret_cast<const float*>(pk));
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(&pa[t]);
         }
-        tmem_st32(p_addr, reinterpret_cast<const float*>(pk));
-        const float2 at = add2(add2(acc[0], acc[1]), add2(acc[2], acc[3]));
-        l_part += at.x + at.y;
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(&p_ready[t]);
+        {
+          uint32_t pk[32];
+          l_sum += exp_pack_64(s + 64, 1.f, neg_m, pk);
+          tmem_st32(s_addr + 32, reinterpret_cast<const float*>(pk));
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(&pb[t]);
+        }
+        if (e + 1 < n_entries) {           // pass the turn to the next entry's tile
+          int tn, kn;
+          entry_of(e + 1, tn, kn);
+          mbar_arrive(&go[tn]);
+        }
         ++et;
       }
     }
 
     // ------------------------------------------------------------ epilogue ---
     if (cnt > 0 && ok) {
-      ok = mbar_wait(&o_final[t], 0);
-      ok = __all_sync(0xffffffffu, ok);
+      ok = __all_sync(0xffffffffu, mbar_wait(&o_final[t], 0));
       if (!ok) misc[5] = 1;
       tc_fence_after();
     }
-    float* red_l = red_t;
-    named_bar_sync(bar_id, 256);
-    red_l[hf * kTileM + r] = l_part;
-    named_bar_sync(bar_id, 256);
-    const float l_sum = l_part + red_l[(hf ^ 1) * kTileM + r];
+    if (m_used == NEG_INF) l_sum = 0.f;
     const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
-    __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * p.N + (row_valid ? row : 0)) * D + hf * kOCols;
+    __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * p.N + (row_valid ? row : 0)) * D;
 #pragma unroll 1
-    for (int c = 0; c < kOCols / 32; ++c) {
+    for (int c = 0; c < D / 32; ++c) {
       float ov[32];
       if (cnt > 0 && ok) {
         tmem_ld32(o_addr + c * 32, ov);
@@ -545,11 +537,10 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
         }
       }
     }
-    if (p.lse && row_valid && hf == 0)
+    if (p.lse && row_valid)
       p.lse[static_cast<size_t>(bh) * p.N + row] =
           l_sum > 0.f ? (log2f(l_sum) + m_used) * 0.69314718055994531f : NEG_INF;
   }
-
   tc_fence_before();
   __syncthreads();
 }
