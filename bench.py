@@ -36,6 +36,11 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "sparse attn ms/call, executed TFLOP/s & % B200 BF16 tensor peak at 75.6K tok"
+# DRAM bytes (read + write) of one attention launch at 75,600 tokens x 40 heads,
+# from the ncu capture summarised in profiles/attn_fwd_wan14b_720p_lite.md
+# (4-head case, 300.5 MB, scaled by 40/4 heads).  Valid for the kernel version
+# that capture names; set to None whenever the kernel changes.
+ATTN_DRAM_BYTES_PER_LAUNCH = 3.0048e9
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -226,7 +231,9 @@ def run_ours(args, rank, world, local):
         "dense_equiv_tflops": round(dense / (statistics.median(kern_ms) * 1e-3) / 1e12, 2),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4), "peak_source": f"{src} bf16_tflops_sustained",
-                     "frac_of_burst": round(achieved / float(peaks["bf16_tflops"]), 4), "traffic": None},
+                     "frac_of_burst": round(achieved / float(peaks["bf16_tflops"]), 4),
+                     "traffic": ATTN_DRAM_BYTES_PER_LAUNCH, "traffic_unit": "bytes per launch",
+                     "algorithmic_bytes": 4 * B * H * N * d * 2},
         "gpu_launches": args.steps,
         "clocks": clk,
         "e2e": e2e,

@@ -4,6 +4,7 @@
     python -m block_sparse_attention_flash_b200.profile_case radial [--reps 2]
     python -m block_sparse_attention_flash_b200.profile_case mask   [--heads 12] [--reps 2]
     python -m block_sparse_attention_flash_b200.profile_case pool   [--heads 12] [--reps 2]
+    python -m block_sparse_attention_flash_b200.profile_case pyr    [--heads 2] [--reps 2]
 
 Each case uses a workload's real token grid with fewer heads, so one launch
 holds a few hundred MB (larger than L2) and a full profiler capture ends in
@@ -12,6 +13,7 @@ seconds.  Inputs are drawn on the device from the seeded generator.
   radial  118,800-token HunyuanVideo-like grid, block 128
   mask    32,760-token 480p grid, block 64, tau = 0.9
   pool    32,760-token 480p grid, block 64
+  pyr     32,760-token 480p grid, block 64, PSA levels from the GPU level builder
 """
 from __future__ import annotations
 
@@ -24,7 +26,7 @@ from . import build, inputs, ops
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["attn", "radial", "mask", "pool"])
+    ap.add_argument("case", choices=["attn", "radial", "mask", "pool", "pyr"])
     ap.add_argument("--heads", type=int, default=0)
     ap.add_argument("--reps", type=int, default=2)
     args = ap.parse_args()
@@ -47,11 +49,18 @@ def main():
         q, k, _ = inputs.rff_qkv(wl, H=args.heads or wl.H, device=dev)
         for _ in range(args.reps):
             ops.sa_build_mask(q, k, wl.block, "tau", tau=wl.tau)
-    else:
+    elif args.case == "pool":
         wl = inputs.WORKLOADS["psa_480p_pyramid"]
         _, k, v = inputs.rff_qkv(wl, H=args.heads or wl.H, device=dev)
         for _ in range(args.reps):
             ops.sa_pyramid_pool(k, v, wl.block)
+    else:
+        wl = inputs.WORKLOADS["psa_480p_pyramid"]
+        q, k, v = inputs.rff_qkv(wl, H=args.heads or 2, device=dev)
+        kp, vp = ops.sa_pyramid_pool(k, v, wl.block)
+        lv = ops.sa_build_mask(q, k, wl.block, "levels", level_frac=wl.level_frac)
+        for _ in range(args.reps):
+            ops.sa_pyramid_attn_fwd(q, k, v, wl.block, lv, kp, vp)
     ops.sa_get_device_status()
     print(f"profile case {args.case}: ok")
 
