@@ -6,30 +6,34 @@
 // ascending order.  Each kv tile is loaded once by TMA and feeds both q-tiles.
 //
 // Roles (384 threads = 12 warps, one CTA per SM):
-//   warp 0       builds the kv-tile list from the mask / skip bytes, then one
-//                lane issues the TMA loads (Q once, K and V through 2-stage
-//                rings released separately; skipped tiles are never loaded:
-//                LiteAttention write-up, sections 3 and 6);
-//   warp 1       owns TMEM (512 columns); its lane 0 issues the tcgen05.mma of
-//                q-tile 0, warp 2's lane 0 those of q-tile 1, so that a tile's
-//                P -> PV hand-off never waits behind the other tile's issue:
-//                S_t = Q_t K^T (both operands in shared memory) and
-//                O_t += P_t V (A operand P_t in TMEM, written over S_t);
+//   warp 0       builds the kv-tile list from the mask / skip bytes, loads Q
+//                and K by TMA (2-slot ring) and issues every S = Q_t K^T
+//                (tcgen05.mma, both operands in shared memory) into the one S
+//                buffer, which the two q-tiles use in turn (skipped tiles are
+//                never loaded: LiteAttention write-up, sections 3 and 6);
+//   warp 3       loads V by TMA (2-slot ring);
+//   warps 1, 2   issue O_t += P_t V for q-tile 0 / 1 (A operand P_t in TMEM,
+//                V in shared memory); warp 1 also owns TMEM (512 columns);
 //   warps 4-7    online softmax of q-tile 0, warps 8-11 of q-tile 1, one row
 //                per thread (a warp may only touch its own TMEM lane quarter).
-//                P goes back in two 64-column halves with one barrier each, so
-//                the first half of PV runs while the second half is computed.
-//                The two softmax warpgroups take turns (a token passed through
-//                the go barriers in list order), so that one tile's softmax
-//                runs while the tensor core works on the other tile instead of
-//                both competing for the same MUFU units.
-//                The skip condition is evaluated on the row maxima the softmax
-//                computes anyway (LiteAttention write-up, section 5), recorded
-//                per warp and reduced across warps at kernel end (section 6).
-// The producer/MMA warpgroup hands registers to the softmax warpgroups
-// (setmaxnreg); each role runs to its own final barrier.
+//                A softmax warpgroup hands the S buffer back as soon as its
+//                tcgen05.ld has landed, so the next S (of the other q-tile)
+//                is computed while it works; P goes to the tile's own P
+//                columns in two 64-column halves, each handed to the PV warp
+//                at once, so the first half of PV runs while the second half
+//                is computed.  The skip condition is evaluated on the row
+//                maxima the softmax computes anyway (LiteAttention write-up,
+//                section 5), recorded per warp and reduced across warps at
+//                kernel end (section 6).
+// Hand-offs between a softmax warpgroup and an issuing warp are named
+// barriers (a few tens of cycles), data arrival and MMA completion are
+// mbarriers.  All MMA issue is warp-wide with one elected lane, so the
+// operands stay in uniform registers.  The producer/MMA warpgroup hands
+// registers to the softmax warpgroups (setmaxnreg); each role runs to its own
+// final barrier.
 //
-// TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [384,384+D).
+// TMEM columns: S [0,128), P0 [128,192), P1 [192,256) (bf16 pairs),
+// O0 [256,256+D), O1 [256+D,256+2D).
 // Shared memory: Q0, Q1, K[2], V[2] tiles of 128 x D bf16 in the 128-byte
 // swizzled layout TMA writes (each 64-column half is a [128 x 128 B] slab),
 // the kv list, the per-warp skip votes and the mbarriers.
@@ -82,14 +86,26 @@ struct AttnSmem {
   static constexpr int kOffList = kOffV + kStages * kTileBytes;
   static constexpr int kVoteWords = kMaxKvTiles * 2 / 32;  // per softmax warp
   static constexpr int kOffVotes = kOffList + kMaxKvTiles * 4;
-  // q_full, k_full[2], v_full[2], k_empty[2], v_empty[2], s_ready[2],
-  // pa[2], pb[2], o_final[2], mma_done[2], go[2]
-  static constexpr int kNumBars = 1 + 4 * kStages + 2 * 6;
+  // q_full, k_full[2], v_full[2], v_empty[2], s_ready[2], pv_done_a[2],
+  // pv_done_b[2], o_final[2], mma_done[3]
+  static constexpr int kNumBars = 1 + 3 * kStages + 2 * 4 + 3;
   static constexpr int kOffBar = kOffVotes + 8 * kVoteWords * 4;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffMisc + 64;
   static constexpr int kAlloc = kBytes + 1024;
 };
+
+// Named barriers (id 0 is __syncthreads): per-warpgroup epilogue syncs, and
+// the hand-offs between softmax warpgroup t (128 threads) and an MMA-issuing
+// warp (32 threads).  Each id joins the same two parties every time, both
+// sides use bar.sync, and every party runs its full, list-determined
+// sequence of syncs (also after an error, skipping only its MMAs and loads),
+// so the syncs pair up in order and none can wait forever.
+constexpr int kBarEpi = 1;      // + t, 128 threads
+constexpr int kBarSFree = 3;    // + t: the S buffer loaded by softmax t <-> S issuer
+constexpr int kBarPA = 5;       // + t: first half of P_t written <-> PV issuer t
+constexpr int kBarPB = 7;       // + t: second half of P_t written <-> PV issuer t
+constexpr int kHandoff = 160;
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
@@ -155,14 +171,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;
   uint64_t* v_full = k_full + kStages;
-  uint64_t* k_empty = v_full + kStages;
-  uint64_t* v_empty = k_empty + kStages;
+  uint64_t* v_empty = v_full + kStages;
   uint64_t* s_ready = v_empty + kStages;
-  uint64_t* pa = s_ready + 2;
-  uint64_t* pb = pa + 2;
-  uint64_t* o_final = pb + 2;
-  uint64_t* mma_done = o_final + 2;
-  uint64_t* go = mma_done + 2;
+  uint64_t* pv_done_a = s_ready + 2;
+  uint64_t* pv_done_b = pv_done_a + 2;
+  uint64_t* o_final = pv_done_b + 2;
+  uint64_t* mma_done = o_final + 2;   // one per MMA-issuing warp
   volatile int* misc = reinterpret_cast<volatile int*>(smem + L::kOffMisc);
   // misc[0] TMEM base, [1] list length, [2] / [3] kv tiles of q-tile 0 / 1, [4] abort flag
 
@@ -214,13 +228,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       misc[3] = c1;
       misc[4] = 0;
       for (int i = 0; i < L::kNumBars; ++i) {
-        uint32_t count = 1;
-        if (&bars[i] == &k_empty[0] || &bars[i] == &k_empty[1] || &bars[i] == &v_empty[0] ||
-            &bars[i] == &v_empty[1])
-          count = 2;  // one arrival from each q-tile's MMA issuer
-        if (&bars[i] == &pa[0] || &bars[i] == &pa[1] || &bars[i] == &pb[0] || &bars[i] == &pb[1] ||
-            &bars[i] == &go[0] || &bars[i] == &go[1])
-          count = 128;  // every softmax thread of the tile
+        // v_empty: one arrival per q-tile per entry (its PV commit; the
+        // commit is doubled when the other q-tile skips the entry)
+        const uint32_t count = (&bars[i] == &v_empty[0] || &bars[i] == &v_empty[1]) ? 2u : 1u;
         mbar_init(&bars[i], count);
       }
       fence_mbar_init();
@@ -241,125 +251,160 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   if (warp < kSoftmaxWarp0) {
     setmaxnreg_dec<56>();
+    auto active = [&](int e, int t) -> bool { return ((list[e] >> (16 + 4 * t)) & 0xFu) != 0; };
+    auto aborted = [&]() -> bool { return __any_sync(0xffffffffu, misc[4] != 0); };
     if (warp == 0) {
-      // ---------------------------------------------------------- producer ---
-      if (lane == 0 && n_list > 0) {
+      // ------------------------------------------- K loads and S issue (warp 0) ---
+      // S number i (the (entry, q-tile) pairs in list order) goes into the one
+      // S buffer once the softmax that consumed S number i-1 has loaded it.
+      // At that point every earlier S has completed, so the K slot of an entry
+      // whose last S was i-1 is free and K of the entry two ahead goes into it.
+      if (n_list > 0) {
         const int cnt0 = misc[2], cnt1 = misc[3];
-        const uint32_t qbytes = static_cast<uint32_t>((cnt0 > 0) + (cnt1 > 0)) * L::kTileBytes;
-        mbar_arrive_expect_tx(q_full, qbytes);
+        const int n_s = cnt0 + cnt1;
+        if (lane == 0) {
+          const uint32_t qbytes = static_cast<uint32_t>((cnt0 > 0) + (cnt1 > 0)) * L::kTileBytes;
+          mbar_arrive_expect_tx(q_full, qbytes);
 #pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          if ((t == 0 ? cnt0 : cnt1) == 0) continue;
+          for (int t = 0; t < 2; ++t) {
+            if ((t == 0 ? cnt0 : cnt1) == 0) continue;
 #pragma unroll
-          for (int hd = 0; hd < D / 64; ++hd)
-            tma_load_3d(&tmQ, q_full, smem + L::kOffQ + t * L::kTileBytes + hd * kHalfBytes, hd * 64,
-                        (qtile0 + t) * kTileM, bh);
+            for (int hd = 0; hd < D / 64; ++hd)
+              tma_load_3d(&tmQ, q_full, smem + L::kOffQ + t * L::kTileBytes + hd * kHalfBytes, hd * 64,
+                          (qtile0 + t) * kTileM, bh);
+          }
         }
+        auto load_k = [&](int e) {
+          if (lane == 0) {
+            const int s = e % kStages;
+            mbar_arrive_expect_tx(&k_full[s], L::kTileBytes);
+#pragma unroll
+            for (int hd = 0; hd < D / 64; ++hd)
+              tma_load_3d(&tmK, &k_full[s], smem + L::kOffK + s * L::kTileBytes + hd * kHalfBytes, hd * 64,
+                          static_cast<int>(list[e] & 0xFFFFu) * kTileN, bh);
+          }
+        };
+        int k_issued = n_list < kStages ? n_list : kStages;   // K loads issued
+        int k_seen = 0;                                        // K loads observed landed
+        for (int e = 0; e < k_issued; ++e) load_k(e);
+        bool ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0));
+        if (!ok && lane == 0) misc[4] = 1;
+        const uint64_t dq0 = smem_desc(smem_addr(smem + L::kOffQ), 16, 1024);
+        const uint64_t dk0 = smem_desc(smem_addr(smem + L::kOffK), 16, 1024);
+        constexpr uint64_t kStageStep = L::kTileBytes >> 4;   // descriptor units
+        int se = 0, st = active(0, 0) ? 0 : 1;
+        int prev_e = 0, prev_t = 0;
+        bool prev_last = false;
+        for (int i = 0; i < n_s; ++i) {
+          if (i > 0) {
+            named_bar_sync(kBarSFree + prev_t, kHandoff);
+            if (prev_last && prev_e + kStages < n_list && !aborted()) {
+              load_k(prev_e + kStages);
+              k_issued = prev_e + kStages + 1;
+            }
+          }
+          ok = ok && !aborted();
+          if (ok && se >= k_seen) {
+            ok = __all_sync(0xffffffffu, mbar_wait(&k_full[se % kStages], (se / kStages) & 1));
+            if (ok) k_seen = se + 1;
+            else if (lane == 0) misc[4] = 1;
+          }
+          if (ok) {
+            tc_fence_after();
+            const uint64_t dq = dq0 + st * kStageStep;
+            const uint64_t dk = dk0 + (se % kStages) * kStageStep;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint64_t off = static_cast<uint64_t>((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+              mma_ss_warp(tmem, dq + off, dk + off, kIdescS, kk > 0 ? 1u : 0u);
+            }
+          }
+          // committed also after an error (with nothing issued), so that the
+          // softmax keeps its place in the sequence of hand-offs
+          mma_commit_warp(&s_ready[st]);
+          prev_e = se;
+          prev_t = st;
+          prev_last = st == 1 || !active(se, 1);
+          if (prev_last) {
+            ++se;
+            st = (se < n_list && active(se, 0)) ? 0 : 1;
+          } else {
+            st = 1;
+          }
+        }
+        named_bar_sync(kBarSFree + prev_t, kHandoff);   // the softmax has loaded the last S
+        // K loads never observed (error path) must land before the CTA exits
+        for (int e = k_seen; e < k_issued; ++e) mbar_wait(&k_full[e % kStages], (e / kStages) & 1);
+        mma_commit_warp(&mma_done[0]);
+        mbar_wait(&mma_done[0], 0);
+      }
+    } else if (warp == 3) {
+      // ------------------------------------------------------- V loads (warp 3) ---
+      if (lane == 0 && n_list > 0) {
         int issued = 0;
         for (int e = 0; e < n_list; ++e) {
           const int s = e % kStages;
-          const uint32_t par = ((e / kStages) - 1) & 1;
-          if (e >= kStages && (misc[4] || !mbar_wait(&k_empty[s], par))) {
+          if (e >= kStages && (misc[4] || !mbar_wait(&v_empty[s], ((e / kStages) - 1) & 1))) {
             misc[4] = 1;
-            break;
-          }
-          const int row = static_cast<int>(list[e] & 0xFFFFu) * kTileN;
-          mbar_arrive_expect_tx(&k_full[s], L::kTileBytes);
-#pragma unroll
-          for (int hd = 0; hd < D / 64; ++hd)
-            tma_load_3d(&tmK, &k_full[s], smem + L::kOffK + s * L::kTileBytes + hd * kHalfBytes, hd * 64, row, bh);
-          if (e >= kStages && !mbar_wait(&v_empty[s], par)) {
-            misc[4] = 1;
-            issued = e;
-            mbar_wait(&k_full[s], (e / kStages) & 1);
             break;
           }
           mbar_arrive_expect_tx(&v_full[s], L::kTileBytes);
 #pragma unroll
           for (int hd = 0; hd < D / 64; ++hd)
-            tma_load_3d(&tmV, &v_full[s], smem + L::kOffV + s * L::kTileBytes + hd * kHalfBytes, hd * 64, row, bh);
+            tma_load_3d(&tmV, &v_full[s], smem + L::kOffV + s * L::kTileBytes + hd * kHalfBytes, hd * 64,
+                        static_cast<int>(list[e] & 0xFFFFu) * kTileN, bh);
           issued = e + 1;
         }
         // Loads still in flight must land before the CTA can exit.
-        for (int e = (issued > kStages ? issued - kStages : 0); e < issued; ++e) {
-          const int s = e % kStages;
-          mbar_wait(&k_full[s], (e / kStages) & 1);
-          mbar_wait(&v_full[s], (e / kStages) & 1);
-        }
-        if ((cnt0 | cnt1) != 0) mbar_wait(q_full, 0);
+        for (int e = (issued > kStages ? issued - kStages : 0); e < issued; ++e)
+          mbar_wait(&v_full[e % kStages], (e / kStages) & 1);
       }
-    } else if (warp <= 2) {
-      // ---------------------------------------------- MMA issue, q-tile t ---
+    } else {
+      // ------------------------------------ PV issue for q-tile t (warps 1, 2) ---
+      // O_t += P_t V, in two halves, each as soon as the softmax warpgroup has
+      // written that half of P_t (A operand from TMEM, V from shared memory).
       const int t = warp - 1;
-      if (lane == 0 && n_list > 0) {
-        const int cnt = misc[2 + t];
-        bool ok = mbar_wait(q_full, 0);
-        const uint64_t dq = smem_desc(smem_addr(smem + L::kOffQ + t * L::kTileBytes), 16, 1024);
-        const uint64_t dk0 = smem_desc(smem_addr(smem + L::kOffK), 16, 1024);
+      const int cnt = misc[2 + t];
+      if (n_list > 0 && cnt > 0) {
         const uint64_t dv0 = smem_desc(smem_addr(smem + L::kOffV), kHalfBytes, 1024);
-        constexpr uint64_t kStageStep = L::kTileBytes >> 4;   // descriptor units
-        const uint32_t s_tmem = tmem + t * 128;
+        constexpr uint64_t kStageStep = L::kTileBytes >> 4;
+        const uint32_t a_tmem = tmem + 128 + 64 * t;
         const uint32_t o_tmem = tmem + 256 + t * D;
-        int pend = -1, done = 0;
-        uint32_t pph = 0;
-        // O_t += P_t V of entry `pend`: first half as soon as it is ready
-        auto issue_pv = [&]() -> bool {
-          const int ps = pend % kStages;
-          const uint64_t dv = dv0 + ps * kStageStep;
-          if (!mbar_wait(&pa[t], pph) || !mbar_wait(&v_full[ps], (pend / kStages) & 1)) return false;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_ts(o_tmem, s_tmem + kk * 8, dv + ((kk * 16 * 128) >> 4), kIdescPV, (done == 0 && kk == 0) ? 0u : 1u);
-          if (!mbar_wait(&pb[t], pph)) return false;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 4; kk < 8; ++kk)
-            mma_ts(o_tmem, s_tmem + kk * 8, dv + ((kk * 16 * 128) >> 4), kIdescPV, 1u);
-          pph ^= 1u;
-          mma_commit(&v_empty[ps]);
-          if (++done == cnt) mma_commit(&o_final[t]);
-          pend = -1;
-          return true;
-        };
-        for (int e = 0; ok && e < n_list; ++e) {
+        int k = 0;
+        for (int e = 0; e < n_list; ++e) {
+          if (!active(e, t)) continue;
           const int s = e % kStages;
-          const uint32_t par = (e / kStages) & 1;
-          if (pend >= 0 && !issue_pv()) {
-            ok = false;
-            break;
+          const uint64_t dv = dv0 + s * kStageStep;
+          named_bar_sync(kBarPA + t, kHandoff);
+          bool ok = !aborted();
+          if (ok) {
+            ok = __all_sync(0xffffffffu, mbar_wait(&v_full[s], (e / kStages) & 1));
+            if (!ok && lane == 0) misc[4] = 1;
           }
-          // every entry's K must have landed before this tile reports the slot
-          // free, so the two arrivals on k_empty / v_empty stay in one phase
-          if (!mbar_wait(&k_full[s], par)) {
-            ok = false;
-            break;
-          }
-          if ((list[e] >> (16 + 4 * t)) & 0xFu) {
+          if (ok) {
             tc_fence_after();
-            const uint64_t dk = dk0 + s * kStageStep;
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint64_t off = static_cast<uint64_t>((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
-              mma_ss(s_tmem, dq + off, dk + off, kIdescS, kk > 0 ? 1u : 0u);
-            }
-            mma_commit(&s_ready[t]);
-            mma_commit(&k_empty[s]);
-            pend = e;
-          } else {
-            mma_commit(&k_empty[s]);
-            if (!mbar_wait(&v_full[s], par)) {
-              ok = false;
-              break;
-            }
-            mma_commit(&v_empty[s]);
+            for (int kk = 0; kk < 4; ++kk)
+              mma_ts_warp(o_tmem, a_tmem + kk * 8, dv + ((kk * 16 * 128) >> 4), kIdescPV,
+                          (k == 0 && kk == 0) ? 0u : 1u);
           }
-          if (misc[4]) ok = false;
+          mma_commit_warp(&pv_done_a[t]);   // also after an error, so that no waiter stalls
+          named_bar_sync(kBarPB + t, kHandoff);
+          if (ok && !aborted()) {
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 4; kk < 8; ++kk)
+              mma_ts_warp(o_tmem, a_tmem + kk * 8, dv + ((kk * 16 * 128) >> 4), kIdescPV, 1u);
+          }
+          // committed also after an error, so that no waiter stalls
+          mma_commit_warp(&pv_done_b[t]);
+          mma_commit_warp(&v_empty[s]);
+          if (!active(e, 1 - t)) mma_commit_warp(&v_empty[s]);   // the other tile's share
+          if (k + 1 == cnt) mma_commit_warp(&o_final[t]);
+          ++k;
         }
-        if (ok && pend >= 0 && !issue_pv()) ok = false;
-        if (!ok) misc[4] = 1;
-        mma_commit(&mma_done[t]);
-        mbar_wait(&mma_done[t], 0);
+        mma_commit_warp(&mma_done[1 + t]);
+        mbar_wait(&mma_done[1 + t], 0);
       }
     }
     tc_fence_before();
@@ -381,15 +426,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const bool row_valid = row < p.N;
     const int qh = (BLK == 64) ? (r >> 6) : 0;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-    const uint32_t s_addr = lane_base + t * 128;
+    const uint32_t s_addr = lane_base;
+    const uint32_t p_addr = lane_base + 128 + 64 * t;
     const uint32_t o_addr = lane_base + 256 + t * D;
     const int cnt = misc[2 + t];
     const float sl2 = p.scale_log2;
     const float NEG_INF = -__int_as_float(0x7f800000);
 
     float m_used = NEG_INF, m_true = NEG_INF, l_sum = 0.f;
-    uint32_t sphase = 0, gphase = 0;
-    int et = 0;
+    int et = 0;   // kv tiles this q-tile has processed
     bool ok = true;
     uint32_t* my_votes = votes + (t * 4 + wq) * L::kVoteWords;
 
@@ -399,23 +444,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const uint32_t bits = (ent >> (16 + 4 * t)) & 0xFu;
         if (!bits) continue;
         const int jt = static_cast<int>(ent & 0xFFFFu);
-        // wait for our turn unless this is the first (entry, tile) phase
-        const bool has_prior = e > 0 || (t == 1 && ((ent >> 16) & 0xFu) != 0);
-        bool w_ok = true;
-        if (has_prior) {
-          w_ok = mbar_wait(&go[t], gphase);
-          gphase ^= 1u;
-        }
-        ok = __all_sync(0xffffffffu, w_ok && mbar_wait(&s_ready[t], sphase)) && misc[4] == 0;
-        if (!ok) {
+        // After an error the loop still runs to the end (its hand-offs keep
+        // the issuing warps' sequences in step); it only stops trusting TMEM.
+        if (!mbar_wait(&s_ready[t], et & 1)) {
           misc[4] = 1;
-          break;
+          ok = false;
         }
-        sphase ^= 1u;
         tc_fence_after();
 
         float s[kTileN];
         tmem_ld128(s_addr, s);
+        // the S buffer is free for the next S (of either q-tile)
+        tc_fence_before();
+        named_bar_sync(kBarSFree + t, kHandoff);
 
         const int valid_cols = min(kTileN, p.N - jt * kTileN);
         if (valid_cols < kTileN || (BLK == 64 && bits != 0xFu)) {
@@ -474,7 +515,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           m_used = mx;
           l_sum *= factor;
         }
-        if (et > 0 && __any_sync(0xffffffffu, factor != 1.f)) {
+        // The previous PV of this tile reads P_t and accumulates into O_t: each
+        // half of P_t is rewritten once that half of the PV has completed, and
+        // O_t is rescaled once all of it has.
+        auto wait_pv = [&](uint64_t* bar) {
+          if (et > 0) {
+            if (!mbar_wait(bar, (et - 1) & 1)) {
+              misc[4] = 1;
+              ok = false;
+            }
+            tc_fence_after();
+          }
+        };
+        const bool rescale = et > 0 && __any_sync(0xffffffffu, factor != 1.f);
+        if (rescale) {
+          wait_pv(&pv_done_b[t]);
 #pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
             float ov[32];
@@ -490,30 +545,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         {
           uint32_t pk[32];
           l_sum += exp_pack_64(s, sl2, neg_m, pk);
-          tmem_st32(s_addr, reinterpret_cast<const float*>(pk));
+          if (!rescale) wait_pv(&pv_done_a[t]);
+          tmem_st32(p_addr, reinterpret_cast<const float*>(pk));
           tmem_st_wait();
           tc_fence_before();
-          mbar_arrive(&pa[t]);
+          named_bar_sync(kBarPA + t, kHandoff);
         }
         {
           uint32_t pk[32];
           l_sum += exp_pack_64(s + 64, sl2, neg_m, pk);
-          tmem_st32(s_addr + 32, reinterpret_cast<const float*>(pk));
+          if (!rescale) wait_pv(&pv_done_b[t]);
+          tmem_st32(p_addr + 32, reinterpret_cast<const float*>(pk));
           tmem_st_wait();
           tc_fence_before();
-          mbar_arrive(&pb[t]);
-        }
-        // pass the turn to the owner of the next (entry, tile) phase
-        if (t == 0 && ((ent >> 20) & 0xFu) != 0) {
-          mbar_arrive(&go[1]);
-        } else if (e + 1 < n_list) {
-          mbar_arrive(&go[((list[e + 1] >> 16) & 0xFu) != 0 ? 0 : 1]);
+          named_bar_sync(kBarPB + t, kHandoff);
         }
         ++et;
       }
     }
 
     // ------------------------------------------------------------ epilogue ---
+    ok = __all_sync(0xffffffffu, ok && misc[4] == 0);
     if (cnt > 0 && ok) {
       ok = __all_sync(0xffffffffu, mbar_wait(&o_final[t], 0));
       if (!ok) misc[4] = 1;
@@ -554,7 +606,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
     // ----------------------------------- skip bits: cross-warp AND at the end ---
     if (p.write_skip && cnt > 0) {
-      named_bar_sync(1 + t, 128);
+      named_bar_sync(kBarEpi + t, 128);
       if (ok && !misc[4]) {
         const int tid = wq * 32 + lane;
         uint32_t* tv = votes + t * 4 * L::kVoteWords;
