@@ -296,13 +296,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         int prev_e = 0, prev_t = 0;
         bool prev_last = false;
         for (int i = 0; i < n_s; ++i) {
-          if (i > 0) {
-            named_bar_sync(kBarSFree + prev_t, kHandoff);
-            if (prev_last && prev_e + kStages < n_list && !aborted()) {
-              load_k(prev_e + kStages);
-              k_issued = prev_e + kStages + 1;
-            }
-          }
+          if (i > 0) named_bar_sync(kBarSFree + prev_t, kHandoff);
           ok = ok && !aborted();
           if (ok && se >= k_seen) {
             ok = __all_sync(0xffffffffu, mbar_wait(&k_full[se % kStages], (se / kStages) & 1));
@@ -322,6 +316,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           // committed also after an error (with nothing issued), so that the
           // softmax keeps its place in the sequence of hand-offs
           mma_commit_warp(&s_ready[st]);
+          // The next K load is issued only now: issuing a TMA load can hold
+          // the issuing warp for hundreds of cycles, and S(i) is on the path.
+          if (i > 0 && prev_last && prev_e + kStages < n_list && !aborted()) {
+            load_k(prev_e + kStages);
+            k_issued = prev_e + kStages + 1;
+          }
           prev_e = se;
           prev_t = st;
           prev_last = st == 1 || !active(se, 1);
