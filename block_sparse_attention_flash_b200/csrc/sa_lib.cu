@@ -323,10 +323,10 @@ sa_status sa_pyramid_attn_fwd(const void* q, const void* k, const void* v, int B
     const int rows = ceil_div(N, 1 << l);
     const void* kb = l == 0 ? k : k_pool[l - 1];
     const void* vb = l == 0 ? v : v_pool[l - 1];
-    if (!encode_rows_map(&maps.k[l], kb, BH, rows, d, block >> l) ||
-        !encode_rows_map(&maps.v[l], vb, BH, rows, d, block >> l))
+    // boxes of at most 64 rows: the kernel fills and releases V by 64-key half
+    const int box = std::min(block >> l, 64);
+    if (!encode_rows_map(&maps.k[l], kb, BH, rows, d, box) || !encode_rows_map(&maps.v[l], vb, BH, rows, d, box))
       return SA_ERR_CUDA;
-    p.pool_rows[l] = rows;
   }
   if (scale == 0.f) scale = 1.0f / std::sqrt(static_cast<float>(d));
   p.B = B;

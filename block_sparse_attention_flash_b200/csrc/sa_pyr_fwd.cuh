@@ -15,16 +15,18 @@
 // the union of their (j, l) pairs; a segment carries a row mask (which of
 // the two q-blocks uses it) that becomes a -inf bias for the other rows.
 //
-// One CTA = two q-tiles with the same roles as sa_attn_fwd.cuh (one MMA issuer
-// per q-tile, one softmax thread per row, P handed over in two halves, the two
-// softmax warpgroups taking turns), but each q-tile has its own packed key
-// tiles; the entries of the two are interleaved.  K and V
-// segments arrive by TMA from one tensor map per pyramid level (level 0 is
-// the original K/V), into 2-stage rings released separately.  The producer
-// warp also writes, per stage, the per-column bias (log2 of the pooled token
-// count, -inf where a column is masked or empty) for both row halves, and
-// zero-fills columns no segment covers so that masked products stay finite.
-// The softmax works in log2 units: x = s * scale * log2(e) + log2(count).
+// One CTA = two q-tiles with the same roles and TMEM layout as
+// sa_attn_fwd.cuh (warp 0 issues every S into the one S buffer, warps 1 and 2
+// issue the PV of q-tile 0 / 1, one softmax thread per row, P handed over in
+// two halves through named barriers), but each q-tile has its own packed key
+// tiles; the entries of the two are interleaved and each entry feeds one
+// q-tile.  Warp 3 is the producer: K and V segments arrive by TMA from one
+// tensor map per pyramid level (level 0 is the original K/V) into 2-slot
+// rings, and the producer also writes, per slot, the per-column bias (log2 of
+// the pooled token count, -inf where a column is masked or empty) for both
+// row halves, and zero-fills columns no segment covers so that masked
+// products stay finite.  The softmax works in log2 units:
+// x = s * scale * log2(e) + log2(count).
 #pragma once
 
 #include "sa_attn_fwd.cuh"
@@ -32,7 +34,7 @@
 namespace sa {
 
 constexpr int kPyrMaxBlocks = 1024;                 // k-blocks per sequence
-// 12 warps: producer, two MMA issuers, one idle, two softmax warpgroups
+// 12 warps: S issuer, two PV issuers, producer, two softmax warpgroups
 constexpr int kPyrWarps = 12;
 constexpr int kPyrThreads = kPyrWarps * 32;
 constexpr int kPyrMaxSegs = 2 * kPyrMaxBlocks;      // per q-tile (union of 2 q-blocks)
@@ -40,7 +42,6 @@ constexpr int kPyrMaxSegs = 2 * kPyrMaxBlocks;      // per q-tile (union of 2 q-
 struct PyrParams {
   int B, H, N;
   int nb;                 // blocks per sequence
-  int pool_rows[4];       // rows of the level-l tensor: ceil(N / 2^l)
   const uint8_t* levels;  // code map: 0 drop, 1 + l level l
   long long lsb, lsh, lsi;
   float scale_log2;
@@ -56,9 +57,11 @@ struct PyrSmem {
   static constexpr int kOffV = kOffK + kStages * kTileBytes;
   static constexpr int kOffSeg = kOffV + kStages * kTileBytes;         // [tile][kPyrMaxSegs] u32
   static constexpr int kOffBias = kOffSeg + 2 * kPyrMaxSegs * 4;       // [stage][half A/B][128] f32
-  // q_full, k_full[2], v_full[2], k_empty[2], v_empty[2], b_full[2],
-  // s_ready[2], pa[2], pb[2], o_final[2], mma_done[2], go[2]
-  static constexpr int kNumBars = 1 + 5 * kStages + 2 * 6;
+  // q_full, k_full[2], v_full[2][2], k_empty[2], v_empty[2][2], b_full[2],
+  // b_empty[2], s_ready[2], pv_done_a[2], pv_done_b[2], o_final[2], mma_done[3]
+  // (V slots are filled and released by 64-key half: rows [0,64) feed the
+  // first half of PV, rows [64,128) the second)
+  static constexpr int kNumBars = 1 + 8 * kStages + 2 * 4 + 3;
   static constexpr int kOffBar = kOffBias + kStages * 2 * kTileN * 4;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffMisc + 128;
@@ -87,19 +90,18 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;
-  uint64_t* v_full = bars + 1 + kStages;
-  uint64_t* k_empty = bars + 1 + 2 * kStages;
-  uint64_t* v_empty = bars + 1 + 3 * kStages;
-  uint64_t* b_full = bars + 1 + 4 * kStages;
-  uint64_t* s_ready = bars + 1 + 5 * kStages;
-  uint64_t* pa = s_ready + 2;
-  uint64_t* pb = pa + 2;
-  uint64_t* o_final = pb + 2;
-  uint64_t* mma_done = o_final + 2;
-  uint64_t* go = mma_done + 2;
+  uint64_t* v_full = bars + 1 + kStages;          // [slot * 2 + half]
+  uint64_t* k_empty = bars + 1 + 3 * kStages;
+  uint64_t* v_empty = bars + 1 + 4 * kStages;     // [slot * 2 + half]
+  uint64_t* b_full = bars + 1 + 6 * kStages;
+  uint64_t* b_empty = bars + 1 + 7 * kStages;
+  uint64_t* s_ready = bars + 1 + 8 * kStages;
+  uint64_t* pv_done_a = s_ready + 2;
+  uint64_t* pv_done_b = pv_done_a + 2;
+  uint64_t* o_final = pv_done_b + 2;
+  uint64_t* mma_done = o_final + 2;   // one per MMA-issuing warp
   volatile int* misc = reinterpret_cast<volatile int*>(smem + L::kOffMisc);
   // misc[0] TMEM base, [1]/[2] segments of q-tile 0/1, [3]/[4] key tiles of q-tile 0/1, [5] abort
-  volatile int* grp = misc + 8;   // producer scratch: owning lane of each 8-column group
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int pair = blockIdx.x, bh = blockIdx.y;
@@ -139,16 +141,8 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
     }
     if (lane == 0) {
       misc[5] = 0;
-      for (int i = 0; i < L::kNumBars; ++i) {
-        uint32_t count = 1;
-        if (&bars[i] == &k_empty[0] || &bars[i] == &k_empty[1] || &bars[i] == &v_empty[0] ||
-            &bars[i] == &v_empty[1])
-          count = 2;  // one arrival from each q-tile's MMA issuer
-        if (&bars[i] == &pa[0] || &bars[i] == &pa[1] || &bars[i] == &pb[0] || &bars[i] == &pb[1] ||
-            &bars[i] == &go[0] || &bars[i] == &go[1])
-          count = 128;  // every softmax thread of the tile
-        mbar_init(&bars[i], count);
-      }
+      for (int i = 0; i < L::kNumBars; ++i)   // b_empty: every softmax thread of the entry's tile
+        mbar_init(&bars[i], (&bars[i] == &b_empty[0] || &bars[i] == &b_empty[1]) ? 128u : 1u);
       fence_mbar_init();
       tma_prefetch_desc(&tmQ);
     }
@@ -161,16 +155,16 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
   tc_fence_after();
 
   const uint32_t tmem = static_cast<uint32_t>(misc[0]);
-  const int ntile[2] = {misc[3], misc[4]};
-  const int n_entries = ntile[0] + ntile[1];
+  const int ntile0 = misc[3], ntile1 = misc[4];   // packed key tiles of q-tile 0 / 1
+  const int n_entries = ntile0 + ntile1;
   // entry e -> (tile, key tile): tiles alternate while both have key tiles left
   auto entry_of = [&](int e, int& t, int& k) {
-    const int m = min(ntile[0], ntile[1]);
+    const int m = min(ntile0, ntile1);
     if (e < 2 * m) {
       t = e & 1;
       k = e >> 1;
     } else {
-      t = ntile[0] > ntile[1] ? 0 : 1;
+      t = ntile0 > ntile1 ? 0 : 1;
       k = m + (e - 2 * m);
     }
   };
@@ -179,221 +173,295 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
 
   if (warp < kSoftmaxWarp0) {
     setmaxnreg_dec<56>();
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer ---
-    if (n_entries > 0) {
-      if (lane == 0) {
-        const uint32_t qbytes = static_cast<uint32_t>((ntile[0] > 0) + (ntile[1] > 0)) * L::kTileBytes;
-        mbar_arrive_expect_tx(q_full, qbytes);
+    // ------------------------------------------- segment gather helpers ---
+    // An entry's segments, one lane per segment (a 128-key tile holds at
+    // most 128 / 8 = 16): a warp scan of the lengths gives each column.
+    struct Seg {
+      uint32_t sg;
+      int lvl, len, col, row, fill;
+      bool mine;
+    };
+    auto scan = [&](int t, int& cursor) -> Seg {
+      const uint32_t* tseg = segs + t * kPyrMaxSegs;
+      const int nseg = misc[1 + t];
+      const int gi = cursor + lane;
+      Seg g;
+      g.sg = (lane < 16 && gi < nseg) ? tseg[gi] : 0u;
+      g.lvl = static_cast<int>((g.sg >> 16) & 3u);
+      g.len = (lane < 16 && gi < nseg) ? (BLK >> g.lvl) : 0;
+      int incl = g.len;
 #pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          if (ntile[t] == 0) continue;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      g.col = incl - g.len;
+      g.mine = g.len > 0 && incl <= kTileN;
+      const int nmine = __popc(__ballot_sync(0xffffffffu, g.mine));
+      g.fill = nmine > 0 ? __shfl_sync(0xffffffffu, incl, nmine - 1) : 0;
+      cursor += nmine;
+      g.row = static_cast<int>(g.sg & 0xFFFFu) * g.len;
+      return g;
+    };
+    // wait (lane 0) for a slot's previous phase; false after an error
+    auto slot_free = [&](uint64_t* bar, int e) -> bool {
+      if (e < kStages) return true;
+      const bool w = lane == 0 ? (misc[5] == 0 && mbar_wait(bar, ((e / kStages) - 1) & 1)) : true;
+      return __shfl_sync(0xffffffffu, w, 0);
+    };
+    // zero rows [r0, r1) of a K or V slot so masked products stay finite
+    auto zero_rows = [&](uint8_t* st, int r0, int r1) {
+      if (r0 < r1) {
+        const int per_half = (r1 - r0) * 8;   // 16-byte chunks per 64-column half
+        for (int idx = lane; idx < per_half * (D / 64); idx += 32) {
+          const int hd = idx >= per_half ? 1 : 0;
+          const int rem = idx - hd * per_half;
+          reinterpret_cast<uint4*>(st + hd * kHalfBytes + (r0 + (rem >> 3)) * 128)[rem & 7] = make_uint4(0, 0, 0, 0);
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      }
+    };
+    // TMA of the segment pieces whose columns lie in [c0, c1); a segment
+    // longer than 64 keys (level 0 of block 128) goes in two 64-row pieces
+    // (the level maps' boxes are at most 64 rows), so no piece crosses 64
+    auto issue = [&](const Seg& g, const CUtensorMap* lvmaps, uint64_t* full, uint8_t* st, int c0, int c1) {
+      const int rows = max(0, min(g.fill, c1) - c0);
+      if (lane == 0) mbar_arrive_expect_tx(full, static_cast<uint32_t>(rows) * D * 2);
+      __syncwarp();
+      if (g.mine) {
 #pragma unroll
-          for (int hd = 0; hd < D / 64; ++hd)
-            tma_load_3d(&tmQ, q_full, smem + L::kOffQ + t * L::kTileBytes + hd * kHalfBytes, hd * 64,
-                        (qtile0 + t) * kTileM, bh);
+        for (int q = 0; q < 2; ++q) {
+          const int cq = g.col + 64 * q;
+          if ((q == 0 || g.len > 64) && cq >= c0 && cq < c1) {
+#pragma unroll
+            for (int hd = 0; hd < D / 64; ++hd)
+              tma_load_3d(&lvmaps[g.lvl], full, st + hd * kHalfBytes + cq * 128, hd * 64, g.row + 64 * q, bh);
+          }
         }
       }
-      int cursor[2] = {0, 0};   // next segment of each q-tile
-      int issued = 0;
-      bool ok = true;
-      const float NEG_INF = -__int_as_float(0x7f800000);
-      for (int e = 0; e < n_entries && ok; ++e) {
-        int t, k;
-        entry_of(e, t, k);
-        const int s = e % kStages;
-        const uint32_t par = ((e / kStages) - 1) & 1;
-        // One lane per segment (a 128-key tile holds at most 128 / 8 = 16):
-        // a warp scan of the lengths gives each segment's column.
-        const uint32_t* tseg = segs + t * kPyrMaxSegs;
-        const int nseg = misc[1 + t];
-        const int gi = cursor[t] + lane;
-        const uint32_t sg = (lane < 16 && gi < nseg) ? tseg[gi] : 0u;
-        const int lvl = static_cast<int>((sg >> 16) & 3u);
-        const int len = (lane < 16 && gi < nseg) ? (BLK >> lvl) : 0;
-        int incl = len;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int y = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += y;
-        }
-        const int col = incl - len;
-        const bool mine = len > 0 && incl <= kTileN;
-        const unsigned ball = __ballot_sync(0xffffffffu, mine);
-        const int nmine = __popc(ball);
-        const int fill = nmine > 0 ? __shfl_sync(0xffffffffu, incl, nmine - 1) : 0;
-        cursor[t] += nmine;
-        const int row = static_cast<int>(sg & 0xFFFFu) * len;
+    };
+    // V half h (keys [64h, 64h+64)) of entry e into its slot
+    auto load_v_half = [&](const Seg& g, int e, int h) -> bool {
+      const int s = e % kStages;
+      if (!slot_free(&v_empty[s * 2 + h], e)) return false;
+      uint8_t* vst = smem + L::kOffV + s * L::kTileBytes;
+      zero_rows(vst, max(g.fill, 64 * h), 64 * h + 64);
+      issue(g, maps.v, &v_full[s * 2 + h], vst, 64 * h, 64 * h + 64);
+      return true;
+    };
+    const float NEG_INF = -__int_as_float(0x7f800000);
 
-        if (e >= kStages) {
-          bool w = lane == 0 ? (misc[5] == 0 && mbar_wait(&k_empty[s], par)) : true;
-          if (!__shfl_sync(0xffffffffu, w, 0)) {
-            ok = false;
-            break;
+    if (warp == 3) {
+      // ------------------------------------ producer of Q, K and bias (warp 3) ---
+      // Per-column bias, log2(pooled token count), for row halves A and B.
+      // Each lane writes the columns of its own segment (one value unless
+      // the segment holds the end of the sequence); lanes 16.. fill the
+      // groups no segment covers.
+      auto write_bias = [&](const Seg& g, float* bst) {
+        if (g.mine) {
+          const uint32_t rm = (g.sg >> 18) & 3u;
+          const bool useA = rm & 1u, useB = QH == 1 ? (rm & 1u) : (rm & 2u);
+          const int lv = g.lvl;
+          const float vl = static_cast<float>(lv);
+          const float4 fA = useA ? make_float4(vl, vl, vl, vl) : make_float4(NEG_INF, NEG_INF, NEG_INF, NEG_INF);
+          const float4 fB = useB ? make_float4(vl, vl, vl, vl) : make_float4(NEG_INF, NEG_INF, NEG_INF, NEG_INF);
+          float4* dA = reinterpret_cast<float4*>(bst + g.col);
+          float4* dB = reinterpret_cast<float4*>(bst + kTileN + g.col);
+          for (int i = 0; i < g.len / 4; ++i) {
+            dA[i] = fA;
+            dB[i] = fB;
           }
-        }
-        uint8_t* kst = smem + L::kOffK + s * L::kTileBytes;
-        uint8_t* vst = smem + L::kOffV + s * L::kTileBytes;
-        // empty columns [fill, 128): zero K rows so masked products stay finite
-        if (fill < kTileN) {
-          for (int idx = lane; idx < (kTileN - fill) * 8 * (D / 64); idx += 32) {
-            const int hd = idx / ((kTileN - fill) * 8);
-            const int rem = idx - hd * (kTileN - fill) * 8;
-            reinterpret_cast<uint4*>(kst + hd * kHalfBytes + (fill + rem / 8) * 128)[rem % 8] = make_uint4(0, 0, 0, 0);
-          }
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        }
-        if (lane == 0) mbar_arrive_expect_tx(&k_full[s], static_cast<uint32_t>(fill) * D * 2);
-        __syncwarp();
-        if (mine) {
-#pragma unroll
-          for (int hd = 0; hd < D / 64; ++hd)
-            tma_load_3d(&maps.k[lvl], &k_full[s], kst + hd * kHalfBytes + col * 128, hd * 64, row, bh);
-        }
-        // V slot and the bias table of this stage are free once PV of entry e-2 is done
-        if (e >= kStages) {
-          bool w = lane == 0 ? mbar_wait(&v_empty[s], par) : true;
-          if (!__shfl_sync(0xffffffffu, w, 0)) {
-            ok = false;
-            if (lane == 0) mbar_wait(&k_full[s], (e / kStages) & 1);
-            break;
-          }
-        }
-        if (fill < kTileN) {
-          for (int idx = lane; idx < (kTileN - fill) * 8 * (D / 64); idx += 32) {
-            const int hd = idx / ((kTileN - fill) * 8);
-            const int rem = idx - hd * (kTileN - fill) * 8;
-            reinterpret_cast<uint4*>(vst + hd * kHalfBytes + (fill + rem / 8) * 128)[rem % 8] = make_uint4(0, 0, 0, 0);
-          }
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        }
-        // per-column log2(pooled token count) for row halves A and B: every
-        // lane takes columns lane, lane+32, ...; the owner of each 8-column
-        // group is looked up in grp[] and its fields fetched by shuffle
-        float* bst = bias + s * 2 * kTileN;
-        if (mine)
-          for (int g = col / 8; g < (col + len) / 8; ++g) grp[g] = lane;
-        __syncwarp();
-#pragma unroll
-        for (int cc = 0; cc < kTileN / 32; ++cc) {
-          const int c = cc * 32 + lane;
-          const int src = c < fill ? grp[c / 8] : 0;
-          const uint32_t sg_o = __shfl_sync(0xffffffffu, sg, src);
-          const int col_o = __shfl_sync(0xffffffffu, col, src);
-          const int row_o = __shfl_sync(0xffffffffu, row, src);
-          float bA = NEG_INF, bB = NEG_INF;
-          if (c < fill) {
-            const int lv = static_cast<int>((sg_o >> 16) & 3u);
-            const uint32_t rm = (sg_o >> 18) & 3u;
-            const int gr = row_o + (c - col_o);
-            float bv = NEG_INF;
-            if (gr < p.pool_rows[lv]) {
-              const int count = min(1 << lv, p.N - (gr << lv));
-              bv = count == (1 << lv) ? static_cast<float>(lv) : log2f(static_cast<float>(count));
+          // the segment that holds the end of the sequence: short last group
+          // (fewer than 2^lv tokens) and rows past the level's end
+          if ((g.row + g.len) << lv > p.N) {
+            const int rows_l = (p.N + (1 << lv) - 1) >> lv;
+            for (int i = 0; i < g.len; ++i) {
+              const int gr = g.row + i;
+              float bv = NEG_INF;
+              if (gr < rows_l) {
+                const int count = min(1 << lv, p.N - (gr << lv));
+                bv = count == (1 << lv) ? vl : log2f(static_cast<float>(count));
+              }
+              bst[g.col + i] = useA ? bv : NEG_INF;
+              bst[kTileN + g.col + i] = useB ? bv : NEG_INF;
             }
-            bA = (rm & 1u) ? bv : NEG_INF;
-            bB = (QH == 1 ? (rm & 1u) : (rm & 2u)) ? bv : NEG_INF;
           }
-          bst[c] = bA;
-          bst[kTileN + c] = bB;
+        }
+        const int g_empty = g.fill / 8 + (lane - 16);   // columns [fill, 128) hold no key
+        if (lane >= 16 && g_empty < kTileN / 8) {
+          const float4 n4 = make_float4(NEG_INF, NEG_INF, NEG_INF, NEG_INF);
+          float4* dA = reinterpret_cast<float4*>(bst + g_empty * 8);
+          float4* dB = reinterpret_cast<float4*>(bst + kTileN + g_empty * 8);
+          dA[0] = n4;
+          dA[1] = n4;
+          dB[0] = n4;
+          dB[1] = n4;
         }
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&b_full[s]);
-          mbar_arrive_expect_tx(&v_full[s], static_cast<uint32_t>(fill) * D * 2);
-        }
-        __syncwarp();
-        if (mine) {
-#pragma unroll
-          for (int hd = 0; hd < D / 64; ++hd)
-            tma_load_3d(&maps.v[lvl], &v_full[s], vst + hd * kHalfBytes + col * 128, hd * 64, row, bh);
-        }
-        issued = e + 1;
-      }
-      if (!ok && lane == 0) misc[5] = 1;
-      if (lane == 0) {
-        for (int e = (issued > kStages ? issued - kStages : 0); e < issued; ++e) {
-          const int s = e % kStages;
-          mbar_wait(&k_full[s], (e / kStages) & 1);
-          mbar_wait(&v_full[s], (e / kStages) & 1);
-        }
-        mbar_wait(q_full, 0);
-      }
-    }
-  } else if (warp <= 2) {
-    // ---------------------------------------------- MMA issue, q-tile t ---
-    const int t = warp - 1;
-    if (lane == 0 && n_entries > 0) {
-      const int cnt = ntile[t];
-      bool ok = mbar_wait(q_full, 0);
-      const uint64_t dq = smem_desc(smem_addr(smem + L::kOffQ + t * L::kTileBytes), 16, 1024);
-      const uint64_t dk0 = smem_desc(sK, 16, 1024);
-      const uint64_t dv0 = smem_desc(sV, kHalfBytes, 1024);
-      constexpr uint64_t kStageStep = L::kTileBytes >> 4;
-      const uint32_t s_tmem = tmem + t * 128;
-      const uint32_t o_tmem = tmem + 256 + t * D;
-      int pend = -1, done = 0;
-      uint32_t pph = 0;
-      auto issue_pv = [&]() -> bool {
-        const int ps = pend % kStages;
-        const uint64_t dv = dv0 + ps * kStageStep;
-        if (!mbar_wait(&pa[t], pph) || !mbar_wait(&v_full[ps], (pend / kStages) & 1)) return false;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_ts(o_tmem, s_tmem + kk * 8, dv + ((kk * 16 * 128) >> 4), kIdescPV, (done == 0 && kk == 0) ? 0u : 1u);
-        if (!mbar_wait(&pb[t], pph)) return false;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 4; kk < 8; ++kk)
-          mma_ts(o_tmem, s_tmem + kk * 8, dv + ((kk * 16 * 128) >> 4), kIdescPV, 1u);
-        pph ^= 1u;
-        mma_commit(&v_empty[ps]);
-        if (++done == cnt) mma_commit(&o_final[t]);
-        pend = -1;
-        return true;
       };
-      for (int e = 0; ok && e < n_entries; ++e) {
-        int te, k;
-        entry_of(e, te, k);
-        const int s = e % kStages;
-        const uint32_t par = (e / kStages) & 1;
-        if (pend >= 0 && !issue_pv()) {
-          ok = false;
-          break;
-        }
-        // every entry's K must have landed before this tile reports the slot free
-        if (!mbar_wait(&k_full[s], par)) {
-          ok = false;
-          break;
-        }
-        if (te == t) {
-          tc_fence_after();
-          const uint64_t dk = dk0 + s * kStageStep;
+      if (n_entries > 0) {
+        if (lane == 0) {
+          const uint32_t qbytes = static_cast<uint32_t>((ntile0 > 0) + (ntile1 > 0)) * L::kTileBytes;
+          mbar_arrive_expect_tx(q_full, qbytes);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t off = static_cast<uint64_t>((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
-            mma_ss(s_tmem, dq + off, dk + off, kIdescS, kk > 0 ? 1u : 0u);
+          for (int t = 0; t < 2; ++t) {
+            if ((t == 0 ? ntile0 : ntile1) == 0) continue;
+#pragma unroll
+            for (int hd = 0; hd < D / 64; ++hd)
+              tma_load_3d(&tmQ, q_full, smem + L::kOffQ + t * L::kTileBytes + hd * kHalfBytes, hd * 64,
+                          (qtile0 + t) * kTileM, bh);
           }
-          mma_commit(&s_ready[t]);
-          mma_commit(&k_empty[s]);
-          pend = e;
-        } else {
-          mma_commit(&k_empty[s]);
-          if (!mbar_wait(&v_full[s], par)) {
+        }
+        int cursor0 = 0, cursor1 = 0, k_issued = 0;
+        bool ok = true;
+        for (int e = 0; e < n_entries; ++e) {
+          int t, k;
+          entry_of(e, t, k);
+          const Seg g = t == 0 ? scan(0, cursor0) : scan(1, cursor1);
+          const int s = e % kStages;
+          if (!slot_free(&k_empty[s], e)) {
             ok = false;
             break;
           }
-          mma_commit(&v_empty[s]);
+          uint8_t* kst = smem + L::kOffK + s * L::kTileBytes;
+          zero_rows(kst, g.fill, kTileN);
+          issue(g, maps.k, &k_full[s], kst, 0, kTileN);
+          k_issued = e + 1;
+          // the bias slot is free once the softmax of entry e-2 has read it
+          if (!slot_free(&b_empty[s], e)) {
+            ok = false;
+            break;
+          }
+          write_bias(g, bias + s * 2 * kTileN);
+          if (lane == 0) mbar_arrive(&b_full[s]);
         }
-        if (misc[5]) ok = false;
+        if (!ok && lane == 0) misc[5] = 1;
+        // Loads still in flight must land before the CTA can exit.
+        if (lane == 0) {
+          for (int e = (k_issued > kStages ? k_issued - kStages : 0); e < k_issued; ++e)
+            mbar_wait(&k_full[e % kStages], (e / kStages) & 1);
+          mbar_wait(q_full, 0);
+        }
       }
-      if (ok && pend >= 0 && !issue_pv()) ok = false;
-      if (!ok) misc[5] = 1;
-      mma_commit(&mma_done[t]);
-      mbar_wait(&mma_done[t], 0);
+    } else if (warp == 0) {
+      // ---------------------------------------------------- S issue (warp 0) ---
+      // Entry e's S = Q_t K_e^T goes into the one S buffer once the softmax that
+      // consumed entry e-1's S has loaded it; warp-wide, one elected lane issues.
+      if (n_entries > 0) {
+        bool ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0));
+        if (!ok && lane == 0) misc[5] = 1;
+        const uint64_t dq0 = smem_desc(smem_addr(smem + L::kOffQ), 16, 1024);
+        const uint64_t dk0 = smem_desc(sK, 16, 1024);
+        constexpr uint64_t kStageStep = L::kTileBytes >> 4;
+        int prev_t = 0;
+        for (int e = 0; e < n_entries; ++e) {
+          int t, k;
+          entry_of(e, t, k);
+          const int s = e % kStages;
+          if (e > 0) named_bar_sync(kBarSFree + prev_t, kHandoff);
+          ok = ok && !__any_sync(0xffffffffu, misc[5] != 0);
+          bool seen = false;
+          if (ok) {
+            seen = __all_sync(0xffffffffu, mbar_wait(&k_full[s], (e / kStages) & 1));
+            if (!seen) {
+              ok = false;
+              if (lane == 0) misc[5] = 1;
+            }
+          }
+          if (ok) {
+            tc_fence_after();
+            const uint64_t dq = dq0 + t * kStageStep;
+            const uint64_t dk = dk0 + s * kStageStep;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint64_t off = static_cast<uint64_t>((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+              mma_ss_warp(tmem, dq + off, dk + off, kIdescS, kk > 0 ? 1u : 0u);
+            }
+          }
+          // committed also after an error, so that the softmax keeps its place
+          mma_commit_warp(&s_ready[t]);
+          // the K slot is free once this S completes (only if its load landed)
+          if (seen) mma_commit_warp(&k_empty[s]);
+          prev_t = t;
+        }
+        named_bar_sync(kBarSFree + prev_t, kHandoff);   // the last S has been loaded
+        mma_commit_warp(&mma_done[0]);
+        mbar_wait(&mma_done[0], 0);
+      }
+    } else {
+      // ------------------------- V loads and PV issue for q-tile t (warps 1, 2) ---
+      // O_t += P_t V in two halves, each as soon as the softmax warpgroup has
+      // written that half of P_t.  This warp also loads V of its own next
+      // entry, each 64-key half as soon as the slot's half is free, so that
+      // the V of an entry is in flight while the previous entry's softmax runs.
+      const int t = warp - 1;
+      const int cnt = t == 0 ? ntile0 : ntile1;
+      if (n_entries > 0 && cnt > 0) {
+        const uint64_t dv0 = smem_desc(sV, kHalfBytes, 1024);
+        constexpr uint64_t kStageStep = L::kTileBytes >> 4;
+        const uint32_t a_tmem = tmem + 128 + 64 * t;
+        const uint32_t o_tmem = tmem + 256 + t * D;
+        int cursor = 0;
+        auto next_own = [&](int e) -> int {   // first entry >= e of this tile, or n_entries
+          for (; e < n_entries; ++e) {
+            int te, k;
+            entry_of(e, te, k);
+            if (te == t) break;
+          }
+          return e;
+        };
+        auto aborted = [&]() -> bool { return __any_sync(0xffffffffu, misc[5] != 0); };
+        // Every V half that was issued is waited for (also after an error), so
+        // that no load is in flight when the CTA exits.
+        int e = next_own(0);
+        Seg g = scan(t, cursor);
+        bool cur_lo = load_v_half(g, e, 0);
+        bool cur_hi = cur_lo && load_v_half(g, e, 1);
+        int done = 0;
+        while (e < n_entries) {
+          const int s = e % kStages;
+          const uint64_t dv = dv0 + s * kStageStep;
+          const int en = next_own(e + 1);
+          Seg gn;
+          if (en < n_entries) gn = scan(t, cursor);
+          named_bar_sync(kBarPA + t, kHandoff);
+          bool landed = cur_lo && __all_sync(0xffffffffu, mbar_wait(&v_full[s * 2], (e / kStages) & 1));
+          bool ok = landed && !aborted();
+          if (ok) {
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_ts_warp(o_tmem, a_tmem + kk * 8, dv + ((kk * 16 * 128) >> 4), kIdescPV,
+                          (done == 0 && kk == 0) ? 0u : 1u);
+            mma_commit_warp(&v_empty[s * 2]);   // first V half free
+          }
+          mma_commit_warp(&pv_done_a[t]);   // also after an error, so that no waiter stalls
+          // first V half of the next entry (its slot half may be the one just read)
+          const bool nxt_lo = en < n_entries && !aborted() && load_v_half(gn, en, 0);
+          named_bar_sync(kBarPB + t, kHandoff);
+          landed = cur_hi && __all_sync(0xffffffffu, mbar_wait(&v_full[s * 2 + 1], (e / kStages) & 1));
+          ok = ok && landed && !aborted();
+          if (ok) {
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 4; kk < 8; ++kk)
+              mma_ts_warp(o_tmem, a_tmem + kk * 8, dv + ((kk * 16 * 128) >> 4), kIdescPV, 1u);
+            mma_commit_warp(&v_empty[s * 2 + 1]);   // second V half free
+          }
+          mma_commit_warp(&pv_done_b[t]);
+          if (++done == cnt) mma_commit_warp(&o_final[t]);
+          if (!ok && lane == 0) misc[5] = 1;
+          const bool nxt_hi = nxt_lo && !aborted() && load_v_half(gn, en, 1);
+          if (en < n_entries && !(nxt_lo && nxt_hi) && lane == 0) misc[5] = 1;
+          e = en;
+          g = gn;
+          cur_lo = nxt_lo;
+          cur_hi = nxt_hi;
+        }
+        mma_commit_warp(&mma_done[1 + t]);
+        mbar_wait(&mma_done[1 + t], 0);
+      }
     }
-  }
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -413,15 +481,15 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
     const bool row_valid = row < p.N;
     const int rh = (QH == 2) ? (r >> 6) : 0;   // which q-block of the tile (bias half)
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-    const uint32_t s_addr = lane_base + t * 128;
+    const uint32_t s_addr = lane_base;
+    const uint32_t p_addr = lane_base + 128 + 64 * t;
     const uint32_t o_addr = lane_base + 256 + t * D;
-    const int cnt = ntile[t];
+    const int cnt = t == 0 ? ntile0 : ntile1;
     const float sl2 = p.scale_log2;
     const float NEG_INF = -__int_as_float(0x7f800000);
 
     float m_used = NEG_INF, l_sum = 0.f;
-    uint32_t sphase = 0, gphase = 0;
-    int et = 0;
+    int et = 0;   // entries of this q-tile processed
     bool ok = true;
     if (cnt > 0) {
       for (int e = 0; e < n_entries; ++e) {
@@ -429,21 +497,23 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
         entry_of(e, te, k);
         if (te != t) continue;
         const int st = e % kStages;
-        bool w_ok = true;
-        if (e > 0) {                       // wait for our turn
-          w_ok = mbar_wait(&go[t], gphase);
-          gphase ^= 1u;
-        }
-        w_ok = w_ok && mbar_wait(&s_ready[t], sphase) && mbar_wait(&b_full[st], (e / kStages) & 1);
-        ok = __all_sync(0xffffffffu, w_ok) && misc[5] == 0;
-        if (!ok) {
+        // After an error the loop still runs to the end (its hand-offs keep
+        // the issuing warps' sequences in step); it only stops trusting TMEM.
+        if (!mbar_wait(&s_ready[t], et & 1)) {
           misc[5] = 1;
-          break;
+          ok = false;
         }
-        sphase ^= 1u;
         tc_fence_after();
         float s[kTileN];
         tmem_ld128(s_addr, s);
+        // the S buffer is free for the next entry's S
+        tc_fence_before();
+        named_bar_sync(kBarSFree + t, kHandoff);
+        // the producer stops after an error, so the bias is then not waited for
+        if (!misc[5] && !mbar_wait(&b_full[st], (e / kStages) & 1)) {
+          misc[5] = 1;
+          ok = false;
+        }
         // x = s * scale * log2e + log2(count), -inf on masked / empty columns
         const float4* bsrc = reinterpret_cast<const float4*>(bias + st * 2 * kTileN + rh * kTileN);
 #pragma unroll
@@ -454,6 +524,7 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
           s[4 * c4 + 2] = fmaf(s[4 * c4 + 2], sl2, bv.z);
           s[4 * c4 + 3] = fmaf(s[4 * c4 + 3], sl2, bv.w);
         }
+        mbar_arrive(&b_empty[st]);   // the producer may now rewrite this bias slot
         float a[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) a[u] = fmaxf(s[2 * u], s[2 * u + 1]);
@@ -469,7 +540,21 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
           m_used = mx;
           l_sum *= factor;
         }
-        if (et > 0 && __any_sync(0xffffffffu, factor != 1.f)) {
+        // The previous PV of this tile reads P_t and accumulates into O_t: each
+        // half of P_t is rewritten once that half of the PV has completed, and
+        // O_t is rescaled once all of it has.
+        auto wait_pv = [&](uint64_t* bar) {
+          if (et > 0) {
+            if (!mbar_wait(bar, (et - 1) & 1)) {
+              misc[5] = 1;
+              ok = false;
+            }
+            tc_fence_after();
+          }
+        };
+        const bool rescale = et > 0 && __any_sync(0xffffffffu, factor != 1.f);
+        if (rescale) {
+          wait_pv(&pv_done_b[t]);
 #pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
             float ov[32];
@@ -484,29 +569,27 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
         {
           uint32_t pk[32];
           l_sum += exp_pack_64(s, 1.f, neg_m, pk);
-          tmem_st32(s_addr, reinterpret_cast<const float*>(pk));
+          if (!rescale) wait_pv(&pv_done_a[t]);
+          tmem_st32(p_addr, reinterpret_cast<const float*>(pk));
           tmem_st_wait();
           tc_fence_before();
-          mbar_arrive(&pa[t]);
+          named_bar_sync(kBarPA + t, kHandoff);
         }
         {
           uint32_t pk[32];
           l_sum += exp_pack_64(s + 64, 1.f, neg_m, pk);
-          tmem_st32(s_addr + 32, reinterpret_cast<const float*>(pk));
+          if (!rescale) wait_pv(&pv_done_b[t]);
+          tmem_st32(p_addr + 32, reinterpret_cast<const float*>(pk));
           tmem_st_wait();
           tc_fence_before();
-          mbar_arrive(&pb[t]);
-        }
-        if (e + 1 < n_entries) {           // pass the turn to the next entry's tile
-          int tn, kn;
-          entry_of(e + 1, tn, kn);
-          mbar_arrive(&go[tn]);
+          named_bar_sync(kBarPB + t, kHandoff);
         }
         ++et;
       }
     }
 
     // ------------------------------------------------------------ epilogue ---
+    ok = __all_sync(0xffffffffu, ok && misc[5] == 0);
     if (cnt > 0 && ok) {
       ok = __all_sync(0xffffffffu, mbar_wait(&o_final[t], 0));
       if (!ok) misc[5] = 1;
