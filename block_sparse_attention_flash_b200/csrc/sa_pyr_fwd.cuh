@@ -38,6 +38,7 @@ constexpr int kPyrMaxBlocks = 1024;                 // k-blocks per sequence
 constexpr int kPyrWarps = 12;
 constexpr int kPyrThreads = kPyrWarps * 32;
 constexpr int kPyrMaxSegs = 2 * kPyrMaxBlocks;      // per q-tile (union of 2 q-blocks)
+constexpr int kPyrMaxEntries = kPyrMaxBlocks;       // packed key tiles per q-tile
 
 struct PyrParams {
   int B, H, N;
@@ -56,7 +57,8 @@ struct PyrSmem {
   static constexpr int kOffK = 2 * kTileBytes;
   static constexpr int kOffV = kOffK + kStages * kTileBytes;
   static constexpr int kOffSeg = kOffV + kStages * kTileBytes;         // [tile][kPyrMaxSegs] u32
-  static constexpr int kOffBias = kOffSeg + 2 * kPyrMaxSegs * 4;       // [stage][half A/B][128] f32
+  static constexpr int kOffEnt = kOffSeg + 2 * kPyrMaxSegs * 4;        // [tile][kPyrMaxEntries] u16
+  static constexpr int kOffBias = kOffEnt + 2 * kPyrMaxEntries * 2;    // [stage][half A/B][128] f32
   // q_full, k_full[2], v_full[2][2], k_empty[2], v_empty[2][2], b_full[2],
   // b_empty[2], s_ready[2], pv_done_a[2], pv_done_b[2], o_final[2], mma_done[3]
   // (V slots are filled and released by 64-key half: rows [0,64) feed the
@@ -86,6 +88,7 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint32_t* segs = reinterpret_cast<uint32_t*>(smem + L::kOffSeg);
+  uint16_t* ents = reinterpret_cast<uint16_t*>(smem + L::kOffEnt);
   float* bias = reinterpret_cast<float*>(smem + L::kOffBias);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
   uint64_t* q_full = bars;
@@ -101,7 +104,8 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
   uint64_t* o_final = pv_done_b + 2;
   uint64_t* mma_done = o_final + 2;   // one per MMA-issuing warp
   volatile int* misc = reinterpret_cast<volatile int*>(smem + L::kOffMisc);
-  // misc[0] TMEM base, [1]/[2] segments of q-tile 0/1, [3]/[4] key tiles of q-tile 0/1, [5] abort
+  // misc[0] TMEM base, [1]/[2] segments of q-tile 0/1, [3]/[4] key tiles of q-tile 0/1, [5] abort,
+  // [6]/[7] packed columns of q-tile 0/1
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int pair = blockIdx.x, bh = blockIdx.y;
@@ -128,8 +132,15 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
             rm = (cA == lvl + 1 ? 1u : 0u) | (cB == lvl + 1 ? 2u : 0u);
           }
           const unsigned ball = __ballot_sync(0xffffffffu, rm != 0);
-          if (rm) segs[t * kPyrMaxSegs + n + __popc(ball & ((1u << lane) - 1u))] =
-              static_cast<uint32_t>(j) | (static_cast<uint32_t>(lvl) << 16) | (rm << 18);
+          if (rm) {
+            // segments of one level have one length, so the packed column
+            // (and with it the key tile) follows from the rank
+            const int rank = __popc(ball & ((1u << lane) - 1u));
+            const int cg = cols + rank * (BLK >> lvl);
+            segs[t * kPyrMaxSegs + n + rank] = static_cast<uint32_t>(j) | (static_cast<uint32_t>(lvl) << 16) |
+                                               (rm << 18) | (static_cast<uint32_t>(cg & (kTileN - 1)) << 24);
+            if ((cg & (kTileN - 1)) == 0) ents[t * kPyrMaxEntries + cg / kTileN] = static_cast<uint16_t>(n + rank);
+          }
           n += __popc(ball);
           cols += __popc(ball) * (BLK >> lvl);
         }
@@ -137,6 +148,7 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
       if (lane == 0) {
         misc[1 + t] = n;
         misc[3 + t] = (cols + kTileN - 1) / kTileN;
+        misc[6 + t] = cols;
       }
     }
     if (lane == 0) {
@@ -175,38 +187,32 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
     setmaxnreg_dec<56>();
     // ------------------------------------------- segment gather helpers ---
     // An entry's segments, one lane per segment (a 128-key tile holds at
-    // most 128 / 8 = 16): a warp scan of the lengths gives each column.
+    // most 128 / 8 = 16), with the columns the list builder assigned.
     struct Seg {
       uint32_t sg;
       int lvl, len, col, row, fill;
       bool mine;
     };
-    auto scan = [&](int t, int& cursor) -> Seg {
-      const uint32_t* tseg = segs + t * kPyrMaxSegs;
-      const int nseg = misc[1 + t];
-      const int gi = cursor + lane;
+    auto seg_of = [&](int t, int k) -> Seg {   // segments of key tile k of q-tile t
+      const int nt = t == 0 ? ntile0 : ntile1;
+      const int start = ents[t * kPyrMaxEntries + k];
+      const int end = k + 1 < nt ? ents[t * kPyrMaxEntries + k + 1] : misc[1 + t];
       Seg g;
-      g.sg = (lane < 16 && gi < nseg) ? tseg[gi] : 0u;
+      g.fill = k + 1 < nt ? kTileN : misc[6 + t] - kTileN * k;
+      g.mine = lane < end - start;
+      g.sg = g.mine ? segs[t * kPyrMaxSegs + start + lane] : 0u;
       g.lvl = static_cast<int>((g.sg >> 16) & 3u);
-      g.len = (lane < 16 && gi < nseg) ? (BLK >> g.lvl) : 0;
-      int incl = g.len;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      g.col = incl - g.len;
-      g.mine = g.len > 0 && incl <= kTileN;
-      const int nmine = __popc(__ballot_sync(0xffffffffu, g.mine));
-      g.fill = nmine > 0 ? __shfl_sync(0xffffffffu, incl, nmine - 1) : 0;
-      cursor += nmine;
+      g.len = g.mine ? (BLK >> g.lvl) : 0;
+      g.col = static_cast<int>((g.sg >> 24) & (kTileN - 1));
       g.row = static_cast<int>(g.sg & 0xFFFFu) * g.len;
       return g;
     };
     // wait (lane 0) for a slot's previous phase; false after an error
     auto slot_free = [&](uint64_t* bar, int e) -> bool {
       if (e < kStages) return true;
-      const bool w = lane == 0 ? (misc[5] == 0 && mbar_wait(bar, ((e / kStages) - 1) & 1)) : true;
+      const uint32_t par = ((e / kStages) - 1) & 1;
+      if (__all_sync(0xffffffffu, mbar_test(bar, par))) return true;   // the common case
+      const bool w = lane == 0 ? (misc[5] == 0 && mbar_wait(bar, par)) : true;
       return __shfl_sync(0xffffffffu, w, 0);
     };
     // zero rows [r0, r1) of a K or V slot so masked products stay finite
@@ -250,55 +256,55 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
       return true;
     };
     const float NEG_INF = -__int_as_float(0x7f800000);
+    // Per-column bias, log2(pooled token count), for row halves A and B.
+    // Each lane writes the columns of its own segment (one value unless
+    // the segment holds the end of the sequence); lanes 16.. fill the
+    // groups no segment covers.
+    auto write_bias = [&](const Seg& g, float* bst) {
+      if (g.mine) {
+        const uint32_t rm = (g.sg >> 18) & 3u;
+        const bool useA = rm & 1u, useB = QH == 1 ? (rm & 1u) : (rm & 2u);
+        const int lv = g.lvl;
+        const float vl = static_cast<float>(lv);
+        const float4 fA = useA ? make_float4(vl, vl, vl, vl) : make_float4(NEG_INF, NEG_INF, NEG_INF, NEG_INF);
+        const float4 fB = useB ? make_float4(vl, vl, vl, vl) : make_float4(NEG_INF, NEG_INF, NEG_INF, NEG_INF);
+        float4* dA = reinterpret_cast<float4*>(bst + g.col);
+        float4* dB = reinterpret_cast<float4*>(bst + kTileN + g.col);
+        for (int i = 0; i < g.len / 4; ++i) {
+          dA[i] = fA;
+          dB[i] = fB;
+        }
+        // the segment that holds the end of the sequence: short last group
+        // (fewer than 2^lv tokens) and rows past the level's end
+        if ((g.row + g.len) << lv > p.N) {
+          const int rows_l = (p.N + (1 << lv) - 1) >> lv;
+          for (int i = 0; i < g.len; ++i) {
+            const int gr = g.row + i;
+            float bv = NEG_INF;
+            if (gr < rows_l) {
+              const int count = min(1 << lv, p.N - (gr << lv));
+              bv = count == (1 << lv) ? vl : log2f(static_cast<float>(count));
+            }
+            bst[g.col + i] = useA ? bv : NEG_INF;
+            bst[kTileN + g.col + i] = useB ? bv : NEG_INF;
+          }
+        }
+      }
+      const int g_empty = g.fill / 8 + (lane - 16);   // columns [fill, 128) hold no key
+      if (lane >= 16 && g_empty < kTileN / 8) {
+        const float4 n4 = make_float4(NEG_INF, NEG_INF, NEG_INF, NEG_INF);
+        float4* dA = reinterpret_cast<float4*>(bst + g_empty * 8);
+        float4* dB = reinterpret_cast<float4*>(bst + kTileN + g_empty * 8);
+        dA[0] = n4;
+        dA[1] = n4;
+        dB[0] = n4;
+        dB[1] = n4;
+      }
+      __syncwarp();
+    };
 
     if (warp == 3) {
       // ------------------------------------ producer of Q, K and bias (warp 3) ---
-      // Per-column bias, log2(pooled token count), for row halves A and B.
-      // Each lane writes the columns of its own segment (one value unless
-      // the segment holds the end of the sequence); lanes 16.. fill the
-      // groups no segment covers.
-      auto write_bias = [&](const Seg& g, float* bst) {
-        if (g.mine) {
-          const uint32_t rm = (g.sg >> 18) & 3u;
-          const bool useA = rm & 1u, useB = QH == 1 ? (rm & 1u) : (rm & 2u);
-          const int lv = g.lvl;
-          const float vl = static_cast<float>(lv);
-          const float4 fA = useA ? make_float4(vl, vl, vl, vl) : make_float4(NEG_INF, NEG_INF, NEG_INF, NEG_INF);
-          const float4 fB = useB ? make_float4(vl, vl, vl, vl) : make_float4(NEG_INF, NEG_INF, NEG_INF, NEG_INF);
-          float4* dA = reinterpret_cast<float4*>(bst + g.col);
-          float4* dB = reinterpret_cast<float4*>(bst + kTileN + g.col);
-          for (int i = 0; i < g.len / 4; ++i) {
-            dA[i] = fA;
-            dB[i] = fB;
-          }
-          // the segment that holds the end of the sequence: short last group
-          // (fewer than 2^lv tokens) and rows past the level's end
-          if ((g.row + g.len) << lv > p.N) {
-            const int rows_l = (p.N + (1 << lv) - 1) >> lv;
-            for (int i = 0; i < g.len; ++i) {
-              const int gr = g.row + i;
-              float bv = NEG_INF;
-              if (gr < rows_l) {
-                const int count = min(1 << lv, p.N - (gr << lv));
-                bv = count == (1 << lv) ? vl : log2f(static_cast<float>(count));
-              }
-              bst[g.col + i] = useA ? bv : NEG_INF;
-              bst[kTileN + g.col + i] = useB ? bv : NEG_INF;
-            }
-          }
-        }
-        const int g_empty = g.fill / 8 + (lane - 16);   // columns [fill, 128) hold no key
-        if (lane >= 16 && g_empty < kTileN / 8) {
-          const float4 n4 = make_float4(NEG_INF, NEG_INF, NEG_INF, NEG_INF);
-          float4* dA = reinterpret_cast<float4*>(bst + g_empty * 8);
-          float4* dB = reinterpret_cast<float4*>(bst + kTileN + g_empty * 8);
-          dA[0] = n4;
-          dA[1] = n4;
-          dB[0] = n4;
-          dB[1] = n4;
-        }
-        __syncwarp();
-      };
       if (n_entries > 0) {
         if (lane == 0) {
           const uint32_t qbytes = static_cast<uint32_t>((ntile0 > 0) + (ntile1 > 0)) * L::kTileBytes;
@@ -312,12 +318,12 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
                           (qtile0 + t) * kTileM, bh);
           }
         }
-        int cursor0 = 0, cursor1 = 0, k_issued = 0;
+        int k_issued = 0;
         bool ok = true;
         for (int e = 0; e < n_entries; ++e) {
           int t, k;
           entry_of(e, t, k);
-          const Seg g = t == 0 ? scan(0, cursor0) : scan(1, cursor1);
+          const Seg g = seg_of(t, k);
           const int s = e % kStages;
           if (!slot_free(&k_empty[s], e)) {
             ok = false;
@@ -401,7 +407,6 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
         constexpr uint64_t kStageStep = L::kTileBytes >> 4;
         const uint32_t a_tmem = tmem + 128 + 64 * t;
         const uint32_t o_tmem = tmem + 256 + t * D;
-        int cursor = 0;
         auto next_own = [&](int e) -> int {   // first entry >= e of this tile, or n_entries
           for (; e < n_entries; ++e) {
             int te, k;
@@ -414,7 +419,8 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
         // Every V half that was issued is waited for (also after an error), so
         // that no load is in flight when the CTA exits.
         int e = next_own(0);
-        Seg g = scan(t, cursor);
+        int k_own = 0;
+        Seg g = seg_of(t, 0);
         bool cur_lo = load_v_half(g, e, 0);
         bool cur_hi = cur_lo && load_v_half(g, e, 1);
         int done = 0;
@@ -423,7 +429,7 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
           const uint64_t dv = dv0 + s * kStageStep;
           const int en = next_own(e + 1);
           Seg gn;
-          if (en < n_entries) gn = scan(t, cursor);
+          if (en < n_entries) gn = seg_of(t, k_own + 1);
           named_bar_sync(kBarPA + t, kHandoff);
           bool landed = cur_lo && __all_sync(0xffffffffu, mbar_wait(&v_full[s * 2], (e / kStages) & 1));
           bool ok = landed && !aborted();
@@ -455,6 +461,7 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
           if (en < n_entries && !(nxt_lo && nxt_hi) && lane == 0) misc[5] = 1;
           e = en;
           g = gn;
+          ++k_own;
           cur_lo = nxt_lo;
           cur_hi = nxt_hi;
         }
