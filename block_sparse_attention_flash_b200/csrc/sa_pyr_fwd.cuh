@@ -257,52 +257,50 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
     };
     const float NEG_INF = -__int_as_float(0x7f800000);
     // Per-column bias, log2(pooled token count), for row halves A and B.
-    // Each lane writes the columns of its own segment (one value unless
-    // the segment holds the end of the sequence); lanes 16.. fill the
-    // groups no segment covers.
+    // Lane L writes columns [4L, 4L+4) of both halves: the segment that
+    // covers them is found from a mask of segment start columns (segments
+    // are in column order) and its fields are fetched by shuffle.  The value
+    // is the level unless the segment holds the end of the sequence (a short
+    // last group, or rows past the level's end); -inf on masked or empty
+    // columns.
     auto write_bias = [&](const Seg& g, float* bst) {
-      if (g.mine) {
-        const uint32_t rm = (g.sg >> 18) & 3u;
+      const uint32_t starts = __reduce_or_sync(0xffffffffu, g.mine ? (1u << (g.col >> 2)) : 0u);
+      const int c0 = 4 * lane;
+      const int owner = __popc(starts & ((2u << lane) - 1u)) - 1;   // the segment's rank = its lane
+      const int src = owner < 0 ? 0 : owner;
+      const uint32_t sg_o = __shfl_sync(0xffffffffu, g.sg, src);
+      const int col_o = __shfl_sync(0xffffffffu, g.col, src);
+      const int row_o = __shfl_sync(0xffffffffu, g.row, src);
+      float4 vA = make_float4(NEG_INF, NEG_INF, NEG_INF, NEG_INF), vB = vA;
+      if (c0 < g.fill) {
+        const int lv = static_cast<int>((sg_o >> 16) & 3u);
+        const uint32_t rm = (sg_o >> 18) & 3u;
         const bool useA = rm & 1u, useB = QH == 1 ? (rm & 1u) : (rm & 2u);
-        const int lv = g.lvl;
-        const float vl = static_cast<float>(lv);
-        const float4 fA = useA ? make_float4(vl, vl, vl, vl) : make_float4(NEG_INF, NEG_INF, NEG_INF, NEG_INF);
-        const float4 fB = useB ? make_float4(vl, vl, vl, vl) : make_float4(NEG_INF, NEG_INF, NEG_INF, NEG_INF);
-        float4* dA = reinterpret_cast<float4*>(bst + g.col);
-        float4* dB = reinterpret_cast<float4*>(bst + kTileN + g.col);
-        for (int i = 0; i < g.len / 4; ++i) {
-          dA[i] = fA;
-          dB[i] = fB;
-        }
-        // the segment that holds the end of the sequence: short last group
-        // (fewer than 2^lv tokens) and rows past the level's end
-        if ((g.row + g.len) << lv > p.N) {
+        const int gr0 = row_o + (c0 - col_o);
+        float v[4];
+        if (((gr0 + 4) << lv) <= p.N) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) v[i] = static_cast<float>(lv);
+        } else {
           const int rows_l = (p.N + (1 << lv) - 1) >> lv;
-          for (int i = 0; i < g.len; ++i) {
-            const int gr = g.row + i;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int gr = gr0 + i;
             float bv = NEG_INF;
             if (gr < rows_l) {
               const int count = min(1 << lv, p.N - (gr << lv));
-              bv = count == (1 << lv) ? vl : log2f(static_cast<float>(count));
+              bv = count == (1 << lv) ? static_cast<float>(lv) : log2f(static_cast<float>(count));
             }
-            bst[g.col + i] = useA ? bv : NEG_INF;
-            bst[kTileN + g.col + i] = useB ? bv : NEG_INF;
+            v[i] = bv;
           }
         }
+        if (useA) vA = make_float4(v[0], v[1], v[2], v[3]);
+        if (useB) vB = make_float4(v[0], v[1], v[2], v[3]);
       }
-      const int g_empty = g.fill / 8 + (lane - 16);   // columns [fill, 128) hold no key
-      if (lane >= 16 && g_empty < kTileN / 8) {
-        const float4 n4 = make_float4(NEG_INF, NEG_INF, NEG_INF, NEG_INF);
-        float4* dA = reinterpret_cast<float4*>(bst + g_empty * 8);
-        float4* dB = reinterpret_cast<float4*>(bst + kTileN + g_empty * 8);
-        dA[0] = n4;
-        dA[1] = n4;
-        dB[0] = n4;
-        dB[1] = n4;
-      }
+      reinterpret_cast<float4*>(bst)[lane] = vA;
+      reinterpret_cast<float4*>(bst + kTileN)[lane] = vB;
       __syncwarp();
     };
-
     if (warp == 3) {
       // ------------------------------------ producer of Q, K and bias (warp 3) ---
       if (n_entries > 0) {
