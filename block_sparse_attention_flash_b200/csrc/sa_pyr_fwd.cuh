@@ -440,8 +440,6 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
             mma_commit_warp(&v_empty[s * 2]);   // first V half free
           }
           mma_commit_warp(&pv_done_a[t]);   // also after an error, so that no waiter stalls
-          // first V half of the next entry (its slot half may be the one just read)
-          const bool nxt_lo = en < n_entries && !aborted() && load_v_half(gn, en, 0);
           named_bar_sync(kBarPB + t, kHandoff);
           landed = cur_hi && __all_sync(0xffffffffu, mbar_wait(&v_full[s * 2 + 1], (e / kStages) & 1));
           ok = ok && landed && !aborted();
@@ -455,6 +453,9 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
           mma_commit_warp(&pv_done_b[t]);
           if (++done == cnt) mma_commit_warp(&o_final[t]);
           if (!ok && lane == 0) misc[5] = 1;
+          // V of the next entry, after this entry's hand-offs so that the
+          // softmax never waits at PB for these gathers
+          const bool nxt_lo = en < n_entries && !aborted() && load_v_half(gn, en, 0);
           const bool nxt_hi = nxt_lo && !aborted() && load_v_half(gn, en, 1);
           if (en < n_entries && !(nxt_lo && nxt_hi) && lane == 0) misc[5] = 1;
           e = en;
