@@ -39,6 +39,10 @@ constexpr int kPyrWarps = 12;
 constexpr int kPyrThreads = kPyrWarps * 32;
 constexpr int kPyrMaxSegs = 2 * kPyrMaxBlocks;      // per q-tile (union of 2 q-blocks)
 constexpr int kPyrMaxEntries = kPyrMaxBlocks;       // packed key tiles per q-tile
+// Raw-logit bias of a masked or empty column, and the row maximum below which
+// a row has no valid column in a tile (real logits are many orders smaller).
+constexpr float kMaskedBias = -30000.f;
+constexpr float kMaskedCut = -10000.f;
 
 struct PyrParams {
   int B, H, N;
@@ -58,13 +62,20 @@ struct PyrSmem {
   static constexpr int kOffV = kOffK + kStages * kTileBytes;
   static constexpr int kOffSeg = kOffV + kStages * kTileBytes;         // [tile][kPyrMaxSegs] u32
   static constexpr int kOffEnt = kOffSeg + 2 * kPyrMaxSegs * 4;        // [tile][kPyrMaxEntries] u16
-  static constexpr int kOffBias = kOffEnt + 2 * kPyrMaxEntries * 2;    // [stage][half A/B][128] f32
-  // q_full, k_full[2], v_full[2][2], k_empty[2], v_empty[2][2], b_full[2],
-  // b_empty[2], s_ready[2], pv_done_a[2], pv_done_b[2], o_final[2], mma_done[3]
+  // The logit bias enters S through one extra K = 16 MMA step: QX holds, per
+  // q row, selector columns (1, 1 on the pair of its q-block), KX per K slot
+  // holds, per key column, the bias in raw logit units split into bf16
+  // hi + lo for each q-block.  Both are 128 x 16 bf16 in the K-major
+  // no-swizzle layout: element (r, c) at (r/8)*256 + (c/8)*128 + (r%8)*16 + (c%8)*2.
+  static constexpr int kOffQX = (kOffEnt + 2 * kPyrMaxEntries * 2 + 1023) / 1024 * 1024;
+  static constexpr int kOffKX = kOffQX + 4096;                          // [slot] 4 KB
+  // q_full, k_full[2], v_full[2][2], k_empty[2], v_empty[2][2], s_ready[2],
+  // pv_done_a[2], pv_done_b[2], o_final[2], mma_done[3]
   // (V slots are filled and released by 64-key half: rows [0,64) feed the
   // first half of PV, rows [64,128) the second)
-  static constexpr int kNumBars = 1 + 8 * kStages + 2 * 4 + 3;
-  static constexpr int kOffBar = kOffBias + kStages * 2 * kTileN * 4;
+  static constexpr int kNumBars = 1 + 6 * kStages + 2 * 4 + 3;
+  static constexpr int kOffKXPat = kOffKX + kStages * 4096;             // 17 KX row patterns
+  static constexpr int kOffBar = kOffKXPat + 17 * 16;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffMisc + 128;
   static constexpr int kAlloc = kBytes + 1024;
@@ -89,16 +100,16 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint32_t* segs = reinterpret_cast<uint32_t*>(smem + L::kOffSeg);
   uint16_t* ents = reinterpret_cast<uint16_t*>(smem + L::kOffEnt);
-  float* bias = reinterpret_cast<float*>(smem + L::kOffBias);
+  uint8_t* qx = smem + L::kOffQX;
+  uint8_t* kx = smem + L::kOffKX;
+  uint4* kxpat = reinterpret_cast<uint4*>(smem + L::kOffKXPat);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;
   uint64_t* v_full = bars + 1 + kStages;          // [slot * 2 + half]
   uint64_t* k_empty = bars + 1 + 3 * kStages;
   uint64_t* v_empty = bars + 1 + 4 * kStages;     // [slot * 2 + half]
-  uint64_t* b_full = bars + 1 + 6 * kStages;
-  uint64_t* b_empty = bars + 1 + 7 * kStages;
-  uint64_t* s_ready = bars + 1 + 8 * kStages;
+  uint64_t* s_ready = bars + 1 + 6 * kStages;
   uint64_t* pv_done_a = s_ready + 2;
   uint64_t* pv_done_b = pv_done_a + 2;
   uint64_t* o_final = pv_done_b + 2;
@@ -153,14 +164,47 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
     }
     if (lane == 0) {
       misc[5] = 0;
-      for (int i = 0; i < L::kNumBars; ++i)   // b_empty: every softmax thread of the entry's tile
-        mbar_init(&bars[i], (&bars[i] == &b_empty[0] || &bars[i] == &b_empty[1]) ? 128u : 1u);
+      for (int i = 0; i < L::kNumBars; ++i)   // k_full: the K loads' arrival and the KX writes' arrival
+        mbar_init(&bars[i], (&bars[i] == &k_full[0] || &bars[i] == &k_full[1]) ? 2u : 1u);
       fence_mbar_init();
       tma_prefetch_desc(&tmQ);
     }
   } else if (warp == 1) {
     tmem_alloc(const_cast<uint32_t*>(reinterpret_cast<volatile uint32_t*>(misc)), 512);
     tmem_relinquish();
+  } else if (warp == 2 || warp == 3) {
+    // QX: q rows of the tile's first q-block select columns 0-1, of its second
+    // 2-3 (block 128: every row 0-1); the KX columns 8-15 of both slots are 0
+    const int i0 = (warp - 2) * 32 + lane;
+    for (int i = i0; i < 128; i += 64) {
+      const bool second = QH == 2 && i >= 64;
+      uint4 w;
+      w.x = second ? 0u : 0x3F803F80u;   // bf16 1.0 in columns 0 and 1
+      w.y = second ? 0x3F803F80u : 0u;   // columns 2 and 3
+      w.z = 0u;
+      w.w = 0u;
+      const int off = (i >> 3) * 256 + (i & 7) * 16;
+      *reinterpret_cast<uint4*>(qx + off) = w;
+      *reinterpret_cast<uint4*>(qx + off + 128) = make_uint4(0, 0, 0, 0);
+      for (int sl = 0; sl < kStages; ++sl) *reinterpret_cast<uint4*>(kx + sl * 4096 + off + 128) = make_uint4(0, 0, 0, 0);
+    }
+    // KX row patterns of full groups: index 4 * level + useA + 2 * useB, and
+    // 16 for a column that holds no key
+    if (warp == 2 && lane < 17) {
+      const float inv_sl2 = 1.f / p.scale_log2;
+      const int lv = lane >> 2;
+      const bool useA = lane < 16 && (lane & 1), useB = lane < 16 && (lane & 2);
+      const float b = static_cast<float>(lv) * inv_sl2;
+      const float bA = useA ? b : kMaskedBias, bB = useB ? b : kMaskedBias;
+      const __nv_bfloat16 hA = __float2bfloat16(bA), hB = __float2bfloat16(bB);
+      const __nv_bfloat16 lA = __float2bfloat16(bA - __bfloat162float(hA));
+      const __nv_bfloat16 lB = __float2bfloat16(bB - __bfloat162float(hB));
+      kxpat[lane] = make_uint4(
+          static_cast<uint32_t>(__bfloat16_as_ushort(hA)) | (static_cast<uint32_t>(__bfloat16_as_ushort(lA)) << 16),
+          static_cast<uint32_t>(__bfloat16_as_ushort(hB)) | (static_cast<uint32_t>(__bfloat16_as_ushort(lB)) << 16), 0u,
+          0u);
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   tc_fence_before();
   __syncthreads();
@@ -256,14 +300,17 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
       return true;
     };
     const float NEG_INF = -__int_as_float(0x7f800000);
-    // Per-column bias, log2(pooled token count), for row halves A and B.
-    // Lane L writes columns [4L, 4L+4) of both halves: the segment that
-    // covers them is found from a mask of segment start columns (segments
-    // are in column order) and its fields are fetched by shuffle.  The value
-    // is the level unless the segment holds the end of the sequence (a short
-    // last group, or rows past the level's end); -inf on masked or empty
+    // The bias of each key column, log2(pooled token count) / (scale log2 e) in
+    // raw logit units, for the tile's two q-blocks, into the K slot's KX rows
+    // (hi and lo bf16 parts, columns 0-1 for q-block A, 2-3 for B; columns
+    // 4-15 stay zero).  Lane L writes key columns [4L, 4L+4): the segment that
+    // covers them is found from a mask of segment start columns (segments are
+    // in column order) and its fields are fetched by shuffle.  The value is the
+    // level unless the segment holds the end of the sequence (a short last
+    // group, or rows past the level's end); kMaskedBias on masked or empty
     // columns.
-    auto write_bias = [&](const Seg& g, float* bst) {
+    const float inv_sl2 = 1.f / p.scale_log2;
+    auto write_kx = [&](const Seg& g, uint8_t* kxs) {
       const uint32_t starts = __reduce_or_sync(0xffffffffu, g.mine ? (1u << (g.col >> 2)) : 0u);
       const int c0 = 4 * lane;
       const int owner = __popc(starts & ((2u << lane) - 1u)) - 1;   // the segment's rank = its lane
@@ -271,38 +318,43 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
       const uint32_t sg_o = __shfl_sync(0xffffffffu, g.sg, src);
       const int col_o = __shfl_sync(0xffffffffu, g.col, src);
       const int row_o = __shfl_sync(0xffffffffu, g.row, src);
-      float4 vA = make_float4(NEG_INF, NEG_INF, NEG_INF, NEG_INF), vB = vA;
-      if (c0 < g.fill) {
-        const int lv = static_cast<int>((sg_o >> 16) & 3u);
-        const uint32_t rm = (sg_o >> 18) & 3u;
-        const bool useA = rm & 1u, useB = QH == 1 ? (rm & 1u) : (rm & 2u);
-        const int gr0 = row_o + (c0 - col_o);
-        float v[4];
-        if (((gr0 + 4) << lv) <= p.N) {
+      const int lv = static_cast<int>((sg_o >> 16) & 3u);
+      const uint32_t rm = (sg_o >> 18) & 3u;
+      const int useA = rm & 1u, useB = QH == 1 ? (rm & 1u) : ((rm >> 1) & 1u);
+      const int gr0 = row_o + (c0 - col_o);
+      if (c0 >= g.fill || ((gr0 + 4) << lv) <= p.N) {
+        // empty, or four full groups of one level: a precomputed row pattern
+        const uint4 w = kxpat[c0 >= g.fill ? 16 : 4 * lv + useA + 2 * useB];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) v[i] = static_cast<float>(lv);
-        } else {
-          const int rows_l = (p.N + (1 << lv) - 1) >> lv;
+        for (int i = 0; i < 4; ++i) *reinterpret_cast<uint4*>(kxs + ((c0 + i) >> 3) * 256 + ((c0 + i) & 7) * 16) = w;
+      } else {
+        // the segment that holds the end of the sequence: short last group
+        // (fewer than 2^lv tokens) and rows past the level's end
+        const int rows_l = (p.N + (1 << lv) - 1) >> lv;
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int gr = gr0 + i;
-            float bv = NEG_INF;
-            if (gr < rows_l) {
-              const int count = min(1 << lv, p.N - (gr << lv));
-              bv = count == (1 << lv) ? static_cast<float>(lv) : log2f(static_cast<float>(count));
-            }
-            v[i] = bv;
+        for (int i = 0; i < 4; ++i) {
+          float braw = kMaskedBias;
+          const int gr = gr0 + i;
+          if (gr < rows_l) {
+            const int count = min(1 << lv, p.N - (gr << lv));
+            braw = (count == (1 << lv) ? static_cast<float>(lv) : log2f(static_cast<float>(count))) * inv_sl2;
           }
+          const float bA = useA ? braw : kMaskedBias, bB = useB ? braw : kMaskedBias;
+          const __nv_bfloat16 hA = __float2bfloat16(bA), hB = __float2bfloat16(bB);
+          const __nv_bfloat16 lA = __float2bfloat16(bA - __bfloat162float(hA));
+          const __nv_bfloat16 lB = __float2bfloat16(bB - __bfloat162float(hB));
+          const int r = c0 + i;   // key column = row of KX
+          *reinterpret_cast<uint4*>(kxs + (r >> 3) * 256 + (r & 7) * 16) = make_uint4(
+              static_cast<uint32_t>(__bfloat16_as_ushort(hA)) | (static_cast<uint32_t>(__bfloat16_as_ushort(lA)) << 16),
+              static_cast<uint32_t>(__bfloat16_as_ushort(hB)) | (static_cast<uint32_t>(__bfloat16_as_ushort(lB)) << 16),
+              0u, 0u);
         }
-        if (useA) vA = make_float4(v[0], v[1], v[2], v[3]);
-        if (useB) vB = make_float4(v[0], v[1], v[2], v[3]);
       }
-      reinterpret_cast<float4*>(bst)[lane] = vA;
-      reinterpret_cast<float4*>(bst + kTileN)[lane] = vB;
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       __syncwarp();
     };
     if (warp == 3) {
-      // ------------------------------------ producer of Q, K and bias (warp 3) ---
+      // ----------------------------------- producer of Q, K and KX (warp 3) ---
       if (n_entries > 0) {
         if (lane == 0) {
           const uint32_t qbytes = static_cast<uint32_t>((ntile0 > 0) + (ntile1 > 0)) * L::kTileBytes;
@@ -331,13 +383,10 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
           zero_rows(kst, g.fill, kTileN);
           issue(g, maps.k, &k_full[s], kst, 0, kTileN);
           k_issued = e + 1;
-          // the bias slot is free once the softmax of entry e-2 has read it
-          if (!slot_free(&b_empty[s], e)) {
-            ok = false;
-            break;
-          }
-          write_bias(g, bias + s * 2 * kTileN);
-          if (lane == 0) mbar_arrive(&b_full[s]);
+          // KX is written while the K segments are in flight; its arrival is
+          // the second of the k_full phase (made visible to the MMA by it)
+          write_kx(g, kx + s * 4096);
+          if (lane == 0) mbar_arrive(&k_full[s]);
         }
         if (!ok && lane == 0) misc[5] = 1;
         // Loads still in flight must land before the CTA can exit.
@@ -356,6 +405,8 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
         if (!ok && lane == 0) misc[5] = 1;
         const uint64_t dq0 = smem_desc(smem_addr(smem + L::kOffQ), 16, 1024);
         const uint64_t dk0 = smem_desc(sK, 16, 1024);
+        const uint64_t dqx = smem_desc_kmajor_noswizzle(smem_addr(qx), 128, 256);
+        const uint64_t dkx0 = smem_desc_kmajor_noswizzle(smem_addr(kx), 128, 256);
         constexpr uint64_t kStageStep = L::kTileBytes >> 4;
         int prev_t = 0;
         for (int e = 0; e < n_entries; ++e) {
@@ -381,6 +432,8 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
               const uint64_t off = static_cast<uint64_t>((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
               mma_ss_warp(tmem, dq + off, dk + off, kIdescS, kk > 0 ? 1u : 0u);
             }
+            // + the bias: selector columns of the row's q-block times its hi + lo parts
+            mma_ss_warp(tmem, dqx, dkx0 + s * (4096 >> 4), kIdescS, 1u);
           }
           // committed also after an error, so that the softmax keeps its place
           mma_commit_warp(&s_ready[t]);
@@ -485,7 +538,6 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
     const int r = wq * 32 + lane;
     const int row = (qtile0 + t) * kTileM + r;
     const bool row_valid = row < p.N;
-    const int rh = (QH == 2) ? (r >> 6) : 0;   // which q-block of the tile (bias half)
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     const uint32_t s_addr = lane_base;
     const uint32_t p_addr = lane_base + 128 + 64 * t;
@@ -515,22 +567,8 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
         // the S buffer is free for the next entry's S
         tc_fence_before();
         named_bar_sync(kBarSFree + t, kHandoff);
-        // the producer stops after an error, so the bias is then not waited for
-        if (!misc[5] && !mbar_wait(&b_full[st], (e / kStages) & 1)) {
-          misc[5] = 1;
-          ok = false;
-        }
-        // x = s * scale * log2e + log2(count), -inf on masked / empty columns
-        const float4* bsrc = reinterpret_cast<const float4*>(bias + st * 2 * kTileN + rh * kTileN);
-#pragma unroll
-        for (int c4 = 0; c4 < 32; ++c4) {
-          const float4 bv = bsrc[c4];
-          s[4 * c4 + 0] = fmaf(s[4 * c4 + 0], sl2, bv.x);
-          s[4 * c4 + 1] = fmaf(s[4 * c4 + 1], sl2, bv.y);
-          s[4 * c4 + 2] = fmaf(s[4 * c4 + 2], sl2, bv.z);
-          s[4 * c4 + 3] = fmaf(s[4 * c4 + 3], sl2, bv.w);
-        }
-        mbar_arrive(&b_empty[st]);   // the producer may now rewrite this bias slot
+        // s already carries the bias (raw logit units): q.k + log2(count) / (scale log2 e),
+        // and about -30000 on masked and empty columns
         float a[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) a[u] = fmaxf(s[2 * u], s[2 * u + 1]);
@@ -539,10 +577,11 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
 #pragma unroll
           for (int u = 0; u < 8; ++u) a[u] = fmax3(a[u], s[c + 2 * u], s[c + 2 * u + 1]);
         }
-        const float mx = fmaxf(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], fmax3(a[5], a[6], a[7])));
+        float mx = fmaxf(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], fmax3(a[5], a[6], a[7])));
+        if (mx < kMaskedCut) mx = NEG_INF;   // no valid column for this row in this tile
         float factor = 1.f;
-        if (mx > m_used && (m_used == NEG_INF || mx - m_used > 8.f)) {
-          factor = (m_used == NEG_INF) ? 0.f : fast_exp2(m_used - mx);
+        if (mx > m_used && (m_used == NEG_INF || (mx - m_used) * sl2 > 8.f)) {
+          factor = (m_used == NEG_INF) ? 0.f : fast_exp2((m_used - mx) * sl2);
           m_used = mx;
           l_sum *= factor;
         }
@@ -571,10 +610,10 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
           }
           tmem_st_wait();
         }
-        const float neg_m = (m_used == NEG_INF) ? 0.f : -m_used;
+        const float neg_m = (m_used == NEG_INF) ? 0.f : -m_used * sl2;
         {
           uint32_t pk[32];
-          l_sum += exp_pack_64(s, 1.f, neg_m, pk);
+          l_sum += exp_pack_64(s, sl2, neg_m, pk);
           if (!rescale) wait_pv(&pv_done_a[t]);
           tmem_st32(p_addr, reinterpret_cast<const float*>(pk));
           tmem_st_wait();
@@ -583,7 +622,7 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
         }
         {
           uint32_t pk[32];
-          l_sum += exp_pack_64(s + 64, 1.f, neg_m, pk);
+          l_sum += exp_pack_64(s + 64, sl2, neg_m, pk);
           if (!rescale) wait_pv(&pv_done_b[t]);
           tmem_st32(p_addr + 32, reinterpret_cast<const float*>(pk));
           tmem_st_wait();
@@ -628,7 +667,7 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
     }
     if (p.lse && row_valid)
       p.lse[static_cast<size_t>(bh) * p.N + row] =
-          l_sum > 0.f ? (log2f(l_sum) + m_used) * 0.69314718055994531f : NEG_INF;
+          l_sum > 0.f ? (log2f(l_sum) + m_used * sl2) * 0.69314718055994531f : NEG_INF;
   }
   tc_fence_before();
   __syncthreads();
