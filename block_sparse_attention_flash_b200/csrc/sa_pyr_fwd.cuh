@@ -13,20 +13,24 @@
 // powers of two that divide 128: they fill 128-key tiles exactly, and no
 // segment crosses a tile edge.  With block 64 the two q-blocks of a tile take
 // the union of their (j, l) pairs; a segment carries a row mask (which of
-// the two q-blocks uses it) that becomes a -inf bias for the other rows.
+// the two q-blocks uses it) that becomes a masking bias for the other rows.
 //
 // One CTA = two q-tiles with the same roles and TMEM layout as
 // sa_attn_fwd.cuh (warp 0 issues every S into the one S buffer, warps 1 and 2
 // issue the PV of q-tile 0 / 1, one softmax thread per row, P handed over in
 // two halves through named barriers), but each q-tile has its own packed key
 // tiles; the entries of the two are interleaved and each entry feeds one
-// q-tile.  Warp 3 is the producer: K and V segments arrive by TMA from one
-// tensor map per pyramid level (level 0 is the original K/V) into 2-slot
-// rings, and the producer also writes, per slot, the per-column bias (log2 of
-// the pooled token count, -inf where a column is masked or empty) for both
-// row halves, and zero-fills columns no segment covers so that masked
-// products stay finite.  The softmax works in log2 units:
-// x = s * scale * log2(e) + log2(count).
+// q-tile.  Warp 3 is the producer: K segments arrive by TMA from one tensor
+// map per pyramid level (level 0 is the original K/V) into a 2-slot ring;
+// the PV warps gather the V segments of their own next key tile the same way.
+// Columns no segment covers are zero-filled so that masked products stay
+// finite.  The bias is not added by the softmax: S gets it from one extra
+// K = 16 MMA step whose A operand (QX) selects, per q row, the pair of
+// columns of its q-block and whose B operand (KX, written per K slot by the
+// producer) holds, per key column, the bias in raw logit units as bf16
+// hi + lo: ln(count) / scale, or a large negative value where the column is
+// masked for that q-block or empty.  The softmax then works on S alone,
+// x = s * scale * log2(e), exactly as in the attention kernel.
 #pragma once
 
 #include "sa_attn_fwd.cuh"
