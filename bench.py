@@ -351,7 +351,20 @@ def run_suite(args):
             ms_a = _time(lambda: ops.sa_sparse_attn_fwd(q, k, v, wl.block, skip_in=skip_a, skip_out=skip_b,
                                                         eps=wl.eps, out=o), args.suite_reps, stream)
             flops = executed_flops(skip_a, N, wl.block, d)
-            out.append(attn_line(wl, name, ms_a, flops, {"eps": wl.eps, "skipped_next_step": int(skip_b.sum())}))
+            skipped = int(skip_b.sum())
+            ms_r = _time(lambda: ops.sa_sparse_attn_fwd(q, k, v, wl.block, skip_in=skip_a, skip_out=skip_b,
+                                                        eps=wl.eps, out=o, order="radial"), args.suite_reps, stream)
+            # diagnostic, clearly not the workload's eps: the share of (q-block, k-block)
+            # pairs that the first step marks for skipping, per visit order and eps
+            diag = {}
+            for order in ("ascending", "radial"):
+                for e in (2.0, 3.0, wl.eps):
+                    ops.sa_sparse_attn_fwd(q, k, v, wl.block, skip_in=skip_a, skip_out=skip_b, eps=e, out=o,
+                                           order=order)
+                    diag[f"{order}_eps{e:g}"] = round(int(skip_b.sum()) / skip_b.numel(), 5)
+            out.append(attn_line(wl, name, ms_a, flops, {"eps": wl.eps, "skipped_next_step": skipped,
+                                                         "radial_order_ms": round(ms_r, 3),
+                                                         "skip_share_diagnostic": diag}))
         else:
             kp, vp = ops.sa_pyramid_pool(k, v, wl.block)
             ms_p = _time(lambda: ops.sa_pyramid_pool(k, v, wl.block, k_pool=kp, v_pool=vp), args.suite_reps, stream)

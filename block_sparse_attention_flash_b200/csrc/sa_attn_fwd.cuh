@@ -3,7 +3,8 @@
 //
 // Work unit: one CTA owns two 128-row q-tiles (rows [256*pair, 256*pair+256))
 // of one (b, h) and walks the union of their kept 128-column kv tiles in
-// ascending order.  Each kv tile is loaded once by TMA and feeds both q-tiles.
+// ascending (or radial-centric) order.  Each kv tile is loaded once by TMA and
+// feeds both q-tiles.
 //
 // Roles (384 threads = 12 warps, one CTA per SM):
 //   warp 0       builds the kv-tile list from the mask / skip bytes, loads Q
@@ -73,6 +74,7 @@ struct AttnParams {
   int carry_skip;   // skip_out != NULL && skip_out != skip_in
   float scale_log2; // scale * log2(e)
   float eps_raw;    // eps / scale: the skip threshold in raw q.k units
+  int radial;       // visit kv tiles in radial-centric order (else ascending)
   __nv_bfloat16* o;
   float* lse;
 };
@@ -189,11 +191,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   if (warp == 0) {
     // ---- kv-tile list: union over the two q-tiles, per-quadrant keep bits ----
+    // Ascending: slot s is kv tile s.  Radial-centric: the CTA's 256 query
+    // rows have diagonal kv tiles qtile0 and qtile0 + 1 (distance 0); slot
+    // 2*dd is tile qtile0 - dd and slot 2*dd + 1 tile qtile0 + 1 + dd, so the
+    // slots run by ascending distance, ties by ascending tile, and a slot
+    // outside [0, n_kv_tiles) holds nothing.
+    const int n_slots = p.radial ? 2 * max(qtile0, p.n_kv_tiles - qtile0 - 1) + 2 : p.n_kv_tiles;
     int n = 0, c0 = 0, c1 = 0;
-    for (int base = 0; base < p.n_kv_tiles; base += 32) {
-      const int jt = base + lane;
+    for (int base = 0; base < n_slots; base += 32) {
+      const int sl = base + lane;
+      const int jt = !p.radial ? sl : (sl < 2 ? qtile0 + sl : ((sl & 1) ? qtile0 + 1 + (sl >> 1) : qtile0 - (sl >> 1)));
       uint32_t bits = 0;
-      if (jt < p.n_kv_tiles) {
+      if (sl < n_slots && jt >= 0 && jt < p.n_kv_tiles) {
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
 #pragma unroll

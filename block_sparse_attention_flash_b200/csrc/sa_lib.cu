@@ -239,9 +239,10 @@ sa_status sa_pyramid_pool(const void* k, const void* v, int B, int H, int N, int
 
 sa_status sa_sparse_attn_fwd(const void* q, const void* k, const void* v, int B, int H, int N, int d, int block,
                              const uint8_t* mask, int64_t mask_sb, int64_t mask_sh, int64_t mask_si,
-                             const uint8_t* skip_in, uint8_t* skip_out, float eps, float scale, void* o,
-                             float* lse, void* stream) {
+                             const uint8_t* skip_in, uint8_t* skip_out, float eps, float scale, int order,
+                             void* o, float* lse, void* stream) {
   if (B < 0 || H < 0 || N < 0) return SA_ERR_INVALID_ARG;
+  if (order != SA_ORDER_ASCENDING && order != SA_ORDER_RADIAL) return SA_ERR_INVALID_ARG;
   if (std::isnan(eps) || eps < 0.f) return SA_ERR_INVALID_ARG;
   if (std::isnan(scale) || scale < 0.f || std::isinf(scale)) return SA_ERR_INVALID_ARG;
   if (B == 0 || H == 0 || N == 0) return SA_OK;
@@ -278,6 +279,7 @@ sa_status sa_sparse_attn_fwd(const void* q, const void* k, const void* v, int B,
   p.carry_skip = skip_out != nullptr && skip_out != skip_in;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.eps_raw = std::isinf(eps) ? INFINITY : eps / scale;
+  p.radial = order == SA_ORDER_RADIAL;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
 

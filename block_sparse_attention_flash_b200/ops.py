@@ -19,6 +19,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libsparse_attn.so")
 
 SA_OK, SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_CUDA, SA_ERR_TIMEOUT = range(5)
+VISIT_ORDERS = {"ascending": 0, "radial": 1}   # sa_visit_order
 SA_MASK_TAU, SA_MASK_LEVELS = 0, 1
 
 _vp, _i32, _i64, _f32, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
@@ -33,7 +34,7 @@ _SIGNATURES = {
     "sa_radial_mask": (_i32, [_i32, _i32, _i32, _i32, _vp, _vp]),
     "sa_pyramid_pool": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
     "sa_sparse_attn_fwd": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _i64, _i64, _i64,
-                                  _vp, _vp, _f32, _f32, _vp, _vp, _vp]),
+                                  _vp, _vp, _f32, _f32, _i32, _vp, _vp, _vp]),
     "sa_pyramid_attn_fwd": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _i64, _i64, _i64,
                                    _vp, _vp, _f32, _vp, _vp, _vp]),
 }
@@ -173,8 +174,12 @@ def sa_sparse_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block:
                        mask: Optional[torch.Tensor] = None, skip_in: Optional[torch.Tensor] = None,
                        skip_out: Optional[torch.Tensor] = None, eps: float = math.inf, scale: float = 0.0,
                        out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-                       stream=None) -> torch.Tensor:
-    """Block-sparse attention forward; returns O (and fills lse / skip_out if given)."""
+                       stream=None, order: str = "ascending") -> torch.Tensor:
+    """Block-sparse attention forward; returns O (and fills lse / skip_out if given).
+
+    ``order`` ("ascending" or "radial") is the k-block visit order of the skip update."""
+    if order not in VISIT_ORDERS:
+        raise ValueError(f"order must be one of {sorted(VISIT_ORDERS)}")
     B, H, N, d = q.shape
     nb = nblocks(N, block)
     if out is None:
@@ -193,8 +198,8 @@ def sa_sparse_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block:
         _dev(q, "q", torch.bfloat16), _dev(k, "k", torch.bfloat16), _dev(v, "v", torch.bfloat16),
         B, H, N, d, block, mptr, sb, sh, si,
         _opt(skip_in, "skip_in", torch.uint8), _opt(skip_out, "skip_out", torch.uint8),
-        float(eps), float(scale), _dev(out, "out", torch.bfloat16), _opt(lse, "lse", torch.float32),
-        _stream(stream))
+        float(eps), float(scale), VISIT_ORDERS[order], _dev(out, "out", torch.bfloat16),
+        _opt(lse, "lse", torch.float32), _stream(stream))
     _check(st, "sa_sparse_attn_fwd")
     return out
 

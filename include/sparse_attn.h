@@ -55,6 +55,13 @@ typedef enum {
   SA_ERR_TIMEOUT = 4        /* a device-side bounded wait ran out           */
 } sa_status;
 
+/* Order in which sa_sparse_attn_fwd visits the kept k-blocks of a q-block
+ * (it decides only the skip update; the output is the same up to rounding). */
+typedef enum {
+  SA_ORDER_ASCENDING = 0,   /* ascending j                                   */
+  SA_ORDER_RADIAL = 1       /* radial-centric, see sa_sparse_attn_fwd         */
+} sa_visit_order;
+
 enum { SA_MASK_TAU = 0, SA_MASK_LEVELS = 1 };
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -183,7 +190,7 @@ SA_API sa_status sa_pyramid_pool(const void* k, const void* v, int B, int H, int
  * == 0, where s_rc = scale * q_r . k_c.  LSE_r = ln sum_c exp(s_rc).  A row
  * with no visited block gets O = 0 and LSE = -inf.
  * Skip update (only when skip_out != NULL): visited k-blocks are taken in
- * ascending j; block j (not the first visited) gets skip_out = 1 iff
+ * the visit order; block j (not the first visited) gets skip_out = 1 iff
  * max_c s_rc over block j < (running max of row r over the blocks visited
  * before j) - eps for every valid row r of the q-block.  Block j still
  * contributes to this call's O.  Every other byte of the row is written as
@@ -200,6 +207,15 @@ SA_API sa_status sa_pyramid_pool(const void* k, const void* v, int B, int H, int
  *   eps           skip threshold in natural-log logit units (>= 0; +inf
  *                 never skips).
  *   scale         logit scale; 0 selects 1/sqrt(d).
+ *   order         SA_ORDER_ASCENDING, or SA_ORDER_RADIAL: the radial-centric
+ *                 ordering of the LiteAttention write-up (section 5; section
+ *                 10 expects 10-20 % more skips from it), read as follows.
+ *                 Keys are cut into tiles of 128, query rows into bands of
+ *                 256; the k-blocks of q-block i are visited by ascending
+ *                 distance of their tile from the two diagonal tiles of the
+ *                 band holding row i*block (distance 0 for both), ties by
+ *                 ascending tile, ascending j inside a tile.  Any other
+ *                 value is SA_ERR_INVALID_ARG.
  *   o             bf16 [B,H,N,d] device, written for every valid row.
  *   lse           NULL or fp32 [B,H,N] device.
  * Limits: d in {64,128}, block in {64,128}, ceil(N/128) <= 4096, B*H <= 65535.
@@ -207,7 +223,7 @@ SA_API sa_status sa_pyramid_pool(const void* k, const void* v, int B, int H, int
 SA_API sa_status sa_sparse_attn_fwd(const void* q, const void* k, const void* v,
                              int B, int H, int N, int d, int block,
                              const uint8_t* mask, int64_t mask_sb, int64_t mask_sh, int64_t mask_si,
-                             const uint8_t* skip_in, uint8_t* skip_out, float eps, float scale,
+                             const uint8_t* skip_in, uint8_t* skip_out, float eps, float scale, int order,
                              void* o, float* lse, void* stream);
 
 /*

@@ -25,10 +25,10 @@ no code with the CUDA library and never imports it.
 from .attention import masked_attention, dense_attention, block_mask_to_token_mask
 from .masks import block_means, block_scores, tau_mask, level_map, radial_mask
 from .pyramid import pyramid_pool, pyramid_attention
-from .lite import lite_step, lite_chain
+from .lite import lite_step, lite_chain, visit_order
 
 __all__ = [
     "masked_attention", "dense_attention", "block_mask_to_token_mask",
     "block_means", "block_scores", "tau_mask", "level_map", "radial_mask",
-    "pyramid_pool", "pyramid_attention", "lite_step", "lite_chain",
+    "pyramid_pool", "pyramid_attention", "lite_step", "lite_chain", "visit_order",
 ]

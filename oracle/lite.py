@@ -17,6 +17,14 @@ Readings (stated because the page gives prose only):
   for every valid row r of the q-block; eps is in natural-log logit units;
 * the output of the detecting step still includes block j; the bit takes
   effect from the next step: skip_out = skip_in | new_bits.
+* radial-centric order (section 5 names it, section 10 expects 10-20 % more
+  sparsity from it; neither defines it): the key axis is cut into tiles of
+  128 tokens and the query axis into bands of 256 rows; the k-blocks of
+  q-block i are visited by ascending distance of their tile from the band's
+  two diagonal tiles (distance 0 for both), ties by ascending tile index, and
+  in ascending j inside a tile.  The band holding q-block i is the one that
+  holds its first row.  Only the order in which blocks are visited changes;
+  the output is the same up to rounding.
 """
 from __future__ import annotations
 
@@ -27,7 +35,29 @@ import numpy as np
 from .attention import _f64, _nblocks, _mask4
 
 
-def lite_qblock(qh, kh, vh, block, keep_row, i, eps, scale):
+RADIAL_TILE = 128     # keys per tile of the radial-centric order
+RADIAL_BAND = 256     # query rows per band of the radial-centric order
+
+
+def visit_order(i, nkb, block, order="ascending"):
+    """k-block indices 0..nkb-1 in the order q-block i visits them."""
+    if order == "ascending":
+        return list(range(nkb))
+    if order != "radial":
+        raise ValueError(f"unknown visit order {order!r}")
+    per_tile = RADIAL_TILE // block
+    n_tiles = -(-nkb // per_tile)
+    c = (i * block // RADIAL_BAND) * (RADIAL_BAND // RADIAL_TILE)   # first diagonal tile of the band
+    last = c + RADIAL_BAND // RADIAL_TILE - 1                      # last diagonal tile
+
+    def dist(t):
+        return c - t if t < c else (t - last if t > last else 0)
+
+    tiles = sorted(range(n_tiles), key=lambda t: (dist(t), t))
+    return [j for t in tiles for j in range(t * per_tile, min(nkb, (t + 1) * per_tile))]
+
+
+def lite_qblock(qh, kh, vh, block, keep_row, i, eps, scale, order="ascending"):
     """(O rows, LSE rows, new-bit row, margin row) for one q-block.
 
     margin[j] = max_r (l_r(j) - m_r + eps) for tested blocks (NaN elsewhere);
@@ -37,7 +67,7 @@ def lite_qblock(qh, kh, vh, block, keep_row, i, eps, scale):
     d = vh.shape[1]
     nkb = keep_row.shape[0]
     r0, r1 = i * block, min(N, (i + 1) * block)
-    visited = np.nonzero(keep_row)[0]
+    visited = np.array([j for j in visit_order(i, nkb, block, order) if keep_row[j]], dtype=np.int64)
     new = np.zeros(nkb, dtype=np.uint8)
     margin = np.full(nkb, np.nan)
     if visited.size == 0:
@@ -63,10 +93,11 @@ def lite_qblock(qh, kh, vh, block, keep_row, i, eps, scale):
     return (e / z) @ vh[c], (m + np.log(z))[:, 0], new, margin
 
 
-def lite_step(q, k, v, block, mask=None, skip_in=None, eps=10.0, scale=None, qblocks=None):
+def lite_step(q, k, v, block, mask=None, skip_in=None, eps=10.0, scale=None, qblocks=None,
+              order="ascending"):
     """One denoising step of block attention with the LiteAttention skip update.
 
-    Effective keep = mask & ~skip_in.  Returns (O, LSE, skip_out, margin) with
+    Effective keep = mask & ~skip_in; ``order`` is "ascending" or "radial".  Returns (O, LSE, skip_out, margin) with
     skip_out = skip_in | new bits, or a dict {(b,h,i): (O, LSE, skip_out_row,
     margin_row)} when ``qblocks`` is given.
     """
@@ -83,7 +114,7 @@ def lite_step(q, k, v, block, mask=None, skip_in=None, eps=10.0, scale=None, qbl
 
     def one(b, h, i):
         keep = (m4[b, h, i] != 0) & (s4[b, h, i] == 0)
-        o, lse, new, mg = lite_qblock(q[b, h], k[b, h], v[b, h], block, keep, i, eps, scale)
+        o, lse, new, mg = lite_qblock(q[b, h], k[b, h], v[b, h], block, keep, i, eps, scale, order)
         return o, lse, (s4[b, h, i] | new).astype(np.uint8), mg
 
     if qblocks is not None:
@@ -100,7 +131,7 @@ def lite_step(q, k, v, block, mask=None, skip_in=None, eps=10.0, scale=None, qbl
     return O, L, S, M
 
 
-def lite_chain(steps_inputs, block, eps, mask=None, skip0=None, feed=None):
+def lite_chain(steps_inputs, block, eps, mask=None, skip0=None, feed=None, order="ascending"):
     """Run lite_step over a sequence of (q, k, v) denoising inputs.
 
     ``feed(s, skip_out)`` may replace the skip mask handed to step s+1 (used
@@ -110,7 +141,7 @@ def lite_chain(steps_inputs, block, eps, mask=None, skip0=None, feed=None):
     out = []
     skip = skip0
     for s, (q, k, v) in enumerate(steps_inputs):
-        O, L, S, M = lite_step(q, k, v, block, mask, skip, eps)
+        O, L, S, M = lite_step(q, k, v, block, mask, skip, eps, order=order)
         out.append((O, L, S, M))
         skip = S if feed is None else feed(s, S)
     return out

@@ -54,11 +54,11 @@ def test_workspace_size(lib):
 
 def _attn(lib, **kw):
     a = dict(q=16, k=16, v=16, B=1, H=1, N=256, d=128, block=128, mask=None, sb=0, sh=0, si=0,
-             skip_in=None, skip_out=None, eps=math.inf, scale=0.0, o=16, lse=None, stream=None)
+             skip_in=None, skip_out=None, eps=math.inf, scale=0.0, order=0, o=16, lse=None, stream=None)
     a.update(kw)
     return lib.sa_sparse_attn_fwd(a["q"], a["k"], a["v"], a["B"], a["H"], a["N"], a["d"], a["block"],
                                   a["mask"], a["sb"], a["sh"], a["si"], a["skip_in"], a["skip_out"],
-                                  a["eps"], a["scale"], a["o"], a["lse"], a["stream"])
+                                  a["eps"], a["scale"], a["order"], a["o"], a["lse"], a["stream"])
 
 
 def test_attention_argument_validation(lib):
@@ -68,6 +68,8 @@ def test_attention_argument_validation(lib):
     assert _attn(lib, k=24) == ops.SA_ERR_INVALID_ARG          # not 16-byte aligned
     assert _attn(lib, eps=float("nan")) == ops.SA_ERR_INVALID_ARG
     assert _attn(lib, eps=-1.0) == ops.SA_ERR_INVALID_ARG
+    assert _attn(lib, order=2) == ops.SA_ERR_INVALID_ARG
+    assert _attn(lib, order=-1) == ops.SA_ERR_INVALID_ARG
     assert _attn(lib, scale=-0.5) == ops.SA_ERR_INVALID_ARG
     assert _attn(lib, N=128 * 4097) == ops.SA_ERR_UNSUPPORTED
     assert _attn(lib, B=256, H=256) == ops.SA_ERR_UNSUPPORTED

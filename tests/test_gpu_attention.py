@@ -20,14 +20,15 @@ def _lib():
     ops.sa_get_device_status()
 
 
-def run_attn(q, k, v, block, mask=None, skip_in=None, skip_out=None, eps=math.inf, with_lse=True):
+def run_attn(q, k, v, block, mask=None, skip_in=None, skip_out=None, eps=math.inf, with_lse=True,
+             order="ascending"):
     qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
     B, H, N, d = q.shape
     # poison the output so unwritten rows show up
     out = torch.full_like(qd, float("nan"))
     lse = torch.full((B, H, N), float("nan"), device="cuda") if with_lse else None
     ops.sa_sparse_attn_fwd(qd, kd, vd, block, mask=None if mask is None else mask.cuda(),
-                           skip_in=skip_in, skip_out=skip_out, eps=eps, out=out, lse=lse)
+                           skip_in=skip_in, skip_out=skip_out, eps=eps, out=out, lse=lse, order=order)
     ops.sa_get_device_status()
     return out.cpu(), (lse.cpu() if lse is not None else None)
 
@@ -94,7 +95,7 @@ def test_radial_mask_broadcast_over_heads():
 
 # ------------------------------------------------------------------ skip ---
 
-def _skip_run(q, k, v, block, mask, skip_in, eps, alias=False):
+def _skip_run(q, k, v, block, mask, skip_in, eps, alias=False, order="ascending"):
     B, H, N, d = q.shape
     nb = -(-N // block)
     si = skip_in.cuda() if skip_in is not None else None
@@ -102,14 +103,14 @@ def _skip_run(q, k, v, block, mask, skip_in, eps, alias=False):
         so = si
     else:
         so = torch.full((B, H, nb, nb), 77, dtype=torch.uint8, device="cuda")
-    O, L = run_attn(q, k, v, block, mask, skip_in=si, skip_out=so, eps=eps)
+    O, L = run_attn(q, k, v, block, mask, skip_in=si, skip_out=so, eps=eps, order=order)
     return O, L, so.cpu()
 
 
-def _check_skip_step(q, k, v, block, mask, skip_in, eps, alias=False):
-    O, L, S = _skip_run(q, k, v, block, mask, skip_in, eps, alias)
+def _check_skip_step(q, k, v, block, mask, skip_in, eps, alias=False, order="ascending"):
+    O, L, S = _skip_run(q, k, v, block, mask, skip_in, eps, alias, order)
     Or, Lr, Sr, M = lite_step(q, k, v, block, None if mask is None else mask.numpy(),
-                              None if skip_in is None else skip_in.numpy(), eps)
+                              None if skip_in is None else skip_in.numpy(), eps, order=order)
     check_o(O, Or, f"skip step eps={eps}")
     check_lse(L, Lr, f"skip step eps={eps}")
     nflag = check_bits(S, Sr, skip_flags(M), f"skip bits eps={eps}")
@@ -173,3 +174,51 @@ def test_skip_in_blocks_are_not_visited():
     check_o(O, Or, "skip_in honoured")
     check_lse(L, Lr, "skip_in honoured")
     assert torch.equal(S, skip_in)                     # eps = inf: carry only
+
+
+# ------------------------------------------------- radial-centric visit order ---
+
+@pytest.mark.parametrize("block", [64, 128])
+def test_radial_order_skip_step(block):
+    """Radial-centric order on an RFF grid of 24 kv tiles (12 q-tile pairs):
+    O, LSE and skip bits against the oracle walking the same order."""
+    wl = inputs.Workload("r", 1, 3, 128, 8, 16, 24, block, "lite", seed=45, sigma_s=2.0, sigma_t=1.5)
+    q, k, v = inputs.rff_qkv(wl)
+    S, Sr, _ = _check_skip_step(q, k, v, block, None, None, eps=1.0, order="radial")
+    _, Sa, _ = _check_skip_step(q, k, v, block, None, None, eps=1.0)
+    assert Sr.sum() > 0 and not np.array_equal(Sr, Sa)   # the order changes the decisions
+
+
+@pytest.mark.parametrize("block", [64, 128])
+def test_radial_order_ragged_masked_chain(block):
+    """Ragged tail (an odd q-tile count, a partial last tile), a random mask and
+    a two-step teacher-forced chain with skip_out aliasing skip_in."""
+    wl = inputs.Workload("rc", 1, 2, 128, 5, 13, 17, block, "lite", seed=46, sigma_s=2.0, sigma_t=1.5)
+    steps = list(inputs.lite_chain_inputs(wl, 2))
+    nb = wl.nblocks
+    mask = inputs.bernoulli_block_mask(1, wl.H, nb, nb, 0.8, seed=47)
+    skip = None
+    for s, (q, k, v) in enumerate(steps):
+        S, Sr, _ = _check_skip_step(q, k, v, block, mask, skip, eps=1.2, alias=skip is not None, order="radial")
+        skip = torch.from_numpy(np.ascontiguousarray(Sr))
+    assert int(skip.sum()) > 0
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_radial_order_reaches_the_row_max_first(d):
+    """Keys of k-blocks 4 and 5 give logit +6, the rest -6: q-blocks 4-7 skip
+    every -6 block under the radial order, only blocks 6 and 7 in ascending order."""
+    block, nb = 64, 8
+    N = block * nb
+    a = math.sqrt(6.0 * math.sqrt(d))
+    u = torch.zeros(d)
+    u[3] = 1.0
+    q = (a * u).repeat(N, 1).view(1, 1, N, d).to(torch.bfloat16)
+    k = (-a * u).repeat(N, 1)
+    k[4 * block:6 * block] = a * u
+    k = k.view(1, 1, N, d).to(torch.bfloat16)
+    v = torch.randn(1, 1, N, d, generator=torch.Generator().manual_seed(2)).to(torch.bfloat16)
+    S, _, _ = _check_skip_step(q, k, v, block, None, None, eps=10.0, order="radial")
+    assert S[0, 0, 4].tolist() == [1, 1, 1, 1, 0, 0, 1, 1]
+    S, _, _ = _check_skip_step(q, k, v, block, None, None, eps=10.0)
+    assert S[0, 0, 4].tolist() == [0, 0, 0, 0, 0, 0, 1, 1]

@@ -6,7 +6,7 @@ import torch
 
 from block_sparse_attention_flash_b200 import inputs
 from oracle import (masked_attention, dense_attention, pyramid_pool, pyramid_attention,
-                    lite_step, lite_chain)
+                    lite_step, lite_chain, visit_order)
 
 
 # ---------------------------------------------------------------- pyramid ---
@@ -175,3 +175,74 @@ def test_running_max_before_or_after_j_is_equivalent():
             bit = j > 0 and bool(np.all(loc < after - 1.2))
             assert bit == bool(S[0, 0, i, j])
             run = after
+
+
+# ------------------------------------------------------ radial-centric order ---
+
+def test_radial_visit_order_hand_listed():
+    """Orders listed by hand from the reading: 128-key tiles, 256-row bands,
+    ascending distance from the band's two diagonal tiles, ties by tile index."""
+    assert visit_order(2, 8, 128, "radial") == [2, 3, 1, 4, 0, 5, 6, 7]
+    assert visit_order(3, 8, 128, "radial") == [2, 3, 1, 4, 0, 5, 6, 7]
+    assert visit_order(0, 5, 128, "radial") == [0, 1, 2, 3, 4]
+    assert visit_order(6, 7, 128, "radial") == [6, 5, 4, 3, 2, 1, 0]
+    assert visit_order(5, 12, 64, "radial") == [4, 5, 6, 7, 2, 3, 8, 9, 0, 1, 10, 11]
+    assert visit_order(9, 11, 64, "radial") == [8, 9, 10, 6, 7, 4, 5, 2, 3, 0, 1]
+    assert visit_order(1, 4, 64, "ascending") == [0, 1, 2, 3]
+    for nkb, block in ((13, 64), (9, 128), (1, 64)):
+        for i in range(nkb):
+            assert sorted(visit_order(i, nkb, block, "radial")) == list(range(nkb))
+
+
+def test_radial_order_changes_no_output_and_keeps_suppression():
+    """The order decides only which blocks are skipped next step: with eps = inf
+    the step equals block attention, and with a finite eps every new bit still
+    marks a block whose probabilities are all <= exp(-eps)."""
+    wl = inputs.Workload("t", 1, 2, 8, 8, 8, 64, 16, "lite", seed=81, sigma_s=2.0)
+    q, k, v = inputs.rff_qkv(wl)
+    block, nb = wl.block, wl.nblocks
+    m = inputs.bernoulli_block_mask(wl.B, wl.H, nb, nb, 0.7, 6)
+    O, L, S, _ = lite_step(q, k, v, block, m, None, eps=math.inf, order="radial")
+    O2, L2 = masked_attention(q, k, v, block, m)
+    assert S.sum() == 0 and np.max(np.abs(O - O2)) < 1e-12 and np.max(np.abs(L - L2)) < 1e-12
+    eps = 0.5
+    _, _, S, _ = lite_step(q, k, v, block, None, None, eps=eps, order="radial")
+    assert S.sum() > 0
+    qd, kd = q.double().numpy(), k.double().numpy()
+    for h in range(wl.H):
+        s = qd[0, h] @ kd[0, h].T / math.sqrt(wl.d)
+        p = np.exp(s - s.max(axis=1, keepdims=True))
+        p /= p.sum(axis=1, keepdims=True)
+        for i, j in zip(*np.nonzero(S[0, h])):
+            assert p[i * block:(i + 1) * block, j * block:(j + 1) * block].max() <= math.exp(-eps)
+
+
+def test_radial_order_reaches_the_row_max_first():
+    """Keys of k-blocks 4 and 5 give logit +6, all others -6; q-block 4 sits in
+    the band whose diagonal tiles hold k-blocks 4-7.  Ascending order meets
+    blocks 0-3 before any +6 block and can skip only 6 and 7; radial order
+    starts at block 4 and skips every -6 block."""
+    d, block, nb = 16, 64, 8
+    a = b = math.sqrt(6.0 * math.sqrt(d))
+    u = np.zeros(d)
+    u[3] = 1.0
+    N = block * nb
+    q = np.tile(a * u, (N, 1))
+    k = np.tile(-b * u, (N, 1))
+    k[4 * block:6 * block] = b * u
+    v = np.random.default_rng(1).normal(size=(N, d))
+    q, k, v = q[None, None], k[None, None], v[None, None]
+    _, _, Sa, _ = lite_step(q, k, v, block, None, None, eps=10.0)
+    _, _, Sr, _ = lite_step(q, k, v, block, None, None, eps=10.0, order="radial")
+    assert Sa[0, 0, 4].tolist() == [0, 0, 0, 0, 0, 0, 1, 1]
+    assert Sr[0, 0, 4].tolist() == [1, 1, 1, 1, 0, 0, 1, 1]
+    # the skip bits of a radial step equal a re-walk of the hand-listed order
+    s = q[0, 0] @ k[0, 0].T / math.sqrt(d)
+    for i in range(nb):
+        rows = s[i * block:(i + 1) * block]
+        order = [4, 5, 6, 7, 2, 3, 0, 1] if 4 <= i < 8 else [0, 1, 2, 3, 4, 5, 6, 7]
+        run = np.full(block, -np.inf)
+        for n_vis, j in enumerate(order):
+            loc = rows[:, j * block:(j + 1) * block].max(axis=1)
+            assert bool(n_vis > 0 and np.all(loc < run - 10.0)) == bool(Sr[0, 0, i, j])
+            run = np.maximum(run, loc)
