@@ -12,7 +12,10 @@ from the pages' descriptions of the methods:
   spatio-temporal decay and static-mask paragraphs;
 * "浙江大学突破视频AI瓶颈:金字塔方法提升视频AI效率10倍" (PSA, arXiv
   2512.04025), the pyramid KV, multi-level mask and distribution-consistent
-  attention paragraphs.
+  attention paragraphs;
+* the backward pass (gradients through the masked attention, needed by the
+  Radial Attention write-up's LoRA length extension) is the derivative of
+  the forward definition, stated in ``oracle/backward.py``.
 
 The pages give prose only; the concrete rules (tau-mass selection, radial
 window S / 2^floor(log2 dt), skip test with epsilon in natural-log logits,
@@ -26,9 +29,11 @@ from .attention import masked_attention, dense_attention, block_mask_to_token_ma
 from .masks import block_means, block_scores, tau_mask, level_map, radial_mask
 from .pyramid import pyramid_pool, pyramid_attention
 from .lite import lite_step, lite_chain, visit_order
+from .backward import masked_attention_bwd, masked_attention_bwd_rows
 
 __all__ = [
     "masked_attention", "dense_attention", "block_mask_to_token_mask",
     "block_means", "block_scores", "tau_mask", "level_map", "radial_mask",
     "pyramid_pool", "pyramid_attention", "lite_step", "lite_chain", "visit_order",
+    "masked_attention_bwd", "masked_attention_bwd_rows",
 ]
