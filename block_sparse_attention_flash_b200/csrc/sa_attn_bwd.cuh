@@ -1,0 +1,627 @@
+// sa_attn_bwd.cuh — backward pass of block-sparse attention for sm_100a.
+//
+// Gradients of O = softmax(scale * Q K^T restricted to the kept blocks) V with
+// respect to Q, K and V, given dO and the forward's LSE (needed by the LoRA
+// length extension of the Radial Attention write-up, "MIT实验室推出Radial
+// Attention", training-cost paragraph; the formulas are the derivative of the
+// forward definition):
+//   P = exp(S - LSE) on kept columns, D_r = dO_r . O_r,
+//   dV = P^T dO,  dS = P * (dO V^T - D),  dK = scale dS^T Q,  dQ = scale dS K.
+//
+// Three launches, no atomics (the result does not depend on scheduling):
+//   bwd_delta_kernel   D_r = dO_r . O_r (HBM-bound: reads O and dO once);
+//   bwd_dkdv_kernel    one CTA per 128-key kv tile: walks the q-tiles that
+//                      keep any of its blocks, S^T = K Q^T and dP^T = V dO^T
+//                      into TMEM, P^T and dS^T packed to bf16 in place, then
+//                      dV += P^T dO and dK += dS^T Q with the A operand in TMEM;
+//   bwd_dq_kernel      one CTA per 128-row q-tile: walks its kept kv tiles,
+//                      S = Q K^T and dP = dO V^T, dS packed in place, then
+//                      dQ += dS K with the A operand in TMEM.
+// Every MMA is one of the two forms of the forward kernel: both operands
+// K-major in shared memory (S, dP), or A from TMEM and B MN-major in shared
+// memory (dV, dK, dQ).  The same 128 x D tile, as TMA writes it, serves as a
+// K-major B operand (Q in S^T, K in S) and as an MN-major B operand (Q in dK,
+// dO in dV, K in dQ).
+//
+// Roles (192 threads = 6 warps, one CTA per SM for the TMEM it holds):
+//   warps 0-3   one thread per row of the CTA's tile (key row in dK/dV, query
+//               row in dQ): P and dS from the TMEM rows, the epilogue;
+//   warp 4      builds the tile list from the mask, issues the TMA loads
+//               (2-stage ring) and stages the per-query LSE / D vectors;
+//   warp 5      allocates TMEM and issues every MMA (warp-wide, one elected lane).
+// Hand-offs: tcgen05.commit to mbarriers from the MMA warp; one named barrier
+// (warps 0-3 + warp 5) when P / dS are in TMEM.  Every party runs the full,
+// list-determined sequence of syncs, also after an error (skipping only its
+// loads and MMAs), and every mbarrier wait is bounded.
+#pragma once
+
+#include "sa_attn_fwd.cuh"
+
+namespace sa {
+
+constexpr int kBwdWarps = 6;
+constexpr int kBwdThreads = kBwdWarps * 32;
+constexpr int kBwdLoadWarp = 4;
+constexpr int kBwdMmaWarp = 5;
+constexpr int kBarBwdP = 1;         // P / dS packed in TMEM: warps 0-3 <-> MMA warp
+constexpr int kBwdHandoff = 160;
+
+struct BwdParams {
+  int B, H, N;
+  int nb;             // blocks per sequence
+  int n_tiles;        // ceil(N / 128)
+  const uint8_t* mask;
+  long long msb, msh, msi;
+  const float* lse;   // [B,H,N] natural-log LSE of the forward
+  const float* delta; // [B,H,N] D_r = dO_r . O_r
+  float scale;        // logit scale
+  float scale_log2;   // scale * log2(e)
+  __nv_bfloat16* dq;
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+};
+
+// D_r = sum_a dO[r,a] O[r,a] in fp32; D / 8 threads per row, 16-byte loads.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_delta_kernel(const __nv_bfloat16* __restrict__ o,
+                                                        const __nv_bfloat16* __restrict__ dout,
+                                                        float* __restrict__ delta, long long rows) {
+  constexpr int kTpr = D / 8;                       // threads per row
+  constexpr int kRowsPerBlock = 256 / kTpr;
+  const int sub = threadIdx.x % kTpr;
+  for (long long r = static_cast<long long>(blockIdx.x) * kRowsPerBlock + threadIdx.x / kTpr; r < rows;
+       r += static_cast<long long>(gridDim.x) * kRowsPerBlock) {
+    const uint4 a = reinterpret_cast<const uint4*>(o + r * D)[sub];
+    const uint4 g = reinterpret_cast<const uint4*>(dout + r * D)[sub];
+    const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+    const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&g);
+    float acc = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 af = __bfloat1622float2(a2[i]), gf = __bfloat1622float2(g2[i]);
+      acc = fmaf(af.x, gf.x, acc);
+      acc = fmaf(af.y, gf.y, acc);
+    }
+#pragma unroll
+    for (int off = kTpr / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (sub == 0) delta[r] = acc;
+  }
+}
+
+template <int D>
+struct BwdSmem {
+  static constexpr int kTileBytes = kTileM * D * 2;
+  // dK/dV kernel: K, V of the CTA's kv tile, then a ring of Q / dO tiles with
+  // their [lse2 | D] vectors (2 x 128 fp32 per stage).
+  // dQ kernel: Q, dO of the CTA's q-tile, then a ring of K / V tiles.
+  static constexpr int kOffFix0 = 0;
+  static constexpr int kOffFix1 = kTileBytes;
+  static constexpr int kOffRing0 = 2 * kTileBytes;                      // [stage]
+  static constexpr int kOffRing1 = kOffRing0 + kStages * kTileBytes;    // [stage]
+  static constexpr int kOffVec = kOffRing1 + kStages * kTileBytes;      // [stage][2][128] f32
+  static constexpr int kOffList = kOffVec + kStages * 2 * 128 * 4;
+  // fix_full, ring_full[2], ring_empty[2], s_ready, mma_done
+  static constexpr int kNumBars = 1 + 2 * kStages + 2;
+  static constexpr int kOffBar = kOffList + kMaxKvTiles * 4;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kBytes = kOffMisc + 64;
+  static constexpr int kAlloc = kBytes + 1024;
+};
+
+// p = 2^(s * sl2 - l2) on kept columns (0 elsewhere), ds = p * (dp - dl), for
+// 32 columns; both packed to bf16 pairs.  l2 / dl are per column (dK/dV
+// kernel, pointers into shared memory) or per row (dQ kernel, l2s / dls).
+template <bool kPerColumn>
+__device__ __forceinline__ void grad_chunk(const float* sv, const float* dp, float sl2, const float* l2,
+                                           const float* dl, float l2s, float dls, uint32_t keep_bits,
+                                           uint32_t* pk, uint32_t* dk) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    float x0, x1, d0, d1;
+    if (kPerColumn) {
+      const float2 l = reinterpret_cast<const float2*>(l2)[i];
+      const float2 g = reinterpret_cast<const float2*>(dl)[i];
+      x0 = fmaf(sv[2 * i], sl2, -l.x);
+      x1 = fmaf(sv[2 * i + 1], sl2, -l.y);
+      d0 = g.x;
+      d1 = g.y;
+    } else {
+      x0 = fmaf(sv[2 * i], sl2, -l2s);
+      x1 = fmaf(sv[2 * i + 1], sl2, -l2s);
+      d0 = dls;
+      d1 = dls;
+    }
+    const float p0 = ((keep_bits >> (2 * i)) & 1u) ? fast_exp2(x0) : 0.f;
+    const float p1 = ((keep_bits >> (2 * i + 1)) & 1u) ? fast_exp2(x1) : 0.f;
+    pk[i] = pack_bf16x2(p0, p1);
+    dk[i] = pack_bf16x2(p0 * (dp[2 * i] - d0), p1 * (dp[2 * i + 1] - d1));
+  }
+}
+
+// One thread's fp32 TMEM row (columns [taddr, taddr + D)) times `mul`, to
+// bf16 at dst (16-byte aligned) when `store`, or zeros when `zero`.  Called by
+// whole warps with warp-uniform `zero` (the TMEM loads are warp-collective).
+template <int D>
+__device__ __forceinline__ void store_row(uint32_t taddr, float mul, __nv_bfloat16* dst, bool zero, bool store) {
+#pragma unroll
+  for (int c = 0; c < D / 32; ++c) {
+    float v[32];
+    if (zero) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = 0.f;
+    } else {
+      tmem_ld32(taddr + 32 * c, v);
+    }
+    if (!store) continue;
+    uint4* out = reinterpret_cast<uint4*>(dst + 32 * c);
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) {
+      uint4 w;
+      w.x = pack_bf16x2(v[q4 * 8 + 0] * mul, v[q4 * 8 + 1] * mul);
+      w.y = pack_bf16x2(v[q4 * 8 + 2] * mul, v[q4 * 8 + 3] * mul);
+      w.z = pack_bf16x2(v[q4 * 8 + 4] * mul, v[q4 * 8 + 5] * mul);
+      w.w = pack_bf16x2(v[q4 * 8 + 6] * mul, v[q4 * 8 + 7] * mul);
+      out[q4] = w;
+    }
+  }
+}
+
+// ------------------------------------------------------------ dK / dV ---
+// CTA = (kv tile jt, head bh).  TMEM columns: dV [0, D), dK [D, 2D),
+// S^T [2D, 2D + 128) (P^T packed to bf16 over its first 64 columns),
+// dP^T [2D + 128, 2D + 256) (dS^T packed over its first 64 columns).
+template <int D, int BLK>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                    const BwdParams p) {
+  using L = BwdSmem<D>;
+  constexpr int QH = kTileM / BLK;  // q-blocks per q-tile
+  constexpr int KH = kTileN / BLK;  // k-blocks per kv tile
+  constexpr uint32_t kIdescS = idesc_bf16_f32(kTileN, kTileM, false);
+  constexpr uint32_t kIdescG = idesc_bf16_f32(kTileN, D, true);
+  constexpr int kHalfBytes = kTileM * 128;  // one 64-column slab of a tile
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint32_t* list = reinterpret_cast<uint32_t*>(smem + L::kOffList);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
+  uint64_t* kv_full = bars;
+  uint64_t* q_full = bars + 1;
+  uint64_t* q_empty = q_full + kStages;
+  uint64_t* s_ready = q_empty + kStages;
+  uint64_t* mma_done = s_ready + 1;
+  volatile int* misc = reinterpret_cast<volatile int*>(smem + L::kOffMisc);
+  // misc[0] TMEM base, [1] list length, [2] abort flag
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int jt = blockIdx.x;
+  const int bh = blockIdx.y;
+  const int b = bh / p.H, h = bh - (bh / p.H) * p.H;
+  auto aborted = [&]() -> bool { return misc[2] != 0; };
+
+  if (warp == kBwdLoadWarp) {
+    // ---- q-tile list: the q-tiles keeping any (q-block, k-block) quadrant ----
+    int n = 0;
+    for (int base = 0; base < p.n_tiles; base += 32) {
+      const int it = base + lane;
+      uint32_t bits = 0;
+      if (it < p.n_tiles) {
+#pragma unroll
+        for (int qh = 0; qh < QH; ++qh) {
+          const int qb = it * QH + qh;
+          if (qb >= p.nb) continue;
+#pragma unroll
+          for (int kh = 0; kh < KH; ++kh) {
+            const int kb = jt * KH + kh;
+            if (kb >= p.nb) continue;
+            const uint8_t keep = p.mask ? p.mask[b * p.msb + h * p.msh + qb * p.msi + kb] : uint8_t(1);
+            if (keep) bits |= (BLK == 128 ? 0xFu : (1u << (qh * 2 + kh)));
+          }
+        }
+      }
+      const unsigned ball = __ballot_sync(0xffffffffu, bits != 0);
+      if (bits) list[n + __popc(ball & ((1u << lane) - 1u))] = static_cast<uint32_t>(it) | (bits << 16);
+      n += __popc(ball);
+    }
+    if (lane == 0) {
+      misc[1] = n;
+      misc[2] = 0;
+      for (int i = 0; i < L::kNumBars; ++i) mbar_init(&bars[i], (&bars[i] >= q_full && &bars[i] < q_empty) ? 2u : 1u);
+      fence_mbar_init();
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmDO);
+    }
+  } else if (warp == kBwdMmaWarp) {
+    tmem_alloc(const_cast<uint32_t*>(reinterpret_cast<volatile uint32_t*>(misc)), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  const uint32_t tmem = static_cast<uint32_t>(misc[0]);
+  const int n_list = misc[1];
+  const uint32_t tm_dv = tmem, tm_dk = tmem + D, tm_s = tmem + 2 * D, tm_dp = tmem + 2 * D + 128;
+
+  if (warp == kBwdLoadWarp) {
+    // ------------------------------------------------------------- loads ---
+    if (n_list > 0) {
+      if (lane == 0) {
+        mbar_arrive_expect_tx(kv_full, 2 * L::kTileBytes);
+#pragma unroll
+        for (int hd = 0; hd < D / 64; ++hd) {
+          tma_load_3d(&tmK, kv_full, smem + L::kOffFix0 + hd * kHalfBytes, hd * 64, jt * kTileN, bh);
+          tma_load_3d(&tmV, kv_full, smem + L::kOffFix1 + hd * kHalfBytes, hd * 64, jt * kTileN, bh);
+        }
+      }
+      for (int e = 0; e < n_list; ++e) {
+        const int s = e % kStages;
+        if (e >= kStages) {
+          // the MMAs of entry e - 2 (the last readers of this stage) have completed
+          if (!mbar_wait(&q_empty[s], ((e / kStages) - 1) & 1) && lane == 0) misc[2] = 1;
+        }
+        if (__any_sync(0xffffffffu, aborted())) continue;
+        const int it = static_cast<int>(list[e] & 0xFFFFu);
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&q_full[s], 2 * L::kTileBytes);
+#pragma unroll
+          for (int hd = 0; hd < D / 64; ++hd) {
+            tma_load_3d(&tmQ, &q_full[s], smem + L::kOffRing0 + s * L::kTileBytes + hd * kHalfBytes, hd * 64,
+                        it * kTileM, bh);
+            tma_load_3d(&tmDO, &q_full[s], smem + L::kOffRing1 + s * L::kTileBytes + hd * kHalfBytes, hd * 64,
+                        it * kTileM, bh);
+          }
+        }
+        // per-query vectors of the tile: lse * log2(e) (+inf past N) and D
+        float* vec = reinterpret_cast<float*>(smem + L::kOffVec) + s * 256;
+        const size_t rbase = static_cast<size_t>(bh) * p.N;
+#pragma unroll
+        for (int k4 = 0; k4 < 4; ++k4) {
+          const int r = k4 * 32 + lane;
+          const int row = it * kTileM + r;
+          const bool valid = row < p.N;
+          vec[r] = valid ? p.lse[rbase + row] * 1.4426950408889634f : __int_as_float(0x7f800000);
+          vec[128 + r] = valid ? p.delta[rbase + row] : 0.f;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&q_full[s]);
+      }
+    }
+  } else if (warp == kBwdMmaWarp) {
+    // -------------------------------------------------------- MMA issue ---
+    if (n_list > 0) {
+      bool ok = __all_sync(0xffffffffu, mbar_wait(kv_full, 0));
+      if (!ok && lane == 0) misc[2] = 1;
+      const uint64_t dk_a = smem_desc(smem_addr(smem + L::kOffFix0), 16, 1024);   // K, A operand
+      const uint64_t dv_a = smem_desc(smem_addr(smem + L::kOffFix1), 16, 1024);   // V, A operand
+      const uint64_t dq_k = smem_desc(smem_addr(smem + L::kOffRing0), 16, 1024);  // Q, K-major B
+      const uint64_t ddo_k = smem_desc(smem_addr(smem + L::kOffRing1), 16, 1024); // dO, K-major B
+      const uint64_t dq_mn = smem_desc(smem_addr(smem + L::kOffRing0), kHalfBytes, 1024);   // Q, MN-major B
+      const uint64_t ddo_mn = smem_desc(smem_addr(smem + L::kOffRing1), kHalfBytes, 1024);  // dO, MN-major B
+      constexpr uint64_t kStageStep = L::kTileBytes >> 4;
+      for (int e = 0; e < n_list; ++e) {
+        const int s = e % kStages;
+        // S^T / dP^T overwrite the columns the previous entry's dV / dK read
+        if (e > 0 && !__all_sync(0xffffffffu, mbar_wait(mma_done, (e - 1) & 1))) {
+          if (lane == 0) misc[2] = 1;
+          ok = false;
+        }
+        ok = __all_sync(0xffffffffu, ok && !aborted());
+        if (ok) {
+          ok = __all_sync(0xffffffffu, mbar_wait(&q_full[s], (e / kStages) & 1));
+          if (!ok && lane == 0) misc[2] = 1;
+        }
+        if (ok) {
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t off = static_cast<uint64_t>((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+            mma_ss_warp(tm_s, dk_a + off, dq_k + s * kStageStep + off, kIdescS, kk > 0 ? 1u : 0u);
+          }
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t off = static_cast<uint64_t>((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+            mma_ss_warp(tm_dp, dv_a + off, ddo_k + s * kStageStep + off, kIdescS, kk > 0 ? 1u : 0u);
+          }
+        }
+        mma_commit_warp(s_ready);   // also after an error, so that no waiter stalls
+        named_bar_sync(kBarBwdP, kBwdHandoff);
+        if (__all_sync(0xffffffffu, ok && !aborted())) {
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < kTileM / 16; ++kk) {
+            const uint64_t off = static_cast<uint64_t>(kk * 16 * 128) >> 4;
+            const uint32_t acc = (e > 0 || kk > 0) ? 1u : 0u;
+            mma_ts_warp(tm_dv, tm_s + kk * 8, ddo_mn + s * kStageStep + off, kIdescG, acc);
+          }
+#pragma unroll
+          for (int kk = 0; kk < kTileM / 16; ++kk) {
+            const uint64_t off = static_cast<uint64_t>(kk * 16 * 128) >> 4;
+            const uint32_t acc = (e > 0 || kk > 0) ? 1u : 0u;
+            mma_ts_warp(tm_dk, tm_dp + kk * 8, dq_mn + s * kStageStep + off, kIdescG, acc);
+          }
+        }
+        mma_commit_warp(&q_empty[s]);
+        mma_commit_warp(mma_done);
+      }
+    }
+  } else {
+    // --------------------------------------- P^T, dS^T and the epilogue ---
+    const int r = threadIdx.x;                       // key row of the kv tile
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const int key = jt * kTileN + r;
+    const bool key_valid = key < p.N;
+    const int kh = BLK == 128 ? 0 : (r >> 6);
+    const float sl2 = p.scale_log2;
+    bool ok = true;
+    for (int e = 0; e < n_list; ++e) {
+      const uint32_t bits = list[e] >> 16;
+      const int it = static_cast<int>(list[e] & 0xFFFFu);
+      const int s = e % kStages;
+      if (!mbar_wait(s_ready, e & 1)) {
+        misc[2] = 1;
+        ok = false;
+      }
+      if (ok && !aborted() && !mbar_wait(&q_full[s], (e / kStages) & 1)) {
+        misc[2] = 1;
+        ok = false;
+      }
+      tc_fence_after();
+      const float* vec = reinterpret_cast<const float*>(smem + L::kOffVec) + s * 256;
+      const int valid_q = min(kTileM, p.N - it * kTileM);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        // chunk c: query columns [32c, 32c + 32) of q-block half c / 2
+        const int qh = BLK == 128 ? 0 : (c >> 1);
+        const bool quad = BLK == 128 ? true : ((bits >> (qh * 2 + kh)) & 1u);
+        const int nv = min(32, max(0, valid_q - 32 * c));
+        const uint32_t keep = (key_valid && quad) ? (nv == 32 ? 0xffffffffu : ((1u << nv) - 1u)) : 0u;
+        float sv[32], dp[32];
+        uint32_t pk[16], dsk[16];
+        tmem_ld32(tm_s + lane_off + 32 * c, sv);
+        tmem_ld32(tm_dp + lane_off + 32 * c, dp);
+        grad_chunk<true>(sv, dp, sl2, vec + 32 * c, vec + 128 + 32 * c, 0.f, 0.f, keep, pk, dsk);
+        tmem_st16(tm_s + lane_off + 16 * c, pk);
+        tmem_st16(tm_dp + lane_off + 16 * c, dsk);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      named_bar_sync(kBarBwdP, kBwdHandoff);
+    }
+    // epilogue: dV and dK rows of this thread's key
+    if (n_list > 0 && !mbar_wait(mma_done, (n_list - 1) & 1)) {
+      misc[2] = 1;
+      ok = false;
+    }
+    tc_fence_after();
+    if (n_list == 0 || __all_sync(0xffffffffu, ok && !aborted())) {
+      const size_t off = (static_cast<size_t>(bh) * p.N + (key_valid ? key : 0)) * D;
+      store_row<D>(tm_dv + lane_off, 1.f, p.dv + off, n_list == 0, key_valid);
+      store_row<D>(tm_dk + lane_off, p.scale, p.dk + off, n_list == 0, key_valid);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kBwdMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ----------------------------------------------------------------- dQ ---
+// CTA = (q-tile it, head bh).  TMEM columns: dQ [0, D), S [128, 256) (dS
+// packed to bf16 over its first 64 columns), dP [256, 384).
+template <int D, int BLK>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                  const BwdParams p) {
+  using L = BwdSmem<D>;
+  constexpr int QH = kTileM / BLK;
+  constexpr int KH = kTileN / BLK;
+  constexpr uint32_t kIdescS = idesc_bf16_f32(kTileM, kTileN, false);
+  constexpr uint32_t kIdescG = idesc_bf16_f32(kTileM, D, true);
+  constexpr int kHalfBytes = kTileM * 128;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint32_t* list = reinterpret_cast<uint32_t*>(smem + L::kOffList);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
+  uint64_t* qd_full = bars;
+  uint64_t* kv_full = bars + 1;
+  uint64_t* kv_empty = kv_full + kStages;
+  uint64_t* s_ready = kv_empty + kStages;
+  uint64_t* mma_done = s_ready + 1;
+  volatile int* misc = reinterpret_cast<volatile int*>(smem + L::kOffMisc);
+  // misc[0] TMEM base, [1] list length, [2] abort flag
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int it = blockIdx.x;
+  const int bh = blockIdx.y;
+  const int b = bh / p.H, h = bh - (bh / p.H) * p.H;
+  auto aborted = [&]() -> bool { return misc[2] != 0; };
+
+  if (warp == kBwdLoadWarp) {
+    // ---- kv-tile list of this q-tile, per-quadrant keep bits ----
+    int n = 0;
+    for (int base = 0; base < p.n_tiles; base += 32) {
+      const int jt = base + lane;
+      uint32_t bits = 0;
+      if (jt < p.n_tiles) {
+#pragma unroll
+        for (int qh = 0; qh < QH; ++qh) {
+          const int qb = it * QH + qh;
+          if (qb >= p.nb) continue;
+#pragma unroll
+          for (int kh = 0; kh < KH; ++kh) {
+            const int kb = jt * KH + kh;
+            if (kb >= p.nb) continue;
+            const uint8_t keep = p.mask ? p.mask[b * p.msb + h * p.msh + qb * p.msi + kb] : uint8_t(1);
+            if (keep) bits |= (BLK == 128 ? 0xFu : (1u << (qh * 2 + kh)));
+          }
+        }
+      }
+      const unsigned ball = __ballot_sync(0xffffffffu, bits != 0);
+      if (bits) list[n + __popc(ball & ((1u << lane) - 1u))] = static_cast<uint32_t>(jt) | (bits << 16);
+      n += __popc(ball);
+    }
+    if (lane == 0) {
+      misc[1] = n;
+      misc[2] = 0;
+      for (int i = 0; i < L::kNumBars; ++i) mbar_init(&bars[i], 1u);
+      fence_mbar_init();
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmDO);
+    }
+  } else if (warp == kBwdMmaWarp) {
+    tmem_alloc(const_cast<uint32_t*>(reinterpret_cast<volatile uint32_t*>(misc)), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  const uint32_t tmem = static_cast<uint32_t>(misc[0]);
+  const int n_list = misc[1];
+  const uint32_t tm_dq = tmem, tm_s = tmem + 128, tm_dp = tmem + 256;
+
+  if (warp == kBwdLoadWarp) {
+    // ------------------------------------------------------------- loads ---
+    if (n_list > 0) {
+      if (lane == 0) {
+        mbar_arrive_expect_tx(qd_full, 2 * L::kTileBytes);
+#pragma unroll
+        for (int hd = 0; hd < D / 64; ++hd) {
+          tma_load_3d(&tmQ, qd_full, smem + L::kOffFix0 + hd * kHalfBytes, hd * 64, it * kTileM, bh);
+          tma_load_3d(&tmDO, qd_full, smem + L::kOffFix1 + hd * kHalfBytes, hd * 64, it * kTileM, bh);
+        }
+      }
+      for (int e = 0; e < n_list; ++e) {
+        const int s = e % kStages;
+        if (e >= kStages && !mbar_wait(&kv_empty[s], ((e / kStages) - 1) & 1) && lane == 0) misc[2] = 1;
+        if (__any_sync(0xffffffffu, aborted())) continue;
+        const int jt = static_cast<int>(list[e] & 0xFFFFu);
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&kv_full[s], 2 * L::kTileBytes);
+#pragma unroll
+          for (int hd = 0; hd < D / 64; ++hd) {
+            tma_load_3d(&tmK, &kv_full[s], smem + L::kOffRing0 + s * L::kTileBytes + hd * kHalfBytes, hd * 64,
+                        jt * kTileN, bh);
+            tma_load_3d(&tmV, &kv_full[s], smem + L::kOffRing1 + s * L::kTileBytes + hd * kHalfBytes, hd * 64,
+                        jt * kTileN, bh);
+          }
+        }
+      }
+    }
+  } else if (warp == kBwdMmaWarp) {
+    // -------------------------------------------------------- MMA issue ---
+    if (n_list > 0) {
+      bool ok = __all_sync(0xffffffffu, mbar_wait(qd_full, 0));
+      if (!ok && lane == 0) misc[2] = 1;
+      const uint64_t dq_a = smem_desc(smem_addr(smem + L::kOffFix0), 16, 1024);    // Q, A operand
+      const uint64_t ddo_a = smem_desc(smem_addr(smem + L::kOffFix1), 16, 1024);   // dO, A operand
+      const uint64_t dk_k = smem_desc(smem_addr(smem + L::kOffRing0), 16, 1024);   // K, K-major B
+      const uint64_t dv_k = smem_desc(smem_addr(smem + L::kOffRing1), 16, 1024);   // V, K-major B
+      const uint64_t dk_mn = smem_desc(smem_addr(smem + L::kOffRing0), kHalfBytes, 1024);  // K, MN-major B
+      constexpr uint64_t kStageStep = L::kTileBytes >> 4;
+      for (int e = 0; e < n_list; ++e) {
+        const int s = e % kStages;
+        // S / dP overwrite the columns the previous entry's dQ MMA read
+        if (e > 0 && !__all_sync(0xffffffffu, mbar_wait(mma_done, (e - 1) & 1))) {
+          if (lane == 0) misc[2] = 1;
+          ok = false;
+        }
+        ok = __all_sync(0xffffffffu, ok && !aborted());
+        if (ok) {
+          ok = __all_sync(0xffffffffu, mbar_wait(&kv_full[s], (e / kStages) & 1));
+          if (!ok && lane == 0) misc[2] = 1;
+        }
+        if (ok) {
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t off = static_cast<uint64_t>((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+            mma_ss_warp(tm_s, dq_a + off, dk_k + s * kStageStep + off, kIdescS, kk > 0 ? 1u : 0u);
+          }
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t off = static_cast<uint64_t>((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+            mma_ss_warp(tm_dp, ddo_a + off, dv_k + s * kStageStep + off, kIdescS, kk > 0 ? 1u : 0u);
+          }
+        }
+        mma_commit_warp(s_ready);   // also after an error, so that no waiter stalls
+        named_bar_sync(kBarBwdP, kBwdHandoff);
+        if (__all_sync(0xffffffffu, ok && !aborted())) {
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < kTileN / 16; ++kk) {
+            const uint64_t off = static_cast<uint64_t>(kk * 16 * 128) >> 4;
+            mma_ts_warp(tm_dq, tm_s + kk * 8, dk_mn + s * kStageStep + off, kIdescG, (e > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        mma_commit_warp(&kv_empty[s]);
+        mma_commit_warp(mma_done);
+      }
+    }
+  } else {
+    // ------------------------------------------------ dS and the epilogue ---
+    const int r = threadIdx.x;                       // query row of the q-tile
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const int row = it * kTileM + r;
+    const bool row_valid = row < p.N;
+    const int qh = BLK == 128 ? 0 : (r >> 6);
+    const float sl2 = p.scale_log2;
+    const size_t rix = static_cast<size_t>(bh) * p.N + (row_valid ? row : 0);
+    const float l2 = row_valid ? p.lse[rix] * 1.4426950408889634f : 0.f;
+    const float dl = row_valid ? p.delta[rix] : 0.f;
+    bool ok = true;
+    for (int e = 0; e < n_list; ++e) {
+      const uint32_t bits = list[e] >> 16;
+      const int jt = static_cast<int>(list[e] & 0xFFFFu);
+      if (!mbar_wait(s_ready, e & 1)) {
+        misc[2] = 1;
+        ok = false;
+      }
+      tc_fence_after();
+      const int valid_k = min(kTileN, p.N - jt * kTileN);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        // chunk c: key columns [32c, 32c + 32) of k-block half c / 2
+        const int kh = BLK == 128 ? 0 : (c >> 1);
+        const bool quad = BLK == 128 ? true : ((bits >> (qh * 2 + kh)) & 1u);
+        const int nv = min(32, max(0, valid_k - 32 * c));
+        const uint32_t keep = (row_valid && quad) ? (nv == 32 ? 0xffffffffu : ((1u << nv) - 1u)) : 0u;
+        float sv[32], dp[32];
+        uint32_t pk[16], dsk[16];
+        tmem_ld32(tm_s + lane_off + 32 * c, sv);
+        tmem_ld32(tm_dp + lane_off + 32 * c, dp);
+        grad_chunk<false>(sv, dp, sl2, nullptr, nullptr, l2, dl, keep, pk, dsk);
+        tmem_st16(tm_s + lane_off + 16 * c, dsk);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      named_bar_sync(kBarBwdP, kBwdHandoff);
+    }
+    if (n_list > 0 && !mbar_wait(mma_done, (n_list - 1) & 1)) {
+      misc[2] = 1;
+      ok = false;
+    }
+    tc_fence_after();
+    if (n_list == 0 || __all_sync(0xffffffffu, ok && !aborted())) {
+      store_row<D>(tm_dq + lane_off, p.scale, p.dq + rix * D, n_list == 0, row_valid);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kBwdMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace sa

@@ -6,11 +6,13 @@
 // launches it on the caller's stream; all arithmetic runs on the GPU.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
 
+#include "sa_attn_bwd.cuh"
 #include "sa_attn_fwd.cuh"
 #include "sa_common.cuh"
 #include "sa_masks.cuh"
@@ -84,6 +86,14 @@ cudaError_t init_device_kernels() {
     set(reinterpret_cast<const void*>(&sa::pyr_fwd_kernel<128, 64>), sa::PyrSmem<128>::kAlloc);
     set(reinterpret_cast<const void*>(&sa::pyr_fwd_kernel<64, 128>), sa::PyrSmem<64>::kAlloc);
     set(reinterpret_cast<const void*>(&sa::pyr_fwd_kernel<64, 64>), sa::PyrSmem<64>::kAlloc);
+    set(reinterpret_cast<const void*>(&sa::bwd_dkdv_kernel<128, 128>), sa::BwdSmem<128>::kAlloc);
+    set(reinterpret_cast<const void*>(&sa::bwd_dkdv_kernel<128, 64>), sa::BwdSmem<128>::kAlloc);
+    set(reinterpret_cast<const void*>(&sa::bwd_dkdv_kernel<64, 128>), sa::BwdSmem<64>::kAlloc);
+    set(reinterpret_cast<const void*>(&sa::bwd_dkdv_kernel<64, 64>), sa::BwdSmem<64>::kAlloc);
+    set(reinterpret_cast<const void*>(&sa::bwd_dq_kernel<128, 128>), sa::BwdSmem<128>::kAlloc);
+    set(reinterpret_cast<const void*>(&sa::bwd_dq_kernel<128, 64>), sa::BwdSmem<128>::kAlloc);
+    set(reinterpret_cast<const void*>(&sa::bwd_dq_kernel<64, 128>), sa::BwdSmem<64>::kAlloc);
+    set(reinterpret_cast<const void*>(&sa::bwd_dq_kernel<64, 64>), sa::BwdSmem<64>::kAlloc);
     set(reinterpret_cast<const void*>(&sa::block_select_kernel),
         static_cast<int>(sa::select_smem_bytes(sa::kMaxSelect)));
     di.err = r;
@@ -426,3 +436,90 @@ extern "C" sa_status sa_build_mask_noalloc(const void* q, const void* k, int B, 
   return sa_build_mask(q, k, B, H, N, d, block, mode, tau, level_frac, mask_out, scores_out, scratch,
                        kNoAllocScratchBytes, stream);
 }
+
+// -------------------------------------------------------- backward pass ---
+extern "C" {
+
+size_t sa_sparse_attn_bwd_workspace(int B, int H, int N) {
+  if (B <= 0 || H <= 0 || N <= 0) return 0;
+  return static_cast<size_t>(B) * H * N * sizeof(float);
+}
+
+sa_status sa_sparse_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                             const float* lse, int B, int H, int N, int d, int block, const uint8_t* mask,
+                             int64_t mask_sb, int64_t mask_sh, int64_t mask_si, float scale, void* dq, void* dk,
+                             void* dv, void* workspace, size_t workspace_bytes, void* stream) {
+  if (B < 0 || H < 0 || N < 0) return SA_ERR_INVALID_ARG;
+  if (std::isnan(scale) || scale < 0.f || std::isinf(scale)) return SA_ERR_INVALID_ARG;
+  if (B == 0 || H == 0 || N == 0) return SA_OK;
+  if (!valid_dim(d) || !valid_block(block)) return SA_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace) return SA_ERR_INVALID_ARG;
+  for (const void* ptr : {q, k, v, o, dout, static_cast<const void*>(dq), static_cast<const void*>(dk),
+                          static_cast<const void*>(dv), static_cast<const void*>(workspace)})
+    if (!aligned16(ptr)) return SA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return SA_ERR_INVALID_ARG;
+  if (workspace_bytes < sa_sparse_attn_bwd_workspace(B, H, N)) return SA_ERR_INVALID_ARG;
+  if (mask && (mask_sb < 0 || mask_sh < 0 || mask_si < 0)) return SA_ERR_INVALID_ARG;
+  const int n_tiles = ceil_div(N, sa::kTileN);
+  if (n_tiles > sa::kMaxKvTiles) return SA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * H > 65535) return SA_ERR_UNSUPPORTED;
+  cudaError_t e = init_device_kernels();
+  if (e != cudaSuccess) return SA_ERR_CUDA;
+
+  const int BH = B * H;
+  CUtensorMap tq, tk, tv, tdo;
+  if (!encode_rows_map(&tq, q, BH, N, d, sa::kTileM) || !encode_rows_map(&tk, k, BH, N, d, sa::kTileN) ||
+      !encode_rows_map(&tv, v, BH, N, d, sa::kTileN) || !encode_rows_map(&tdo, dout, BH, N, d, sa::kTileM))
+    return SA_ERR_CUDA;
+
+  if (scale == 0.f) scale = 1.0f / std::sqrt(static_cast<float>(d));
+  float* delta = static_cast<float*>(workspace);
+  sa::BwdParams p;
+  p.B = B;
+  p.H = H;
+  p.N = N;
+  p.nb = ceil_div(N, block);
+  p.n_tiles = n_tiles;
+  p.mask = mask;
+  p.msb = mask_sb;
+  p.msh = mask_sh;
+  p.msi = mask_si;
+  p.lse = lse;
+  p.delta = delta;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.dq = static_cast<__nv_bfloat16*>(dq);
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+
+  cudaStream_t s = as_stream(stream);
+  const long long rows = static_cast<long long>(BH) * N;
+  const int rows_per_block = 256 / (d / 8);
+  const int grid_d = static_cast<int>(std::min<long long>((rows + rows_per_block - 1) / rows_per_block, 148LL * 16));
+  const __nv_bfloat16* ob = static_cast<const __nv_bfloat16*>(o);
+  const __nv_bfloat16* gb = static_cast<const __nv_bfloat16*>(dout);
+  if (d == 128)
+    sa::bwd_delta_kernel<128><<<grid_d, 256, 0, s>>>(ob, gb, delta, rows);
+  else
+    sa::bwd_delta_kernel<64><<<grid_d, 256, 0, s>>>(ob, gb, delta, rows);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return SA_ERR_CUDA;
+
+  const dim3 grid(n_tiles, BH);
+  if (d == 128 && block == 128) {
+    sa::bwd_dkdv_kernel<128, 128><<<grid, sa::kBwdThreads, sa::BwdSmem<128>::kAlloc, s>>>(tq, tk, tv, tdo, p);
+    sa::bwd_dq_kernel<128, 128><<<grid, sa::kBwdThreads, sa::BwdSmem<128>::kAlloc, s>>>(tq, tk, tv, tdo, p);
+  } else if (d == 128) {
+    sa::bwd_dkdv_kernel<128, 64><<<grid, sa::kBwdThreads, sa::BwdSmem<128>::kAlloc, s>>>(tq, tk, tv, tdo, p);
+    sa::bwd_dq_kernel<128, 64><<<grid, sa::kBwdThreads, sa::BwdSmem<128>::kAlloc, s>>>(tq, tk, tv, tdo, p);
+  } else if (block == 128) {
+    sa::bwd_dkdv_kernel<64, 128><<<grid, sa::kBwdThreads, sa::BwdSmem<64>::kAlloc, s>>>(tq, tk, tv, tdo, p);
+    sa::bwd_dq_kernel<64, 128><<<grid, sa::kBwdThreads, sa::BwdSmem<64>::kAlloc, s>>>(tq, tk, tv, tdo, p);
+  } else {
+    sa::bwd_dkdv_kernel<64, 64><<<grid, sa::kBwdThreads, sa::BwdSmem<64>::kAlloc, s>>>(tq, tk, tv, tdo, p);
+    sa::bwd_dq_kernel<64, 64><<<grid, sa::kBwdThreads, sa::BwdSmem<64>::kAlloc, s>>>(tq, tk, tv, tdo, p);
+  }
+  return cuda_status(cudaGetLastError());
+}
+
+}  // extern "C"

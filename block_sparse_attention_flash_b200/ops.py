@@ -37,6 +37,9 @@ _SIGNATURES = {
                                   _vp, _vp, _f32, _f32, _i32, _vp, _vp, _vp]),
     "sa_pyramid_attn_fwd": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _i64, _i64, _i64,
                                    _vp, _vp, _f32, _vp, _vp, _vp]),
+    "sa_sparse_attn_bwd_workspace": (_sz, [_i32, _i32, _i32]),
+    "sa_sparse_attn_bwd": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _i64, _i64, _i64,
+                                  _f32, _vp, _vp, _vp, _vp, _sz, _vp]),
 }
 
 _lib = None
@@ -224,3 +227,37 @@ def sa_pyramid_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block
         _dev(out, "out", torch.bfloat16), _opt(lse, "lse", torch.float32), _stream(stream))
     _check(st, "sa_pyramid_attn_fwd")
     return out
+
+
+def sa_sparse_attn_bwd_workspace(B: int, H: int, N: int) -> int:
+    return int(lib().sa_sparse_attn_bwd_workspace(B, H, N))
+
+
+def sa_sparse_attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, dout: torch.Tensor,
+                       lse: torch.Tensor, block: int, mask: Optional[torch.Tensor] = None, scale: float = 0.0,
+                       dq: Optional[torch.Tensor] = None, dk: Optional[torch.Tensor] = None,
+                       dv: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                       stream=None):
+    """Gradients (dQ, dK, dV) of sa_sparse_attn_fwd given dO and the forward's O and LSE."""
+    B, H, N, d = q.shape
+    nb = nblocks(N, block)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if workspace is None:
+        workspace = torch.empty(max(16, sa_sparse_attn_bwd_workspace(B, H, N)), dtype=torch.uint8, device=q.device)
+    sb = sh = si = 0
+    mptr = None
+    if mask is not None:
+        if mask.dtype != torch.uint8 or not mask.is_cuda:
+            raise ValueError("mask must be a CUDA uint8 tensor")
+        sb, sh, si = _mask_strides(mask, B, H, nb)
+        mptr = mask.data_ptr()
+    st = lib().sa_sparse_attn_bwd(
+        _dev(q, "q", torch.bfloat16), _dev(k, "k", torch.bfloat16), _dev(v, "v", torch.bfloat16),
+        _dev(o, "o", torch.bfloat16), _dev(dout, "dout", torch.bfloat16), _dev(lse, "lse", torch.float32),
+        B, H, N, d, block, mptr, sb, sh, si, float(scale),
+        _dev(dq, "dq", torch.bfloat16), _dev(dk, "dk", torch.bfloat16), _dev(dv, "dv", torch.bfloat16),
+        _dev(workspace, "workspace", torch.uint8), workspace.numel(), _stream(stream))
+    _check(st, "sa_sparse_attn_bwd")
+    return dq, dk, dv

@@ -10,6 +10,7 @@
  *   sa_pyramid_pool    PSA pyramid: mean-pooled K/V at 2, 4 and 8 tokens per key
  *   sa_sparse_attn_fwd FlashAttention-style forward over kept tiles, with the
  *                      LiteAttention skip-mask update fused in
+ *   sa_sparse_attn_bwd its gradients with respect to Q, K and V
  *
  * Conventions shared by every entry point
  *   - Tensors are caller-owned DEVICE memory.  Q, K, V and O are bf16,
@@ -245,6 +246,41 @@ SA_API sa_status sa_pyramid_attn_fwd(const void* q, const void* k, const void* v
                               const uint8_t* levels, int64_t lv_sb, int64_t lv_sh, int64_t lv_si,
                               const void* const* k_pool, const void* const* v_pool,
                               float scale, void* o, float* lse, void* stream);
+
+/*
+ * sa_sparse_attn_bwd — gradients of sa_sparse_attn_fwd with respect to Q, K, V.
+ *   Needed by the LoRA length extension of the Radial Attention write-up
+ *   ("MIT实验室推出Radial Attention", arXiv 2506.19852, training-cost
+ *   paragraph), which trains through the sparse attention.  The formulas are
+ *   the derivative of the forward's definition; no page states them:
+ *     P_rc = exp(s_rc - LSE_r) on the kept columns of row r (0 elsewhere),
+ *     D_r  = dO_r . O_r,
+ *     dV_c = sum_r P_rc dO_r,
+ *     dS   = P * (dO V^T - D),
+ *     dQ_r = scale sum_c dS_rc k_c,   dK_c = scale sum_r dS_rc q_r.
+ * Arguments
+ *   q, k, v       bf16 [B,H,N,d] device, the forward's inputs.
+ *   o, lse        the forward's outputs for the same q, k, v, mask and scale
+ *                 (bf16 [B,H,N,d]; fp32 [B,H,N], natural log).  A row with no
+ *                 kept block (LSE = -inf) gets dQ = 0.
+ *   dout          bf16 [B,H,N,d] device, the gradient of the loss w.r.t. O.
+ *   mask, mask_s* as sa_sparse_attn_fwd (NULL keeps every block; any nonzero
+ *                 byte keeps).  Pass the forward's effective mask (mask AND
+ *                 NOT skip_in when the forward skipped blocks).
+ *   scale         logit scale; 0 selects 1/sqrt(d).
+ *   dq, dk, dv    bf16 [B,H,N,d] device, written for every valid row (zero
+ *                 where the row or key takes part in no kept block).
+ *   workspace     device scratch of at least sa_sparse_attn_bwd_workspace()
+ *                 bytes (16-byte aligned): holds D_r as fp32 [B,H,N].
+ * Deterministic: no atomics; dK/dV and dQ come from separate passes.
+ * Limits: as sa_sparse_attn_fwd.
+ */
+SA_API size_t sa_sparse_attn_bwd_workspace(int B, int H, int N);
+SA_API sa_status sa_sparse_attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                             const void* dout, const float* lse, int B, int H, int N, int d, int block,
+                             const uint8_t* mask, int64_t mask_sb, int64_t mask_sh, int64_t mask_si,
+                             float scale, void* dq, void* dk, void* dv, void* workspace,
+                             size_t workspace_bytes, void* stream);
 
 #ifdef __cplusplus
 }

@@ -76,11 +76,12 @@ def masked_attention_bwd_rows(q, k, v, block, mask, dout, b, h, q_rows, k_rows, 
     gradients, so all rows are visited; only the selected outputs are kept.
     Returns (dQ [len(q_rows), d], dK [len(k_rows), d], dV [len(k_rows), d]).
     """
+    B, H = q.shape[0], q.shape[1]
     qh, kh, vh, doh = (_f64(x[b, h]) for x in (q, k, v, dout))
     N, d = qh.shape
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     nb = _nblocks(N, block)
-    m = np.asarray(_mask4(mask, b + 1, h + 1, nb, nb)[b, h]) != 0
+    m = np.asarray(_mask4(mask, B, H, nb, nb)[b, h]) != 0
     q_rows = np.asarray(q_rows, dtype=np.int64)
     k_rows = np.asarray(k_rows, dtype=np.int64)
     kblk = np.arange(N) // block

@@ -5,7 +5,8 @@ Tolerances (bf16 inputs and output, unit-variance data):
   LSE  abs <= 1e-3 (finite rows), identical -inf on rows with no visited block;
   masks / skip bits: bit-exact except bits whose decision margin lies within
   1e-3 of the cut (flagged by the oracle); flagged mismatches are counted and
-  returned, not failed.
+  returned, not failed;
+  gradients: relative to the reference's size (check_grad below).
 """
 import numpy as np
 import torch
@@ -62,3 +63,27 @@ def skip_flags(margin, eps_margin=1e-3):
     """Flag skip decisions whose margin max_r(l_r - m_r + eps) is within 1e-3 of 0."""
     m = np.asarray(margin)
     return np.isfinite(m) & (np.abs(m) < eps_margin)
+
+
+# Gradients (attention backward): their scale shrinks like 1/sqrt(kept keys),
+# so the bar is relative to the reference.  The kernel rounds P and dS to bf16
+# for the MMAs (relative 2^-9 each), takes D_r from the bf16 forward output and
+# rounds the result to bf16: about 0.5 % per element.  Bar: max-abs error
+# <= 2e-2 x max |ref| and mean-abs error <= 1e-2 x mean |ref|.
+GRAD_MAX_REL = 2e-2
+GRAD_MEAN_REL = 1e-2
+
+
+def check_grad(g_gpu, g_ref, what=""):
+    g = as_np(g_gpu).astype(np.float64)
+    r = np.asarray(g_ref, dtype=np.float64)
+    assert g.shape == r.shape, (g.shape, r.shape)
+    assert np.all(np.isfinite(g)), f"{what}: non-finite gradient"
+    err = np.abs(g - r)
+    ref_max, ref_mean = np.abs(r).max(), np.abs(r).mean()
+    if ref_max == 0.0:
+        assert err.max() == 0.0, f"{what}: nonzero where the gradient is zero"
+        return 0.0, 0.0
+    assert err.max() <= GRAD_MAX_REL * ref_max, f"{what}: max-abs {err.max():.3e} vs max|ref| {ref_max:.3e}"
+    assert err.mean() <= GRAD_MEAN_REL * ref_mean, f"{what}: mean-abs {err.mean():.3e} vs mean|ref| {ref_mean:.3e}"
+    return float(err.max() / ref_max), float(err.mean() / ref_mean)

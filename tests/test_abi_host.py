@@ -29,7 +29,8 @@ def _declared_symbols():
 def test_header_declares_the_entry_points():
     names = _declared_symbols()
     for n in ("sa_build_mask", "sa_radial_mask", "sa_pyramid_pool", "sa_sparse_attn_fwd",
-              "sa_pyramid_attn_fwd", "sa_get_device_status", "sa_build_mask_workspace"):
+              "sa_pyramid_attn_fwd", "sa_get_device_status", "sa_build_mask_workspace",
+              "sa_sparse_attn_bwd", "sa_sparse_attn_bwd_workspace"):
         assert n in names
 
 
@@ -111,3 +112,29 @@ def test_ops_refuse_cpu_tensors():
     q = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16)
     with pytest.raises((ValueError, RuntimeError)):
         ops.sa_sparse_attn_fwd(q, q, q, 64, out=q.clone())
+
+
+def _bwd(lib, **kw):
+    a = dict(q=16, k=16, v=16, o=16, dout=16, lse=16, B=1, H=1, N=256, d=128, block=128, mask=None, sb=0, sh=0,
+             si=0, scale=0.0, dq=16, dk=16, dv=16, ws=16, ws_bytes=1 << 20, stream=None)
+    a.update(kw)
+    return lib.sa_sparse_attn_bwd(a["q"], a["k"], a["v"], a["o"], a["dout"], a["lse"], a["B"], a["H"], a["N"],
+                                  a["d"], a["block"], a["mask"], a["sb"], a["sh"], a["si"], a["scale"], a["dq"],
+                                  a["dk"], a["dv"], a["ws"], a["ws_bytes"], a["stream"])
+
+
+def test_backward_workspace_and_argument_validation(lib):
+    assert ops.sa_sparse_attn_bwd_workspace(2, 3, 100) == 2 * 3 * 100 * 4
+    assert ops.sa_sparse_attn_bwd_workspace(0, 3, 100) == 0
+    assert _bwd(lib, B=0) == ops.SA_OK                          # nothing to do
+    assert _bwd(lib, N=-1) == ops.SA_ERR_INVALID_ARG
+    assert _bwd(lib, d=96) == ops.SA_ERR_UNSUPPORTED
+    assert _bwd(lib, block=256) == ops.SA_ERR_UNSUPPORTED
+    assert _bwd(lib, lse=None) == ops.SA_ERR_INVALID_ARG
+    assert _bwd(lib, dout=None) == ops.SA_ERR_INVALID_ARG
+    assert _bwd(lib, dk=24) == ops.SA_ERR_INVALID_ARG           # not 16-byte aligned
+    assert _bwd(lib, lse=18) == ops.SA_ERR_INVALID_ARG          # not 4-byte aligned
+    assert _bwd(lib, ws_bytes=256 * 4 - 1) == ops.SA_ERR_INVALID_ARG
+    assert _bwd(lib, scale=float("nan")) == ops.SA_ERR_INVALID_ARG
+    assert _bwd(lib, mask=16, si=-1) == ops.SA_ERR_INVALID_ARG
+

@@ -80,15 +80,16 @@ def test_sampled_rows_equal_full_gradients():
     dq, dk, dv = masked_attention_bwd(q, k, v, wl.block, mask, do)
     qr = [0, 5, 63, 64, 200, wl.N - 1]
     kr = [1, 64, 127, 150, wl.N - 1]
-    sq, sk, sv = masked_attention_bwd_rows(q, k, v, wl.block, mask, do, 0, 1, qr, kr, chunk=96)
-    assert np.max(np.abs(sq - dq[0, 1, qr])) < 1e-12
-    assert np.max(np.abs(sk - dk[0, 1, kr])) < 1e-12
-    assert np.max(np.abs(sv - dv[0, 1, kr])) < 1e-12
+    for h in range(2):
+        sq, sk, sv = masked_attention_bwd_rows(q, k, v, wl.block, mask, do, 0, h, qr, kr, chunk=96)
+        assert np.max(np.abs(sq - dq[0, h, qr])) < 1e-12
+        assert np.max(np.abs(sk - dk[0, h, kr])) < 1e-12
+        assert np.max(np.abs(sv - dv[0, h, kr])) < 1e-12
 
 
 def test_pins_catch_planted_mistakes(monkeypatch):
-    """Each planted mistake (dropped D term, transposed dS in dK, missing scale
-    in dQ) must break the key-shift invariance or the finite-difference pin."""
+    """Each planted mistake (dropped D term, missing scale in dQ) must break
+    the key-shift invariance or the finite-difference pin."""
     import oracle.backward as ob
 
     q, k, v, dout, block, mask = _case(N=24, d=4, block=8, seed=21)
