@@ -43,7 +43,9 @@ constexpr int kBwdWarps = 6;
 constexpr int kBwdThreads = kBwdWarps * 32;
 constexpr int kBwdLoadWarp = 4;
 constexpr int kBwdMmaWarp = 5;
-constexpr int kBarBwdP = 1;         // P / dS packed in TMEM: warps 0-3 <-> MMA warp
+// P / dS of the first / second 64-column half packed in TMEM: warps 0-3 <-> MMA warp
+constexpr int kBarBwdA = 1;
+constexpr int kBarBwdB = 2;
 constexpr int kBwdHandoff = 160;
 
 struct BwdParams {
@@ -100,8 +102,8 @@ struct BwdSmem {
   static constexpr int kOffRing1 = kOffRing0 + kStages * kTileBytes;    // [stage]
   static constexpr int kOffVec = kOffRing1 + kStages * kTileBytes;      // [stage][2][128] f32
   static constexpr int kOffList = kOffVec + kStages * 2 * 128 * 4;
-  // fix_full, ring_full[2], ring_empty[2], s_ready, mma_done
-  static constexpr int kNumBars = 1 + 2 * kStages + 2;
+  // fix_full, ring_full[2], ring_empty[2], ready_a, ready_b, half_a_done, half_b_done
+  static constexpr int kNumBars = 1 + 2 * kStages + 4;
   static constexpr int kOffBar = kOffList + kMaxKvTiles * 4;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffMisc + 64;
@@ -138,6 +140,32 @@ __device__ __forceinline__ void grad_chunk(const float* sv, const float* dp, flo
   }
 }
 
+// Half hh (columns [64 hh, 64 hh + 64)) of this thread's S and dP rows: P
+// packed over the half's first 32 S columns (when kStoreP) and dS over the
+// half's first 32 columns at ds_base.  The second chunk's loads are issued
+// before the first chunk's stores (disjoint columns); each chunk's stores
+// land on columns its own or the previous chunk already read.
+template <bool kPerColumn, bool kStoreP>
+__device__ __forceinline__ void grad_half(uint32_t ts, uint32_t tdp, uint32_t ds_base, int hh, float sl2,
+                                          const float* l2, const float* dl, float l2s, float dls, uint32_t keep0,
+                                          uint32_t keep1) {
+  float s0[32], d0[32], s1[32], d1[32];
+  uint32_t pk[16], dk[16];
+  const uint32_t cs = ts + 64 * hh, cd = tdp + 64 * hh, cq = ds_base + 64 * hh;
+  tmem_ld32x2_nowait(cs, cd, s0, d0);
+  tmem_ld_wait2(s0, d0);
+  tmem_ld32x2_nowait(cs + 32, cd + 32, s1, d1);
+  grad_chunk<kPerColumn>(s0, d0, sl2, kPerColumn ? l2 + 64 * hh : nullptr, kPerColumn ? dl + 64 * hh : nullptr,
+                         l2s, dls, keep0, pk, dk);
+  if (kStoreP) tmem_st16(cs, pk);
+  tmem_st16(cq, dk);
+  tmem_ld_wait2(s1, d1);
+  grad_chunk<kPerColumn>(s1, d1, sl2, kPerColumn ? l2 + 64 * hh + 32 : nullptr,
+                         kPerColumn ? dl + 64 * hh + 32 : nullptr, l2s, dls, keep1, pk, dk);
+  if (kStoreP) tmem_st16(cs + 16, pk);
+  tmem_st16(cq + 16, dk);
+}
+
 // One thread's fp32 TMEM row (columns [taddr, taddr + D)) times `mul`, to
 // bf16 at dst (16-byte aligned) when `store`, or zeros when `zero`.  Called by
 // whole warps with warp-uniform `zero` (the TMEM loads are warp-collective).
@@ -166,10 +194,16 @@ __device__ __forceinline__ void store_row(uint32_t taddr, float mul, __nv_bfloat
   }
 }
 
+
 // ------------------------------------------------------------ dK / dV ---
 // CTA = (kv tile jt, head bh).  TMEM columns: dV [0, D), dK [D, 2D),
-// S^T [2D, 2D + 128) (P^T packed to bf16 over its first 64 columns),
-// dP^T [2D + 128, 2D + 256) (dS^T packed over its first 64 columns).
+// S^T [2D, 2D + 128) and dP^T [2D + 128, 2D + 256), each in two 64-query
+// halves; P^T / dS^T of a half are packed to bf16 over the half's first 32
+// columns.  Per entry (q-tile) the MMA warp issues, for each half: S^T_h and
+// dP^T_h (N = 64), and once warps 0-3 have packed the half, dV += P^T_h dO_h
+// and dK += dS^T_h Q_h (K = 64).  The next entry's S^T_h goes into a half as
+// soon as the gradient MMAs that read it have completed, so one half's MMAs
+// run while warps 0-3 work on the other.
 template <int D, int BLK>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -178,7 +212,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   using L = BwdSmem<D>;
   constexpr int QH = kTileM / BLK;  // q-blocks per q-tile
   constexpr int KH = kTileN / BLK;  // k-blocks per kv tile
-  constexpr uint32_t kIdescS = idesc_bf16_f32(kTileN, kTileM, false);
+  constexpr uint32_t kIdescH = idesc_bf16_f32(kTileN, 64, false);   // S^T / dP^T half: 128 keys x 64 queries
   constexpr uint32_t kIdescG = idesc_bf16_f32(kTileN, D, true);
   constexpr int kHalfBytes = kTileM * 128;  // one 64-column slab of a tile
 
@@ -189,8 +223,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* kv_full = bars;
   uint64_t* q_full = bars + 1;
   uint64_t* q_empty = q_full + kStages;
-  uint64_t* s_ready = q_empty + kStages;
-  uint64_t* mma_done = s_ready + 1;
+  uint64_t* ready = q_empty + kStages;       // [2]: S^T_h and dP^T_h of the current entry computed
+  uint64_t* half_done = ready + 2;           // [2]: the gradient MMAs of half h completed
   volatile int* misc = reinterpret_cast<volatile int*>(smem + L::kOffMisc);
   // misc[0] TMEM base, [1] list length, [2] abort flag
 
@@ -227,6 +261,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (lane == 0) {
       misc[1] = n;
       misc[2] = 0;
+      // q_full: the TMA bytes' arrival and the LSE / D writer's arrival
       for (int i = 0; i < L::kNumBars; ++i) mbar_init(&bars[i], (&bars[i] >= q_full && &bars[i] < q_empty) ? 2u : 1u);
       fence_mbar_init();
       tma_prefetch_desc(&tmQ);
@@ -259,10 +294,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       for (int e = 0; e < n_list; ++e) {
         const int s = e % kStages;
-        if (e >= kStages) {
-          // the MMAs of entry e - 2 (the last readers of this stage) have completed
-          if (!mbar_wait(&q_empty[s], ((e / kStages) - 1) & 1) && lane == 0) misc[2] = 1;
-        }
+        // the MMAs of entry e - 2 (the last readers of this stage) have completed
+        if (e >= kStages && !mbar_wait(&q_empty[s], ((e / kStages) - 1) & 1) && lane == 0) misc[2] = 1;
         if (__any_sync(0xffffffffu, aborted())) continue;
         const int it = static_cast<int>(list[e] & 0xFFFFu);
         if (lane == 0) {
@@ -302,50 +335,78 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint64_t dq_mn = smem_desc(smem_addr(smem + L::kOffRing0), kHalfBytes, 1024);   // Q, MN-major B
       const uint64_t ddo_mn = smem_desc(smem_addr(smem + L::kOffRing1), kHalfBytes, 1024);  // dO, MN-major B
       constexpr uint64_t kStageStep = L::kTileBytes >> 4;
-      for (int e = 0; e < n_list; ++e) {
-        const int s = e % kStages;
-        // S^T / dP^T overwrite the columns the previous entry's dV / dK read
-        if (e > 0 && !__all_sync(0xffffffffu, mbar_wait(mma_done, (e - 1) & 1))) {
+      // S^T_hh, dP^T_hh of entry e: queries [64 hh, 64 hh + 64) = rows 64 hh.. of
+      // each 64-column slab of the Q / dO tile (8 KB into the slab)
+      auto issue_sdp = [&](int e, int hh) {
+        const uint64_t base = (e % kStages) * kStageStep + (static_cast<uint64_t>(hh * 64 * 128) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t off = static_cast<uint64_t>((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+          mma_ss_warp(tm_s + 64 * hh, dk_a + off, dq_k + base + off, kIdescH, kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t off = static_cast<uint64_t>((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+          mma_ss_warp(tm_dp + 64 * hh, dv_a + off, ddo_k + base + off, kIdescH, kk > 0 ? 1u : 0u);
+        }
+      };
+      // dV += P^T_hh dO_hh and dK += dS^T_hh Q_hh: K = the half's 64 queries
+      auto issue_grad = [&](int e, int hh) {
+        const uint64_t base = (e % kStages) * kStageStep;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t off = static_cast<uint64_t>((hh * 64 + kk * 16) * 128) >> 4;
+          const uint32_t acc = (e > 0 || hh > 0 || kk > 0) ? 1u : 0u;
+          mma_ts_warp(tm_dv, tm_s + 64 * hh + kk * 8, ddo_mn + base + off, kIdescG, acc);
+          mma_ts_warp(tm_dk, tm_dp + 64 * hh + kk * 8, dq_mn + base + off, kIdescG, acc);
+        }
+      };
+      auto wait_q = [&](int e) {
+        ok = __all_sync(0xffffffffu, ok && !aborted());
+        if (ok) {
+          ok = __all_sync(0xffffffffu, mbar_wait(&q_full[e % kStages], (e / kStages) & 1));
+          if (!ok && lane == 0) misc[2] = 1;
+        }
+        if (ok) tc_fence_after();
+      };
+      auto wait_half = [&](int hh, int e) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&half_done[hh], e & 1))) {
           if (lane == 0) misc[2] = 1;
           ok = false;
         }
         ok = __all_sync(0xffffffffu, ok && !aborted());
-        if (ok) {
-          ok = __all_sync(0xffffffffu, mbar_wait(&q_full[s], (e / kStages) & 1));
-          if (!ok && lane == 0) misc[2] = 1;
-        }
-        if (ok) {
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t off = static_cast<uint64_t>((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
-            mma_ss_warp(tm_s, dk_a + off, dq_k + s * kStageStep + off, kIdescS, kk > 0 ? 1u : 0u);
-          }
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t off = static_cast<uint64_t>((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
-            mma_ss_warp(tm_dp, dv_a + off, ddo_k + s * kStageStep + off, kIdescS, kk > 0 ? 1u : 0u);
-          }
-        }
-        mma_commit_warp(s_ready);   // also after an error, so that no waiter stalls
-        named_bar_sync(kBarBwdP, kBwdHandoff);
+        if (ok) tc_fence_after();
+      };
+      wait_q(0);
+      if (ok) issue_sdp(0, 0);
+      mma_commit_warp(&ready[0]);   // every commit also after an error, so that no waiter stalls
+      if (ok) issue_sdp(0, 1);
+      mma_commit_warp(&ready[1]);
+      for (int e = 0; e < n_list; ++e) {
+        named_bar_sync(kBarBwdA, kBwdHandoff);
         if (__all_sync(0xffffffffu, ok && !aborted())) {
           tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < kTileM / 16; ++kk) {
-            const uint64_t off = static_cast<uint64_t>(kk * 16 * 128) >> 4;
-            const uint32_t acc = (e > 0 || kk > 0) ? 1u : 0u;
-            mma_ts_warp(tm_dv, tm_s + kk * 8, ddo_mn + s * kStageStep + off, kIdescG, acc);
-          }
-#pragma unroll
-          for (int kk = 0; kk < kTileM / 16; ++kk) {
-            const uint64_t off = static_cast<uint64_t>(kk * 16 * 128) >> 4;
-            const uint32_t acc = (e > 0 || kk > 0) ? 1u : 0u;
-            mma_ts_warp(tm_dk, tm_dp + kk * 8, dq_mn + s * kStageStep + off, kIdescG, acc);
-          }
+          issue_grad(e, 0);
         }
-        mma_commit_warp(&q_empty[s]);
-        mma_commit_warp(mma_done);
+        mma_commit_warp(&half_done[0]);
+        if (e + 1 < n_list) {
+          wait_half(0, e);            // S^T_0 of e + 1 overwrites what the MMAs above read
+          wait_q(e + 1);
+          if (ok) issue_sdp(e + 1, 0);
+          mma_commit_warp(&ready[0]);
+        }
+        named_bar_sync(kBarBwdB, kBwdHandoff);
+        if (__all_sync(0xffffffffu, ok && !aborted())) {
+          tc_fence_after();
+          issue_grad(e, 1);
+        }
+        mma_commit_warp(&half_done[1]);
+        mma_commit_warp(&q_empty[e % kStages]);
+        if (e + 1 < n_list) {
+          wait_half(1, e);
+          if (ok) issue_sdp(e + 1, 1);
+          mma_commit_warp(&ready[1]);
+        }
       }
     }
   } else {
@@ -361,38 +422,33 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint32_t bits = list[e] >> 16;
       const int it = static_cast<int>(list[e] & 0xFFFFu);
       const int s = e % kStages;
-      if (!mbar_wait(s_ready, e & 1)) {
-        misc[2] = 1;
-        ok = false;
-      }
-      if (ok && !aborted() && !mbar_wait(&q_full[s], (e / kStages) & 1)) {
-        misc[2] = 1;
-        ok = false;
-      }
-      tc_fence_after();
       const float* vec = reinterpret_cast<const float*>(smem + L::kOffVec) + s * 256;
       const int valid_q = min(kTileM, p.N - it * kTileM);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        // chunk c: query columns [32c, 32c + 32) of q-block half c / 2
-        const int qh = BLK == 128 ? 0 : (c >> 1);
-        const bool quad = BLK == 128 ? true : ((bits >> (qh * 2 + kh)) & 1u);
-        const int nv = min(32, max(0, valid_q - 32 * c));
-        const uint32_t keep = (key_valid && quad) ? (nv == 32 ? 0xffffffffu : ((1u << nv) - 1u)) : 0u;
-        float sv[32], dp[32];
-        uint32_t pk[16], dsk[16];
-        tmem_ld32(tm_s + lane_off + 32 * c, sv);
-        tmem_ld32(tm_dp + lane_off + 32 * c, dp);
-        grad_chunk<true>(sv, dp, sl2, vec + 32 * c, vec + 128 + 32 * c, 0.f, 0.f, keep, pk, dsk);
-        tmem_st16(tm_s + lane_off + 16 * c, pk);
-        tmem_st16(tm_dp + lane_off + 16 * c, dsk);
+      for (int hh = 0; hh < 2; ++hh) {
+        if (!mbar_wait(&ready[hh], e & 1)) {
+          misc[2] = 1;
+          ok = false;
+        }
+        if (hh == 0 && ok && !aborted() && !mbar_wait(&q_full[s], (e / kStages) & 1)) {
+          misc[2] = 1;
+          ok = false;
+        }
+        tc_fence_after();
+        // half hh: query columns [64 hh, 64 hh + 64), q-block half hh for block 64
+        const bool quad = BLK == 128 ? true : ((bits >> (hh * 2 + kh)) & 1u);
+        const int nv0 = min(32, max(0, valid_q - 64 * hh)), nv1 = min(32, max(0, valid_q - 64 * hh - 32));
+        const uint32_t keep0 = (key_valid && quad) ? (nv0 == 32 ? 0xffffffffu : ((1u << nv0) - 1u)) : 0u;
+        const uint32_t keep1 = (key_valid && quad) ? (nv1 == 32 ? 0xffffffffu : ((1u << nv1) - 1u)) : 0u;
+        grad_half<true, true>(tm_s + lane_off, tm_dp + lane_off, tm_dp + lane_off, hh, sl2, vec, vec + 128, 0.f,
+                              0.f, keep0, keep1);
+        tmem_st_wait();
+        tc_fence_before();
+        named_bar_sync(hh == 0 ? kBarBwdA : kBarBwdB, kBwdHandoff);
       }
-      tmem_st_wait();
-      tc_fence_before();
-      named_bar_sync(kBarBwdP, kBwdHandoff);
     }
-    // epilogue: dV and dK rows of this thread's key
-    if (n_list > 0 && !mbar_wait(mma_done, (n_list - 1) & 1)) {
+    // epilogue: dV and dK rows of this thread's key, once the last MMAs completed
+    if (n_list > 0 && !mbar_wait(&half_done[1], (n_list - 1) & 1)) {
       misc[2] = 1;
       ok = false;
     }
@@ -412,8 +468,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 }
 
 // ----------------------------------------------------------------- dQ ---
-// CTA = (q-tile it, head bh).  TMEM columns: dQ [0, D), S [128, 256) (dS
-// packed to bf16 over its first 64 columns), dP [256, 384).
+// CTA = (q-tile it, head bh).  TMEM columns: dQ [0, D), S [128, 256) and
+// dP [256, 384), each in two 64-key halves; dS of a half is packed to bf16
+// over the half's first 32 S columns.  The same two-half pipeline as the
+// dK / dV kernel: S_h, dP_h (N = 64 keys), then dQ += dS_h K_h (K = 64).
 template <int D, int BLK>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -422,7 +480,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   using L = BwdSmem<D>;
   constexpr int QH = kTileM / BLK;
   constexpr int KH = kTileN / BLK;
-  constexpr uint32_t kIdescS = idesc_bf16_f32(kTileM, kTileN, false);
+  constexpr uint32_t kIdescH = idesc_bf16_f32(kTileM, 64, false);   // S / dP half: 128 queries x 64 keys
   constexpr uint32_t kIdescG = idesc_bf16_f32(kTileM, D, true);
   constexpr int kHalfBytes = kTileM * 128;
 
@@ -433,8 +491,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* qd_full = bars;
   uint64_t* kv_full = bars + 1;
   uint64_t* kv_empty = kv_full + kStages;
-  uint64_t* s_ready = kv_empty + kStages;
-  uint64_t* mma_done = s_ready + 1;
+  uint64_t* ready = kv_empty + kStages;
+  uint64_t* half_done = ready + 2;
   volatile int* misc = reinterpret_cast<volatile int*>(smem + L::kOffMisc);
   // misc[0] TMEM base, [1] list length, [2] abort flag
 
@@ -529,43 +587,76 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint64_t dv_k = smem_desc(smem_addr(smem + L::kOffRing1), 16, 1024);   // V, K-major B
       const uint64_t dk_mn = smem_desc(smem_addr(smem + L::kOffRing0), kHalfBytes, 1024);  // K, MN-major B
       constexpr uint64_t kStageStep = L::kTileBytes >> 4;
-      for (int e = 0; e < n_list; ++e) {
-        const int s = e % kStages;
-        // S / dP overwrite the columns the previous entry's dQ MMA read
-        if (e > 0 && !__all_sync(0xffffffffu, mbar_wait(mma_done, (e - 1) & 1))) {
+      // S_hh, dP_hh of entry e: keys [64 hh, 64 hh + 64) of its kv tile
+      auto issue_sdp = [&](int e, int hh) {
+        const uint64_t base = (e % kStages) * kStageStep + (static_cast<uint64_t>(hh * 64 * 128) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t off = static_cast<uint64_t>((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+          mma_ss_warp(tm_s + 64 * hh, dq_a + off, dk_k + base + off, kIdescH, kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t off = static_cast<uint64_t>((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+          mma_ss_warp(tm_dp + 64 * hh, ddo_a + off, dv_k + base + off, kIdescH, kk > 0 ? 1u : 0u);
+        }
+      };
+      // dQ += dS_hh K_hh: K = the half's 64 keys
+      auto issue_grad = [&](int e, int hh) {
+        const uint64_t base = (e % kStages) * kStageStep;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t off = static_cast<uint64_t>((hh * 64 + kk * 16) * 128) >> 4;
+          mma_ts_warp(tm_dq, tm_s + 64 * hh + kk * 8, dk_mn + base + off, kIdescG,
+                      (e > 0 || hh > 0 || kk > 0) ? 1u : 0u);
+        }
+      };
+      auto wait_kv = [&](int e) {
+        ok = __all_sync(0xffffffffu, ok && !aborted());
+        if (ok) {
+          ok = __all_sync(0xffffffffu, mbar_wait(&kv_full[e % kStages], (e / kStages) & 1));
+          if (!ok && lane == 0) misc[2] = 1;
+        }
+        if (ok) tc_fence_after();
+      };
+      auto wait_half = [&](int hh, int e) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&half_done[hh], e & 1))) {
           if (lane == 0) misc[2] = 1;
           ok = false;
         }
         ok = __all_sync(0xffffffffu, ok && !aborted());
-        if (ok) {
-          ok = __all_sync(0xffffffffu, mbar_wait(&kv_full[s], (e / kStages) & 1));
-          if (!ok && lane == 0) misc[2] = 1;
-        }
-        if (ok) {
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t off = static_cast<uint64_t>((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
-            mma_ss_warp(tm_s, dq_a + off, dk_k + s * kStageStep + off, kIdescS, kk > 0 ? 1u : 0u);
-          }
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t off = static_cast<uint64_t>((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
-            mma_ss_warp(tm_dp, ddo_a + off, dv_k + s * kStageStep + off, kIdescS, kk > 0 ? 1u : 0u);
-          }
-        }
-        mma_commit_warp(s_ready);   // also after an error, so that no waiter stalls
-        named_bar_sync(kBarBwdP, kBwdHandoff);
+        if (ok) tc_fence_after();
+      };
+      wait_kv(0);
+      if (ok) issue_sdp(0, 0);
+      mma_commit_warp(&ready[0]);   // every commit also after an error, so that no waiter stalls
+      if (ok) issue_sdp(0, 1);
+      mma_commit_warp(&ready[1]);
+      for (int e = 0; e < n_list; ++e) {
+        named_bar_sync(kBarBwdA, kBwdHandoff);
         if (__all_sync(0xffffffffu, ok && !aborted())) {
           tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < kTileN / 16; ++kk) {
-            const uint64_t off = static_cast<uint64_t>(kk * 16 * 128) >> 4;
-            mma_ts_warp(tm_dq, tm_s + kk * 8, dk_mn + s * kStageStep + off, kIdescG, (e > 0 || kk > 0) ? 1u : 0u);
-          }
+          issue_grad(e, 0);
         }
-        mma_commit_warp(&kv_empty[s]);
-        mma_commit_warp(mma_done);
+        mma_commit_warp(&half_done[0]);
+        if (e + 1 < n_list) {
+          wait_half(0, e);            // S_0 of e + 1 overwrites what the MMAs above read
+          wait_kv(e + 1);
+          if (ok) issue_sdp(e + 1, 0);
+          mma_commit_warp(&ready[0]);
+        }
+        named_bar_sync(kBarBwdB, kBwdHandoff);
+        if (__all_sync(0xffffffffu, ok && !aborted())) {
+          tc_fence_after();
+          issue_grad(e, 1);
+        }
+        mma_commit_warp(&half_done[1]);
+        mma_commit_warp(&kv_empty[e % kStages]);
+        if (e + 1 < n_list) {
+          wait_half(1, e);
+          if (ok) issue_sdp(e + 1, 1);
+          mma_commit_warp(&ready[1]);
+        }
       }
     }
   } else {
@@ -583,31 +674,27 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int e = 0; e < n_list; ++e) {
       const uint32_t bits = list[e] >> 16;
       const int jt = static_cast<int>(list[e] & 0xFFFFu);
-      if (!mbar_wait(s_ready, e & 1)) {
-        misc[2] = 1;
-        ok = false;
-      }
-      tc_fence_after();
       const int valid_k = min(kTileN, p.N - jt * kTileN);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        // chunk c: key columns [32c, 32c + 32) of k-block half c / 2
-        const int kh = BLK == 128 ? 0 : (c >> 1);
-        const bool quad = BLK == 128 ? true : ((bits >> (qh * 2 + kh)) & 1u);
-        const int nv = min(32, max(0, valid_k - 32 * c));
-        const uint32_t keep = (row_valid && quad) ? (nv == 32 ? 0xffffffffu : ((1u << nv) - 1u)) : 0u;
-        float sv[32], dp[32];
-        uint32_t pk[16], dsk[16];
-        tmem_ld32(tm_s + lane_off + 32 * c, sv);
-        tmem_ld32(tm_dp + lane_off + 32 * c, dp);
-        grad_chunk<false>(sv, dp, sl2, nullptr, nullptr, l2, dl, keep, pk, dsk);
-        tmem_st16(tm_s + lane_off + 16 * c, dsk);
+      for (int hh = 0; hh < 2; ++hh) {
+        if (!mbar_wait(&ready[hh], e & 1)) {
+          misc[2] = 1;
+          ok = false;
+        }
+        tc_fence_after();
+        // half hh: key columns [64 hh, 64 hh + 64), k-block half hh for block 64
+        const bool quad = BLK == 128 ? true : ((bits >> (qh * 2 + hh)) & 1u);
+        const int nv0 = min(32, max(0, valid_k - 64 * hh)), nv1 = min(32, max(0, valid_k - 64 * hh - 32));
+        const uint32_t keep0 = (row_valid && quad) ? (nv0 == 32 ? 0xffffffffu : ((1u << nv0) - 1u)) : 0u;
+        const uint32_t keep1 = (row_valid && quad) ? (nv1 == 32 ? 0xffffffffu : ((1u << nv1) - 1u)) : 0u;
+        grad_half<false, false>(tm_s + lane_off, tm_dp + lane_off, tm_s + lane_off, hh, sl2, nullptr, nullptr, l2,
+                                dl, keep0, keep1);
+        tmem_st_wait();
+        tc_fence_before();
+        named_bar_sync(hh == 0 ? kBarBwdA : kBarBwdB, kBwdHandoff);
       }
-      tmem_st_wait();
-      tc_fence_before();
-      named_bar_sync(kBarBwdP, kBwdHandoff);
     }
-    if (n_list > 0 && !mbar_wait(mma_done, (n_list - 1) & 1)) {
+    if (n_list > 0 && !mbar_wait(&half_done[1], (n_list - 1) & 1)) {
       misc[2] = 1;
       ok = false;
     }

@@ -313,6 +313,39 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float* v) {
 #undef SA_R8
 }
 
+// Two 32 lanes x 32 columns loads (columns at a0 and at a1), not waited: the
+// registers are valid only after tmem_ld_wait2 on the same arrays.
+__device__ __forceinline__ void tmem_ld32x2_nowait(uint32_t a0, uint32_t a1, float* v0, float* v1) {
+  uint32_t* r = reinterpret_cast<uint32_t*>(v0);
+  uint32_t* q = reinterpret_cast<uint32_t*>(v1);
+#define SA_R8(x, b) "=r"(x[b]), "=r"(x[b + 1]), "=r"(x[b + 2]), "=r"(x[b + 3]), "=r"(x[b + 4]), "=r"(x[b + 5]), \
+                    "=r"(x[b + 6]), "=r"(x[b + 7])
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%64];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, "
+      "%45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%65];"
+      : SA_R8(r, 0), SA_R8(r, 8), SA_R8(r, 16), SA_R8(r, 24), SA_R8(q, 0), SA_R8(q, 8), SA_R8(q, 16), SA_R8(q, 24)
+      : "r"(a0), "r"(a1)
+      : "memory");
+#undef SA_R8
+}
+
+// Wait for this thread's outstanding TMEM loads.  The 64 registers of v0 / v1
+// are tied to the wait so that the compiler moves no use of them above it.
+__device__ __forceinline__ void tmem_ld_wait2(float* v0, float* v1) {
+  uint32_t* r = reinterpret_cast<uint32_t*>(v0);
+  uint32_t* q = reinterpret_cast<uint32_t*>(v1);
+#define SA_T8(x, b) "+r"(x[b]), "+r"(x[b + 1]), "+r"(x[b + 2]), "+r"(x[b + 3]), "+r"(x[b + 4]), "+r"(x[b + 5]), \
+                    "+r"(x[b + 6]), "+r"(x[b + 7])
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : SA_T8(r, 0), SA_T8(r, 8), SA_T8(r, 16), SA_T8(r, 24), SA_T8(q, 0), SA_T8(q, 8), SA_T8(q, 16),
+                 SA_T8(q, 24)
+               :
+               : "memory");
+#undef SA_T8
+}
+
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));

@@ -5,6 +5,7 @@
     python -m block_sparse_attention_flash_b200.profile_case mask   [--heads 12] [--reps 2]
     python -m block_sparse_attention_flash_b200.profile_case pool   [--heads 12] [--reps 2]
     python -m block_sparse_attention_flash_b200.profile_case pyr    [--heads 2] [--reps 2]
+    python -m block_sparse_attention_flash_b200.profile_case bwd    [--heads 2] [--reps 2]
 
 Each case uses a workload's real token grid with fewer heads, so one launch
 holds a few hundred MB (larger than L2) and a full profiler capture ends in
@@ -14,6 +15,7 @@ seconds.  Inputs are drawn on the device from the seeded generator.
   mask    32,760-token 480p grid, block 64, tau = 0.9
   pool    32,760-token 480p grid, block 64
   pyr     32,760-token 480p grid, block 64, PSA levels from the GPU level builder
+  bwd     32,760-token 480p grid, block 64, all kept: forward once, then the backward
 """
 from __future__ import annotations
 
@@ -26,7 +28,7 @@ from . import build, inputs, ops
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["attn", "radial", "mask", "pool", "pyr"])
+    ap.add_argument("case", choices=["attn", "radial", "mask", "pool", "pyr", "bwd"])
     ap.add_argument("--heads", type=int, default=0)
     ap.add_argument("--reps", type=int, default=2)
     args = ap.parse_args()
@@ -54,6 +56,15 @@ def main():
         _, k, v = inputs.rff_qkv(wl, H=args.heads or wl.H, device=dev)
         for _ in range(args.reps):
             ops.sa_pyramid_pool(k, v, wl.block)
+    elif args.case == "bwd":
+        wl = inputs.WORKLOADS["wan13b_480p_tau"]
+        q, k, v = inputs.rff_qkv(wl, H=args.heads or 2, device=dev)
+        g = torch.Generator(device=dev).manual_seed(wl.seed + 7)
+        dout = torch.randn(q.shape, generator=g, device=dev).to(torch.bfloat16)
+        lse = torch.empty(q.shape[:3], device=dev)
+        o = ops.sa_sparse_attn_fwd(q, k, v, wl.block, lse=lse)
+        for _ in range(args.reps):
+            ops.sa_sparse_attn_bwd(q, k, v, o, dout, lse, wl.block)
     else:
         wl = inputs.WORKLOADS["psa_480p_pyramid"]
         q, k, v = inputs.rff_qkv(wl, H=args.heads or 2, device=dev)
