@@ -23,14 +23,16 @@
 // K-major B operand (Q in S^T, K in S) and as an MN-major B operand (Q in dK,
 // dO in dV, K in dQ).
 //
-// Roles (192 threads = 6 warps, one CTA per SM for the TMEM it holds):
+// Roles (320 threads = 10 warps, one CTA per SM for the TMEM it holds):
 //   warps 0-3   one thread per row of the CTA's tile (key row in dK/dV, query
-//               row in dQ): P and dS from the TMEM rows, the epilogue;
-//   warp 4      builds the tile list from the mask, issues the TMA loads
+//               row in dQ): P and dS of the first 64-column half of each S;
+//   warps 4-7   the same rows, second half (the two halves run concurrently);
+//               both warpgroups share the epilogue;
+//   warp 8      builds the tile list from the mask, issues the TMA loads
 //               (2-stage ring) and stages the per-query LSE / D vectors;
-//   warp 5      allocates TMEM and issues every MMA (warp-wide, one elected lane).
+//   warp 9      allocates TMEM and issues every MMA (warp-wide, one elected lane).
 // Hand-offs: tcgen05.commit to mbarriers from the MMA warp; one named barrier
-// (warps 0-3 + warp 5) when P / dS are in TMEM.  Every party runs the full,
+// per half (its warpgroup + warp 9) when that half's P / dS are in TMEM.  Every party runs the full,
 // list-determined sequence of syncs, also after an error (skipping only its
 // loads and MMAs), and every mbarrier wait is bounded.
 #pragma once
@@ -39,11 +41,12 @@
 
 namespace sa {
 
-constexpr int kBwdWarps = 6;
+constexpr int kBwdWarps = 10;
 constexpr int kBwdThreads = kBwdWarps * 32;
-constexpr int kBwdLoadWarp = 4;
-constexpr int kBwdMmaWarp = 5;
-// P / dS of the first / second 64-column half packed in TMEM: warps 0-3 <-> MMA warp
+constexpr int kBwdLoadWarp = 8;
+constexpr int kBwdMmaWarp = 9;
+// P / dS of the first / second 64-column half packed in TMEM: warps 0-3 /
+// warps 4-7 <-> MMA warp
 constexpr int kBarBwdA = 1;
 constexpr int kBarBwdB = 2;
 constexpr int kBwdHandoff = 160;
@@ -102,8 +105,8 @@ struct BwdSmem {
   static constexpr int kOffRing1 = kOffRing0 + kStages * kTileBytes;    // [stage]
   static constexpr int kOffVec = kOffRing1 + kStages * kTileBytes;      // [stage][2][128] f32
   static constexpr int kOffList = kOffVec + kStages * 2 * 128 * 4;
-  // fix_full, ring_full[2], ring_empty[2], ready_a, ready_b, half_a_done, half_b_done
-  static constexpr int kNumBars = 1 + 2 * kStages + 4;
+  // fix_full, ring_full[2], ring_empty[2], ready[2], half_done[2], final_done
+  static constexpr int kNumBars = 1 + 2 * kStages + 5;
   static constexpr int kOffBar = kOffList + kMaxKvTiles * 4;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffMisc + 64;
@@ -200,10 +203,10 @@ __device__ __forceinline__ void store_row(uint32_t taddr, float mul, __nv_bfloat
 // S^T [2D, 2D + 128) and dP^T [2D + 128, 2D + 256), each in two 64-query
 // halves; P^T / dS^T of a half are packed to bf16 over the half's first 32
 // columns.  Per entry (q-tile) the MMA warp issues, for each half: S^T_h and
-// dP^T_h (N = 64), and once warps 0-3 have packed the half, dV += P^T_h dO_h
+// dP^T_h (N = 64), and once its warpgroup has packed the half, dV += P^T_h dO_h
 // and dK += dS^T_h Q_h (K = 64).  The next entry's S^T_h goes into a half as
 // soon as the gradient MMAs that read it have completed, so one half's MMAs
-// run while warps 0-3 work on the other.
+// run while the warpgroups work on the halves.
 template <int D, int BLK>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -225,6 +228,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* q_empty = q_full + kStages;
   uint64_t* ready = q_empty + kStages;       // [2]: S^T_h and dP^T_h of the current entry computed
   uint64_t* half_done = ready + 2;           // [2]: the gradient MMAs of half h completed
+  uint64_t* final_done = half_done + 2;
   volatile int* misc = reinterpret_cast<volatile int*>(smem + L::kOffMisc);
   // misc[0] TMEM base, [1] list length, [2] abort flag
 
@@ -294,10 +298,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       for (int e = 0; e < n_list; ++e) {
         const int s = e % kStages;
+        const int it = static_cast<int>(list[e] & 0xFFFFu);
+        // per-query vectors of the tile, read before the wait for the stage:
+        // lse * log2(e) (+inf past N) and D
+        float lv[4], dv4[4];
+        const size_t rbase = static_cast<size_t>(bh) * p.N;
+#pragma unroll
+        for (int k4 = 0; k4 < 4; ++k4) {
+          const int row = it * kTileM + k4 * 32 + lane;
+          const bool valid = row < p.N;
+          lv[k4] = valid ? p.lse[rbase + row] * 1.4426950408889634f : __int_as_float(0x7f800000);
+          dv4[k4] = valid ? p.delta[rbase + row] : 0.f;
+        }
         // the MMAs of entry e - 2 (the last readers of this stage) have completed
         if (e >= kStages && !mbar_wait(&q_empty[s], ((e / kStages) - 1) & 1) && lane == 0) misc[2] = 1;
         if (__any_sync(0xffffffffu, aborted())) continue;
-        const int it = static_cast<int>(list[e] & 0xFFFFu);
         if (lane == 0) {
           mbar_arrive_expect_tx(&q_full[s], 2 * L::kTileBytes);
 #pragma unroll
@@ -308,16 +323,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                         it * kTileM, bh);
           }
         }
-        // per-query vectors of the tile: lse * log2(e) (+inf past N) and D
         float* vec = reinterpret_cast<float*>(smem + L::kOffVec) + s * 256;
-        const size_t rbase = static_cast<size_t>(bh) * p.N;
 #pragma unroll
         for (int k4 = 0; k4 < 4; ++k4) {
-          const int r = k4 * 32 + lane;
-          const int row = it * kTileM + r;
-          const bool valid = row < p.N;
-          vec[r] = valid ? p.lse[rbase + row] * 1.4426950408889634f : __int_as_float(0x7f800000);
-          vec[128 + r] = valid ? p.delta[rbase + row] : 0.f;
+          vec[k4 * 32 + lane] = lv[k4];
+          vec[128 + k4 * 32 + lane] = dv4[k4];
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&q_full[s]);
@@ -382,6 +392,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mma_commit_warp(&ready[0]);   // every commit also after an error, so that no waiter stalls
       if (ok) issue_sdp(0, 1);
       mma_commit_warp(&ready[1]);
+      // Per half: once its warpgroup has packed it, the gradient MMAs; once
+      // those have completed (they read the half's columns), the next
+      // entry's S / dP of the half.  The other half's MMAs keep the pipe busy
+      // while this warp waits.
       for (int e = 0; e < n_list; ++e) {
         named_bar_sync(kBarBwdA, kBwdHandoff);
         if (__all_sync(0xffffffffu, ok && !aborted())) {
@@ -390,7 +404,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         mma_commit_warp(&half_done[0]);
         if (e + 1 < n_list) {
-          wait_half(0, e);            // S^T_0 of e + 1 overwrites what the MMAs above read
+          wait_half(0, e);
           wait_q(e + 1);
           if (ok) issue_sdp(e + 1, 0);
           mma_commit_warp(&ready[0]);
@@ -408,11 +422,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           mma_commit_warp(&ready[1]);
         }
       }
+      mma_commit_warp(final_done);   // every MMA of the CTA has completed
     }
   } else {
-    // --------------------------------------- P^T, dS^T and the epilogue ---
-    const int r = threadIdx.x;                       // key row of the kv tile
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    // ------------------------------- P^T, dS^T of one half; the epilogue ---
+    const int hh = warp >> 2;                        // half of each S^T this warpgroup packs
+    const int r = (warp & 3) * 32 + lane;            // key row of the kv tile
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const int key = jt * kTileN + r;
     const bool key_valid = key < p.N;
     const int kh = BLK == 128 ? 0 : (r >> 6);
@@ -424,39 +440,38 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int s = e % kStages;
       const float* vec = reinterpret_cast<const float*>(smem + L::kOffVec) + s * 256;
       const int valid_q = min(kTileM, p.N - it * kTileM);
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        if (!mbar_wait(&ready[hh], e & 1)) {
-          misc[2] = 1;
-          ok = false;
-        }
-        if (hh == 0 && ok && !aborted() && !mbar_wait(&q_full[s], (e / kStages) & 1)) {
-          misc[2] = 1;
-          ok = false;
-        }
-        tc_fence_after();
-        // half hh: query columns [64 hh, 64 hh + 64), q-block half hh for block 64
-        const bool quad = BLK == 128 ? true : ((bits >> (hh * 2 + kh)) & 1u);
-        const int nv0 = min(32, max(0, valid_q - 64 * hh)), nv1 = min(32, max(0, valid_q - 64 * hh - 32));
-        const uint32_t keep0 = (key_valid && quad) ? (nv0 == 32 ? 0xffffffffu : ((1u << nv0) - 1u)) : 0u;
-        const uint32_t keep1 = (key_valid && quad) ? (nv1 == 32 ? 0xffffffffu : ((1u << nv1) - 1u)) : 0u;
-        grad_half<true, true>(tm_s + lane_off, tm_dp + lane_off, tm_dp + lane_off, hh, sl2, vec, vec + 128, 0.f,
-                              0.f, keep0, keep1);
-        tmem_st_wait();
-        tc_fence_before();
-        named_bar_sync(hh == 0 ? kBarBwdA : kBarBwdB, kBwdHandoff);
+      if (!mbar_wait(&ready[hh], e & 1)) {
+        misc[2] = 1;
+        ok = false;
       }
+      if (ok && !aborted() && !mbar_wait(&q_full[s], (e / kStages) & 1)) {
+        misc[2] = 1;
+        ok = false;
+      }
+      tc_fence_after();
+      // half hh: query columns [64 hh, 64 hh + 64), q-block half hh for block 64
+      const bool quad = BLK == 128 ? true : ((bits >> (hh * 2 + kh)) & 1u);
+      const int nv0 = min(32, max(0, valid_q - 64 * hh)), nv1 = min(32, max(0, valid_q - 64 * hh - 32));
+      const uint32_t keep0 = (key_valid && quad) ? (nv0 == 32 ? 0xffffffffu : ((1u << nv0) - 1u)) : 0u;
+      const uint32_t keep1 = (key_valid && quad) ? (nv1 == 32 ? 0xffffffffu : ((1u << nv1) - 1u)) : 0u;
+      grad_half<true, true>(tm_s + lane_off, tm_dp + lane_off, tm_dp + lane_off, hh, sl2, vec, vec + 128, 0.f, 0.f,
+                            keep0, keep1);
+      tmem_st_wait();
+      tc_fence_before();
+      named_bar_sync(hh == 0 ? kBarBwdA : kBarBwdB, kBwdHandoff);
     }
-    // epilogue: dV and dK rows of this thread's key, once the last MMAs completed
-    if (n_list > 0 && !mbar_wait(&half_done[1], (n_list - 1) & 1)) {
+    // epilogue: warps 0-3 write dV, warps 4-7 dK, once every MMA has completed
+    if (n_list > 0 && !mbar_wait(final_done, 0)) {
       misc[2] = 1;
       ok = false;
     }
     tc_fence_after();
     if (n_list == 0 || __all_sync(0xffffffffu, ok && !aborted())) {
       const size_t off = (static_cast<size_t>(bh) * p.N + (key_valid ? key : 0)) * D;
-      store_row<D>(tm_dv + lane_off, 1.f, p.dv + off, n_list == 0, key_valid);
-      store_row<D>(tm_dk + lane_off, p.scale, p.dk + off, n_list == 0, key_valid);
+      if (hh == 0)
+        store_row<D>(tm_dv + lane_off, 1.f, p.dv + off, n_list == 0, key_valid);
+      else
+        store_row<D>(tm_dk + lane_off, p.scale, p.dk + off, n_list == 0, key_valid);
     }
   }
   tc_fence_before();
@@ -493,6 +508,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* kv_empty = kv_full + kStages;
   uint64_t* ready = kv_empty + kStages;
   uint64_t* half_done = ready + 2;
+  uint64_t* final_done = half_done + 2;
   volatile int* misc = reinterpret_cast<volatile int*>(smem + L::kOffMisc);
   // misc[0] TMEM base, [1] list length, [2] abort flag
 
@@ -632,6 +648,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mma_commit_warp(&ready[0]);   // every commit also after an error, so that no waiter stalls
       if (ok) issue_sdp(0, 1);
       mma_commit_warp(&ready[1]);
+      // Per half: once its warpgroup has packed it, the gradient MMAs; once
+      // those have completed (they read the half's columns), the next
+      // entry's S / dP of the half.  The other half's MMAs keep the pipe busy
+      // while this warp waits.
       for (int e = 0; e < n_list; ++e) {
         named_bar_sync(kBarBwdA, kBwdHandoff);
         if (__all_sync(0xffffffffu, ok && !aborted())) {
@@ -640,7 +660,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         mma_commit_warp(&half_done[0]);
         if (e + 1 < n_list) {
-          wait_half(0, e);            // S_0 of e + 1 overwrites what the MMAs above read
+          wait_half(0, e);
           wait_kv(e + 1);
           if (ok) issue_sdp(e + 1, 0);
           mma_commit_warp(&ready[0]);
@@ -658,11 +678,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           mma_commit_warp(&ready[1]);
         }
       }
+      mma_commit_warp(final_done);   // every MMA of the CTA has completed
     }
   } else {
-    // ------------------------------------------------ dS and the epilogue ---
-    const int r = threadIdx.x;                       // query row of the q-tile
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    // ---------------------------------------- dS of one half; the epilogue ---
+    const int hh = warp >> 2;                        // half of each S this warpgroup packs
+    const int r = (warp & 3) * 32 + lane;            // query row of the q-tile
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const int row = it * kTileM + r;
     const bool row_valid = row < p.N;
     const int qh = BLK == 128 ? 0 : (r >> 6);
@@ -675,32 +697,31 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint32_t bits = list[e] >> 16;
       const int jt = static_cast<int>(list[e] & 0xFFFFu);
       const int valid_k = min(kTileN, p.N - jt * kTileN);
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        if (!mbar_wait(&ready[hh], e & 1)) {
-          misc[2] = 1;
-          ok = false;
-        }
-        tc_fence_after();
-        // half hh: key columns [64 hh, 64 hh + 64), k-block half hh for block 64
-        const bool quad = BLK == 128 ? true : ((bits >> (qh * 2 + hh)) & 1u);
-        const int nv0 = min(32, max(0, valid_k - 64 * hh)), nv1 = min(32, max(0, valid_k - 64 * hh - 32));
-        const uint32_t keep0 = (row_valid && quad) ? (nv0 == 32 ? 0xffffffffu : ((1u << nv0) - 1u)) : 0u;
-        const uint32_t keep1 = (row_valid && quad) ? (nv1 == 32 ? 0xffffffffu : ((1u << nv1) - 1u)) : 0u;
-        grad_half<false, false>(tm_s + lane_off, tm_dp + lane_off, tm_s + lane_off, hh, sl2, nullptr, nullptr, l2,
-                                dl, keep0, keep1);
-        tmem_st_wait();
-        tc_fence_before();
-        named_bar_sync(hh == 0 ? kBarBwdA : kBarBwdB, kBwdHandoff);
+      if (!mbar_wait(&ready[hh], e & 1)) {
+        misc[2] = 1;
+        ok = false;
       }
+      tc_fence_after();
+      // half hh: key columns [64 hh, 64 hh + 64), k-block half hh for block 64
+      const bool quad = BLK == 128 ? true : ((bits >> (qh * 2 + hh)) & 1u);
+      const int nv0 = min(32, max(0, valid_k - 64 * hh)), nv1 = min(32, max(0, valid_k - 64 * hh - 32));
+      const uint32_t keep0 = (row_valid && quad) ? (nv0 == 32 ? 0xffffffffu : ((1u << nv0) - 1u)) : 0u;
+      const uint32_t keep1 = (row_valid && quad) ? (nv1 == 32 ? 0xffffffffu : ((1u << nv1) - 1u)) : 0u;
+      grad_half<false, false>(tm_s + lane_off, tm_dp + lane_off, tm_s + lane_off, hh, sl2, nullptr, nullptr, l2, dl,
+                              keep0, keep1);
+      tmem_st_wait();
+      tc_fence_before();
+      named_bar_sync(hh == 0 ? kBarBwdA : kBarBwdB, kBwdHandoff);
     }
-    if (n_list > 0 && !mbar_wait(&half_done[1], (n_list - 1) & 1)) {
+    // epilogue: warps 0-3 write dQ columns [0, D/2), warps 4-7 [D/2, D)
+    if (n_list > 0 && !mbar_wait(final_done, 0)) {
       misc[2] = 1;
       ok = false;
     }
     tc_fence_after();
     if (n_list == 0 || __all_sync(0xffffffffu, ok && !aborted())) {
-      store_row<D>(tm_dq + lane_off, p.scale, p.dq + rix * D, n_list == 0, row_valid);
+      store_row<D / 2>(tm_dq + lane_off + hh * (D / 2), p.scale, p.dq + rix * D + hh * (D / 2), n_list == 0,
+                       row_valid);
     }
   }
   tc_fence_before();
