@@ -97,7 +97,7 @@ template <int D>
 struct BwdSmem {
   static constexpr int kTileBytes = kTileM * D * 2;
   // dK/dV kernel: K, V of the CTA's kv tile, then a ring of Q / dO tiles with
-  // their [lse2 | D] vectors (2 x 128 fp32 per stage).
+  // their [-lse * log2(e) | D] vectors (2 x 128 fp32 per stage).
   // dQ kernel: Q, dO of the CTA's q-tile, then a ring of K / V tiles.
   static constexpr int kOffFix0 = 0;
   static constexpr int kOffFix1 = kTileBytes;
@@ -105,42 +105,62 @@ struct BwdSmem {
   static constexpr int kOffRing1 = kOffRing0 + kStages * kTileBytes;    // [stage]
   static constexpr int kOffVec = kOffRing1 + kStages * kTileBytes;      // [stage][2][128] f32
   static constexpr int kOffList = kOffVec + kStages * 2 * 128 * 4;
-  // fix_full, ring_full[2], ring_empty[2], ready[2], half_done[2], final_done
-  static constexpr int kNumBars = 1 + 2 * kStages + 5;
+  // fix_full, ring_full[2], ring_empty[2], ready[2], half_done[2], final_done,
+  // fix_tmem (dQ kernel: Q and dO copied into TMEM)
+  static constexpr int kNumBars = 1 + 2 * kStages + 6;
   static constexpr int kOffBar = kOffList + kMaxKvTiles * 4;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffMisc + 64;
   static constexpr int kAlloc = kBytes + 1024;
 };
 
-// p = 2^(s * sl2 - l2) on kept columns (0 elsewhere), ds = p * (dp - dl), for
-// 32 columns; both packed to bf16 pairs.  l2 / dl are per column (dK/dV
-// kernel, pointers into shared memory) or per row (dQ kernel, l2s / dls).
-template <bool kPerColumn>
-__device__ __forceinline__ void grad_chunk(const float* sv, const float* dp, float sl2, const float* l2,
-                                           const float* dl, float l2s, float dls, uint32_t keep_bits,
+// p = 2^(s * sl2 + nl) on kept columns (0 elsewhere), ds = p * (dp - dl), for
+// 32 columns; both packed to bf16 pairs.  nl = -lse * log2(e) and dl = D are
+// per column (dK/dV kernel: pointers into shared memory, 16-byte aligned) or
+// per row (dQ kernel: nls / dls).  kAll: every column kept (no selects).
+template <bool kPerColumn, bool kAll>
+__device__ __forceinline__ void grad_chunk(const float* sv, const float* dp, float sl2, const float* nl,
+                                           const float* dl, float nls, float dls, uint32_t keep_bits,
                                            uint32_t* pk, uint32_t* dk) {
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    float x0, x1, d0, d1;
+  for (int q = 0; q < 8; ++q) {
+    float x[4], g[4], pv[4];
     if (kPerColumn) {
-      const float2 l = reinterpret_cast<const float2*>(l2)[i];
-      const float2 g = reinterpret_cast<const float2*>(dl)[i];
-      x0 = fmaf(sv[2 * i], sl2, -l.x);
-      x1 = fmaf(sv[2 * i + 1], sl2, -l.y);
-      d0 = g.x;
-      d1 = g.y;
+      const float4 l4 = reinterpret_cast<const float4*>(nl)[q];
+      const float4 g4 = reinterpret_cast<const float4*>(dl)[q];
+      x[0] = fmaf(sv[4 * q + 0], sl2, l4.x);
+      x[1] = fmaf(sv[4 * q + 1], sl2, l4.y);
+      x[2] = fmaf(sv[4 * q + 2], sl2, l4.z);
+      x[3] = fmaf(sv[4 * q + 3], sl2, l4.w);
+      g[0] = g4.x;
+      g[1] = g4.y;
+      g[2] = g4.z;
+      g[3] = g4.w;
     } else {
-      x0 = fmaf(sv[2 * i], sl2, -l2s);
-      x1 = fmaf(sv[2 * i + 1], sl2, -l2s);
-      d0 = dls;
-      d1 = dls;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        x[j] = fmaf(sv[4 * q + j], sl2, nls);
+        g[j] = dls;
+      }
     }
-    const float p0 = ((keep_bits >> (2 * i)) & 1u) ? fast_exp2(x0) : 0.f;
-    const float p1 = ((keep_bits >> (2 * i + 1)) & 1u) ? fast_exp2(x1) : 0.f;
-    pk[i] = pack_bf16x2(p0, p1);
-    dk[i] = pack_bf16x2(p0 * (dp[2 * i] - d0), p1 * (dp[2 * i + 1] - d1));
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      pv[j] = (kAll || ((keep_bits >> (4 * q + j)) & 1u)) ? fast_exp2(x[j]) : 0.f;
+    pk[2 * q] = pack_bf16x2(pv[0], pv[1]);
+    pk[2 * q + 1] = pack_bf16x2(pv[2], pv[3]);
+    dk[2 * q] = pack_bf16x2(pv[0] * (dp[4 * q] - g[0]), pv[1] * (dp[4 * q + 1] - g[1]));
+    dk[2 * q + 1] = pack_bf16x2(pv[2] * (dp[4 * q + 2] - g[2]), pv[3] * (dp[4 * q + 3] - g[3]));
   }
+}
+
+template <bool kPerColumn>
+__device__ __forceinline__ void grad_chunk_any(const float* sv, const float* dp, float sl2, const float* nl,
+                                               const float* dl, float nls, float dls, uint32_t keep_bits,
+                                               uint32_t* pk, uint32_t* dk) {
+  if (keep_bits == 0xffffffffu)
+    grad_chunk<kPerColumn, true>(sv, dp, sl2, nl, dl, nls, dls, keep_bits, pk, dk);
+  else
+    grad_chunk<kPerColumn, false>(sv, dp, sl2, nl, dl, nls, dls, keep_bits, pk, dk);
 }
 
 // Half hh (columns [64 hh, 64 hh + 64)) of this thread's S and dP rows: P
@@ -158,13 +178,13 @@ __device__ __forceinline__ void grad_half(uint32_t ts, uint32_t tdp, uint32_t ds
   tmem_ld32x2_nowait(cs, cd, s0, d0);
   tmem_ld_wait2(s0, d0);
   tmem_ld32x2_nowait(cs + 32, cd + 32, s1, d1);
-  grad_chunk<kPerColumn>(s0, d0, sl2, kPerColumn ? l2 + 64 * hh : nullptr, kPerColumn ? dl + 64 * hh : nullptr,
-                         l2s, dls, keep0, pk, dk);
+  grad_chunk_any<kPerColumn>(s0, d0, sl2, kPerColumn ? l2 + 64 * hh : nullptr,
+                             kPerColumn ? dl + 64 * hh : nullptr, l2s, dls, keep0, pk, dk);
   if (kStoreP) tmem_st16(cs, pk);
   tmem_st16(cq, dk);
   tmem_ld_wait2(s1, d1);
-  grad_chunk<kPerColumn>(s1, d1, sl2, kPerColumn ? l2 + 64 * hh + 32 : nullptr,
-                         kPerColumn ? dl + 64 * hh + 32 : nullptr, l2s, dls, keep1, pk, dk);
+  grad_chunk_any<kPerColumn>(s1, d1, sl2, kPerColumn ? l2 + 64 * hh + 32 : nullptr,
+                             kPerColumn ? dl + 64 * hh + 32 : nullptr, l2s, dls, keep1, pk, dk);
   if (kStoreP) tmem_st16(cs + 16, pk);
   tmem_st16(cq + 16, dk);
 }
@@ -300,14 +320,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int s = e % kStages;
         const int it = static_cast<int>(list[e] & 0xFFFFu);
         // per-query vectors of the tile, read before the wait for the stage:
-        // lse * log2(e) (+inf past N) and D
+        // -lse * log2(e) (-inf past N) and D
         float lv[4], dv4[4];
         const size_t rbase = static_cast<size_t>(bh) * p.N;
 #pragma unroll
         for (int k4 = 0; k4 < 4; ++k4) {
           const int row = it * kTileM + k4 * 32 + lane;
           const bool valid = row < p.N;
-          lv[k4] = valid ? p.lse[rbase + row] * 1.4426950408889634f : __int_as_float(0x7f800000);
+          lv[k4] = valid ? p.lse[rbase + row] * -1.4426950408889634f : -__int_as_float(0x7f800000);
           dv4[k4] = valid ? p.delta[rbase + row] : 0.f;
         }
         // the MMAs of entry e - 2 (the last readers of this stage) have completed
@@ -485,7 +505,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 // ----------------------------------------------------------------- dQ ---
 // CTA = (q-tile it, head bh).  TMEM columns: dQ [0, D), S [128, 256) and
 // dP [256, 384), each in two 64-key halves; dS of a half is packed to bf16
-// over the half's first 32 S columns.  The same two-half pipeline as the
+// over the half's first 32 S columns; Q and dO as bf16 pairs at [384, 384 +
+// D/2) and [384 + D/2, 384 + D), copied there once per CTA from the TMA
+// tiles, so that S_h = Q K_h^T and dP_h = dO V_h^T read only K_h / V_h from
+// shared memory (an N = 64 MMA with both operands in shared memory is bound
+// by the shared-memory bandwidth).  The same two-half pipeline as the
 // dK / dV kernel: S_h, dP_h (N = 64 keys), then dQ += dS_h K_h (K = 64).
 template <int D, int BLK>
 __global__ void __launch_bounds__(kBwdThreads, 1)
@@ -509,6 +533,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* ready = kv_empty + kStages;
   uint64_t* half_done = ready + 2;
   uint64_t* final_done = half_done + 2;
+  uint64_t* qd_tmem = final_done + 1;        // Q and dO rows stored into TMEM (256 arrivals)
   volatile int* misc = reinterpret_cast<volatile int*>(smem + L::kOffMisc);
   // misc[0] TMEM base, [1] list length, [2] abort flag
 
@@ -545,7 +570,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (lane == 0) {
       misc[1] = n;
       misc[2] = 0;
-      for (int i = 0; i < L::kNumBars; ++i) mbar_init(&bars[i], 1u);
+      for (int i = 0; i < L::kNumBars; ++i) mbar_init(&bars[i], &bars[i] == qd_tmem ? 256u : 1u);
       fence_mbar_init();
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
@@ -563,6 +588,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t tmem = static_cast<uint32_t>(misc[0]);
   const int n_list = misc[1];
   const uint32_t tm_dq = tmem, tm_s = tmem + 128, tm_dp = tmem + 256;
+  const uint32_t tm_q = tmem + 384, tm_do = tmem + 384 + D / 2;
 
   if (warp == kBwdLoadWarp) {
     // ------------------------------------------------------------- loads ---
@@ -595,10 +621,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else if (warp == kBwdMmaWarp) {
     // -------------------------------------------------------- MMA issue ---
     if (n_list > 0) {
-      bool ok = __all_sync(0xffffffffu, mbar_wait(qd_full, 0));
+      bool ok = __all_sync(0xffffffffu, mbar_wait(qd_tmem, 0));   // Q, dO in TMEM
       if (!ok && lane == 0) misc[2] = 1;
-      const uint64_t dq_a = smem_desc(smem_addr(smem + L::kOffFix0), 16, 1024);    // Q, A operand
-      const uint64_t ddo_a = smem_desc(smem_addr(smem + L::kOffFix1), 16, 1024);   // dO, A operand
       const uint64_t dk_k = smem_desc(smem_addr(smem + L::kOffRing0), 16, 1024);   // K, K-major B
       const uint64_t dv_k = smem_desc(smem_addr(smem + L::kOffRing1), 16, 1024);   // V, K-major B
       const uint64_t dk_mn = smem_desc(smem_addr(smem + L::kOffRing0), kHalfBytes, 1024);  // K, MN-major B
@@ -609,12 +633,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t off = static_cast<uint64_t>((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
-          mma_ss_warp(tm_s + 64 * hh, dq_a + off, dk_k + base + off, kIdescH, kk > 0 ? 1u : 0u);
+          mma_ts_warp(tm_s + 64 * hh, tm_q + kk * 8, dk_k + base + off, kIdescH, kk > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t off = static_cast<uint64_t>((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
-          mma_ss_warp(tm_dp + 64 * hh, ddo_a + off, dv_k + base + off, kIdescH, kk > 0 ? 1u : 0u);
+          mma_ts_warp(tm_dp + 64 * hh, tm_do + kk * 8, dv_k + base + off, kIdescH, kk > 0 ? 1u : 0u);
         }
       };
       // dQ += dS_hh K_hh: K = the half's 64 keys
@@ -690,9 +714,35 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int qh = BLK == 128 ? 0 : (r >> 6);
     const float sl2 = p.scale_log2;
     const size_t rix = static_cast<size_t>(bh) * p.N + (row_valid ? row : 0);
-    const float l2 = row_valid ? p.lse[rix] * 1.4426950408889634f : 0.f;
+    const float l2 = row_valid ? p.lse[rix] * -1.4426950408889634f : 0.f;   // -lse * log2(e)
     const float dl = row_valid ? p.delta[rix] : 0.f;
     bool ok = true;
+    if (n_list > 0) {
+      // row r of Q (warps 0-3) or dO (warps 4-7) from the 128-byte swizzled TMA
+      // tile (16-byte chunk j of a row at chunk j ^ (r % 8)) into TMEM as bf16
+      // pairs: the A operand layout of the MMAs above
+      if (!mbar_wait(qd_full, 0)) {
+        misc[2] = 1;
+        ok = false;
+      }
+      const uint8_t* tile = smem + (hh == 0 ? L::kOffFix0 : L::kOffFix1);
+#pragma unroll
+      for (int hd = 0; hd < D / 64; ++hd) {
+        uint32_t w[32];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint4 c = *reinterpret_cast<const uint4*>(tile + hd * kHalfBytes + r * 128 + ((j ^ (r & 7)) << 4));
+          w[4 * j] = c.x;
+          w[4 * j + 1] = c.y;
+          w[4 * j + 2] = c.z;
+          w[4 * j + 3] = c.w;
+        }
+        tmem_st32((hh == 0 ? tm_q : tm_do) + lane_off + 32 * hd, reinterpret_cast<const float*>(w));
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(qd_tmem);
+    }
     for (int e = 0; e < n_list; ++e) {
       const uint32_t bits = list[e] >> 16;
       const int jt = static_cast<int>(list[e] & 0xFFFFu);
