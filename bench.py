@@ -337,6 +337,28 @@ def run_suite(args):
             out.append(attn_line(wl, name, ms_a, flops, {
                 "mask_ms": round(ms_m, 4), "mask_gbs": round(qk_bytes / ms_m / 1e6, 1),
                 "mask_frac_of_hbm": round(qk_bytes / ms_m / 1e6 / hbm, 4)}))
+            # backward pass over the same mask (dQ, dK, dV from dO, O, LSE)
+            lse = torch.empty(B, H, N, device=dev)
+            ops.sa_sparse_attn_fwd(q, k, v, wl.block, mask=m, out=o, lse=lse)
+            gen = torch.Generator(device=dev).manual_seed(wl.seed + 11)
+            dout = torch.randn(q.shape, generator=gen, device=dev).to(torch.bfloat16)
+            dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+            bws = torch.empty(ops.sa_sparse_attn_bwd_workspace(B, H, N), dtype=torch.uint8, device=dev)
+            ms_b = _time(lambda: ops.sa_sparse_attn_bwd(q, k, v, o, dout, lse, wl.block, mask=m, dq=dq, dk=dk, dv=dv,
+                                                        workspace=bws), args.suite_reps, stream)
+            # algorithmic backward work: 5 GEMMs (dV, dP, dS K, dS^T Q and the recomputed S) per kept
+            # element; the kernels execute 7 (S and dP are recomputed in the dQ pass)
+            out.append(attn_line(wl, name + "_backward", ms_b, 2.5 * flops, {
+                "executed_tflops_7gemm": round(3.5 * flops / ms_b / 1e9, 1)}))
+            # token permutation of Q, K, V: per-head PARO axis orders, 3 x 5 x 4 cells
+            orders = (torch.arange(H, device=dev) % 6).to(torch.uint8)
+            pout = [torch.empty_like(q) for _ in range(3)]
+            ms_p = _time(lambda: ops.sa_token_permute([q, k, v], wl.T, wl.Hh, wl.Ww, head_order=orders, cells=(3, 5, 4),
+                                                      out=pout), args.suite_reps, stream)
+            pbytes = 2 * 3 * B * H * N * d * 2
+            out.append({"workload": name + "_permute_qkv", "N": N, "H": H, "d": d, "ms_per_call": round(ms_p, 4),
+                        "gbs": round(pbytes / ms_p / 1e6, 1), "frac_of_hbm": round(pbytes / ms_p / 1e6 / hbm, 4),
+                        "peak_source": src})
         elif wl.kind == "radial":
             rm = ops.sa_radial_mask(wl.T, wl.Hh, wl.Ww, wl.block)
             ms_r = _time(lambda: ops.sa_radial_mask(wl.T, wl.Hh, wl.Ww, wl.block, out=rm), args.suite_reps, stream)

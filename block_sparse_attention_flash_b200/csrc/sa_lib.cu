@@ -16,6 +16,7 @@
 #include "sa_attn_fwd.cuh"
 #include "sa_common.cuh"
 #include "sa_masks.cuh"
+#include "sa_permute.cuh"
 #include "sa_pyr_fwd.cuh"
 #include "sparse_attn.h"
 
@@ -519,6 +520,55 @@ sa_status sa_sparse_attn_bwd(const void* q, const void* k, const void* v, const 
     sa::bwd_dkdv_kernel<64, 64><<<grid, sa::kBwdThreads, sa::BwdSmem<64>::kAlloc, s>>>(tq, tk, tv, tdo, p);
     sa::bwd_dq_kernel<64, 64><<<grid, sa::kBwdThreads, sa::BwdSmem<64>::kAlloc, s>>>(tq, tk, tv, tdo, p);
   }
+  return cuda_status(cudaGetLastError());
+}
+
+}  // extern "C"
+
+// ----------------------------------------------------- token permutation ---
+extern "C" {
+
+sa_status sa_token_permute(const void* const* src, void* const* dst, int n_tensors, int B, int H, int T, int Hh,
+                           int Ww, int d, int order, const uint8_t* head_order, int ct, int ch, int cw, int inverse,
+                           void* stream) {
+  if (n_tensors < 1 || n_tensors > sa::kPermMaxTensors || !src || !dst) return SA_ERR_INVALID_ARG;
+  if (B < 0 || H < 0 || T < 0 || Hh < 0 || Ww < 0) return SA_ERR_INVALID_ARG;
+  if (order < 0 || order > 5 || (inverse != 0 && inverse != 1)) return SA_ERR_INVALID_ARG;
+  if (ct < 1 || ch < 1 || cw < 1) return SA_ERR_INVALID_ARG;
+  const long long N = static_cast<long long>(T) * Hh * Ww;
+  if (B == 0 || H == 0 || N == 0) return SA_OK;
+  if (T % ct || Hh % ch || Ww % cw) return SA_ERR_INVALID_ARG;
+  if (N > (1LL << 30)) return SA_ERR_UNSUPPORTED;
+  if (!valid_dim(d)) return SA_ERR_UNSUPPORTED;
+  sa::PermParams p;
+  for (int i = 0; i < n_tensors; ++i) {
+    if (!src[i] || !dst[i] || !aligned16(src[i]) || !aligned16(dst[i]) || src[i] == dst[i]) return SA_ERR_INVALID_ARG;
+    p.src[i] = static_cast<const __nv_bfloat16*>(src[i]);
+    p.dst[i] = static_cast<__nv_bfloat16*>(dst[i]);
+  }
+  for (int i = n_tensors; i < sa::kPermMaxTensors; ++i) {
+    p.src[i] = nullptr;
+    p.dst[i] = nullptr;
+  }
+  p.n_tensors = n_tensors;
+  p.H = H;
+  p.N = static_cast<int>(N);
+  p.g[0] = T;
+  p.g[1] = Hh;
+  p.g[2] = Ww;
+  p.c[0] = ct;
+  p.c[1] = ch;
+  p.c[2] = cw;
+  p.order = order;
+  p.head_order = head_order;
+  p.inverse = inverse;
+  if (static_cast<long long>(B) * H > 65535) return SA_ERR_UNSUPPORTED;
+  const dim3 grid(static_cast<unsigned>((N + 255) / 256), static_cast<unsigned>(B * H), static_cast<unsigned>(n_tensors));
+  cudaStream_t s = as_stream(stream);
+  if (d == 128)
+    sa::token_permute_kernel<128><<<grid, 256, 0, s>>>(p);
+  else
+    sa::token_permute_kernel<64><<<grid, 256, 0, s>>>(p);
   return cuda_status(cudaGetLastError());
 }
 

@@ -38,6 +38,8 @@ _SIGNATURES = {
     "sa_pyramid_attn_fwd": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _i64, _i64, _i64,
                                    _vp, _vp, _f32, _vp, _vp, _vp]),
     "sa_sparse_attn_bwd_workspace": (_sz, [_i32, _i32, _i32]),
+    "sa_token_permute": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _i32, _i32, _i32,
+                                _i32, _vp]),
     "sa_sparse_attn_bwd": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _i64, _i64, _i64,
                                   _f32, _vp, _vp, _vp, _vp, _sz, _vp]),
 }
@@ -261,3 +263,36 @@ def sa_sparse_attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: tor
         _dev(workspace, "workspace", torch.uint8), workspace.numel(), _stream(stream))
     _check(st, "sa_sparse_attn_bwd")
     return dq, dk, dv
+
+
+AXIS_ORDERS = ("thw", "twh", "htw", "hwt", "wth", "wht")   # the library's order codes 0..5
+
+
+def sa_token_permute(tensors, T: int, Hh: int, Ww: int, order="thw", head_order: Optional[torch.Tensor] = None,
+                     cells=(1, 1, 1), inverse: bool = False, out=None, stream=None):
+    """Reorder the tokens of up to four [B,H,N,d] bf16 tensors in one launch
+    (PARO axis orders / VMoBA cell partitions); returns the list of outputs."""
+    tensors = list(tensors)
+    if not 1 <= len(tensors) <= 4:
+        raise ValueError("one to four tensors")
+    B, H, N, d = tensors[0].shape
+    if N != T * Hh * Ww:
+        raise ValueError("N must equal T * Hh * Ww")
+    for t in tensors:
+        if tuple(t.shape) != (B, H, N, d):
+            raise ValueError("all tensors must have the same shape")
+    code = AXIS_ORDERS.index(order) if isinstance(order, str) else int(order)
+    hptr = None
+    if head_order is not None:
+        if head_order.dtype != torch.uint8 or not head_order.is_cuda or head_order.numel() != H:
+            raise ValueError("head_order must be a CUDA uint8 tensor of H codes")
+        hptr = head_order.data_ptr()
+    out = [torch.empty_like(t) for t in tensors] if out is None else list(out)
+    src = (ctypes.c_void_p * 4)(*[_dev(t, "tensor", torch.bfloat16) for t in tensors])
+    dst = (ctypes.c_void_p * 4)(*[_dev(t, "out", torch.bfloat16) for t in out])
+    st = lib().sa_token_permute(ctypes.cast(src, ctypes.c_void_p), ctypes.cast(dst, ctypes.c_void_p), len(tensors),
+                                B, H, T, Hh, Ww, d, code, hptr, int(cells[0]), int(cells[1]), int(cells[2]),
+                                int(bool(inverse)), _stream(stream))
+    _check(st, "sa_token_permute")
+    return out
+

@@ -11,6 +11,7 @@
  *   sa_sparse_attn_fwd FlashAttention-style forward over kept tiles, with the
  *                      LiteAttention skip-mask update fused in
  *   sa_sparse_attn_bwd its gradients with respect to Q, K and V
+ *   sa_token_permute   PARO axis orders / VMoBA cell partitions of the grid
  *
  * Conventions shared by every entry point
  *   - Tensors are caller-owned DEVICE memory.  Q, K, V and O are bf16,
@@ -281,6 +282,34 @@ SA_API sa_status sa_sparse_attn_bwd(const void* q, const void* k, const void* v,
                              const uint8_t* mask, int64_t mask_sb, int64_t mask_sh, int64_t mask_si,
                              float scale, void* dq, void* dk, void* dv, void* workspace,
                              size_t workspace_bytes, void* stream);
+
+/*
+ * sa_token_permute — reorder the tokens of the (t, h, w) grid, per head.
+ *   PAROAttention write-up (pattern-aware reordering paragraphs: 6 orders of
+ *   the three axes, one chosen per head, so that scattered attention becomes
+ *   blocks) and VMoBA write-up (layer-wise recurrent 1D / 2D / 3D block
+ *   partition of the video into temporal, spatial and spatio-temporal cells).
+ *
+ * Tokens are ordered by (cell coordinates, coordinates inside the cell), both
+ * tuples in the head's axis order, slowest axis first.  Axis order codes:
+ * 0 t,h,w (raster)  1 t,w,h  2 h,t,w  3 h,w,t  4 w,t,h  5 w,h,t.  Cells are
+ * ct x ch x cw and must divide the grid; 1 x 1 x 1 cells give the pure axis
+ * orders, order 0 with cells (ct, Hh, Ww) / (T, ch, cw) / (ct, ch, cw) the 1D
+ * / 2D / 3D partitions.  The blocks of the attention calls are then runs of
+ * `block` consecutive tokens of the permuted sequence.
+ * Arguments
+ *   src, dst      HOST arrays of n_tensors (1..4) device pointers, each bf16
+ *                 [B,H,N,d], N = T*Hh*Ww, 16-byte aligned; dst[i] != src[i].
+ *   order         axis order code of every head when head_order is NULL.
+ *   head_order    NULL, or uint8 [H] device array of per-head codes (0..5).
+ *   inverse       0: dst holds the permuted sequence of src (raster order);
+ *                 1: src is permuted, dst gets raster order back.
+ * Limits: d in {64,128}, N <= 2^30, B*H <= 65535.  Invalid codes in head_order are not
+ * checked on the device; they read as code 5.
+ */
+SA_API sa_status sa_token_permute(const void* const* src, void* const* dst, int n_tensors, int B, int H,
+                           int T, int Hh, int Ww, int d, int order, const uint8_t* head_order,
+                           int ct, int ch, int cw, int inverse, void* stream);
 
 #ifdef __cplusplus
 }

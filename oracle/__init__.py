@@ -13,6 +13,8 @@ from the pages' descriptions of the methods:
 * "浙江大学突破视频AI瓶颈:金字塔方法提升视频AI效率10倍" (PSA, arXiv
   2512.04025), the pyramid KV, multi-level mask and distribution-consistent
   attention paragraphs;
+* PAROAttention write-up (pattern-aware reordering) and VMoBA's recurrent
+  1D / 2D / 3D partitions: token permutations of the grid, ``oracle/permute.py``;
 * the backward pass (gradients through the masked attention, needed by the
   Radial Attention write-up's LoRA length extension) is the derivative of
   the forward definition, stated in ``oracle/backward.py``.
@@ -30,10 +32,11 @@ from .masks import block_means, block_scores, tau_mask, level_map, radial_mask
 from .pyramid import pyramid_pool, pyramid_attention
 from .lite import lite_step, lite_chain, visit_order
 from .backward import masked_attention_bwd, masked_attention_bwd_rows
+from .permute import permutation, permute_tokens
 
 __all__ = [
     "masked_attention", "dense_attention", "block_mask_to_token_mask",
     "block_means", "block_scores", "tau_mask", "level_map", "radial_mask",
     "pyramid_pool", "pyramid_attention", "lite_step", "lite_chain", "visit_order",
-    "masked_attention_bwd", "masked_attention_bwd_rows",
+    "masked_attention_bwd", "masked_attention_bwd_rows", "permutation", "permute_tokens",
 ]

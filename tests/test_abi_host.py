@@ -30,7 +30,7 @@ def test_header_declares_the_entry_points():
     names = _declared_symbols()
     for n in ("sa_build_mask", "sa_radial_mask", "sa_pyramid_pool", "sa_sparse_attn_fwd",
               "sa_pyramid_attn_fwd", "sa_get_device_status", "sa_build_mask_workspace",
-              "sa_sparse_attn_bwd", "sa_sparse_attn_bwd_workspace"):
+              "sa_sparse_attn_bwd", "sa_sparse_attn_bwd_workspace", "sa_token_permute"):
         assert n in names
 
 
@@ -137,4 +137,23 @@ def test_backward_workspace_and_argument_validation(lib):
     assert _bwd(lib, ws_bytes=256 * 4 - 1) == ops.SA_ERR_INVALID_ARG
     assert _bwd(lib, scale=float("nan")) == ops.SA_ERR_INVALID_ARG
     assert _bwd(lib, mask=16, si=-1) == ops.SA_ERR_INVALID_ARG
+
+
+def test_permute_argument_validation(lib):
+    import ctypes
+    src = (ctypes.c_void_p * 4)(16, 32, 48, 64)
+    dst = (ctypes.c_void_p * 4)(80, 96, 112, 128)
+    same = (ctypes.c_void_p * 4)(16, 32, 48, 64)
+
+    def call(n=1, B=1, H=1, T=2, Hh=3, Ww=4, d=128, order=0, ct=1, ch=1, cw=1, inverse=0, s=src, t=dst):
+        return lib.sa_token_permute(ctypes.cast(s, ctypes.c_void_p), ctypes.cast(t, ctypes.c_void_p), n, B, H, T,
+                                    Hh, Ww, d, order, None, ct, ch, cw, inverse, None)
+    assert call(B=0) == ops.SA_OK
+    assert call(n=0) == ops.SA_ERR_INVALID_ARG and call(n=5) == ops.SA_ERR_INVALID_ARG
+    assert call(order=6) == ops.SA_ERR_INVALID_ARG and call(order=-1) == ops.SA_ERR_INVALID_ARG
+    assert call(inverse=2) == ops.SA_ERR_INVALID_ARG
+    assert call(ch=2) == ops.SA_ERR_INVALID_ARG                 # 2 does not divide Hh = 3
+    assert call(cw=0) == ops.SA_ERR_INVALID_ARG
+    assert call(d=96) == ops.SA_ERR_UNSUPPORTED
+    assert call(t=same) == ops.SA_ERR_INVALID_ARG               # dst == src
 
