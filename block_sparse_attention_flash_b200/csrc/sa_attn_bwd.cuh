@@ -61,6 +61,7 @@ struct BwdParams {
   const float* delta; // [B,H,N] D_r = dO_r . O_r
   float scale;        // logit scale
   float scale_log2;   // scale * log2(e)
+  int causal;         // key c visible to row r only if c <= r (blocks j > i dropped)
   __nv_bfloat16* dq;
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
@@ -161,6 +162,11 @@ __device__ __forceinline__ void grad_chunk_any(const float* sv, const float* dp,
     grad_chunk<kPerColumn, true>(sv, dp, sl2, nl, dl, nls, dls, keep_bits, pk, dk);
   else
     grad_chunk<kPerColumn, false>(sv, dp, sl2, nl, dl, nls, dls, keep_bits, pk, dk);
+}
+
+// Bits i of a 32-column chunk with i >= lo (all for lo <= 0, none for lo >= 32).
+__device__ __forceinline__ uint32_t causal_from(int lo) {
+  return lo <= 0 ? 0xffffffffu : (lo >= 32 ? 0u : ~((1u << lo) - 1u));
 }
 
 // Half hh (columns [64 hh, 64 hh + 64)) of this thread's S and dP rows: P
@@ -274,7 +280,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const int kb = jt * KH + kh;
             if (kb >= p.nb) continue;
             const uint8_t keep = p.mask ? p.mask[b * p.msb + h * p.msh + qb * p.msi + kb] : uint8_t(1);
-            if (keep) bits |= (BLK == 128 ? 0xFu : (1u << (qh * 2 + kh)));
+            if (keep && (!p.causal || kb <= qb)) bits |= (BLK == 128 ? 0xFu : (1u << (qh * 2 + kh)));
           }
         }
       }
@@ -472,8 +478,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // half hh: query columns [64 hh, 64 hh + 64), q-block half hh for block 64
       const bool quad = BLK == 128 ? true : ((bits >> (hh * 2 + kh)) & 1u);
       const int nv0 = min(32, max(0, valid_q - 64 * hh)), nv1 = min(32, max(0, valid_q - 64 * hh - 32));
-      const uint32_t keep0 = (key_valid && quad) ? (nv0 == 32 ? 0xffffffffu : ((1u << nv0) - 1u)) : 0u;
-      const uint32_t keep1 = (key_valid && quad) ? (nv1 == 32 ? 0xffffffffu : ((1u << nv1) - 1u)) : 0u;
+      uint32_t keep0 = (key_valid && quad) ? (nv0 == 32 ? 0xffffffffu : ((1u << nv0) - 1u)) : 0u;
+      uint32_t keep1 = (key_valid && quad) ? (nv1 == 32 ? 0xffffffffu : ((1u << nv1) - 1u)) : 0u;
+      if (p.causal && it == jt) {
+        // diagonal tile: query column c sees this key (row r) only if c >= r
+        keep0 &= causal_from(r - 64 * hh);
+        keep1 &= causal_from(r - 64 * hh - 32);
+      }
       grad_half<true, true>(tm_s + lane_off, tm_dp + lane_off, tm_dp + lane_off, hh, sl2, vec, vec + 128, 0.f, 0.f,
                             keep0, keep1);
       tmem_st_wait();
@@ -559,7 +570,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const int kb = jt * KH + kh;
             if (kb >= p.nb) continue;
             const uint8_t keep = p.mask ? p.mask[b * p.msb + h * p.msh + qb * p.msi + kb] : uint8_t(1);
-            if (keep) bits |= (BLK == 128 ? 0xFu : (1u << (qh * 2 + kh)));
+            if (keep && (!p.causal || kb <= qb)) bits |= (BLK == 128 ? 0xFu : (1u << (qh * 2 + kh)));
           }
         }
       }
@@ -755,8 +766,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // half hh: key columns [64 hh, 64 hh + 64), k-block half hh for block 64
       const bool quad = BLK == 128 ? true : ((bits >> (qh * 2 + hh)) & 1u);
       const int nv0 = min(32, max(0, valid_k - 64 * hh)), nv1 = min(32, max(0, valid_k - 64 * hh - 32));
-      const uint32_t keep0 = (row_valid && quad) ? (nv0 == 32 ? 0xffffffffu : ((1u << nv0) - 1u)) : 0u;
-      const uint32_t keep1 = (row_valid && quad) ? (nv1 == 32 ? 0xffffffffu : ((1u << nv1) - 1u)) : 0u;
+      uint32_t keep0 = (row_valid && quad) ? (nv0 == 32 ? 0xffffffffu : ((1u << nv0) - 1u)) : 0u;
+      uint32_t keep1 = (row_valid && quad) ? (nv1 == 32 ? 0xffffffffu : ((1u << nv1) - 1u)) : 0u;
+      if (p.causal && jt == it) {
+        // diagonal tile: key column c is visible to row r only if c <= r
+        keep0 &= ~causal_from(r - 64 * hh + 1);
+        keep1 &= ~causal_from(r - 64 * hh - 32 + 1);
+      }
       grad_half<false, false>(tm_s + lane_off, tm_dp + lane_off, tm_s + lane_off, hh, sl2, nullptr, nullptr, l2, dl,
                               keep0, keep1);
       tmem_st_wait();

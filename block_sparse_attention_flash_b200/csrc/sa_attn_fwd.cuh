@@ -75,6 +75,7 @@ struct AttnParams {
   float scale_log2; // scale * log2(e)
   float eps_raw;    // eps / scale: the skip threshold in raw q.k units
   int radial;       // visit kv tiles in radial-centric order (else ascending)
+  int causal;       // key c visible to row r only if c <= r (blocks j > i dropped)
   __nv_bfloat16* o;
   float* lse;
 };
@@ -216,7 +217,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               const uint8_t keep = p.mask ? p.mask[b * p.msb + h * p.msh + qb * p.msi + kb] : uint8_t(1);
               const size_t sidx = (static_cast<size_t>(bh) * p.nb + qb) * p.nb + kb;
               const uint8_t sk = p.skip_in ? p.skip_in[sidx] : uint8_t(0);
-              if (keep && !sk) {
+              if (keep && !sk && (!p.causal || kb <= qb)) {
                 bits |= (BLK == 128 ? 0xFu : (1u << (qh * 2 + kh))) << (16 + 4 * t);
               } else if (p.carry_skip) {
                 p.skip_out[sidx] = sk;
@@ -468,12 +469,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         named_bar_sync(kBarSFree + t, kHandoff);
 
         const int valid_cols = min(kTileN, p.N - jt * kTileN);
-        if (valid_cols < kTileN || (BLK == 64 && bits != 0xFu)) {
+        // causal: in the diagonal tile (kv tile = q-tile) key c needs c <= r
+        const int cmax = (p.causal && jt == qtile0 + t) ? r : kTileN - 1;
+        if (valid_cols < kTileN || (BLK == 64 && bits != 0xFu) || cmax < kTileN - 1) {
           const bool k0 = BLK == 128 ? true : ((bits >> (qh * 2 + 0)) & 1u);
           const bool k1 = BLK == 128 ? true : ((bits >> (qh * 2 + 1)) & 1u);
 #pragma unroll
           for (int c = 0; c < kTileN; ++c) {
-            const bool keep = (c < valid_cols) && (c < 64 ? k0 : k1);
+            const bool keep = (c < valid_cols) && (c < 64 ? k0 : k1) && c <= cmax;
             s[c] = keep ? s[c] : NEG_INF;
           }
         }

@@ -251,9 +251,10 @@ sa_status sa_pyramid_pool(const void* k, const void* v, int B, int H, int N, int
 sa_status sa_sparse_attn_fwd(const void* q, const void* k, const void* v, int B, int H, int N, int d, int block,
                              const uint8_t* mask, int64_t mask_sb, int64_t mask_sh, int64_t mask_si,
                              const uint8_t* skip_in, uint8_t* skip_out, float eps, float scale, int order,
-                             void* o, float* lse, void* stream) {
+                             int causal, void* o, float* lse, void* stream) {
   if (B < 0 || H < 0 || N < 0) return SA_ERR_INVALID_ARG;
   if (order != SA_ORDER_ASCENDING && order != SA_ORDER_RADIAL) return SA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return SA_ERR_INVALID_ARG;
   if (std::isnan(eps) || eps < 0.f) return SA_ERR_INVALID_ARG;
   if (std::isnan(scale) || scale < 0.f || std::isinf(scale)) return SA_ERR_INVALID_ARG;
   if (B == 0 || H == 0 || N == 0) return SA_OK;
@@ -291,6 +292,7 @@ sa_status sa_sparse_attn_fwd(const void* q, const void* k, const void* v, int B,
   p.scale_log2 = scale * 1.4426950408889634f;
   p.eps_raw = std::isinf(eps) ? INFINITY : eps / scale;
   p.radial = order == SA_ORDER_RADIAL;
+  p.causal = causal;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
 
@@ -448,9 +450,10 @@ size_t sa_sparse_attn_bwd_workspace(int B, int H, int N) {
 
 sa_status sa_sparse_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
                              const float* lse, int B, int H, int N, int d, int block, const uint8_t* mask,
-                             int64_t mask_sb, int64_t mask_sh, int64_t mask_si, float scale, void* dq, void* dk,
-                             void* dv, void* workspace, size_t workspace_bytes, void* stream) {
+                             int64_t mask_sb, int64_t mask_sh, int64_t mask_si, float scale, int causal, void* dq,
+                             void* dk, void* dv, void* workspace, size_t workspace_bytes, void* stream) {
   if (B < 0 || H < 0 || N < 0) return SA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return SA_ERR_INVALID_ARG;
   if (std::isnan(scale) || scale < 0.f || std::isinf(scale)) return SA_ERR_INVALID_ARG;
   if (B == 0 || H == 0 || N == 0) return SA_OK;
   if (!valid_dim(d) || !valid_block(block)) return SA_ERR_UNSUPPORTED;
@@ -489,6 +492,7 @@ sa_status sa_sparse_attn_bwd(const void* q, const void* k, const void* v, const 
   p.delta = delta;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.causal = causal;
   p.dq = static_cast<__nv_bfloat16*>(dq);
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);

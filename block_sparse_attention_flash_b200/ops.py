@@ -34,14 +34,14 @@ _SIGNATURES = {
     "sa_radial_mask": (_i32, [_i32, _i32, _i32, _i32, _vp, _vp]),
     "sa_pyramid_pool": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
     "sa_sparse_attn_fwd": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _i64, _i64, _i64,
-                                  _vp, _vp, _f32, _f32, _i32, _vp, _vp, _vp]),
+                                  _vp, _vp, _f32, _f32, _i32, _i32, _vp, _vp, _vp]),
     "sa_pyramid_attn_fwd": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _i64, _i64, _i64,
                                    _vp, _vp, _f32, _vp, _vp, _vp]),
     "sa_sparse_attn_bwd_workspace": (_sz, [_i32, _i32, _i32]),
     "sa_token_permute": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _i32, _i32, _i32,
                                 _i32, _vp]),
     "sa_sparse_attn_bwd": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _i64, _i64, _i64,
-                                  _f32, _vp, _vp, _vp, _vp, _sz, _vp]),
+                                  _f32, _i32, _vp, _vp, _vp, _vp, _sz, _vp]),
 }
 
 _lib = None
@@ -179,7 +179,7 @@ def sa_sparse_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block:
                        mask: Optional[torch.Tensor] = None, skip_in: Optional[torch.Tensor] = None,
                        skip_out: Optional[torch.Tensor] = None, eps: float = math.inf, scale: float = 0.0,
                        out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-                       stream=None, order: str = "ascending") -> torch.Tensor:
+                       stream=None, order: str = "ascending", causal: bool = False) -> torch.Tensor:
     """Block-sparse attention forward; returns O (and fills lse / skip_out if given).
 
     ``order`` ("ascending" or "radial") is the k-block visit order of the skip update."""
@@ -203,7 +203,7 @@ def sa_sparse_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block:
         _dev(q, "q", torch.bfloat16), _dev(k, "k", torch.bfloat16), _dev(v, "v", torch.bfloat16),
         B, H, N, d, block, mptr, sb, sh, si,
         _opt(skip_in, "skip_in", torch.uint8), _opt(skip_out, "skip_out", torch.uint8),
-        float(eps), float(scale), VISIT_ORDERS[order], _dev(out, "out", torch.bfloat16),
+        float(eps), float(scale), VISIT_ORDERS[order], int(bool(causal)), _dev(out, "out", torch.bfloat16),
         _opt(lse, "lse", torch.float32), _stream(stream))
     _check(st, "sa_sparse_attn_fwd")
     return out
@@ -239,7 +239,7 @@ def sa_sparse_attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: tor
                        lse: torch.Tensor, block: int, mask: Optional[torch.Tensor] = None, scale: float = 0.0,
                        dq: Optional[torch.Tensor] = None, dk: Optional[torch.Tensor] = None,
                        dv: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
-                       stream=None):
+                       stream=None, causal: bool = False):
     """Gradients (dQ, dK, dV) of sa_sparse_attn_fwd given dO and the forward's O and LSE."""
     B, H, N, d = q.shape
     nb = nblocks(N, block)
@@ -258,7 +258,7 @@ def sa_sparse_attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: tor
     st = lib().sa_sparse_attn_bwd(
         _dev(q, "q", torch.bfloat16), _dev(k, "k", torch.bfloat16), _dev(v, "v", torch.bfloat16),
         _dev(o, "o", torch.bfloat16), _dev(dout, "dout", torch.bfloat16), _dev(lse, "lse", torch.float32),
-        B, H, N, d, block, mptr, sb, sh, si, float(scale),
+        B, H, N, d, block, mptr, sb, sh, si, float(scale), int(bool(causal)),
         _dev(dq, "dq", torch.bfloat16), _dev(dk, "dk", torch.bfloat16), _dev(dv, "dv", torch.bfloat16),
         _dev(workspace, "workspace", torch.uint8), workspace.numel(), _stream(stream))
     _check(st, "sa_sparse_attn_bwd")

@@ -218,6 +218,13 @@ SA_API sa_status sa_pyramid_pool(const void* k, const void* v, int B, int H, int
  *                 band holding row i*block (distance 0 for both), ties by
  *                 ascending tile, ascending j inside a tile.  Any other
  *                 value is SA_ERR_INVALID_ARG.
+ *   causal        0, or 1: key c is visible to row r only if c <= r (token
+ *                 index in the sequence as given).  The PSA page notes the
+ *                 method serves causal video generation as well as
+ *                 bidirectional understanding; read as: the effective mask
+ *                 is mask AND (j <= i), and inside the diagonal block the
+ *                 key must not come after the row.  Blocks j > i are neither
+ *                 visited nor tested; their skip_out bytes copy skip_in.
  *   o             bf16 [B,H,N,d] device, written for every valid row.
  *   lse           NULL or fp32 [B,H,N] device.
  * Limits: d in {64,128}, block in {64,128}, ceil(N/128) <= 4096, B*H <= 65535.
@@ -226,7 +233,7 @@ SA_API sa_status sa_sparse_attn_fwd(const void* q, const void* k, const void* v,
                              int B, int H, int N, int d, int block,
                              const uint8_t* mask, int64_t mask_sb, int64_t mask_sh, int64_t mask_si,
                              const uint8_t* skip_in, uint8_t* skip_out, float eps, float scale, int order,
-                             void* o, float* lse, void* stream);
+                             int causal, void* o, float* lse, void* stream);
 
 /*
  * sa_pyramid_attn_fwd — PSA multi-level attention forward.
@@ -269,6 +276,7 @@ SA_API sa_status sa_pyramid_attn_fwd(const void* q, const void* k, const void* v
  *                 byte keeps).  Pass the forward's effective mask (mask AND
  *                 NOT skip_in when the forward skipped blocks).
  *   scale         logit scale; 0 selects 1/sqrt(d).
+ *   causal        as sa_sparse_attn_fwd (use the forward's value).
  *   dq, dk, dv    bf16 [B,H,N,d] device, written for every valid row (zero
  *                 where the row or key takes part in no kept block).
  *   workspace     device scratch of at least sa_sparse_attn_bwd_workspace()
@@ -280,7 +288,7 @@ SA_API size_t sa_sparse_attn_bwd_workspace(int B, int H, int N);
 SA_API sa_status sa_sparse_attn_bwd(const void* q, const void* k, const void* v, const void* o,
                              const void* dout, const float* lse, int B, int H, int N, int d, int block,
                              const uint8_t* mask, int64_t mask_sb, int64_t mask_sh, int64_t mask_si,
-                             float scale, void* dq, void* dk, void* dv, void* workspace,
+                             float scale, int causal, void* dq, void* dk, void* dv, void* workspace,
                              size_t workspace_bytes, void* stream);
 
 /*

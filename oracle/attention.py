@@ -14,6 +14,10 @@ Blocks are consecutive runs of ``block`` tokens in raster (t,h,w) order; the
 last block may be partial and then holds only its valid tokens.  A row with
 no kept column gets O_r = 0 and LSE_r = -inf.  ``scale`` defaults to
 1/sqrt(d) (natural-log units).
+
+Causal option (the PSA page says the method serves causal video generation
+as well as bidirectional understanding; reading): key column c is visible to
+row r only if it is kept by the block mask and c <= r.
 """
 from __future__ import annotations
 
@@ -41,12 +45,13 @@ def _mask4(mask, B, H, nqb, nkb):
     return np.broadcast_to(m, (B, H, nqb, nkb))
 
 
-def attention_qblock(qh, kh, vh, block, keep_row, i, scale):
+def attention_qblock(qh, kh, vh, block, keep_row, i, scale, causal=False):
     """O (rows x d) and LSE (rows,) for q-block ``i`` of one head.
 
     ``keep_row`` is the boolean row of the block mask for q-block ``i``.
     The kept key columns are gathered in ascending order and one fp64 matmul
-    gives the logits; softmax is the textbook max-subtracted form.
+    gives the logits; softmax is the textbook max-subtracted form.  With
+    ``causal``, logits of columns after the row are -inf.
     """
     N = qh.shape[0]
     r0, r1 = i * block, min(N, (i + 1) * block)
@@ -57,15 +62,19 @@ def attention_qblock(qh, kh, vh, block, keep_row, i, scale):
         return np.zeros((r1 - r0, d)), np.full(r1 - r0, -np.inf)
     c = np.concatenate(cols)
     s = (qh[r0:r1] @ kh[c].T) * scale
+    if causal:
+        s = np.where(c[None, :] <= np.arange(r0, r1)[:, None], s, -np.inf)
     m = s.max(axis=1, keepdims=True)
+    m = np.where(np.isfinite(m), m, 0.0)
     e = np.exp(s - m)
     z = e.sum(axis=1, keepdims=True)
-    o = (e / z) @ vh[c]
-    lse = (m + np.log(z))[:, 0]
+    o = np.divide(e, z, out=np.zeros_like(e), where=z > 0) @ vh[c]
+    with np.errstate(divide="ignore"):
+        lse = (m + np.log(z))[:, 0]
     return o, lse
 
 
-def masked_attention(q, k, v, block, mask=None, scale=None, qblocks=None):
+def masked_attention(q, k, v, block, mask=None, scale=None, qblocks=None, causal=False):
     """Block-masked attention over [B, H, N, d] inputs.
 
     mask: None (all kept) or anything broadcastable to uint8 [B, H, Nqb, Nkb].
@@ -83,7 +92,7 @@ def masked_attention(q, k, v, block, mask=None, scale=None, qblocks=None):
         out = {}
         for (b, h, i) in qblocks:
             out[(b, h, i)] = attention_qblock(q[b, h], k[b, h], v[b, h], block,
-                                              m4[b, h, i] != 0, i, scale)
+                                              m4[b, h, i] != 0, i, scale, causal)
         return out
     O = np.zeros((B, H, N, d))
     L = np.zeros((B, H, N))
@@ -92,7 +101,7 @@ def masked_attention(q, k, v, block, mask=None, scale=None, qblocks=None):
             for i in range(nqb):
                 r0, r1 = i * block, min(N, (i + 1) * block)
                 O[b, h, r0:r1], L[b, h, r0:r1] = attention_qblock(
-                    q[b, h], k[b, h], v[b, h], block, m4[b, h, i] != 0, i, scale)
+                    q[b, h], k[b, h], v[b, h], block, m4[b, h, i] != 0, i, scale, causal)
     return O, L
 
 

@@ -9,7 +9,8 @@ with respect to Q, K and V over the same block masks.
 The gradient is the derivative of the forward definition in
 ``oracle/attention.py`` (no page states it; it follows from the chain rule
 through the row softmax).  For one head, with M the token keep matrix
-expanded from the block mask and dO the incoming gradient of O:
+expanded from the block mask (and, with the causal option, restricted to
+key c <= row r) and dO the incoming gradient of O:
 
     S    = scale * Q K^T,  S_rc = -inf where M_rc = 0
     P    = row softmax of S (a row with no kept column is all zero)
@@ -49,7 +50,7 @@ def attention_bwd_head(qh, kh, vh, doh, keep, scale):
     return scale * (ds @ kh), scale * (ds.T @ qh), dv
 
 
-def masked_attention_bwd(q, k, v, block, mask, dout, scale=None):
+def masked_attention_bwd(q, k, v, block, mask, dout, scale=None, causal=False):
     """Gradients (dQ, dK, dV), fp64 [B,H,N,d] each, of block-masked attention.
 
     mask: None (all kept) or anything broadcastable to uint8 [B, H, Nb, Nb];
@@ -64,11 +65,14 @@ def masked_attention_bwd(q, k, v, block, mask, dout, scale=None):
     for b in range(B):
         for h in range(H):
             keep = block_mask_to_token_mask(m4[b, h], N, block)
+            if causal:
+                keep = keep & np.tri(N, dtype=bool)
             dq[b, h], dk[b, h], dv[b, h] = attention_bwd_head(q[b, h], k[b, h], v[b, h], do[b, h], keep, scale)
     return dq, dk, dv
 
 
-def masked_attention_bwd_rows(q, k, v, block, mask, dout, b, h, q_rows, k_rows, scale=None, chunk=1024):
+def masked_attention_bwd_rows(q, k, v, block, mask, dout, b, h, q_rows, k_rows, scale=None, chunk=1024,
+                              causal=False):
     """Selected rows of dQ (query rows ``q_rows``) and of dK, dV (key rows
     ``k_rows``) of head (b, h), for sizes where the full N x N matrices do not
     fit.  The same formulas as ``attention_bwd_head``, evaluated over chunks of
@@ -92,6 +96,8 @@ def masked_attention_bwd_rows(q, k, v, block, mask, dout, b, h, q_rows, k_rows, 
         r1 = min(N, r0 + chunk)
         rows = np.arange(r0, r1)
         keep = m[(rows // block)[:, None], kblk[None, :]]
+        if causal:
+            keep = keep & (np.arange(N)[None, :] <= rows[:, None])
         s = np.where(keep, (qh[r0:r1] @ kh.T) * scale, -np.inf)
         p = _softmax_rows(s)
         o = p @ vh

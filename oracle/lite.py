@@ -16,7 +16,9 @@ Readings (stated because the page gives prose only):
 * block j (not the first visited) gets a new skip bit iff l_r(j) < m_r - eps
   for every valid row r of the q-block; eps is in natural-log logit units;
 * the output of the detecting step still includes block j; the bit takes
-  effect from the next step: skip_out = skip_in | new_bits.
+  effect from the next step: skip_out = skip_in | new_bits;
+* causal option: blocks j > i are not visited; in the diagonal block a row's
+  maximum is over the columns at or before it.
 * radial-centric order (section 5 names it, section 10 expects 10-20 % more
   sparsity from it; neither defines it): the key axis is cut into tiles of
   128 tokens and the query axis into bands of 256 rows; the k-blocks of
@@ -57,7 +59,7 @@ def visit_order(i, nkb, block, order="ascending"):
     return [j for t in tiles for j in range(t * per_tile, min(nkb, (t + 1) * per_tile))]
 
 
-def lite_qblock(qh, kh, vh, block, keep_row, i, eps, scale, order="ascending"):
+def lite_qblock(qh, kh, vh, block, keep_row, i, eps, scale, order="ascending", causal=False):
     """(O rows, LSE rows, new-bit row, margin row) for one q-block.
 
     margin[j] = max_r (l_r(j) - m_r + eps) for tested blocks (NaN elsewhere);
@@ -67,7 +69,8 @@ def lite_qblock(qh, kh, vh, block, keep_row, i, eps, scale, order="ascending"):
     d = vh.shape[1]
     nkb = keep_row.shape[0]
     r0, r1 = i * block, min(N, (i + 1) * block)
-    visited = np.array([j for j in visit_order(i, nkb, block, order) if keep_row[j]], dtype=np.int64)
+    visited = np.array([j for j in visit_order(i, nkb, block, order) if keep_row[j] and (not causal or j <= i)],
+                       dtype=np.int64)
     new = np.zeros(nkb, dtype=np.uint8)
     margin = np.full(nkb, np.nan)
     if visited.size == 0:
@@ -75,6 +78,8 @@ def lite_qblock(qh, kh, vh, block, keep_row, i, eps, scale, order="ascending"):
     cols = [np.arange(j * block, min(N, (j + 1) * block)) for j in visited]
     c = np.concatenate(cols)
     s = (qh[r0:r1] @ kh[c].T) * scale
+    if causal:
+        s = np.where(c[None, :] <= np.arange(r0, r1)[:, None], s, -np.inf)
     running = np.full(r1 - r0, -np.inf)
     off = 0
     for n_vis, j in enumerate(visited):
@@ -94,7 +99,7 @@ def lite_qblock(qh, kh, vh, block, keep_row, i, eps, scale, order="ascending"):
 
 
 def lite_step(q, k, v, block, mask=None, skip_in=None, eps=10.0, scale=None, qblocks=None,
-              order="ascending"):
+              order="ascending", causal=False):
     """One denoising step of block attention with the LiteAttention skip update.
 
     Effective keep = mask & ~skip_in; ``order`` is "ascending" or "radial".  Returns (O, LSE, skip_out, margin) with
@@ -114,7 +119,7 @@ def lite_step(q, k, v, block, mask=None, skip_in=None, eps=10.0, scale=None, qbl
 
     def one(b, h, i):
         keep = (m4[b, h, i] != 0) & (s4[b, h, i] == 0)
-        o, lse, new, mg = lite_qblock(q[b, h], k[b, h], v[b, h], block, keep, i, eps, scale, order)
+        o, lse, new, mg = lite_qblock(q[b, h], k[b, h], v[b, h], block, keep, i, eps, scale, order, causal)
         return o, lse, (s4[b, h, i] | new).astype(np.uint8), mg
 
     if qblocks is not None:

@@ -55,11 +55,11 @@ def test_workspace_size(lib):
 
 def _attn(lib, **kw):
     a = dict(q=16, k=16, v=16, B=1, H=1, N=256, d=128, block=128, mask=None, sb=0, sh=0, si=0,
-             skip_in=None, skip_out=None, eps=math.inf, scale=0.0, order=0, o=16, lse=None, stream=None)
+             skip_in=None, skip_out=None, eps=math.inf, scale=0.0, order=0, causal=0, o=16, lse=None, stream=None)
     a.update(kw)
     return lib.sa_sparse_attn_fwd(a["q"], a["k"], a["v"], a["B"], a["H"], a["N"], a["d"], a["block"],
                                   a["mask"], a["sb"], a["sh"], a["si"], a["skip_in"], a["skip_out"],
-                                  a["eps"], a["scale"], a["order"], a["o"], a["lse"], a["stream"])
+                                  a["eps"], a["scale"], a["order"], a["causal"], a["o"], a["lse"], a["stream"])
 
 
 def test_attention_argument_validation(lib):
@@ -71,6 +71,7 @@ def test_attention_argument_validation(lib):
     assert _attn(lib, eps=-1.0) == ops.SA_ERR_INVALID_ARG
     assert _attn(lib, order=2) == ops.SA_ERR_INVALID_ARG
     assert _attn(lib, order=-1) == ops.SA_ERR_INVALID_ARG
+    assert _attn(lib, causal=2) == ops.SA_ERR_INVALID_ARG
     assert _attn(lib, scale=-0.5) == ops.SA_ERR_INVALID_ARG
     assert _attn(lib, N=128 * 4097) == ops.SA_ERR_UNSUPPORTED
     assert _attn(lib, B=256, H=256) == ops.SA_ERR_UNSUPPORTED
@@ -116,10 +117,10 @@ def test_ops_refuse_cpu_tensors():
 
 def _bwd(lib, **kw):
     a = dict(q=16, k=16, v=16, o=16, dout=16, lse=16, B=1, H=1, N=256, d=128, block=128, mask=None, sb=0, sh=0,
-             si=0, scale=0.0, dq=16, dk=16, dv=16, ws=16, ws_bytes=1 << 20, stream=None)
+             si=0, scale=0.0, causal=0, dq=16, dk=16, dv=16, ws=16, ws_bytes=1 << 20, stream=None)
     a.update(kw)
     return lib.sa_sparse_attn_bwd(a["q"], a["k"], a["v"], a["o"], a["dout"], a["lse"], a["B"], a["H"], a["N"],
-                                  a["d"], a["block"], a["mask"], a["sb"], a["sh"], a["si"], a["scale"], a["dq"],
+                                  a["d"], a["block"], a["mask"], a["sb"], a["sh"], a["si"], a["scale"], a["causal"], a["dq"],
                                   a["dk"], a["dv"], a["ws"], a["ws_bytes"], a["stream"])
 
 
@@ -137,6 +138,7 @@ def test_backward_workspace_and_argument_validation(lib):
     assert _bwd(lib, ws_bytes=256 * 4 - 1) == ops.SA_ERR_INVALID_ARG
     assert _bwd(lib, scale=float("nan")) == ops.SA_ERR_INVALID_ARG
     assert _bwd(lib, mask=16, si=-1) == ops.SA_ERR_INVALID_ARG
+    assert _bwd(lib, causal=3) == ops.SA_ERR_INVALID_ARG
 
 
 def test_permute_argument_validation(lib):

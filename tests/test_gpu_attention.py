@@ -21,14 +21,15 @@ def _lib():
 
 
 def run_attn(q, k, v, block, mask=None, skip_in=None, skip_out=None, eps=math.inf, with_lse=True,
-             order="ascending"):
+             order="ascending", causal=False):
     qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
     B, H, N, d = q.shape
     # poison the output so unwritten rows show up
     out = torch.full_like(qd, float("nan"))
     lse = torch.full((B, H, N), float("nan"), device="cuda") if with_lse else None
     ops.sa_sparse_attn_fwd(qd, kd, vd, block, mask=None if mask is None else mask.cuda(),
-                           skip_in=skip_in, skip_out=skip_out, eps=eps, out=out, lse=lse, order=order)
+                           skip_in=skip_in, skip_out=skip_out, eps=eps, out=out, lse=lse, order=order,
+                           causal=causal)
     ops.sa_get_device_status()
     return out.cpu(), (lse.cpu() if lse is not None else None)
 
@@ -95,7 +96,7 @@ def test_radial_mask_broadcast_over_heads():
 
 # ------------------------------------------------------------------ skip ---
 
-def _skip_run(q, k, v, block, mask, skip_in, eps, alias=False, order="ascending"):
+def _skip_run(q, k, v, block, mask, skip_in, eps, alias=False, order="ascending", causal=False):
     B, H, N, d = q.shape
     nb = -(-N // block)
     si = skip_in.cuda() if skip_in is not None else None
@@ -103,14 +104,14 @@ def _skip_run(q, k, v, block, mask, skip_in, eps, alias=False, order="ascending"
         so = si
     else:
         so = torch.full((B, H, nb, nb), 77, dtype=torch.uint8, device="cuda")
-    O, L = run_attn(q, k, v, block, mask, skip_in=si, skip_out=so, eps=eps, order=order)
+    O, L = run_attn(q, k, v, block, mask, skip_in=si, skip_out=so, eps=eps, order=order, causal=causal)
     return O, L, so.cpu()
 
 
-def _check_skip_step(q, k, v, block, mask, skip_in, eps, alias=False, order="ascending"):
-    O, L, S = _skip_run(q, k, v, block, mask, skip_in, eps, alias, order)
+def _check_skip_step(q, k, v, block, mask, skip_in, eps, alias=False, order="ascending", causal=False):
+    O, L, S = _skip_run(q, k, v, block, mask, skip_in, eps, alias, order, causal)
     Or, Lr, Sr, M = lite_step(q, k, v, block, None if mask is None else mask.numpy(),
-                              None if skip_in is None else skip_in.numpy(), eps, order=order)
+                              None if skip_in is None else skip_in.numpy(), eps, order=order, causal=causal)
     check_o(O, Or, f"skip step eps={eps}")
     check_lse(L, Lr, f"skip step eps={eps}")
     nflag = check_bits(S, Sr, skip_flags(M), f"skip bits eps={eps}")
@@ -222,3 +223,40 @@ def test_radial_order_reaches_the_row_max_first(d):
     assert S[0, 0, 4].tolist() == [1, 1, 1, 1, 0, 0, 1, 1]
     S, _, _ = _check_skip_step(q, k, v, block, None, None, eps=10.0)
     assert S[0, 0, 4].tolist() == [0, 0, 0, 0, 0, 0, 1, 1]
+
+
+# ------------------------------------------------------------------ causal ---
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("block", [64, 128])
+def test_causal_ragged_masks(d, block):
+    """Causal option on a ragged sequence: all kept, then a Bernoulli mask with
+    one q-block keeping only future blocks (no visible key) and one without
+    its diagonal block."""
+    B, H, N = 1, 2, 128 * 5 + 72
+    q, k, v = inputs.normal_qkv(B, H, N, d, seed=d * 3 + block)
+    nb = -(-N // block)
+    O, L = run_attn(q, k, v, block, None, causal=True)
+    Or, Lr = masked_attention(q, k, v, block, None, causal=True)
+    check_o(O, Or, f"causal all d={d} block={block}")
+    check_lse(L, Lr, f"causal all d={d} block={block}")
+    mask = inputs.bernoulli_block_mask(B, H, nb, nb, 0.6, seed=block + 3)
+    mask[:, :, 1, :] = 0
+    mask[:, :, 1, 4] = 1
+    mask[:, :, 3, 3] = 0
+    O, L = run_attn(q, k, v, block, mask, causal=True)
+    Or, Lr = masked_attention(q, k, v, block, mask, causal=True)
+    check_o(O, Or, f"causal masked d={d} block={block}")
+    check_lse(L, Lr, f"causal masked d={d} block={block}")
+
+
+@pytest.mark.parametrize("block", [64, 128])
+def test_causal_skip_step_and_radial(block):
+    wl = inputs.Workload("cs", 1, 2, 128, 4, 16, 24, block, "lite", seed=47, sigma_s=2.0, sigma_t=1.5)
+    q, k, v = inputs.rff_qkv(wl)
+    for order in ("ascending", "radial"):
+        S, Sr, _ = _check_skip_step(q, k, v, block, None, None, eps=1.0, order=order, causal=True)
+        nb = wl.nblocks
+        iu = np.triu_indices(nb, 1)
+        assert not S.numpy()[0, :, iu[0], iu[1]].any()        # future blocks never marked
+        assert Sr.sum() > 0

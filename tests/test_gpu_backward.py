@@ -25,15 +25,15 @@ def _lib():
     ops.sa_get_device_status()
 
 
-def run_bwd(q, k, v, dout, block, mask=None):
+def run_bwd(q, k, v, dout, block, mask=None, causal=False):
     """Forward then backward on the GPU; returns (dq, dk, dv) on the host."""
     qd, kd, vd, gd = q.cuda(), k.cuda(), v.cuda(), dout.cuda()
     B, H, N, d = q.shape
     md = None if mask is None else mask.cuda()
     lse = torch.empty(B, H, N, device="cuda")
-    o = ops.sa_sparse_attn_fwd(qd, kd, vd, block, mask=md, lse=lse)
+    o = ops.sa_sparse_attn_fwd(qd, kd, vd, block, mask=md, lse=lse, causal=causal)
     dq, dk, dv = (torch.full_like(qd, float("nan")) for _ in range(3))
-    ops.sa_sparse_attn_bwd(qd, kd, vd, o, gd, lse, block, mask=md, dq=dq, dk=dk, dv=dv)
+    ops.sa_sparse_attn_bwd(qd, kd, vd, o, gd, lse, block, mask=md, dq=dq, dk=dk, dv=dv, causal=causal)
     ops.sa_get_device_status()
     return dq.cpu(), dk.cpu(), dv.cpu()
 
@@ -119,3 +119,15 @@ def test_full_size_480p_sampled_rows():
         check_grad(dq[0, h, rows], rq, f"480p dQ head {h}")
         check_grad(dk[0, h, rows], rk, f"480p dK head {h}")
         check_grad(dv[0, h, rows], rv, f"480p dV head {h}")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("block", [64, 128])
+def test_causal_ragged(d, block):
+    B, H, N = 1, 2, 128 * 5 + 72
+    q, k, v = inputs.normal_qkv(B, H, N, d, seed=d + block + 7)
+    dout = inputs.normal_qkv(B, H, N, d, seed=d + block + 8)[0]
+    nb = -(-N // block)
+    mask = inputs.bernoulli_block_mask(B, H, nb, nb, 0.7, seed=block + 9)
+    got = run_bwd(q, k, v, dout, block, mask, causal=True)
+    check_all(got, masked_attention_bwd(q, k, v, block, mask, dout, causal=True), f"causal d={d} block={block}")

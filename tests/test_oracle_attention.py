@@ -120,3 +120,40 @@ def test_sampled_qblocks_equal_full_computation():
     for (b, h, i), (o, l) in part.items():
         sl = slice(i * wl.block, (i + 1) * wl.block)
         assert np.array_equal(o, O[b, h, sl]) and np.array_equal(l, L[b, h, sl])
+
+
+# ------------------------------------------------------------------ causal ---
+
+def test_causal_all_ones_equals_sdpa_is_causal():
+    g = torch.Generator().manual_seed(21)
+    B, H, N, d, block = 1, 2, 200, 32, 64
+    q, k, v = (torch.randn(B, H, N, d, generator=g, dtype=torch.float64) for _ in range(3))
+    ref = torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=True)
+    O, L = masked_attention(q.numpy(), k.numpy(), v.numpy(), block, None, causal=True)
+    assert np.max(np.abs(O - ref.numpy())) < 1e-12
+    s = (q @ k.transpose(-1, -2)).numpy() / math.sqrt(d)
+    s = np.where(np.tri(N, dtype=bool), s, -np.inf)
+    assert np.max(np.abs(L - logsumexp(s, axis=-1))) < 1e-12
+
+
+def test_causal_block_mask_equals_token_level_brute_force():
+    """Causal with a block mask (diagonal kept or not, empty rows included)
+    against a per-row loop over the visible keys written out directly."""
+    g = np.random.default_rng(22)
+    N, d, block = 150, 8, 32
+    q, k, v = (g.normal(size=(1, 1, N, d)) for _ in range(3))
+    nb = -(-N // block)
+    mask = (g.random((1, 1, nb, nb)) < 0.5).astype(np.uint8)
+    mask[0, 0, 1, :] = 0
+    mask[0, 0, 1, 3] = 1                      # q-block 1 keeps only a future block: no visible key
+    mask[0, 0, 2, 2] = 0                      # q-block 2 without its diagonal block
+    O, L = masked_attention(q, k, v, block, mask, causal=True)
+    for r in range(N):
+        vis = [c for c in range(N) if mask[0, 0, r // block, c // block] and c <= r]
+        if not vis:
+            assert np.all(O[0, 0, r] == 0) and L[0, 0, r] == -np.inf
+            continue
+        s = np.array([q[0, 0, r] @ k[0, 0, c] for c in vis]) / math.sqrt(d)
+        p = np.exp(s - s.max())
+        assert np.max(np.abs(O[0, 0, r] - (p / p.sum()) @ v[0, 0, vis])) < 1e-12
+        assert abs(L[0, 0, r] - (s.max() + math.log(p.sum()))) < 1e-12

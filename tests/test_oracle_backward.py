@@ -121,3 +121,26 @@ def test_pins_catch_planted_mistakes(monkeypatch):
         fd_ok = all(abs(fd_q(i) - dq[0, 0, i, 0]) < 1e-7 for i in range(block, 24))
         assert not (shift_ok and fd_ok), bad.__name__
     monkeypatch.setattr(ob, "attention_bwd_head", good)
+
+
+def test_causal_finite_differences():
+    q, k, v, dout, block, mask = _case(N=24, d=4, block=8, seed=31)
+    mask[:] = 1
+    mask[0, 0, 2, 1] = 0
+    dq, dk, dv = masked_attention_bwd(q, k, v, block, mask, dout, causal=True)
+    h = 1e-5
+
+    def loss(q_, k_, v_):
+        o, _ = masked_attention(q_, k_, v_, block, mask, causal=True)
+        return float(np.sum(o * dout))
+
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        for idx in [(0, 0, 0, 0), (0, 0, 5, 1), (0, 0, 13, 2), (0, 0, 23, 3), (0, 0, 17, 0)]:
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args = {"q": lambda y: (y, k, v), "k": lambda y: (q, y, v), "v": lambda y: (q, k, y)}[name]
+            num = (loss(*args(xp)) - loss(*args(xm))) / (2 * h)
+            assert abs(num - g[idx]) < 1e-7, (name, idx)
+    # the last key takes part only in the last row: its gradients come from that row alone
+    assert np.max(np.abs(dk[0, 0, :23].sum(axis=0) + dk[0, 0, 23])) < 1e-12
