@@ -148,8 +148,8 @@ sa_status sa_build_mask(const void* q, const void* k, int B, int H, int N, int d
                         const float* level_frac, uint8_t* mask_out, float* scores_out, void* workspace,
                         size_t workspace_bytes, void* stream) {
   if (B < 0 || H < 0 || N < 0) return SA_ERR_INVALID_ARG;
-  if (mode != SA_MASK_TAU && mode != SA_MASK_LEVELS) return SA_ERR_INVALID_ARG;
-  if (mode == SA_MASK_TAU && !(tau > 0.f && tau <= 1.f)) return SA_ERR_INVALID_ARG;
+  if (mode != SA_MASK_TAU && mode != SA_MASK_LEVELS && mode != SA_MASK_GLOBAL) return SA_ERR_INVALID_ARG;
+  if ((mode == SA_MASK_TAU || mode == SA_MASK_GLOBAL) && !(tau > 0.f && tau <= 1.f)) return SA_ERR_INVALID_ARG;
   int c0 = 0, c1 = 0, c2 = 0;
   if (B == 0 || H == 0 || N == 0) return SA_OK;
   if (!valid_dim(d) || !valid_block(block)) return SA_ERR_UNSUPPORTED;
@@ -191,6 +191,28 @@ sa_status sa_build_mask(const void* q, const void* k, int B, int H, int N, int d
   }
   const long long nrows = static_cast<long long>(BH) * nb;
   const unsigned warp_grid = static_cast<unsigned>((nrows + 3) / 4);
+  if (mode == SA_MASK_GLOBAL) {
+    // the block means are no longer needed: their space holds the row
+    // statistics, then (Nb > 64) the heads' bins and search state
+    float2* stats = reinterpret_cast<float2*>(qmean);
+    sa::global_row_stats_kernel<<<warp_grid, 128, 0, s>>>(scores, nb, nrows, stats);
+    if (nb <= 64) {
+      sa::global_select_kernel<<<BH, sa::kGlobalThreads, 0, s>>>(scores, stats, nb, tau, mask_out);
+      return cuda_status(cudaGetLastError());
+    }
+    const size_t stats_bytes = (static_cast<size_t>(BH) * nb * sizeof(float2) + 255) / 256 * 256;
+    float* hist = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(qmean) + stats_bytes);
+    auto* state = reinterpret_cast<unsigned long long*>(hist + static_cast<size_t>(BH) * 256);
+    const int per_head = std::max(1, std::min(64, (148 * 4 + BH - 1) / BH));
+    const dim3 gs(per_head, BH);
+    sa::global_init_kernel<<<BH, 256, 0, s>>>(hist, state);
+    for (int pass = 0; pass < 8; ++pass) {
+      sa::global_hist_kernel<<<gs, sa::kGlobalSliceThreads, 0, s>>>(scores, stats, nb, pass, state, hist);
+      sa::global_decide_kernel<<<BH, 256, 0, s>>>(hist, state, nb, tau, pass);
+    }
+    sa::global_mark_kernel<<<gs, sa::kGlobalSliceThreads, 0, s>>>(scores, stats, nb, state, mask_out);
+    return cuda_status(cudaGetLastError());
+  }
   if (nb <= 32)
     sa::block_select_warp_kernel<1><<<warp_grid, 128, 0, s>>>(scores, nb, nrows, mode, tau, c0, c1, c2, mask_out);
   else if (nb <= 64)

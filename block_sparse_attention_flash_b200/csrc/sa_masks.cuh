@@ -488,4 +488,204 @@ __global__ void __launch_bounds__(128) pyramid_pool_kernel(const __nv_bfloat16* 
   store(o8, n8, static_cast<size_t>(r0 / 8), s8, 1.f / rows);
 }
 
+// ------------------------------------------------ global block selection ---
+// VMoBA write-up, "global block selection" and "threshold dynamic selection"
+// paragraphs: the (q-block, k-block) pairs of a head compete with each other
+// rather than within a row, and the head's own concentration decides how many
+// survive.  Reading: P_ij = softmax_j(S_ij) per row; all pairs of the head are
+// visited by descending P (ties: lower i * Nb + j first) and a pair is kept
+// iff the mass visited before it is < tau * Nb (the head's total mass is Nb).
+//
+// Row statistics (max, 1 / sum of exp) first, one warp per row.
+__global__ void __launch_bounds__(128) global_row_stats_kernel(const float* __restrict__ scores, int nb, long long nrows,
+                                                               float2* __restrict__ stats) {
+  const long long row = static_cast<long long>(blockIdx.x) * 4 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= nrows) return;
+  const float* srow = scores + row * nb;
+  float mx = -__int_as_float(0x7f800000);
+  for (int j = lane; j < nb; j += 32) mx = fmaxf(mx, srow[j]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  float sum = 0.f;
+  for (int j = lane; j < nb; j += 32) sum += expf(srow[j] - mx);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+  if (lane == 0) stats[row] = make_float2(mx, 1.f / sum);
+}
+
+// Then one CTA per head finds the last kept pair by a most-significant-first
+// radix search over the 64-bit key (fp32 bits of P, then the complement of the
+// pair index): pass k histograms, by the key's next 8 bits, the mass of the
+// pairs that match the bits fixed so far; the bin where the mass counted from
+// the top first reaches tau * Nb holds the last kept pair.  After 8 passes the
+// key is known and a pair is kept iff its key is >= it.  P is recomputed from
+// the scores in every pass with the same instructions, so it is the same value
+// each time.
+constexpr int kGlobalThreads = 1024;
+constexpr int kGlobalWarps = kGlobalThreads / 32;
+
+__device__ __forceinline__ unsigned long long global_key(const float* srow_scores, const float2 st, int j, int lin) {
+  const float p = expf(srow_scores[j] - st.x) * st.y;
+  return (static_cast<unsigned long long>(__float_as_uint(p)) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(lin));
+}
+
+__global__ void __launch_bounds__(kGlobalThreads) global_select_kernel(const float* __restrict__ scores,
+                                                                       const float2* __restrict__ stats, int nb,
+                                                                       float tau, uint8_t* __restrict__ mask) {
+  __shared__ float hist[kGlobalWarps][256];
+  __shared__ float bin_mass[256];
+  __shared__ unsigned long long s_prefix;
+  __shared__ double s_above;
+  __shared__ int s_keep_all;
+  const int bh = blockIdx.x;
+  const int warp = threadIdx.x >> 5;
+  const float* sc = scores + static_cast<size_t>(bh) * nb * nb;
+  const float2* st = stats + static_cast<size_t>(bh) * nb;
+  const int total = nb * nb;
+  const double target = static_cast<double>(tau) * nb;
+  if (threadIdx.x == 0) {
+    s_prefix = 0ull;
+    s_above = 0.0;
+    s_keep_all = 0;
+  }
+  for (int pass = 0; pass < 8; ++pass) {
+    const int shift = 56 - 8 * pass;
+    for (int i = threadIdx.x; i < kGlobalWarps * 256; i += kGlobalThreads) (&hist[0][0])[i] = 0.f;
+    __syncthreads();
+    const unsigned long long prefix = s_prefix;
+    const unsigned long long hi_mask = pass == 0 ? 0ull : (~0ull << (shift + 8));
+    for (int e = threadIdx.x; e < total; e += kGlobalThreads) {
+      const int i = e / nb, j = e - (e / nb) * nb;
+      const unsigned long long key = global_key(sc + static_cast<size_t>(i) * nb, st[i], j, e);
+      if ((key & hi_mask) == prefix) {
+        const float p = __uint_as_float(static_cast<uint32_t>(key >> 32));
+        atomicAdd(&hist[warp][(key >> shift) & 255u], p);
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x < 256) {
+      float m = 0.f;
+      for (int w = 0; w < kGlobalWarps; ++w) m += hist[w][threadIdx.x];
+      bin_mass[threadIdx.x] = m;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && !s_keep_all) {
+      // bins from the top: the first whose inclusive cumulative mass reaches the target
+      double cum = s_above;
+      int bin = -1;
+      for (int b = 255; b >= 0; --b) {
+        if (cum + bin_mass[b] >= target) {
+          bin = b;
+          break;
+        }
+        cum += bin_mass[b];
+      }
+      if (bin < 0) {
+        s_keep_all = 1;   // the head's mass never reaches the target: keep every pair
+      } else {
+        s_prefix = prefix | (static_cast<unsigned long long>(bin) << shift);
+        s_above = cum;
+      }
+    }
+    __syncthreads();
+    if (s_keep_all) break;
+  }
+  const unsigned long long cut = s_prefix;
+  const bool all = s_keep_all != 0;
+  uint8_t* mk = mask + static_cast<size_t>(bh) * total;
+  for (int e = threadIdx.x; e < total; e += kGlobalThreads) {
+    const int i = e / nb, j = e - (e / nb) * nb;
+    mk[e] = (all || global_key(sc + static_cast<size_t>(i) * nb, st[i], j, e) >= cut) ? uint8_t(1) : uint8_t(0);
+  }
+}
+
+// Many-CTA form of the same search for large heads (Nb > 64): G CTAs per
+// head each histogram a slice of the head's pairs into the head's global bins
+// (one launch per pass), and one CTA per head then picks the bin.  State per
+// head: [0] key prefix, [1] mass above the prefix (double bits), [2] keep-all.
+constexpr int kGlobalSliceThreads = 512;
+
+__global__ void global_init_kernel(float* __restrict__ hist, unsigned long long* __restrict__ state) {
+  const int bh = blockIdx.x;
+  for (int b = threadIdx.x; b < 256; b += blockDim.x) hist[bh * 256 + b] = 0.f;
+  if (threadIdx.x < 4) state[bh * 4 + threadIdx.x] = 0ull;
+}
+
+__global__ void __launch_bounds__(kGlobalSliceThreads) global_hist_kernel(
+    const float* __restrict__ scores, const float2* __restrict__ stats, int nb, int pass,
+    const unsigned long long* __restrict__ state, float* __restrict__ hist) {
+  __shared__ float wh[kGlobalSliceThreads / 32][256];
+  const int bh = blockIdx.y;
+  if (state[bh * 4 + 2]) return;
+  const int warp = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < (kGlobalSliceThreads / 32) * 256; i += kGlobalSliceThreads) (&wh[0][0])[i] = 0.f;
+  __syncthreads();
+  const int shift = 56 - 8 * pass;
+  const unsigned long long prefix = state[bh * 4];
+  const unsigned long long hi_mask = pass == 0 ? 0ull : (~0ull << (shift + 8));
+  const float* sc = scores + static_cast<size_t>(bh) * nb * nb;
+  const float2* st = stats + static_cast<size_t>(bh) * nb;
+  const int total = nb * nb;
+  const int per = (total + gridDim.x - 1) / gridDim.x;
+  const int e0 = blockIdx.x * per, e1 = min(total, e0 + per);
+  for (int e = e0 + threadIdx.x; e < e1; e += kGlobalSliceThreads) {
+    const int i = e / nb, j = e - (e / nb) * nb;
+    const unsigned long long key = global_key(sc + static_cast<size_t>(i) * nb, st[i], j, e);
+    if ((key & hi_mask) == prefix) atomicAdd(&wh[warp][(key >> shift) & 255u], __uint_as_float(static_cast<uint32_t>(key >> 32)));
+  }
+  __syncthreads();
+  if (threadIdx.x < 256) {
+    float m = 0.f;
+    for (int w = 0; w < kGlobalSliceThreads / 32; ++w) m += wh[w][threadIdx.x];
+    if (m != 0.f) atomicAdd(&hist[bh * 256 + threadIdx.x], m);
+  }
+}
+
+__global__ void global_decide_kernel(float* __restrict__ hist, unsigned long long* __restrict__ state, int nb,
+                                     float tau, int pass) {
+  const int bh = blockIdx.x;
+  if (threadIdx.x == 0 && !state[bh * 4 + 2]) {
+    const int shift = 56 - 8 * pass;
+    const double target = static_cast<double>(tau) * nb;
+    double cum = __longlong_as_double(static_cast<long long>(state[bh * 4 + 1]));
+    int bin = -1;
+    for (int b = 255; b >= 0; --b) {
+      const double m = hist[bh * 256 + b];
+      if (cum + m >= target) {
+        bin = b;
+        break;
+      }
+      cum += m;
+    }
+    if (bin < 0) {
+      state[bh * 4 + 2] = 1ull;
+    } else {
+      state[bh * 4] |= static_cast<unsigned long long>(bin) << shift;
+      state[bh * 4 + 1] = static_cast<unsigned long long>(__double_as_longlong(cum));
+    }
+  }
+  __syncthreads();
+  for (int b = threadIdx.x; b < 256; b += blockDim.x) hist[bh * 256 + b] = 0.f;
+}
+
+__global__ void __launch_bounds__(kGlobalSliceThreads) global_mark_kernel(
+    const float* __restrict__ scores, const float2* __restrict__ stats, int nb,
+    const unsigned long long* __restrict__ state, uint8_t* __restrict__ mask) {
+  const int bh = blockIdx.y;
+  const unsigned long long cut = state[bh * 4];
+  const bool all = state[bh * 4 + 2] != 0ull;
+  const float* sc = scores + static_cast<size_t>(bh) * nb * nb;
+  const float2* st = stats + static_cast<size_t>(bh) * nb;
+  const int total = nb * nb;
+  const int per = (total + gridDim.x - 1) / gridDim.x;
+  const int e0 = blockIdx.x * per, e1 = min(total, e0 + per);
+  uint8_t* mk = mask + static_cast<size_t>(bh) * total;
+  for (int e = e0 + threadIdx.x; e < e1; e += kGlobalSliceThreads) {
+    const int i = e / nb, j = e - (e / nb) * nb;
+    mk[e] = (all || global_key(sc + static_cast<size_t>(i) * nb, st[i], j, e) >= cut) ? uint8_t(1) : uint8_t(0);
+  }
+}
+
 }  // namespace sa
+

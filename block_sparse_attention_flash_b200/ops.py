@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(_PKG, "libsparse_attn.so")
 
 SA_OK, SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_CUDA, SA_ERR_TIMEOUT = range(5)
 VISIT_ORDERS = {"ascending": 0, "radial": 1}   # sa_visit_order
-SA_MASK_TAU, SA_MASK_LEVELS = 0, 1
+SA_MASK_TAU, SA_MASK_LEVELS, SA_MASK_GLOBAL = 0, 1, 2
 
 _vp, _i32, _i64, _f32, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
 
@@ -148,7 +148,10 @@ def sa_build_mask(q: torch.Tensor, k: torch.Tensor, block: int, mode: str = "tau
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
     fr = (ctypes.c_float * 3)(*[float(x) for x in level_frac])
-    m = SA_MASK_TAU if mode == "tau" else SA_MASK_LEVELS
+    modes = {"tau": SA_MASK_TAU, "levels": SA_MASK_LEVELS, "global": SA_MASK_GLOBAL}
+    if mode not in modes:
+        raise ValueError(f"mode must be one of {sorted(modes)}")
+    m = modes[mode]
     st = lib().sa_build_mask(_dev(q, "q", torch.bfloat16), _dev(k, "k", torch.bfloat16), B, H, N, d, block, m,
                              float(tau), ctypes.cast(fr, ctypes.c_void_p), _dev(mask_out, "mask_out", torch.uint8),
                              _opt(scores_out, "scores_out", torch.float32), _dev(workspace, "workspace", torch.uint8),

@@ -64,7 +64,7 @@ typedef enum {
   SA_ORDER_RADIAL = 1       /* radial-centric, see sa_sparse_attn_fwd         */
 } sa_visit_order;
 
-enum { SA_MASK_TAU = 0, SA_MASK_LEVELS = 1 };
+enum { SA_MASK_TAU = 0, SA_MASK_LEVELS = 1, SA_MASK_GLOBAL = 2 };
 
 /* Human-readable name of a status code (static string, never NULL). */
 SA_API const char* sa_status_string(sa_status s);
@@ -101,13 +101,19 @@ SA_API size_t sa_build_mask_workspace(int B, int H, int N, int d, int block);
  *   SA_MASK_TAU:    P_i = softmax_j(S_i); visit j by descending S (ties: lower
  *                   j first); mask[j] = 1 iff the mass of the blocks visited
  *                   before j is < tau (the block that crosses tau is kept).
+ *   SA_MASK_GLOBAL: P as for SA_MASK_TAU, but the pairs of a head compete
+ *                   with each other (VMoBA's global selection; the threshold
+ *                   then adapts the count to the head's concentration):
+ *                   visit all (i, j) of the head by descending P_ij (ties:
+ *                   lower i * Nb + j first); mask[i][j] = 1 iff the mass
+ *                   visited before it is < tau * Nb.  A row may keep nothing.
  *   SA_MASK_LEVELS: rank r_j of S_ij in the same order; with quotas
  *                   c_l = ceil(level_frac[l] * Nb) (cumulative fractions,
  *                   non-decreasing), code = 1 if r < c_0, 2 if r < c_1,
  *                   3 if r < c_2, else 4 (code = pyramid level + 1).
  * Arguments
  *   q, k        bf16 [B,H,N,d] device, read only.
- *   tau         (0, 1]; used for SA_MASK_TAU.
+ *   tau         (0, 1]; used for SA_MASK_TAU and SA_MASK_GLOBAL.
  *   level_frac  HOST pointer to 3 floats in [0,1]; used for SA_MASK_LEVELS.
  *   mask_out    uint8 [B,H,Nb,Nb] device, written in full.
  *   scores_out  optional fp32 [B,H,Nb,Nb] device (NULL: kept in workspace).

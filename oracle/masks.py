@@ -11,6 +11,13 @@
   by descending probability (ties: lower k-block index first) and keep a block
   iff the mass of the blocks ranked strictly before it is < tau.  The block
   that crosses tau is kept, so every row keeps at least one block.
+* ``global_mask``: the "global block selection" paragraph (pairs of a head
+  compete with each other instead of within a row) with the threshold of the
+  "threshold dynamic selection" paragraph (the head's concentration sets the
+  count).  Reading: P = per-row softmax of the scores as above; all (i, j) of
+  the head are visited by descending P (ties: lower i * Nkb + j first) and a
+  pair is kept iff the mass visited before it is < tau * Nqb, the head's
+  total mass.  A row may keep nothing.
 * ``level_map``: the PSA page's multi-level mask generator with the fixed
   level quotas: ranks (same order as above, on the scores) below
   ceil(f1*Nkb) get level 0, below ceil(f2*Nkb) level 1, below ceil(f3*Nkb)
@@ -155,3 +162,40 @@ def radial_mask(T, Hh, Ww, block):
                 kexp = t.bit_length() - 1          # floor(log2 t)
                 out[i, j] = 1 if int(dp[i, j]) * (1 << kexp) < S else 0
     return out
+
+
+def global_head(scores_head, tau):
+    """Keep bits and margin flags of one head's [Nqb, Nkb] scores, global selection."""
+    s = np.asarray(scores_head, dtype=np.float64)
+    nqb, nkb = s.shape
+    p = np.exp(s - s.max(axis=1, keepdims=True))
+    p = p / p.sum(axis=1, keepdims=True)
+    flat = p.ravel()
+    order = np.lexsort((np.arange(flat.size), -flat))     # descending P, lower index first
+    mass_before = np.empty_like(flat)
+    mass_before[order] = np.concatenate(([0.0], np.cumsum(flat[order])[:-1]))
+    target = tau * nqb
+    keep = mass_before < target
+    flag = np.abs(mass_before - target) < MARGIN * nqb
+    if keep.any() and (~keep).any():
+        p_in, p_out = flat[keep].min(), flat[~keep].max()
+        flag |= keep & (np.abs(flat - p_out) <= MARGIN * p_out)
+        flag |= (~keep) & (np.abs(flat - p_in) <= MARGIN * p_in)
+    return keep.reshape(nqb, nkb), flag.reshape(nqb, nkb)
+
+
+def global_mask(q, k, block, tau, scale=None, return_info=False):
+    """uint8 [B,H,Nqb,Nkb] mask of the global (per-head) top-mass selection."""
+    S = block_scores(q, k, block, scale)
+    B, H = S.shape[:2]
+    mask = np.zeros(S.shape, dtype=np.uint8)
+    flags = np.zeros(S.shape, dtype=bool)
+    for b in range(B):
+        for h in range(H):
+            keep, flag = global_head(S[b, h], tau)
+            mask[b, h] = keep
+            flags[b, h] = flag
+    if return_info:
+        return mask, flags, S
+    return mask
+

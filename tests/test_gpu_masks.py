@@ -4,7 +4,7 @@ import pytest
 import torch
 
 from block_sparse_attention_flash_b200 import build, inputs, ops
-from oracle import radial_mask, tau_mask, level_map, pyramid_pool
+from oracle import radial_mask, tau_mask, level_map, pyramid_pool, global_mask
 from _parity import check_bits
 
 pytestmark = pytest.mark.gpu
@@ -117,3 +117,25 @@ def test_select_paths_for_long_rows(nb, mode):
     else:
         ref, flags, _ = level_map(q, k, block, (0.1, 0.3, 0.6), return_info=True)
     check_bits(m.cpu(), ref, flags, f"{mode} nb={nb}")
+
+
+@pytest.mark.parametrize("block", [64, 128])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("tau", [0.3, 0.9])
+def test_global_mask_small(block, d, tau):
+    q, k, _ = _small_rff(block, d)
+    m = ops.sa_build_mask(q.cuda(), k.cuda(), block, "global", tau=tau)
+    ops.sa_get_device_status()
+    mr, flags, _ = global_mask(q, k, block, tau, return_info=True)
+    check_bits(m.cpu(), mr, flags, f"global block={block} d={d} tau={tau}")
+
+
+def test_global_mask_480p_grid():
+    """The 480p workload (12 heads, 512 x 512 block pairs per head), tau 0.9."""
+    wl = inputs.WORKLOADS["wan13b_480p_tau"]
+    q, k, _ = inputs.rff_qkv(wl)
+    m = ops.sa_build_mask(q.cuda(), k.cuda(), wl.block, "global", tau=wl.tau)
+    ops.sa_get_device_status()
+    mr, flags, _ = global_mask(q, k, wl.block, wl.tau, return_info=True)
+    nflag = check_bits(m.cpu(), mr, flags, "global 480p")
+    assert nflag <= 0.001 * mr.size

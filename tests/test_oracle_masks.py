@@ -163,3 +163,51 @@ def test_radial_density_hunyuan_720p_grid():
     m = radial_mask(wl.T, wl.Hh, wl.Ww, wl.block)
     assert m.shape == (929, 929)
     assert abs(m.mean() - 0.3707) < 5e-5
+
+
+# ------------------------------------------------------- global selection ---
+
+def test_global_single_row_equals_tau_row():
+    from oracle.masks import global_head, tau_row
+    g = np.random.default_rng(3)
+    for tau in (0.3, 0.5, 0.9):
+        s = g.normal(size=(1, 37)) * 2.0
+        keep, _ = global_head(s, tau)
+        keep_t, _, _, _ = tau_row(s[0], tau)
+        assert np.array_equal(keep[0], keep_t)
+
+
+def test_global_hand_built_peaked_and_uniform_rows():
+    """Row 0 has one dominant block, row 1 is uniform: the head's mass (2) is
+    reached with the peak and then row 1's blocks in index order."""
+    from oracle.masks import global_head
+    s = np.array([[20.0, 0.0, 0.0, 0.0], [0.0, 0.0, 0.0, 0.0]])
+    keep, _ = global_head(s, 0.5)                  # target mass 1.0
+    assert keep.astype(int).tolist() == [[1, 0, 0, 0], [1, 0, 0, 0]]
+    keep, _ = global_head(s, 0.7)                  # target mass 1.4
+    assert keep.astype(int).tolist() == [[1, 0, 0, 0], [1, 1, 0, 0]]
+    keep, _ = global_head(s, 1.0)
+    assert keep.all()
+
+
+def test_global_brute_force_shortest_prefix():
+    """Pure-Python brute force: the kept pairs are the shortest prefix of the
+    pairs sorted by (descending P, index) whose mass reaches tau * Nqb."""
+    from oracle.masks import global_head
+    g = np.random.default_rng(4)
+    s = g.normal(size=(5, 7)) * 1.5
+    for tau in (0.2, 0.55, 0.8):
+        keep, _ = global_head(s, tau)
+        rows = []
+        for i in range(5):
+            e = [math.exp(x - max(s[i])) for x in s[i]]
+            z = sum(e)
+            rows.append([x / z for x in e])
+        pairs = sorted(((rows[i][j], -(i * 7 + j), i, j) for i in range(5) for j in range(7)), reverse=True)
+        acc, want = 0.0, np.zeros((5, 7), dtype=bool)
+        for p, _, i, j in pairs:
+            if acc >= tau * 5:
+                break
+            want[i, j] = True
+            acc += p
+        assert np.array_equal(keep, want)
