@@ -6,6 +6,7 @@
     python -m block_sparse_attention_flash_b200.profile_case pool   [--heads 12] [--reps 2]
     python -m block_sparse_attention_flash_b200.profile_case pyr    [--heads 2] [--reps 2]
     python -m block_sparse_attention_flash_b200.profile_case bwd    [--heads 2] [--reps 2]
+    python -m block_sparse_attention_flash_b200.profile_case perm   [--heads 12] [--reps 2]
 
 Each case uses a workload's real token grid with fewer heads, so one launch
 holds a few hundred MB (larger than L2) and a full profiler capture ends in
@@ -16,6 +17,7 @@ seconds.  Inputs are drawn on the device from the seeded generator.
   pool    32,760-token 480p grid, block 64
   pyr     32,760-token 480p grid, block 64, PSA levels from the GPU level builder
   bwd     32,760-token 480p grid, block 64, all kept: forward once, then the backward
+  perm    32,760-token 480p grid: Q, K, V permuted in one launch (per-head orders, 3x5x4 cells)
 """
 from __future__ import annotations
 
@@ -28,7 +30,7 @@ from . import build, inputs, ops
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["attn", "radial", "mask", "pool", "pyr", "bwd"])
+    ap.add_argument("case", choices=["attn", "radial", "mask", "pool", "pyr", "bwd", "perm"])
     ap.add_argument("--heads", type=int, default=0)
     ap.add_argument("--reps", type=int, default=2)
     args = ap.parse_args()
@@ -65,6 +67,12 @@ def main():
         o = ops.sa_sparse_attn_fwd(q, k, v, wl.block, lse=lse)
         for _ in range(args.reps):
             ops.sa_sparse_attn_bwd(q, k, v, o, dout, lse, wl.block)
+    elif args.case == "perm":
+        wl = inputs.WORKLOADS["wan13b_480p_tau"]
+        q, k, v = inputs.rff_qkv(wl, H=args.heads or wl.H, device=dev)
+        orders = (torch.arange(q.shape[1], device=dev) % 6).to(torch.uint8)
+        for _ in range(args.reps):
+            ops.sa_token_permute([q, k, v], wl.T, wl.Hh, wl.Ww, head_order=orders, cells=(3, 5, 4))
     else:
         wl = inputs.WORKLOADS["psa_480p_pyramid"]
         q, k, v = inputs.rff_qkv(wl, H=args.heads or 2, device=dev)
