@@ -334,9 +334,10 @@ sa_status sa_sparse_attn_fwd(const void* q, const void* k, const void* v, int B,
 
 sa_status sa_pyramid_attn_fwd(const void* q, const void* k, const void* v, int B, int H, int N, int d, int block,
                               const uint8_t* levels, int64_t lv_sb, int64_t lv_sh, int64_t lv_si,
-                              const void* const* k_pool, const void* const* v_pool, float scale, void* o, float* lse,
-                              void* stream) {
+                              const void* const* k_pool, const void* const* v_pool, float scale, int causal, void* o,
+                              float* lse, void* stream) {
   if (B < 0 || H < 0 || N < 0) return SA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return SA_ERR_INVALID_ARG;
   if (std::isnan(scale) || scale < 0.f || std::isinf(scale)) return SA_ERR_INVALID_ARG;
   if (B == 0 || H == 0 || N == 0) return SA_OK;
   if (!valid_dim(d) || !valid_block(block)) return SA_ERR_UNSUPPORTED;
@@ -375,6 +376,7 @@ sa_status sa_pyramid_attn_fwd(const void* q, const void* k, const void* v, int B
   p.lsh = lv_sh;
   p.lsi = lv_si;
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.causal = causal;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   const int n_pairs = ceil_div(ceil_div(N, sa::kTileM), 2);

@@ -54,6 +54,7 @@ struct PyrParams {
   const uint8_t* levels;  // code map: 0 drop, 1 + l level l
   long long lsb, lsh, lsi;
   float scale_log2;
+  int causal;             // k-blocks j > i dropped, the diagonal block at level 0 cut per row
   __nv_bfloat16* o;
   float* lse;
 };
@@ -120,7 +121,8 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
   uint64_t* mma_done = o_final + 2;   // one per MMA-issuing warp
   volatile int* misc = reinterpret_cast<volatile int*>(smem + L::kOffMisc);
   // misc[0] TMEM base, [1]/[2] segments of q-tile 0/1, [3]/[4] key tiles of q-tile 0/1, [5] abort,
-  // [6]/[7] packed columns of q-tile 0/1
+  // [6]/[7] packed columns of q-tile 0/1, [8 + 2t + x] causal: key tile * 256 + column of the
+  // diagonal segment of q-block x of q-tile t (-1: none)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int pair = blockIdx.x, bh = blockIdx.y;
@@ -135,6 +137,11 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
       const int qbA = (qtile0 + t) * QH;
       const int qbB = qbA + QH - 1;
       const bool validA = qbA < p.nb, validB = qbB < p.nb;
+      if (lane == 0) {
+        misc[8 + 2 * t] = -1;
+        misc[9 + 2 * t] = -1;
+      }
+      __syncwarp();
 #pragma unroll 1
       for (int lvl = 0; lvl < 4; ++lvl) {
         for (int base = 0; base < p.nb; base += 32) {
@@ -142,8 +149,14 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
           uint32_t rm = 0;
           if (j < p.nb) {
             const long long rowoff = b * p.lsb + h * p.lsh + j;
-            const int cA = validA ? p.levels[rowoff + qbA * p.lsi] : 0;
-            const int cB = validB ? p.levels[rowoff + qbB * p.lsi] : 0;
+            int cA = validA ? p.levels[rowoff + qbA * p.lsi] : 0;
+            int cB = validB ? p.levels[rowoff + qbB * p.lsi] : 0;
+            if (p.causal) {
+              // blocks after the q-block are dropped; its own block, if kept, is
+              // attended at level 0 (its pooled keys would mix in later tokens)
+              cA = j > qbA ? 0 : (j == qbA && cA ? 1 : cA);
+              cB = j > qbB ? 0 : (j == qbB && cB ? 1 : cB);
+            }
             rm = (cA == lvl + 1 ? 1u : 0u) | (cB == lvl + 1 ? 2u : 0u);
           }
           const unsigned ball = __ballot_sync(0xffffffffu, rm != 0);
@@ -155,6 +168,11 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
             segs[t * kPyrMaxSegs + n + rank] = static_cast<uint32_t>(j) | (static_cast<uint32_t>(lvl) << 16) |
                                                (rm << 18) | (static_cast<uint32_t>(cg & (kTileN - 1)) << 24);
             if ((cg & (kTileN - 1)) == 0) ents[t * kPyrMaxEntries + cg / kTileN] = static_cast<uint16_t>(n + rank);
+            if (p.causal && lvl == 0) {
+              const int where = (cg / kTileN) * 256 + (cg & (kTileN - 1));
+              if ((rm & 1u) && j == qbA) misc[8 + 2 * t] = where;
+              if ((rm & 2u) && j == qbB) misc[9 + 2 * t] = where;
+            }
           }
           n += __popc(ball);
           cols += __popc(ball) * (BLK >> lvl);
@@ -549,6 +567,10 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
     const int cnt = t == 0 ? ntile0 : ntile1;
     const float sl2 = p.scale_log2;
     const float NEG_INF = -__int_as_float(0x7f800000);
+    // causal: where this row's own block sits in the packed key tiles
+    const int xq = (BLK == 64) ? (r >> 6) : 0;
+    const int diag = p.causal ? misc[8 + 2 * t + xq] : -1;
+    const int r_in_blk = r & (BLK - 1);
 
     float m_used = NEG_INF, l_sum = 0.f;
     int et = 0;   // entries of this q-tile processed
@@ -571,6 +593,14 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
         // the S buffer is free for the next entry's S
         tc_fence_before();
         named_bar_sync(kBarSFree + t, kHandoff);
+        if (diag >= 0 && (diag >> 8) == k) {
+          // causal: the diagonal segment's key x (from the block start) is
+          // visible to the row only if x <= the row's position in its block
+          const int c0 = diag & 255;
+#pragma unroll
+          for (int c = 0; c < kTileN; ++c)
+            if (c >= c0 && c < c0 + BLK && c - c0 > r_in_blk) s[c] = NEG_INF;
+        }
         // s already carries the bias (raw logit units): q.k + log2(count) / (scale log2 e),
         // and about -30000 on masked and empty columns
         float a[8];

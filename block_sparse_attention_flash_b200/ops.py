@@ -36,7 +36,7 @@ _SIGNATURES = {
     "sa_sparse_attn_fwd": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _i64, _i64, _i64,
                                   _vp, _vp, _f32, _f32, _i32, _i32, _vp, _vp, _vp]),
     "sa_pyramid_attn_fwd": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _i64, _i64, _i64,
-                                   _vp, _vp, _f32, _vp, _vp, _vp]),
+                                   _vp, _vp, _f32, _i32, _vp, _vp, _vp]),
     "sa_sparse_attn_bwd_workspace": (_sz, [_i32, _i32, _i32]),
     "sa_token_permute": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _i32, _i32, _i32,
                                 _i32, _vp]),
@@ -214,7 +214,7 @@ def sa_sparse_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block:
 
 def sa_pyramid_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block: int, levels: torch.Tensor,
                         k_pool, v_pool, scale: float = 0.0, out: Optional[torch.Tensor] = None,
-                        lse: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+                        lse: Optional[torch.Tensor] = None, stream=None, causal: bool = False) -> torch.Tensor:
     """PSA multi-level attention forward over a level-code map (0 drop, 1+l level l)."""
     B, H, N, d = q.shape
     nb = nblocks(N, block)
@@ -228,7 +228,7 @@ def sa_pyramid_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block
     st = lib().sa_pyramid_attn_fwd(
         _dev(q, "q", torch.bfloat16), _dev(k, "k", torch.bfloat16), _dev(v, "v", torch.bfloat16),
         B, H, N, d, block, levels.data_ptr(), sb, sh, si,
-        ctypes.cast(kp, ctypes.c_void_p), ctypes.cast(vp, ctypes.c_void_p), float(scale),
+        ctypes.cast(kp, ctypes.c_void_p), ctypes.cast(vp, ctypes.c_void_p), float(scale), int(bool(causal)),
         _dev(out, "out", torch.bfloat16), _opt(lse, "lse", torch.float32), _stream(stream))
     _check(st, "sa_pyramid_attn_fwd")
     return out

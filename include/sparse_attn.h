@@ -253,13 +253,18 @@ SA_API sa_status sa_sparse_attn_fwd(const void* q, const void* k, const void* v,
  * by c = 2/4/8 (k_pool/v_pool from sa_pyramid_pool).  A pooled key of a group
  * holding n tokens gets logit scale * q . k_pooled + ln(n).
  *   k_pool, v_pool  HOST arrays of 3 device pointers (c = 2, 4, 8).
+ *   causal          0, or 1 (PSA page: the method serves causal generation
+ *                   too).  Read as: k-blocks j > i are dropped; block i itself,
+ *                   if kept, is attended at level 0 (pooled keys of that block
+ *                   would mix in later tokens) with key c visible to row r
+ *                   only if c <= r; blocks j < i keep their codes.
  * Limits: as sa_sparse_attn_fwd, block == 64 or 128.
  */
 SA_API sa_status sa_pyramid_attn_fwd(const void* q, const void* k, const void* v,
                               int B, int H, int N, int d, int block,
                               const uint8_t* levels, int64_t lv_sb, int64_t lv_sh, int64_t lv_si,
                               const void* const* k_pool, const void* const* v_pool,
-                              float scale, void* o, float* lse, void* stream);
+                              float scale, int causal, void* o, float* lse, void* stream);
 
 /*
  * sa_sparse_attn_bwd — gradients of sa_sparse_attn_fwd with respect to Q, K, V.

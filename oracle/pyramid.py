@@ -13,7 +13,11 @@ Readings:
 * a pooled key stands for the n_g tokens of its group, so its logit gets
   + ln(n_g): if the n_g keys were equal, full attention would weight them
   n_g * exp(s), which is exactly exp(s + ln n_g);
-* level codes: 0 = dropped, 1 + l = attend at level l.
+* level codes: 0 = dropped, 1 + l = attend at level l;
+* causal option (the page: PSA serves causal generation too): k-blocks j > i
+  are dropped; block i itself, if kept, is attended at level 0 (a pooled key
+  of that block would mix in later tokens) with key c visible to row r only
+  if c <= r; blocks j < i keep their codes (all their tokens are earlier).
 """
 from __future__ import annotations
 
@@ -47,7 +51,7 @@ def _level_keys(kh, vh, pooled_k, pooled_v, N, block, j, level):
     return pooled_k[level][g0:g1], pooled_v[level][g0:g1], np.log(counts)
 
 
-def pyramid_attention(q, k, v, block, levels, scale=None, qblocks=None):
+def pyramid_attention(q, k, v, block, levels, scale=None, qblocks=None, causal=False):
     """Multi-level block attention over [B,H,N,d] with a level-code map.
 
     levels: anything broadcastable to uint8 [B,H,Nqb,Nkb] (0 drop, 1+l level l).
@@ -63,19 +67,29 @@ def pyramid_attention(q, k, v, block, levels, scale=None, qblocks=None):
 
     def one(b, h, i):
         r0, r1 = i * block, min(N, (i + 1) * block)
-        ks, vs, bs = [], [], []
+        ks, vs, bs, ids = [], [], [], []
         for j in range(nkb):
             code = int(lv[b, h, i, j])
+            if causal and j > i:
+                code = 0
+            if causal and j == i and code:
+                code = 1
             if code == 0:
                 continue
             kk, vv, bb = _level_keys(k[b, h], v[b, h],
                                      {l: pk[l][b, h] for l in pk},
                                      {l: pv[l][b, h] for l in pv}, N, block, j, code - 1)
             ks.append(kk), vs.append(vv), bs.append(bb)
+            # key index of level-0 columns of the diagonal block, -1 elsewhere
+            ids.append(np.arange(j * block, j * block + kk.shape[0]) if (causal and j == i) else
+                       np.full(kk.shape[0], -1))
         if not ks:
             return np.zeros((r1 - r0, d)), np.full(r1 - r0, -np.inf)
         K, V, bias = np.concatenate(ks), np.concatenate(vs), np.concatenate(bs)
         s = (q[b, h, r0:r1] @ K.T) * scale + bias[None, :]
+        if causal:
+            kid = np.concatenate(ids)
+            s = np.where(kid[None, :] > np.arange(r0, r1)[:, None], -np.inf, s)
         m = s.max(axis=1, keepdims=True)
         e = np.exp(s - m)
         z = e.sum(axis=1, keepdims=True)

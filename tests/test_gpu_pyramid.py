@@ -23,13 +23,13 @@ def _lib():
     ops.sa_get_device_status()
 
 
-def run_pyr(q, k, v, block, codes):
+def run_pyr(q, k, v, block, codes, causal=False):
     qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
     B, H, N, d = q.shape
     kp, vp = ops.sa_pyramid_pool(kd, vd, block)
     out = torch.full_like(qd, float("nan"))
     lse = torch.full((B, H, N), float("nan"), device="cuda")
-    ops.sa_pyramid_attn_fwd(qd, kd, vd, block, codes.cuda(), kp, vp, out=out, lse=lse)
+    ops.sa_pyramid_attn_fwd(qd, kd, vd, block, codes.cuda(), kp, vp, out=out, lse=lse, causal=causal)
     ops.sa_get_device_status()
     return out.cpu(), lse.cpu()
 
@@ -116,3 +116,21 @@ def test_psa_480p_full_sampled():
         want_o.append(o), want_l.append(l)
     check_o(torch.cat(got_o), np.concatenate(want_o), "psa 480p")
     check_lse(torch.cat(got_l), np.concatenate(want_l), "psa 480p")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("block", [64, 128])
+@pytest.mark.parametrize("N", [1031, 2048 + 64 * 3 + 8])
+def test_causal_random_levels_ragged(d, block, N):
+    """Causal option: future blocks dropped, the diagonal block at level 0 with
+    the per-row cut, earlier blocks at their levels; one q-block whose
+    diagonal block is dropped by the map."""
+    B, H = 1, 2
+    q, k, v = inputs.normal_qkv(B, H, N, d, seed=N + d + block + 1)
+    nb = -(-N // block)
+    codes = _codes(B, H, nb, seed=N * 5 + block)
+    codes[0, 0, 3, 3] = 0
+    O, L = run_pyr(q, k, v, block, codes, causal=True)
+    Or, Lr = pyramid_attention(q, k, v, block, codes.numpy(), causal=True)
+    check_o(O, Or, f"causal pyramid N={N} d={d} block={block}")
+    check_lse(L, Lr, f"causal pyramid N={N} d={d} block={block}")

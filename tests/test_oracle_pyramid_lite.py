@@ -53,6 +53,27 @@ def test_constant_groups_make_any_level_mix_exact():
     assert np.max(np.abs(Oc - Od)) < 1e-12
 
 
+def test_causal_constant_groups_equal_causal_attention():
+    """Causal option with K/V constant over 8-token groups: earlier blocks at
+    any level are exact, so pyramid attention equals causal masked attention
+    with the same kept blocks; all-level-0 codes equal it for any K/V."""
+    N, d, block = 64 * 5 + 24, 16, 64
+    g = torch.Generator().manual_seed(23)
+    q = torch.randn(1, 2, N, d, generator=g).to(torch.bfloat16)
+    k, v = inputs.const_group_kv(1, 2, N, d, 8, seed=24)
+    nb = -(-N // block)
+    codes = torch.randint(0, 5, (1, 2, nb, nb), generator=g).numpy().astype(np.uint8)
+    O, L = pyramid_attention(q, k, v, block, codes, causal=True)
+    Om, Lm = masked_attention(q, k, v, block, (codes != 0).astype(np.uint8), causal=True)
+    assert np.max(np.abs(O - Om)) < 1e-12
+    fin = np.isfinite(Lm)
+    assert np.array_equal(fin, np.isfinite(L)) and np.max(np.abs(L[fin] - Lm[fin])) < 1e-12
+    q2, k2, v2 = inputs.normal_qkv(1, 2, N, d, seed=25)
+    O1, _ = pyramid_attention(q2, k2, v2, block, np.ones_like(codes), causal=True)
+    Om1, _ = masked_attention(q2, k2, v2, block, None, causal=True)
+    assert np.max(np.abs(O1 - Om1)) < 1e-12
+
+
 def test_exactness_pin_catches_a_wrong_correction(monkeypatch):
     """Plant a sign error in the oracle's ln(count) bias: the pin must fail."""
     import oracle.pyramid as pyr
