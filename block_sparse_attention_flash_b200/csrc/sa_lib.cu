@@ -213,6 +213,21 @@ sa_status sa_build_mask(const void* q, const void* k, int B, int H, int N, int d
     sa::global_mark_kernel<<<gs, sa::kGlobalSliceThreads, 0, s>>>(scores, stats, nb, state, mask_out);
     return cuda_status(cudaGetLastError());
   }
+  if (mode == SA_MASK_TAU && nb <= 1024) {
+    if (nb <= 32)
+      sa::tau_select_warp_kernel<1><<<warp_grid, 128, 0, s>>>(scores, nb, nrows, tau, mask_out);
+    else if (nb <= 64)
+      sa::tau_select_warp_kernel<2><<<warp_grid, 128, 0, s>>>(scores, nb, nrows, tau, mask_out);
+    else if (nb <= 128)
+      sa::tau_select_warp_kernel<4><<<warp_grid, 128, 0, s>>>(scores, nb, nrows, tau, mask_out);
+    else if (nb <= 256)
+      sa::tau_select_warp_kernel<8><<<warp_grid, 128, 0, s>>>(scores, nb, nrows, tau, mask_out);
+    else if (nb <= 512)
+      sa::tau_select_warp_kernel<16><<<warp_grid, 128, 0, s>>>(scores, nb, nrows, tau, mask_out);
+    else
+      sa::tau_select_warp_kernel<32><<<warp_grid, 128, 0, s>>>(scores, nb, nrows, tau, mask_out);
+    return cuda_status(cudaGetLastError());
+  }
   if (nb <= 32)
     sa::block_select_warp_kernel<1><<<warp_grid, 128, 0, s>>>(scores, nb, nrows, mode, tau, c0, c1, c2, mask_out);
   else if (nb <= 64)

@@ -421,6 +421,88 @@ __global__ void __launch_bounds__(128) block_select_warp_kernel(const float* __r
   for (int j = lane; j < nb; j += 32) mrow[j] = stage[warp][j];
 }
 
+// TAU rows without a sort (rows of at most 32*E blocks, one warp per row):
+// the kept set is the shortest prefix, in (descending score, ascending j)
+// order, whose probability mass reaches tau.  Its last key K* is the smallest
+// 32-bit score key whose cumulative mass reaches tau; it is found bit by bit
+// from the most significant end (32 rounds of a masked warp sum).  Blocks
+// with a key below K* are kept; blocks whose key equals K* (equal scores) are
+// kept in ascending j while the mass before them is < tau.
+template <int E>
+__global__ void __launch_bounds__(128) tau_select_warp_kernel(const float* __restrict__ scores, int nb,
+                                                              long long nrows, float tau,
+                                                              uint8_t* __restrict__ mask_out) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long row = static_cast<long long>(blockIdx.x) * 4 + warp;
+  if (row >= nrows) return;
+  const float* srow = scores + row * nb;
+  float sc[E], pr[E];
+  uint32_t key[E];
+  float mx = -__int_as_float(0x7f800000);
+#pragma unroll
+  for (int k = 0; k < E; ++k) {
+    const int i = lane * E + k;
+    sc[k] = i < nb ? srow[i] : -__int_as_float(0x7f800000);
+    mx = fmaxf(mx, sc[k]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  float sum = 0.f;
+#pragma unroll
+  for (int k = 0; k < E; ++k) {
+    const int i = lane * E + k;
+    pr[k] = i < nb ? expf(sc[k] - mx) : 0.f;
+    sum += pr[k];
+    key[k] = i < nb ? ~float_order_key(sc[k]) : 0xFFFFFFFFu;   // ascending key = descending score
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  const float inv = 1.f / sum;
+#pragma unroll
+  for (int k = 0; k < E; ++k) pr[k] *= inv;
+  // smallest K with mass(key <= K) >= tau (all ones when the total stays below tau)
+  uint32_t kstar = 0u;
+#pragma unroll 1
+  for (int b = 31; b >= 0; --b) {
+    const uint32_t cand = kstar | ((1u << b) - 1u);
+    float m = 0.f;
+#pragma unroll
+    for (int k = 0; k < E; ++k) m += key[k] <= cand ? pr[k] : 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m += __shfl_xor_sync(0xffffffffu, m, o);
+    if (!(m >= tau)) kstar |= 1u << b;
+  }
+  // mass strictly before K*, and the rank in j of each block tied at K*
+  float below = 0.f;
+  int ties = 0;
+#pragma unroll
+  for (int k = 0; k < E; ++k) {
+    below += key[k] < kstar ? pr[k] : 0.f;
+    ties += key[k] == kstar && (lane * E + k) < nb ? 1 : 0;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) below += __shfl_xor_sync(0xffffffffu, below, o);
+  int tie_before = ties;   // exclusive prefix over lanes (blocks are numbered lane * E + k)
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, tie_before, o);
+    if (lane >= o) tie_before += y;
+  }
+  tie_before -= ties;
+  uint8_t* mrow = mask_out + row * nb;
+#pragma unroll
+  for (int k = 0; k < E; ++k) {
+    const int i = lane * E + k;
+    if (i >= nb) continue;
+    uint8_t keep = key[k] < kstar ? 1 : 0;
+    if (key[k] == kstar) {
+      keep = below + static_cast<float>(tie_before) * pr[k] < tau ? 1 : 0;
+      ++tie_before;
+    }
+    mrow[i] = keep;
+  }
+}
+
 // ----------------------------------------------------------- pyramid pool ---
 // grid (ceil(N / (8 * GPB)), B*H, 2); z = 0 pools K, z = 1 pools V.  Thread
 // (g, ch) owns the 8-token group g of the CTA and 16-byte chunk ch: it loads
