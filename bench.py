@@ -111,6 +111,29 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def replica_seed(base_seed, rank):
+    """Seed of a rank's drift noise: every replica runs its own copy of the workload."""
+    return base_seed + 1 + 1000 * rank
+
+
+def reduce_over_ranks(total_ms, work, world, device):
+    """(max over ranks of the timed region, sum over ranks of the work done).
+
+    Every rank calls this with its own numbers; the whole-job value is the
+    summed work over the slowest rank's time."""
+    if world == 1:
+        return float(total_ms), float(work)
+    t = torch.tensor([float(total_ms)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    w = torch.tensor([float(work)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(w, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item()), float(w.item())
+
+
+def whole_job_tflops(work_all, ms_max):
+    return work_all / (ms_max * 1e-3) / 1e12
+
+
 def executed_flops(skip_in, N, block, d, mask=None):
     """4 * d * sum over visited (i, j) of valid rows_i * valid cols_j."""
     nb = -(-N // block)
@@ -142,7 +165,7 @@ def run_ours(args, rank, world, local):
     # Per-step inputs, drawn on the device before timing (the chain's drift).
     q0, k0, v0 = inputs.rff_qkv(wl, device=dev)
     g = torch.Generator(device=dev)
-    g.manual_seed(wl.seed + 1 + 1000 * rank)
+    g.manual_seed(replica_seed(wl.seed, rank))
     qkv = [(q0, k0, v0)]
     for s in range(1, nsteps):
         q, k, v = qkv[-1]
@@ -182,15 +205,7 @@ def run_ours(args, rank, world, local):
     kern_ms = [ev[s][0].elapsed_time(ev[s][1]) for s in range(args.warmup, nsteps)]
     flops = [executed_flops(skips[s], N, block, d) for s in range(args.warmup, nsteps)]
     dense = 4.0 * d * N * N * B * H
-    my = torch.tensor([total_ms, sum(flops)], dtype=torch.float64, device=dev)
-    if world > 1:
-        t = my[:1].clone()
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        f = my[1:].clone()
-        torch.distributed.all_reduce(f, op=torch.distributed.ReduceOp.SUM)
-        total_ms_max, flops_all = float(t.item()), float(f.item())
-    else:
-        total_ms_max, flops_all = total_ms, sum(flops)
+    total_ms_max, flops_all = reduce_over_ranks(total_ms, sum(flops), world, dev)
 
     # end-to-end through the public API with host buffers (rank-local)
     e2e = None
@@ -211,7 +226,7 @@ def run_ours(args, rank, world, local):
     skip_rate = 1.0 - sum(flops) / (dense * len(flops))
     line = {
         "metric": METRIC,
-        "value": round(flops_all / (total_ms_max * 1e-3) / 1e12, 2),
+        "value": round(whole_job_tflops(flops_all, total_ms_max), 2),
         "unit": "TFLOP/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -270,12 +285,9 @@ def run_e2e(ops, qkv0, block, eps, nb, dev, stream, steps, world):
     b.record(stream)
     torch.cuda.synchronize(dev)
     ms = a.elapsed_time(b)
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
-    flops = sum(executed_flops(skips[s], N, block, d) for s in range(1, steps + 1)) * world
-    return {"value": round(flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+    ms, flops = reduce_over_ranks(ms, sum(executed_flops(skips[s], N, block, d) for s in range(1, steps + 1)),
+                                  world, dev)
+    return {"value": round(whole_job_tflops(flops, ms), 2), "unit": "TFLOP/s",
             "h2d_bytes_per_step": 3 * q0.numel() * 2, "d2h_bytes_per_step": q0.numel() * 2,
             "ms_per_step": round(ms / steps, 3), "steps": steps}
 
