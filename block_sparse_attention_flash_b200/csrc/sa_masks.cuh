@@ -122,20 +122,32 @@ __global__ void __launch_bounds__(256) block_scores_kernel(const float* __restri
   for (int a = 0; a < 4; ++a)
 #pragma unroll
     for (int c = 0; c < 4; ++c) acc[a][c] = 0.f;
+  // the next chunk's operands are loaded into registers while this chunk is
+  // multiplied (512 float4 per operand chunk, two per thread)
+  float4 pa[2], pb[2];
+  auto fetch = [&](int kc) {
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int idx = threadIdx.x + u * 256;
+      const int rr = idx >> 3, c4 = (idx & 7) * 4;
+      pa[u] = (i0 + rr < nb) ? *reinterpret_cast<const float4*>(qm + static_cast<size_t>(i0 + rr) * D + kc + c4)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+      pb[u] = (j0 + rr < nb) ? *reinterpret_cast<const float4*>(km + static_cast<size_t>(j0 + rr) * D + kc + c4)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  fetch(0);
 #pragma unroll 1
   for (int kc = 0; kc < D; kc += 32) {
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
-      const int idx = threadIdx.x + u * 256;   // 512 float4 per operand chunk
+      const int idx = threadIdx.x + u * 256;
       const int rr = idx >> 3, c4 = (idx & 7) * 4;
-      const float4 av = (i0 + rr < nb) ? *reinterpret_cast<const float4*>(qm + static_cast<size_t>(i0 + rr) * D + kc + c4)
-                                       : make_float4(0.f, 0.f, 0.f, 0.f);
-      const float4 bv = (j0 + rr < nb) ? *reinterpret_cast<const float4*>(km + static_cast<size_t>(j0 + rr) * D + kc + c4)
-                                       : make_float4(0.f, 0.f, 0.f, 0.f);
-      sa[c4 + 0][rr] = av.x; sa[c4 + 1][rr] = av.y; sa[c4 + 2][rr] = av.z; sa[c4 + 3][rr] = av.w;
-      sb[c4 + 0][rr] = bv.x; sb[c4 + 1][rr] = bv.y; sb[c4 + 2][rr] = bv.z; sb[c4 + 3][rr] = bv.w;
+      sa[c4 + 0][rr] = pa[u].x; sa[c4 + 1][rr] = pa[u].y; sa[c4 + 2][rr] = pa[u].z; sa[c4 + 3][rr] = pa[u].w;
+      sb[c4 + 0][rr] = pb[u].x; sb[c4 + 1][rr] = pb[u].y; sb[c4 + 2][rr] = pb[u].z; sb[c4 + 3][rr] = pb[u].w;
     }
     __syncthreads();
+    if (kc + 32 < D) fetch(kc + 32);
 #pragma unroll 8
     for (int k = 0; k < 32; ++k) {
       const float4 a = *reinterpret_cast<const float4*>(&sa[k][ty * 4]);
