@@ -131,3 +131,31 @@ def test_causal_ragged(d, block):
     mask = inputs.bernoulli_block_mask(B, H, nb, nb, 0.7, seed=block + 9)
     got = run_bwd(q, k, v, dout, block, mask, causal=True)
     check_all(got, masked_attention_bwd(q, k, v, block, mask, dout, causal=True), f"causal d={d} block={block}")
+
+
+@pytest.mark.parametrize("layout", ["2d", "3d", "4d"])
+def test_batch_two_mask_layouts(layout):
+    """B = 2 with the mask given as [Nb, Nb] (broadcast), [H, Nb, Nb] or a full
+    [B, H, Nb, Nb] array: the element strides reach the kernels unchanged."""
+    B, H, N, d, block = 2, 3, 128 * 4 + 56, 128, 64
+    q, k, v = inputs.normal_qkv(B, H, N, d, seed=81)
+    dout = inputs.normal_qkv(B, H, N, d, seed=82)[0]
+    nb = -(-N // block)
+    full = inputs.bernoulli_block_mask(B, H, nb, nb, 0.5, seed=83)
+    if layout == "2d":
+        m = full[0, 0]
+        ref_mask = m.view(1, 1, nb, nb).expand(B, H, nb, nb)
+    elif layout == "3d":
+        m = full[0]
+        ref_mask = m.view(1, H, nb, nb).expand(B, H, nb, nb)
+    else:
+        m = full
+        ref_mask = full
+    md = m.cuda()
+    qd, kd, vd, gd = q.cuda(), k.cuda(), v.cuda(), dout.cuda()
+    lse = torch.empty(B, H, N, device="cuda")
+    o = ops.sa_sparse_attn_fwd(qd, kd, vd, block, mask=md, lse=lse)
+    dq, dk, dv = ops.sa_sparse_attn_bwd(qd, kd, vd, o, gd, lse, block, mask=md)
+    ops.sa_get_device_status()
+    ref = masked_attention_bwd(q, k, v, block, ref_mask.numpy(), dout)
+    check_all((dq.cpu(), dk.cpu(), dv.cpu()), ref, f"batch 2 mask {layout}")

@@ -134,3 +134,19 @@ def test_causal_random_levels_ragged(d, block, N):
     Or, Lr = pyramid_attention(q, k, v, block, codes.numpy(), causal=True)
     check_o(O, Or, f"causal pyramid N={N} d={d} block={block}")
     check_lse(L, Lr, f"causal pyramid N={N} d={d} block={block}")
+
+
+def test_batch_two_broadcast_levels():
+    """B = 2, H = 3 with one [Nb, Nb] level map broadcast over batch and heads."""
+    B, H, N, d, block = 2, 3, 64 * 11 + 40, 128, 64
+    q, k, v = inputs.normal_qkv(B, H, N, d, seed=84)
+    nb = -(-N // block)
+    codes = _codes(1, 1, nb, seed=85)[0, 0]
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    kp, vp = ops.sa_pyramid_pool(kd, vd, block)
+    lse = torch.empty(B, H, N, device="cuda")
+    out = ops.sa_pyramid_attn_fwd(qd, kd, vd, block, codes.cuda(), kp, vp, lse=lse)
+    ops.sa_get_device_status()
+    Or, Lr = pyramid_attention(q, k, v, block, codes.numpy())
+    check_o(out.cpu(), Or, "pyramid batch 2")
+    check_lse(lse.cpu(), Lr, "pyramid batch 2")
