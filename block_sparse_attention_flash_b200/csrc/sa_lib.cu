@@ -616,3 +616,117 @@ sa_status sa_token_permute(const void* const* src, void* const* dst, int n_tenso
 }
 
 }  // extern "C"
+
+// ------------------------------------------- forward from host buffers ---
+// Q, K, V come from host memory and O goes back to it: the (b, h) rows are
+// streamed through the device in chunks of `heads_per_chunk` heads, two chunk
+// buffers in turn, so that the copy of chunk c + 1 in, the attention of chunk
+// c and the copy of chunk c - 1 out run at the same time (host-to-device and
+// device-to-host on two streams of their own, the attention on the caller's
+// stream).  One cudaMemcpyAsync per tensor and chunk.
+namespace {
+
+size_t host_chunk_elems(int N, int d, int hc) { return static_cast<size_t>(hc) * N * d; }
+
+}  // namespace
+
+extern "C" {
+
+size_t sa_sparse_attn_fwd_host_workspace(int N, int d, int heads_per_chunk) {
+  if (N <= 0 || d <= 0 || heads_per_chunk <= 0) return 0;
+  return 2 * 4 * host_chunk_elems(N, d, heads_per_chunk) * 2;   // 2 buffers x (Q, K, V, O) x bf16
+}
+
+sa_status sa_sparse_attn_fwd_host(const void* q, const void* k, const void* v, int B, int H, int N, int d,
+                                  int block, const uint8_t* mask, int64_t mask_sb, int64_t mask_sh,
+                                  int64_t mask_si, const uint8_t* skip_in, uint8_t* skip_out, float eps,
+                                  float scale, int order, int causal, void* o, float* lse, void* workspace,
+                                  size_t workspace_bytes, int heads_per_chunk, void* stream) {
+  if (B < 0 || H < 0 || N < 0 || heads_per_chunk <= 0) return SA_ERR_INVALID_ARG;
+  if (B == 0 || H == 0 || N == 0) return SA_OK;
+  if (!q || !k || !v || !o || !workspace) return SA_ERR_INVALID_ARG;
+  if (!valid_dim(d) || !valid_block(block)) return SA_ERR_UNSUPPORTED;
+  const int hc = std::min(heads_per_chunk, H);
+  if (workspace_bytes < sa_sparse_attn_fwd_host_workspace(N, d, hc)) return SA_ERR_INVALID_ARG;
+  if (!aligned16(workspace)) return SA_ERR_INVALID_ARG;
+  const size_t ce = host_chunk_elems(N, d, hc);
+  auto* ws = static_cast<__nv_bfloat16*>(workspace);
+  __nv_bfloat16* buf[2][4];
+  for (int s = 0; s < 2; ++s)
+    for (int t = 0; t < 4; ++t) buf[s][t] = ws + (static_cast<size_t>(s) * 4 + t) * ce;
+  const auto* hq = static_cast<const __nv_bfloat16*>(q);
+  const auto* hk = static_cast<const __nv_bfloat16*>(k);
+  const auto* hv = static_cast<const __nv_bfloat16*>(v);
+  auto* ho = static_cast<__nv_bfloat16*>(o);
+  const size_t nb = static_cast<size_t>(ceil_div(N, block));
+  const size_t head_elems = static_cast<size_t>(N) * d;
+
+  cudaStream_t cs = as_stream(stream);
+  cudaStream_t in_s = nullptr, out_s = nullptr;
+  cudaEvent_t loaded[2] = {nullptr, nullptr}, computed[2] = {nullptr, nullptr}, stored[2] = {nullptr, nullptr};
+  sa_status st = SA_OK;
+  auto ok = [&](cudaError_t e) {
+    if (e != cudaSuccess && st == SA_OK) st = SA_ERR_CUDA;
+    return st == SA_OK;
+  };
+  ok(cudaStreamCreateWithFlags(&in_s, cudaStreamNonBlocking));
+  ok(cudaStreamCreateWithFlags(&out_s, cudaStreamNonBlocking));
+  for (int s = 0; s < 2 && st == SA_OK; ++s) {
+    ok(cudaEventCreateWithFlags(&loaded[s], cudaEventDisableTiming));
+    ok(cudaEventCreateWithFlags(&computed[s], cudaEventDisableTiming));
+    ok(cudaEventCreateWithFlags(&stored[s], cudaEventDisableTiming));
+  }
+  // the copies in must not overtake work the caller queued on its stream before this call
+  cudaEvent_t start = nullptr;
+  if (ok(cudaEventCreateWithFlags(&start, cudaEventDisableTiming)) && ok(cudaEventRecord(start, cs)))
+    ok(cudaStreamWaitEvent(in_s, start, 0));
+  int chunk = 0;
+  for (int b = 0; b < B && st == SA_OK; ++b) {
+    for (int h0 = 0; h0 < H && st == SA_OK; h0 += hc, ++chunk) {
+      const int nh = std::min(hc, H - h0);
+      const int s = chunk & 1;
+      const size_t off = (static_cast<size_t>(b) * H + h0) * head_elems;
+      const size_t bytes = static_cast<size_t>(nh) * head_elems * 2;
+      // buffer s was last read by chunk - 2's attention and its O copied out
+      if (chunk >= 2) {
+        ok(cudaStreamWaitEvent(in_s, computed[s], 0));
+      }
+      ok(cudaMemcpyAsync(buf[s][0], hq + off, bytes, cudaMemcpyHostToDevice, in_s));
+      ok(cudaMemcpyAsync(buf[s][1], hk + off, bytes, cudaMemcpyHostToDevice, in_s));
+      ok(cudaMemcpyAsync(buf[s][2], hv + off, bytes, cudaMemcpyHostToDevice, in_s));
+      ok(cudaEventRecord(loaded[s], in_s));
+      ok(cudaStreamWaitEvent(cs, loaded[s], 0));
+      if (chunk >= 2) ok(cudaStreamWaitEvent(cs, stored[s], 0));
+      if (st != SA_OK) break;
+      const uint8_t* mk = mask ? mask + b * mask_sb + static_cast<int64_t>(h0) * mask_sh : nullptr;
+      const size_t so = (static_cast<size_t>(b) * H + h0) * nb * nb;
+      const sa_status a = sa_sparse_attn_fwd(buf[s][0], buf[s][1], buf[s][2], 1, nh, N, d, block, mk, 0, mask_sh,
+                                             mask_si, skip_in ? skip_in + so : nullptr,
+                                             skip_out ? skip_out + so : nullptr, eps, scale, order, causal,
+                                             buf[s][3], lse ? lse + (static_cast<size_t>(b) * H + h0) * N : nullptr,
+                                             stream);
+      if (a != SA_OK) {
+        st = a;
+        break;
+      }
+      ok(cudaEventRecord(computed[s], cs));
+      ok(cudaStreamWaitEvent(out_s, computed[s], 0));
+      ok(cudaMemcpyAsync(ho + off, buf[s][3], bytes, cudaMemcpyDeviceToHost, out_s));
+      ok(cudaEventRecord(stored[s], out_s));
+    }
+  }
+  // the caller's stream sees every copy out before anything it queues next
+  for (int s = 0; s < 2; ++s)
+    if (stored[s]) cudaStreamWaitEvent(cs, stored[s], 0);
+  for (int s = 0; s < 2; ++s) {
+    if (loaded[s]) cudaEventDestroy(loaded[s]);
+    if (computed[s]) cudaEventDestroy(computed[s]);
+    if (stored[s]) cudaEventDestroy(stored[s]);
+  }
+  if (start) cudaEventDestroy(start);
+  if (in_s) cudaStreamDestroy(in_s);
+  if (out_s) cudaStreamDestroy(out_s);
+  return st;
+}
+
+}  // extern "C"

@@ -38,6 +38,9 @@ _SIGNATURES = {
     "sa_pyramid_attn_fwd": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _i64, _i64, _i64,
                                    _vp, _vp, _f32, _i32, _vp, _vp, _vp]),
     "sa_sparse_attn_bwd_workspace": (_sz, [_i32, _i32, _i32]),
+    "sa_sparse_attn_fwd_host_workspace": (_sz, [_i32, _i32, _i32]),
+    "sa_sparse_attn_fwd_host": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _i64, _i64, _i64,
+                                       _vp, _vp, _f32, _f32, _i32, _i32, _vp, _vp, _vp, _sz, _i32, _vp]),
     "sa_token_permute": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _i32, _i32, _i32,
                                 _i32, _vp]),
     "sa_sparse_attn_bwd": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _i64, _i64, _i64,
@@ -297,5 +300,50 @@ def sa_token_permute(tensors, T: int, Hh: int, Ww: int, order="thw", head_order:
                                 B, H, T, Hh, Ww, d, code, hptr, int(cells[0]), int(cells[1]), int(cells[2]),
                                 int(bool(inverse)), _stream(stream))
     _check(st, "sa_token_permute")
+    return out
+
+
+def _host(t: torch.Tensor, name: str, dtype: torch.dtype) -> int:
+    if not isinstance(t, torch.Tensor) or t.is_cuda:
+        raise ValueError(f"{name} must be a host tensor")
+    if t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {dtype} tensor")
+    return t.data_ptr()
+
+
+def sa_sparse_attn_fwd_host_workspace(N: int, d: int, heads_per_chunk: int) -> int:
+    return int(lib().sa_sparse_attn_fwd_host_workspace(N, d, heads_per_chunk))
+
+
+def sa_sparse_attn_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block: int, out: torch.Tensor,
+                            mask: Optional[torch.Tensor] = None, skip_in: Optional[torch.Tensor] = None,
+                            skip_out: Optional[torch.Tensor] = None, eps: float = math.inf, scale: float = 0.0,
+                            lse: Optional[torch.Tensor] = None, heads_per_chunk: int = 4,
+                            workspace: Optional[torch.Tensor] = None, stream=None, order: str = "ascending",
+                            causal: bool = False, device=None) -> torch.Tensor:
+    """sa_sparse_attn_fwd with q, k, v and out in host memory (pin them for overlap)."""
+    B, H, N, d = q.shape
+    nb = nblocks(N, block)
+    hc = min(heads_per_chunk, H)
+    if workspace is None:
+        dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
+        workspace = torch.empty(sa_sparse_attn_fwd_host_workspace(N, d, hc), dtype=torch.uint8, device=dev)
+    sb = sh = si = 0
+    mptr = None
+    if mask is not None:
+        if mask.dtype != torch.uint8 or not mask.is_cuda:
+            raise ValueError("mask must be a CUDA uint8 tensor")
+        sb, sh, si = _mask_strides(mask, B, H, nb)
+        mptr = mask.data_ptr()
+    for name, t in (("skip_in", skip_in), ("skip_out", skip_out)):
+        if t is not None and tuple(t.shape) != (B, H, nb, nb):
+            raise ValueError(f"{name} must be [{B}, {H}, {nb}, {nb}]")
+    st = lib().sa_sparse_attn_fwd_host(
+        _host(q, "q", torch.bfloat16), _host(k, "k", torch.bfloat16), _host(v, "v", torch.bfloat16),
+        B, H, N, d, block, mptr, sb, sh, si, _opt(skip_in, "skip_in", torch.uint8),
+        _opt(skip_out, "skip_out", torch.uint8), float(eps), float(scale), VISIT_ORDERS[order], int(bool(causal)),
+        _host(out, "out", torch.bfloat16), _opt(lse, "lse", torch.float32), _dev(workspace, "workspace", torch.uint8),
+        workspace.numel(), hc, _stream(stream))
+    _check(st, "sa_sparse_attn_fwd_host")
     return out
 

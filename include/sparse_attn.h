@@ -303,6 +303,36 @@ SA_API sa_status sa_sparse_attn_bwd(const void* q, const void* k, const void* v,
                              size_t workspace_bytes, void* stream);
 
 /*
+ * sa_sparse_attn_fwd_host — sa_sparse_attn_fwd with Q, K, V and O in HOST memory.
+ *   No page counterpart: the pages run attention inside a model on the GPU.
+ *   This entry point serves callers whose tensors live in host memory; it
+ *   streams the (b, h) rows through the device so the transfers overlap the
+ *   attention.
+ *
+ * q, k, v, o are HOST bf16 [B,H,N,d] (page-locked memory makes the copies
+ * asynchronous; pageable memory works but serialises them).  Every other
+ * argument is as sa_sparse_attn_fwd (mask, skip_in, skip_out, lse: device).
+ * The heads go through the device in chunks of heads_per_chunk heads of one
+ * batch entry, two chunk buffers in turn: the copies in of chunk c + 1, the
+ * attention of chunk c (on `stream`) and the copy out of chunk c - 1 run
+ * concurrently (the copies on two streams this call creates and releases).
+ * Work queued on `stream` before the call completes before the first copy;
+ * work queued after it starts after the last copy out.  Each chunk gives the
+ * same results as one sa_sparse_attn_fwd call over all heads.
+ *   workspace     device scratch of sa_sparse_attn_fwd_host_workspace(N, d,
+ *                 min(heads_per_chunk, H)) bytes, 16-byte aligned.
+ * Returns the first error; a call that fails part way may have written some
+ * chunks.
+ */
+SA_API size_t sa_sparse_attn_fwd_host_workspace(int N, int d, int heads_per_chunk);
+SA_API sa_status sa_sparse_attn_fwd_host(const void* q, const void* k, const void* v,
+                                  int B, int H, int N, int d, int block,
+                                  const uint8_t* mask, int64_t mask_sb, int64_t mask_sh, int64_t mask_si,
+                                  const uint8_t* skip_in, uint8_t* skip_out, float eps, float scale,
+                                  int order, int causal, void* o, float* lse, void* workspace,
+                                  size_t workspace_bytes, int heads_per_chunk, void* stream);
+
+/*
  * sa_token_permute — reorder the tokens of the (t, h, w) grid, per head.
  *   PAROAttention write-up (pattern-aware reordering paragraphs: 6 orders of
  *   the three axes, one chosen per head, so that scattered attention becomes

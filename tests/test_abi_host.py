@@ -30,7 +30,8 @@ def test_header_declares_the_entry_points():
     names = _declared_symbols()
     for n in ("sa_build_mask", "sa_radial_mask", "sa_pyramid_pool", "sa_sparse_attn_fwd",
               "sa_pyramid_attn_fwd", "sa_get_device_status", "sa_build_mask_workspace",
-              "sa_sparse_attn_bwd", "sa_sparse_attn_bwd_workspace", "sa_token_permute"):
+              "sa_sparse_attn_bwd", "sa_sparse_attn_bwd_workspace", "sa_token_permute",
+              "sa_sparse_attn_fwd_host", "sa_sparse_attn_fwd_host_workspace"):
         assert n in names
 
 
@@ -159,3 +160,19 @@ def test_permute_argument_validation(lib):
     assert call(d=96) == ops.SA_ERR_UNSUPPORTED
     assert call(t=same) == ops.SA_ERR_INVALID_ARG               # dst == src
 
+
+
+def test_host_entry_workspace_and_validation(lib):
+    assert ops.sa_sparse_attn_fwd_host_workspace(1000, 128, 4) == 2 * 4 * 4 * 1000 * 128 * 2
+    assert ops.sa_sparse_attn_fwd_host_workspace(1000, 128, 0) == 0
+
+    def call(q=16, o=16, B=1, H=2, N=256, d=128, block=128, ws=16, ws_bytes=1 << 30, hc=1):
+        return lib.sa_sparse_attn_fwd_host(q, 16, 16, B, H, N, d, block, None, 0, 0, 0, None, None, math.inf, 0.0,
+                                           0, 0, o, None, ws, ws_bytes, hc, None)
+    assert call(B=0) == ops.SA_OK
+    assert call(hc=0) == ops.SA_ERR_INVALID_ARG
+    assert call(q=None) == ops.SA_ERR_INVALID_ARG
+    assert call(o=None) == ops.SA_ERR_INVALID_ARG
+    assert call(d=96) == ops.SA_ERR_UNSUPPORTED
+    assert call(ws_bytes=100) == ops.SA_ERR_INVALID_ARG
+    assert call(ws=24) == ops.SA_ERR_INVALID_ARG

@@ -260,3 +260,32 @@ def test_causal_skip_step_and_radial(block):
         iu = np.triu_indices(nb, 1)
         assert not S.numpy()[0, :, iu[0], iu[1]].any()        # future blocks never marked
         assert Sr.sum() > 0
+
+
+# ------------------------------------------------------ host-buffer entry ---
+
+@pytest.mark.parametrize("hc", [1, 2, 5])
+def test_host_buffers_equal_device_path(hc):
+    """Q, K, V, O in pinned host memory, streamed in chunks of hc heads (B = 2,
+    H = 5, chunks that do not divide H): O, LSE and skip_out are identical to
+    one device-path call, with a mask, a skip chain and the radial order."""
+    B, H, N, d, block = 2, 5, 128 * 4 + 40, 128, 64
+    q, k, v = inputs.normal_qkv(B, H, N, d, seed=95)
+    nb = -(-N // block)
+    mask = inputs.bernoulli_block_mask(B, H, nb, nb, 0.7, seed=96).cuda()
+    skip_in = inputs.bernoulli_block_mask(B, H, nb, nb, 0.2, seed=97, force_diagonal=False).cuda()
+    lse_d = torch.empty(B, H, N, device="cuda")
+    so_d = torch.zeros(B, H, nb, nb, dtype=torch.uint8, device="cuda")
+    o_d = ops.sa_sparse_attn_fwd(q.cuda(), k.cuda(), v.cuda(), block, mask=mask, skip_in=skip_in, skip_out=so_d,
+                                 eps=1.0, lse=lse_d, order="radial")
+    hq, hk, hv = (t.pin_memory() for t in (q, k, v))
+    ho = torch.empty_like(hq).pin_memory()
+    lse_h = torch.empty(B, H, N, device="cuda")
+    so_h = torch.zeros(B, H, nb, nb, dtype=torch.uint8, device="cuda")
+    ops.sa_sparse_attn_fwd_host(hq, hk, hv, block, out=ho, mask=mask, skip_in=skip_in, skip_out=so_h, eps=1.0,
+                                lse=lse_h, heads_per_chunk=hc, order="radial")
+    torch.cuda.synchronize()
+    ops.sa_get_device_status()
+    assert torch.equal(ho, o_d.cpu())
+    assert torch.equal(lse_h, lse_d)
+    assert torch.equal(so_h, so_d)
