@@ -353,7 +353,7 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
         // the segment that holds the end of the sequence: short last group
         // (fewer than 2^lv tokens) and rows past the level's end
         const int rows_l = (p.N + (1 << lv) - 1) >> lv;
-#pragma unroll
+#pragma unroll 1
         for (int i = 0; i < 4; ++i) {
           float braw = kMaskedBias;
           const int gr = gr0 + i;
