@@ -75,7 +75,7 @@ struct AttnParams {
   float scale_log2; // scale * log2(e)
   float eps_raw;    // eps / scale: the skip threshold in raw q.k units
   int radial;       // visit kv tiles in radial-centric order (else ascending)
-  int causal;       // key c visible to row r only if c <= r (blocks j > i dropped)
+  int causal;       // key c visible to row r only if c <= r (blocks j > i dropped); selects the kernel
   __nv_bfloat16* o;
   float* lse;
 };
@@ -155,7 +155,9 @@ __device__ __forceinline__ float exp_pack_64(const float* s, float sl2, float ne
   return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
 }
 
-template <int D, int BLK>
+// CAUSAL is a template parameter: the causal mask adds code to the softmax
+// loop, and measured at block 64 even its never-taken form cost 7 % there.
+template <int D, int BLK, bool CAUSAL>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
@@ -217,7 +219,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               const uint8_t keep = p.mask ? p.mask[b * p.msb + h * p.msh + qb * p.msi + kb] : uint8_t(1);
               const size_t sidx = (static_cast<size_t>(bh) * p.nb + qb) * p.nb + kb;
               const uint8_t sk = p.skip_in ? p.skip_in[sidx] : uint8_t(0);
-              if (keep && !sk && (!p.causal || kb <= qb)) {
+              if (keep && !sk && (!CAUSAL || kb <= qb)) {
                 bits |= (BLK == 128 ? 0xFu : (1u << (qh * 2 + kh))) << (16 + 4 * t);
               } else if (p.carry_skip) {
                 p.skip_out[sidx] = sk;
@@ -469,16 +471,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         named_bar_sync(kBarSFree + t, kHandoff);
 
         const int valid_cols = min(kTileN, p.N - jt * kTileN);
-        // causal: in the diagonal tile (kv tile = q-tile) key c needs c <= r
-        const int cmax = (p.causal && jt == qtile0 + t) ? r : kTileN - 1;
-        if (valid_cols < kTileN || (BLK == 64 && bits != 0xFu) || cmax < kTileN - 1) {
+        if (valid_cols < kTileN || (BLK == 64 && bits != 0xFu)) {
           const bool k0 = BLK == 128 ? true : ((bits >> (qh * 2 + 0)) & 1u);
           const bool k1 = BLK == 128 ? true : ((bits >> (qh * 2 + 1)) & 1u);
 #pragma unroll
           for (int c = 0; c < kTileN; ++c) {
-            const bool keep = (c < valid_cols) && (c < 64 ? k0 : k1) && c <= cmax;
+            const bool keep = (c < valid_cols) && (c < 64 ? k0 : k1);
             s[c] = keep ? s[c] : NEG_INF;
           }
+        }
+        // causal: in the diagonal tile (kv tile = q-tile) key c needs c <= r
+        // (a separate loop, so that the common path is unchanged)
+        if (CAUSAL && jt == qtile0 + t) {
+#pragma unroll
+          for (int c = 0; c < kTileN; ++c) s[c] = c <= r ? s[c] : NEG_INF;
         }
         // row maxima of the two 64-column halves: four independent chains each
         float mxh[2];

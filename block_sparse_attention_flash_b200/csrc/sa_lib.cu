@@ -79,10 +79,14 @@ cudaError_t init_device_kernels() {
     auto set = [&r](const void* fn, int bytes) {
       if (r == cudaSuccess) r = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     };
-    set(reinterpret_cast<const void*>(&sa::attn_fwd_kernel<128, 128>), sa::AttnSmem<128>::kAlloc);
-    set(reinterpret_cast<const void*>(&sa::attn_fwd_kernel<128, 64>), sa::AttnSmem<128>::kAlloc);
-    set(reinterpret_cast<const void*>(&sa::attn_fwd_kernel<64, 128>), sa::AttnSmem<64>::kAlloc);
-    set(reinterpret_cast<const void*>(&sa::attn_fwd_kernel<64, 64>), sa::AttnSmem<64>::kAlloc);
+    set(reinterpret_cast<const void*>(&sa::attn_fwd_kernel<128, 128, false>), sa::AttnSmem<128>::kAlloc);
+    set(reinterpret_cast<const void*>(&sa::attn_fwd_kernel<128, 64, false>), sa::AttnSmem<128>::kAlloc);
+    set(reinterpret_cast<const void*>(&sa::attn_fwd_kernel<64, 128, false>), sa::AttnSmem<64>::kAlloc);
+    set(reinterpret_cast<const void*>(&sa::attn_fwd_kernel<64, 64, false>), sa::AttnSmem<64>::kAlloc);
+    set(reinterpret_cast<const void*>(&sa::attn_fwd_kernel<128, 128, true>), sa::AttnSmem<128>::kAlloc);
+    set(reinterpret_cast<const void*>(&sa::attn_fwd_kernel<128, 64, true>), sa::AttnSmem<128>::kAlloc);
+    set(reinterpret_cast<const void*>(&sa::attn_fwd_kernel<64, 128, true>), sa::AttnSmem<64>::kAlloc);
+    set(reinterpret_cast<const void*>(&sa::attn_fwd_kernel<64, 64, true>), sa::AttnSmem<64>::kAlloc);
     set(reinterpret_cast<const void*>(&sa::pyr_fwd_kernel<128, 128>), sa::PyrSmem<128>::kAlloc);
     set(reinterpret_cast<const void*>(&sa::pyr_fwd_kernel<128, 64>), sa::PyrSmem<128>::kAlloc);
     set(reinterpret_cast<const void*>(&sa::pyr_fwd_kernel<64, 128>), sa::PyrSmem<64>::kAlloc);
@@ -336,14 +340,17 @@ sa_status sa_sparse_attn_fwd(const void* q, const void* k, const void* v, int B,
   const int n_pairs = ceil_div(ceil_div(N, sa::kTileM), 2);
   dim3 grid(n_pairs, BH);
   cudaStream_t s = as_stream(stream);
+#define SA_ATTN_LAUNCH(DD, BB, CC) \
+  sa::attn_fwd_kernel<DD, BB, CC><<<grid, sa::kAttnThreads, sa::AttnSmem<DD>::kAlloc, s>>>(tq, tk, tv, p)
   if (d == 128 && block == 128)
-    sa::attn_fwd_kernel<128, 128><<<grid, sa::kAttnThreads, sa::AttnSmem<128>::kAlloc, s>>>(tq, tk, tv, p);
+    causal ? SA_ATTN_LAUNCH(128, 128, true) : SA_ATTN_LAUNCH(128, 128, false);
   else if (d == 128 && block == 64)
-    sa::attn_fwd_kernel<128, 64><<<grid, sa::kAttnThreads, sa::AttnSmem<128>::kAlloc, s>>>(tq, tk, tv, p);
+    causal ? SA_ATTN_LAUNCH(128, 64, true) : SA_ATTN_LAUNCH(128, 64, false);
   else if (d == 64 && block == 128)
-    sa::attn_fwd_kernel<64, 128><<<grid, sa::kAttnThreads, sa::AttnSmem<64>::kAlloc, s>>>(tq, tk, tv, p);
+    causal ? SA_ATTN_LAUNCH(64, 128, true) : SA_ATTN_LAUNCH(64, 128, false);
   else
-    sa::attn_fwd_kernel<64, 64><<<grid, sa::kAttnThreads, sa::AttnSmem<64>::kAlloc, s>>>(tq, tk, tv, p);
+    causal ? SA_ATTN_LAUNCH(64, 64, true) : SA_ATTN_LAUNCH(64, 64, false);
+#undef SA_ATTN_LAUNCH
   return cuda_status(cudaGetLastError());
 }
 
