@@ -155,8 +155,8 @@ __device__ __forceinline__ float exp_pack_64(const float* s, float sl2, float ne
   return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
 }
 
-// CAUSAL is a template parameter: the causal mask adds code to the softmax
-// loop, and measured at block 64 even its never-taken form cost 7 % there.
+// CAUSAL is a template parameter, so that the non-causal instantiation
+// carries no causal code in its softmax loop.
 template <int D, int BLK, bool CAUSAL>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
