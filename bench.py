@@ -134,6 +134,13 @@ def whole_job_tflops(work_all, ms_max):
     return work_all / (ms_max * 1e-3) / 1e12
 
 
+def workload_config(wl, world):
+    """The `config` object of both arms' JSON lines."""
+    return {"workload": wl.name, "B": wl.B, "H": wl.H, "N": wl.N, "grid": [wl.T, wl.Hh, wl.Ww], "d": wl.d,
+            "block": wl.block, "eps": wl.eps, "mask": "all kept + LiteAttention skip chain",
+            "l2": "inputs larger than L2 (3 x 774 MB per step)", "parallelism": f"replicas x{world}"}
+
+
 def executed_flops(skip_in, N, block, d, mask=None):
     """4 * d * sum over visited (i, j) of valid rows_i * valid cols_j."""
     nb = -(-N // block)
@@ -237,9 +244,7 @@ def run_ours(args, rank, world, local):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded random-Fourier-feature locality generator + denoising drift, drawn on device)",
-        "config": {"workload": wl.name, "B": B, "H": H, "N": N, "grid": [wl.T, wl.Hh, wl.Ww], "d": d,
-                   "block": block, "eps": eps, "mask": "all kept + LiteAttention skip chain",
-                   "l2": "inputs larger than L2 (3 x 774 MB per step)", "parallelism": f"replicas x{world}"},
+        "config": workload_config(wl, world),
         "ms_per_call": round(statistics.median(kern_ms), 3),
         "density": round(1.0 - skip_rate, 6),
         "executed_tflops": round(achieved, 2),
@@ -477,8 +482,7 @@ def run_reference(args, rank, world):
             "warmup": args.warmup, "ms_per_step": round(dt * 1e3 / max(1, args.steps), 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded random-Fourier-feature locality generator)", "impl": "reference",
-            "config": {"workload": wl.name, "B": wl.B, "H": wl.H, "N": wl.N, "d": wl.d, "block": wl.block,
-                       "eps": wl.eps},
+            "config": workload_config(wl, world),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": last["cores"], "kind": "oracle",
                              "sample": last["sample"]},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
