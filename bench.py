@@ -262,7 +262,7 @@ def run_ours(args, rank, world, local):
     return line
 
 
-E2E_HEADS_PER_CHUNK = 4
+E2E_HEADS_PER_CHUNK = 2   # measured: 2 heads 98.2 ms per step, 4 heads 100.5, 8 heads 105
 
 
 def run_e2e(ops, qkv0, block, eps, nb, dev, stream, steps, world):
