@@ -17,11 +17,12 @@
 //   bwd_dq_kernel      one CTA per 128-row q-tile: walks its kept kv tiles,
 //                      S = Q K^T and dP = dO V^T, dS packed in place, then
 //                      dQ += dS K with the A operand in TMEM.
-// Every MMA is one of the two forms of the forward kernel: both operands
-// K-major in shared memory (S, dP), or A from TMEM and B MN-major in shared
+// The MMAs take one of three forms: both operands K-major in shared memory
+// (S^T, dP^T in dK/dV), A from TMEM and B K-major in shared memory (S, dP in
+// dQ, with Q and dO copied into TMEM), or A from TMEM and B MN-major in shared
 // memory (dV, dK, dQ).  The same 128 x D tile, as TMA writes it, serves as a
 // K-major B operand (Q in S^T, K in S) and as an MN-major B operand (Q in dK,
-// dO in dV, K in dQ).
+// dO in dV, K in dQ).  Each S is computed in two 64-column halves.
 //
 // Roles (320 threads = 10 warps, one CTA per SM for the TMEM it holds):
 //   warps 0-3   one thread per row of the CTA's tile (key row in dK/dV, query
@@ -32,9 +33,9 @@
 //               (2-stage ring) and stages the per-query LSE / D vectors;
 //   warp 9      allocates TMEM and issues every MMA (warp-wide, one elected lane).
 // Hand-offs: tcgen05.commit to mbarriers from the MMA warp; one named barrier
-// per half (its warpgroup + warp 9) when that half's P / dS are in TMEM.  Every party runs the full,
-// list-determined sequence of syncs, also after an error (skipping only its
-// loads and MMAs), and every mbarrier wait is bounded.
+// per half (its warpgroup + warp 9) when that half's P / dS are in TMEM.
+// Every party runs the full, list-determined sequence of syncs, also after an
+// error (skipping only its loads and MMAs), and every mbarrier wait is bounded.
 #pragma once
 
 #include "sa_attn_fwd.cuh"
