@@ -289,3 +289,21 @@ def test_host_buffers_equal_device_path(hc):
     assert torch.equal(ho, o_d.cpu())
     assert torch.equal(lse_h, lse_d)
     assert torch.equal(so_h, so_d)
+
+
+def test_maximum_sequence_sampled_qblocks():
+    """The longest supported sequence (4096 kv tiles: N = 524,288 - 40 tokens,
+    d = 64, block 128) with a 5 % Bernoulli mask: sampled q-blocks (first,
+    middle, last, ragged) against the oracle."""
+    B, H, d, block = 1, 1, 64, 128
+    N = 128 * 4096 - 40
+    q, k, v = inputs.normal_qkv(B, H, N, d, seed=4097)
+    nb = -(-N // block)
+    mask = inputs.bernoulli_block_mask(B, H, nb, nb, 0.05, seed=4098)
+    O, L = run_attn(q, k, v, block, mask)
+    picks = [(0, 0, 0), (0, 0, 1), (0, 0, 2047), (0, 0, nb - 1)]
+    ref = masked_attention(q, k, v, block, mask, qblocks=picks)
+    for (b, h, i), (Or, Lr) in ref.items():
+        r0, r1 = i * block, min(N, (i + 1) * block)
+        check_o(O[b, h, r0:r1], Or, f"max N q-block {i}")
+        check_lse(L[b, h, r0:r1], Lr, f"max N q-block {i}")

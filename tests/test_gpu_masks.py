@@ -139,3 +139,23 @@ def test_global_mask_480p_grid():
     mr, flags, _ = global_mask(q, k, wl.block, wl.tau, return_info=True)
     nflag = check_bits(m.cpu(), mr, flags, "global 480p")
     assert nflag <= 0.001 * mr.size
+
+
+@pytest.mark.parametrize("mode", ["tau", "global"])
+def test_maximum_rows_4096_blocks(mode):
+    """The largest supported row (Nb = 4096 blocks of 64 tokens, N = 262,144 -
+    17): the shared-memory select path (tau) and the many-CTA global search."""
+    from oracle import global_mask
+    block, d, nb = 64, 64, 4096
+    N = block * nb - 17
+    g = torch.Generator().manual_seed(4096)
+    q = (torch.randn(1, 1, N, d, generator=g) * 0.5).to(torch.bfloat16)
+    k = (torch.randn(1, 1, N, d, generator=g) * 0.5).to(torch.bfloat16)
+    m = ops.sa_build_mask(q.cuda(), k.cuda(), block, mode, tau=0.6)
+    ops.sa_get_device_status()
+    if mode == "tau":
+        ref, flags, _ = tau_mask(q, k, block, 0.6, return_info=True)
+    else:
+        ref, flags, _ = global_mask(q, k, block, 0.6, return_info=True)
+    nflag = check_bits(m.cpu(), ref, flags, f"{mode} nb=4096")
+    assert nflag <= 0.001 * ref.size
