@@ -1,0 +1,56 @@
+"""Oracle pins from the hand-worked fixtures in tests/golden/ (CPU only).
+
+The pages print no numeric worked example, so each fixture is a small case
+worked out by hand from the rule a page states (the citation and the reading
+head each file).  No value in them comes from code.
+"""
+import math
+
+import numpy as np
+import pytest
+
+from oracle import lite_step, permutation, radial_mask
+from oracle.masks import global_head, tau_row
+
+from _golden import floats as _floats, ints as _ints, matrix, records as _records
+
+
+@pytest.mark.parametrize("rec", _records("axis_orders.txt"), ids=lambda r: f"{r['grid']}/{r['cells']}/{r['order']}")
+def test_axis_orders(rec):
+    T, Hh, Ww = _ints(rec["grid"])
+    perm = permutation(T, Hh, Ww, rec["order"], tuple(_ints(rec["cells"])))
+    assert perm.tolist() == rec["list"]
+
+
+@pytest.mark.parametrize("rec", _records("tau_rows.txt"), ids=lambda r: f"{r['p']}@{r['tau']}")
+def test_tau_rows(rec):
+    p = np.array(_floats(rec["p"]))
+    keep, _, _, _ = tau_row(np.log(p), float(rec["tau"]))
+    assert np.nonzero(keep)[0].tolist() == _ints(rec["keep"])
+
+
+@pytest.mark.parametrize("rec", _records("global_heads.txt"), ids=lambda r: f"{r['p']}@{r['tau']}")
+def test_global_heads(rec):
+    p = np.array(matrix(rec["p"]))
+    keep = global_head(np.log(p), float(rec["tau"]))[0]
+    expect = np.array(matrix(rec["keep"], _ints))
+    assert np.array_equal(np.asarray(keep, dtype=np.int64), expect)
+
+
+@pytest.mark.parametrize("rec", _records("radial_rows.txt"), ids=lambda r: f"{r['grid']}/{r['block']}/{r['row']}")
+def test_radial_rows(rec):
+    T, Hh, Ww = _ints(rec["grid"])
+    m = radial_mask(T, Hh, Ww, int(rec["block"]))
+    assert np.nonzero(m[int(rec["row"])])[0].tolist() == _ints(rec["keep"])
+
+
+@pytest.mark.parametrize("rec", _records("lite_skip.txt"), ids=lambda r: f"q{r['q']}/eps{r['eps']}")
+def test_lite_skip(rec):
+    q = np.array(_floats(rec["q"])).reshape(1, 1, 6, 1)
+    k = np.array(_floats(rec["k"])).reshape(1, 1, 6, 1)
+    v = np.arange(6, dtype=np.float64).reshape(1, 1, 6, 1)
+    _, _, skip, margin = lite_step(q, k, v, 2, eps=float(rec["eps"]), scale=1.0)
+    assert skip[0, 0, 0].tolist() == _ints(rec["bits"])
+    got = margin[0, 0, 0]
+    assert math.isnan(got[0])
+    assert np.allclose(got[1:], _floats(rec["margins"]), rtol=0, atol=1e-12)
