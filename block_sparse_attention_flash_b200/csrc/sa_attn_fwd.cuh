@@ -75,6 +75,8 @@ struct AttnParams {
   float eps_raw;    // eps / scale: the skip threshold in raw q.k units
   int radial;       // visit kv tiles in radial-centric order (else ascending)
   int causal;       // key c visible to row r only if c <= r (blocks j > i dropped); selects the kernel
+  int n_pairs;      // q-tile pairs per head
+  int n_full;       // CTAs [0, n_full) take a whole pair; each later pair runs as two CTAs, one per q-tile
   __nv_bfloat16* o;
   float* lse;
 };
@@ -188,7 +190,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   // misc[0] TMEM base, [1] list length, [2] / [3] kv tiles of q-tile 0 / 1, [4] abort flag
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int pair = blockIdx.x, bh = blockIdx.y;
+  // Work unit u = bh * n_pairs + pair, in launch order.  Units from n_full on
+  // (the last, partial wave of a launch) run as two CTAs each; a CTA then
+  // treats the pair's other q-tile as absent: no list bits, no writes.
+  int unit = blockIdx.x, skip_t = -1;
+  if (unit >= p.n_full) {
+    const int x = unit - p.n_full;
+    unit = p.n_full + (x >> 1);
+    skip_t = 1 - (x & 1);
+  }
+  const int bh = unit / p.n_pairs, pair = unit - bh * p.n_pairs;
   const int b = bh / p.H, h = bh - (bh / p.H) * p.H;
   const int qtile0 = 2 * pair;
 
@@ -213,7 +224,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
           for (int qh = 0; qh < QH; ++qh) {
             const int qb = (qtile0 + t) * QH + qh;
-            if (qb >= p.nb) continue;
+            if (qb >= p.nb || t == skip_t) continue;
 #pragma unroll
             for (int kh = 0; kh < KH; ++kh) {
               const int kb = jt * KH + kh;
@@ -437,7 +448,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int wq = warp & 3;
     const int r = wq * 32 + lane;
     const int row = (qtile0 + t) * kTileM + r;
-    const bool row_valid = row < p.N;
+    const bool row_valid = row < p.N && t != skip_t;
     const int qh = (BLK == 64) ? (r >> 6) : 0;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     const uint32_t s_addr = lane_base;

@@ -65,6 +65,7 @@ bool encode_rows_map(CUtensorMap* map, const void* base, int BH, int rows, int D
 struct DeviceInit {
   std::once_flag flag;
   cudaError_t err = cudaSuccess;
+  int n_sm = 1;
 };
 DeviceInit g_dev_init[kMaxDevices];
 
@@ -101,9 +102,33 @@ cudaError_t init_device_kernels() {
     set(reinterpret_cast<const void*>(&sa::bwd_dq_kernel<64, 64>), sa::BwdSmem<64>::kAlloc);
     set(reinterpret_cast<const void*>(&sa::block_select_kernel),
         static_cast<int>(sa::select_smem_bytes(sa::kMaxSelect)));
+    int dev = 0, n_sm = 0;
+    if (r == cudaSuccess) r = cudaGetDevice(&dev);
+    if (r == cudaSuccess) r = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+    if (r == cudaSuccess && n_sm > 0) di.n_sm = n_sm;
     di.err = r;
   });
   return di.err;
+}
+
+// SM count of the current device (valid after init_device_kernels succeeded).
+int device_sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 1;
+  return g_dev_init[dev].n_sm;
+}
+
+// Number of work units, out of `units` launched one CTA each, to run as two
+// CTAs each (one per q-tile of the pair).  The attention kernel allocates all
+// 512 TMEM columns, so one CTA per SM is active and a launch runs in waves of
+// n_sm CTAs.  When the last wave holds no more than half of the SMs, its units
+// are split: twice as many CTAs, each with half the rows, finish that wave
+// sooner (each still streams all of its K/V tiles, so a full wave is left
+// alone).
+long long tail_units_to_split(long long units, int n_sm) {
+  if (n_sm <= 0) return 0;
+  const long long tail = units % n_sm;
+  return (tail > 0 && 2 * tail <= n_sm) ? tail : 0;
 }
 
 bool valid_dim(int d) { return d == 64 || d == 128; }
@@ -338,7 +363,11 @@ sa_status sa_sparse_attn_fwd(const void* q, const void* k, const void* v, int B,
   p.lse = lse;
 
   const int n_pairs = ceil_div(ceil_div(N, sa::kTileM), 2);
-  dim3 grid(n_pairs, BH);
+  const long long units = static_cast<long long>(n_pairs) * BH;
+  const long long n_split = tail_units_to_split(units, device_sm_count());
+  p.n_pairs = n_pairs;
+  p.n_full = static_cast<int>(units - n_split);
+  dim3 grid(static_cast<unsigned>(units + n_split));
   cudaStream_t s = as_stream(stream);
 #define SA_ATTN_LAUNCH(DD, BB, CC) \
   sa::attn_fwd_kernel<DD, BB, CC><<<grid, sa::kAttnThreads, sa::AttnSmem<DD>::kAlloc, s>>>(tq, tk, tv, p)
@@ -402,7 +431,11 @@ sa_status sa_pyramid_attn_fwd(const void* q, const void* k, const void* v, int B
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   const int n_pairs = ceil_div(ceil_div(N, sa::kTileM), 2);
-  dim3 grid(n_pairs, BH);
+  const long long units = static_cast<long long>(n_pairs) * BH;
+  const long long n_split = tail_units_to_split(units, device_sm_count());
+  p.n_pairs = n_pairs;
+  p.n_full = static_cast<int>(units - n_split);
+  dim3 grid(static_cast<unsigned>(units + n_split));
   cudaStream_t s = as_stream(stream);
   if (d == 128 && block == 128)
     sa::pyr_fwd_kernel<128, 128><<<grid, sa::kPyrThreads, sa::PyrSmem<128>::kAlloc, s>>>(tq, maps, p);

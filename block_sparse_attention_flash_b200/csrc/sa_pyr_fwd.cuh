@@ -55,6 +55,8 @@ struct PyrParams {
   long long lsb, lsh, lsi;
   float scale_log2;
   int causal;             // k-blocks j > i dropped, the diagonal block at level 0 cut per row
+  int n_pairs;            // q-tile pairs per head
+  int n_full;             // CTAs [0, n_full) take a whole pair; each later pair runs as two CTAs, one per q-tile
   __nv_bfloat16* o;
   float* lse;
 };
@@ -125,7 +127,16 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
   // diagonal segment of q-block x of q-tile t (-1: none)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int pair = blockIdx.x, bh = blockIdx.y;
+  // Work unit u = bh * n_pairs + pair, in launch order.  Units from n_full on
+  // (the last, partial wave of a launch) run as two CTAs each; a CTA then
+  // treats the pair's other q-tile as absent: no segments, no writes.
+  int unit = blockIdx.x, skip_t = -1;
+  if (unit >= p.n_full) {
+    const int x = unit - p.n_full;
+    unit = p.n_full + (x >> 1);
+    skip_t = 1 - (x & 1);
+  }
+  const int bh = unit / p.n_pairs, pair = unit - bh * p.n_pairs;
   const int b = bh / p.H, h = bh - (bh / p.H) * p.H;
   const int qtile0 = 2 * pair;
 
@@ -136,7 +147,7 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
       int n = 0, cols = 0;
       const int qbA = (qtile0 + t) * QH;
       const int qbB = qbA + QH - 1;
-      const bool validA = qbA < p.nb, validB = qbB < p.nb;
+      const bool validA = qbA < p.nb && t != skip_t, validB = qbB < p.nb && t != skip_t;
       if (lane == 0) {
         misc[8 + 2 * t] = -1;
         misc[9 + 2 * t] = -1;
@@ -559,7 +570,7 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
     const int wq = warp & 3;
     const int r = wq * 32 + lane;
     const int row = (qtile0 + t) * kTileM + r;
-    const bool row_valid = row < p.N;
+    const bool row_valid = row < p.N && t != skip_t;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     const uint32_t s_addr = lane_base;
     const uint32_t p_addr = lane_base + 128 + 64 * t;

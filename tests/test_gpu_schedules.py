@@ -105,3 +105,52 @@ def test_pyramid_unbalanced_tiles(block):
     check_lse(lse.cpu(), Lr, f"pyramid unbalanced block={block}")
     rows3 = slice(3 * 128, 4 * 128)                        # q-tile 3 keeps nothing
     assert torch.all(out.cpu()[:, :, rows3] == 0) and torch.all(lse.cpu()[:, :, rows3] == -math.inf)
+
+
+@pytest.mark.parametrize("block", [64, 128])
+@pytest.mark.parametrize("kernel", ["attention", "pyramid"])
+def test_tail_wave_split_is_bit_identical(block, kernel):
+    """A launch whose last wave would hold at most half of the SMs runs the
+    pairs of that wave as two CTAs each, one per q-tile.  With 148 SMs: 20
+    heads of 9 q-tiles (5 pairs each, the last one ragged) make 100 pairs, a
+    last wave of more than half the SMs, so no pair is split; the first 3
+    heads alone (15 pairs) are all split.  The same heads must give
+    bit-identical O, LSE and skip bits both ways, and match the oracle."""
+    H, N, d = 20, 128 * 8 + 40, 128
+    q, k, v = inputs.normal_qkv(1, H, N, d, seed=block + 91)
+    nb = -(-N // block)
+    g = torch.Generator().manual_seed(block + 92)
+    if kernel == "attention":
+        mask = (torch.rand(1, H, nb, nb, generator=g) < 0.6).to(torch.uint8)
+        skip_in = (torch.rand(1, H, nb, nb, generator=g) < 0.1).to(torch.uint8)
+    else:
+        codes = torch.randint(0, 5, (1, H, nb, nb), generator=g, dtype=torch.uint8)
+
+    def run(h):
+        qd, kd, vd = q[:, :h].cuda(), k[:, :h].cuda(), v[:, :h].cuda()
+        out = torch.full_like(qd, float("nan"))
+        lse = torch.full((1, h, N), float("nan"), device="cuda")
+        if kernel == "attention":
+            so = torch.full((1, h, nb, nb), 7, dtype=torch.uint8, device="cuda")
+            ops.sa_sparse_attn_fwd(qd, kd, vd, block, mask=mask[:, :h].contiguous().cuda(),
+                                   skip_in=skip_in[:, :h].contiguous().cuda(), skip_out=so, eps=2.0,
+                                   out=out, lse=lse)
+        else:
+            kp, vp = ops.sa_pyramid_pool(kd, vd, block)
+            ops.sa_pyramid_attn_fwd(qd, kd, vd, block, codes[:, :h].contiguous().cuda(), kp, vp, out=out, lse=lse)
+            so = torch.zeros(1)
+        ops.sa_get_device_status()
+        return out.cpu(), lse.cpu(), so.cpu()
+
+    O20, L20, S20 = run(H)
+    O3, L3, S3 = run(3)
+    assert torch.equal(O20[:, :3].view(torch.int16), O3.view(torch.int16))
+    assert torch.equal(L20[:, :3], L3)
+    if kernel == "attention":
+        assert torch.equal(S20[:, :3], S3)
+        keep = mask & (1 - skip_in)
+        Or, Lr = masked_attention(q, k, v, block, keep)
+    else:
+        Or, Lr = pyramid_attention(q, k, v, block, codes.numpy())
+    check_o(O20, Or, f"{kernel} block={block}")
+    check_lse(L20, Lr, f"{kernel} block={block}")
