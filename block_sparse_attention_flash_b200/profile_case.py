@@ -1,6 +1,7 @@
 """Small, self-contained launches of each kernel, for profiler captures.
 
     python -m block_sparse_attention_flash_b200.profile_case attn   [--heads 4] [--reps 2]
+    python -m block_sparse_attention_flash_b200.profile_case tau    [--heads 12] [--reps 2]
     python -m block_sparse_attention_flash_b200.profile_case radial [--reps 2]
     python -m block_sparse_attention_flash_b200.profile_case mask   [--heads 12] [--reps 2]
     python -m block_sparse_attention_flash_b200.profile_case pool   [--heads 12] [--reps 2]
@@ -12,6 +13,7 @@ Each case uses a workload's real token grid with fewer heads, so one launch
 holds a few hundred MB (larger than L2) and a full profiler capture ends in
 seconds.  Inputs are drawn on the device from the seeded generator.
   attn    75,600-token LiteAttention grid (block 128, d 128), all kept, skip update on
+  tau     32,760-token 480p grid (block 64, d 128): the tau = 0.9 mask, then the attention
   radial  118,800-token HunyuanVideo-like grid, block 128
   mask    32,760-token 480p grid, block 64, tau = 0.9
   pool    32,760-token 480p grid, block 64
@@ -30,7 +32,7 @@ from . import build, inputs, ops
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["attn", "radial", "mask", "pool", "pyr", "bwd", "perm"])
+    ap.add_argument("case", choices=["attn", "tau", "radial", "mask", "pool", "pyr", "bwd", "perm"])
     ap.add_argument("--heads", type=int, default=0)
     ap.add_argument("--reps", type=int, default=2)
     args = ap.parse_args()
@@ -44,6 +46,13 @@ def main():
         skip = [torch.zeros(1, q.shape[1], nb, nb, dtype=torch.uint8, device=dev) for _ in range(args.reps + 1)]
         for r in range(args.reps):
             ops.sa_sparse_attn_fwd(q, k, v, wl.block, skip_in=skip[r], skip_out=skip[r + 1], eps=wl.eps)
+    elif args.case == "tau":
+        wl = inputs.WORKLOADS["wan13b_480p_tau"]
+        q, k, v = inputs.rff_qkv(wl, H=args.heads or wl.H, device=dev)
+        m = ops.sa_build_mask(q, k, wl.block, "tau", tau=wl.tau)
+        o = torch.empty_like(q)
+        for _ in range(args.reps):
+            ops.sa_sparse_attn_fwd(q, k, v, wl.block, mask=m, out=o)
     elif args.case == "radial":
         wl = inputs.WORKLOADS["hunyuan_720p_radial"]
         for _ in range(args.reps):
