@@ -44,6 +44,15 @@ def test_tau_uniform_scores_keep_first_ceil_tau_n():
     assert (m[..., :8] == 1).all() and (m[..., 8:] == 0).all()
 
 
+def test_tau_block_exactly_at_the_threshold_is_dropped():
+    """Keep a block iff the mass strictly before it is < tau, checked where the
+    mass before a block equals tau exactly: four equal blocks (p = 1/4, sums
+    exact in binary) and tau = 1/2 keep two blocks, not three."""
+    keep, _, p, mass_before = tau_row(np.zeros(4), 0.5)
+    assert p.tolist() == [0.25] * 4 and mass_before.tolist() == [0.0, 0.25, 0.5, 0.75]
+    assert keep.tolist() == [True, True, False, False]
+
+
 def test_tau_to_zero_keeps_only_argmax():
     g = np.random.default_rng(1)
     for _ in range(20):
@@ -188,6 +197,15 @@ def test_global_hand_built_peaked_and_uniform_rows():
     assert keep.astype(int).tolist() == [[1, 0, 0, 0], [1, 1, 0, 0]]
     keep, _ = global_head(s, 1.0)
     assert keep.all()
+
+
+def test_global_pair_exactly_at_the_threshold_is_dropped():
+    """Two uniform rows of two blocks (every P = 1/2 exactly) and tau = 1/2:
+    the head's target mass is 1, reached exactly before the third pair in
+    index order, so two pairs are kept."""
+    from oracle.masks import global_head
+    keep, _ = global_head(np.zeros((2, 2)), 0.5)
+    assert keep.astype(int).tolist() == [[1, 1], [0, 0]]
 
 
 def test_global_brute_force_shortest_prefix():

@@ -1,0 +1,186 @@
+"""Planted mistakes in the oracle must be caught by its pins (CPU only).
+
+Each case rewrites one line of one oracle function into a plausible
+mistake: a dropped term, a wrong sign, a non-strict comparison, a
+transposed operand, an off-by-one exponent, a reversed tie order.  Then it
+runs the pins that guard that function, and at least one of them must
+fail.  A case that every pin lets through would mark a gap in the pins.
+
+The rewrite works on the function's source text, so the mutant is the
+oracle's own code with the one change.  It replaces every reference to the
+original function in the oracle package and in the pin modules for the
+duration of the case.
+"""
+import inspect
+import sys
+import textwrap
+
+import pytest
+
+import oracle
+import oracle.attention
+import oracle.backward
+import oracle.lite
+import oracle.masks
+import oracle.permute
+import oracle.pyramid
+import test_golden as pins_golden
+import test_oracle_attention as pins_attn
+import test_oracle_backward as pins_bwd
+import test_oracle_masks as pins_masks
+import test_oracle_permute as pins_perm
+import test_oracle_pyramid_lite as pins_pl
+
+
+def _mutant(module, name, old, new):
+    fn = getattr(module, name)
+    src = textwrap.dedent(inspect.getsource(fn))
+    assert src.count(old) == 1, f"{name}: the text to mutate must occur exactly once: {old!r}"
+    ns = dict(module.__dict__)
+    exec(compile(src.replace(old, new), f"<mutant of {module.__name__}.{name}>", "exec"), ns)
+    return fn, ns[name]
+
+
+def _install(monkeypatch, original, mutant):
+    """Replace every module-level reference to `original` in the oracle and pin modules."""
+    mods = [m for k, m in list(sys.modules.items())
+            if m is not None and (k == "oracle" or k.startswith("oracle.") or k.startswith("test_"))]
+    for m in mods:
+        for attr, val in list(vars(m).items()):
+            if val is original:
+                monkeypatch.setattr(m, attr, mutant)
+
+
+def _golden(test, name):
+    """One parametrized golden pin over all records of its fixture."""
+    from _golden import records
+    fixture = {"test_axis_orders": "axis_orders.txt", "test_tau_rows": "tau_rows.txt",
+               "test_global_heads": "global_heads.txt", "test_radial_rows": "radial_rows.txt",
+               "test_lite_skip": "lite_skip.txt"}[name]
+
+    def run():
+        for rec in records(fixture):
+            test(rec)
+    return run
+
+
+PIN_SETS = {
+    "attention": [pins_attn.test_all_ones_mask_equals_dense_sdpa_tiny_config,
+                  lambda: pins_attn.test_brute_force_token_level_matches_block_path(21, 8),
+                  pins_attn.test_rows_sum_to_one_with_unit_values,
+                  pins_attn.test_single_kept_block_is_attention_over_that_block,
+                  pins_attn.test_lse_matches_scipy_logsumexp_on_kept_columns,
+                  pins_attn.test_causal_all_ones_equals_sdpa_is_causal,
+                  pins_attn.test_causal_block_mask_equals_token_level_brute_force],
+    "tau": [pins_masks.test_tau_uniform_scores_keep_first_ceil_tau_n,
+            pins_masks.test_tau_block_exactly_at_the_threshold_is_dropped,
+            pins_masks.test_tau_to_zero_keeps_only_argmax,
+            pins_masks.test_tau_brute_force_minimum_cardinality_prefix,
+            pins_masks.test_tau_monotone,
+            _golden(pins_golden.test_tau_rows, "test_tau_rows")],
+    "levels": [pins_masks.test_level_quotas_and_order, pins_masks.test_level_ties_break_by_index],
+    "scores": [pins_masks.test_block_means_closed_form_with_partial_tail, pins_masks.test_block_scores_closed_form],
+    "radial": [lambda: pins_masks.test_radial_matches_bruteforce(17, 4, 9, 8),
+               lambda: pins_masks.test_radial_matches_bruteforce(9, 8, 16, 16),
+               pins_masks.test_radial_structure,
+               _golden(pins_golden.test_radial_rows, "test_radial_rows")],
+    "global": [pins_masks.test_global_single_row_equals_tau_row,
+               pins_masks.test_global_hand_built_peaked_and_uniform_rows,
+               pins_masks.test_global_pair_exactly_at_the_threshold_is_dropped,
+               pins_masks.test_global_brute_force_shortest_prefix,
+               _golden(pins_golden.test_global_heads, "test_global_heads")],
+    "lite": [pins_pl.test_infinite_eps_never_skips_and_equals_block_attention,
+             pins_pl.test_hand_built_gap_of_twelve,
+             pins_pl.test_skipped_blocks_are_exponentially_suppressed,
+             pins_pl.test_first_visited_block_never_skipped_and_chain_monotone,
+             _golden(pins_golden.test_lite_skip, "test_lite_skip")],
+    "visit": [pins_pl.test_radial_visit_order_hand_listed],
+    "permute": [lambda: pins_perm.test_axis_orders_equal_grid_transposes("hwt"),
+                pins_perm.test_hand_listed_hwt,
+                pins_perm.test_cell_partitions_equal_blocked_transposes,
+                _golden(pins_golden.test_axis_orders, "test_axis_orders")],
+    "pyramid": [pins_pl.test_pool_partial_group_and_progressive_equals_direct,
+                pins_pl.test_all_level_zero_equals_block_attention,
+                pins_pl.test_constant_groups_make_any_level_mix_exact,
+                pins_pl.test_causal_constant_groups_equal_causal_attention],
+    "backward": [pins_bwd.test_empty_rows_and_columns_and_key_shift_invariance,
+                 pins_bwd.test_dense_case_equals_torch_autograd,
+                 pins_bwd.test_causal_finite_differences],
+}
+
+A, M, L, P, Y, W = (oracle.attention, oracle.masks, oracle.lite, oracle.permute, oracle.pyramid,
+                    oracle.backward)
+MUTATIONS = [
+    # (id, module, function, original text, mistaken text, pin set)
+    ("attn-no-scale", A, "attention_qblock", "s = (qh[r0:r1] @ kh[c].T) * scale", "s = (qh[r0:r1] @ kh[c].T)",
+     "attention"),
+    ("attn-lse-without-max", A, "attention_qblock", "lse = (m + np.log(z))", "lse = (np.log(z))", "attention"),
+    ("attn-mask-ignored", A, "attention_qblock", "for j in np.nonzero(keep_row)[0]]", "for j in range(len(keep_row))]",
+     "attention"),
+    ("attn-causal-drops-diagonal", A, "attention_qblock", "c[None, :] <= np.arange(r0, r1)[:, None]",
+     "c[None, :] < np.arange(r0, r1)[:, None]", "attention"),
+    ("tau-non-strict", M, "tau_row", "keep = mass_before < tau", "keep = mass_before <= tau", "tau"),
+    ("tau-mass-includes-self", M, "tau_row", "mass_before[j] = acc\n        acc += p[j]",
+     "acc += p[j]\n        mass_before[j] = acc", "tau"),
+    ("rank-ascending", M, "_order", "np.lexsort((np.arange(row.shape[0]), -row))",
+     "np.lexsort((np.arange(row.shape[0]), row))", "tau"),
+    ("rank-ties-reversed", M, "_order", "np.lexsort((np.arange(row.shape[0]), -row))",
+     "np.lexsort((-np.arange(row.shape[0]), -row))", "tau"),
+    ("level-quota-floor", M, "level_counts", "math.ceil(f * nkb - 1e-9)", "math.floor(f * nkb + 1e-9)", "levels"),
+    ("level-ties-reversed", M, "_order", "np.lexsort((np.arange(row.shape[0]), -row))",
+     "np.lexsort((-np.arange(row.shape[0]), -row))", "levels"),
+    ("means-divide-by-block", M, "block_means", "/ (r1 - r0)", "/ block", "scores"),
+    ("scores-no-scale", M, "block_scores", 'qm, km) * scale', 'qm, km)', "scores"),
+    # (Δt = 1 needs no band of its own: the window rule keeps every offset there.)
+    ("radial-band-too-wide", M, "radial_mask", "if t <= 1:", "if t <= 2:", "radial"),
+    ("radial-log2-off-by-one", M, "radial_mask", "kexp = t.bit_length() - 1", "kexp = t.bit_length()", "radial"),
+    ("radial-non-strict-window", M, "radial_mask", "(1 << kexp) < S", "(1 << kexp) <= S", "radial"),
+    ("radial-last-token-position", M, "radial_mask", "first = np.arange(nb, dtype=np.int64) * block",
+     "first = np.minimum(np.arange(nb, dtype=np.int64) * block + block - 1, N - 1)", "radial"),
+    ("global-non-strict", M, "global_head", "keep = mass_before < target", "keep = mass_before <= target", "global"),
+    ("global-target-per-row", M, "global_head", "target = tau * nqb", "target = tau", "global"),
+    ("global-ties-reversed", M, "global_head", "np.lexsort((np.arange(flat.size), -flat))",
+     "np.lexsort((-np.arange(flat.size), -flat))", "global"),
+    ("skip-any-row", L, "lite_qblock", "mg = np.max(local - running + eps)", "mg = np.min(local - running + eps)",
+     "lite"),
+    ("skip-eps-sign", L, "lite_qblock", "mg = np.max(local - running + eps)", "mg = np.max(local - running - eps)",
+     "lite"),
+    ("skip-last-block-max", L, "lite_qblock", "running = np.maximum(running, local)", "running = local", "lite"),
+    ("skip-first-block-tested", L, "lite_qblock", "if n_vis > 0:", "if n_vis >= 0:", "lite"),
+    ("skip-never-tested", L, "lite_qblock", "if n_vis > 0:", "if n_vis < 0:", "lite"),
+    ("radial-order-ties-descending", L, "visit_order", "key=lambda t: (dist(t), t)", "key=lambda t: (dist(t), -t)",
+     "visit"),
+    ("perm-slowest-axis-last", P, "permutation", "np.lexsort(keys[::-1])", "np.lexsort(keys)", "permute"),
+    ("perm-cell-and-inner-swapped", P, "permutation",
+     "keys = [coord[a] // cell[a] for a in order] + [coord[a] % cell[a] for a in order]",
+     "keys = [coord[a] % cell[a] for a in order] + [coord[a] // cell[a] for a in order]", "permute"),
+    ("pool-divide-by-c", Y, "pyramid_pool", "/ (r1 - r0)", "/ c", "pyramid"),
+    ("pyramid-bias-sign", Y, "_level_keys", "np.log(counts)", "-np.log(counts)", "pyramid"),
+    ("pyramid-bias-missing", Y, "_level_keys", "np.log(counts)", "0.0 * counts", "pyramid"),
+    ("pyramid-causal-diagonal-pooled", Y, "pyramid_attention", "if causal and j == i and code:\n                code = 1",
+     "if causal and j == i and code:\n                code = code", "pyramid"),
+    ("bwd-no-delta", W, "attention_bwd_head", "dr = np.sum(p * dp, axis=1, keepdims=True)", "dr = 0.0", "backward"),
+    ("bwd-dk-no-scale", W, "attention_bwd_head", "scale * (ds.T @ qh)", "(ds.T @ qh)", "backward"),
+    ("bwd-dv-transposed", W, "attention_bwd_head", "dv = p.T @ doh", "dv = p @ doh", "backward"),
+]
+
+
+@pytest.mark.parametrize("case", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_planted_mistake_is_caught(case, monkeypatch):
+    _, module, name, old, new, pin_set = case
+    original, mutant = _mutant(module, name, old, new)
+    _install(monkeypatch, original, mutant)
+    caught = []
+    for pin in PIN_SETS[pin_set]:
+        try:
+            pin()
+        except Exception as e:          # an AssertionError, or the mutant breaking a shape or index
+            caught.append(type(e).__name__)
+    assert caught, f"no pin of '{pin_set}' fails with the planted mistake {case[0]}"
+
+
+def test_unmutated_pins_pass():
+    """Control: every pin set passes on the oracle as it is."""
+    for pins in PIN_SETS.values():
+        for pin in pins:
+            pin()
