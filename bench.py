@@ -38,9 +38,10 @@ sys.path.insert(0, ROOT)
 METRIC = "sparse attn ms/call, executed TFLOP/s & % B200 BF16 tensor peak at 75.6K tok"
 # DRAM bytes (read + write) of one attention launch at 75,600 tokens x 40 heads,
 # from the ncu capture summarised in profiles/attn_fwd_wan14b_720p_lite.md
-# (4-head case, 300.8 MB, scaled by 40/4 heads).  Valid for the kernel version
-# that capture names; set to None whenever the kernel changes.
-ATTN_DRAM_BYTES_PER_LAUNCH = 3.0080e9
+# (4-head case, 239.5 MB read + 61.4 MB written, scaled by 40/4 heads).  Valid
+# for the kernel version that capture names; set to None whenever the kernel
+# changes.
+ATTN_DRAM_BYTES_PER_LAUNCH = 3.0087e9
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
