@@ -4,14 +4,19 @@
  *
  * The library computes non-causal softmax attention over the 3D
  * (frame x height x width) token grid of a video diffusion transformer, where
- * only selected (q-block, k-block) tiles are executed.  It has four parts:
- *   sa_build_mask      mean-pooled block scores -> tau-mass mask or PSA level map
- *   sa_radial_mask     static radial mask (window halves as frame distance doubles)
- *   sa_pyramid_pool    PSA pyramid: mean-pooled K/V at 2, 4 and 8 tokens per key
- *   sa_sparse_attn_fwd FlashAttention-style forward over kept tiles, with the
- *                      LiteAttention skip-mask update fused in
- *   sa_sparse_attn_bwd its gradients with respect to Q, K and V
- *   sa_token_permute   PARO axis orders / VMoBA cell partitions of the grid
+ * only selected (q-block, k-block) tiles are executed.  Entry points:
+ *   sa_build_mask           mean-pooled block scores -> tau-mass mask (per row
+ *                           or per head) or PSA level map
+ *   sa_build_mask_noalloc   the same without a caller workspace
+ *   sa_radial_mask          static radial mask (window halves as frame
+ *                           distance doubles)
+ *   sa_pyramid_pool         PSA pyramid: mean-pooled K/V at 2, 4 and 8 tokens
+ *   sa_sparse_attn_fwd      FlashAttention-style forward over kept tiles, with
+ *                           the LiteAttention skip-mask update fused in
+ *   sa_sparse_attn_fwd_host the same with Q/K/V/O in host memory, streamed
+ *   sa_pyramid_attn_fwd     PSA multi-level attention over a level map
+ *   sa_sparse_attn_bwd      gradients of sa_sparse_attn_fwd for Q, K and V
+ *   sa_token_permute        PARO axis orders / VMoBA cell partitions of the grid
  *
  * Conventions shared by every entry point
  *   - Tensors are caller-owned DEVICE memory.  Q, K, V and O are bf16,
@@ -28,8 +33,11 @@
  *   - Device-side waits are bounded.  A wait that runs out records
  *     SA_ERR_TIMEOUT in a per-device error word that sa_get_device_status
  *     reads; the kernel then returns without hanging the GPU.
- *   - The library allocates no device memory.  Scratch memory is passed in
- *     by the caller (sa_build_mask's workspace).
+ *   - The library allocates no device memory at run time.  Scratch memory
+ *     is passed in by the caller (the workspace arguments); the one
+ *     exception, sa_build_mask_noalloc, uses a static device array.
+ *     sa_sparse_attn_fwd_host creates and destroys its own copy streams and
+ *     events inside the call.
  *
  * Citations name the web page the operation comes from and its section.
  */
