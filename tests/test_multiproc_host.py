@@ -39,7 +39,7 @@ def _worker(rank, world, port, results):
 def test_two_gloo_ranks_max_time_sum_work():
     world = 2
     port = _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:   # no fork of a multi-threaded process
         results = m.dict()
         mp.spawn(_worker, args=(world, port, results), nprocs=world, join=True)
         res = dict(results)
