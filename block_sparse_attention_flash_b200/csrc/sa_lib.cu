@@ -134,6 +134,35 @@ long long tail_units_to_split(long long units, int n_sm) {
 bool valid_dim(int d) { return d == 64 || d == 128; }
 bool valid_block(int b) { return b == 64 || b == 128; }
 
+// Host-side checks shared by sa_build_mask and sa_build_mask_noalloc (all but
+// the workspace).  *empty is set for a call with no rows (nothing to launch).
+sa_status check_build_mask_args(const void* q, const void* k, int B, int H, int N, int d, int block, int mode,
+                                float tau, const float* level_frac, const uint8_t* mask_out, bool* empty) {
+  *empty = false;
+  if (B < 0 || H < 0 || N < 0) return SA_ERR_INVALID_ARG;
+  if (mode != SA_MASK_TAU && mode != SA_MASK_LEVELS && mode != SA_MASK_GLOBAL) return SA_ERR_INVALID_ARG;
+  if ((mode == SA_MASK_TAU || mode == SA_MASK_GLOBAL) && !(tau > 0.f && tau <= 1.f)) return SA_ERR_INVALID_ARG;
+  if (B == 0 || H == 0 || N == 0) {
+    *empty = true;
+    return SA_OK;
+  }
+  if (!valid_dim(d) || !valid_block(block)) return SA_ERR_UNSUPPORTED;
+  if (!q || !k || !mask_out) return SA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k)) return SA_ERR_INVALID_ARG;
+  if (ceil_div(N, block) > sa::kMaxSelect) return SA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * H > 65535) return SA_ERR_UNSUPPORTED;
+  if (mode == SA_MASK_LEVELS) {
+    if (!level_frac) return SA_ERR_INVALID_ARG;
+    float prev = 0.f;
+    for (int i = 0; i < 3; ++i) {
+      const float f = level_frac[i];
+      if (!(f >= prev && f <= 1.f)) return SA_ERR_INVALID_ARG;
+      prev = f;
+    }
+  }
+  return SA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -176,26 +205,14 @@ size_t sa_build_mask_workspace(int B, int H, int N, int d, int block) {
 sa_status sa_build_mask(const void* q, const void* k, int B, int H, int N, int d, int block, int mode, float tau,
                         const float* level_frac, uint8_t* mask_out, float* scores_out, void* workspace,
                         size_t workspace_bytes, void* stream) {
-  if (B < 0 || H < 0 || N < 0) return SA_ERR_INVALID_ARG;
-  if (mode != SA_MASK_TAU && mode != SA_MASK_LEVELS && mode != SA_MASK_GLOBAL) return SA_ERR_INVALID_ARG;
-  if ((mode == SA_MASK_TAU || mode == SA_MASK_GLOBAL) && !(tau > 0.f && tau <= 1.f)) return SA_ERR_INVALID_ARG;
-  int c0 = 0, c1 = 0, c2 = 0;
-  if (B == 0 || H == 0 || N == 0) return SA_OK;
-  if (!valid_dim(d) || !valid_block(block)) return SA_ERR_UNSUPPORTED;
-  if (!q || !k || !mask_out || !workspace) return SA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return SA_ERR_INVALID_ARG;
-  const int nb = ceil_div(N, block);
-  if (nb > sa::kMaxSelect) return SA_ERR_UNSUPPORTED;
-  if (static_cast<long long>(B) * H > 65535) return SA_ERR_UNSUPPORTED;
+  bool empty = false;
+  const sa_status st = check_build_mask_args(q, k, B, H, N, d, block, mode, tau, level_frac, mask_out, &empty);
+  if (st != SA_OK || empty) return st;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return SA_ERR_INVALID_ARG;
   if (workspace_bytes < sa_build_mask_workspace(B, H, N, d, block)) return SA_ERR_INVALID_ARG;
+  const int nb = ceil_div(N, block);
+  int c0 = 0, c1 = 0, c2 = 0;
   if (mode == SA_MASK_LEVELS) {
-    if (!level_frac) return SA_ERR_INVALID_ARG;
-    float prev = 0.f;
-    for (int i = 0; i < 3; ++i) {
-      const float f = level_frac[i];
-      if (!(f >= prev && f <= 1.f)) return SA_ERR_INVALID_ARG;
-      prev = f;
-    }
     c0 = static_cast<int>(std::ceil(static_cast<double>(level_frac[0]) * nb - 1e-9));
     c1 = static_cast<int>(std::ceil(static_cast<double>(level_frac[1]) * nb - 1e-9));
     c2 = static_cast<int>(std::ceil(static_cast<double>(level_frac[2]) * nb - 1e-9));
@@ -454,19 +471,20 @@ sa_status sa_pyramid_attn_fwd(const void* q, const void* k, const void* v, int B
 // sa_build_mask_noalloc: sa_build_mask for callers that must not allocate.
 //
 // Some callers cannot call cudaMalloc at the moment they need a mask:
-//   - code running inside CUDA stream capture, where an allocation would break
-//     the capture;
-//   - runtimes that own all device memory through their own pool and forbid
-//     libraries from allocating behind their back;
-//   - latency-critical loops that must never block on the allocator.
-// For them this variant takes its scratch (block means and block scores) from
+//   - serving runtimes that reserve all device memory up front in their own
+//     pool and do not let a library allocate behind their back (a cudaMalloc
+//     there fails, or takes memory the pool has promised elsewhere);
+//   - latency-critical denoising loops: cudaMalloc and cudaFree can
+//     synchronise the device, which stalls every stream of the process.
+// For them this variant takes its scratch (block means and block scores, or
+// the global selection's row statistics, histograms and search state) from
 // one file-scope device array instead of a caller-provided workspace.  The
-// array is created when the library's device code is loaded on a GPU and is
-// held on every such GPU until the process exits.
+// array exists on every GPU that loads the library's device code and stays
+// allocated there until the process exits.
 //
 // Everything that runs on the GPU is the same as in sa_build_mask: this entry
-// point looks up the array's device address and then calls sa_build_mask with
-// it as the workspace.
+// point checks the arguments, looks up the array's device address and then
+// calls sa_build_mask with it as the workspace.
 // ===========================================================================
 namespace {
 
@@ -480,29 +498,32 @@ static __device__ __align__(256) unsigned char g_build_mask_scratch[kNoAllocScra
 
 namespace {
 
-struct ScratchAddress {
-  std::once_flag flag;
-  void* ptr = nullptr;
-  cudaError_t err = cudaSuccess;
-};
-ScratchAddress g_scratch_address[kMaxDevices];
+std::mutex g_scratch_mutex;
+void* g_scratch_address[kMaxDevices] = {};
 
 // Device address of g_build_mask_scratch on the current device.  In host code
 // the array's name is only a host-side stand-in, so the address has to be
-// asked from the runtime: once per device, with that device current.
+// asked from the runtime, with the device current.  Only a successful lookup
+// is kept: a lookup that failed (no context yet, a capture in progress) is
+// tried again on the next call.
 cudaError_t build_mask_scratch(void** out) {
+  *out = nullptr;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  ScratchAddress& s = g_scratch_address[dev];
-  std::call_once(s.flag, [&s] {
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (g_scratch_address[dev] == nullptr) {
     void* p = nullptr;
-    s.err = cudaGetSymbolAddress(&p, g_build_mask_scratch);
-    s.ptr = (s.err == cudaSuccess) ? p : nullptr;
-  });
-  *out = s.ptr;
-  return s.err;
+    e = cudaGetSymbolAddress(&p, g_build_mask_scratch);
+    if (e != cudaSuccess) {
+      cudaGetLastError();  // reset the last-error state: a later launch check must not see this failure
+      return e;
+    }
+    g_scratch_address[dev] = p;
+  }
+  *out = g_scratch_address[dev];
+  return cudaSuccess;
 }
 
 }  // namespace
@@ -510,8 +531,9 @@ cudaError_t build_mask_scratch(void** out) {
 extern "C" sa_status sa_build_mask_noalloc(const void* q, const void* k, int B, int H, int N, int d, int block,
                                            int mode, float tau, const float* level_frac, uint8_t* mask_out,
                                            float* scores_out, void* stream) {
-  if (B < 0 || H < 0 || N < 0) return SA_ERR_INVALID_ARG;
-  if (B == 0 || H == 0 || N == 0) return SA_OK;
+  bool empty = false;
+  const sa_status st = check_build_mask_args(q, k, B, H, N, d, block, mode, tau, level_frac, mask_out, &empty);
+  if (st != SA_OK || empty) return st;
   if (sa_build_mask_workspace(B, H, N, d, block) > kNoAllocScratchBytes) return SA_ERR_UNSUPPORTED;
   void* scratch = nullptr;
   if (build_mask_scratch(&scratch) != cudaSuccess || scratch == nullptr) return SA_ERR_CUDA;

@@ -135,25 +135,29 @@ SA_API sa_status sa_build_mask(const void* q, const void* k, int B, int H, int N
 
 /*
  * sa_build_mask_noalloc — sa_build_mask without a caller-provided workspace.
- *   The pages have no counterpart to this entry point: it exists for callers
- *   that cannot allocate device memory when they need a mask (code inside
- *   CUDA stream capture, runtimes that forbid libraries from allocating, or
- *   loops that must not wait on an allocator).
+ *   The pages have no counterpart to this entry point.  It serves callers
+ *   that cannot allocate device memory when they need a mask: serving
+ *   runtimes that reserve all device memory up front in their own pool and
+ *   do not let a library allocate beside it, and latency-critical loops that
+ *   cannot afford cudaMalloc / cudaFree (they can synchronise the device).
  *
  * Same arguments, computation and results as sa_build_mask, minus the
  * workspace.  The scratch comes from one static device array of 32 MiB
  * (33,554,432 bytes) that every GPU loading this library holds until the
  * process exits.  Rules:
  *   - Size limit: sizes whose sa_build_mask_workspace(B, H, N, d, block)
- *     exceeds 32 MiB are rejected with SA_ERR_UNSUPPORTED before any launch.
+ *     exceeds 32 MiB are rejected with SA_ERR_UNSUPPORTED before any launch
+ *     (the other arguments are checked first, with sa_build_mask's codes).
  *   - Set-up: the first call on a device, with that device current, looks up
- *     the array's device address (cudaGetSymbolAddress) and keeps it.  Make
- *     that first call before any stream capture.
+ *     the array's device address (cudaGetSymbolAddress) and keeps it; a
+ *     lookup that fails returns SA_ERR_CUDA and is tried again on the next
+ *     call.  Make that first call before any stream capture.
  *   - Sharing: all calls on a device share the one array, and it keeps the
- *     previous call's contents.  Nothing in it needs to start at zero (every
- *     byte read is first written by the same call).  Calls whose kernels
- *     overlap on the GPU (different streams, no ordering between them) race
- *     on the array and give wrong masks: serialise them.
+ *     previous call's contents.  What has to start at zero (the histograms
+ *     and search state of SA_MASK_GLOBAL) is cleared by each call itself;
+ *     every other byte it reads was written earlier in the same call.  Calls
+ *     whose kernels overlap on the GPU (different streams, no ordering
+ *     between them) race on the array and give wrong masks: serialise them.
  *   - No memory is allocated or freed by this call.
  */
 SA_API sa_status sa_build_mask_noalloc(const void* q, const void* k, int B, int H, int N, int d, int block,

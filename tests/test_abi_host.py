@@ -96,6 +96,30 @@ def test_mask_builder_argument_validation(lib):
     assert f(16, 16, 1, 1, 0, 64, 64, 0, 0.9, None, 16, None, 256, 0, None) == ops.SA_OK
 
 
+
+def test_noalloc_mask_builder_checks_arguments_before_its_scratch_lookup(lib):
+    """Argument errors of sa_build_mask_noalloc keep sa_build_mask's codes.
+
+    The checks run on the host before the entry point asks the runtime for
+    its scratch array's address, so they come back the same with no GPU
+    present (where that lookup would fail with SA_ERR_CUDA)."""
+    fr = (ctypes.c_float * 3)(0.1, 0.3, 0.6)
+    bad = (ctypes.c_float * 3)(0.5, 0.3, 0.6)
+    f = lib.sa_build_mask_noalloc
+    frp, badp = ctypes.cast(fr, ctypes.c_void_p), ctypes.cast(bad, ctypes.c_void_p)
+    assert f(16, 16, 1, 1, 512, 64, 64, 0, 1.5, None, 16, None, None) == ops.SA_ERR_INVALID_ARG   # tau
+    assert f(16, 16, 1, 1, 512, 64, 64, 7, 0.9, None, 16, None, None) == ops.SA_ERR_INVALID_ARG   # mode
+    assert f(16, 16, 1, 1, 512, 64, 64, 1, 0.9, badp, 16, None, None) == ops.SA_ERR_INVALID_ARG   # fractions
+    assert f(16, 16, 1, 1, 512, 64, 64, 1, 0.9, None, 16, None, None) == ops.SA_ERR_INVALID_ARG   # no fractions
+    assert f(16, 16, 1, 1, 512, 80, 64, 0, 0.9, None, 16, None, None) == ops.SA_ERR_UNSUPPORTED   # d
+    assert f(16, 16, 1, 1, 512, 64, 32, 0, 0.9, None, 16, None, None) == ops.SA_ERR_UNSUPPORTED   # block
+    assert f(24, 16, 1, 1, 512, 64, 64, 0, 0.9, None, 16, None, None) == ops.SA_ERR_INVALID_ARG   # alignment
+    assert f(16, 16, 1, 1, 512, 64, 64, 0, 0.9, None, None, None, None) == ops.SA_ERR_INVALID_ARG  # no mask
+    assert f(16, 16, -1, 1, 512, 64, 64, 0, 0.9, None, 16, None, None) == ops.SA_ERR_INVALID_ARG
+    assert f(16, 16, 1, 1, 0, 64, 64, 0, 0.9, frp, 16, None, None) == ops.SA_OK                   # empty
+    # beyond the 32 MiB scratch: 12 heads, 118,800 tokens, block 64
+    assert f(16, 16, 1, 12, 118800, 128, 64, 0, 0.9, None, 16, None, None) == ops.SA_ERR_UNSUPPORTED
+
 def test_pool_and_radial_argument_validation(lib):
     three = (ctypes.c_void_p * 3)(16, 32, 48)
     holes = (ctypes.c_void_p * 3)(16, None, 48)
