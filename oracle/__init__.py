@@ -30,13 +30,13 @@ no code with the CUDA library and never imports it.
 from .attention import masked_attention, dense_attention, block_mask_to_token_mask
 from .masks import block_means, block_scores, tau_mask, level_map, radial_mask, global_mask
 from .pyramid import pyramid_pool, pyramid_attention
-from .lite import lite_step, lite_chain, visit_order
+from .lite import lite_step, lite_chain, visit_order, skip_flags
 from .backward import masked_attention_bwd, masked_attention_bwd_rows
 from .permute import permutation, permute_tokens
 
 __all__ = [
     "masked_attention", "dense_attention", "block_mask_to_token_mask",
     "block_means", "block_scores", "tau_mask", "level_map", "radial_mask", "global_mask",
-    "pyramid_pool", "pyramid_attention", "lite_step", "lite_chain", "visit_order",
+    "pyramid_pool", "pyramid_attention", "lite_step", "lite_chain", "visit_order", "skip_flags",
     "masked_attention_bwd", "masked_attention_bwd_rows", "permutation", "permute_tokens",
 ]

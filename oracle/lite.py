@@ -35,6 +35,7 @@ import math
 import numpy as np
 
 from .attention import _f64, _nblocks, _mask4
+from .masks import MARGIN
 
 
 RADIAL_TILE = 128     # keys per tile of the radial-centric order
@@ -96,6 +97,18 @@ def lite_qblock(qh, kh, vh, block, keep_row, i, eps, scale, order="ascending", c
     e = np.exp(s - m)
     z = e.sum(axis=1, keepdims=True)
     return (e / z) @ vh[c], (m + np.log(z))[:, 0], new, margin
+
+
+def skip_flags(margin):
+    """Skip decisions within MARGIN of the cut, from lite_step's margin rows.
+
+    The comparison rule for skip bits is bit-exact except where the decision
+    margin max_r (l_r(j) - m_r + eps) lies within 1e-3 of 0 (absolute, in
+    natural-log logit units): there fp32 and fp64 may decide differently.
+    Untested blocks (NaN margin) are never flagged.
+    """
+    m = np.asarray(margin, dtype=np.float64)
+    return np.isfinite(m) & (np.abs(m) < MARGIN)
 
 
 def lite_step(q, k, v, block, mask=None, skip_in=None, eps=10.0, scale=None, qblocks=None,

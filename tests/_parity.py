@@ -4,12 +4,14 @@ Tolerances (bf16 inputs and output, unit-variance data):
   O    max-abs <= 2e-2 and mean-abs <= 2e-3 against the fp64 oracle;
   LSE  abs <= 1e-3 (finite rows), identical -inf on rows with no visited block;
   masks / skip bits: bit-exact except bits whose decision margin lies within
-  1e-3 of the cut (flagged by the oracle); flagged mismatches are counted and
-  returned, not failed;
+  1e-3 of the cut (flagged by the oracle); flagged mismatches are counted,
+  printed and bounded (at most 0.1 % of the compared bits), not failed;
   gradients: relative to the reference's size (check_grad below).
 """
 import numpy as np
 import torch
+
+from oracle.lite import skip_flags  # noqa: F401  (the skip bits' margin rule, for the parity tests)
 
 O_MAX_ABS = 2e-2
 O_MEAN_ABS = 2e-3
@@ -44,25 +46,32 @@ def check_lse(l_gpu, l_ref, what=""):
         assert err <= LSE_ABS, f"{what}: LSE abs {err:.3e}"
 
 
-def check_bits(b_gpu, b_ref, flags=None, what=""):
-    """Bit-exact compare; mismatches on flagged positions are tolerated and counted."""
+# Flagged mismatches allowed per comparison: a decision only flips between
+# fp32 and fp64 when its margin is within rounding of the cut, so flagged
+# bits that do differ must stay rare.  Bound: 0.1 % of the compared bits, and
+# at least 2 (small masks with one near-tie).
+FLAG_MAX_FRAC = 1e-3
+FLAG_MIN_ALLOWED = 2
+
+
+def check_bits(b_gpu, b_ref, flags=None, what="", max_frac=FLAG_MAX_FRAC):
+    """Bit-exact compare; mismatches on flagged positions are counted, bounded
+    and reported (printed), any other mismatch fails.  Returns the count."""
     g = as_np(b_gpu).astype(np.int64)
     r = np.asarray(b_ref).astype(np.int64)
     assert g.shape == r.shape, (g.shape, r.shape)
     bad = g != r
-    if flags is not None:
-        f = np.asarray(flags, dtype=bool)
-        unflagged = bad & ~f
-        assert not unflagged.any(), f"{what}: {int(unflagged.sum())} unflagged mismatches"
-        return int((bad & f).sum())
-    assert not bad.any(), f"{what}: {int(bad.sum())} mismatches"
-    return 0
-
-
-def skip_flags(margin, eps_margin=1e-3):
-    """Flag skip decisions whose margin max_r(l_r - m_r + eps) is within 1e-3 of 0."""
-    m = np.asarray(margin)
-    return np.isfinite(m) & (np.abs(m) < eps_margin)
+    if flags is None:
+        assert not bad.any(), f"{what}: {int(bad.sum())} mismatches"
+        return 0
+    f = np.asarray(flags, dtype=bool)
+    unflagged = bad & ~f
+    assert not unflagged.any(), f"{what}: {int(unflagged.sum())} unflagged mismatches"
+    n = int((bad & f).sum())
+    allowed = max(FLAG_MIN_ALLOWED, int(max_frac * g.size))
+    print(f"[flagged] {what}: {n} flagged mismatches of {g.size} bits ({int(f.sum())} flagged)")
+    assert n <= allowed, f"{what}: {n} flagged mismatches, more than the {allowed} allowed"
+    return n
 
 
 # Gradients (attention backward): their scale shrinks like 1/sqrt(kept keys),

@@ -10,7 +10,8 @@ import numpy as np
 import pytest
 
 from oracle import lite_step, permutation, radial_mask
-from oracle.masks import global_head, tau_row
+from oracle.lite import skip_flags
+from oracle.masks import global_head, level_row, tau_row
 
 from _golden import floats as _floats, ints as _ints, matrix, records as _records
 
@@ -54,3 +55,30 @@ def test_lite_skip(rec):
     got = margin[0, 0, 0]
     assert math.isnan(got[0])
     assert np.allclose(got[1:], _floats(rec["margins"]), rtol=0, atol=1e-12)
+
+
+def check_margin_flags(rec):
+    """One record of margin_flags.txt: decisions and their margin flags."""
+    kind = rec["kind"]
+    if kind == "tau":
+        keep, flag, _, _ = tau_row(np.log(np.array(_floats(rec["p"]))), float(rec["tau"]))
+        assert np.nonzero(keep)[0].tolist() == _ints(rec["keep"])
+        assert np.nonzero(flag)[0].tolist() == _ints(rec["flag"])
+    elif kind == "level":
+        code, flag = level_row(np.array(_floats(rec["s"])), _ints(rec["counts"]))
+        assert code.tolist() == _ints(rec["code"])
+        assert np.nonzero(flag)[0].tolist() == _ints(rec["flag"])
+    elif kind == "global":
+        keep, flag = global_head(np.log(np.array(matrix(rec["p"]))), float(rec["tau"]))
+        assert np.array_equal(np.asarray(keep, dtype=np.int64), np.array(matrix(rec["keep"], _ints)))
+        assert np.array_equal(np.asarray(flag, dtype=np.int64), np.array(matrix(rec["flag"], _ints)))
+    else:
+        assert kind == "skip"
+        flag = skip_flags(np.array(_floats(rec["margin"])))
+        assert np.nonzero(flag)[0].tolist() == _ints(rec["flag"])
+
+
+@pytest.mark.parametrize("rec", _records("margin_flags.txt"),
+                         ids=lambda r: "-".join(f"{k}{v}" for k, v in r.items() if k in ("kind", "p", "s", "tau")))
+def test_margin_flags(rec):
+    check_margin_flags(rec)

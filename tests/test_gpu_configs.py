@@ -105,8 +105,10 @@ def test_wan14b_720p_lite_step_full(eps):
     _compare_rows(O[:, heads].cpu(), lse[:, heads].cpu(), {key: val[:2] for key, val in ref.items()}, wl.block,
                   wl.N, f"lite 720p eps={eps}")
     S = skip_out[:, heads].cpu().numpy()
-    nflag_total = 0
-    for (b, hh, i), (_, _, srow, mrow) in ref.items():
-        nflag_total += check_bits(S[b, hh, i], srow, skip_flags(mrow), f"skip row {hh},{i}")
+    keys = list(ref)
+    got = np.stack([S[b, hh, i] for (b, hh, i) in keys])
+    want = np.stack([ref[key][2] for key in keys])
+    flags = np.stack([skip_flags(ref[key][3]) for key in keys])
+    check_bits(got, want, flags, f"skip rows 720p eps={eps}")
     if eps == 2.0:
         assert S.sum() > 0

@@ -64,6 +64,17 @@ def _golden(test, name):
     return run
 
 
+def _margin(kind):
+    """The margin-flag pins of one decision kind (tests/golden/margin_flags.txt)."""
+    from _golden import records
+
+    def run():
+        for rec in records("margin_flags.txt"):
+            if rec["kind"] == kind:
+                pins_golden.check_margin_flags(rec)
+    return run
+
+
 PIN_SETS = {
     "attention": [pins_attn.test_all_ones_mask_equals_dense_sdpa_tiny_config,
                   lambda: pins_attn.test_brute_force_token_level_matches_block_path(21, 8),
@@ -77,8 +88,9 @@ PIN_SETS = {
             pins_masks.test_tau_to_zero_keeps_only_argmax,
             pins_masks.test_tau_brute_force_minimum_cardinality_prefix,
             pins_masks.test_tau_monotone,
-            _golden(pins_golden.test_tau_rows, "test_tau_rows")],
-    "levels": [pins_masks.test_level_quotas_and_order, pins_masks.test_level_ties_break_by_index],
+            _golden(pins_golden.test_tau_rows, "test_tau_rows"),
+            _margin("tau")],
+    "levels": [pins_masks.test_level_quotas_and_order, pins_masks.test_level_ties_break_by_index, _margin("level")],
     "scores": [pins_masks.test_block_means_closed_form_with_partial_tail, pins_masks.test_block_scores_closed_form],
     "radial": [lambda: pins_masks.test_radial_matches_bruteforce(17, 4, 9, 8),
                lambda: pins_masks.test_radial_matches_bruteforce(9, 8, 16, 16),
@@ -88,7 +100,9 @@ PIN_SETS = {
                pins_masks.test_global_hand_built_peaked_and_uniform_rows,
                pins_masks.test_global_pair_exactly_at_the_threshold_is_dropped,
                pins_masks.test_global_brute_force_shortest_prefix,
-               _golden(pins_golden.test_global_heads, "test_global_heads")],
+               _golden(pins_golden.test_global_heads, "test_global_heads"),
+               _margin("global")],
+    "skipflags": [_margin("skip")],
     "lite": [pins_pl.test_infinite_eps_never_skips_and_equals_block_attention,
              pins_pl.test_hand_built_gap_of_twelve,
              pins_pl.test_skipped_blocks_are_exponentially_suppressed,
@@ -141,6 +155,27 @@ MUTATIONS = [
     ("global-target-per-row", M, "global_head", "target = tau * nqb", "target = tau", "global"),
     ("global-ties-reversed", M, "global_head", "np.lexsort((np.arange(flat.size), -flat))",
      "np.lexsort((-np.arange(flat.size), -flat))", "global"),
+    # margin flags: each decision's "within 1e-3 of the cut" rule
+    ("tau-flag-margin-wide", M, "tau_row", "flag = np.abs(mass_before - tau) < MARGIN",
+     "flag = np.abs(mass_before - tau) < 10 * MARGIN", "tau"),
+    ("tau-flag-margin-narrow", M, "tau_row", "flag = np.abs(mass_before - tau) < MARGIN",
+     "flag = np.abs(mass_before - tau) < 0.1 * MARGIN", "tau"),
+    ("tau-flag-mass-after", M, "tau_row", "np.abs(mass_before - tau)", "np.abs(mass_before + p - tau)", "tau"),
+    ("tau-flag-no-swap-kept", M, "tau_row", "flag |= keep & (np.abs(p - p_out) <= MARGIN * p_out)", "pass", "tau"),
+    ("tau-flag-no-swap-dropped", M, "tau_row", "flag |= (~keep) & (np.abs(p - p_in) <= MARGIN * p_in)", "pass",
+     "tau"),
+    ("tau-flag-swap-absolute", M, "tau_row", "<= MARGIN * p_out", "<= MARGIN", "tau"),
+    ("level-flag-margin-wide", M, "level_row", "(s - s_out < MARGIN)", "(s - s_out < 10 * MARGIN)", "levels"),
+    ("level-flag-sign", M, "level_row", "(s - s_out < MARGIN)", "(s_out - s < MARGIN)", "levels"),
+    ("level-flag-no-lower-side", M, "level_row", "flag |= (rank >= c) & (s_in - s < MARGIN)", "pass", "levels"),
+    ("level-flag-relative", M, "level_row", "(s_in - s < MARGIN)", "(s_in - s < MARGIN * abs(s_in))", "levels"),
+    ("global-flag-margin-absolute", M, "global_head", "< MARGIN * nqb", "< MARGIN", "global"),
+    ("global-flag-margin-wide", M, "global_head", "< MARGIN * nqb", "< 10 * MARGIN * nqb", "global"),
+    ("global-flag-no-swap-kept", M, "global_head", "flag |= keep & (np.abs(flat - p_out) <= MARGIN * p_out)",
+     "pass", "global"),
+    ("global-flag-swap-absolute", M, "global_head", "<= MARGIN * p_in)", "<= MARGIN)", "global"),
+    ("skip-flag-wide", L, "skip_flags", "np.abs(m) < MARGIN", "np.abs(m) < 10 * MARGIN", "skipflags"),
+    ("skip-flag-signed", L, "skip_flags", "np.abs(m) < MARGIN", "m < MARGIN", "skipflags"),
     ("skip-any-row", L, "lite_qblock", "mg = np.max(local - running + eps)", "mg = np.min(local - running + eps)",
      "lite"),
     ("skip-eps-sign", L, "lite_qblock", "mg = np.max(local - running + eps)", "mg = np.max(local - running - eps)",
