@@ -55,11 +55,6 @@ constexpr int kMaxKvTiles = 4096;
 constexpr int kAttnWarps = 12;
 constexpr int kAttnThreads = kAttnWarps * 32;
 constexpr int kSoftmaxWarp0 = 4;
-// Within each 16-pair chunk of a row, pairs [kPolyPairFrom, 16) take 2^x from
-// the FMA-pipe polynomial instead of the MUFU unit.  Measured on B200,
-// offloading any share of the pairs was slower than none (the polynomial's
-// issue cost exceeds the MUFU time it frees), so the offload is off.
-constexpr int kPolyPairFrom = 16;
 
 struct AttnParams {
   int B, H, N;
@@ -134,9 +129,9 @@ __device__ __forceinline__ bool named_bar_and(int id, int nthreads, bool v) {
 // returns the fp32 sum.  The scale-and-shift and the sums run on packed
 // f32x2 FMA / ADD (two lanes per instruction): the softmax loop is partly
 // bound by instruction issue, and halving these instructions measured 4.8 %
-// faster end to end at 75.6K tokens.  2^x itself comes from the MUFU ex2;
-// moving a share of it to the FMA-pipe polynomial (kPolyPairFrom < 16) was
-// slower (12.5 % of the pairs: -2.4 %; 25 %: -5.5 %).
+// faster end to end at 75.6K tokens.  2^x itself comes from the MUFU ex2
+// (moving a share of it to an FMA-pipe polynomial measured slower: 12.5 % of
+// the pairs -2.4 %, 25 % -5.5 %).
 __device__ __forceinline__ float exp_pack_64(const float* s, float sl2, float neg_m, uint32_t* pk) {
   float2 acc[4];
 #pragma unroll
@@ -145,15 +140,7 @@ __device__ __forceinline__ float exp_pack_64(const float* s, float sl2, float ne
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
     const float2 x = fma2(make_float2(s[2 * i], s[2 * i + 1]), sl2v, nmv);
-    float p0, p1;
-    if ((i & 15) >= kPolyPairFrom) {
-      const float2 pp = exp2_poly2(x);
-      p0 = pp.x;
-      p1 = pp.y;
-    } else {
-      p0 = fast_exp2(x.x);
-      p1 = fast_exp2(x.y);
-    }
+    const float p0 = fast_exp2(x.x), p1 = fast_exp2(x.y);
     acc[i & 3] = add2(acc[i & 3], make_float2(p0, p1));
     pk[i] = pack_bf16x2(p0, p1);
   }
@@ -603,7 +590,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       tc_fence_after();
     }
     // A row that never saw a valid column keeps m_used = -inf: it is empty
-    // (O = 0, LSE = -inf) whatever the polynomial left in l_sum.
+    // (O = 0, LSE = -inf) whatever its exponentials left in l_sum.
     if (m_used == NEG_INF) l_sum = 0.f;
     const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
     __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * p.N + (row_valid ? row : 0)) * D;

@@ -84,17 +84,37 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete.  Returns false (and
-// records SA_ERR_TIMEOUT) if it has not completed within kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// records SA_ERR_TIMEOUT) if it has not completed within limit_ns of the
+// global timer; each try_wait suspends for at most kSuspendHintNs, so the
+// wait ends within about limit_ns + kSuspendHintNs.
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, unsigned long long limit_ns) {
   // a phase that has already completed is seen without the suspend machinery
   if (mbar_test(bar, parity) || mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_timer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
+    if (global_timer_ns() - t0 > limit_ns) {
       record_error(SA_ERR_TIMEOUT);
       return false;
     }
+  }
+}
+
+// The kernels' wait: mbar_wait_for with the library's limit (kWaitLimitNs).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  return mbar_wait_for(bar, parity, kWaitLimitNs);
+}
+
+// Self-test of the failure path: one thread waits, through mbar_wait_for, on
+// an mbarrier that nothing arrives on, so the wait runs out after limit_ns,
+// records SA_ERR_TIMEOUT and the kernel returns.  No other thread, copy or
+// MMA is involved, so nothing is left in flight.
+__global__ void __launch_bounds__(32) self_test_timeout_kernel(unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    mbar_wait_for(&bar, 0, limit_ns);
   }
 }
 
@@ -367,47 +387,6 @@ __device__ __forceinline__ float2 add2(float2 a, float2 b) {
       : "=l"(*reinterpret_cast<unsigned long long*>(&d))
       : "l"(*reinterpret_cast<unsigned long long*>(&a)), "l"(*reinterpret_cast<unsigned long long*>(&b)));
   return d;
-}
-
-// 2^x for a pair on the FMA pipe: Cody-Waite split x = n + f (n = round(x),
-// |f| <= 1/2), 2^f by the degree-3 minimax polynomial fitted in
-// exp2_poly_fit.py (max relative error 7.5e-5), 2^n added to the exponent
-// field.  Inputs at or below -125 (masked logits are -inf) return exactly 0;
-// such terms are below 2^-124 and cannot register in a bf16 probability or
-// an fp32 row sum anyway.
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: x + kRound rounds x to an integer
-  constexpr float kC0 = 0.99992806f, kC1 = 0.69326097f, kC2 = 0.24261113f, kC3 = 0.05517167f;
-  x.x = fmaxf(x.x, -125.f);
-  x.y = fmaxf(x.y, -125.f);
-  const float2 j = add2(x, make_float2(kRound, kRound));
-  const float2 n = add2(j, make_float2(-kRound, -kRound));
-  const float2 f = fma2(n, make_float2(-1.f, -1.f), x);
-  float2 p = fma2(make_float2(kC3, kC3), f, make_float2(kC2, kC2));
-  p = fma2(p, f, make_float2(kC1, kC1));
-  p = fma2(p, f, make_float2(kC0, kC0));
-  float2 r = make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(j.x) << 23)),
-                         __int_as_float(__float_as_int(p.y) + (__float_as_int(j.y) << 23)));
-  // masked logits arrive as -inf and must give exactly 0
-  r.x = x.x <= -125.f ? 0.f : r.x;
-  r.y = x.y <= -125.f ? 0.f : r.y;
-  return r;
-}
-
-// Scalar 2^x on the FMA pipe, same split and polynomial as exp2_poly2 but
-// without the exact-zero guard: inputs at or below -125 (masked logits) give
-// a value below 2^-124 instead of 0.  Callers that can see a row made only of
-// masked logits must treat that row as empty themselves.
-__device__ __forceinline__ float exp2_poly(float x) {
-  constexpr float kRound = 12582912.0f;
-  x = fmaxf(x, -125.f);
-  const float j = x + kRound;
-  const float n = j - kRound;
-  const float f = x - n;
-  float q = fmaf(0.05517167f, f, 0.24261113f);
-  q = fmaf(q, f, 0.69326097f);
-  q = fmaf(q, f, 0.99992806f);
-  return __int_as_float(__float_as_int(q) + (__float_as_int(j) << 23));
 }
 
 // Per-warpgroup register budget changes (all four warps of a warpgroup

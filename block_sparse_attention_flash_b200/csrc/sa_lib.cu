@@ -195,6 +195,12 @@ sa_status sa_get_device_status(void* stream) {
   return word ? SA_ERR_CUDA : SA_OK;
 }
 
+sa_status sa_self_test_timeout(uint64_t wait_ns, void* stream) {
+  if (wait_ns == 0 || wait_ns > 1000000000ull) return SA_ERR_INVALID_ARG;
+  sa::self_test_timeout_kernel<<<1, 32, 0, as_stream(stream)>>>(static_cast<unsigned long long>(wait_ns));
+  return cuda_status(cudaGetLastError());
+}
+
 size_t sa_build_mask_workspace(int B, int H, int N, int d, int block) {
   if (B <= 0 || H <= 0 || N <= 0 || d <= 0 || block <= 0) return 0;
   const size_t nb = static_cast<size_t>(ceil_div(N, block));

@@ -28,6 +28,7 @@ _SIGNATURES = {
     "sa_status_string": (ctypes.c_char_p, [_i32]),
     "sa_version": (_i32, []),
     "sa_get_device_status": (_i32, [_vp]),
+    "sa_self_test_timeout": (_i32, [ctypes.c_uint64, _vp]),
     "sa_build_mask_workspace": (_sz, [_i32, _i32, _i32, _i32, _i32]),
     "sa_build_mask": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _vp, _vp, _vp, _sz, _vp]),
     "sa_build_mask_noalloc": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _vp, _vp, _vp]),
@@ -123,6 +124,12 @@ def nblocks(N: int, block: int) -> int:
 def sa_get_device_status(stream=None) -> None:
     """Synchronise the stream and raise if a kernel recorded a device-side error."""
     _check(lib().sa_get_device_status(_stream(stream)), "sa_get_device_status")
+
+
+def sa_self_test_timeout(wait_ns: int, stream=None) -> None:
+    """Queue the failure-path self-test: one bounded device wait that runs out
+    after wait_ns; the next sa_get_device_status reports SA_ERR_TIMEOUT."""
+    _check(lib().sa_self_test_timeout(int(wait_ns), _stream(stream)), "sa_self_test_timeout")
 
 
 def sa_radial_mask(T: int, Hh: int, Ww: int, block: int, out: Optional[torch.Tensor] = None,

@@ -17,6 +17,8 @@
  *   sa_pyramid_attn_fwd     PSA multi-level attention over a level map
  *   sa_sparse_attn_bwd      gradients of sa_sparse_attn_fwd for Q, K and V
  *   sa_token_permute        PARO axis orders / VMoBA cell partitions of the grid
+ *   sa_get_device_status    read and clear the device error word
+ *   sa_self_test_timeout    make one bounded wait run out on purpose
  *
  * Conventions shared by every entry point
  *   - Tensors are caller-owned DEVICE memory.  Q, K, V and O are bf16,
@@ -87,6 +89,24 @@ SA_API int sa_version(void);
  * synchronisation itself failed).
  */
 SA_API sa_status sa_get_device_status(void* stream);
+
+/*
+ * sa_self_test_timeout — exercise the failure-detection path on purpose.
+ *   No page counterpart: the pages describe no error handling.  This entry
+ *   point lets a caller (or a test) check, without faulting or hanging the
+ *   GPU, that a device-side wait which runs out is reported.
+ *
+ * Launches one CTA on `stream` whose single thread waits, through the same
+ * bounded mbarrier wait the kernels use, on an mbarrier that nothing arrives
+ * on.  The wait gives up after wait_ns nanoseconds of the global timer (plus
+ * at most 0.1 ms), records SA_ERR_TIMEOUT in the device error word and the
+ * kernel returns; no copy or MMA is left in flight.  The next
+ * sa_get_device_status on the device returns SA_ERR_TIMEOUT and clears the
+ * word, after which the library works as before.
+ *   wait_ns   1 .. 1,000,000,000 (1 s); anything else is SA_ERR_INVALID_ARG.
+ * Returns SA_OK once the kernel is queued.
+ */
+SA_API sa_status sa_self_test_timeout(uint64_t wait_ns, void* stream);
 
 /*
  * sa_build_mask_workspace — bytes of device scratch sa_build_mask needs:

@@ -31,7 +31,8 @@ def test_header_declares_the_entry_points():
     for n in ("sa_build_mask", "sa_radial_mask", "sa_pyramid_pool", "sa_sparse_attn_fwd",
               "sa_pyramid_attn_fwd", "sa_get_device_status", "sa_build_mask_workspace",
               "sa_sparse_attn_bwd", "sa_sparse_attn_bwd_workspace", "sa_token_permute",
-              "sa_sparse_attn_fwd_host", "sa_sparse_attn_fwd_host_workspace"):
+              "sa_sparse_attn_fwd_host", "sa_sparse_attn_fwd_host_workspace", "sa_self_test_timeout",
+              "sa_build_mask_noalloc"):
         assert n in names
 
 
@@ -45,6 +46,12 @@ def test_status_strings_and_version(lib):
     assert ops.status_string(0) == "SA_OK"
     assert ops.status_string(4) == "SA_ERR_TIMEOUT"
     assert lib.sa_version() >= 100
+
+
+def test_self_test_timeout_argument_validation(lib):
+    assert lib.sa_self_test_timeout(0, None) == ops.SA_ERR_INVALID_ARG
+    assert lib.sa_self_test_timeout(1_000_000_001, None) == ops.SA_ERR_INVALID_ARG
+    assert lib.sa_self_test_timeout(2**64 - 1, None) == ops.SA_ERR_INVALID_ARG
 
 
 def test_workspace_size(lib):

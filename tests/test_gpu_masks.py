@@ -51,6 +51,20 @@ def test_level_map_small(block):
     check_bits(m.cpu(), lr, flags, f"levels block={block}")
 
 
+@pytest.mark.parametrize("grid,block,width", [((4, 16, 20), 64, 1), ((8, 40, 40), 64, 8), ((21, 30, 52), 64, 16)])
+def test_level_map_each_select_width(grid, block, width):
+    """LEVELS rows through the warp selection kernel at E = 1, 8 and 16 keys
+    per lane (20, 200 and 512 blocks per row; the last is the PSA 480p grid)."""
+    T, Hh, Ww = grid
+    wl = inputs.Workload("w", 1, 2, 128, T, Hh, Ww, block, "pyramid", seed=70 + width)
+    assert 32 * width // 2 < wl.nblocks <= 32 * width
+    q, k, _ = inputs.rff_qkv(wl)
+    m = ops.sa_build_mask(q.cuda(), k.cuda(), block, "levels", level_frac=wl.level_frac)
+    ops.sa_get_device_status()
+    lr, flags, _ = level_map(q, k, block, wl.level_frac, return_info=True)
+    check_bits(m.cpu(), lr, flags, f"levels nb={wl.nblocks} E={width}")
+
+
 def test_scores_out_matches_oracle_scores():
     q, k, _ = _small_rff(64)
     nb = -(-q.shape[2] // 64)

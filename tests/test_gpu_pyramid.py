@@ -1,8 +1,10 @@
 """GPU parity: PSA pyramid attention (sa_pyramid_pool + sa_pyramid_attn_fwd) vs the oracle.
 
 The oracle pools K/V in fp64 and the GPU pools in fp32 and stores bf16; the
-difference is absorbed by the O tolerance.  Level maps handed to the GPU come
-from the oracle or from seeded draws, never from the GPU mask builder.
+difference is absorbed by the O tolerance.  Level maps handed to the oracle
+come from the oracle itself or from seeded draws, never from the GPU mask
+builder; the end-to-end case runs the GPU attention on the GPU-built map and
+compares only q-blocks whose GPU row equals the oracle's row.
 """
 import numpy as np
 import pytest
@@ -10,7 +12,7 @@ import torch
 
 from block_sparse_attention_flash_b200 import build, inputs, ops
 from oracle import pyramid_attention, masked_attention, dense_attention, level_map
-from _parity import check_o, check_lse
+from _parity import check_o, check_lse, check_bits
 
 pytestmark = pytest.mark.gpu
 
@@ -116,6 +118,46 @@ def test_psa_480p_full_sampled():
         want_o.append(o), want_l.append(l)
     check_o(torch.cat(got_o), np.concatenate(want_o), "psa 480p")
     check_lse(torch.cat(got_l), np.concatenate(want_l), "psa 480p")
+
+
+def test_psa_480p_gpu_pipeline():
+    """The PSA workload as the bench runs it, all on the GPU: level map from
+    sa_build_mask (12 heads x 512 x 512, the E = 16 warp selection), pooling,
+    then pyramid attention on that map.  The map is checked against the
+    oracle's for every head (flag-aware); the attention on sampled q-blocks of
+    three heads whose GPU level row is identical to the oracle's row, against
+    the oracle's attention on its own map."""
+    wl = inputs.WORKLOADS["psa_480p_pyramid"]
+    q, k, v = inputs.rff_qkv(wl, device="cuda")
+    nb = wl.nblocks
+    lv = ops.sa_build_mask(q, k, wl.block, "levels", level_frac=wl.level_frac)
+    kp, vp = ops.sa_pyramid_pool(k, v, wl.block)
+    lse = torch.empty(1, wl.H, wl.N, device="cuda")
+    O = ops.sa_pyramid_attn_fwd(q, k, v, wl.block, lv, kp, vp, lse=lse)
+    ops.sa_get_device_status()
+    qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
+    lv_ref, flags, _ = level_map(qc, kc, wl.block, wl.level_frac, return_info=True)
+    lv_gpu = lv.cpu().numpy()
+    check_bits(lv_gpu, lv_ref, flags, "levels 480p, 12 heads")
+    heads = [0, 6, 11]
+    same = (lv_gpu == lv_ref).all(axis=-1)[0]              # [H, nb]: rows the two maps agree on
+    g = np.random.default_rng(17)
+    samples = []
+    for hh, h in enumerate(heads):
+        ok = np.nonzero(same[h])[0]
+        assert ok.size >= nb - 8, f"head {h}: {nb - ok.size} level rows differ"
+        pick = set(g.choice(ok, size=4, replace=False).tolist())
+        pick |= {i for i in (0, nb - 1) if same[h, i]}
+        samples += [(0, hh, int(i)) for i in sorted(pick)]
+    ref = pyramid_attention(qc[:, heads], kc[:, heads], vc[:, heads], wl.block, lv_ref[:, heads], qblocks=samples)
+    Oh, Lh = O[:, heads].cpu(), lse[:, heads].cpu()
+    got_o, got_l, want_o, want_l = [], [], [], []
+    for (b, hh, i), (o, l) in ref.items():
+        r0, r1 = i * wl.block, min(wl.N, (i + 1) * wl.block)
+        got_o.append(Oh[b, hh, r0:r1]), got_l.append(Lh[b, hh, r0:r1])
+        want_o.append(o), want_l.append(l)
+    check_o(torch.cat(got_o), np.concatenate(want_o), "psa 480p GPU pipeline")
+    check_lse(torch.cat(got_l), np.concatenate(want_l), "psa 480p GPU pipeline")
 
 
 @pytest.mark.parametrize("d", [64, 128])
