@@ -1,7 +1,8 @@
 """Benchmark: block-sparse attention with the LiteAttention skip chain on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME] [--no-e2e] [--no-cpu-baseline]
+                    [--workload NAME] [--no-e2e] [--no-cpu-baseline] [--no-configs]
+    python bench.py --suite     (every workload's path, one JSON line each)
 
 Default workload: the Wan2.1-14B-like 720p LiteAttention step (B=1, H=40,
 d=128, 21 x 45 x 80 grid = 75,600 tokens, block 128, eps = 10): each bench
@@ -18,6 +19,13 @@ call, density and the dense-equivalent rate alongside.  With N > 1 GPUs each
 rank runs its own copy of the workload (heads are independent; weak scaling,
 no collective on the data path) and the value is total FLOPs / max-over-ranks
 time.
+
+The same JSON line carries, under "configs" (single-GPU runs), the other
+workloads' paths, each device-timed with its roofline fraction and an oracle
+sample on the host (with the GPU-vs-oracle mask bit counts): the 480p
+tau-mask path, the 720p radial path, the 480p PSA pyramid path, and a
+labelled eps = 2 run of the 75.6K-token chain whose steps consume the skip
+bits of the step before (the time per step against the executed tiles).
 """
 from __future__ import annotations
 
@@ -37,10 +45,9 @@ sys.path.insert(0, ROOT)
 
 METRIC = "sparse attn ms/call, executed TFLOP/s & % B200 BF16 tensor peak at 75.6K tok"
 # DRAM bytes (read + write) of one attention launch at 75,600 tokens x 40 heads,
-# from the ncu capture summarised in profiles/attn_fwd_wan14b_720p_lite.md
-# (4-head case, 239.5 MB read + 61.4 MB written, scaled by 40/4 heads).  Valid
-# for the kernel version that capture names; set to None whenever the kernel
-# changes.
+# from an ncu capture of the 4-head case (239.5 MB read + 61.4 MB written,
+# scaled by 40/4 heads).  Valid for the kernel version that capture measured;
+# set to None whenever the kernel changes.
 ATTN_DRAM_BYTES_PER_LAUNCH = 3.0087e9
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -215,12 +222,22 @@ def run_ours(args, rank, world, local):
     dense = 4.0 * d * N * N * B * H
     total_ms_max, flops_all = reduce_over_ranks(total_ms, sum(flops), world, dev)
 
-    # end-to-end through the public API with host buffers (rank-local)
+    # end-to-end through the public API with host buffers, over the same drifted steps
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(ops, qkv[0], block, eps, nb, dev, stream, args.e2e_steps, world)
+        e2e = run_e2e(ops, qkv, args.warmup, block, eps, nb, dev, stream, world)
 
-    del qkv
+    # the other workloads' paths and the eps = 2 chain (rank 0 of a single-GPU run)
+    configs = None
+    if rank == 0 and world == 1 and not args.no_configs:
+        configs = {"lite_eps2_chain": lite_eps2_chain(ops, qkv, wl, dev, stream, statistics.median(kern_ms),
+                                                      args.cpu_seconds_config)}
+        del qkv
+        torch.cuda.empty_cache()
+        configs.update(run_configs(args, ops, dev, stream))
+    else:
+        del qkv
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         q, k, v = (t[:, :1].cpu() for t in (q0, k0, v0))
@@ -259,6 +276,7 @@ def run_ours(args, rank, world, local):
         "clocks": clk,
         "e2e": e2e,
         "cpu_baseline": cpu,
+        "configs": configs,
     }
     return line
 
@@ -266,38 +284,209 @@ def run_ours(args, rank, world, local):
 E2E_HEADS_PER_CHUNK = 2   # measured: 2 heads 98.2 ms per step, 4 heads 100.5, 8 heads 105
 
 
-def run_e2e(ops, qkv0, block, eps, nb, dev, stream, steps, world):
+def run_e2e(ops, qkv, first, block, eps, nb, dev, stream, world):
     """Same metric through the public C-ABI call with host buffers
-    (sa_sparse_attn_fwd_host): every step copies Q/K/V in from pinned host
-    memory and O back out, inside the timed region; the library overlaps the
-    copies of one chunk of heads with the attention of another."""
-    q0, k0, v0 = qkv0
-    B, H, N, d = q0.shape
-    hq, hk, hv = (t.cpu().pin_memory() for t in (q0, k0, v0))
-    ho = torch.empty_like(hq).pin_memory()
+    (sa_sparse_attn_fwd_host), over the same drifted denoising steps as the
+    device-timed value (steps first .. end of qkv) with the skip mask carried:
+    every step copies that step's Q/K/V in from pinned host memory and O back
+    out, inside the timed region; the library overlaps the copies of one chunk
+    of heads with the attention of another.  One untimed warm-up call first."""
+    steps = len(qkv) - first
+    B, H, N, d = qkv[0][0].shape
+    host = [tuple(t.cpu().pin_memory() for t in qkv[s]) for s in range(first - 1, len(qkv))]
+    ho = torch.empty_like(host[0][0]).pin_memory()
     ws = torch.empty(ops.sa_sparse_attn_fwd_host_workspace(N, d, min(E2E_HEADS_PER_CHUNK, H)), dtype=torch.uint8,
                      device=dev)
     skips = [torch.zeros(B, H, nb, nb, dtype=torch.uint8, device=dev) for _ in range(steps + 2)]
 
-    def one(s):
-        ops.sa_sparse_attn_fwd_host(hq, hk, hv, block, out=ho, skip_in=skips[s], skip_out=skips[s + 1], eps=eps,
+    def one(i):
+        hq, hk, hv = host[i]
+        ops.sa_sparse_attn_fwd_host(hq, hk, hv, block, out=ho, skip_in=skips[i], skip_out=skips[i + 1], eps=eps,
                                     heads_per_chunk=E2E_HEADS_PER_CHUNK, workspace=ws, stream=stream)
 
     one(0)
     torch.cuda.synchronize(dev)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
-    for s in range(1, steps + 1):
-        one(s)
+    for i in range(1, steps + 1):
+        one(i)
     b.record(stream)
     torch.cuda.synchronize(dev)
+    ops.sa_get_device_status(stream)
     ms = a.elapsed_time(b)
-    ms, flops = reduce_over_ranks(ms, sum(executed_flops(skips[s], N, block, d) for s in range(1, steps + 1)),
+    ms, flops = reduce_over_ranks(ms, sum(executed_flops(skips[i], N, block, d) for i in range(1, steps + 1)),
                                   world, dev)
+    n = qkv[0][0].numel()
     return {"value": round(whole_job_tflops(flops, ms), 2), "unit": "TFLOP/s",
-            "h2d_bytes_per_step": 3 * q0.numel() * 2, "d2h_bytes_per_step": q0.numel() * 2,
+            "h2d_bytes_per_step": 3 * n * 2, "d2h_bytes_per_step": n * 2,
             "ms_per_step": round(ms / steps, 3), "steps": steps,
+            "inputs": "the same drifted denoising steps as the device-timed value, skip mask carried",
             "api": f"sa_sparse_attn_fwd_host, {E2E_HEADS_PER_CHUNK} heads per chunk"}
+
+
+# ------------------------------------------------ the other workloads' paths ---
+
+CONFIG_REPS = 10
+LITE_DIAG_EPS = 2.0
+LITE_DIAG_STEPS = 6
+
+
+def lite_eps2_chain(ops, qkv, wl, dev, stream, ms_eps10, cpu_seconds):
+    """Diagnostic, labelled: the same 75.6K-token chain at eps = 2 (the
+    workload's eps = 10 skips nothing on this generator).  Step s consumes the
+    skip bits of step s - 1, so its executed tiles fall; the time per step
+    should fall with them (skipped tiles are neither loaded, multiplied nor
+    exponentiated).  The oracle sample recomputes step 0 for q-blocks of
+    head 0 and checks their skip rows."""
+    B, H, N, d, block = wl.B, wl.H, wl.N, wl.d, wl.block
+    nb = wl.nblocks
+    n = min(LITE_DIAG_STEPS, len(qkv))
+    skips = [torch.zeros(B, H, nb, nb, dtype=torch.uint8, device=dev) for _ in range(n + 1)]
+    out = torch.empty_like(qkv[0][0])
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for s in range(n):                      # untimed pass: the chain's skip masks
+        q, k, v = qkv[s]
+        ops.sa_sparse_attn_fwd(q, k, v, block, skip_in=skips[s], skip_out=skips[s + 1], eps=LITE_DIAG_EPS, out=out,
+                               stream=stream)
+    torch.cuda.synchronize(dev)
+    ms = []
+    for rep in range(3):                    # timed: each step on its own skip_in (skip_out to a scratch mask)
+        scratch = torch.empty_like(skips[0])
+        for s in range(n):
+            q, k, v = qkv[s]
+            ev[s][0].record(stream)
+            ops.sa_sparse_attn_fwd(q, k, v, block, skip_in=skips[s], skip_out=scratch, eps=LITE_DIAG_EPS, out=out,
+                                   stream=stream)
+            ev[s][1].record(stream)
+        torch.cuda.synchronize(dev)
+        ms.append([ev[s][0].elapsed_time(ev[s][1]) for s in range(n)])
+    ops.sa_get_device_status(stream)
+    dense = 4.0 * d * N * N * B * H
+    per_step = []
+    for s in range(n):
+        t = statistics.median(m[s] for m in ms)
+        fl = executed_flops(skips[s], N, block, d)
+        per_step.append({"step": s, "ms": round(t, 3), "density": round(fl / dense, 4),
+                         "executed_tflops": round(fl / t / 1e9, 1), "time_vs_eps10": round(t / ms_eps10, 4)})
+    cpu = None
+    if cpu_seconds > 0:
+        q, k, v = (t[:, :1].cpu() for t in qkv[0])
+        cpu = cpu_sample(q, k, v, block, LITE_DIAG_EPS, cpu_seconds, gpu_skip=skips[1][:, :1].cpu().numpy())
+    return {"what": f"diagnostic: eps = {LITE_DIAG_EPS:g} instead of the workload's {wl.eps:g}, same inputs",
+            "eps": LITE_DIAG_EPS, "ms_eps10": round(ms_eps10, 3), "steps": per_step, "cpu_baseline": cpu}
+
+
+def run_configs(args, ops, dev, stream):
+    """The three other workloads' hot paths, one entry each (device-timed,
+    CUDA-event medians of CONFIG_REPS calls after 3 warm-ups)."""
+    from block_sparse_attention_flash_b200 import inputs
+
+    peaks, src = load_peaks()
+    out = {}
+    for name in ("wan13b_480p_tau", "hunyuan_720p_radial", "psa_480p_pyramid"):
+        wl = inputs.WORKLOADS[name]
+        q, k, v = inputs.rff_qkv(wl, device=dev)
+        if wl.kind == "tau":
+            out[name] = config_tau(ops, wl, q, k, v, dev, stream, peaks, src, args.cpu_seconds_config)
+        elif wl.kind == "radial":
+            out[name] = config_radial(ops, wl, q, k, v, dev, stream, peaks, src, args.cpu_seconds_config)
+        else:
+            out[name] = config_psa(ops, wl, q, k, v, dev, stream, peaks, src, args.cpu_seconds_config)
+        ops.sa_get_device_status(stream)
+        del q, k, v
+        torch.cuda.empty_cache()
+    return out
+
+
+def _attn_entry(wl, ms, flops, peaks, src, algorithmic_flops=None):
+    dense = 4.0 * wl.d * wl.N * wl.N * wl.B * wl.H
+    alg = flops if algorithmic_flops is None else algorithmic_flops
+    burst, sust = float(peaks["bf16_tflops"]), float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+    tf = alg / ms / 1e9
+    return {"ms_per_call": round(ms, 3), "density": round(alg / dense, 5), "executed_tflops": round(tf, 1),
+            "dense_equiv_tflops": round(dense / ms / 1e9, 1),
+            "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": burst, "unit": "TFLOP/s",
+                         "frac": round(tf / burst, 4), "frac_of_sustained": round(tf / sust, 4),
+                         "peak_source": f"{src} bf16_tflops (burst: a kernel timed alone)"}}
+
+
+def _hbm_entry(ms, nbytes, peaks, src):
+    gbs = nbytes / ms / 1e6
+    return {"ms_per_call": round(ms, 4), "roofline": {"bound": "hbm", "achieved": round(gbs, 1),
+                                                      "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                                                      "frac": round(gbs / float(peaks["hbm_gbs"]), 4),
+                                                      "algorithmic_bytes": nbytes, "peak_source": f"{src} hbm_gbs"}}
+
+
+def config_tau(ops, wl, q, k, v, dev, stream, peaks, src, cpu_seconds):
+    B, H, N, d = q.shape
+    nb = wl.nblocks
+    ws = torch.empty(ops.sa_build_mask_workspace(B, H, N, d, wl.block), dtype=torch.uint8, device=dev)
+    m = torch.empty(B, H, nb, nb, dtype=torch.uint8, device=dev)
+    o = torch.empty_like(q)
+    ms_m = _time(lambda: ops.sa_build_mask(q, k, wl.block, "tau", tau=wl.tau, mask_out=m, workspace=ws),
+                 CONFIG_REPS, stream, SHORT_CALL_BATCH)
+    ms_a = _time(lambda: ops.sa_sparse_attn_fwd(q, k, v, wl.block, mask=m, out=o), CONFIG_REPS, stream)
+    flops = executed_flops(torch.zeros_like(m), N, wl.block, d, mask=m)
+    mask_bytes = 2 * B * H * N * d * 2 + B * H * nb * nb
+    entry = {"path": "sa_build_mask (tau) + sa_sparse_attn_fwd", "attention": _attn_entry(wl, ms_a, flops, peaks, src),
+             "mask_builder": _hbm_entry(ms_m, mask_bytes, peaks, src)}
+    if cpu_seconds > 0:
+        entry["cpu_baseline"] = cpu_config_sample(wl, q, k, v, m, cpu_seconds, "tau")
+    return entry
+
+
+def config_radial(ops, wl, q, k, v, dev, stream, peaks, src, cpu_seconds):
+    B, H, N, d = q.shape
+    nb = wl.nblocks
+    rm = ops.sa_radial_mask(wl.T, wl.Hh, wl.Ww, wl.block)
+    o = torch.empty_like(q)
+    ms_r = _time(lambda: ops.sa_radial_mask(wl.T, wl.Hh, wl.Ww, wl.block, out=rm), CONFIG_REPS, stream,
+                 SHORT_CALL_BATCH)
+    ms_a = _time(lambda: ops.sa_sparse_attn_fwd(q, k, v, wl.block, mask=rm, out=o), CONFIG_REPS, stream)
+    m4 = rm.view(1, 1, nb, nb).expand(B, H, nb, nb)
+    flops = executed_flops(torch.zeros(B, H, nb, nb, dtype=torch.uint8, device=dev), N, wl.block, d, mask=m4)
+    entry = {"path": "sa_radial_mask + sa_sparse_attn_fwd", "attention": _attn_entry(wl, ms_a, flops, peaks, src),
+             "radial_mask": _hbm_entry(ms_r, nb * nb, peaks, src)}
+    if cpu_seconds > 0:
+        entry["cpu_baseline"] = cpu_config_sample(wl, q, k, v, rm, cpu_seconds, "radial")
+    return entry
+
+
+def pyramid_flops(lv, N, block, d):
+    """Algorithmic pyramid work: 4 d x valid rows x pooled keys of each (i, j) at its level."""
+    B, H, nb, _ = lv.shape
+    rows = torch.full((nb,), float(block), device=lv.device, dtype=torch.float64)
+    rows[-1] = N - (nb - 1) * block
+    cols = torch.zeros(B, H, nb, nb, dtype=torch.float64, device=lv.device)
+    for lvl in range(4):
+        cnt = torch.full((nb,), float(block >> lvl), device=lv.device, dtype=torch.float64)
+        cnt[-1] = -(-int(rows[-1].item()) // (1 << lvl))
+        cols += (lv == lvl + 1).to(torch.float64) * cnt.view(1, 1, 1, nb)
+    return float(4.0 * d * torch.einsum("i,bhij->", rows, cols).item())
+
+
+def config_psa(ops, wl, q, k, v, dev, stream, peaks, src, cpu_seconds):
+    B, H, N, d = q.shape
+    nb = wl.nblocks
+    ws = torch.empty(ops.sa_build_mask_workspace(B, H, N, d, wl.block), dtype=torch.uint8, device=dev)
+    lv = torch.empty(B, H, nb, nb, dtype=torch.uint8, device=dev)
+    kp, vp = ops.sa_pyramid_pool(k, v, wl.block)
+    o = torch.empty_like(q)
+    ms_l = _time(lambda: ops.sa_build_mask(q, k, wl.block, "levels", level_frac=wl.level_frac, mask_out=lv,
+                                           workspace=ws), CONFIG_REPS, stream, SHORT_CALL_BATCH)
+    ms_p = _time(lambda: ops.sa_pyramid_pool(k, v, wl.block, k_pool=kp, v_pool=vp), CONFIG_REPS, stream,
+                 SHORT_CALL_BATCH)
+    ms_a = _time(lambda: ops.sa_pyramid_attn_fwd(q, k, v, wl.block, lv, kp, vp, out=o), CONFIG_REPS, stream)
+    flops = pyramid_flops(lv, N, wl.block, d)
+    kv_bytes = 2 * B * H * N * d * 2
+    entry = {"path": "sa_build_mask (levels) + sa_pyramid_pool + sa_pyramid_attn_fwd",
+             "attention": _attn_entry(wl, ms_a, flops, peaks, src),
+             "level_map": _hbm_entry(ms_l, kv_bytes + B * H * nb * nb, peaks, src),
+             "pool": _hbm_entry(ms_p, kv_bytes + kv_bytes * 7 // 8, peaks, src)}
+    if cpu_seconds > 0:
+        entry["cpu_baseline"] = cpu_config_sample(wl, q, k, v, lv, cpu_seconds, "levels")
+    return entry
 
 
 # -------------------------------------------------------------- suite mode ---
@@ -425,15 +614,7 @@ def run_suite(args):
             lv = ops.sa_build_mask(q, k, wl.block, "levels", level_frac=wl.level_frac)
             ms_a = _time(lambda: ops.sa_pyramid_attn_fwd(q, k, v, wl.block, lv, kp, vp, out=o), args.suite_reps,
                          stream)
-            # executed keys per (i, j): block >> level (valid rows x pooled cols)
-            rows = torch.full((nb,), float(wl.block), device=dev, dtype=torch.float64)
-            rows[-1] = N - (nb - 1) * wl.block
-            cols = torch.zeros(B, H, nb, nb, dtype=torch.float64, device=dev)
-            for lvl in range(4):
-                cnt = torch.full((nb,), float(wl.block >> lvl), device=dev, dtype=torch.float64)
-                cnt[-1] = -(-int(rows[-1].item()) // (1 << lvl))
-                cols += (lv == lvl + 1).to(torch.float64) * cnt.view(1, 1, 1, nb)
-            flops = float(4.0 * d * torch.einsum("i,bhij->", rows, cols).item())
+            flops = pyramid_flops(lv, N, wl.block, d)
             pool_bytes = qk_bytes + qk_bytes * 7 // 8
             out.append(attn_line(wl, name, ms_a, flops, {
                 "pool_ms": round(ms_p, 4), "pool_gbs": round(pool_bytes / ms_p / 1e6, 1),
@@ -447,29 +628,98 @@ def run_suite(args):
 
 # ------------------------------------------------------------ oracle timing ---
 
-def cpu_sample(q, k, v, block, eps, seconds):
-    """Time the fp64 oracle's lite_step on q-blocks of head 0, step 0, for about
-    `seconds` of host time; report its executed TFLOP/s."""
-    import numpy as np
+def _threads():
     from threadpoolctl import threadpool_info
+    return max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+
+
+def _bit_check(got, want, flags=None):
+    """Counts of a GPU-vs-oracle mask comparison (flags: the oracle's margin flags)."""
+    import numpy as np
+    bad = np.asarray(got) != np.asarray(want)
+    out = {"bits": int(bad.size), "mismatches": int(bad.sum())}
+    if flags is not None:
+        f = np.asarray(flags, dtype=bool)
+        out.update({"flagged": int(f.sum()), "flagged_mismatches": int((bad & f).sum()),
+                    "unflagged_mismatches": int((bad & ~f).sum())})
+    return out
+
+
+def cpu_sample(q, k, v, block, eps, seconds, gpu_skip=None):
+    """Time the fp64 oracle's lite_step on q-blocks of head 0, step 0, for about
+    `seconds` of host time; report its executed TFLOP/s.  With gpu_skip (the
+    GPU's skip_out of that step for head 0) the oracle's skip rows of the
+    sampled q-blocks are compared with it (bit counts, margin-flag aware)."""
+    import numpy as np
     import oracle
 
     N, d = q.shape[2], q.shape[3]
     nb = -(-N // block)
-    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    order = list(range(0, nb, max(1, nb // 64)))
+    done, flops = 0, 0.0
+    got, want, flags = [], [], []
+    t0 = time.perf_counter()
+    for i in order:
+        ref = oracle.lite_step(q, k, v, block, None, None, eps, qblocks=[(0, 0, i)])
+        rows = min(block, N - i * block)
+        flops += 4.0 * d * rows * N
+        done += 1
+        if gpu_skip is not None:
+            _, _, srow, mrow = ref[(0, 0, i)]
+            got.append(gpu_skip[0, 0, i]), want.append(srow), flags.append(oracle.skip_flags(mrow))
+        if time.perf_counter() - t0 > seconds:
+            break
+    dt = time.perf_counter() - t0
+    out = {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": _threads(), "kind": "oracle",
+           "sample": f"{done} q-blocks of head 0 at denoising step 0 (all {N} keys each), {dt:.1f} s"}
+    if gpu_skip is not None:
+        out["skip_check"] = _bit_check(np.stack(got), np.stack(want), np.stack(flags))
+    return out
+
+
+def cpu_config_sample(wl, q, k, v, gpu_mask, seconds, kind):
+    """The oracle on head 0 of one workload: its mask builder (timed, and its
+    mask compared with the GPU's, margin-flag aware), then its attention on
+    its own mask for q-blocks spread over the sequence, for about `seconds`;
+    the value is executed TFLOP/s of the attention (algorithmic work)."""
+    import numpy as np
+    import oracle
+
+    qh, kh, vh = (t[:, :1].cpu() for t in (q, k, v))
+    N, d, block = wl.N, wl.d, wl.block
+    nb = wl.nblocks
+    t0 = time.perf_counter()
+    if kind == "tau":
+        ref, flags, _ = oracle.tau_mask(qh, kh, block, wl.tau, return_info=True)
+    elif kind == "levels":
+        ref, flags, _ = oracle.level_map(qh, kh, block, wl.level_frac, return_info=True)
+    else:
+        ref, flags = oracle.radial_mask(wl.T, wl.Hh, wl.Ww, block)[None, None], None
+    t_mask = time.perf_counter() - t0
+    g = gpu_mask.cpu().numpy()
+    g = g[:1, :1] if g.ndim == 4 else g[None, None]
+    check = _bit_check(g, ref, flags)
+    valid = np.full(nb, block, dtype=np.int64)
+    valid[-1] = N - (nb - 1) * block
     order = list(range(0, nb, max(1, nb // 64)))
     done, flops = 0, 0.0
     t0 = time.perf_counter()
     for i in order:
-        oracle.lite_step(q, k, v, block, None, None, eps, qblocks=[(0, 0, i)])
-        rows = min(block, N - i * block)
-        flops += 4.0 * d * rows * N
+        if kind == "levels":
+            oracle.pyramid_attention(qh, kh, vh, block, ref, qblocks=[(0, 0, i)])
+            cols = sum(-(-int(valid[j]) // (1 << (int(ref[0, 0, i, j]) - 1))) for j in range(nb) if ref[0, 0, i, j])
+        else:
+            oracle.masked_attention(qh, kh, vh, block, ref, qblocks=[(0, 0, i)])
+            cols = int(valid[ref[0, 0, i] != 0].sum())
+        flops += 4.0 * d * int(valid[i]) * cols
         done += 1
         if time.perf_counter() - t0 > seconds:
             break
     dt = time.perf_counter() - t0
-    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-            "sample": f"{done} q-blocks of head 0 at denoising step 0 (all {N} keys each), {dt:.1f} s"}
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": _threads(), "kind": "oracle",
+            "sample": f"mask builder on head 0 ({t_mask:.1f} s), then attention on the oracle's mask for {done} "
+                      f"q-blocks of head 0 ({dt:.1f} s)",
+            "mask_check": check}
 
 
 def run_reference(args, rank, world):
@@ -509,9 +759,11 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="wan14b_720p_lite")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the other workloads' entries")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--cpu-seconds-config", type=float, default=5.0,
+                    help="oracle seconds per entry of `configs` (0: no oracle sample there)")
     ap.add_argument("--ref-seconds", type=float, default=60.0)
     ap.add_argument("--suite", action="store_true", help="time every workload's hot path (one line each)")
     ap.add_argument("--suite-reps", type=int, default=10)

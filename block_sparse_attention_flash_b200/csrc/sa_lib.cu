@@ -134,6 +134,15 @@ long long tail_units_to_split(long long units, int n_sm) {
 bool valid_dim(int d) { return d == 64 || d == 128; }
 bool valid_block(int b) { return b == 64 || b == 128; }
 
+// Cumulative level quota ceil(f * nb) for a fraction passed as fp32.  The fp32
+// value of a decimal fraction can sit just above it (0.1f = 0.10000000149),
+// which would lift an exact product (0.1 * 1000 = 100) past the integer; a
+// product within 1e-3 blocks above an integer is taken as that integer.  The
+// representation error is below 2^-24 * nb <= 2.5e-4 blocks for nb <= 4096.
+int level_quota(float f, int nb) {
+  return static_cast<int>(std::ceil(static_cast<double>(f) * nb - 1e-3));
+}
+
 // Host-side checks shared by sa_build_mask and sa_build_mask_noalloc (all but
 // the workspace).  *empty is set for a call with no rows (nothing to launch).
 sa_status check_build_mask_args(const void* q, const void* k, int B, int H, int N, int d, int block, int mode,
@@ -219,9 +228,9 @@ sa_status sa_build_mask(const void* q, const void* k, int B, int H, int N, int d
   const int nb = ceil_div(N, block);
   int c0 = 0, c1 = 0, c2 = 0;
   if (mode == SA_MASK_LEVELS) {
-    c0 = static_cast<int>(std::ceil(static_cast<double>(level_frac[0]) * nb - 1e-9));
-    c1 = static_cast<int>(std::ceil(static_cast<double>(level_frac[1]) * nb - 1e-9));
-    c2 = static_cast<int>(std::ceil(static_cast<double>(level_frac[2]) * nb - 1e-9));
+    c0 = level_quota(level_frac[0], nb);
+    c1 = level_quota(level_frac[1], nb);
+    c2 = level_quota(level_frac[2], nb);
   }
   cudaError_t e = init_device_kernels();
   if (e != cudaSuccess) return SA_ERR_CUDA;

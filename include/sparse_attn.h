@@ -137,8 +137,11 @@ SA_API size_t sa_build_mask_workspace(int B, int H, int N, int d, int block);
  *                   visited before it is < tau * Nb.  A row may keep nothing.
  *   SA_MASK_LEVELS: rank r_j of S_ij in the same order; with quotas
  *                   c_l = ceil(level_frac[l] * Nb) (cumulative fractions,
- *                   non-decreasing), code = 1 if r < c_0, 2 if r < c_1,
- *                   3 if r < c_2, else 4 (code = pyramid level + 1).
+ *                   non-decreasing; a product within 1e-3 above an integer
+ *                   counts as that integer, so that 0.1f * 1000 gives 100
+ *                   although 0.1f is slightly above 0.1), code = 1 if
+ *                   r < c_0, 2 if r < c_1, 3 if r < c_2, else 4 (code =
+ *                   pyramid level + 1).
  * Arguments
  *   q, k        bf16 [B,H,N,d] device, read only.
  *   tau         (0, 1]; used for SA_MASK_TAU and SA_MASK_GLOBAL.
