@@ -293,7 +293,12 @@ def run_e2e(ops, qkv, first, block, eps, nb, dev, stream, world):
     of heads with the attention of another.  One untimed warm-up call first."""
     steps = len(qkv) - first
     B, H, N, d = qkv[0][0].shape
-    host = [tuple(t.cpu().pin_memory() for t in qkv[s]) for s in range(first - 1, len(qkv))]
+    def pinned(t):
+        h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        h.copy_(t)
+        return h
+
+    host = [tuple(pinned(t) for t in qkv[s]) for s in range(first - 1, len(qkv))]
     ho = torch.empty_like(host[0][0]).pin_memory()
     ws = torch.empty(ops.sa_sparse_attn_fwd_host_workspace(N, d, min(E2E_HEADS_PER_CHUNK, H)), dtype=torch.uint8,
                      device=dev)

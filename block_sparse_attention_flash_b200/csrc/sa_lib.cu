@@ -88,10 +88,14 @@ cudaError_t init_device_kernels() {
     set(reinterpret_cast<const void*>(&sa::attn_fwd_kernel<128, 64, true>), sa::AttnSmem<128>::kAlloc);
     set(reinterpret_cast<const void*>(&sa::attn_fwd_kernel<64, 128, true>), sa::AttnSmem<64>::kAlloc);
     set(reinterpret_cast<const void*>(&sa::attn_fwd_kernel<64, 64, true>), sa::AttnSmem<64>::kAlloc);
-    set(reinterpret_cast<const void*>(&sa::pyr_fwd_kernel<128, 128>), sa::PyrSmem<128>::kAlloc);
-    set(reinterpret_cast<const void*>(&sa::pyr_fwd_kernel<128, 64>), sa::PyrSmem<128>::kAlloc);
-    set(reinterpret_cast<const void*>(&sa::pyr_fwd_kernel<64, 128>), sa::PyrSmem<64>::kAlloc);
-    set(reinterpret_cast<const void*>(&sa::pyr_fwd_kernel<64, 64>), sa::PyrSmem<64>::kAlloc);
+    set(reinterpret_cast<const void*>(&sa::pyr_fwd_kernel<128, 128, false>), sa::PyrSmem<128>::kAlloc);
+    set(reinterpret_cast<const void*>(&sa::pyr_fwd_kernel<128, 64, false>), sa::PyrSmem<128>::kAlloc);
+    set(reinterpret_cast<const void*>(&sa::pyr_fwd_kernel<64, 128, false>), sa::PyrSmem<64>::kAlloc);
+    set(reinterpret_cast<const void*>(&sa::pyr_fwd_kernel<64, 64, false>), sa::PyrSmem<64>::kAlloc);
+    set(reinterpret_cast<const void*>(&sa::pyr_fwd_kernel<128, 128, true>), sa::PyrSmem<128>::kAlloc);
+    set(reinterpret_cast<const void*>(&sa::pyr_fwd_kernel<128, 64, true>), sa::PyrSmem<128>::kAlloc);
+    set(reinterpret_cast<const void*>(&sa::pyr_fwd_kernel<64, 128, true>), sa::PyrSmem<64>::kAlloc);
+    set(reinterpret_cast<const void*>(&sa::pyr_fwd_kernel<64, 64, true>), sa::PyrSmem<64>::kAlloc);
     set(reinterpret_cast<const void*>(&sa::bwd_dkdv_kernel<128, 128>), sa::BwdSmem<128>::kAlloc);
     set(reinterpret_cast<const void*>(&sa::bwd_dkdv_kernel<128, 64>), sa::BwdSmem<128>::kAlloc);
     set(reinterpret_cast<const void*>(&sa::bwd_dkdv_kernel<64, 128>), sa::BwdSmem<64>::kAlloc);
@@ -459,7 +463,6 @@ sa_status sa_pyramid_attn_fwd(const void* q, const void* k, const void* v, int B
   p.lsh = lv_sh;
   p.lsi = lv_si;
   p.scale_log2 = scale * 1.4426950408889634f;
-  p.causal = causal;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   const int n_pairs = ceil_div(ceil_div(N, sa::kTileM), 2);
@@ -469,14 +472,17 @@ sa_status sa_pyramid_attn_fwd(const void* q, const void* k, const void* v, int B
   p.n_full = static_cast<int>(units - n_split);
   dim3 grid(static_cast<unsigned>(units + n_split));
   cudaStream_t s = as_stream(stream);
+#define SA_PYR_LAUNCH(DD, BB, CC) \
+  sa::pyr_fwd_kernel<DD, BB, CC><<<grid, sa::kPyrThreads, sa::PyrSmem<DD>::kAlloc, s>>>(tq, maps, p)
   if (d == 128 && block == 128)
-    sa::pyr_fwd_kernel<128, 128><<<grid, sa::kPyrThreads, sa::PyrSmem<128>::kAlloc, s>>>(tq, maps, p);
+    causal ? SA_PYR_LAUNCH(128, 128, true) : SA_PYR_LAUNCH(128, 128, false);
   else if (d == 128 && block == 64)
-    sa::pyr_fwd_kernel<128, 64><<<grid, sa::kPyrThreads, sa::PyrSmem<128>::kAlloc, s>>>(tq, maps, p);
+    causal ? SA_PYR_LAUNCH(128, 64, true) : SA_PYR_LAUNCH(128, 64, false);
   else if (d == 64 && block == 128)
-    sa::pyr_fwd_kernel<64, 128><<<grid, sa::kPyrThreads, sa::PyrSmem<64>::kAlloc, s>>>(tq, maps, p);
+    causal ? SA_PYR_LAUNCH(64, 128, true) : SA_PYR_LAUNCH(64, 128, false);
   else
-    sa::pyr_fwd_kernel<64, 64><<<grid, sa::kPyrThreads, sa::PyrSmem<64>::kAlloc, s>>>(tq, maps, p);
+    causal ? SA_PYR_LAUNCH(64, 64, true) : SA_PYR_LAUNCH(64, 64, false);
+#undef SA_PYR_LAUNCH
   return cuda_status(cudaGetLastError());
 }
 

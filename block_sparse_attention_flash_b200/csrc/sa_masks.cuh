@@ -327,27 +327,30 @@ __global__ void __launch_bounds__(kSelectThreads) block_select_kernel(const floa
   for (int j = threadIdx.x; j < nb; j += kSelectThreads) mrow[j] = out_row[j];
 }
 
-// Warp-per-row variant for rows of at most 32*E blocks (E <= 32): the keys
+// Score row accessor: element i of a row at `base`, either plain (a row of
+// the scores array in global memory) or skewed by one word per 32 (a row
+// staged in shared memory, so that lane l reading element l*E + k hits a
+// bank of its own for every E).
+template <bool SKEW>
+__device__ __forceinline__ int score_index(int i) {
+  return SKEW ? i + (i >> 5) : i;
+}
+
+// Warp-per-row selection for rows of at most 32*E blocks (E <= 32): the keys
 // live in registers (E per lane, blocked: lane l holds ranks l*E .. l*E+E-1
 // after the sort) and the bitonic network uses in-register swaps for strides
-// below E and shuffles above.  Four rows per 128-thread CTA.
-template <int E>
-__global__ void __launch_bounds__(128) block_select_warp_kernel(const float* __restrict__ scores, int nb,
-                                                                long long nrows, int mode, float tau, int c0,
-                                                                int c1, int c2, uint8_t* __restrict__ mask_out) {
+// below E and shuffles above.  `stage` is the warp's P-byte staging row.
+template <int E, bool SKEW>
+__device__ __forceinline__ void block_select_row(const float* srow, int nb, int mode, float tau, int c0, int c1,
+                                                 int c2, uint8_t* stage, uint8_t* __restrict__ mrow, int lane) {
   constexpr int P = 32 * E;
-  __shared__ uint8_t stage[4][P];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long row = static_cast<long long>(blockIdx.x) * 4 + warp;
-  if (row >= nrows) return;
-  const float* srow = scores + row * nb;
   unsigned long long key[E];
   float mx = -__int_as_float(0x7f800000);
 #pragma unroll
   for (int k = 0; k < E; ++k) {
     const int i = lane * E + k;
     if (i < nb) {
-      const float sc = srow[i];
+      const float sc = srow[score_index<SKEW>(i)];
       mx = fmaxf(mx, sc);
       key[k] = (static_cast<unsigned long long>(~float_order_key(sc)) << 32) | static_cast<unsigned>(i);
     } else {
@@ -362,7 +365,7 @@ __global__ void __launch_bounds__(128) block_select_warp_kernel(const float* __r
 #pragma unroll
     for (int k = 0; k < E; ++k) {
       const int i = lane * E + k;
-      if (i < nb) sum += expf(srow[i] - mx);
+      if (i < nb) sum += expf(srow[score_index<SKEW>(i)] - mx);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
@@ -405,7 +408,7 @@ __global__ void __launch_bounds__(128) block_select_warp_kernel(const float* __r
 #pragma unroll
     for (int k = 0; k < E; ++k) {
       const unsigned j = static_cast<unsigned>(key[k]);
-      pk[k] = key[k] != ~0ull ? expf(srow[j] - mx) * inv : 0.f;
+      pk[k] = key[k] != ~0ull ? expf(srow[score_index<SKEW>(static_cast<int>(j))] - mx) * inv : 0.f;
       lsum += pk[k];
     }
     float inc = lsum;
@@ -417,7 +420,7 @@ __global__ void __launch_bounds__(128) block_select_warp_kernel(const float* __r
     float before = inc - lsum;
 #pragma unroll
     for (int k = 0; k < E; ++k) {
-      if (key[k] != ~0ull) stage[warp][static_cast<unsigned>(key[k])] = before < tau ? 1 : 0;
+      if (key[k] != ~0ull) stage[static_cast<unsigned>(key[k])] = before < tau ? 1 : 0;
       before += pk[k];
     }
   } else {
@@ -425,12 +428,31 @@ __global__ void __launch_bounds__(128) block_select_warp_kernel(const float* __r
     for (int k = 0; k < E; ++k) {
       const int r = lane * E + k;
       if (key[k] != ~0ull)
-        stage[warp][static_cast<unsigned>(key[k])] = r < c0 ? 1 : (r < c1 ? 2 : (r < c2 ? 3 : 4));
+        stage[static_cast<unsigned>(key[k])] = r < c0 ? 1 : (r < c1 ? 2 : (r < c2 ? 3 : 4));
     }
   }
   __syncwarp();
-  uint8_t* mrow = mask_out + row * nb;
-  for (int j = lane; j < nb; j += 32) mrow[j] = stage[warp][j];
+  for (int j = lane; j < nb; j += 32) mrow[j] = stage[j];
+  __syncwarp();
+}
+
+// Four rows per 128-thread CTA, one warp each.  The row is read from global
+// memory with consecutive lanes on consecutive blocks and staged in shared
+// memory (skewed), so the blocked reads of the sort hit distinct banks.
+template <int E>
+__global__ void __launch_bounds__(128) block_select_warp_kernel(const float* __restrict__ scores, int nb,
+                                                                long long nrows, int mode, float tau, int c0,
+                                                                int c1, int c2, uint8_t* __restrict__ mask_out) {
+  constexpr int P = 32 * E;
+  __shared__ uint8_t stage[4][P];
+  __shared__ float row_s[4][P + P / 32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long row = static_cast<long long>(blockIdx.x) * 4 + warp;
+  if (row >= nrows) return;
+  const float* srow = scores + row * nb;
+  for (int i = lane; i < nb; i += 32) row_s[warp][score_index<true>(i)] = srow[i];
+  __syncwarp();
+  block_select_row<E, true>(row_s[warp], nb, mode, tau, c0, c1, c2, stage[warp], mask_out + row * nb, lane);
 }
 
 // TAU rows without a sort (rows of at most 32*E blocks, one warp per row):
@@ -439,21 +461,17 @@ __global__ void __launch_bounds__(128) block_select_warp_kernel(const float* __r
 // 32-bit score key whose cumulative mass reaches tau; it is found bit by bit
 // from the most significant end (32 rounds of a masked warp sum).  Blocks
 // with a key below K* are kept; blocks whose key equals K* (equal scores) are
-// kept in ascending j while the mass before them is < tau.
+// kept in ascending j while the mass before them is < tau.  Lane l holds
+// blocks j = 32 k + l (k < E), so the row is read with coalesced loads.
 template <int E>
-__global__ void __launch_bounds__(128) tau_select_warp_kernel(const float* __restrict__ scores, int nb,
-                                                              long long nrows, float tau,
-                                                              uint8_t* __restrict__ mask_out) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long row = static_cast<long long>(blockIdx.x) * 4 + warp;
-  if (row >= nrows) return;
-  const float* srow = scores + row * nb;
+__device__ __forceinline__ void tau_select_row(const float* __restrict__ srow, int nb, float tau,
+                                               uint8_t* __restrict__ mrow, int lane) {
   float sc[E], pr[E];
   uint32_t key[E];
   float mx = -__int_as_float(0x7f800000);
 #pragma unroll
   for (int k = 0; k < E; ++k) {
-    const int i = lane * E + k;
+    const int i = 32 * k + lane;
     sc[k] = i < nb ? srow[i] : -__int_as_float(0x7f800000);
     mx = fmaxf(mx, sc[k]);
   }
@@ -462,7 +480,7 @@ __global__ void __launch_bounds__(128) tau_select_warp_kernel(const float* __res
   float sum = 0.f;
 #pragma unroll
   for (int k = 0; k < E; ++k) {
-    const int i = lane * E + k;
+    const int i = 32 * k + lane;
     pr[k] = i < nb ? expf(sc[k] - mx) : 0.f;
     sum += pr[k];
     key[k] = i < nb ? ~float_order_key(sc[k]) : 0xFFFFFFFFu;   // ascending key = descending score
@@ -484,35 +502,37 @@ __global__ void __launch_bounds__(128) tau_select_warp_kernel(const float* __res
     for (int o = 16; o > 0; o >>= 1) m += __shfl_xor_sync(0xffffffffu, m, o);
     if (!(m >= tau)) kstar |= 1u << b;
   }
-  // mass strictly before K*, and the rank in j of each block tied at K*
+  // mass strictly before K*
   float below = 0.f;
-  int ties = 0;
 #pragma unroll
-  for (int k = 0; k < E; ++k) {
-    below += key[k] < kstar ? pr[k] : 0.f;
-    ties += key[k] == kstar && (lane * E + k) < nb ? 1 : 0;
-  }
+  for (int k = 0; k < E; ++k) below += key[k] < kstar ? pr[k] : 0.f;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) below += __shfl_xor_sync(0xffffffffu, below, o);
-  int tie_before = ties;   // exclusive prefix over lanes (blocks are numbered lane * E + k)
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, tie_before, o);
-    if (lane >= o) tie_before += y;
-  }
-  tie_before -= ties;
-  uint8_t* mrow = mask_out + row * nb;
+  // blocks tied at K*, in ascending j: chunk by chunk, lanes in order
+  int tie_before = 0;
+  const unsigned lower = (1u << lane) - 1u;
 #pragma unroll
   for (int k = 0; k < E; ++k) {
-    const int i = lane * E + k;
-    if (i >= nb) continue;
-    uint8_t keep = key[k] < kstar ? 1 : 0;
-    if (key[k] == kstar) {
-      keep = below + static_cast<float>(tie_before) * pr[k] < tau ? 1 : 0;
-      ++tie_before;
+    const int i = 32 * k + lane;
+    const bool tied = key[k] == kstar && i < nb;
+    const unsigned ball = __ballot_sync(0xffffffffu, tied);
+    if (i < nb) {
+      uint8_t keep = key[k] < kstar ? 1 : 0;
+      if (tied) keep = below + static_cast<float>(tie_before + __popc(ball & lower)) * pr[k] < tau ? 1 : 0;
+      mrow[i] = keep;
     }
-    mrow[i] = keep;
+    tie_before += __popc(ball);
   }
+}
+
+template <int E>
+__global__ void __launch_bounds__(128) tau_select_warp_kernel(const float* __restrict__ scores, int nb,
+                                                              long long nrows, float tau,
+                                                              uint8_t* __restrict__ mask_out) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long row = static_cast<long long>(blockIdx.x) * 4 + warp;
+  if (row >= nrows) return;
+  tau_select_row<E>(scores + row * nb, nb, tau, mask_out + row * nb, lane);
 }
 
 // ----------------------------------------------------------- pyramid pool ---

@@ -43,6 +43,12 @@ constexpr int kPyrWarps = 12;
 constexpr int kPyrThreads = kPyrWarps * 32;
 constexpr int kPyrMaxSegs = 2 * kPyrMaxBlocks;      // per q-tile (union of 2 q-blocks)
 constexpr int kPyrMaxEntries = kPyrMaxBlocks;       // packed key tiles per q-tile
+// Entry word of a packed key tile: index of its first segment (bits 0-10),
+// uniform flag (bit 11: every segment has the same level and row mask and
+// holds full groups, so the bias is one constant per q-block), level (bits
+// 12-13) and row mask (bits 14-15) of its first segment.
+constexpr uint32_t kEntStartMask = 0x7FFu;
+constexpr uint32_t kEntUniform = 1u << 11;
 // Raw-logit bias of a masked or empty column, and the row maximum below which
 // a row has no valid column in a tile (real logits are many orders smaller).
 constexpr float kMaskedBias = -30000.f;
@@ -54,7 +60,6 @@ struct PyrParams {
   const uint8_t* levels;  // code map: 0 drop, 1 + l level l
   long long lsb, lsh, lsi;
   float scale_log2;
-  int causal;             // k-blocks j > i dropped, the diagonal block at level 0 cut per row
   int n_pairs;            // q-tile pairs per head
   int n_full;             // CTAs [0, n_full) take a whole pair; each later pair runs as two CTAs, one per q-tile
   __nv_bfloat16* o;
@@ -93,7 +98,7 @@ struct PyrMaps {
   CUtensorMap v[4];
 };
 
-template <int D, int BLK>
+template <int D, int BLK, bool CAUSAL>
 __global__ void __launch_bounds__(kPyrThreads, 1)
     pyr_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ PyrMaps maps,
                    const PyrParams p) {
@@ -124,7 +129,8 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
   volatile int* misc = reinterpret_cast<volatile int*>(smem + L::kOffMisc);
   // misc[0] TMEM base, [1]/[2] segments of q-tile 0/1, [3]/[4] key tiles of q-tile 0/1, [5] abort,
   // [6]/[7] packed columns of q-tile 0/1, [8 + 2t + x] causal: key tile * 256 + column of the
-  // diagonal segment of q-block x of q-tile t (-1: none)
+  // diagonal segment of q-block x of q-tile t (-1: none), [12 + 2t + x] key tiles of q-tile t
+  // holding a segment of the last block (-1: none)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // Work unit u = bh * n_pairs + pair, in launch order.  Units from n_full on
@@ -140,62 +146,143 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
   const int b = bh / p.H, h = bh - (bh / p.H) * p.H;
   const int qtile0 = 2 * pair;
 
-  if (warp == 0) {
-    // ---- per q-tile segment lists, sorted by level (pass l collects level l) ----
-#pragma unroll 1
-    for (int t = 0; t < 2; ++t) {
-      int n = 0, cols = 0;
-      const int qbA = (qtile0 + t) * QH;
-      const int qbB = qbA + QH - 1;
-      const bool validA = qbA < p.nb && t != skip_t, validB = qbB < p.nb && t != skip_t;
-      if (lane == 0) {
-        misc[8 + 2 * t] = -1;
-        misc[9 + 2 * t] = -1;
+  if (warp == 0 || warp == 3) {
+    // ---- the segment list of q-tile t (warp 0: t = 0, warp 3: t = 1) ----
+    // Segments are sorted by group: by level (lengths non-increasing, so they
+    // fill 128-key tiles exactly) and, within a level, by row mask: used by
+    // both q-blocks, by the first only, by the second only (block 128: one
+    // group per level); ascending j within a group.  A key tile whose
+    // segments all share a group and hold full pooled groups needs no
+    // per-column bias (uniform).  Two passes over j: count the segments of
+    // each group, then place each one at its group's offset plus its rank.
+    const int t = warp == 0 ? 0 : 1;
+    constexpr int NR = QH == 2 ? 3 : 1;   // row-mask groups per level
+    constexpr int NG = 4 * NR;
+    // The level codes of the two q-blocks (after the causal adjustment) and
+    // the per-group running offsets are staged in the V ring, unused until
+    // the main loop.
+    uint8_t* cd = smem + L::kOffV + t * 2 * kPyrMaxBlocks;
+    int* gpos = reinterpret_cast<int*>(smem + L::kOffV + 4 * kPyrMaxBlocks + t * 128);
+    int* gcol = gpos + 16;
+    const int qbA = (qtile0 + t) * QH;
+    const int qbB = qbA + QH - 1;
+    const bool validA = qbA < p.nb && t != skip_t, validB = qbB < p.nb && t != skip_t;
+    for (int j = lane; j < p.nb; j += 32) {
+      const long long rowoff = b * p.lsb + h * p.lsh + j;
+      int cA = validA ? p.levels[rowoff + qbA * p.lsi] : 0;
+      int cB = validB ? p.levels[rowoff + qbB * p.lsi] : 0;
+      if (CAUSAL) {
+        // blocks after the q-block are dropped; its own block, if kept, is
+        // attended at level 0 (its pooled keys would mix in later tokens)
+        cA = j > qbA ? 0 : (j == qbA && cA ? 1 : cA);
+        cB = j > qbB ? 0 : (j == qbB && cB ? 1 : cB);
       }
-      __syncwarp();
-#pragma unroll 1
-      for (int lvl = 0; lvl < 4; ++lvl) {
-        for (int base = 0; base < p.nb; base += 32) {
-          const int j = base + lane;
-          uint32_t rm = 0;
-          if (j < p.nb) {
-            const long long rowoff = b * p.lsb + h * p.lsh + j;
-            int cA = validA ? p.levels[rowoff + qbA * p.lsi] : 0;
-            int cB = validB ? p.levels[rowoff + qbB * p.lsi] : 0;
-            if (p.causal) {
-              // blocks after the q-block are dropped; its own block, if kept, is
-              // attended at level 0 (its pooled keys would mix in later tokens)
-              cA = j > qbA ? 0 : (j == qbA && cA ? 1 : cA);
-              cB = j > qbB ? 0 : (j == qbB && cB ? 1 : cB);
-            }
-            rm = (cA == lvl + 1 ? 1u : 0u) | (cB == lvl + 1 ? 2u : 0u);
-          }
-          const unsigned ball = __ballot_sync(0xffffffffu, rm != 0);
-          if (rm) {
-            // segments of one level have one length, so the packed column
-            // (and with it the key tile) follows from the rank
-            const int rank = __popc(ball & ((1u << lane) - 1u));
-            const int cg = cols + rank * (BLK >> lvl);
-            segs[t * kPyrMaxSegs + n + rank] = static_cast<uint32_t>(j) | (static_cast<uint32_t>(lvl) << 16) |
-                                               (rm << 18) | (static_cast<uint32_t>(cg & (kTileN - 1)) << 24);
-            if ((cg & (kTileN - 1)) == 0) ents[t * kPyrMaxEntries + cg / kTileN] = static_cast<uint16_t>(n + rank);
-            if (p.causal && lvl == 0) {
-              const int where = (cg / kTileN) * 256 + (cg & (kTileN - 1));
-              if ((rm & 1u) && j == qbA) misc[8 + 2 * t] = where;
-              if ((rm & 2u) && j == qbB) misc[9 + 2 * t] = where;
-            }
-          }
-          n += __popc(ball);
-          cols += __popc(ball) * (BLK >> lvl);
-        }
+      cd[j] = static_cast<uint8_t>(cA);
+      cd[kPyrMaxBlocks + j] = static_cast<uint8_t>(cB);
+    }
+    __syncwarp();
+    // group of each of a block's (at most two) segments, -1 for none
+    auto groups_of = [&](int j, int& gA, int& gB) {
+      gA = -1;
+      gB = -1;
+      if (j >= p.nb) return;
+      const int cA = cd[j], cB = cd[kPyrMaxBlocks + j];
+      if (QH == 1 || cA == cB) {
+        if (cA) gA = (cA - 1) * NR;
+      } else {
+        if (cA) gA = (cA - 1) * NR + 1;
+        if (cB) gB = (cB - 1) * NR + 2;
       }
-      if (lane == 0) {
-        misc[1 + t] = n;
-        misc[3 + t] = (cols + kTileN - 1) / kTileN;
-        misc[6 + t] = cols;
+    };
+    // pass 1: segments per group, as 16-bit fields of three 64-bit words
+    unsigned long long cw[3] = {0ull, 0ull, 0ull};
+    for (int base = 0; base < p.nb; base += 32) {
+      int gA, gB;
+      groups_of(base + lane, gA, gB);
+#pragma unroll
+      for (int w = 0; w < 3; ++w) {
+        if (gA >= 0 && (gA >> 2) == w) cw[w] += 1ull << (16 * (gA & 3));
+        if (gB >= 0 && (gB >> 2) == w) cw[w] += 1ull << (16 * (gB & 3));
       }
     }
+#pragma unroll
+    for (int w = 0; w < 3; ++w)
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) cw[w] += __shfl_xor_sync(0xffffffffu, cw[w], o);
+    int n = 0, cols = 0;
+#pragma unroll
+    for (int g = 0; g < NG; ++g) {
+      const int c = static_cast<int>((cw[g >> 2] >> (16 * (g & 3))) & 0xFFFFull);
+      if (lane == g) {
+        gpos[g] = n;
+        gcol[g] = cols;
+      }
+      n += c;
+      cols += c * (BLK >> (g / NR));
+    }
     if (lane == 0) {
+      misc[8 + 2 * t] = -1;
+      misc[9 + 2 * t] = -1;
+      misc[12 + 2 * t] = -1;
+      misc[13 + 2 * t] = -1;
+    }
+    __syncwarp();
+    // pass 2: each segment at its group's running offset plus its rank among
+    // the chunk's lanes of the same group (lanes hold ascending j)
+    for (int base = 0; base < p.nb; base += 32) {
+      const int j = base + lane;
+      int gA, gB;
+      groups_of(j, gA, gB);
+#pragma unroll
+      for (int x = 0; x < 2; ++x) {
+        const int g = x == 0 ? gA : gB;
+        const unsigned peers = __match_any_sync(0xffffffffu, g);
+        const int rank = __popc(peers & ((1u << lane) - 1u));
+        if (g >= 0) {
+          const int lvl = g / NR;
+          const uint32_t rm = NR == 1 ? 3u : (g % NR == 0 ? 3u : static_cast<uint32_t>(g % NR));
+          const int pos = gpos[g] + rank;
+          const int cg = gcol[g] + rank * (BLK >> lvl);
+          segs[t * kPyrMaxSegs + pos] = static_cast<uint32_t>(j) | (static_cast<uint32_t>(lvl) << 16) | (rm << 18) |
+                                        (static_cast<uint32_t>(cg & (kTileN - 1)) << 24);
+          if ((cg & (kTileN - 1)) == 0) ents[t * kPyrMaxEntries + cg / kTileN] = static_cast<uint16_t>(pos);
+          if (CAUSAL && lvl == 0) {
+            const int where = (cg / kTileN) * 256 + (cg & (kTileN - 1));
+            if ((rm & 1u) && j == qbA) misc[8 + 2 * t] = where;
+            if ((rm & 2u) && j == qbB) misc[9 + 2 * t] = where;
+          }
+          if (j == p.nb - 1) misc[12 + 2 * t + x] = cg / kTileN;   // a tile holding a segment of the last block
+        }
+        __syncwarp();
+        if (g >= 0 && rank == 0) {
+          gpos[g] += __popc(peers);
+          gcol[g] += __popc(peers) * (BLK >> (g / NR));
+        }
+        __syncwarp();
+      }
+    }
+    // key-tile descriptors, packed above the first-segment index (11 bits):
+    // bit 11 uniform, bits 12-13 level, bits 14-15 row mask
+    const bool last_partial = p.N - (p.nb - 1) * BLK < BLK;
+    const int part0 = misc[12 + 2 * t], part1 = misc[13 + 2 * t];
+    const int nt = (cols + kTileN - 1) / kTileN;
+    for (int k = lane; k < nt; k += 32) {
+      // (the start bits are masked: a neighbour lane may already have added
+      // the descriptor bits of tile k + 1)
+      const int s0 = ents[t * kPyrMaxEntries + k] & kEntStartMask;
+      const int s1 = (k + 1 < nt ? (ents[t * kPyrMaxEntries + k + 1] & kEntStartMask) : n) - 1;
+      const uint32_t g0 = (segs[t * kPyrMaxSegs + s0] >> 16) & 15u;
+      const uint32_t g1 = (segs[t * kPyrMaxSegs + s1] >> 16) & 15u;
+      const bool full = (k + 1) * kTileN <= cols;
+      const bool uni = g0 == g1 && full && !(last_partial && (k == part0 || k == part1));
+      ents[t * kPyrMaxEntries + k] = static_cast<uint16_t>(s0 | (uni ? kEntUniform : 0u) | (g0 << 12));
+    }
+    if (lane == 0) {
+      misc[1 + t] = n;
+      misc[3 + t] = nt;
+      misc[6 + t] = cols;
+    }
+    if (warp == 0 && lane == 0) {
       misc[5] = 0;
       for (int i = 0; i < L::kNumBars; ++i)   // k_full: the K loads' arrival and the KX writes' arrival
         mbar_init(&bars[i], (&bars[i] == &k_full[0] || &bars[i] == &k_full[1]) ? 2u : 1u);
@@ -205,11 +292,11 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
   } else if (warp == 1) {
     tmem_alloc(const_cast<uint32_t*>(reinterpret_cast<volatile uint32_t*>(misc)), 512);
     tmem_relinquish();
-  } else if (warp == 2 || warp == 3) {
-    // QX: q rows of the tile's first q-block select columns 0-1, of its second
-    // 2-3 (block 128: every row 0-1); the KX columns 8-15 of both slots are 0
-    const int i0 = (warp - 2) * 32 + lane;
-    for (int i = i0; i < 128; i += 64) {
+  } else {
+    // QX (warp 2): q rows of the tile's first q-block select columns 0-1, of
+    // its second 2-3 (block 128: every row 0-1); the KX columns 8-15 of both
+    // slots are 0
+    for (int i = lane; i < 128; i += 32) {
       const bool second = QH == 2 && i >= 64;
       uint4 w;
       w.x = second ? 0u : 0x3F803F80u;   // bf16 1.0 in columns 0 and 1
@@ -223,7 +310,7 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
     }
     // KX row patterns of full groups: index 4 * level + useA + 2 * useB, and
     // 16 for a column that holds no key
-    if (warp == 2 && lane < 17) {
+    if (lane < 17) {
       const float inv_sl2 = 1.f / p.scale_log2;
       const int lv = lane >> 2;
       const bool useA = lane < 16 && (lane & 1), useB = lane < 16 && (lane & 2);
@@ -272,8 +359,8 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
     };
     auto seg_of = [&](int t, int k) -> Seg {   // segments of key tile k of q-tile t
       const int nt = t == 0 ? ntile0 : ntile1;
-      const int start = ents[t * kPyrMaxEntries + k];
-      const int end = k + 1 < nt ? ents[t * kPyrMaxEntries + k + 1] : misc[1 + t];
+      const int start = ents[t * kPyrMaxEntries + k] & kEntStartMask;
+      const int end = k + 1 < nt ? (ents[t * kPyrMaxEntries + k + 1] & kEntStartMask) : misc[1 + t];
       Seg g;
       g.fill = k + 1 < nt ? kTileN : misc[6 + t] - kTileN * k;
       g.mine = lane < end - start;
@@ -416,9 +503,10 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
           zero_rows(kst, g.fill, kTileN);
           issue(g, maps.k, &k_full[s], kst, 0, kTileN);
           k_issued = e + 1;
-          // KX is written while the K segments are in flight; its arrival is
-          // the second of the k_full phase (made visible to the MMA by it)
-          write_kx(g, kx + s * 4096);
+          // KX is written while the K segments are in flight (mixed tiles
+          // only: a uniform tile's bias is added by the softmax); its arrival
+          // is the second of the k_full phase (made visible to the MMA by it)
+          if (!(ents[t * kPyrMaxEntries + k] & kEntUniform)) write_kx(g, kx + s * 4096);
           if (lane == 0) mbar_arrive(&k_full[s]);
         }
         if (!ok && lane == 0) misc[5] = 1;
@@ -465,8 +553,10 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
               const uint64_t off = static_cast<uint64_t>((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
               mma_ss_warp(tmem, dq + off, dk + off, kIdescS, kk > 0 ? 1u : 0u);
             }
-            // + the bias: selector columns of the row's q-block times its hi + lo parts
-            mma_ss_warp(tmem, dqx, dkx0 + s * (4096 >> 4), kIdescS, 1u);
+            // + the bias of a mixed tile: selector columns of the row's q-block
+            // times its hi + lo parts
+            if (!(ents[t * kPyrMaxEntries + k] & kEntUniform))
+              mma_ss_warp(tmem, dqx, dkx0 + s * (4096 >> 4), kIdescS, 1u);
           }
           // committed also after an error, so that the softmax keeps its place
           mma_commit_warp(&s_ready[t]);
@@ -580,56 +670,28 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
     const float NEG_INF = -__int_as_float(0x7f800000);
     // causal: where this row's own block sits in the packed key tiles
     const int xq = (BLK == 64) ? (r >> 6) : 0;
-    const int diag = p.causal ? misc[8 + 2 * t + xq] : -1;
+    const int diag = CAUSAL ? misc[8 + 2 * t + xq] : -1;
     const int r_in_blk = r & (BLK - 1);
 
+    const float inv_sl2 = 1.f / sl2;
     float m_used = NEG_INF, l_sum = 0.f;
-    int et = 0;   // entries of this q-tile processed
+    int et = 0;            // entries of this q-tile processed
+    bool p_zero = false;   // this warp's rows of P_t hold zeros (the last entry skipped them)
     bool ok = true;
     if (cnt > 0) {
       for (int e = 0; e < n_entries; ++e) {
         int te, k;
         entry_of(e, te, k);
         if (te != t) continue;
-        const int st = e % kStages;
-        // After an error the loop still runs to the end (its hand-offs keep
-        // the issuing warps' sequences in step); it only stops trusting TMEM.
-        if (!mbar_wait(&s_ready[t], et & 1)) {
-          misc[5] = 1;
-          ok = false;
-        }
-        tc_fence_after();
-        float s[kTileN];
-        tmem_ld128(s_addr, s);
-        // the S buffer is free for the next entry's S
-        tc_fence_before();
-        named_bar_sync(kBarSFree + t, kHandoff);
-        if (diag >= 0 && (diag >> 8) == k) {
-          // causal: the diagonal segment's key x (from the block start) is
-          // visible to the row only if x <= the row's position in its block
-          const int c0 = diag & 255;
-#pragma unroll
-          for (int c = 0; c < kTileN; ++c)
-            if (c >= c0 && c < c0 + BLK && c - c0 > r_in_blk) s[c] = NEG_INF;
-        }
-        // s already carries the bias (raw logit units): q.k + log2(count) / (scale log2 e),
-        // and about -30000 on masked and empty columns
-        float a[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) a[u] = fmaxf(s[2 * u], s[2 * u + 1]);
-#pragma unroll
-        for (int c = 16; c < kTileN; c += 16) {
-#pragma unroll
-          for (int u = 0; u < 8; ++u) a[u] = fmax3(a[u], s[c + 2 * u], s[c + 2 * u + 1]);
-        }
-        float mx = fmaxf(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], fmax3(a[5], a[6], a[7])));
-        if (mx < kMaskedCut) mx = NEG_INF;   // no valid column for this row in this tile
-        float factor = 1.f;
-        if (mx > m_used && (m_used == NEG_INF || (mx - m_used) * sl2 > 8.f)) {
-          factor = (m_used == NEG_INF) ? 0.f : fast_exp2((m_used - mx) * sl2);
-          m_used = mx;
-          l_sum *= factor;
-        }
+        // A uniform tile (same level and row mask throughout, full groups):
+        // its bias is one constant, lv in log2 units (lv * inv_sl2 in raw
+        // logit units), added here instead of by the bias MMA, and the rows
+        // of a q-block that does not use the tile skip it (their P is zero).
+        const uint32_t ed = ents[t * kPyrMaxEntries + k];
+        const bool uni = (ed & kEntUniform) != 0;
+        const int lv = static_cast<int>((ed >> 12) & 3u);
+        const uint32_t erm = (ed >> 14) & 3u;
+        const bool use = !uni || QH == 1 || ((erm >> xq) & 1u);
         // The previous PV of this tile reads P_t and accumulates into O_t: each
         // half of P_t is rewritten once that half of the PV has completed, and
         // O_t is rescaled once all of it has.
@@ -642,6 +704,73 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
             tc_fence_after();
           }
         };
+        if (!use) {
+          // these rows' P stays zero: written once, then left alone (the PV
+          // of a later entry reads it again)
+          named_bar_sync(kBarSFree + t, kHandoff);
+          uint32_t zk[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) zk[i] = 0u;
+          if (!p_zero) wait_pv(&pv_done_a[t]);
+          if (!p_zero) {
+            tmem_st32(p_addr, reinterpret_cast<const float*>(zk));
+            tmem_st_wait();
+          }
+          tc_fence_before();
+          named_bar_sync(kBarPA + t, kHandoff);
+          if (!p_zero) {
+            wait_pv(&pv_done_b[t]);
+            tmem_st32(p_addr + 32, reinterpret_cast<const float*>(zk));
+            tmem_st_wait();
+          }
+          tc_fence_before();
+          named_bar_sync(kBarPB + t, kHandoff);
+          p_zero = true;
+          ++et;
+          continue;
+        }
+        // After an error the loop still runs to the end (its hand-offs keep
+        // the issuing warps' sequences in step); it only stops trusting TMEM.
+        if (!mbar_wait(&s_ready[t], et & 1)) {
+          misc[5] = 1;
+          ok = false;
+        }
+        tc_fence_after();
+        float s[kTileN];
+        tmem_ld128(s_addr, s);
+        // the S buffer is free for the next entry's S
+        tc_fence_before();
+        named_bar_sync(kBarSFree + t, kHandoff);
+        if (CAUSAL && diag >= 0 && (diag >> 8) == k) {
+          // causal: the diagonal segment's key x (from the block start) is
+          // visible to the row only if x <= the row's position in its block
+          const int c0 = diag & 255;
+#pragma unroll
+          for (int c = 0; c < kTileN; ++c)
+            if (c >= c0 && c < c0 + BLK && c - c0 > r_in_blk) s[c] = NEG_INF;
+        }
+        // a mixed tile's s already carries the bias (raw logit units): q.k +
+        // log2(count) / (scale log2 e), and about -30000 on masked and empty
+        // columns; a uniform tile's bias is lv * inv_sl2 on every column
+        float a[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) a[u] = fmaxf(s[2 * u], s[2 * u + 1]);
+#pragma unroll
+        for (int c = 16; c < kTileN; c += 16) {
+#pragma unroll
+          for (int u = 0; u < 8; ++u) a[u] = fmax3(a[u], s[c + 2 * u], s[c + 2 * u + 1]);
+        }
+        float mx = fmaxf(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], fmax3(a[5], a[6], a[7])));
+        if (uni)
+          mx += static_cast<float>(lv) * inv_sl2;
+        else if (mx < kMaskedCut)
+          mx = NEG_INF;   // no valid column for this row in this tile
+        float factor = 1.f;
+        if (mx > m_used && (m_used == NEG_INF || (mx - m_used) * sl2 > 8.f)) {
+          factor = (m_used == NEG_INF) ? 0.f : fast_exp2((m_used - mx) * sl2);
+          m_used = mx;
+          l_sum *= factor;
+        }
         const bool rescale = et > 0 && __any_sync(0xffffffffu, factor != 1.f);
         if (rescale) {
           wait_pv(&pv_done_b[t]);
@@ -655,7 +784,8 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
           }
           tmem_st_wait();
         }
-        const float neg_m = (m_used == NEG_INF) ? 0.f : -m_used * sl2;
+        // x = s sl2 + (uniform: lv) - m sl2
+        const float neg_m = (m_used == NEG_INF) ? 0.f : (uni ? static_cast<float>(lv) : 0.f) - m_used * sl2;
         {
           uint32_t pk[32];
           l_sum += exp_pack_64(s, sl2, neg_m, pk);
@@ -674,6 +804,7 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
           tc_fence_before();
           named_bar_sync(kBarPB + t, kHandoff);
         }
+        p_zero = false;
         ++et;
       }
     }
