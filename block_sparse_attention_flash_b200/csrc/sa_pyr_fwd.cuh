@@ -676,7 +676,6 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
     const float inv_sl2 = 1.f / sl2;
     float m_used = NEG_INF, l_sum = 0.f;
     int et = 0;            // entries of this q-tile processed
-    bool p_zero = false;   // this warp's rows of P_t hold zeros (the last entry skipped them)
     bool ok = true;
     if (cnt > 0) {
       for (int e = 0; e < n_entries; ++e) {
@@ -684,14 +683,13 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
         entry_of(e, te, k);
         if (te != t) continue;
         // A uniform tile (same level and row mask throughout, full groups):
-        // its bias is one constant, lv in log2 units (lv * inv_sl2 in raw
-        // logit units), added here instead of by the bias MMA, and the rows
-        // of a q-block that does not use the tile skip it (their P is zero).
+        // its bias is one constant, ln(2^l) (l * inv_sl2 in raw logit units),
+        // added here instead of by the bias MMA, and the rows of a q-block
+        // that does not use the tile skip it (their P is zero).
         const uint32_t ed = ents[t * kPyrMaxEntries + k];
-        const bool uni = (ed & kEntUniform) != 0;
-        const int lv = static_cast<int>((ed >> 12) & 3u);
-        const uint32_t erm = (ed >> 14) & 3u;
-        const bool use = !uni || QH == 1 || ((erm >> xq) & 1u);
+        const bool use = !(ed & kEntUniform) || QH == 1 || ((ed >> (14 + xq)) & 1u);
+        // the tile's bias in raw logit units (0 for a mixed tile, whose S carries it)
+        const float bias = (ed & kEntUniform) ? static_cast<float>((ed >> 12) & 3u) * inv_sl2 : 0.f;
         // The previous PV of this tile reads P_t and accumulates into O_t: each
         // half of P_t is rewritten once that half of the PV has completed, and
         // O_t is rescaled once all of it has.
@@ -705,27 +703,22 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
           }
         };
         if (!use) {
-          // these rows' P stays zero: written once, then left alone (the PV
-          // of a later entry reads it again)
+          // these rows' P is zero (no S load, no exponentials); the hand-offs
+          // run as for any entry
           named_bar_sync(kBarSFree + t, kHandoff);
           uint32_t zk[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) zk[i] = 0u;
-          if (!p_zero) wait_pv(&pv_done_a[t]);
-          if (!p_zero) {
-            tmem_st32(p_addr, reinterpret_cast<const float*>(zk));
-            tmem_st_wait();
-          }
+          wait_pv(&pv_done_a[t]);
+          tmem_st32(p_addr, reinterpret_cast<const float*>(zk));
+          tmem_st_wait();
           tc_fence_before();
           named_bar_sync(kBarPA + t, kHandoff);
-          if (!p_zero) {
-            wait_pv(&pv_done_b[t]);
-            tmem_st32(p_addr + 32, reinterpret_cast<const float*>(zk));
-            tmem_st_wait();
-          }
+          wait_pv(&pv_done_b[t]);
+          tmem_st32(p_addr + 32, reinterpret_cast<const float*>(zk));
+          tmem_st_wait();
           tc_fence_before();
           named_bar_sync(kBarPB + t, kHandoff);
-          p_zero = true;
           ++et;
           continue;
         }
@@ -751,7 +744,8 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
         }
         // a mixed tile's s already carries the bias (raw logit units): q.k +
         // log2(count) / (scale log2 e), and about -30000 on masked and empty
-        // columns; a uniform tile's bias is lv * inv_sl2 on every column
+        // columns; a uniform tile's bias is `bias` on every column (and its
+        // row maximum is a real logit, never below the cut)
         float a[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) a[u] = fmaxf(s[2 * u], s[2 * u + 1]);
@@ -761,10 +755,7 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
           for (int u = 0; u < 8; ++u) a[u] = fmax3(a[u], s[c + 2 * u], s[c + 2 * u + 1]);
         }
         float mx = fmaxf(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], fmax3(a[5], a[6], a[7])));
-        if (uni)
-          mx += static_cast<float>(lv) * inv_sl2;
-        else if (mx < kMaskedCut)
-          mx = NEG_INF;   // no valid column for this row in this tile
+        mx = mx < kMaskedCut ? NEG_INF : mx + bias;   // -inf: no valid column for this row in this tile
         float factor = 1.f;
         if (mx > m_used && (m_used == NEG_INF || (mx - m_used) * sl2 > 8.f)) {
           factor = (m_used == NEG_INF) ? 0.f : fast_exp2((m_used - mx) * sl2);
@@ -784,8 +775,8 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
           }
           tmem_st_wait();
         }
-        // x = s sl2 + (uniform: lv) - m sl2
-        const float neg_m = (m_used == NEG_INF) ? 0.f : (uni ? static_cast<float>(lv) : 0.f) - m_used * sl2;
+        // x = (s + bias - m) sl2
+        const float neg_m = (m_used == NEG_INF) ? 0.f : (bias - m_used) * sl2;
         {
           uint32_t pk[32];
           l_sum += exp_pack_64(s, sl2, neg_m, pk);
@@ -804,7 +795,6 @@ __global__ void __launch_bounds__(kPyrThreads, 1)
           tc_fence_before();
           named_bar_sync(kBarPB + t, kHandoff);
         }
-        p_zero = false;
         ++et;
       }
     }
