@@ -124,6 +124,22 @@ def replica_seed(base_seed, rank):
     return base_seed + 1 + 1000 * rank
 
 
+def replica_chain(wl, rank, nsteps, device, H=None):
+    """The denoising inputs of one replica: the workload's step-0 draw (the same
+    on every rank) and nsteps - 1 drift steps whose noise comes from the
+    rank's own seed, so the replicas run different chains."""
+    from block_sparse_attention_flash_b200 import inputs
+
+    q0, k0, v0 = inputs.rff_qkv(wl, H=H, device=device)
+    g = torch.Generator(device=device)
+    g.manual_seed(replica_seed(wl.seed, rank))
+    qkv = [(q0, k0, v0)]
+    for _ in range(1, nsteps):
+        q, k, v = qkv[-1]
+        qkv.append((inputs.drift(q, g), inputs.drift(k, g), inputs.drift(v, g)))
+    return qkv
+
+
 def reduce_over_ranks(total_ms, work, world, device):
     """(max over ranks of the timed region, sum over ranks of the work done).
 
@@ -178,13 +194,8 @@ def run_ours(args, rank, world, local):
     nsteps = args.warmup + args.steps
 
     # Per-step inputs, drawn on the device before timing (the chain's drift).
-    q0, k0, v0 = inputs.rff_qkv(wl, device=dev)
-    g = torch.Generator(device=dev)
-    g.manual_seed(replica_seed(wl.seed, rank))
-    qkv = [(q0, k0, v0)]
-    for s in range(1, nsteps):
-        q, k, v = qkv[-1]
-        qkv.append((inputs.drift(q, g), inputs.drift(k, g), inputs.drift(v, g)))
+    qkv = replica_chain(wl, rank, nsteps, dev)
+    q0, k0, v0 = qkv[0]
     skips = [torch.zeros(B, H, nb, nb, dtype=torch.uint8, device=dev) for _ in range(nsteps + 1)]
     out = torch.empty_like(q0)
     stream = torch.cuda.current_stream(dev)
@@ -219,7 +230,6 @@ def run_ours(args, rank, world, local):
     total_ms = t0.elapsed_time(t1)
     kern_ms = [ev[s][0].elapsed_time(ev[s][1]) for s in range(args.warmup, nsteps)]
     flops = [executed_flops(skips[s], N, block, d) for s in range(args.warmup, nsteps)]
-    dense = 4.0 * d * N * N * B * H
     total_ms_max, flops_all = reduce_over_ranks(total_ms, sum(flops), world, dev)
 
     # end-to-end through the public API with host buffers, over the same drifted steps
@@ -245,18 +255,29 @@ def run_ours(args, rank, world, local):
 
     if rank != 0:
         return None
+    line = assemble_line(wl, world, args.steps, args.warmup, total_ms_max, flops_all, kern_ms, flops)
+    line.update({"clocks": clk, "e2e": e2e, "cpu_baseline": cpu, "configs": configs})
+    return line
+
+
+def assemble_line(wl, world, steps, warmup, total_ms_max, flops_all, kern_ms, flops):
+    """The JSON line of the device-timed run (rank 0): the whole-job value is
+    the work summed over ranks divided by the slowest rank's timed region;
+    the per-call figures and the roofline are rank 0's own launches."""
+    B, H, N, d = wl.B, wl.H, wl.N, wl.d
+    dense = 4.0 * d * N * N * B * H
     peaks, src = load_peaks()
     achieved = sum(flops) / (sum(kern_ms) * 1e-3) / 1e12
     peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
     skip_rate = 1.0 - sum(flops) / (dense * len(flops))
-    line = {
+    return {
         "metric": METRIC,
         "value": round(whole_job_tflops(flops_all, total_ms_max), 2),
         "unit": "TFLOP/s",
         "n_gpus": world,
-        "steps": args.steps,
-        "warmup": args.warmup,
-        "ms_per_step": round(total_ms_max / args.steps, 3),
+        "steps": steps,
+        "warmup": warmup,
+        "ms_per_step": round(total_ms_max / steps, 3),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -272,13 +293,8 @@ def run_ours(args, rank, world, local):
                      "frac_of_burst": round(achieved / float(peaks["bf16_tflops"]), 4),
                      "traffic": ATTN_DRAM_BYTES_PER_LAUNCH, "traffic_unit": "bytes per launch",
                      "algorithmic_bytes": 4 * B * H * N * d * 2},
-        "gpu_launches": args.steps,
-        "clocks": clk,
-        "e2e": e2e,
-        "cpu_baseline": cpu,
-        "configs": configs,
+        "gpu_launches": steps,
     }
-    return line
 
 
 E2E_HEADS_PER_CHUNK = 2   # measured: 2 heads 98.2 ms per step, 4 heads 100.5, 8 heads 105
