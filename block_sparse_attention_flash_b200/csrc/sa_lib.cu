@@ -294,17 +294,17 @@ sa_status sa_build_mask(const void* q, const void* k, int B, int H, int N, int d
     return cuda_status(cudaGetLastError());
   }
   if (nb <= 32)
-    sa::block_select_warp_kernel<1><<<warp_grid, 128, 0, s>>>(scores, nb, nrows, mode, tau, c0, c1, c2, mask_out);
+    sa::level_select_warp_kernel<1><<<warp_grid, 128, 0, s>>>(scores, nb, nrows, c0, c1, c2, mask_out);
   else if (nb <= 64)
-    sa::block_select_warp_kernel<2><<<warp_grid, 128, 0, s>>>(scores, nb, nrows, mode, tau, c0, c1, c2, mask_out);
+    sa::level_select_warp_kernel<2><<<warp_grid, 128, 0, s>>>(scores, nb, nrows, c0, c1, c2, mask_out);
   else if (nb <= 128)
-    sa::block_select_warp_kernel<4><<<warp_grid, 128, 0, s>>>(scores, nb, nrows, mode, tau, c0, c1, c2, mask_out);
+    sa::level_select_warp_kernel<4><<<warp_grid, 128, 0, s>>>(scores, nb, nrows, c0, c1, c2, mask_out);
   else if (nb <= 256)
-    sa::block_select_warp_kernel<8><<<warp_grid, 128, 0, s>>>(scores, nb, nrows, mode, tau, c0, c1, c2, mask_out);
+    sa::level_select_warp_kernel<8><<<warp_grid, 128, 0, s>>>(scores, nb, nrows, c0, c1, c2, mask_out);
   else if (nb <= 512)
-    sa::block_select_warp_kernel<16><<<warp_grid, 128, 0, s>>>(scores, nb, nrows, mode, tau, c0, c1, c2, mask_out);
+    sa::level_select_warp_kernel<16><<<warp_grid, 128, 0, s>>>(scores, nb, nrows, c0, c1, c2, mask_out);
   else if (nb <= 1024)
-    sa::block_select_warp_kernel<32><<<warp_grid, 128, 0, s>>>(scores, nb, nrows, mode, tau, c0, c1, c2, mask_out);
+    sa::level_select_warp_kernel<32><<<warp_grid, 128, 0, s>>>(scores, nb, nrows, c0, c1, c2, mask_out);
   else
     sa::block_select_kernel<<<static_cast<unsigned>(nrows), sa::kSelectThreads, sa::select_smem_bytes(nb), s>>>(
         scores, nb, mode, tau, c0, c1, c2, mask_out);

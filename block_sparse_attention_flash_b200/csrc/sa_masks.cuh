@@ -105,11 +105,17 @@ __global__ void __launch_bounds__(128) block_means_kernel(const __nv_bfloat16* _
 // ----------------------------------------------------------- block scores ---
 // grid (ceil(nb/64), ceil(nb/64), B*H), 256 threads; each thread owns a 4 x 4
 // patch of a 64 x 64 tile of S = scale * Qbar Kbar^T, fp32 throughout.  The
-// d dimension is walked in chunks of 32 staged (transposed) in shared memory.
+// d dimension is walked in chunks of 32 staged transposed in shared memory:
+// element (row r, column k of the chunk) sits at [k][r ^ sw(k)], where the
+// XOR sw(k) = 4 * ((k / 4) % 8) permutes whole groups of four rows.  The
+// transposed stores of a warp then fall in 32 distinct banks, and a thread
+// still reads its four rows of one column as one aligned float4.  At most 42
+// registers a thread let six CTAs share an SM, so the 768 tiles of 12 heads
+// of 512 blocks run as one wave on 148 SMs.
 template <int D>
-__global__ void __launch_bounds__(256) block_scores_kernel(const float* __restrict__ qmean,
-                                                           const float* __restrict__ kmean, int nb, float scale,
-                                                           float* __restrict__ scores) {
+__global__ void __launch_bounds__(256, 6) block_scores_kernel(const float* __restrict__ qmean,
+                                                              const float* __restrict__ kmean, int nb, float scale,
+                                                              float* __restrict__ scores) {
   __shared__ __align__(16) float sa[32][68];
   __shared__ __align__(16) float sb[32][68];
   const int bh = blockIdx.z;
@@ -117,41 +123,33 @@ __global__ void __launch_bounds__(256) block_scores_kernel(const float* __restri
   const float* qm = qmean + static_cast<size_t>(bh) * nb * D;
   const float* km = kmean + static_cast<size_t>(bh) * nb * D;
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  auto sw = [](int k) { return ((k >> 2) & 7) << 2; };
   float acc[4][4];
 #pragma unroll
   for (int a = 0; a < 4; ++a)
 #pragma unroll
     for (int c = 0; c < 4; ++c) acc[a][c] = 0.f;
-  // the next chunk's operands are loaded into registers while this chunk is
-  // multiplied (512 float4 per operand chunk, two per thread)
-  float4 pa[2], pb[2];
-  auto fetch = [&](int kc) {
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int idx = threadIdx.x + u * 256;
-      const int rr = idx >> 3, c4 = (idx & 7) * 4;
-      pa[u] = (i0 + rr < nb) ? *reinterpret_cast<const float4*>(qm + static_cast<size_t>(i0 + rr) * D + kc + c4)
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
-      pb[u] = (j0 + rr < nb) ? *reinterpret_cast<const float4*>(km + static_cast<size_t>(j0 + rr) * D + kc + c4)
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-  };
-  fetch(0);
 #pragma unroll 1
   for (int kc = 0; kc < D; kc += 32) {
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
       const int idx = threadIdx.x + u * 256;
-      const int rr = idx >> 3, c4 = (idx & 7) * 4;
-      sa[c4 + 0][rr] = pa[u].x; sa[c4 + 1][rr] = pa[u].y; sa[c4 + 2][rr] = pa[u].z; sa[c4 + 3][rr] = pa[u].w;
-      sb[c4 + 0][rr] = pb[u].x; sb[c4 + 1][rr] = pb[u].y; sb[c4 + 2][rr] = pb[u].z; sb[c4 + 3][rr] = pb[u].w;
+      const int rr = idx >> 3, c4 = (idx & 7) * 4;   // 8 lanes read one row's 32 columns
+      const float4 pa = (i0 + rr < nb)
+                            ? *reinterpret_cast<const float4*>(qm + static_cast<size_t>(i0 + rr) * D + kc + c4)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4 pb = (j0 + rr < nb)
+                            ? *reinterpret_cast<const float4*>(km + static_cast<size_t>(j0 + rr) * D + kc + c4)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+      const int col = rr ^ sw(c4);   // c4 .. c4 + 3 share k / 4, so one swizzle for the four
+      sa[c4 + 0][col] = pa.x; sa[c4 + 1][col] = pa.y; sa[c4 + 2][col] = pa.z; sa[c4 + 3][col] = pa.w;
+      sb[c4 + 0][col] = pb.x; sb[c4 + 1][col] = pb.y; sb[c4 + 2][col] = pb.z; sb[c4 + 3][col] = pb.w;
     }
     __syncthreads();
-    if (kc + 32 < D) fetch(kc + 32);
 #pragma unroll 8
     for (int k = 0; k < 32; ++k) {
-      const float4 a = *reinterpret_cast<const float4*>(&sa[k][ty * 4]);
-      const float4 bq = *reinterpret_cast<const float4*>(&sb[k][tx * 4]);
+      const float4 a = *reinterpret_cast<const float4*>(&sa[k][(ty * 4) ^ sw(k)]);
+      const float4 bq = *reinterpret_cast<const float4*>(&sb[k][(tx * 4) ^ sw(k)]);
       const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {bq.x, bq.y, bq.z, bq.w};
 #pragma unroll
       for (int u = 0; u < 4; ++u)
@@ -327,132 +325,76 @@ __global__ void __launch_bounds__(kSelectThreads) block_select_kernel(const floa
   for (int j = threadIdx.x; j < nb; j += kSelectThreads) mrow[j] = out_row[j];
 }
 
-// Score row accessor: element i of a row at `base`, either plain (a row of
-// the scores array in global memory) or skewed by one word per 32 (a row
-// staged in shared memory, so that lane l reading element l*E + k hits a
-// bank of its own for every E).
-template <bool SKEW>
-__device__ __forceinline__ int score_index(int i) {
-  return SKEW ? i + (i >> 5) : i;
-}
-
-// Warp-per-row selection for rows of at most 32*E blocks (E <= 32): the keys
-// live in registers (E per lane, blocked: lane l holds ranks l*E .. l*E+E-1
-// after the sort) and the bitonic network uses in-register swaps for strides
-// below E and shuffles above.  `stage` is the warp's P-byte staging row.
-template <int E, bool SKEW>
-__device__ __forceinline__ void block_select_row(const float* srow, int nb, int mode, float tau, int c0, int c1,
-                                                 int c2, uint8_t* stage, uint8_t* __restrict__ mrow, int lane) {
-  constexpr int P = 32 * E;
-  unsigned long long key[E];
-  float mx = -__int_as_float(0x7f800000);
+// LEVELS rows without a sort (rows of at most 32*E blocks, one warp per row).
+// A block's level follows its rank r in (descending score, ascending j)
+// order: code 1 for r < c0, 2 for r < c1, 3 for r < c2, else 4.  For each
+// cut c the 32-bit score key K_c of the block of rank c - 1 is found bit by
+// bit from the most significant end: the smallest K with count(key <= K) >=
+// c (32 rounds of a warp count, the three cuts side by side).  A block is
+// below cut c if its key is below K_c, or if its key equals K_c (equal
+// scores) and fewer than c blocks precede it: those with a smaller key, then
+// the tied ones in ascending j.  Lane l holds blocks j = 32 k + l (k < E), so
+// the row is read and the codes written with coalesced accesses.
+template <int E>
+__device__ __forceinline__ void level_select_row(const float* __restrict__ srow, int nb, int c0, int c1, int c2,
+                                                 uint8_t* __restrict__ mrow, int lane) {
+  uint32_t key[E];
 #pragma unroll
   for (int k = 0; k < E; ++k) {
-    const int i = lane * E + k;
-    if (i < nb) {
-      const float sc = srow[score_index<SKEW>(i)];
-      mx = fmaxf(mx, sc);
-      key[k] = (static_cast<unsigned long long>(~float_order_key(sc)) << 32) | static_cast<unsigned>(i);
-    } else {
-      key[k] = ~0ull;
+    const int i = 32 * k + lane;
+    key[k] = i < nb ? ~float_order_key(srow[i]) : 0xFFFFFFFFu;   // ascending key = descending score
+  }
+  const uint32_t cut[3] = {static_cast<uint32_t>(max(c0, 0)), static_cast<uint32_t>(max(c1, 0)),
+                           static_cast<uint32_t>(max(c2, 0))};
+  uint32_t kst[3] = {0u, 0u, 0u};
+#pragma unroll 1
+  for (int b = 31; b >= 0; --b) {
+    const uint32_t low = (1u << b) - 1u;
+#pragma unroll
+    for (int c = 0; c < 3; ++c) {
+      const uint32_t cand = kst[c] | low;
+      uint32_t n = 0;
+#pragma unroll
+      for (int k = 0; k < E; ++k) n += (32 * k + lane < nb && key[k] <= cand) ? 1u : 0u;
+      n = __reduce_add_sync(0xffffffffu, n);
+      if (n < cut[c]) kst[c] |= 1u << b;
     }
   }
-  float inv = 0.f;
-  if (mode == SA_MASK_TAU) {
+  uint32_t less[3];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    float sum = 0.f;
+  for (int c = 0; c < 3; ++c) {
+    uint32_t n = 0;
 #pragma unroll
-    for (int k = 0; k < E; ++k) {
-      const int i = lane * E + k;
-      if (i < nb) sum += expf(srow[score_index<SKEW>(i)] - mx);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    inv = 1.f / sum;
+    for (int k = 0; k < E; ++k) n += (32 * k + lane < nb && key[k] < kst[c]) ? 1u : 0u;
+    less[c] = __reduce_add_sync(0xffffffffu, n);
   }
-  // bitonic sort, ascending keys (descending score, then ascending j)
+  uint32_t tie_before[3] = {0u, 0u, 0u};
+  const unsigned lower = (1u << lane) - 1u;
 #pragma unroll
-  for (int size = 2; size <= P; size <<= 1) {
+  for (int k = 0; k < E; ++k) {
+    const int i = 32 * k + lane;
+    uint8_t code = 1;
 #pragma unroll
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      if (stride >= E) {
-        const int lm = stride / E;
-        const bool lower = (lane & lm) == 0;
-#pragma unroll
-        for (int k = 0; k < E; ++k) {
-          const unsigned long long other = __shfl_xor_sync(0xffffffffu, key[k], lm);
-          const bool up = ((lane * E + k) & size) == 0;
-          const bool take_min = (up == lower);
-          key[k] = take_min ? (key[k] < other ? key[k] : other) : (key[k] > other ? key[k] : other);
-        }
-      } else {
-#pragma unroll
-        for (int k = 0; k < E; ++k) {
-          if ((k & stride) == 0) {
-            const int k2 = k | stride;
-            const bool up = ((lane * E + k) & size) == 0;
-            const unsigned long long a = key[k], b = key[k2];
-            if ((a > b) == up) {
-              key[k] = b;
-              key[k2] = a;
-            }
-          }
-        }
-      }
+    for (int c = 0; c < 3; ++c) {
+      const bool tied = i < nb && key[k] == kst[c];
+      const unsigned ball = __ballot_sync(0xffffffffu, tied);
+      const bool below =
+          key[k] < kst[c] || (tied && less[c] + tie_before[c] + static_cast<uint32_t>(__popc(ball & lower)) < cut[c]);
+      code += below ? 0 : 1;
+      tie_before[c] += static_cast<uint32_t>(__popc(ball));
     }
+    if (i < nb) mrow[i] = code;
   }
-  if (mode == SA_MASK_TAU) {
-    float pk[E];
-    float lsum = 0.f;
-#pragma unroll
-    for (int k = 0; k < E; ++k) {
-      const unsigned j = static_cast<unsigned>(key[k]);
-      pk[k] = key[k] != ~0ull ? expf(srow[score_index<SKEW>(static_cast<int>(j))] - mx) * inv : 0.f;
-      lsum += pk[k];
-    }
-    float inc = lsum;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const float y = __shfl_up_sync(0xffffffffu, inc, o);
-      if (lane >= o) inc += y;
-    }
-    float before = inc - lsum;
-#pragma unroll
-    for (int k = 0; k < E; ++k) {
-      if (key[k] != ~0ull) stage[static_cast<unsigned>(key[k])] = before < tau ? 1 : 0;
-      before += pk[k];
-    }
-  } else {
-#pragma unroll
-    for (int k = 0; k < E; ++k) {
-      const int r = lane * E + k;
-      if (key[k] != ~0ull)
-        stage[static_cast<unsigned>(key[k])] = r < c0 ? 1 : (r < c1 ? 2 : (r < c2 ? 3 : 4));
-    }
-  }
-  __syncwarp();
-  for (int j = lane; j < nb; j += 32) mrow[j] = stage[j];
-  __syncwarp();
 }
 
-// Four rows per 128-thread CTA, one warp each.  The row is read from global
-// memory with consecutive lanes on consecutive blocks and staged in shared
-// memory (skewed), so the blocked reads of the sort hit distinct banks.
 template <int E>
-__global__ void __launch_bounds__(128) block_select_warp_kernel(const float* __restrict__ scores, int nb,
-                                                                long long nrows, int mode, float tau, int c0,
-                                                                int c1, int c2, uint8_t* __restrict__ mask_out) {
-  constexpr int P = 32 * E;
-  __shared__ uint8_t stage[4][P];
-  __shared__ float row_s[4][P + P / 32];
+__global__ void __launch_bounds__(128) level_select_warp_kernel(const float* __restrict__ scores, int nb,
+                                                                long long nrows, int c0, int c1, int c2,
+                                                                uint8_t* __restrict__ mask_out) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long row = static_cast<long long>(blockIdx.x) * 4 + warp;
   if (row >= nrows) return;
-  const float* srow = scores + row * nb;
-  for (int i = lane; i < nb; i += 32) row_s[warp][score_index<true>(i)] = srow[i];
-  __syncwarp();
-  block_select_row<E, true>(row_s[warp], nb, mode, tau, c0, c1, c2, stage[warp], mask_out + row * nb, lane);
+  level_select_row<E>(scores + row * nb, nb, c0, c1, c2, mask_out + row * nb, lane);
 }
 
 // TAU rows without a sort (rows of at most 32*E blocks, one warp per row):
