@@ -104,6 +104,8 @@ cudaError_t init_device_kernels() {
     set(reinterpret_cast<const void*>(&sa::bwd_dq_kernel<128, 64>), sa::BwdSmem<128>::kAlloc);
     set(reinterpret_cast<const void*>(&sa::bwd_dq_kernel<64, 128>), sa::BwdSmem<64>::kAlloc);
     set(reinterpret_cast<const void*>(&sa::bwd_dq_kernel<64, 64>), sa::BwdSmem<64>::kAlloc);
+    set(reinterpret_cast<const void*>(&sa::block_scores_tc_kernel<128>), sa::kScoresTcSmem + 1024);
+    set(reinterpret_cast<const void*>(&sa::block_scores_tc_kernel<64>), sa::kScoresTcSmem + 1024);
     set(reinterpret_cast<const void*>(&sa::block_select_kernel),
         static_cast<int>(sa::select_smem_bytes(sa::kMaxSelect)));
     int dev = 0, n_sm = 0;
@@ -246,13 +248,14 @@ sa_status sa_build_mask(const void* q, const void* k, int B, int H, int N, int d
   const float scale = 1.0f / std::sqrt(static_cast<float>(d));
   const auto* qb = static_cast<const __nv_bfloat16*>(q);
   const auto* kb = static_cast<const __nv_bfloat16*>(k);
-  dim3 g1(nb, BH, 2), g2(ceil_div(nb, 64), ceil_div(nb, 64), BH);
+  dim3 g1(nb, BH, 2), g2(ceil_div(nb, 128), ceil_div(nb, 128), BH);
+  constexpr int kScoresSmem = sa::kScoresTcSmem + 1024;
   if (d == 128) {
     sa::block_means_kernel<128><<<g1, 128, 0, s>>>(qb, kb, N, block, nb, qmean, kmean);
-    sa::block_scores_kernel<128><<<g2, 256, 0, s>>>(qmean, kmean, nb, scale, scores);
+    sa::block_scores_tc_kernel<128><<<g2, 128, kScoresSmem, s>>>(qmean, kmean, nb, scale, scores);
   } else {
     sa::block_means_kernel<64><<<g1, 128, 0, s>>>(qb, kb, N, block, nb, qmean, kmean);
-    sa::block_scores_kernel<64><<<g2, 256, 0, s>>>(qmean, kmean, nb, scale, scores);
+    sa::block_scores_tc_kernel<64><<<g2, 128, kScoresSmem, s>>>(qmean, kmean, nb, scale, scores);
   }
   const long long nrows = static_cast<long long>(BH) * nb;
   const unsigned warp_grid = static_cast<unsigned>((nrows + 3) / 4);

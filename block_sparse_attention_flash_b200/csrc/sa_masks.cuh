@@ -4,8 +4,8 @@
 //                          exponential-decay mask paragraphs)
 //   block_means_kernel     mean of each token block of Q and K (VMoBA write-up,
 //                          block scoring with pooled queries/keys)
-//   block_scores_kernel    S_ij = scale * qbar_i . kbar_j (one small fp32 GEMM
-//                          per head)
+//   block_scores_tc_kernel S_ij = scale * qbar_i . kbar_j (one small GEMM per
+//                          head, fp32 accuracy from three tf32 tensor-core passes)
 //   block_select_kernel    per q-block row: tau-mass selection (VMoBA write-up,
 //                          threshold dynamic selection) or PSA level quotas
 //                          (PSA page, multi-level mask generator)
@@ -102,71 +102,134 @@ __global__ void __launch_bounds__(128) block_means_kernel(const __nv_bfloat16* _
   }
 }
 
-// ----------------------------------------------------------- block scores ---
-// grid (ceil(nb/64), ceil(nb/64), B*H), 256 threads; each thread owns a 4 x 4
-// patch of a 64 x 64 tile of S = scale * Qbar Kbar^T, fp32 throughout.  The
-// d dimension is walked in chunks of 32 staged transposed in shared memory:
-// element (row r, column k of the chunk) sits at [k][r ^ sw(k)], where the
-// XOR sw(k) = 4 * ((k / 4) % 8) permutes whole groups of four rows.  The
-// transposed stores of a warp then fall in 32 distinct banks, and a thread
-// still reads its four rows of one column as one aligned float4.  At most 42
-// registers a thread let six CTAs share an SM, so the 768 tiles of 12 heads
-// of 512 blocks run as one wave on 148 SMs.
+// ------------------------------------------- block scores on tensor cores ---
+// grid (ceil(nb/128), ceil(nb/128), B*H), 128 threads, one 128 x 128 tile of
+// S = scale * Qbar Kbar^T per CTA, fp32 in and out.  The means are split into
+// tf32 parts, x = hi + lo with hi = x with its 13 low mantissa bits cleared
+// (exact in tf32) and lo = x - hi (exact in fp32), and
+//   S ~= hi_q hi_k^T + hi_q lo_k^T + lo_q hi_k^T
+// runs as three tcgen05 kind::tf32 MMA passes accumulating in fp32 in TMEM
+// (the dropped lo_q lo_k^T term and the tf32 rounding of lo are below 2^-20
+// of each product, close to fp32's own rounding).  The d dimension goes in
+// chunks of 32 (one 128-byte row of a 128-byte-swizzled K-major operand):
+// the threads stage the chunk's hi and lo parts of 128 Q rows and 128 K rows
+// (64 KB), one elected lane issues 12 MMAs (3 passes x 4 steps of K = 8), and
+// the staging of the next chunk (whose loads are already in registers) waits
+// for them to complete.  Epilogue: one
+// thread per row loads its 128 fp32 accumulators from TMEM, scales and stores.
+constexpr int kScoresTcSmem = 4 * 16384;   // A hi, A lo, B hi, B lo: 128 rows x 128 bytes each
+
 template <int D>
-__global__ void __launch_bounds__(256, 6) block_scores_kernel(const float* __restrict__ qmean,
+__global__ void __launch_bounds__(128) block_scores_tc_kernel(const float* __restrict__ qmean,
                                                               const float* __restrict__ kmean, int nb, float scale,
                                                               float* __restrict__ scores) {
-  __shared__ __align__(16) float sa[32][68];
-  __shared__ __align__(16) float sb[32][68];
-  const int bh = blockIdx.z;
-  const int i0 = blockIdx.y * 64, j0 = blockIdx.x * 64;
+  constexpr int kChunks = D / 32;
+  // kind::tf32: D f32 (bits 4-5 = 1), A and B tf32 (bits 7-9, 10-12 = 2), both
+  // K-major, N = 128 (bits 17-22 = N >> 3), M = 128 (bits 24-28 = M >> 4)
+  constexpr uint32_t kIdesc = (1u << 4) | (2u << 7) | (2u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ uint64_t done_bar;
+  __shared__ uint32_t tmem_base;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.z, i0 = blockIdx.y * 128, j0 = blockIdx.x * 128;
   const float* qm = qmean + static_cast<size_t>(bh) * nb * D;
   const float* km = kmean + static_cast<size_t>(bh) * nb * D;
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  auto sw = [](int k) { return ((k >> 2) & 7) << 2; };
-  float acc[4][4];
-#pragma unroll
-  for (int a = 0; a < 4; ++a)
-#pragma unroll
-    for (int c = 0; c < 4; ++c) acc[a][c] = 0.f;
-#pragma unroll 1
-  for (int kc = 0; kc < D; kc += 32) {
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int idx = threadIdx.x + u * 256;
-      const int rr = idx >> 3, c4 = (idx & 7) * 4;   // 8 lanes read one row's 32 columns
-      const float4 pa = (i0 + rr < nb)
-                            ? *reinterpret_cast<const float4*>(qm + static_cast<size_t>(i0 + rr) * D + kc + c4)
-                            : make_float4(0.f, 0.f, 0.f, 0.f);
-      const float4 pb = (j0 + rr < nb)
-                            ? *reinterpret_cast<const float4*>(km + static_cast<size_t>(j0 + rr) * D + kc + c4)
-                            : make_float4(0.f, 0.f, 0.f, 0.f);
-      const int col = rr ^ sw(c4);   // c4 .. c4 + 3 share k / 4, so one swizzle for the four
-      sa[c4 + 0][col] = pa.x; sa[c4 + 1][col] = pa.y; sa[c4 + 2][col] = pa.z; sa[c4 + 3][col] = pa.w;
-      sb[c4 + 0][col] = pb.x; sb[c4 + 1][col] = pb.y; sb[c4 + 2][col] = pb.z; sb[c4 + 3][col] = pb.w;
-    }
-    __syncthreads();
-#pragma unroll 8
-    for (int k = 0; k < 32; ++k) {
-      const float4 a = *reinterpret_cast<const float4*>(&sa[k][(ty * 4) ^ sw(k)]);
-      const float4 bq = *reinterpret_cast<const float4*>(&sb[k][(tx * 4) ^ sw(k)]);
-      const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {bq.x, bq.y, bq.z, bq.w};
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-#pragma unroll
-        for (int w = 0; w < 4; ++w) acc[u][w] = fmaf(av[u], bv[w], acc[u][w]);
-    }
-    __syncthreads();
+  if (warp == 0) {
+    tmem_alloc(&tmem_base, 128);
+    tmem_relinquish();
   }
+  if (threadIdx.x == 32) {
+    mbar_init(&done_bar, 1);
+    fence_mbar_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base;
+  const uint32_t sbase = smem_addr(smem);
+  const uint64_t d_ahi = smem_desc(sbase, 16, 1024), d_alo = smem_desc(sbase + 16384, 16, 1024);
+  const uint64_t d_bhi = smem_desc(sbase + 32768, 16, 1024), d_blo = smem_desc(sbase + 49152, 16, 1024);
+  // 2 operands x 128 rows x 8 float4 per chunk, 16 per thread: element
+  // (it, thread) is operand op, row rr, 16-byte unit u; it lands at
+  // rr * 128 + (u ^ (rr % 8)) * 16 of the operand's part.  A chunk's 16 loads
+  // are issued together, and the next chunk's are in flight during the MMAs.
+  float4 xr[16];
+  auto load_chunk = [&](int c) {
 #pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const int i = i0 + ty * 4 + u;
-    if (i >= nb) continue;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      const int j = j0 + tx * 4 + w;
-      if (j < nb) scores[(static_cast<size_t>(bh) * nb + i) * nb + j] = acc[u][w] * scale;
+    for (int it = 0; it < 16; ++it) {
+      const int idx = static_cast<int>(threadIdx.x) + 128 * it;
+      const int op = idx >> 10, rr = (idx >> 3) & 127, u = idx & 7;
+      const int grow = (op == 0 ? i0 : j0) + rr;
+      xr[it] = grow < nb ? *reinterpret_cast<const float4*>((op == 0 ? qm : km) + static_cast<size_t>(grow) * D +
+                                                             c * 32 + u * 4)
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
     }
+  };
+  auto store_chunk = [&]() {
+    auto hi_of = [](float v) { return __uint_as_float(__float_as_uint(v) & 0xFFFFE000u); };
+#pragma unroll
+    for (int it = 0; it < 16; ++it) {
+      const int idx = static_cast<int>(threadIdx.x) + 128 * it;
+      const int op = idx >> 10, rr = (idx >> 3) & 127, u = idx & 7;
+      const float4 x = xr[it];
+      const float4 hi = make_float4(hi_of(x.x), hi_of(x.y), hi_of(x.z), hi_of(x.w));
+      const float4 lo = make_float4(x.x - hi.x, x.y - hi.y, x.z - hi.z, x.w - hi.w);
+      const int off = op * 32768 + rr * 128 + ((u ^ (rr & 7)) << 4);
+      *reinterpret_cast<float4*>(smem + off) = hi;
+      *reinterpret_cast<float4*>(smem + off + 16384) = lo;
+    }
+  };
+  bool ok = true;
+  load_chunk(0);
+#pragma unroll 1
+  for (int c = 0; c < kChunks; ++c) {
+    store_chunk();
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (c + 1 < kChunks) load_chunk(c + 1);
+    if (warp == 0) {
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t off = static_cast<uint64_t>(kk * 32) >> 4;
+        mma_tf32_warp(tmem, d_ahi + off, d_bhi + off, kIdesc, (c > 0 || kk > 0) ? 1u : 0u);
+        mma_tf32_warp(tmem, d_ahi + off, d_blo + off, kIdesc, 1u);
+        mma_tf32_warp(tmem, d_alo + off, d_bhi + off, kIdesc, 1u);
+      }
+      mma_commit_warp(&done_bar);
+    }
+    // the MMAs read the staging area: the next chunk overwrites it only after they complete
+    ok = mbar_wait(&done_bar, c & 1) && ok;
+    tc_fence_after();
+  }
+  // epilogue: thread = row i0 + 32 warp + lane, columns j0 .. j0 + 127
+  const int i = i0 + warp * 32 + lane;
+  float* srow = scores + (static_cast<size_t>(bh) * nb + (i < nb ? i : 0)) * nb;
+#pragma unroll 1
+  for (int cc = 0; cc < 4; ++cc) {
+    float v[32];
+    tmem_ld32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + cc * 32, v);
+    if (i < nb && ok) {
+      const int jb = j0 + cc * 32;
+      if (jb + 32 <= nb && (nb & 3) == 0) {
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4)
+          *reinterpret_cast<float4*>(srow + jb + q4 * 4) =
+              make_float4(v[q4 * 4] * scale, v[q4 * 4 + 1] * scale, v[q4 * 4 + 2] * scale, v[q4 * 4 + 3] * scale);
+      } else {
+#pragma unroll
+        for (int t = 0; t < 32; ++t)
+          if (jb + t < nb) srow[jb + t] = v[t] * scale;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
   }
 }
 
