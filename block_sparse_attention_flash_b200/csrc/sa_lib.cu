@@ -48,6 +48,20 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
 
 // [B*H, rows, D] bf16 viewed as a 3D tensor (D innermost), 64 x 128 x 1 boxes,
 // 128-byte swizzle, zero fill outside the tensor.
+// [BH][rows][D] fp32, box 32 columns (128 bytes) x box_rows rows, 128-byte swizzle.
+bool encode_f32_map(CUtensorMap* map, const void* base, int BH, int rows, int D, int box_rows) {
+  auto fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 4, static_cast<cuuint64_t>(rows) * D * 4};
+  cuuint32_t box[3] = {32, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool encode_rows_map(CUtensorMap* map, const void* base, int BH, int rows, int D, int box_rows) {
   auto fn = get_encode_fn();
   if (!fn) return false;
@@ -220,7 +234,7 @@ size_t sa_build_mask_workspace(int B, int H, int N, int d, int block) {
   if (B <= 0 || H <= 0 || N <= 0 || d <= 0 || block <= 0) return 0;
   const size_t nb = static_cast<size_t>(ceil_div(N, block));
   const size_t bh = static_cast<size_t>(B) * H;
-  return (2 * bh * nb * d + bh * nb * nb) * sizeof(float);
+  return (4 * bh * nb * d + bh * nb * nb) * sizeof(float);
 }
 
 sa_status sa_build_mask(const void* q, const void* k, int B, int H, int N, int d, int block, int mode, float tau,
@@ -241,21 +255,29 @@ sa_status sa_build_mask(const void* q, const void* k, int B, int H, int N, int d
   cudaError_t e = init_device_kernels();
   if (e != cudaSuccess) return SA_ERR_CUDA;
   const int BH = B * H;
+  // the block means as tf32 hi / lo parts, then the scores
+  const size_t mean_n = static_cast<size_t>(BH) * nb * d;
   float* qmean = static_cast<float*>(workspace);
-  float* kmean = qmean + static_cast<size_t>(BH) * nb * d;
-  float* scores = scores_out ? scores_out : kmean + static_cast<size_t>(BH) * nb * d;
+  float* qlo = qmean + mean_n;
+  float* khi = qlo + mean_n;
+  float* klo = khi + mean_n;
+  float* scores = scores_out ? scores_out : klo + mean_n;
   cudaStream_t s = as_stream(stream);
   const float scale = 1.0f / std::sqrt(static_cast<float>(d));
   const auto* qb = static_cast<const __nv_bfloat16*>(q);
   const auto* kb = static_cast<const __nv_bfloat16*>(k);
-  dim3 g1(nb, BH, 2), g2(ceil_div(nb, 128), ceil_div(nb, 128), BH);
+  sa::ScoresMaps smaps;
+  if (!encode_f32_map(&smaps.qhi, qmean, BH, nb, d, 128) || !encode_f32_map(&smaps.qlo, qlo, BH, nb, d, 128) ||
+      !encode_f32_map(&smaps.khi, khi, BH, nb, d, 256) || !encode_f32_map(&smaps.klo, klo, BH, nb, d, 256))
+    return SA_ERR_CUDA;
+  dim3 g1(nb, BH, 2), g2(ceil_div(nb, 256), ceil_div(nb, 128), BH);
   constexpr int kScoresSmem = sa::kScoresTcSmem + 1024;
   if (d == 128) {
-    sa::block_means_kernel<128><<<g1, 128, 0, s>>>(qb, kb, N, block, nb, qmean, kmean);
-    sa::block_scores_tc_kernel<128><<<g2, 128, kScoresSmem, s>>>(qmean, kmean, nb, scale, scores);
+    sa::block_means_kernel<128><<<g1, 128, 0, s>>>(qb, kb, N, block, nb, qmean, qlo, khi, klo);
+    sa::block_scores_tc_kernel<128><<<g2, 128, kScoresSmem, s>>>(smaps, nb, scale, scores);
   } else {
-    sa::block_means_kernel<64><<<g1, 128, 0, s>>>(qb, kb, N, block, nb, qmean, kmean);
-    sa::block_scores_tc_kernel<64><<<g2, 128, kScoresSmem, s>>>(qmean, kmean, nb, scale, scores);
+    sa::block_means_kernel<64><<<g1, 128, 0, s>>>(qb, kb, N, block, nb, qmean, qlo, khi, klo);
+    sa::block_scores_tc_kernel<64><<<g2, 128, kScoresSmem, s>>>(smaps, nb, scale, scores);
   }
   const long long nrows = static_cast<long long>(BH) * nb;
   const unsigned warp_grid = static_cast<unsigned>((nrows + 3) / 4);
@@ -513,7 +535,7 @@ sa_status sa_pyramid_attn_fwd(const void* q, const void* k, const void* v, int B
 namespace {
 
 // Upper bound of the shared scratch: large enough for the 480p workload
-// (12 heads, 32,760 tokens, block 64, d 128 needs 18.9 MB).
+// (12 heads, 32,760 tokens, block 64, d 128 needs 25.2 MB).
 constexpr size_t kNoAllocScratchBytes = static_cast<size_t>(32) << 20;  // 32 MiB
 
 }  // namespace

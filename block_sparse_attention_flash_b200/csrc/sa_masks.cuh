@@ -56,11 +56,16 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float* f) {
 // ------------------------------------------------------------ block means ---
 // grid (nb, B*H, 2): z = 0 averages Q, z = 1 averages K.  128 threads: thread
 // (rg, ch) sums 16-byte chunk ch of rows rg, rg + RG, ...; smem reduces over rg.
+// Each fp32 mean x is written as two tf32 parts for the scores GEMM: hi = x
+// with its 13 low mantissa bits cleared (exact in tf32) and lo = x - hi
+// (exact in fp32); hi + lo = x.
+__device__ __forceinline__ float tf32_hi(float v) { return __uint_as_float(__float_as_uint(v) & 0xFFFFE000u); }
+
 template <int D>
 __global__ void __launch_bounds__(128) block_means_kernel(const __nv_bfloat16* __restrict__ q,
                                                           const __nv_bfloat16* __restrict__ k, int N, int block,
-                                                          int nb, float* __restrict__ qmean,
-                                                          float* __restrict__ kmean) {
+                                                          int nb, float* __restrict__ qhi, float* __restrict__ qlo,
+                                                          float* __restrict__ khi, float* __restrict__ klo) {
   constexpr int CH = D / 8;      // 16-byte chunks per row
   constexpr int RG = 128 / CH;   // row groups
   __shared__ float red[RG][D];
@@ -97,122 +102,116 @@ __global__ void __launch_bounds__(128) block_means_kernel(const __nv_bfloat16* _
     float s = 0.f;
 #pragma unroll
     for (int g = 0; g < RG; ++g) s += red[g][c];
-    float* out = (z == 0 ? qmean : kmean) + (static_cast<size_t>(bh) * nb + i) * D;
-    out[c] = s / static_cast<float>(rows);
+    const size_t o = (static_cast<size_t>(bh) * nb + i) * D + c;
+    const float m = s / static_cast<float>(rows);
+    const float hi = tf32_hi(m);
+    (z == 0 ? qhi : khi)[o] = hi;
+    (z == 0 ? qlo : klo)[o] = m - hi;
   }
 }
 
 // ------------------------------------------- block scores on tensor cores ---
-// grid (ceil(nb/128), ceil(nb/128), B*H), 128 threads, one 128 x 128 tile of
-// S = scale * Qbar Kbar^T per CTA, fp32 in and out.  The means are split into
-// tf32 parts, x = hi + lo with hi = x with its 13 low mantissa bits cleared
-// (exact in tf32) and lo = x - hi (exact in fp32), and
+// grid (ceil(nb/256), ceil(nb/128), B*H), 128 threads, one 128 x 256 tile of
+// S = scale * Qbar Kbar^T per CTA, fp32 out.  The means arrive as tf32 parts
+// (x = hi + lo, block_means_kernel), and
 //   S ~= hi_q hi_k^T + hi_q lo_k^T + lo_q hi_k^T
 // runs as three tcgen05 kind::tf32 MMA passes accumulating in fp32 in TMEM
 // (the dropped lo_q lo_k^T term and the tf32 rounding of lo are below 2^-20
 // of each product, close to fp32's own rounding).  The d dimension goes in
-// chunks of 32 (one 128-byte row of a 128-byte-swizzled K-major operand):
-// the threads stage the chunk's hi and lo parts of 128 Q rows and 128 K rows
-// (64 KB), one elected lane issues 12 MMAs (3 passes x 4 steps of K = 8), and
-// the staging of the next chunk (whose loads are already in registers) waits
-// for them to complete.  Epilogue: one
-// thread per row loads its 128 fp32 accumulators from TMEM, scales and stores.
-constexpr int kScoresTcSmem = 4 * 16384;   // A hi, A lo, B hi, B lo: 128 rows x 128 bytes each
+// chunks of 32 (one 128-byte row of a 128-byte-swizzled K-major operand)
+// through a 2-stage ring that TMA fills (Q hi / lo: 128 rows, K hi / lo: 256
+// rows; rows past a head's last block read as zero); per chunk one elected
+// lane issues 12 MMAs (3 passes x 4 steps of K = 8) and releases the stage.
+// Epilogue: one thread per row loads its 256 fp32 accumulators from TMEM,
+// scales and stores the columns below nb.
+constexpr int kScoresStage = 2 * 16384 + 2 * 32768;   // A hi, A lo (128 rows), B hi, B lo (256 rows) x 128 B
+constexpr int kScoresTcSmem = 2 * kScoresStage;
+
+struct ScoresMaps {
+  CUtensorMap qhi, qlo, khi, klo;   // fp32 [B*H][nb][D], box 32 columns x 128 (Q) or 256 (K) rows
+};
 
 template <int D>
-__global__ void __launch_bounds__(128) block_scores_tc_kernel(const float* __restrict__ qmean,
-                                                              const float* __restrict__ kmean, int nb, float scale,
-                                                              float* __restrict__ scores) {
+__global__ void __launch_bounds__(128, 1) block_scores_tc_kernel(const __grid_constant__ ScoresMaps maps, int nb,
+                                                                 float scale, float* __restrict__ scores) {
   constexpr int kChunks = D / 32;
   // kind::tf32: D f32 (bits 4-5 = 1), A and B tf32 (bits 7-9, 10-12 = 2), both
-  // K-major, N = 128 (bits 17-22 = N >> 3), M = 128 (bits 24-28 = M >> 4)
-  constexpr uint32_t kIdesc = (1u << 4) | (2u << 7) | (2u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+  // K-major, N = 256 (bits 17-22 = N >> 3), M = 128 (bits 24-28 = M >> 4)
+  constexpr uint32_t kIdesc = (1u << 4) | (2u << 7) | (2u << 10) | ((256u >> 3) << 17) | ((128u >> 4) << 24);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ uint64_t done_bar;
+  __shared__ uint64_t full_bar[2], empty_bar[2], done_bar;
   __shared__ uint32_t tmem_base;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.z, i0 = blockIdx.y * 128, j0 = blockIdx.x * 128;
-  const float* qm = qmean + static_cast<size_t>(bh) * nb * D;
-  const float* km = kmean + static_cast<size_t>(bh) * nb * D;
-  if (warp == 0) {
-    tmem_alloc(&tmem_base, 128);
+  const int bh = blockIdx.z, i0 = blockIdx.y * 128, j0 = blockIdx.x * 256;
+  if (warp == 2) {
+    tmem_alloc(&tmem_base, 256);
     tmem_relinquish();
   }
-  if (threadIdx.x == 32) {
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&full_bar[i], 1);
+      mbar_init(&empty_bar[i], 1);
+    }
     mbar_init(&done_bar, 1);
     fence_mbar_init();
+    tma_prefetch_desc(&maps.qhi);
+    tma_prefetch_desc(&maps.qlo);
+    tma_prefetch_desc(&maps.khi);
+    tma_prefetch_desc(&maps.klo);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base;
-  const uint32_t sbase = smem_addr(smem);
-  const uint64_t d_ahi = smem_desc(sbase, 16, 1024), d_alo = smem_desc(sbase + 16384, 16, 1024);
-  const uint64_t d_bhi = smem_desc(sbase + 32768, 16, 1024), d_blo = smem_desc(sbase + 49152, 16, 1024);
-  // 2 operands x 128 rows x 8 float4 per chunk, 16 per thread: element
-  // (it, thread) is operand op, row rr, 16-byte unit u; it lands at
-  // rr * 128 + (u ^ (rr % 8)) * 16 of the operand's part.  A chunk's 16 loads
-  // are issued together, and the next chunk's are in flight during the MMAs.
-  float4 xr[16];
-  auto load_chunk = [&](int c) {
-#pragma unroll
-    for (int it = 0; it < 16; ++it) {
-      const int idx = static_cast<int>(threadIdx.x) + 128 * it;
-      const int op = idx >> 10, rr = (idx >> 3) & 127, u = idx & 7;
-      const int grow = (op == 0 ? i0 : j0) + rr;
-      xr[it] = grow < nb ? *reinterpret_cast<const float4*>((op == 0 ? qm : km) + static_cast<size_t>(grow) * D +
-                                                             c * 32 + u * 4)
-                         : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-  };
-  auto store_chunk = [&]() {
-    auto hi_of = [](float v) { return __uint_as_float(__float_as_uint(v) & 0xFFFFE000u); };
-#pragma unroll
-    for (int it = 0; it < 16; ++it) {
-      const int idx = static_cast<int>(threadIdx.x) + 128 * it;
-      const int op = idx >> 10, rr = (idx >> 3) & 127, u = idx & 7;
-      const float4 x = xr[it];
-      const float4 hi = make_float4(hi_of(x.x), hi_of(x.y), hi_of(x.z), hi_of(x.w));
-      const float4 lo = make_float4(x.x - hi.x, x.y - hi.y, x.z - hi.z, x.w - hi.w);
-      const int off = op * 32768 + rr * 128 + ((u ^ (rr & 7)) << 4);
-      *reinterpret_cast<float4*>(smem + off) = hi;
-      *reinterpret_cast<float4*>(smem + off + 16384) = lo;
-    }
-  };
-  bool ok = true;
-  load_chunk(0);
-#pragma unroll 1
-  for (int c = 0; c < kChunks; ++c) {
-    store_chunk();
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (c + 1 < kChunks) load_chunk(c + 1);
-    if (warp == 0) {
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t off = static_cast<uint64_t>(kk * 32) >> 4;
-        mma_tf32_warp(tmem, d_ahi + off, d_bhi + off, kIdesc, (c > 0 || kk > 0) ? 1u : 0u);
-        mma_tf32_warp(tmem, d_ahi + off, d_blo + off, kIdesc, 1u);
-        mma_tf32_warp(tmem, d_alo + off, d_bhi + off, kIdesc, 1u);
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer ---
+    if (lane == 0) {
+      for (int c = 0; c < kChunks; ++c) {
+        const int st = c & 1;
+        if (c >= 2 && !mbar_wait(&empty_bar[st], ((c >> 1) - 1) & 1)) break;
+        uint8_t* base = smem + st * kScoresStage;
+        mbar_arrive_expect_tx(&full_bar[st], static_cast<uint32_t>(kScoresStage));
+        tma_load_3d(&maps.qhi, &full_bar[st], base, c * 32, i0, bh);
+        tma_load_3d(&maps.qlo, &full_bar[st], base + 16384, c * 32, i0, bh);
+        tma_load_3d(&maps.khi, &full_bar[st], base + 32768, c * 32, j0, bh);
+        tma_load_3d(&maps.klo, &full_bar[st], base + 65536, c * 32, j0, bh);
       }
-      mma_commit_warp(&done_bar);
     }
-    // the MMAs read the staging area: the next chunk overwrites it only after they complete
-    ok = mbar_wait(&done_bar, c & 1) && ok;
-    tc_fence_after();
+  } else if (warp == 1) {
+    // -------------------------------------------------------- MMA issue ---
+    bool ok = true;
+    for (int c = 0; c < kChunks; ++c) {
+      const int st = c & 1;
+      ok = ok && __all_sync(0xffffffffu, mbar_wait(&full_bar[st], (c >> 1) & 1));
+      if (ok) {
+        tc_fence_after();
+        const uint32_t sbase = smem_addr(smem + st * kScoresStage);
+        const uint64_t d_ahi = smem_desc(sbase, 16, 1024), d_alo = smem_desc(sbase + 16384, 16, 1024);
+        const uint64_t d_bhi = smem_desc(sbase + 32768, 16, 1024), d_blo = smem_desc(sbase + 65536, 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t off = static_cast<uint64_t>(kk * 32) >> 4;
+          mma_tf32_warp(tmem, d_ahi + off, d_bhi + off, kIdesc, (c > 0 || kk > 0) ? 1u : 0u);
+          mma_tf32_warp(tmem, d_ahi + off, d_blo + off, kIdesc, 1u);
+          mma_tf32_warp(tmem, d_alo + off, d_bhi + off, kIdesc, 1u);
+        }
+      }
+      mma_commit_warp(&empty_bar[st]);   // also after an error, so that the producer never stalls
+    }
+    mma_commit_warp(&done_bar);
   }
-  // epilogue: thread = row i0 + 32 warp + lane, columns j0 .. j0 + 127
+  // epilogue: thread = row i0 + 32 warp + lane, columns j0 .. j0 + 255
+  const bool ok = mbar_wait(&done_bar, 0);
+  tc_fence_after();
   const int i = i0 + warp * 32 + lane;
   float* srow = scores + (static_cast<size_t>(bh) * nb + (i < nb ? i : 0)) * nb;
 #pragma unroll 1
-  for (int cc = 0; cc < 4; ++cc) {
+  for (int cc = 0; cc < 8; ++cc) {
     float v[32];
     tmem_ld32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + cc * 32, v);
-    if (i < nb && ok) {
-      const int jb = j0 + cc * 32;
+    const int jb = j0 + cc * 32;
+    if (i < nb && ok && jb < nb) {
       if (jb + 32 <= nb && (nb & 3) == 0) {
 #pragma unroll
         for (int q4 = 0; q4 < 8; ++q4)
@@ -227,9 +226,9 @@ __global__ void __launch_bounds__(128) block_scores_tc_kernel(const float* __res
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 2) {
     tc_fence_after();
-    tmem_dealloc(tmem, 128);
+    tmem_dealloc(tmem, 256);
   }
 }
 

@@ -110,7 +110,8 @@ SA_API sa_status sa_self_test_timeout(uint64_t wait_ns, void* stream);
 
 /*
  * sa_build_mask_workspace — bytes of device scratch sa_build_mask needs:
- * the fp32 block means of Q and K (2 * B*H*Nb*d floats) plus the fp32 block
+ * the block means of Q and K, each as two fp32 arrays (tf32 high and low
+ * parts for the tensor-core scores: 4 * B*H*Nb*d floats), plus the fp32 block
  * scores (B*H*Nb*Nb floats).  The caller allocates it (any 256-byte aligned
  * buffer of at least this size).
  */

@@ -57,7 +57,7 @@ def test_self_test_timeout_argument_validation(lib):
 def test_workspace_size(lib):
     B, H, N, d, block = 1, 12, 32760, 128, 64
     nb = -(-N // block)
-    assert ops.sa_build_mask_workspace(B, H, N, d, block) == 4 * (2 * B * H * nb * d + B * H * nb * nb)
+    assert ops.sa_build_mask_workspace(B, H, N, d, block) == 4 * (4 * B * H * nb * d + B * H * nb * nb)
     assert ops.sa_build_mask_workspace(0, H, N, d, block) == 0
 
 

@@ -75,6 +75,38 @@ def test_scores_out_matches_oracle_scores():
     assert np.abs(sc.cpu().numpy() - S).max() < 1e-4
 
 
+def test_block_scores_480p_accuracy():
+    """The block scores at the 480p size (2 heads, Nb = 512) against the oracle's fp64 scores.
+
+    The GPU forms the means in fp32 and the scores on tensor cores from three
+    tf32 passes of a hi / lo split of the means.  Per score the error is
+    bounded by the magnitude m = scale * sum_a |qbar_a| |kbar_a| times: the
+    fp32 means (at most 64 additions of 2^-24 each, for both factors), the
+    split (the dropped lo * lo term and the tf32 rounding of lo, below 2^-20
+    per product) and the fp32 accumulation over d = 128 terms (128 * 2^-24):
+    about 2 * 64 * 2^-24 + 2^-20 + 128 * 2^-24 = 1.6e-5.  The test asserts
+    2e-5 * m."""
+    wl = inputs.WORKLOADS["wan13b_480p_tau"]
+    q, k, _ = inputs.rff_qkv(wl, H=2)
+    nb = wl.nblocks
+    sc = torch.empty(1, 2, nb, nb, device="cuda")
+    ops.sa_build_mask(q.cuda(), k.cuda(), wl.block, "tau", tau=wl.tau, scores_out=sc)
+    ops.sa_get_device_status()
+    _, _, S = tau_mask(q, k, wl.block, wl.tau, return_info=True)
+    d = q.shape[-1]
+    pad = nb * wl.block - q.shape[2]
+    qa = np.pad(q.double().numpy(), ((0, 0), (0, 0), (0, pad), (0, 0)))
+    ka = np.pad(k.double().numpy(), ((0, 0), (0, 0), (0, pad), (0, 0)))
+    cnt = np.minimum(wl.block, q.shape[2] - np.arange(nb) * wl.block)[None, None, :, None]
+    qbar = qa.reshape(1, 2, nb, wl.block, d).sum(3) / cnt
+    kbar = ka.reshape(1, 2, nb, wl.block, d).sum(3) / cnt
+    mag = np.einsum("bhid,bhjd->bhij", np.abs(qbar), np.abs(kbar)) / np.sqrt(d)
+    err = np.abs(sc.cpu().double().numpy() - S)
+    worst = float((err / np.maximum(mag, 1e-30)).max())
+    print(f"480p block scores: max |error| / magnitude = {worst:.2e}")
+    assert np.all(err <= 2e-5 * mag + 1e-12), worst
+
+
 def test_uniform_scores_keep_first_blocks():
     """Q == 0 makes every score equal: the GPU must break ties by index."""
     N, block = 64 * 42, 64            # tau * Nb = 31.5: no exact tie with the threshold
