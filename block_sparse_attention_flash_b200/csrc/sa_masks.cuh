@@ -6,9 +6,11 @@
 //                          block scoring with pooled queries/keys)
 //   block_scores_tc_kernel S_ij = scale * qbar_i . kbar_j (one small GEMM per
 //                          head, fp32 accuracy from three tf32 tensor-core passes)
-//   block_select_kernel    per q-block row: tau-mass selection (VMoBA write-up,
-//                          threshold dynamic selection) or PSA level quotas
-//                          (PSA page, multi-level mask generator)
+//   tau_select_warp_kernel per q-block row, one warp: tau-mass selection
+//                          (VMoBA write-up, threshold dynamic selection)
+//   level_select_warp_kernel  per q-block row, one warp: PSA level quotas (PSA
+//                          page, multi-level mask generator)
+//   block_select_kernel    either, one CTA per row, for rows above 1024 blocks
 //   pyramid_pool_kernel    mean of 2, 4, 8 consecutive tokens (PSA page,
 //                          pyramid KV by progressive average pooling)
 //
