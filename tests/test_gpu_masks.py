@@ -136,6 +136,27 @@ def test_pyramid_pool(d, N):
             assert np.all(err <= np.abs(ref) * 2.0 ** -8 + 1e-6), (c, float(err.max()))
 
 
+@pytest.mark.parametrize("block", [64, 128])
+@pytest.mark.parametrize("d", [64, 128])
+def test_mask_builder_batch2_ragged(block, d):
+    """B = 2 (every mask kernel folds the batch into B*H) with a ragged last block (4,320 tokens):
+    the block scores against the oracle's fp64 scores, and the tau and level masks flag-aware."""
+    wl = inputs.Workload("b2", 2, 2, d, 9, 20, 24, block, "tau", seed=83 + d + block)
+    q, k, _ = inputs.rff_qkv(wl)
+    nb = wl.nblocks
+    assert q.shape[0] == 2 and q.shape[2] % block != 0
+    fr = (0.1, 0.3, 0.6)
+    sc = torch.empty(2, 2, nb, nb, device="cuda")
+    m = ops.sa_build_mask(q.cuda(), k.cuda(), block, "tau", tau=0.9, scores_out=sc)
+    lv = ops.sa_build_mask(q.cuda(), k.cuda(), block, "levels", level_frac=fr)
+    ops.sa_get_device_status()
+    mr, flags, S = tau_mask(q, k, block, 0.9, return_info=True)
+    assert np.abs(sc.cpu().numpy() - S).max() < 1e-4
+    check_bits(m.cpu(), mr, flags, f"tau B=2 d={d} block={block}")
+    lr, lflags, _ = level_map(q, k, block, fr, return_info=True)
+    check_bits(lv.cpu(), lr, lflags, f"levels B=2 d={d} block={block}")
+
+
 def test_tau_mask_wan13b_480p_full():
     """Full-size tau mask of the 480p Wan2.1-1.3B-like workload (12 heads, 512 x 512 blocks)."""
     wl = inputs.WORKLOADS["wan13b_480p_tau"]
