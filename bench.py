@@ -452,6 +452,32 @@ def config_tau(ops, wl, q, k, v, dev, stream, peaks, src, cpu_seconds):
     mask_bytes = 2 * B * H * N * d * 2 + B * H * nb * nb
     entry = {"path": "sa_build_mask (tau) + sa_sparse_attn_fwd", "attention": _attn_entry(wl, ms_a, flops, peaks, src),
              "mask_builder": _hbm_entry(ms_m, mask_bytes, peaks, src)}
+    # backward over the same mask (dQ, dK, dV from dO, O, LSE): algorithmic work is 5 GEMMs per
+    # kept element (S, dP, dV, dK, dQ); the kernels execute 7 (S and dP again in the dQ pass)
+    lse = torch.empty(B, H, N, device=dev)
+    ops.sa_sparse_attn_fwd(q, k, v, wl.block, mask=m, out=o, lse=lse)
+    gen = torch.Generator(device=dev).manual_seed(wl.seed + 11)
+    dout = torch.randn(q.shape, generator=gen, device=dev).to(torch.bfloat16)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    bws = torch.empty(ops.sa_sparse_attn_bwd_workspace(B, H, N), dtype=torch.uint8, device=dev)
+    ms_b = _time(lambda: ops.sa_sparse_attn_bwd(q, k, v, o, dout, lse, wl.block, mask=m, dq=dq, dk=dk, dv=dv,
+                                                workspace=bws), CONFIG_REPS, stream)
+    burst = float(peaks["bf16_tflops"])
+    alg_tf = 2.5 * flops / ms_b / 1e9
+    entry["backward"] = {"path": "sa_sparse_attn_bwd", "ms_per_call": round(ms_b, 3),
+                         "algorithmic_tflops": round(alg_tf, 1),
+                         "executed_tflops_7gemm": round(3.5 * flops / ms_b / 1e9, 1),
+                         "roofline": {"bound": "tensor", "achieved": round(alg_tf, 1), "peak": burst,
+                                      "unit": "TFLOP/s", "frac": round(alg_tf / burst, 4),
+                                      "peak_source": f"{src} bf16_tflops (burst: a kernel timed alone)"}}
+    del dout, dq, dk, dv, bws, lse
+    # token permutation of Q, K, V: per-head PARO axis orders and 3 x 5 x 4 VMoBA cells
+    orders = (torch.arange(H, device=dev) % 6).to(torch.uint8)
+    pout = [torch.empty_like(q) for _ in range(3)]
+    ms_p = _time(lambda: ops.sa_token_permute([q, k, v], wl.T, wl.Hh, wl.Ww, head_order=orders, cells=(3, 5, 4),
+                                              out=pout), CONFIG_REPS, stream, SHORT_CALL_BATCH)
+    entry["permute_qkv"] = dict(path="sa_token_permute", **_hbm_entry(ms_p, 2 * 3 * B * H * N * d * 2, peaks, src))
+    del pout
     if cpu_seconds > 0:
         entry["cpu_baseline"] = cpu_config_sample(wl, q, k, v, m, cpu_seconds, "tau")
     return entry
