@@ -451,8 +451,12 @@ __device__ __forceinline__ void level_select_row(const float* __restrict__ srow,
   }
 }
 
+// At E = 16 (rows of up to 512 blocks) the registers are capped so that 11
+// CTAs share an SM: the 1,536 CTAs of 12 heads of 512 rows then run as one
+// wave (50.1 against 55.5 us at 480p).  The same cap costs the tau kernel
+// spills and time, so it keeps its 64 registers.
 template <int E>
-__global__ void __launch_bounds__(128) level_select_warp_kernel(const float* __restrict__ scores, int nb,
+__global__ void __launch_bounds__(128, E == 16 ? 11 : 1) level_select_warp_kernel(const float* __restrict__ scores, int nb,
                                                                 long long nrows, int c0, int c1, int c2,
                                                                 uint8_t* __restrict__ mask_out) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
