@@ -297,7 +297,7 @@ def assemble_line(wl, world, steps, warmup, total_ms_max, flops_all, kern_ms, fl
     }
 
 
-E2E_HEADS_PER_CHUNK = 2   # measured: 2 heads 98.2 ms per step, 4 heads 100.5, 8 heads 105
+E2E_HEADS_PER_CHUNK = 1   # measured: 1 head 95.9-96.6 ms per step, 2 heads 97.2-97.7 (same process), 4 heads 100.5, 8 heads 105
 
 
 def run_e2e(ops, qkv, first, block, eps, nb, dev, stream, world):
