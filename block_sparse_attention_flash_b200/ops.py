@@ -322,16 +322,26 @@ def sa_sparse_attn_fwd_host_workspace(N: int, d: int, heads_per_chunk: int) -> i
     return int(lib().sa_sparse_attn_fwd_host_workspace(N, d, heads_per_chunk))
 
 
+def default_heads_per_chunk(N: int, H: int, n_sm: int = 148) -> int:
+    """Heads per chunk for sa_sparse_attn_fwd_host: the fewest heads whose
+    q-tile pairs (ceil(N / 256) per head) fill two waves of the SMs.  The
+    first chunk's copy in and the last chunk's copy out are not overlapped, so
+    smaller chunks hide more; one 75,600-token head is already 296 pairs."""
+    pairs = -(-N // 256)
+    return max(1, min(H, -(-2 * n_sm // max(pairs, 1))))
+
+
 def sa_sparse_attn_fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block: int, out: torch.Tensor,
                             mask: Optional[torch.Tensor] = None, skip_in: Optional[torch.Tensor] = None,
                             skip_out: Optional[torch.Tensor] = None, eps: float = math.inf, scale: float = 0.0,
-                            lse: Optional[torch.Tensor] = None, heads_per_chunk: int = 4,
+                            lse: Optional[torch.Tensor] = None, heads_per_chunk: Optional[int] = None,
                             workspace: Optional[torch.Tensor] = None, stream=None, order: str = "ascending",
                             causal: bool = False, device=None) -> torch.Tensor:
-    """sa_sparse_attn_fwd with q, k, v and out in host memory (pin them for overlap)."""
+    """sa_sparse_attn_fwd with q, k, v and out in host memory (pin them for overlap).
+    heads_per_chunk None: default_heads_per_chunk(N, H)."""
     B, H, N, d = q.shape
     nb = nblocks(N, block)
-    hc = min(heads_per_chunk, H)
+    hc = min(heads_per_chunk if heads_per_chunk is not None else default_heads_per_chunk(N, H), H)
     if workspace is None:
         dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
         workspace = torch.empty(sa_sparse_attn_fwd_host_workspace(N, d, hc), dtype=torch.uint8, device=dev)

@@ -207,3 +207,12 @@ def test_host_entry_workspace_and_validation(lib):
     assert call(d=96) == ops.SA_ERR_UNSUPPORTED
     assert call(ws_bytes=100) == ops.SA_ERR_INVALID_ARG
     assert call(ws=24) == ops.SA_ERR_INVALID_ARG
+
+
+def test_default_heads_per_chunk():
+    """Host-buffer forward: the fewest heads whose q-tile pairs fill two waves of 148 SMs."""
+    from block_sparse_attention_flash_b200.ops import default_heads_per_chunk
+    assert default_heads_per_chunk(75600, 40) == 1      # 296 pairs a head: two waves already
+    assert default_heads_per_chunk(32760, 12) == 3      # 128 pairs a head
+    assert default_heads_per_chunk(256, 8) == 8         # one pair a head: capped at H
+    assert default_heads_per_chunk(1, 1) == 1
