@@ -110,21 +110,6 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-// Named barrier over `nthreads` threads that also returns the AND of `v`
-// over all of them, so that every participant takes the same branch.
-__device__ __forceinline__ bool named_bar_and(int id, int nthreads, bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred pi, po;\n\t"
-      "setp.ne.u32 pi, %2, 0;\n\t"
-      "bar.red.and.pred po, %1, %3, pi;\n\t"
-      "selp.u32 %0, 1, 0, po;\n\t}"
-      : "=r"(r)
-      : "r"(id), "r"(static_cast<uint32_t>(v)), "r"(nthreads)
-      : "memory");
-  return r != 0;
-}
-
 // p = 2^x for 64 logits s[c] (x = s * sl2 + neg_m), packed to 32 bf16 pairs;
 // returns the fp32 sum.  The scale-and-shift and the sums run on packed
 // f32x2 FMA / ADD (two lanes per instruction): the softmax loop is partly

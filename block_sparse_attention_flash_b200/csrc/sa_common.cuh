@@ -155,33 +155,13 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::f16 (bf16 in, fp32 acc).
-__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                       uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// D[tmem] (+)= A[tmem] * B[smem desc], kind::f16.
-__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                       uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// Warp-wide forms: the whole warp calls them with warp-uniform operands (so
-// the descriptors can live in uniform registers) and one elected lane issues.
-// A single-lane caller pays a register-to-uniform move per operand on every
-// MMA; measured on B200, 8 back-to-back 128x128x16 MMAs issue in 171 clocks
-// warp-wide against 386 from one lane.
+// MMA issue, warp-wide: the whole warp calls these with warp-uniform operands
+// (so the descriptors can live in uniform registers) and one elected lane
+// issues.  Issuing from a single lane instead pays a register-to-uniform move
+// per operand on every MMA; measured on B200, 8 back-to-back 128x128x16 MMAs
+// issue in 171 clocks warp-wide against 386 from one lane.
+//
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::f16 (bf16 in, fp32 accumulate).
 __device__ __forceinline__ void mma_ss_warp(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                             uint32_t accumulate) {
   asm volatile(
@@ -205,6 +185,7 @@ __device__ __forceinline__ void mma_tf32_warp(uint32_t d_tmem, uint64_t a_desc, 
       : "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem desc], kind::f16.
 __device__ __forceinline__ void mma_ts_warp(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
                                             uint32_t accumulate) {
   asm volatile(
@@ -216,19 +197,14 @@ __device__ __forceinline__ void mma_ts_warp(uint32_t d_tmem, uint32_t a_tmem, ui
       : "memory");
 }
 
+// Arrive once on `bar` (from one elected lane) when every tcgen05 op issued so
+// far by the issuing thread has completed.
 __device__ __forceinline__ void mma_commit_warp(uint64_t* bar) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t"
       "elect.sync _|e, 0xffffffff;\n\t"
       "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_addr(bar))
       : "memory");
-}
-
-// Arrive once on `bar` when every tcgen05 op issued so far by this thread completes.
-__device__ __forceinline__ void mma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   smem_addr(bar))
-               : "memory");
 }
 
 // Shared-memory matrix descriptor (sm_100 format): start address, leading and
@@ -324,23 +300,6 @@ __device__ __forceinline__ void tmem_ld128(uint32_t taddr, float* v) {
       : SA_R8(0), SA_R8(8), SA_R8(16), SA_R8(24), SA_R8(32), SA_R8(40), SA_R8(48), SA_R8(56), SA_R8(64),
         SA_R8(72), SA_R8(80), SA_R8(88), SA_R8(96), SA_R8(104), SA_R8(112), SA_R8(120)
       : "r"(taddr), "r"(taddr + 32), "r"(taddr + 64), "r"(taddr + 96)
-      : "memory");
-#undef SA_R8
-}
-
-// 2 x (32 lanes x 32 columns) from TMEM into v[0..63], one wait for both.
-__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float* v) {
-  uint32_t* r = reinterpret_cast<uint32_t*>(v);
-#define SA_R8(b) "=r"(r[b]), "=r"(r[b + 1]), "=r"(r[b + 2]), "=r"(r[b + 3]), "=r"(r[b + 4]), "=r"(r[b + 5]), \
-                 "=r"(r[b + 6]), "=r"(r[b + 7])
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%64];\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, "
-      "%45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%65];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : SA_R8(0), SA_R8(8), SA_R8(16), SA_R8(24), SA_R8(32), SA_R8(40), SA_R8(48), SA_R8(56)
-      : "r"(taddr), "r"(taddr + 32)
       : "memory");
 #undef SA_R8
 }
