@@ -166,7 +166,8 @@ int level_quota(float f, int nb) {
 // Host-side checks shared by sa_build_mask and sa_build_mask_noalloc (all but
 // the workspace).  *empty is set for a call with no rows (nothing to launch).
 sa_status check_build_mask_args(const void* q, const void* k, int B, int H, int N, int d, int block, int mode,
-                                float tau, const float* level_frac, const uint8_t* mask_out, bool* empty) {
+                                float tau, const float* level_frac, const uint8_t* mask_out, const float* scores_out,
+                                bool* empty) {
   *empty = false;
   if (B < 0 || H < 0 || N < 0) return SA_ERR_INVALID_ARG;
   if (mode != SA_MASK_TAU && mode != SA_MASK_LEVELS && mode != SA_MASK_GLOBAL) return SA_ERR_INVALID_ARG;
@@ -178,6 +179,7 @@ sa_status check_build_mask_args(const void* q, const void* k, int B, int H, int 
   if (!valid_dim(d) || !valid_block(block)) return SA_ERR_UNSUPPORTED;
   if (!q || !k || !mask_out) return SA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k)) return SA_ERR_INVALID_ARG;
+  if (scores_out && !aligned16(scores_out)) return SA_ERR_INVALID_ARG;   // rows are stored as float4
   if (ceil_div(N, block) > sa::kMaxSelect) return SA_ERR_UNSUPPORTED;
   if (static_cast<long long>(B) * H > 65535) return SA_ERR_UNSUPPORTED;
   if (mode == SA_MASK_LEVELS) {
@@ -241,7 +243,8 @@ sa_status sa_build_mask(const void* q, const void* k, int B, int H, int N, int d
                         const float* level_frac, uint8_t* mask_out, float* scores_out, void* workspace,
                         size_t workspace_bytes, void* stream) {
   bool empty = false;
-  const sa_status st = check_build_mask_args(q, k, B, H, N, d, block, mode, tau, level_frac, mask_out, &empty);
+  const sa_status st =
+      check_build_mask_args(q, k, B, H, N, d, block, mode, tau, level_frac, mask_out, scores_out, &empty);
   if (st != SA_OK || empty) return st;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return SA_ERR_INVALID_ARG;
   if (workspace_bytes < sa_build_mask_workspace(B, H, N, d, block)) return SA_ERR_INVALID_ARG;
@@ -578,7 +581,8 @@ extern "C" sa_status sa_build_mask_noalloc(const void* q, const void* k, int B, 
                                            int mode, float tau, const float* level_frac, uint8_t* mask_out,
                                            float* scores_out, void* stream) {
   bool empty = false;
-  const sa_status st = check_build_mask_args(q, k, B, H, N, d, block, mode, tau, level_frac, mask_out, &empty);
+  const sa_status st =
+      check_build_mask_args(q, k, B, H, N, d, block, mode, tau, level_frac, mask_out, scores_out, &empty);
   if (st != SA_OK || empty) return st;
   if (sa_build_mask_workspace(B, H, N, d, block) > kNoAllocScratchBytes) return SA_ERR_UNSUPPORTED;
   void* scratch = nullptr;

@@ -150,7 +150,8 @@ SA_API size_t sa_build_mask_workspace(int B, int H, int N, int d, int block);
  *   tau         (0, 1]; used for SA_MASK_TAU and SA_MASK_GLOBAL.
  *   level_frac  HOST pointer to 3 floats in [0,1]; used for SA_MASK_LEVELS.
  *   mask_out    uint8 [B,H,Nb,Nb] device, written in full.
- *   scores_out  optional fp32 [B,H,Nb,Nb] device (NULL: kept in workspace).
+ *   scores_out  optional fp32 [B,H,Nb,Nb] device, 16-byte aligned (NULL:
+ *               kept in workspace).
  *   workspace   device scratch of sa_build_mask_workspace() bytes.
  * Limits: d in {64,128}, block in {64,128}, Nb <= 4096.
  */

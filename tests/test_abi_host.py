@@ -100,6 +100,7 @@ def test_mask_builder_argument_validation(lib):
              None) == ops.SA_ERR_INVALID_ARG                   # workspace too small
     assert f(16, 16, 1, 1, 512, 64, 64, 0, 0.9, None, 16, None, 200, 1 << 20, None) == ops.SA_ERR_INVALID_ARG
     assert f(16, 16, 1, 1, 512, 80, 64, 0, 0.9, None, 16, None, 256, 1 << 20, None) == ops.SA_ERR_UNSUPPORTED
+    assert f(16, 16, 1, 1, 512, 64, 64, 0, 0.9, None, 16, 20, 256, 1 << 20, None) == ops.SA_ERR_INVALID_ARG  # scores_out
     assert f(16, 16, 1, 1, 0, 64, 64, 0, 0.9, None, 16, None, 256, 0, None) == ops.SA_OK
 
 
@@ -121,6 +122,7 @@ def test_noalloc_mask_builder_checks_arguments_before_its_scratch_lookup(lib):
     assert f(16, 16, 1, 1, 512, 80, 64, 0, 0.9, None, 16, None, None) == ops.SA_ERR_UNSUPPORTED   # d
     assert f(16, 16, 1, 1, 512, 64, 32, 0, 0.9, None, 16, None, None) == ops.SA_ERR_UNSUPPORTED   # block
     assert f(24, 16, 1, 1, 512, 64, 64, 0, 0.9, None, 16, None, None) == ops.SA_ERR_INVALID_ARG   # alignment
+    assert f(16, 16, 1, 1, 512, 64, 64, 0, 0.9, None, 16, 20, None) == ops.SA_ERR_INVALID_ARG     # scores_out
     assert f(16, 16, 1, 1, 512, 64, 64, 0, 0.9, None, None, None, None) == ops.SA_ERR_INVALID_ARG  # no mask
     assert f(16, 16, -1, 1, 512, 64, 64, 0, 0.9, None, 16, None, None) == ops.SA_ERR_INVALID_ARG
     assert f(16, 16, 1, 1, 0, 64, 64, 0, 0.9, frp, 16, None, None) == ops.SA_OK                   # empty
