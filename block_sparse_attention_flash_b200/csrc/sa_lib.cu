@@ -151,6 +151,31 @@ long long tail_units_to_split(long long units, int n_sm) {
   return (tail > 0 && 2 * tail <= n_sm) ? tail : 0;
 }
 
+// Launch with programmatic stream serialization (128 threads a CTA): the
+// kernel's CTAs may be scheduled, and run their set-up, while the previous
+// kernel on the stream is still finishing.  Only the mask builder's scores
+// and warp selections are launched this way; each executes
+// griddepcontrol.wait, which returns once the previous kernel has completed
+// and its writes are visible, before it touches global memory that a kernel
+// before it reads or writes.  A kernel lets its dependents start early
+// (griddepcontrol.launch_dependents) only after its own wait, or, for the
+// block means (an ordinary launch), at its start: each kernel therefore runs
+// ahead of its immediate predecessor only, never of a kernel further back.
+template <typename... P, typename... A>
+cudaError_t launch_pdl(void (*kern)(P...), dim3 grid, int smem, cudaStream_t s, A... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<P>(args)...);
+}
+
 bool valid_dim(int d) { return d == 64 || d == 128; }
 bool valid_block(int b) { return b == 64 || b == 128; }
 
@@ -277,11 +302,12 @@ sa_status sa_build_mask(const void* q, const void* k, int B, int H, int N, int d
   constexpr int kScoresSmem = sa::kScoresTcSmem + 1024;
   if (d == 128) {
     sa::block_means_kernel<128><<<g1, 128, 0, s>>>(qb, kb, N, block, nb, qmean, qlo, khi, klo);
-    sa::block_scores_tc_kernel<128><<<g2, 128, kScoresSmem, s>>>(smaps, nb, scale, scores);
+    e = launch_pdl(sa::block_scores_tc_kernel<128>, g2, kScoresSmem, s, smaps, nb, scale, scores);
   } else {
     sa::block_means_kernel<64><<<g1, 128, 0, s>>>(qb, kb, N, block, nb, qmean, qlo, khi, klo);
-    sa::block_scores_tc_kernel<64><<<g2, 128, kScoresSmem, s>>>(smaps, nb, scale, scores);
+    e = launch_pdl(sa::block_scores_tc_kernel<64>, g2, kScoresSmem, s, smaps, nb, scale, scores);
   }
+  if (e != cudaSuccess) return SA_ERR_CUDA;
   const long long nrows = static_cast<long long>(BH) * nb;
   const unsigned warp_grid = static_cast<unsigned>((nrows + 3) / 4);
   if (mode == SA_MASK_GLOBAL) {
@@ -306,37 +332,44 @@ sa_status sa_build_mask(const void* q, const void* k, int B, int H, int N, int d
     sa::global_mark_kernel<<<gs, sa::kGlobalSliceThreads, 0, s>>>(scores, stats, nb, state, mask_out);
     return cuda_status(cudaGetLastError());
   }
+  const float* cscores = scores;
+  auto tau_rows = [&](auto kern) {
+    return launch_pdl(kern, dim3(warp_grid), 0, s, cscores, nb, nrows, tau, mask_out);
+  };
+  auto level_rows = [&](auto kern) {
+    return launch_pdl(kern, dim3(warp_grid), 0, s, cscores, nb, nrows, c0, c1, c2, mask_out);
+  };
   if (mode == SA_MASK_TAU && nb <= 1024) {
     if (nb <= 32)
-      sa::tau_select_warp_kernel<1><<<warp_grid, 128, 0, s>>>(scores, nb, nrows, tau, mask_out);
+      e = tau_rows(sa::tau_select_warp_kernel<1>);
     else if (nb <= 64)
-      sa::tau_select_warp_kernel<2><<<warp_grid, 128, 0, s>>>(scores, nb, nrows, tau, mask_out);
+      e = tau_rows(sa::tau_select_warp_kernel<2>);
     else if (nb <= 128)
-      sa::tau_select_warp_kernel<4><<<warp_grid, 128, 0, s>>>(scores, nb, nrows, tau, mask_out);
+      e = tau_rows(sa::tau_select_warp_kernel<4>);
     else if (nb <= 256)
-      sa::tau_select_warp_kernel<8><<<warp_grid, 128, 0, s>>>(scores, nb, nrows, tau, mask_out);
+      e = tau_rows(sa::tau_select_warp_kernel<8>);
     else if (nb <= 512)
-      sa::tau_select_warp_kernel<16><<<warp_grid, 128, 0, s>>>(scores, nb, nrows, tau, mask_out);
+      e = tau_rows(sa::tau_select_warp_kernel<16>);
     else
-      sa::tau_select_warp_kernel<32><<<warp_grid, 128, 0, s>>>(scores, nb, nrows, tau, mask_out);
-    return cuda_status(cudaGetLastError());
+      e = tau_rows(sa::tau_select_warp_kernel<32>);
+    return cuda_status(e != cudaSuccess ? e : cudaGetLastError());
   }
   if (nb <= 32)
-    sa::level_select_warp_kernel<1><<<warp_grid, 128, 0, s>>>(scores, nb, nrows, c0, c1, c2, mask_out);
+    e = level_rows(sa::level_select_warp_kernel<1>);
   else if (nb <= 64)
-    sa::level_select_warp_kernel<2><<<warp_grid, 128, 0, s>>>(scores, nb, nrows, c0, c1, c2, mask_out);
+    e = level_rows(sa::level_select_warp_kernel<2>);
   else if (nb <= 128)
-    sa::level_select_warp_kernel<4><<<warp_grid, 128, 0, s>>>(scores, nb, nrows, c0, c1, c2, mask_out);
+    e = level_rows(sa::level_select_warp_kernel<4>);
   else if (nb <= 256)
-    sa::level_select_warp_kernel<8><<<warp_grid, 128, 0, s>>>(scores, nb, nrows, c0, c1, c2, mask_out);
+    e = level_rows(sa::level_select_warp_kernel<8>);
   else if (nb <= 512)
-    sa::level_select_warp_kernel<16><<<warp_grid, 128, 0, s>>>(scores, nb, nrows, c0, c1, c2, mask_out);
+    e = level_rows(sa::level_select_warp_kernel<16>);
   else if (nb <= 1024)
-    sa::level_select_warp_kernel<32><<<warp_grid, 128, 0, s>>>(scores, nb, nrows, c0, c1, c2, mask_out);
+    e = level_rows(sa::level_select_warp_kernel<32>);
   else
     sa::block_select_kernel<<<static_cast<unsigned>(nrows), sa::kSelectThreads, sa::select_smem_bytes(nb), s>>>(
         scores, nb, mode, tau, c0, c1, c2, mask_out);
-  return cuda_status(cudaGetLastError());
+  return cuda_status(e != cudaSuccess ? e : cudaGetLastError());
 }
 
 sa_status sa_radial_mask(int T, int Hh, int Ww, int block, uint8_t* mask_out, void* stream) {

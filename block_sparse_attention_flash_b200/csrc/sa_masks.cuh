@@ -71,6 +71,9 @@ __global__ void __launch_bounds__(128) block_means_kernel(const __nv_bfloat16* _
   constexpr int CH = D / 8;      // 16-byte chunks per row
   constexpr int RG = 128 / CH;   // row groups
   __shared__ float red[RG][D];
+  // the scores kernel after this one may be scheduled once every CTA here
+  // has started; it waits for this grid's completion before reading
+  asm volatile("griddepcontrol.launch_dependents;");
   const int i = blockIdx.x, bh = blockIdx.y, z = blockIdx.z;
   const __nv_bfloat16* x = (z == 0 ? q : k) + (static_cast<size_t>(bh) * N + static_cast<size_t>(i) * block) * D;
   const int rows = min(block, N - i * block);
@@ -165,6 +168,11 @@ __global__ void __launch_bounds__(128, 1) block_scores_tc_kernel(const __grid_co
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // launched with programmatic stream serialization: the set-up above may run
+  // beside the block means; wait until they are complete and visible, then
+  // let the selection after this kernel be scheduled
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;");
   const uint32_t tmem = tmem_base;
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer ---
@@ -459,6 +467,8 @@ template <int E>
 __global__ void __launch_bounds__(128, E == 16 ? 11 : 1) level_select_warp_kernel(const float* __restrict__ scores, int nb,
                                                                 long long nrows, int c0, int c1, int c2,
                                                                 uint8_t* __restrict__ mask_out) {
+  // launched with programmatic stream serialization after the scores kernel
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long row = static_cast<long long>(blockIdx.x) * 4 + warp;
   if (row >= nrows) return;
@@ -539,6 +549,8 @@ template <int E>
 __global__ void __launch_bounds__(128) tau_select_warp_kernel(const float* __restrict__ scores, int nb,
                                                               long long nrows, float tau,
                                                               uint8_t* __restrict__ mask_out) {
+  // launched with programmatic stream serialization after the scores kernel
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long row = static_cast<long long>(blockIdx.x) * 4 + warp;
   if (row >= nrows) return;

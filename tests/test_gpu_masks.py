@@ -157,6 +157,53 @@ def test_mask_builder_batch2_ragged(block, d):
     check_bits(lv.cpu(), lr, lflags, f"levels B=2 d={d} block={block}")
 
 
+@pytest.mark.parametrize("mode", ["tau", "levels"])
+def test_mask_builder_on_a_non_default_stream(mode):
+    """Three heads built on a non-default stream and read back on it right after the call, with
+    no synchronisation in between: every launch must go to the caller's stream; against the
+    oracle, flag-aware."""
+    wl = inputs.Workload("h3", 1, 3, 128, 9, 20, 24, 64, "tau", seed=97)
+    q, k, _ = inputs.rff_qkv(wl)
+    nb = wl.nblocks
+    fr = (0.1, 0.3, 0.6)
+    qd, kd = q.cuda(), k.cuda()
+    m = torch.full((1, 3, nb, nb), 0xFF, dtype=torch.uint8, device="cuda")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        ops.sa_build_mask(qd, kd, 64, mode, tau=0.9, level_frac=fr, mask_out=m)
+        got = m.clone()
+    torch.cuda.synchronize()
+    ops.sa_get_device_status()
+    if mode == "tau":
+        ref, flags, _ = tau_mask(q, k, 64, 0.9, return_info=True)
+    else:
+        ref, flags, _ = level_map(q, k, 64, fr, return_info=True)
+    check_bits(got.cpu(), ref, flags, f"{mode} H=3 on a side stream")
+
+
+@pytest.mark.parametrize("mode", ["tau", "levels"])
+def test_mask_builder_graph_capture_matches_eager(mode):
+    """A CUDA-graph capture of the builder (caller's workspace and output) replays to the same
+    bytes as an eager call; 12 heads, 8,192 tokens."""
+    wl = inputs.Workload("g12", 1, 12, 128, 8, 32, 32, 64, "tau", seed=101)
+    q, k, _ = inputs.rff_qkv(wl, device="cuda")
+    B, H, N, d = q.shape
+    nb = wl.nblocks
+    fr = (0.1, 0.3, 0.6)
+    ws = torch.empty(ops.sa_build_mask_workspace(B, H, N, d, 64), dtype=torch.uint8, device="cuda")
+    eager = ops.sa_build_mask(q, k, 64, mode, tau=0.9, level_frac=fr, workspace=ws)
+    m = torch.zeros(B, H, nb, nb, dtype=torch.uint8, device="cuda")
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        ops.sa_build_mask(q, k, 64, mode, tau=0.9, level_frac=fr, mask_out=m, workspace=ws)
+    g.replay()
+    torch.cuda.synchronize()
+    ops.sa_get_device_status()
+    assert torch.equal(m, eager)
+    del g
+
+
 def test_tau_mask_wan13b_480p_full():
     """Full-size tau mask of the 480p Wan2.1-1.3B-like workload (12 heads, 512 x 512 blocks)."""
     wl = inputs.WORKLOADS["wan13b_480p_tau"]
