@@ -40,6 +40,12 @@
  *     exception, sa_build_mask_noalloc, uses a static device array.
  *     sa_sparse_attn_fwd_host creates and destroys its own copy streams and
  *     events inside the call.
+ *   - Every device entry point only launches kernels on `stream` (no copy,
+ *     allocation or synchronisation), so it can be captured in a CUDA graph
+ *     (after one eager call on the device, which sets kernel attributes).
+ *     sa_build_mask launches its scores and selection kernels with
+ *     programmatic stream serialization: each may start while the kernel
+ *     before it finishes, and waits for that kernel's results on the device.
  *
  * Citations name the web page the operation comes from and its section.
  */
