@@ -9,6 +9,7 @@ a constant, so the key gradients sum to zero).
 import math
 
 import numpy as np
+import pytest
 import torch
 
 from block_sparse_attention_flash_b200 import inputs
@@ -71,17 +72,21 @@ def test_empty_rows_and_columns_and_key_shift_invariance():
     assert np.max(np.abs(dv.sum(axis=2) - dout[0, 0, block:].sum(axis=0))) < 1e-12  # rows of P sum to 1
 
 
-def test_sampled_rows_equal_full_gradients():
+@pytest.mark.parametrize("causal", [False, True])
+def test_sampled_rows_equal_full_gradients(causal):
+    """The chunked row sampler agrees with the full backward (itself pinned by finite
+    differences and autograd), on a random block mask with and without the causal cut; the
+    sampled rows include block edges (63, 64, 127) and the last, partial block's rows."""
     wl = inputs.Workload("b", 1, 2, 32, 3, 10, 10, 64, "tau", seed=11)
     q, k, v = inputs.rff_qkv(wl)
     do = inputs.normal_qkv(1, 2, wl.N, 32, seed=12)[0]
     nb = wl.nblocks
     mask = inputs.bernoulli_block_mask(1, 2, nb, nb, 0.5, seed=13)
-    dq, dk, dv = masked_attention_bwd(q, k, v, wl.block, mask, do)
+    dq, dk, dv = masked_attention_bwd(q, k, v, wl.block, mask, do, causal=causal)
     qr = [0, 5, 63, 64, 200, wl.N - 1]
     kr = [1, 64, 127, 150, wl.N - 1]
     for h in range(2):
-        sq, sk, sv = masked_attention_bwd_rows(q, k, v, wl.block, mask, do, 0, h, qr, kr, chunk=96)
+        sq, sk, sv = masked_attention_bwd_rows(q, k, v, wl.block, mask, do, 0, h, qr, kr, chunk=96, causal=causal)
         assert np.max(np.abs(sq - dq[0, h, qr])) < 1e-12
         assert np.max(np.abs(sk - dk[0, h, kr])) < 1e-12
         assert np.max(np.abs(sv - dv[0, h, kr])) < 1e-12

@@ -112,6 +112,7 @@ PIN_SETS = {
     "permute": [lambda: pins_perm.test_axis_orders_equal_grid_transposes("hwt"),
                 pins_perm.test_hand_listed_hwt,
                 pins_perm.test_cell_partitions_equal_blocked_transposes,
+                pins_perm.test_bijection_inverse_and_per_head_orders,
                 _golden(pins_golden.test_axis_orders, "test_axis_orders")],
     "pyramid": [pins_pl.test_pool_partial_group_and_progressive_equals_direct,
                 pins_pl.test_all_level_zero_equals_block_attention,
@@ -120,6 +121,9 @@ PIN_SETS = {
     "backward": [pins_bwd.test_empty_rows_and_columns_and_key_shift_invariance,
                  pins_bwd.test_dense_case_equals_torch_autograd,
                  pins_bwd.test_causal_finite_differences],
+    "backward_rows": [lambda: pins_bwd.test_sampled_rows_equal_full_gradients(False),
+                      lambda: pins_bwd.test_sampled_rows_equal_full_gradients(True)],
+    "chain": [pins_pl.test_first_visited_block_never_skipped_and_chain_monotone],
 }
 
 A, M, L, P, Y, W = (oracle.attention, oracle.masks, oracle.lite, oracle.permute, oracle.pyramid,
@@ -197,6 +201,16 @@ MUTATIONS = [
     ("bwd-no-delta", W, "attention_bwd_head", "dr = np.sum(p * dp, axis=1, keepdims=True)", "dr = 0.0", "backward"),
     ("bwd-dk-no-scale", W, "attention_bwd_head", "scale * (ds.T @ qh)", "(ds.T @ qh)", "backward"),
     ("bwd-dv-transposed", W, "attention_bwd_head", "dv = p.T @ doh", "dv = p @ doh", "backward"),
+    ("bwd-rows-no-delta", W, "masked_attention_bwd_rows", "dr = np.sum(doh[r0:r1] * o, axis=1, keepdims=True)",
+     "dr = 0.0", "backward_rows"),
+    ("bwd-rows-causal-drops-diagonal", W, "masked_attention_bwd_rows",
+     "np.arange(N)[None, :] <= rows[:, None]", "np.arange(N)[None, :] < rows[:, None]", "backward_rows"),
+    ("bwd-rows-dk-no-scale", W, "masked_attention_bwd_rows", "dk += scale * (dsc.T @ qh[r0:r1])",
+     "dk += dsc.T @ qh[r0:r1]", "backward_rows"),
+    ("perm-inverse-applies-forward", P, "permute_tokens", "out[:, h, perm] = x[:, h]", "out[:, h] = x[:, h, perm]",
+     "permute"),
+    ("chain-skip-not-carried", L, "lite_chain", "skip = S if feed is None else feed(s, S)",
+     "skip = skip0 if feed is None else feed(s, S)", "chain"),
 ]
 
 
