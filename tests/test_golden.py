@@ -11,7 +11,7 @@ import pytest
 
 from oracle import lite_step, permutation, radial_mask
 from oracle.lite import skip_flags
-from oracle.masks import global_head, level_row, tau_row
+from oracle.masks import global_head, level_counts, level_row, tau_row
 
 from _golden import floats as _floats, ints as _ints, matrix, records as _records
 
@@ -28,6 +28,13 @@ def test_tau_rows(rec):
     p = np.array(_floats(rec["p"]))
     keep, _, _, _ = tau_row(np.log(p), float(rec["tau"]))
     assert np.nonzero(keep)[0].tolist() == _ints(rec["keep"])
+
+
+@pytest.mark.parametrize("rec", _records("level_rows.txt"), ids=lambda r: f"{r['p']}@{r['fr']}")
+def test_level_rows(rec):
+    p = np.array(_floats(rec["p"]))
+    code, _ = level_row(np.log(p), level_counts(p.size, _floats(rec["fr"])))
+    assert code.tolist() == _ints(rec["code"])
 
 
 @pytest.mark.parametrize("rec", _records("global_heads.txt"), ids=lambda r: f"{r['p']}@{r['tau']}")

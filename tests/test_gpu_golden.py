@@ -72,6 +72,16 @@ def test_tau_rows(rec):
         assert np.nonzero(m[i])[0].tolist() == ints(rec["keep"]), i
 
 
+@pytest.mark.parametrize("rec", records("level_rows.txt"), ids=lambda r: f"{r['p']}@{r['fr']}")
+def test_level_rows(rec):
+    p = np.array(floats(rec["p"]))
+    P = np.tile(p, (p.size, 1))                 # every q-block sees the fixture's row
+    q, k = _scores_qk(P)
+    m = ops.sa_build_mask(q, k, 64, mode="levels", level_frac=tuple(floats(rec["fr"]))).cpu().numpy()[0, 0]
+    for i in range(p.size):
+        assert m[i].tolist() == ints(rec["code"]), i
+
+
 @pytest.mark.parametrize("rec", [r for r in records("global_heads.txt") if len(matrix(r["p"])) == len(matrix(r["p"])[0])],
                          ids=lambda r: f"{r['p']}@{r['tau']}")
 def test_global_heads(rec):

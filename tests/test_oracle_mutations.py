@@ -56,6 +56,7 @@ def _golden(test, name):
     from _golden import records
     fixture = {"test_axis_orders": "axis_orders.txt", "test_tau_rows": "tau_rows.txt",
                "test_global_heads": "global_heads.txt", "test_radial_rows": "radial_rows.txt",
+               "test_level_rows": "level_rows.txt",
                "test_lite_skip": "lite_skip.txt"}[name]
 
     def run():
@@ -90,7 +91,8 @@ PIN_SETS = {
             pins_masks.test_tau_monotone,
             _golden(pins_golden.test_tau_rows, "test_tau_rows"),
             _margin("tau")],
-    "levels": [pins_masks.test_level_quotas_and_order, pins_masks.test_level_ties_break_by_index, _margin("level")],
+    "levels": [pins_masks.test_level_quotas_and_order, pins_masks.test_level_ties_break_by_index, _margin("level"),
+               _golden(pins_golden.test_level_rows, "test_level_rows")],
     "scores": [pins_masks.test_block_means_closed_form_with_partial_tail, pins_masks.test_block_scores_closed_form],
     "radial": [lambda: pins_masks.test_radial_matches_bruteforce(17, 4, 9, 8),
                lambda: pins_masks.test_radial_matches_bruteforce(9, 8, 16, 16),
@@ -169,6 +171,9 @@ MUTATIONS = [
     ("tau-flag-no-swap-dropped", M, "tau_row", "flag |= (~keep) & (np.abs(p - p_in) <= MARGIN * p_in)", "pass",
      "tau"),
     ("tau-flag-swap-absolute", M, "tau_row", "<= MARGIN * p_out", "<= MARGIN", "tau"),
+    ("level-code-is-level", M, "level_row", "code[rank < counts[lvl]] = lvl + 1", "code[rank < counts[lvl]] = lvl",
+     "levels"),
+    ("level-coarse-overwrites-fine", M, "level_row", "for lvl in (2, 1, 0):", "for lvl in (0, 1, 2):", "levels"),
     ("level-flag-margin-wide", M, "level_row", "(s - s_out < MARGIN)", "(s - s_out < 10 * MARGIN)", "levels"),
     ("level-flag-sign", M, "level_row", "(s - s_out < MARGIN)", "(s_out - s < MARGIN)", "levels"),
     ("level-flag-no-lower-side", M, "level_row", "flag |= (rank >= c) & (s_in - s < MARGIN)", "pass", "levels"),
