@@ -51,6 +51,7 @@ def test_all_ones_mask_equals_dense_sdpa_tiny_config():
     ref = _sdpa64(q, k, v)
     assert np.max(np.abs(O - ref)) < 1e-12
     Od, Ld = dense_attention(q, k, v)
+    assert np.max(np.abs(Od - ref)) < 1e-12
     assert np.max(np.abs(L - Ld)) < 1e-12
 
 

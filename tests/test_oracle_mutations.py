@@ -84,6 +84,7 @@ PIN_SETS = {
                   pins_attn.test_lse_matches_scipy_logsumexp_on_kept_columns,
                   pins_attn.test_causal_all_ones_equals_sdpa_is_causal,
                   pins_attn.test_causal_block_mask_equals_token_level_brute_force],
+    "dense": [pins_attn.test_all_ones_mask_equals_dense_sdpa_tiny_config],
     "tau": [pins_masks.test_tau_uniform_scores_keep_first_ceil_tau_n,
             pins_masks.test_tau_block_exactly_at_the_threshold_is_dropped,
             pins_masks.test_tau_to_zero_keeps_only_argmax,
@@ -139,6 +140,10 @@ MUTATIONS = [
      "attention"),
     ("attn-causal-drops-diagonal", A, "attention_qblock", "c[None, :] <= np.arange(r0, r1)[:, None]",
      "c[None, :] < np.arange(r0, r1)[:, None]", "attention"),
+    ("dense-unnormalised", A, "dense_attention", "e / z, v)", "e, v)", "dense"),
+    ("dense-lse-without-max", A, "dense_attention", "(m + np.log(z))", "(np.log(z))", "dense"),
+    ("token-mask-transposed", A, "block_mask_to_token_mask", "return m[idx][:, idx]", "return m.T[idx][:, idx]",
+     "backward"),
     ("tau-non-strict", M, "tau_row", "keep = mass_before < tau", "keep = mass_before <= tau", "tau"),
     ("tau-mass-includes-self", M, "tau_row", "mass_before[j] = acc\n        acc += p[j]",
      "acc += p[j]\n        mass_before[j] = acc", "tau"),
