@@ -11,7 +11,7 @@ import pytest
 
 from oracle import lite_step, permutation, radial_mask
 from oracle.lite import skip_flags
-from oracle.masks import global_head, level_counts, level_row, tau_row
+from oracle.masks import global_head, global_mask, level_counts, level_map, level_row, tau_mask, tau_row
 
 from _golden import floats as _floats, ints as _ints, matrix, records as _records
 
@@ -89,3 +89,71 @@ def check_margin_flags(rec):
                          ids=lambda r: "-".join(f"{k}{v}" for k, v in r.items() if k in ("kind", "p", "s", "tau")))
 def test_margin_flags(rec):
     check_margin_flags(rec)
+
+
+def _qk_for_scores(heads, block=3):
+    """fp64 Q, K [1, len(heads), nb * block, d] whose block scores are ln P for each head's
+    [nb, nb] matrix P (d = nb, scale 1 / sqrt(d)): every row of q-block i is sqrt(d) e_i and
+    every row of k-block j holds ln P[i, j] in dimension i, so the block means are those rows and
+    S[i, j] = (1 / sqrt(d)) * sqrt(d) * ln P[i, j]."""
+    nb = heads[0].shape[0]
+    d, N = nb, nb * block
+    q = np.zeros((1, len(heads), N, d))
+    k = np.zeros((1, len(heads), N, d))
+    for h, P in enumerate(heads):
+        for i in range(nb):
+            q[0, h, i * block:(i + 1) * block, i] = math.sqrt(d)
+            for j in range(nb):
+                k[0, h, j * block:(j + 1) * block, i] = math.log(P[i, j])
+    return q, k
+
+
+def _fixture_row_heads(p):
+    """Head 0: row 0 is the fixture's row, the other rows uniform; head 1: every row uniform."""
+    nb = p.size
+    uniform = np.full((nb, nb), 1.0 / nb)
+    h0 = uniform.copy()
+    h0[0] = p
+    return [h0, uniform]
+
+
+@pytest.mark.parametrize("rec", _records("tau_rows.txt"), ids=lambda r: f"{r['p']}@{r['tau']}")
+def test_tau_rows_through_the_mask_wrapper(rec):
+    """The whole oracle path (block means, scores, per-row selection over every head and row)
+    reproduces the fixture's row; uniform rows keep the first ceil(tau * Nb) blocks."""
+    p = np.array(_floats(rec["p"]))
+    nb, tau = p.size, float(rec["tau"])
+    q, k = _qk_for_scores(_fixture_row_heads(p))
+    m = tau_mask(q, k, 3, tau)
+    first = list(range(math.ceil(tau * nb - 1e-9)))
+    assert np.nonzero(m[0, 0, 0])[0].tolist() == _ints(rec["keep"])
+    for h, i in [(0, i) for i in range(1, nb)] + [(1, i) for i in range(nb)]:
+        assert np.nonzero(m[0, h, i])[0].tolist() == first, (h, i)
+
+
+@pytest.mark.parametrize("rec", _records("level_rows.txt"), ids=lambda r: f"{r['p']}@{r['fr']}")
+def test_level_rows_through_the_map_wrapper(rec):
+    """As above for the level map; uniform rows take the codes in index order."""
+    p = np.array(_floats(rec["p"]))
+    nb = p.size
+    q, k = _qk_for_scores(_fixture_row_heads(p))
+    lv = level_map(q, k, 3, _floats(rec["fr"]))
+    counts = level_counts(nb, _floats(rec["fr"]))
+    uniform = [1 if r < counts[0] else 2 if r < counts[1] else 3 if r < counts[2] else 4 for r in range(nb)]
+    assert lv[0, 0, 0].tolist() == _ints(rec["code"])
+    for h, i in [(0, i) for i in range(1, nb)] + [(1, i) for i in range(nb)]:
+        assert lv[0, h, i].tolist() == uniform, (h, i)
+
+
+@pytest.mark.parametrize("rec", [r for r in _records("global_heads.txt") if len(matrix(r["p"])) == len(matrix(r["p"])[0])],
+                         ids=lambda r: f"{r['p']}@{r['tau']}")
+def test_global_heads_through_the_mask_wrapper(rec):
+    """As above for the global selection (the square fixtures); head 1's uniform scores keep the
+    first ceil(tau * Nb * Nb) pairs in index order."""
+    P = np.array(matrix(rec["p"]))
+    nb, tau = P.shape[0], float(rec["tau"])
+    q, k = _qk_for_scores([P, np.full((nb, nb), 1.0 / nb)])
+    m = global_mask(q, k, 3, tau)
+    assert np.array_equal(m[0, 0].astype(np.int64), np.array(matrix(rec["keep"], _ints)))
+    n_keep = math.ceil(tau * nb * nb - 1e-9)
+    assert m[0, 1].ravel().tolist() == [1] * n_keep + [0] * (nb * nb - n_keep)

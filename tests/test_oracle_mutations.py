@@ -25,6 +25,7 @@ import oracle.masks
 import oracle.permute
 import oracle.pyramid
 import test_golden as pins_golden
+from _golden import matrix
 import test_oracle_attention as pins_attn
 import test_oracle_backward as pins_bwd
 import test_oracle_masks as pins_masks
@@ -56,11 +57,21 @@ def _golden(test, name):
     from _golden import records
     fixture = {"test_axis_orders": "axis_orders.txt", "test_tau_rows": "tau_rows.txt",
                "test_global_heads": "global_heads.txt", "test_radial_rows": "radial_rows.txt",
-               "test_level_rows": "level_rows.txt",
+               "test_level_rows": "level_rows.txt", "test_tau_rows_through_the_mask_wrapper": "tau_rows.txt",
+               "test_level_rows_through_the_map_wrapper": "level_rows.txt",
+               "test_global_heads_through_the_mask_wrapper": "global_heads.txt",
                "test_lite_skip": "lite_skip.txt"}[name]
 
     def run():
         for rec in records(fixture):
+            test(rec)
+    return run
+
+
+def _square(test):
+    """The global wrapper pin takes the square fixtures only (the library's masks are Nb x Nb)."""
+    def run(rec):
+        if len(matrix(rec["p"])) == len(matrix(rec["p"])[0]):
             test(rec)
     return run
 
@@ -124,6 +135,11 @@ PIN_SETS = {
     "backward": [pins_bwd.test_empty_rows_and_columns_and_key_shift_invariance,
                  pins_bwd.test_dense_case_equals_torch_autograd,
                  pins_bwd.test_causal_finite_differences],
+    "wrappers": [_golden(pins_golden.test_tau_rows_through_the_mask_wrapper, "test_tau_rows_through_the_mask_wrapper"),
+                 _golden(pins_golden.test_level_rows_through_the_map_wrapper,
+                         "test_level_rows_through_the_map_wrapper"),
+                 _golden(_square(pins_golden.test_global_heads_through_the_mask_wrapper),
+                         "test_global_heads_through_the_mask_wrapper")],
     "backward_rows": [lambda: pins_bwd.test_sampled_rows_equal_full_gradients(False),
                       lambda: pins_bwd.test_sampled_rows_equal_full_gradients(True)],
     "chain": [pins_pl.test_first_visited_block_never_skipped_and_chain_monotone],
@@ -144,6 +160,13 @@ MUTATIONS = [
     ("dense-lse-without-max", A, "dense_attention", "(m + np.log(z))", "(np.log(z))", "dense"),
     ("token-mask-transposed", A, "block_mask_to_token_mask", "return m[idx][:, idx]", "return m.T[idx][:, idx]",
      "backward"),
+    ("tau-mask-first-row-only", M, "tau_mask", "tau_row(S[b, h, i], tau)", "tau_row(S[b, h, 0], tau)", "wrappers"),
+    ("tau-mask-first-head-only", M, "tau_mask", "tau_row(S[b, h, i], tau)", "tau_row(S[b, 0, i], tau)", "wrappers"),
+    ("level-map-first-row-only", M, "level_map", "level_row(S[b, h, i], counts)", "level_row(S[b, h, 0], counts)",
+     "wrappers"),
+    ("global-mask-first-head-only", M, "global_mask", "global_head(S[b, h], tau)", "global_head(S[b, 0], tau)",
+     "wrappers"),
+    ("scores-transposed", M, "block_scores", '"bhid,bhjd->bhij"', '"bhid,bhjd->bhji"', "wrappers"),
     ("tau-non-strict", M, "tau_row", "keep = mass_before < tau", "keep = mass_before <= tau", "tau"),
     ("tau-mass-includes-self", M, "tau_row", "mass_before[j] = acc\n        acc += p[j]",
      "acc += p[j]\n        mass_before[j] = acc", "tau"),
