@@ -267,3 +267,29 @@ def test_radial_order_reaches_the_row_max_first():
             loc = rows[:, j * block:(j + 1) * block].max(axis=1)
             assert bool(n_vis > 0 and np.all(loc < run - 10.0)) == bool(Sr[0, 0, i, j])
             run = np.maximum(run, loc)
+
+
+def test_sampled_qblocks_equal_full_for_lite_and_pyramid():
+    """The q-block samplers that the full-size GPU tests use (``qblocks=``) return exactly the
+    full computation's rows, for the skip update (with a carried skip mask and a block mask) and
+    for pyramid attention over a mixed level map; the samples include the partial last q-block."""
+    wl = inputs.Workload("s", 1, 2, 16, 3, 5, 7, 16, "lite", seed=91)   # 105 tokens, 7 blocks
+    q, k, v = inputs.rff_qkv(wl)
+    nb, N = wl.nblocks, wl.N
+    g = np.random.default_rng(92)
+    mask = (g.random((1, 2, nb, nb)) < 0.8).astype(np.uint8)
+    skip0 = (g.random((1, 2, nb, nb)) < 0.2).astype(np.uint8)
+    picks = [(0, 1, 0), (0, 0, 3), (0, 1, nb - 1)]
+    O, L, S, M = lite_step(q, k, v, wl.block, mask, skip0, eps=2.0)
+    part = lite_step(q, k, v, wl.block, mask, skip0, eps=2.0, qblocks=picks)
+    assert list(part) == picks
+    for (b, h, i), (o, l, srow, mrow) in part.items():
+        sl = slice(i * wl.block, min(N, (i + 1) * wl.block))
+        assert np.array_equal(o, O[b, h, sl]) and np.array_equal(l, L[b, h, sl])
+        assert np.array_equal(srow, S[b, h, i]) and np.array_equal(mrow, M[b, h, i], equal_nan=True)
+    codes = g.integers(0, 5, size=(1, 2, nb, nb)).astype(np.uint8)
+    Op, Lp = pyramid_attention(q, k, v, wl.block, codes)
+    pp = pyramid_attention(q, k, v, wl.block, codes, qblocks=picks)
+    for (b, h, i), (o, l) in pp.items():
+        sl = slice(i * wl.block, min(N, (i + 1) * wl.block))
+        assert np.array_equal(o, Op[b, h, sl]) and np.array_equal(l, Lp[b, h, sl])
