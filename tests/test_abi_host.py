@@ -149,6 +149,20 @@ def test_ops_refuse_cpu_tensors():
         ops.sa_sparse_attn_fwd(q, q, q, 64, out=q.clone())
 
 
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """Without the built library every op raises; nothing falls back to another implementation."""
+    import torch
+    monkeypatch.setattr(ops, "LIB_PATH", str(tmp_path / "libsparse_attn.so"))
+    monkeypatch.setattr(ops, "_lib", None)
+    with pytest.raises(RuntimeError, match="is missing"):
+        ops.lib()
+    q = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16)
+    with pytest.raises(RuntimeError, match="is missing"):
+        ops.sa_build_mask_workspace(1, 1, 128, 64, 64)
+    with pytest.raises((RuntimeError, ValueError)):
+        ops.sa_sparse_attn_fwd(q, q, q, 64)
+
+
 def _bwd(lib, **kw):
     a = dict(q=16, k=16, v=16, o=16, dout=16, lse=16, B=1, H=1, N=256, d=128, block=128, mask=None, sb=0, sh=0,
              si=0, scale=0.0, causal=0, dq=16, dk=16, dv=16, ws=16, ws_bytes=1 << 20, stream=None)
