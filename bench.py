@@ -47,7 +47,10 @@ METRIC = "sparse attn ms/call, executed TFLOP/s & % B200 BF16 tensor peak at 75.
 # DRAM bytes (read + write) of one attention launch at 75,600 tokens x 40 heads,
 # from an ncu capture of the 4-head case (239.5 MB read + 61.4 MB written,
 # scaled by 40/4 heads).  Valid for the kernel version that capture measured;
-# set to None whenever the kernel changes.
+# set to None whenever the kernel changes.  The source edits since that capture
+# removed only code that never ran (a polynomial branch whose condition was
+# false at compile time, an unused barrier helper), so the executed kernel is
+# the one measured.
 ATTN_DRAM_BYTES_PER_LAUNCH = 3.0087e9
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
