@@ -9,7 +9,7 @@ import math
 import numpy as np
 import pytest
 
-from oracle import lite_step, permutation, radial_mask
+from oracle import lite_step, permutation, pyramid_attention, radial_mask
 from oracle.lite import skip_flags
 from oracle.masks import global_head, global_mask, level_counts, level_map, level_row, tau_mask, tau_row
 
@@ -157,3 +157,15 @@ def test_global_heads_through_the_mask_wrapper(rec):
     assert np.array_equal(m[0, 0].astype(np.int64), np.array(matrix(rec["keep"], _ints)))
     n_keep = math.ceil(tau * nb * nb - 1e-9)
     assert m[0, 1].ravel().tolist() == [1] * n_keep + [0] * (nb * nb - n_keep)
+
+
+@pytest.mark.parametrize("rec", _records("pyramid_rows.txt"), ids=lambda r: f"codes{r['codes']}")
+def test_pyramid_rows(rec):
+    """d = 1, scale 1, block 8, 16 tokens, every query 1; k-block 0: keys 0, values 1."""
+    k = np.array([0.0] * 8 + _floats(rec["k1"])).reshape(1, 1, 16, 1)
+    v = np.array([1.0] * 8 + _floats(rec["v1"])).reshape(1, 1, 16, 1)
+    q = np.ones((1, 1, 16, 1))
+    codes = np.array([_ints(rec["codes"])] * 2, dtype=np.uint8)
+    O, L = pyramid_attention(q, k, v, 8, codes, scale=1.0)
+    assert np.allclose(O[0, 0, :8, 0], float(rec["o"]), rtol=0, atol=1e-12)
+    assert np.allclose(L[0, 0, :8], float(rec["lse"]), rtol=0, atol=1e-12)

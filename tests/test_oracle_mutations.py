@@ -57,7 +57,7 @@ def _golden(test, name):
     from _golden import records
     fixture = {"test_axis_orders": "axis_orders.txt", "test_tau_rows": "tau_rows.txt",
                "test_global_heads": "global_heads.txt", "test_radial_rows": "radial_rows.txt",
-               "test_level_rows": "level_rows.txt", "test_tau_rows_through_the_mask_wrapper": "tau_rows.txt",
+               "test_level_rows": "level_rows.txt", "test_pyramid_rows": "pyramid_rows.txt", "test_tau_rows_through_the_mask_wrapper": "tau_rows.txt",
                "test_level_rows_through_the_map_wrapper": "level_rows.txt",
                "test_global_heads_through_the_mask_wrapper": "global_heads.txt",
                "test_lite_skip": "lite_skip.txt"}[name]
@@ -131,7 +131,8 @@ PIN_SETS = {
     "pyramid": [pins_pl.test_pool_partial_group_and_progressive_equals_direct,
                 pins_pl.test_all_level_zero_equals_block_attention,
                 pins_pl.test_constant_groups_make_any_level_mix_exact,
-                pins_pl.test_causal_constant_groups_equal_causal_attention],
+                pins_pl.test_causal_constant_groups_equal_causal_attention,
+                _golden(pins_golden.test_pyramid_rows, "test_pyramid_rows")],
     "backward": [pins_bwd.test_empty_rows_and_columns_and_key_shift_invariance,
                  pins_bwd.test_dense_case_equals_torch_autograd,
                  pins_bwd.test_causal_finite_differences],
@@ -229,6 +230,8 @@ MUTATIONS = [
     ("pool-divide-by-c", Y, "pyramid_pool", "/ (r1 - r0)", "/ c", "pyramid"),
     ("pyramid-bias-sign", Y, "_level_keys", "np.log(counts)", "-np.log(counts)", "pyramid"),
     ("pyramid-bias-missing", Y, "_level_keys", "np.log(counts)", "0.0 * counts", "pyramid"),
+    ("pyramid-values-subsampled", Y, "_level_keys", "pooled_v[level][g0:g1], np.log(counts)",
+     "vh[r0:r1:c], np.log(counts)", "pyramid"),
     ("pyramid-causal-diagonal-pooled", Y, "pyramid_attention", "if causal and j == i and code:\n                code = 1",
      "if causal and j == i and code:\n                code = code", "pyramid"),
     ("bwd-no-delta", W, "attention_bwd_head", "dr = np.sum(p * dp, axis=1, keepdims=True)", "dr = 0.0", "backward"),
